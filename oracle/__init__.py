@@ -1,0 +1,51 @@
+"""fp64 CPU oracle of the timestep-forced streaming denoising step.
+
+TEST INFRASTRUCTURE ONLY.  Only the test-suite, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline / reference leg may import or run anything in this
+package.  The CUDA path in ``streaming_causal_video_timestep_b200`` shares no
+code with it: neither imports the other; both take their inputs from the
+seeded generators in ``workloads``.
+
+What it computes (Live Avatar, arXiv 2512.04677, as described on the pages):
+  * block-causal attention of a 3-latent-frame block over [sink | rolling
+    window | itself] (10100.com article, training-framework figure caption:
+    "block-independent noise + causal mask"; papernotes note, 整体框架);
+  * a noisy rolling KV cache kept per timestep, never refreshed with a clean
+    forward (papernotes note, 关键设计 2 "History Corrupt"; gitcode blog,
+    question 4);
+  * timestep forcing: the cache read at step t_i holds K/V computed at t_i
+    (papernotes note, 关键设计 4; gitcode blog, question 6);
+  * Rolling RoPE: the sink frame's temporal position is re-offset each block so
+    its distance to the active block is constant (papernotes note, 关键设计 3;
+    admirer.cn article, "滾動位置編碼");
+  * Adaptive Attention Sink: the first generated latent replaces the reference
+    sink once (papernotes note, 关键设计 3; gitcode blog, question 5);
+  * flow-matching velocity v ~ x1 - x0 and an Euler step between the 4
+    distilled timesteps (papernotes note, 损失函数 / L_FM);
+  * the timestep-pipelined order of the 4 in-flight blocks (10100.com article,
+    TPP figure caption; gitcode blog, question 6).
+
+Everything is fp64 numpy with a dict-indexed cache, an explicit mask matrix and
+a naive softmax.  The readings taken where the pages are silent are listed in
+the design doc of this repository.
+
+Pins (tests/test_oracle_*.py): brute force on tiny inputs, SDPA on the visible
+segments, softmax rows summing to 1, single-key passthrough, RoPE norm and
+relative-position identities against a complex-number formulation, the Rolling
+RoPE offset up to 10,000 blocks, (block, step) cache tags, the flow-matching
+straight-line closed form, pipelined == sequential order with the sink fixed,
+and closed forms of the layer with special weights.  Agreement with the real
+14B Live Avatar model is parity unpinned: the pages give no weights, code or
+worked example.
+"""
+from .rope import axis_frequencies, rope_rotate, block_positions, sink_positions
+from .attention import block_causal_attention
+from .flow import euler_step
+from .schedule import TickScheduler, index_state_layout
+from .stream import OracleStream
+
+__all__ = [
+    "axis_frequencies", "rope_rotate", "block_positions", "sink_positions",
+    "block_causal_attention", "euler_step", "TickScheduler", "index_state_layout",
+    "OracleStream",
+]

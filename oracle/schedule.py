@@ -1,0 +1,128 @@
+"""Integer state of the stream: tick schedule, ring entries, positions, sink generation.
+
+Timestep-forcing pipeline (10100.com article, TPP figure caption; papernotes
+note, 关键设计 4; gitcode blog, question 6): worker i is pinned to the step
+t_i -> t_{i+1} and keeps its own cache.  On one device the 4 workers become 4
+slots of one tick: at tick k slot i holds the block that slot i-1 held at tick
+k-1 and slot 0 takes the new block, so in an uninterrupted stream slot i runs
+block k - i.  The block in the last slot is finished at the end of its tick.
+
+Ring (readings of the rolling cache, gitcode blog question 1 table: only the
+most recent N blocks are kept): each (layer, slot) ring has window+1 entries;
+block b writes entry b mod (window+1), which evicts block b - window - 1.  The
+block reads the resident blocks b-window .. b-1 oldest first, then itself.
+
+Index-state record (int32), identical to the C-ABI's debug export:
+  header  [tick, blocks_in, blocks_out, sink_generation]
+  per slot i (num_steps records):
+    [active_block, write_entry, evicted_block, sink_tpos, frame_tpos,
+     sink_generation_used, step_index, n_resident,
+     resident[E] (oldest -> newest, -1 padded), tags[E] x (block, step)]
+active_block, write_entry and evicted_block are -1 and sink_tpos, frame_tpos,
+sink_generation_used are 0 for a slot idle this tick; step_index is the slot
+index; n_resident, resident and tags always describe the ring contents.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from workloads import SCHED_PIPELINED, SINK_AAS
+
+
+def index_state_layout(cfg):
+    E = cfg.ring_entries
+    per_slot = 8 + 3 * E
+    return 4, per_slot, 4 + cfg.num_steps * per_slot
+
+
+class TickScheduler:
+    def __init__(self, cfg):
+        self.cfg = cfg
+        S, E = cfg.num_steps, cfg.ring_entries
+        self.S, self.E = S, E
+        self.slots = [-1] * S          # block held by each slot after the last tick
+        self.tick = -1
+        self.blocks_in = 0
+        self.blocks_out = 0
+        self.sink_generation = 0
+        self.tags = [[(-1, -1)] * E for _ in range(S)]
+        self._records = [self._idle_record(i) for i in range(S)]
+
+    # -- one tick ---------------------------------------------------------
+    def begin_tick(self, has_new: bool):
+        """Start a call.  Returns (run, finished): run = [(slot, block)] in
+        execution order, finished = the block completed by this call or -1.
+        The caller appends each (slot, block) with append() right before it
+        computes that step."""
+        S = self.S
+        if self.cfg.schedule == SCHED_PIPELINED:
+            new_block = self.blocks_in if has_new else -1
+            slots = [new_block] + self.slots[:-1]
+            run = [(i, b) for i, b in enumerate(slots) if b >= 0]
+            finished = slots[S - 1]
+            self.slots = slots
+        else:
+            if not has_new:
+                raise ValueError("the sequential schedule needs a new block on every call")
+            b = self.blocks_in
+            run = [(i, b) for i in range(S)]
+            finished = b
+        self.tick += 1
+        if has_new:
+            self.blocks_in += 1
+        self._records = [self._idle_record(i) for i in range(S)]
+        return run, finished
+
+    def end_tick(self, finished: int):
+        """Close a call; returns True when the sink must be replaced now (AAS)."""
+        if finished >= 0:
+            self.blocks_out += 1
+        if finished == 0 and self.cfg.sink_mode == SINK_AAS and self.sink_generation == 0:
+            self.sink_generation = 1
+            return True
+        return False
+
+    def append(self, i: int, b: int):
+        """Ring append of block b in slot i; returns the slot's record."""
+        cfg, E = self.cfg, self.E
+        e = b % E
+        evicted = self.tags[i][e][0]
+        self.tags[i][e] = (b, i)
+        resident = self.resident(i)
+        rec = [b, e, evicted, self.sink_tpos(b), cfg.frames_per_block * b,
+               self.sink_generation, i, len(resident)]
+        rec = rec + self._pad(resident) + [v for tag in self.tags[i] for v in tag]
+        self._records[i] = rec
+        return rec
+
+    # -- queries ------------------------------------------------------------
+    def resident(self, i):
+        return sorted(t[0] for t in self.tags[i] if t[0] >= 0)
+
+    def window_blocks(self, i, b):
+        """Prior blocks block b reads in slot i, oldest first."""
+        return [x for x in self.resident(i) if b - self.cfg.window_blocks <= x < b]
+
+    def sink_tpos(self, b: int) -> int:
+        cfg = self.cfg
+        if cfg.rolling_rope:
+            return cfg.frames_per_block * b - cfg.sink_offset_frames
+        return -cfg.sink_offset_frames
+
+    def index_state(self) -> np.ndarray:
+        head = [self.tick, self.blocks_in, self.blocks_out, self.sink_generation]
+        body = []
+        for i in range(self.S):
+            rec = list(self._records[i])
+            # ring-content fields always reflect the current ring
+            rec[7] = len(self.resident(i))
+            rec[8:8 + self.E] = self._pad(self.resident(i))
+            rec[8 + self.E:] = [v for tag in self.tags[i] for v in tag]
+            body += rec
+        return np.asarray(head + body, dtype=np.int32)
+
+    def _pad(self, xs):
+        return list(xs) + [-1] * (self.E - len(xs))
+
+    def _idle_record(self, i):
+        return [-1, -1, -1, 0, 0, 0, i, 0] + [-1] * self.E + [-1] * (2 * self.E)

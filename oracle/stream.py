@@ -1,0 +1,147 @@
+"""The stream: sink set-up, slot passes, ticks and the Adaptive Attention Sink, fp64.
+
+One slot pass (block b at step i), per the pages' description of the
+streaming DiT step (papernotes note, 整体框架 and 关键设计 2-4):
+    h = x W_in^T                       (identity when latent_ch == hidden)
+    for each layer l:
+        [q | k | v] = h W_qkv[l]^T      (heads of width d, q/k/v in that order)
+        q, k = RoPE at (3b + f, r, c)
+        cache[(l, i, b)] = (k, v)       noisy K/V of THIS step: timestep forcing
+        drop cache[(l, i, b - window - 1)]
+        sink K re-roped at (3b - 3, r, c) (Rolling RoPE), sink V as stored
+        o = block-causal attention over [sink | window | block]
+        h = h + o W_out[l]^T
+    v = h W_head^T                       (identity when latent_ch == hidden)
+    x <- x + (t_{i+1} - t_i) v
+The synthetic sublayers have no norm, FFN or conditioning (the pages give no
+layer internals; the sublayer is the attention step the pages describe).
+
+Sink (reading: the sink frame passes through the same stack attending only to
+itself; its un-roped K and its V are kept per layer and shared by all slots).
+Adaptive Attention Sink (papernotes note, 关键设计 3; gitcode blog, question 5):
+once block 0 is finished, frame 0 of its final latent replaces the sink and the
+sink is never replaced again.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .attention import block_causal_attention
+from .flow import euler_step
+from .rope import block_positions, rope_rotate, sink_positions
+from .schedule import TickScheduler
+
+
+class OracleStream:
+    def __init__(self, cfg, weights, trace: bool = False):
+        self.cfg = cfg
+        f64 = lambda a: None if a is None else np.asarray(a, dtype=np.float64)
+        self.w_qkv = [f64(w) for w in weights.w_qkv]
+        self.w_out = [f64(w) for w in weights.w_out]
+        self.w_in = f64(weights.w_in)
+        self.w_head = f64(weights.w_head)
+        self.sched = TickScheduler(cfg)
+        self.cache = {}            # (layer, slot, block) -> (k_roped, v, (block, step))
+        self.sink_k = None         # per layer, un-roped [F, H, d]
+        self.sink_v = None
+        self.sink_latent = None
+        self.latents = {}          # block -> current latent (fp64)
+        self.trace = {} if trace else None
+
+    # -- pieces -------------------------------------------------------------
+    def _split_heads(self, qkv):
+        c = self.cfg
+        T = qkv.shape[0]
+        D, H, d = c.hidden, c.heads, c.head_dim
+        q = qkv[:, 0:D].reshape(T, H, d)
+        k = qkv[:, D:2 * D].reshape(T, H, d)
+        v = qkv[:, 2 * D:3 * D].reshape(T, H, d)
+        return q, k, v
+
+    def project_in(self, x):
+        x = np.asarray(x, np.float64)
+        return x.copy() if self.w_in is None else x @ self.w_in.T
+
+    def project_head(self, h):
+        return h.copy() if self.w_head is None else h @ self.w_head.T
+
+    # -- sink -----------------------------------------------------------------
+    def set_sink(self, latent):
+        c = self.cfg
+        latent = np.asarray(latent, np.float64)
+        self.sink_latent = latent.copy()
+        h = self.project_in(latent)
+        t0 = -c.sink_offset_frames
+        pt, ph, pw = sink_positions(c, t0)
+        self.sink_k, self.sink_v = [], []
+        for l in range(c.num_layers):
+            q, k, v = self._split_heads(h @ self.w_qkv[l].T)
+            self.sink_k.append(k.copy())
+            self.sink_v.append(v.copy())
+            qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
+            kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
+            o = block_causal_attention(qr, {}, (kr, v), qblock=0, window=c.window_blocks)
+            h = h + o.reshape(h.shape[0], -1) @ self.w_out[l].T
+            if self.trace is not None:
+                self.trace[("sink", l)] = dict(k=k.copy(), v=v.copy(), o=o, h=h.copy())
+
+    # -- one step of one block --------------------------------------------------
+    def slot_pass(self, x, b: int, i: int):
+        c = self.cfg
+        rec = self.sched.append(i, b)
+        x = np.asarray(x, np.float64)
+        h = self.project_in(x)
+        pt, ph, pw = block_positions(c, b)
+        st, sh, sw = sink_positions(c, self.sched.sink_tpos(b))
+        tr = {} if self.trace is not None else None
+        if tr is not None:
+            tr["x_in"] = x.copy()
+            tr["h_in"] = h.copy()
+            tr["record"] = list(rec)
+        for l in range(c.num_layers):
+            q, k, v = self._split_heads(h @ self.w_qkv[l].T)
+            qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
+            kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
+            self.cache[(l, i, b)] = (kr, v.copy(), (b, i))
+            self.cache.pop((l, i, b - c.window_blocks - 1), None)
+            sk = rope_rotate(self.sink_k[l], st, sh, sw, c.pairs, c.rope_theta)
+            blocks = {bb: (kk, vv) for (ll, ii, bb), (kk, vv, _) in self.cache.items()
+                      if ll == l and ii == i}
+            o = block_causal_attention(qr, blocks, (sk, self.sink_v[l]), qblock=b,
+                                       window=c.window_blocks)
+            h = h + o.reshape(h.shape[0], -1) @ self.w_out[l].T
+            if tr is not None:
+                tr[("layer", l)] = dict(q=qr, k=kr, v=v.copy(), sink_k=sk, o=o, h=h.copy())
+        vel = self.project_head(h)
+        x_next = euler_step(x, vel, c.timesteps[i], c.timesteps[i + 1])
+        if tr is not None:
+            tr["v"] = vel
+            tr["x_out"] = x_next.copy()
+            self.trace[(b, i)] = tr
+        return x_next
+
+    # -- one call of the C-ABI's la_denoise_step ---------------------------------
+    def denoise_step(self, x_new=None, inputs=None):
+        """x_new: noise of the next block (or None to drain).  inputs: optional
+        {(block, step): latent} overriding the latent a step starts from
+        (teacher forcing).  Returns (finished latent or None, finished id)."""
+        if self.sink_k is None:
+            raise RuntimeError("set_sink first")
+        has_new = x_new is not None
+        run, finished = self.sched.begin_tick(has_new)
+        if has_new:
+            self.latents[self.sched.blocks_in - 1] = np.asarray(x_new, np.float64)
+        for i, b in run:
+            x = self.latents[b]
+            if inputs is not None and (b, i) in inputs:
+                x = np.asarray(inputs[(b, i)], np.float64)
+            self.latents[b] = self.slot_pass(x, b, i)
+        out = None
+        if finished >= 0:
+            out = self.latents.pop(finished)
+        if self.sched.end_tick(finished):
+            self.set_sink(out[: self.cfg.sink_tokens])
+        return out, finished
+
+    def index_state(self):
+        return self.sched.index_state()

@@ -1,0 +1,147 @@
+"""Brute-force, scalar-loop restatement of the streaming step for tiny inputs.
+
+Written independently of the oracle (no numpy matmul, no shared helpers): every
+projection is an explicit sum, RoPE is an explicit 2x2 rotation per pair with
+math.cos / math.sin, attention loops over keys and decides visibility from the
+block rule, and the schedule uses the closed form "at tick k slot i runs block
+k - i".  Used only to pin the oracle on tiny configs.
+"""
+import math
+
+
+def matvec_rows(X, W):
+    """Y[t][n] = sum_k X[t][k] * W[n][k] (W in [out, in] layout)."""
+    out = []
+    for row in X:
+        out.append([sum(row[k] * wn[k] for k in range(len(row))) for wn in W])
+    return out
+
+
+def rotate(vec, t, r, c, pairs, theta):
+    pt, ph, pw = pairs
+    res = list(vec)
+    for j in range(len(vec) // 2):
+        if j < pt:
+            ang = t * theta ** (-(j) / pt)
+        elif j < pt + ph:
+            ang = r * theta ** (-(j - pt) / ph)
+        else:
+            ang = c * theta ** (-(j - pt - ph) / pw)
+        a, b = vec[2 * j], vec[2 * j + 1]
+        res[2 * j] = a * math.cos(ang) - b * math.sin(ang)
+        res[2 * j + 1] = a * math.sin(ang) + b * math.cos(ang)
+    return res
+
+
+class BruteStream:
+    def __init__(self, cfg, W):
+        self.c = cfg
+        tolist = lambda a: None if a is None else [[float(v) for v in row] for row in a]
+        self.wqkv = [tolist(w) for w in W.w_qkv]
+        self.wout = [tolist(w) for w in W.w_out]
+        self.win = tolist(W.w_in)
+        self.whead = tolist(W.w_head)
+        self.keys = []        # entries (layer, slot, block, token_pos, k_vec_per_head, v_vec_per_head)
+        self.sink = None      # per layer: list of (r, c, k_heads (unroped), v_heads)
+        self.replaced = False
+        self.lat = {}
+
+    def _heads(self, vec, part):
+        c = self.c
+        D, d = c.hidden, c.head_dim
+        return [vec[part * D + h * d: part * D + (h + 1) * d] for h in range(c.heads)]
+
+    def _tok_rc(self, n):
+        F, gw = self.c.frame_tokens, self.c.grid_w
+        f, rem = divmod(n, F)
+        return f, rem // gw, rem % gw
+
+    def _layer_attend(self, qs_heads, key_list):
+        """qs_heads: per query, per head rotated q; key_list: [(k_heads, v_heads)]."""
+        c = self.c
+        outs = []
+        for qh in qs_heads:
+            row = []
+            for h in range(c.heads):
+                logits = [sum(qh[h][e] * kh[h][e] for e in range(c.head_dim)) / math.sqrt(c.head_dim)
+                          for kh, _ in key_list]
+                mx = max(logits)
+                ws = [math.exp(z - mx) for z in logits]
+                tot = sum(ws)
+                acc = [0.0] * c.head_dim
+                for wgt, (_, vh) in zip(ws, key_list):
+                    for e in range(c.head_dim):
+                        acc[e] += wgt / tot * vh[h][e]
+                row.extend(acc)
+            outs.append(row)
+        return outs
+
+    def set_sink(self, latent):
+        c = self.c
+        h = [list(map(float, r)) for r in latent]
+        if self.win is not None:
+            h = matvec_rows(h, self.win)
+        t0 = -c.sink_offset_frames
+        self.sink = []
+        for l in range(c.num_layers):
+            qkv = matvec_rows(h, self.wqkv[l])
+            entries, qrot, krot = [], [], []
+            for n, vec in enumerate(qkv):
+                _, r, cc = self._tok_rc(n)
+                qh, kh, vh = self._heads(vec, 0), self._heads(vec, 1), self._heads(vec, 2)
+                entries.append((r, cc, kh, vh))
+                qrot.append([rotate(x, t0, r, cc, c.pairs, c.rope_theta) for x in qh])
+                krot.append(([rotate(x, t0, r, cc, c.pairs, c.rope_theta) for x in kh], vh))
+            self.sink.append(entries)
+            o = self._layer_attend(qrot, krot)
+            proj = matvec_rows(o, self.wout[l])
+            h = [[a + b for a, b in zip(hr, pr)] for hr, pr in zip(h, proj)]
+
+    def step(self, x, b, i):
+        c = self.c
+        h = [list(map(float, r)) for r in x]
+        if self.win is not None:
+            h = matvec_rows(h, self.win)
+        fpb = c.frames_per_block
+        t_sink = fpb * b - c.sink_offset_frames if c.rolling_rope else -c.sink_offset_frames
+        for l in range(c.num_layers):
+            qkv = matvec_rows(h, self.wqkv[l])
+            qrot = []
+            for n, vec in enumerate(qkv):
+                f, r, cc = self._tok_rc(n)
+                t = fpb * b + f
+                qrot.append([rotate(x_, t, r, cc, c.pairs, c.rope_theta) for x_ in self._heads(vec, 0)])
+                kr = [rotate(x_, t, r, cc, c.pairs, c.rope_theta) for x_ in self._heads(vec, 1)]
+                self.keys.append((l, i, b, kr, self._heads(vec, 2)))
+            visible = []
+            for (r, cc, kh, vh) in self.sink[l]:
+                visible.append(([rotate(x_, t_sink, r, cc, c.pairs, c.rope_theta) for x_ in kh], vh))
+            for (ll, ii, bb, kr, vh) in self.keys:
+                if ll == l and ii == i and b - c.window_blocks <= bb <= b:
+                    visible.append((kr, vh))
+            o = self._layer_attend(qrot, visible)
+            proj = matvec_rows(o, self.wout[l])
+            h = [[a + bq for a, bq in zip(hr, pr)] for hr, pr in zip(h, proj)]
+        v = h if self.whead is None else matvec_rows(h, self.whead)
+        dt = c.timesteps[i + 1] - c.timesteps[i]
+        return [[xa + dt * va for xa, va in zip(xr, vr)] for xr, vr in zip(x, v)]
+
+    def run_pipelined(self, noises):
+        """Tick k: slot i runs block k - i.  Returns {block: final latent}."""
+        c = self.c
+        S = c.num_steps
+        nb = len(noises)
+        done = {}
+        for k in range(nb + S - 1):
+            for i in range(S):
+                b = k - i
+                if 0 <= b < nb:
+                    x = self.lat.get(b, [list(map(float, r)) for r in noises[b]]) if i == 0 else self.lat[b]
+                    self.lat[b] = self.step(x, b, i)
+            fin = k - (S - 1)
+            if 0 <= fin < nb:
+                done[fin] = self.lat.pop(fin)
+                if fin == 0 and c.sink_mode == 1 and not self.replaced:
+                    self.replaced = True
+                    self.set_sink(done[0][: c.sink_tokens])
+        return done

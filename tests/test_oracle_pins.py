@@ -1,0 +1,397 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+Brute force on tiny inputs, a library special case (SDPA), closed forms,
+invariants, and values the Live Avatar pages print (tests/golden).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import OracleStream, TickScheduler, block_causal_attention, euler_step, rope_rotate
+from oracle.rope import axis_frequencies, block_positions, sink_positions, sink_temporal_position
+from workloads import (SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_AAS, SINK_FIXED, TINY,
+                       StreamConfig, Workload, block_noise, make_weights, random_array)
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pages_facts.json")
+
+
+def _facts():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _tiny_blocks(rng, nblocks, T, H, d):
+    return {b: (rng.standard_normal((T, H, d)), rng.standard_normal((T, H, d))) for b in nblocks}
+
+
+# ---------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------
+def test_attention_matches_per_query_brute_force():
+    rng = np.random.default_rng(1)
+    T, F, H, d, window = 12, 4, 2, 4, 2
+    qblock = 5
+    # blocks 2 (evicted: outside the window), 3, 4 (window), 5 (self), 6 (future)
+    blocks = _tiny_blocks(rng, [2, 3, 4, 5, 6], T, H, d)
+    sink = (rng.standard_normal((F, H, d)), rng.standard_normal((F, H, d)))
+    q = rng.standard_normal((T, H, d))
+    got = block_causal_attention(q, blocks, sink, qblock=qblock, window=window)
+    for t in range(T):
+        for h in range(H):
+            keys = [(sink[0][n, h], sink[1][n, h]) for n in range(F)]
+            for b, (k, v) in blocks.items():
+                if qblock - window <= b <= qblock:
+                    keys += [(k[n, h], v[n, h]) for n in range(T)]
+            logits = [sum(q[t, h, e] * kk[e] for e in range(d)) / math.sqrt(d) for kk, _ in keys]
+            mx = max(logits)
+            w = [math.exp(z - mx) for z in logits]
+            tot = sum(w)
+            want = [sum(wi / tot * vv[e] for wi, (_, vv) in zip(w, keys)) for e in range(d)]
+            np.testing.assert_allclose(got[t, h], want, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_matches_sdpa_on_visible_segments():
+    rng = np.random.default_rng(2)
+    T, F, H, d, window = 48, 16, 3, 8, 2
+    qblock = 7
+    blocks = _tiny_blocks(rng, [3, 4, 5, 6, 7], T, H, d)
+    sink = (rng.standard_normal((F, H, d)), rng.standard_normal((F, H, d)))
+    q = rng.standard_normal((T, H, d))
+    got = block_causal_attention(q, blocks, sink, qblock=qblock, window=window)
+    seg_k = [sink[0]] + [blocks[b][0] for b in (5, 6, 7)]
+    seg_v = [sink[1]] + [blocks[b][1] for b in (5, 6, 7)]
+    K = torch.from_numpy(np.concatenate(seg_k)).permute(1, 0, 2)
+    V = torch.from_numpy(np.concatenate(seg_v)).permute(1, 0, 2)
+    Q = torch.from_numpy(q).permute(1, 0, 2)
+    want = torch.nn.functional.scaled_dot_product_attention(Q, K, V).permute(1, 0, 2).numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-12)
+
+
+def test_softmax_rows_sum_to_one_and_masked_keys_get_zero():
+    rng = np.random.default_rng(3)
+    T, F, H, d = 12, 4, 2, 4
+    blocks = _tiny_blocks(rng, [0, 1, 2, 3], T, H, d)
+    sink = (rng.standard_normal((F, H, d)), rng.standard_normal((F, H, d)))
+    q = rng.standard_normal((T, H, d)) * 3
+    _, p, mask = block_causal_attention(q, blocks, sink, qblock=3, window=1, return_probs=True)
+    np.testing.assert_allclose(p.sum(axis=2), 1.0, rtol=0, atol=1e-14)
+    assert np.all(p[:, :, ~mask[0]] == 0.0)
+    # visible keys: 4 sink + block 2 + block 3
+    assert mask[0].sum() == F + 2 * T
+
+
+def test_single_visible_key_passes_its_value_through():
+    rng = np.random.default_rng(4)
+    H, d = 2, 8
+    sink = (rng.standard_normal((1, H, d)), rng.standard_normal((1, H, d)))
+    q = rng.standard_normal((5, H, d)) * 10
+    got = block_causal_attention(q, {}, sink, qblock=0, window=2)
+    np.testing.assert_array_equal(got, np.broadcast_to(sink[1], got.shape))
+
+
+# ---------------------------------------------------------------------------
+# RoPE
+# ---------------------------------------------------------------------------
+PAIRS = (22, 21, 21)
+
+
+def _complex_rope(x, t, r, c, pairs, theta):
+    """Independent formulation: pairs as complex numbers times exp(i * angle)."""
+    z = x[..., 0::2] + 1j * x[..., 1::2]
+    pt, ph, pw = pairs
+    ang = np.concatenate([t * theta ** (-np.arange(pt) / pt), r * theta ** (-np.arange(ph) / ph),
+                          c * theta ** (-np.arange(pw) / pw)])
+    z = z * np.exp(1j * ang)
+    out = np.empty_like(x)
+    out[..., 0::2] = z.real
+    out[..., 1::2] = z.imag
+    return out
+
+
+def test_rope_matches_complex_rotation():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 3, 128))
+    t = np.array([0, 1, 5, 29999, -3, 7])
+    r = np.array([0, 3, 29, 1, 0, 12])
+    c = np.array([0, 51, 2, 7, 0, 40])
+    got = rope_rotate(x, t, r, c, PAIRS, 10000.0)
+    for n in range(6):
+        want = _complex_rope(x[n], t[n], r[n], c[n], PAIRS, 10000.0)
+        np.testing.assert_allclose(got[n], want, rtol=1e-12, atol=1e-12)
+
+
+def test_rope_preserves_norm_and_identity_at_origin():
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((10, 2, 64))
+    pos = rng.integers(-50, 5000, size=(3, 10))
+    y = rope_rotate(x, *pos, (12, 10, 10), 10000.0)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-13)
+    z = rope_rotate(x, np.zeros(10), np.zeros(10), np.zeros(10), (12, 10, 10), 10000.0)
+    np.testing.assert_allclose(z, x, rtol=0, atol=0)
+
+
+def test_rope_relative_position_identity():
+    """R(a)^T R(b) = R(b - a): q(P) . k(p) depends only on P - p, per axis."""
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((1, 128))
+    k = rng.standard_normal((1, 128))
+    P = np.array([[40], [3], [9]])
+    p = np.array([[37], [5], [1]])
+    base = (rope_rotate(q, *P, PAIRS, 1e4) * rope_rotate(k, *p, PAIRS, 1e4)).sum()
+    for shift in ([100, 0, 0], [0, 7, -2], [29996, 11, 13]):
+        s = np.array(shift)[:, None]
+        moved = (rope_rotate(q, *(P + s), PAIRS, 1e4) * rope_rotate(k, *(p + s), PAIRS, 1e4)).sum()
+        assert abs(moved - base) < 1e-9 * max(1.0, abs(base))
+    # and equals q . R(p - P) k
+    rel = (q * rope_rotate(k, *(p - P), PAIRS, 1e4)).sum()
+    assert abs(rel - base) < 1e-10 * max(1.0, abs(base))
+
+
+def test_axis_frequencies_follow_theta_power_rule():
+    wt, wh, ww = axis_frequencies((22, 21, 21), 10000.0)
+    assert wt[0] == 1.0 and wh[0] == 1.0 and ww[0] == 1.0
+    np.testing.assert_allclose(wt[11] ** 2, 10000.0 ** (-1.0), rtol=1e-14)   # theta^(-11/22)
+    np.testing.assert_allclose(wh[7] ** 3, 10000.0 ** (-1.0), rtol=1e-14)    # theta^(-7/21)
+
+
+def test_block_positions_frame_major_then_row_then_column():
+    cfg = TINY.cfg.replace(grid_h=2, grid_w=3)
+    t, r, c = block_positions(cfg, 4)
+    assert list(t) == [12] * 6 + [13] * 6 + [14] * 6
+    assert list(r[:6]) == [0, 0, 0, 1, 1, 1]
+    assert list(c[:6]) == [0, 1, 2, 0, 1, 2]
+
+
+# ---------------------------------------------------------------------------
+# Rolling RoPE
+# ---------------------------------------------------------------------------
+def test_rolling_rope_keeps_sink_offset_constant_to_10000_blocks():
+    cfg = TINY.cfg
+    for b in range(0, 10001):
+        assert sink_temporal_position(cfg, b) - cfg.frames_per_block * b == -3
+    fixed = cfg.replace(rolling_rope=0)
+    assert sink_temporal_position(fixed, 10000) == -3
+
+
+def test_rolling_rope_sink_logits_identical_at_block_1_and_10000():
+    cfg = TINY.cfg.replace(head_dim=128, hidden=128, rope_split=PAIRS)
+    rng = np.random.default_rng(8)
+    qb = rng.standard_normal((cfg.block_tokens, 1, 128))
+    ks = rng.standard_normal((cfg.sink_tokens, 1, 128))
+
+    def logits(b):
+        q = rope_rotate(qb, *block_positions(cfg, b), cfg.pairs, cfg.rope_theta)
+        k = rope_rotate(ks, *sink_positions(cfg, sink_temporal_position(cfg, b)), cfg.pairs,
+                        cfg.rope_theta)
+        return q[:, 0] @ k[:, 0].T
+
+    np.testing.assert_allclose(logits(10000), logits(1), rtol=1e-9, atol=1e-9)
+    # without rolling the sink's distance grows and the logits differ
+    cfg_fixed = cfg.replace(rolling_rope=0)
+    q = rope_rotate(qb, *block_positions(cfg_fixed, 10000), cfg.pairs, cfg.rope_theta)
+    k = rope_rotate(ks, *sink_positions(cfg_fixed, -3), cfg.pairs, cfg.rope_theta)
+    assert np.abs(q[:, 0] @ k[:, 0].T - logits(1)).max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# flow matching
+# ---------------------------------------------------------------------------
+def test_constant_velocity_reproduces_straight_path_exactly():
+    rng = np.random.default_rng(9)
+    x0 = rng.standard_normal((48, 64))
+    x1 = rng.standard_normal((48, 64))
+    ts = TINY.cfg.timesteps
+    x = x1.copy()                 # t = 1
+    for i in range(len(ts) - 1):
+        x = euler_step(x, x1 - x0, ts[i], ts[i + 1])
+        np.testing.assert_allclose(x, ts[i + 1] * x1 + (1 - ts[i + 1]) * x0, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(x, x0, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# schedule, timestep forcing, AAS
+# ---------------------------------------------------------------------------
+def test_scheduler_closed_form_uninterrupted_stream():
+    cfg = TINY.cfg
+    sch = TickScheduler(cfg)
+    S, E, nw = cfg.num_steps, cfg.ring_entries, cfg.window_blocks
+    nb = 40
+    for k in range(nb + S - 1):
+        run, fin = sch.begin_tick(k < nb)
+        assert run == [(i, k - i) for i in range(S) if 0 <= k - i < nb]
+        assert fin == (k - S + 1 if k - S + 1 >= 0 else -1)
+        for i, b in run:
+            rec = sch.append(i, b)
+            assert rec[0] == b and rec[1] == b % E
+            assert rec[2] == (b - E if b >= E else -1)
+            assert rec[3] == 3 * b - 3 and rec[4] == 3 * b
+            resident = list(range(max(0, b - nw), b + 1))
+            assert rec[7] == len(resident) and rec[8:8 + len(resident)] == resident
+            assert sch.window_blocks(i, b) == resident[:-1]
+        sch.end_tick(fin)
+    assert sch.blocks_out == nb
+
+
+def test_timestep_forcing_every_cache_entry_holds_its_own_step():
+    wl = TINY
+    W = make_weights(wl)
+    s = OracleStream(wl.cfg, W)
+    s.set_sink(W.sink)
+    for k in range(wl.num_blocks + 3):
+        s.denoise_step(block_noise(wl, k) if k < wl.num_blocks else None)
+        for (l, i, b), (_, _, tag) in s.cache.items():
+            assert tag == (b, i)
+        for i in range(wl.cfg.num_steps):
+            for (blk, step) in s.sched.tags[i]:
+                assert blk == -1 or step == i
+
+
+def test_each_block_takes_exactly_nfe_forward_passes_and_sink_replaced_once():
+    facts = _facts()
+    wl = TINY
+    W = make_weights(wl)
+    s = OracleStream(wl.cfg, W, trace=True)
+    s.set_sink(W.sink)
+    gens = []
+    out0 = None
+    for k in range(wl.num_blocks + 3):
+        out, fin = s.denoise_step(block_noise(wl, k) if k < wl.num_blocks else None)
+        if fin == 0:
+            out0 = out
+        gens.append(s.sched.sink_generation)
+    passes = {}
+    for key in s.trace:
+        if isinstance(key[0], int):
+            passes[key[0]] = passes.get(key[0], 0) + 1
+    assert set(passes.values()) == {facts["nfe_per_block_no_refresh"]["value"]}
+    assert wl.cfg.frames_per_block == facts["frames_per_block"]["value"]
+    assert wl.cfg.num_steps == facts["pipeline_workers"]["value"]
+    # sink replaced once, right after block 0 finished (tick 3), never again
+    assert gens == [0, 0, 0, 1, 1, 1, 1, 1, 1]
+    assert gens.count(0) == 3 and sorted(set(gens)) == [0, facts["sink_replacements"]["value"]]
+    np.testing.assert_array_equal(s.sink_latent, out0[: wl.cfg.sink_tokens])
+
+
+def test_pipelined_order_equals_sequential_order_with_fixed_sink():
+    wl = Workload("t", TINY.cfg.replace(sink_mode=SINK_FIXED, num_layers=2), 3, 7, 0.125)
+    W = make_weights(wl)
+    outs = {}
+    for sched in (SCHED_PIPELINED, SCHED_SEQUENTIAL):
+        cfg = wl.cfg.replace(schedule=sched)
+        s = OracleStream(cfg, W)
+        s.set_sink(W.sink)
+        res = {}
+        n_calls = wl.num_blocks + (3 if sched == SCHED_PIPELINED else 0)
+        for k in range(n_calls):
+            out, fin = s.denoise_step(block_noise(wl, k) if k < wl.num_blocks else None)
+            if fin >= 0:
+                res[fin] = out
+        outs[sched] = res
+    assert sorted(outs[0]) == list(range(wl.num_blocks))
+    for b in range(wl.num_blocks):
+        np.testing.assert_array_equal(outs[SCHED_PIPELINED][b], outs[SCHED_SEQUENTIAL][b])
+
+
+def test_pipelined_differs_from_sequential_with_aas():
+    """The AAS sink reaches blocks 1-3 only for their later steps in pipelined order."""
+    wl = Workload("t", TINY.cfg.replace(sink_mode=SINK_AAS), 3, 5, 0.125)
+    W = make_weights(wl)
+    res = {}
+    for sched in (SCHED_PIPELINED, SCHED_SEQUENTIAL):
+        s = OracleStream(wl.cfg.replace(schedule=sched), W)
+        s.set_sink(W.sink)
+        got = {}
+        for k in range(wl.num_blocks + (3 if sched == SCHED_PIPELINED else 0)):
+            out, fin = s.denoise_step(block_noise(wl, k) if k < wl.num_blocks else None)
+            if fin >= 0:
+                got[fin] = out
+        res[sched] = got
+    np.testing.assert_array_equal(res[0][0], res[1][0])
+    assert np.abs(res[0][1] - res[1][1]).max() > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# closed forms of the whole step with special weights
+# ---------------------------------------------------------------------------
+def _special_weights(cfg, q_scale=0.0, k_scale=0.0, out_scale=1.0, sink=None):
+    D = cfg.hidden
+    wqkv = np.zeros((3 * D, D), np.float32)
+    wqkv[0:D] = np.eye(D) * q_scale
+    wqkv[D:2 * D] = np.eye(D) * k_scale
+    wqkv[2 * D:3 * D] = np.eye(D)
+    wout = np.eye(D, dtype=np.float32) * out_scale
+
+    class W:
+        pass
+    w = W()
+    w.w_qkv = [wqkv] * cfg.num_layers
+    w.w_out = [wout] * cfg.num_layers
+    w.w_in = None
+    w.w_head = None
+    w.sink = sink
+    return w
+
+
+def test_uniform_attention_closed_form_counts_the_visible_tokens():
+    """With W_q = W_k = 0, W_v = W_out = I and identity in/head projections the
+    layer adds the mean of the visible tokens' inputs, so one step gives
+    x' = x + dt (x + mean(sink_h, window inputs at this step, x))."""
+    cfg = TINY.cfg.replace(sink_mode=SINK_FIXED, window_blocks=2)
+    rng = np.random.default_rng(10)
+    sink = rng.standard_normal((cfg.sink_tokens, cfg.hidden)).astype(np.float32)
+    W = _special_weights(cfg, sink=sink)
+    s = OracleStream(cfg, W, trace=True)
+    s.set_sink(sink)
+    # the sink's own layer: uniform over itself, so sink h_1 = sink + mean(sink) (unused later)
+    np.testing.assert_allclose(s.sink_v[0].reshape(cfg.sink_tokens, -1), sink, atol=0)
+    nb = 6
+    for k in range(nb + 3):
+        s.denoise_step(block_noise(Workload("n", cfg, 5, nb, 0.1), k) if k < nb else None)
+    for (b, i), tr in [(key, v) for key, v in s.trace.items() if isinstance(key[0], int)]:
+        x = tr["x_in"]
+        toks = [sink] + [s.trace[(bb, i)]["x_in"] for bb in range(max(0, b - 2), b)] + [x]
+        mean = np.concatenate(toks).mean(axis=0)
+        dt = cfg.timesteps[i + 1] - cfg.timesteps[i]
+        np.testing.assert_allclose(tr["x_out"], x + dt * (x + mean[None, :]), rtol=1e-12, atol=1e-12)
+
+
+def test_oracle_stream_matches_scalar_brute_force_stream():
+    from _brute import BruteStream
+    cfg = StreamConfig(num_layers=2, hidden=16, heads=2, head_dim=8, latent_ch=16, grid_h=2,
+                       grid_w=2, window_blocks=1, rope_split=(2, 1, 1), sink_mode=SINK_AAS,
+                       dtype=1)
+    wl = Workload("brute", cfg, 11, 5, 0.25)
+    W = make_weights(wl)
+    noises = [block_noise(wl, b) for b in range(wl.num_blocks)]
+    bs = BruteStream(cfg, W)
+    bs.set_sink(W.sink)
+    want = bs.run_pipelined(noises)
+    s = OracleStream(cfg, W)
+    s.set_sink(W.sink)
+    for k in range(wl.num_blocks + 3):
+        out, fin = s.denoise_step(noises[k] if k < wl.num_blocks else None)
+        if fin >= 0:
+            np.testing.assert_allclose(out, np.array(want[fin]), rtol=1e-11, atol=1e-11)
+
+
+def test_oracle_stream_matches_brute_force_with_projections_and_no_rolling():
+    from _brute import BruteStream
+    cfg = StreamConfig(num_layers=1, hidden=16, heads=1, head_dim=16, latent_ch=4, grid_h=1,
+                       grid_w=3, window_blocks=2, rope_split=(4, 2, 2), sink_mode=SINK_FIXED,
+                       rolling_rope=0, timesteps=(1.0, 0.6, 0.2, 0.0), dtype=1)
+    wl = Workload("brute2", cfg, 12, 6, 0.3, head_std=0.3)
+    W = make_weights(wl)
+    noises = [block_noise(wl, b) for b in range(wl.num_blocks)]
+    bs = BruteStream(cfg, W)
+    bs.set_sink(W.sink)
+    want = bs.run_pipelined(noises)
+    s = OracleStream(cfg, W)
+    s.set_sink(W.sink)
+    for k in range(wl.num_blocks + cfg.num_steps - 1):
+        out, fin = s.denoise_step(noises[k] if k < wl.num_blocks else None)
+        if fin >= 0:
+            np.testing.assert_allclose(out, np.array(want[fin]), rtol=1e-11, atol=1e-11)
