@@ -1,0 +1,272 @@
+/*
+ * la_stream.h -- C ABI of the timestep-forced streaming denoising step.
+ *
+ * The operation is the streaming generator step of Live Avatar (arXiv
+ * 2512.04677) as the pages describe it:
+ *   - blocks of 3 latent frames advance autoregressively under a block-causal
+ *     mask (papernotes.org ECCV2026 note, 整体框架; 10100.com article,
+ *     training-framework caption);
+ *   - the KV cache keeps the noisy K/V of the step that produced them and is
+ *     never refreshed by a clean forward (papernotes note, 关键设计 2 "History
+ *     Corrupt"; gitcode blog, question 4);
+ *   - every denoising step t_i has its own cache (timestep forcing) and the 4
+ *     steps of 4 consecutive blocks run as a pipeline (papernotes note,
+ *     关键设计 4 "TPP"; 10100.com article, TPP caption).  On one GPU the 4
+ *     pipeline stages run as one grouped launch per tick;
+ *   - the sink frame is re-offset in RoPE time each block so its distance to
+ *     the active block stays constant (Rolling RoPE, papernotes note 关键设计 3)
+ *     and is replaced once by the first generated latent (Adaptive Attention
+ *     Sink, papernotes note 关键设计 3; gitcode blog question 5);
+ *   - each step ends with the flow-matching Euler update
+ *     x_{t_{i+1}} = x_{t_i} + (t_{i+1} - t_i) v (papernotes note, 损失函数).
+ *
+ * Conventions for every function:
+ *   - Return value: LA_OK (0) or a negative LA_E* status.  No C++ exception
+ *     crosses this boundary.  la_last_error() gives a text for the last
+ *     failure of a stream.
+ *   - "device" pointers are CUDA device memory of the stream's device;
+ *     "host" pointers are CPU memory (pinned memory makes copies asynchronous).
+ *   - Work is enqueued asynchronously on the CUDA stream given at creation;
+ *     host-side state (tick counter, ring indices, finished block id) is
+ *     updated synchronously.  la_synchronize() waits and reports device-side
+ *     errors (LA_EDEVICE) raised by bounded waits inside the kernels.
+ *   - The caller owns inputs, outputs and weights; the library owns the ring
+ *     caches, the sink buffers, scratch and the tick state.
+ *   - There is no CPU fallback: without a usable sm_100 device creation fails
+ *     with LA_ECUDA.
+ */
+#ifndef LA_STREAM_H
+#define LA_STREAM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define LA_OK        0
+#define LA_EINVAL   -1   /* bad argument or configuration                   */
+#define LA_ESTATE   -2   /* call not valid in the stream's current state    */
+#define LA_ENOMEM   -3   /* device memory would not fit (checked up front)  */
+#define LA_ECUDA    -4   /* a CUDA runtime / driver call failed             */
+#define LA_EDEVICE  -5   /* a kernel raised the device error word           */
+
+/* ---- enums ------------------------------------------------------------- */
+#define LA_SINK_FIXED        0  /* reference sink kept for the whole stream           */
+#define LA_SINK_AAS          1  /* sink replaced once by frame 0 of finished block 0  */
+#define LA_SCHED_PIPELINED   0  /* one call = one tick: slot i runs step i of block k-i */
+#define LA_SCHED_SEQUENTIAL  1  /* one call = one block through all steps in order     */
+#define LA_BF16              0  /* bf16 weights/activations, fp32 accumulate, fp32 x   */
+#define LA_FP32              1  /* fp32 everywhere (SIMT path, no TF32)                */
+
+/* Limits of this build. */
+#define LA_MAX_STEPS     8
+#define LA_MAX_WINDOW   14
+#define LA_MAX_FPB       7
+
+/*
+ * Stream configuration.  D = heads*head_dim, F = grid_h*grid_w tokens per
+ * latent frame, T_b = frames_per_block*F tokens per block.
+ */
+typedef struct la_config {
+  int32_t num_layers;          /* >= 1 attention sublayers                               */
+  int32_t hidden;              /* D; must equal heads*head_dim                           */
+  int32_t heads;               /* H                                                      */
+  int32_t head_dim;            /* d; bf16 path: 128; fp32 path: even, <= 128             */
+  int32_t latent_ch;           /* C; C == D with NULL w_in/w_head means identity maps   */
+  int32_t grid_h, grid_w;      /* latent frame token grid                                */
+  int32_t frames_per_block;    /* 3 on the pages; 1..LA_MAX_FPB                          */
+  int32_t sink_frames;         /* 1 (only value supported)                               */
+  int32_t window_blocks;       /* N_w: prior blocks each timestep slot keeps, 0..LA_MAX_WINDOW */
+  int32_t num_steps;           /* S: timestep slots, 1..LA_MAX_STEPS                      */
+  const float* timesteps;      /* HOST, num_steps+1 values, strictly descending, finite;
+                                  step i integrates from timesteps[i] to timesteps[i+1].
+                                  Copied at creation.                                    */
+  int32_t rope_split[3];       /* rotary PAIRS for (t, h, w); sum == head_dim/2         */
+  double  rope_theta;          /* > 0, e.g. 10000                                        */
+  int32_t sink_mode;           /* LA_SINK_FIXED | LA_SINK_AAS                            */
+  int32_t rolling_rope;        /* 1: sink t-pos = frames_per_block*b - sink_offset_frames;
+                                  0: fixed at -sink_offset_frames                         */
+  int32_t sink_offset_frames;  /* 3                                                      */
+  int32_t schedule;            /* LA_SCHED_PIPELINED | LA_SCHED_SEQUENTIAL               */
+  int32_t dtype;               /* LA_BF16 | LA_FP32                                      */
+} la_config;
+
+/*
+ * Weights: DEVICE pointers, BORROWED (they must outlive the stream and must
+ * not change while it exists).  Element type = config dtype (bf16 or fp32).
+ * Layout [out_features, in_features], row-major, i.e. y = x W^T.
+ */
+typedef struct la_weights {
+  const void* w_in;              /* [D, C] or NULL (identity; needs C == D)     */
+  const void* w_head;            /* [C, D] or NULL (identity; needs C == D)     */
+  const void* const* w_qkv;      /* HOST array of num_layers DEVICE pointers, each [3D, D];
+                                    rows 0..D-1 give q, D..2D-1 k, 2D..3D-1 v; head h
+                                    owns rows h*d .. h*d+d-1 of each part        */
+  const void* const* w_out;      /* HOST array of num_layers DEVICE pointers, each [D, D] */
+} la_weights;
+
+typedef struct la_stream la_stream;
+
+/*
+ * Create a stream on the current CUDA device.  cuda_stream is a cudaStream_t
+ * (NULL = legacy default stream).  Allocates every buffer up front after a
+ * cudaMemGetInfo check (LA_ENOMEM if it would not fit).  *out is set to NULL
+ * on failure.  LA_EINVAL: invalid config (sizes <= 0, hidden != heads*head_dim,
+ * head_dim unsupported for the dtype, timesteps not strictly descending,
+ * window out of range, rope_split not summing to head_dim/2, NULL weights).
+ */
+int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_stream,
+                     la_stream** out);
+
+/*
+ * Set the reference sink: DEVICE fp32 [sink_frames*F, C].  Runs the sink
+ * frame through the layers (self-attention over the sink only, RoPE time
+ * -sink_offset_frames) and stores, per layer, the un-roped sink K and the
+ * sink V shared by all slots.  Must precede the first la_denoise_step; may
+ * only be called before it (LA_ESTATE afterwards).
+ */
+int la_set_sink(la_stream* s, const float* sink_latent);
+
+/*
+ * One call.  Pipelined schedule: one tick.  x_new (DEVICE fp32 [T_b, C]) is
+ * the noise of the next block at timesteps[0]; it enters slot 0.  NULL drains
+ * the pipeline (no new block).  Every in-flight block advances one step in
+ * its slot.  If the block in the last slot finishes, its latent is copied to
+ * x_out (DEVICE fp32 [T_b, C]) and its id is written to *finished_block
+ * (HOST), else *finished_block = -1 and x_out is untouched.
+ * Sequential schedule: x_new must be non-NULL; the block runs all steps in
+ * order and always finishes.
+ * When the sink mode is LA_SINK_AAS and block 0 finishes, frame 0 of its
+ * latent becomes the sink for every later step (once per stream).
+ * LA_ESTATE before la_set_sink; LA_EINVAL for NULL x_out / finished_block or
+ * a NULL x_new in the sequential schedule.
+ */
+int la_denoise_step(la_stream* s, const float* x_new, float* x_out, int64_t* finished_block);
+
+/* Same as la_denoise_step with HOST x_new / x_out: the host->device copy of
+ * the new block and the device->host copy of the finished block are enqueued
+ * on the stream (asynchronous if the host memory is pinned); the call returns
+ * after enqueueing, so read x_out only after la_synchronize(). */
+int la_denoise_step_host(la_stream* s, const float* x_new_host, float* x_out_host,
+                         int64_t* finished_block);
+
+/* Wait for all work of the stream; LA_EDEVICE if a kernel raised the device
+ * error word (the word is cleared after being reported). */
+int la_synchronize(la_stream* s);
+
+/* Free everything.  NULL is a no-op.  The pointer is invalid afterwards. */
+int la_stream_destroy(la_stream* s);
+
+/* Text of the last error on s (never NULL; "" if none); static text if s is NULL. */
+const char* la_last_error(const la_stream* s);
+const char* la_status_string(int status);
+
+/* ---- debug / test exports ------------------------------------------------ */
+
+/* Number of int32 values of the index state (see la_get_index_state). */
+int64_t la_index_state_size(const la_stream* s);
+
+/*
+ * Integer state after the last call, HOST buffer of n >= la_index_state_size
+ * int32: header [tick, blocks_in, blocks_out, sink_generation] then, for each
+ * slot i < num_steps, E = window_blocks+1 and R = 8 + 3E values:
+ *   [active_block, write_entry, evicted_block, sink_tpos, frame_tpos,
+ *    sink_generation_used, step_index, n_resident,
+ *    resident[E] (oldest -> newest, -1 padded), tags[E] x (block, step)].
+ * active_block/write_entry/evicted_block are -1 and sink_tpos/frame_tpos/
+ * sink_generation_used are 0 for a slot that was idle in the last call.
+ */
+int la_get_index_state(const la_stream* s, int32_t* host_buf, int64_t n);
+
+/* Enable (1) / disable (0) capture of per-slot intermediates for la_debug_tap.
+ * Allocates capture buffers on enable. */
+int la_debug_capture(la_stream* s, int32_t enable);
+
+#define LA_TAP_X_IN      0  /* fp32 [T_b, C]   latent the slot's last step started from        */
+#define LA_TAP_X_OUT     1  /* fp32 [T_b, C]   latent after the slot's last step               */
+#define LA_TAP_H         2  /* fp32 [T_b, D]   residual after layer `layer` (-1: after in-proj) */
+#define LA_TAP_Q         3  /* dtype [H, T_b, d] roped queries of layer                          */
+#define LA_TAP_O         4  /* dtype [T_b, D]   attention output of layer                        */
+#define LA_TAP_V         5  /* fp32 [T_b, C]    velocity of the slot's last step                 */
+#define LA_TAP_RING_K    6  /* dtype [E, H, T_b, d] ring K of (layer, slot), by entry            */
+#define LA_TAP_RING_V    7  /* dtype [E, H, T_b, d] ring V of (layer, slot)                      */
+#define LA_TAP_SINK_K    8  /* dtype [H, F, d] un-roped sink K of layer (slot ignored)           */
+#define LA_TAP_SINK_V    9  /* dtype [H, F, d] sink V of layer (slot ignored)                    */
+#define LA_TAP_SINK_KROPE 10 /* dtype [H, F, d] sink K as roped for the slot's last step         */
+
+/* Copy one tapped tensor into dst (DEVICE, dst_bytes >= the tensor's size),
+ * ordered on the stream.  Taps other than ring / sink need capture enabled
+ * before the call being inspected.  LA_EINVAL on bad what/layer/slot/size. */
+int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* dst,
+                 int64_t dst_bytes);
+
+/* Overwrite the latent that `slot` will start its next step from (DEVICE fp32
+ * [T_b, C]).  Slot 0 of the pipelined schedule is fed by x_new instead.
+ * Used to inject fresh per-step inputs in soak tests.  LA_ESTATE if the slot
+ * will be idle in the next tick. */
+int la_debug_set_slot_input(la_stream* s, int32_t slot, const float* x);
+
+/* Kernel timing with CUDA events on the stream.  kind: LA_KIND_*. */
+#define LA_KIND_IN_PROJ   0
+#define LA_KIND_QKV_GEMM  1
+#define LA_KIND_ROPE      2
+#define LA_KIND_ATTN      3
+#define LA_KIND_OUT_GEMM  4
+#define LA_KIND_HEAD      5
+#define LA_KIND_OTHER     6
+#define LA_NUM_KINDS      7
+int la_profile_enable(la_stream* s, int32_t enable);   /* resets the counters */
+int la_profile_read(la_stream* s, int32_t kind, int64_t* launches, double* total_ms);
+/* Kernels launched by this stream since creation. */
+int64_t la_launch_count(const la_stream* s);
+
+/* ---- op-level entry points (unit tests, microbenchmarks) ------------------
+ * Each enqueues one kernel on cuda_stream (a cudaStream_t, NULL = default).
+ * They allocate nothing except where stated.
+ */
+
+/*
+ * C = A W^T with an epilogue.  A: DEVICE [M, K] row-major, W: DEVICE [N, K]
+ * row-major, both of `dtype` (bf16 path: tcgen05 tensor cores, fp32
+ * accumulate; fp32 path: SIMT fp32).  K % 8 == 0 for bf16.
+ *   LA_EPI_STORE:   out (dtype [M, N]) = acc
+ *   LA_EPI_RESID:   h32 (fp32 [M, N]) += acc; out (dtype [M, N]) = h32
+ *   LA_EPI_SET32:   h32 = acc; out (dtype [M, N]) = acc   (out may be NULL)
+ *   LA_EPI_EULER:   h32[m, n] += dt[m / rows_per_group] * acc (the Euler update;
+ *                   dt: HOST array of ceil(M/rows_per_group) floats, <= LA_MAX_STEPS)
+ * For LA_FP32 "out" of RESID/SET32 may alias h32.
+ */
+#define LA_EPI_STORE  0
+#define LA_EPI_RESID  1
+#define LA_EPI_SET32  2
+#define LA_EPI_EULER  3
+int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, void* out,
+               float* h32, int64_t M, int64_t N, int64_t K, const float* dt,
+               int64_t rows_per_group, void* cuda_stream);
+
+/*
+ * Block attention over a list of KV segments for one group of Tq queries:
+ * O[t, h*d + e] = sum_j softmax_j(q_h[t] . k_h[j] / sqrt(d)) v_h[j][e] over the
+ * concatenation of the segments (every key visible; the block-causal mask is
+ * expressed by which segments are passed).  q: DEVICE [H, Tq, d]; segment s:
+ * k_seg[s], v_seg[s] DEVICE [H, seg_len[s], d] (HOST arrays of nseg pointers /
+ * lengths, 1 <= nseg <= LA_MAX_WINDOW + 2, seg_len >= 1); out DEVICE [Tq, H*d].
+ * dtype LA_BF16 needs d == 128 (tcgen05), LA_FP32 any even d <= 128.
+ */
+int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t d,
+                    int32_t nseg, const void* const* k_seg, const void* const* v_seg,
+                    const int64_t* seg_len, void* out, void* cuda_stream);
+
+/*
+ * Standalone Euler update x[r, :] += dt[r / rows_per_group] * v[r, :] over
+ * `rows` rows of C fp32 values (DEVICE x, v); dt HOST, <= LA_MAX_STEPS groups.
+ */
+int la_op_euler(float* x, const float* v, int64_t rows, int64_t C, const float* dt,
+                int64_t rows_per_group, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LA_STREAM_H */

@@ -121,10 +121,11 @@ class OracleStream:
         return x_next
 
     # -- one call of the C-ABI's la_denoise_step ---------------------------------
-    def denoise_step(self, x_new=None, inputs=None):
+    def denoise_step(self, x_new=None, inputs=None, aas_latent=None):
         """x_new: noise of the next block (or None to drain).  inputs: optional
-        {(block, step): latent} overriding the latent a step starts from
-        (teacher forcing).  Returns (finished latent or None, finished id)."""
+        {(block, step): latent} overriding the latent a step starts from, and
+        aas_latent: optional finished latent of block 0 to take the new sink
+        from (teacher forcing).  Returns (finished latent or None, finished id)."""
         if self.sink_k is None:
             raise RuntimeError("set_sink first")
         has_new = x_new is not None
@@ -140,7 +141,8 @@ class OracleStream:
         if finished >= 0:
             out = self.latents.pop(finished)
         if self.sched.end_tick(finished):
-            self.set_sink(out[: self.cfg.sink_tokens])
+            src = out if aas_latent is None else np.asarray(aas_latent, np.float64)
+            self.set_sink(src[: self.cfg.sink_tokens])
         return out, finished
 
     def index_state(self):

@@ -1,0 +1,100 @@
+"""ctypes declarations of the C ABI in include/la_stream.h (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_double, c_float, c_int, c_int32, c_int64, c_void_p
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libla.so")
+
+LA_OK, LA_EINVAL, LA_ESTATE, LA_ENOMEM, LA_ECUDA, LA_EDEVICE = 0, -1, -2, -3, -4, -5
+LA_SINK_FIXED, LA_SINK_AAS = 0, 1
+LA_SCHED_PIPELINED, LA_SCHED_SEQUENTIAL = 0, 1
+LA_BF16, LA_FP32 = 0, 1
+LA_MAX_STEPS, LA_MAX_WINDOW, LA_MAX_FPB = 8, 14, 7
+LA_EPI_STORE, LA_EPI_RESID, LA_EPI_SET32, LA_EPI_EULER = 0, 1, 2, 3
+
+TAP = dict(x_in=0, x_out=1, h=2, q=3, o=4, v=5, ring_k=6, ring_v=7, sink_k=8, sink_v=9, sink_k_rope=10)
+KIND = dict(in_proj=0, qkv_gemm=1, rope=2, attn=3, out_gemm=4, head=5, other=6)
+
+
+class LaConfig(ctypes.Structure):
+    _fields_ = [
+        ("num_layers", c_int32), ("hidden", c_int32), ("heads", c_int32), ("head_dim", c_int32),
+        ("latent_ch", c_int32), ("grid_h", c_int32), ("grid_w", c_int32), ("frames_per_block", c_int32),
+        ("sink_frames", c_int32), ("window_blocks", c_int32), ("num_steps", c_int32),
+        ("timesteps", POINTER(c_float)), ("rope_split", c_int32 * 3), ("rope_theta", c_double),
+        ("sink_mode", c_int32), ("rolling_rope", c_int32), ("sink_offset_frames", c_int32),
+        ("schedule", c_int32), ("dtype", c_int32),
+    ]
+
+
+class LaWeights(ctypes.Structure):
+    _fields_ = [("w_in", c_void_p), ("w_head", c_void_p), ("w_qkv", POINTER(c_void_p)),
+                ("w_out", POINTER(c_void_p))]
+
+
+class LaError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{msg} (status {code})")
+        self.code = code
+
+
+_lib = None
+
+
+def load():
+    """Load libla.so; raises if it is missing (there is no fallback path)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} not built: run python -m streaming_causal_video_timestep_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "la_stream_create": (c_int, [POINTER(LaConfig), POINTER(LaWeights), c_void_p, POINTER(c_void_p)]),
+        "la_set_sink": (c_int, [c_void_p, c_void_p]),
+        "la_denoise_step": (c_int, [c_void_p, c_void_p, c_void_p, POINTER(c_int64)]),
+        "la_denoise_step_host": (c_int, [c_void_p, c_void_p, c_void_p, POINTER(c_int64)]),
+        "la_synchronize": (c_int, [c_void_p]),
+        "la_stream_destroy": (c_int, [c_void_p]),
+        "la_last_error": (c_char_p, [c_void_p]),
+        "la_status_string": (c_char_p, [c_int]),
+        "la_index_state_size": (c_int64, [c_void_p]),
+        "la_get_index_state": (c_int, [c_void_p, POINTER(c_int32), c_int64]),
+        "la_debug_capture": (c_int, [c_void_p, c_int32]),
+        "la_debug_tap": (c_int, [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_int64]),
+        "la_debug_set_slot_input": (c_int, [c_void_p, c_int32, c_void_p]),
+        "la_profile_enable": (c_int, [c_void_p, c_int32]),
+        "la_profile_read": (c_int, [c_void_p, c_int32, POINTER(c_int64), POINTER(c_double)]),
+        "la_launch_count": (c_int64, [c_void_p]),
+        "la_op_gemm": (c_int, [c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64,
+                               c_int64, POINTER(c_float), c_int64, c_void_p]),
+        "la_op_attention": (c_int, [c_int32, c_void_p, c_int64, c_int32, c_int32, c_int32, POINTER(c_void_p),
+                                    POINTER(c_void_p), POINTER(c_int64), c_void_p, c_void_p]),
+        "la_op_euler": (c_int, [c_void_p, c_void_p, c_int64, c_int64, POINTER(c_float), c_int64, c_void_p]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def exported_symbols():
+    """Names of the C-ABI functions declared in include/la_stream.h."""
+    return [
+        "la_stream_create", "la_set_sink", "la_denoise_step", "la_denoise_step_host", "la_synchronize",
+        "la_stream_destroy", "la_last_error", "la_status_string", "la_index_state_size", "la_get_index_state",
+        "la_debug_capture", "la_debug_tap", "la_debug_set_slot_input", "la_profile_enable", "la_profile_read",
+        "la_launch_count", "la_op_gemm", "la_op_attention", "la_op_euler",
+    ]
+
+
+def check(code, handle=None):
+    if code != LA_OK:
+        lib = load()
+        msg = lib.la_last_error(handle).decode() if handle else lib.la_status_string(code).decode()
+        raise LaError(code, msg or lib.la_status_string(code).decode())

@@ -1,0 +1,83 @@
+// Internal definitions shared by the kernels and the host library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "la_stream.h"
+
+#define LA_MAX_SEG (LA_MAX_WINDOW + 2)
+#define LA_MAX_PT 64          // temporal rotary pairs (head_dim <= 128)
+#define LA_TROWS (LA_MAX_FPB + 1)
+
+// Device error word codes (first error wins).
+#define LA_DEVERR_WAIT_TIMEOUT 1
+#define LA_DEVERR_BAD_DESC     2
+
+// Per-pass description of the buffers: which blocks the grouped launch
+// processes, in which timestep slot, and where their cache entries live.
+struct PassDesc {
+  int nbuf;                          // buffers covered by the row range (rows = nbuf*T)
+  int nactive;                       // active buffers, listed in active_buf
+  int active_buf[LA_MAX_STEPS];
+  int active[LA_MAX_STEPS];          // per buffer: 1 if it runs a step this pass
+  int slot[LA_MAX_STEPS];            // timestep slot of the buffer's block
+  int block[LA_MAX_STEPS];
+  int write_entry[LA_MAX_STEPS];     // ring entry the block's K/V go to
+  int nwin[LA_MAX_STEPS];            // prior blocks read, oldest first
+  int win_entry[LA_MAX_STEPS][LA_MAX_WINDOW];
+  int frame_tpos[LA_MAX_STEPS];      // RoPE time of the block's frame 0
+  int sink_tpos[LA_MAX_STEPS];       // RoPE time of the sink for this block
+  float dt[LA_MAX_STEPS];            // t_{i+1} - t_i of the buffer's slot
+};
+
+// One KV segment for attention: K from map kmap, V from map vmap (indices into
+// the kernel's map arrays), each a stack of [H, rows, d] planes.
+struct AttnSeg {
+  int kmap, vmap;
+  int kslice, vslice;   // outermost coordinate in the map (which [H, rows, d] plane)
+  int len;              // keys
+};
+
+struct AttnGroup {
+  int nseg;
+  AttnSeg seg[LA_MAX_SEG];
+  int q_slice;          // slice of the q map
+  int out_row0;         // first output row of this group
+};
+
+#define LA_MAX_GROUPS LA_MAX_STEPS
+
+struct AttnParams {
+  int ngroups;
+  AttnGroup g[LA_MAX_GROUPS];
+  int Tq;               // queries per group
+  int H, d;
+  float scale_log2;     // log2(e) / sqrt(d)
+  void* out;            // [rows, H*d] dtype
+  long long out_ld;     // elements per output row
+  int* err;
+  // raw pointers for the SIMT path: element offset of (slice, h, n, e) is
+  // ((slice*H + h)*rows + n)*d + e, rows = krows/vrows[m] (q: Tq)
+  const void* qbase;
+  const void* kbase[LA_MAX_SEG];
+  const void* vbase[LA_MAX_SEG];
+  int krows[LA_MAX_SEG];
+  int vrows[LA_MAX_SEG];
+};
+
+enum GemmEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SET32 = 2, EPI_EULER = 3 };
+
+struct GemmEpiParams {
+  int kind;
+  void* out;            // dtype [M, N]
+  float* h32;           // fp32 [M, N]
+  long long ld;         // N
+  int rows_per_group;   // EULER: rows of one buffer
+  float dt[LA_MAX_STEPS];
+  int active[LA_MAX_STEPS];   // EULER: only active groups update
+  float* vtap;          // optional fp32 [M, N] copy of acc (velocity capture)
+};
+
+static inline int ceil_div_i(long long a, long long b) { return (int)((a + b - 1) / b); }

@@ -1,0 +1,273 @@
+// Bandwidth-bound kernels: RoPE tables, fused Rolling RoPE + ring append +
+// sink re-rope, the sink's K/V split, in-projection helpers and the Euler update.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace {
+
+template <typename T> struct Vec8;
+template <> struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(b[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
+    uint4 w;
+    w.x = pack_bf16x2(v[0], v[1]);
+    w.y = pack_bf16x2(v[2], v[3]);
+    w.z = pack_bf16x2(v[4], v[5]);
+    w.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = w;
+  }
+};
+template <> struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0];
+    const float4 b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+};
+
+// Rotate the 4 pairs of an 8-element chunk; pair j = 4*ch + jj.
+__device__ __forceinline__ void rotate8(float (&v)[8], int ch, int buf, int trow, int rr, int cc,
+                                        const RopeArgs& a) {
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    const int j = 4 * ch + jj;
+    float c, s;
+    if (j < a.pt) {
+      const int idx = (buf * LA_TROWS + trow) * LA_MAX_PT + j;
+      c = a.tcos[idx];
+      s = a.tsin[idx];
+    } else if (j < a.pt + a.ph) {
+      const int idx = rr * a.ph + (j - a.pt);
+      c = a.rcos[idx];
+      s = a.rsin[idx];
+    } else {
+      const int idx = cc * a.pw + (j - a.pt - a.ph);
+      c = a.ccos[idx];
+      s = a.csin[idx];
+    }
+    const float x0 = v[2 * jj], x1 = v[2 * jj + 1];
+    v[2 * jj] = x0 * c - x1 * s;
+    v[2 * jj + 1] = x0 * s + x1 * c;
+  }
+}
+
+__global__ void k_rope_ttab(const __grid_constant__ PassDesc pd, int fpb, int pt, const double* __restrict__ omega,
+                            float* tcos, float* tsin) {
+  const int rows = fpb + 1;
+  const int per_buf = rows * pt;
+  for (int i = threadIdx.x; i < pd.nactive * per_buf; i += blockDim.x) {
+    const int ai = i / per_buf, rem = i % per_buf;
+    const int f = rem / pt, j = rem % pt;
+    const int buf = pd.active_buf[ai];
+    const int pos = f < fpb ? pd.frame_tpos[buf] + f : pd.sink_tpos[buf];
+    double s, c;
+    sincos(static_cast<double>(pos) * omega[j], &s, &c);
+    const int idx = (buf * LA_TROWS + f) * LA_MAX_PT + j;
+    tcos[idx] = static_cast<float>(c);
+    tsin[idx] = static_cast<float>(s);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_rope_append(const __grid_constant__ PassDesc pd,
+                                                     const __grid_constant__ RopeArgs a, long long n_main,
+                                                     long long n_sink) {
+  const int chunks = a.d / 8;
+  const T* qkv = reinterpret_cast<const T*>(a.qkv);
+  const long long total = n_main + n_sink;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    if (idx < n_main) {
+      long long rest = idx;
+      const int ch = static_cast<int>(rest % chunks); rest /= chunks;
+      const int h = static_cast<int>(rest % a.H); rest /= a.H;
+      const int part = static_cast<int>(rest % 3); rest /= 3;
+      const int n = static_cast<int>(rest % a.T); rest /= a.T;
+      const int buf = pd.active_buf[rest];
+      const long long row = static_cast<long long>(buf) * a.T + n;
+      float v[8];
+      Vec8<T>::load(qkv + row * 3 * a.D + part * a.D + h * a.d + ch * 8, v);
+      if (part < 2) {
+        const int f = n / a.F, rem = n % a.F;
+        rotate8(v, ch, buf, f, rem / a.grid_w, rem % a.grid_w, a);
+      }
+      T* dst;
+      const long long tok = static_cast<long long>(n) * a.d + ch * 8;
+      if (part == 0) {
+        dst = reinterpret_cast<T*>(a.q_rope) + (static_cast<long long>(buf) * a.H + h) * a.T * a.d + tok;
+      } else {
+        const long long slice = a.ring_slice0 + static_cast<long long>(pd.slot[buf]) * a.E + pd.write_entry[buf];
+        T* base = reinterpret_cast<T*>(part == 1 ? a.ring_k : a.ring_v);
+        dst = base + (slice * a.H + h) * a.T * a.d + tok;
+      }
+      Vec8<T>::store(dst, v);
+    } else {
+      long long rest = idx - n_main;
+      const int ch = static_cast<int>(rest % chunks); rest /= chunks;
+      const int m = static_cast<int>(rest % a.F); rest /= a.F;
+      const int h = static_cast<int>(rest % a.H); rest /= a.H;
+      const int buf = pd.active_buf[rest];
+      const long long off = (static_cast<long long>(h) * a.F + m) * a.d + ch * 8;
+      float v[8];
+      Vec8<T>::load(reinterpret_cast<const T*>(a.sink_k) + off, v);
+      rotate8(v, ch, buf, a.fpb, m / a.grid_w, m % a.grid_w, a);
+      Vec8<T>::store(reinterpret_cast<T*>(a.sink_k_rope) + static_cast<long long>(buf) * a.H * a.F * a.d + off, v);
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_sink_qkv(const __grid_constant__ RopeArgs a, T* sink_k_raw, T* sink_v,
+                                                  T* q_rope, T* k_rope) {
+  const int chunks = a.d / 8;
+  const long long total = static_cast<long long>(a.F) * 3 * a.H * chunks;
+  const T* qkv = reinterpret_cast<const T*>(a.qkv);
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    long long rest = idx;
+    const int ch = static_cast<int>(rest % chunks); rest /= chunks;
+    const int h = static_cast<int>(rest % a.H); rest /= a.H;
+    const int part = static_cast<int>(rest % 3); rest /= 3;
+    const int m = static_cast<int>(rest);
+    float v[8];
+    Vec8<T>::load(qkv + static_cast<long long>(m) * 3 * a.D + part * a.D + h * a.d + ch * 8, v);
+    const long long off = (static_cast<long long>(h) * a.F + m) * a.d + ch * 8;
+    if (part == 2) {
+      Vec8<T>::store(sink_v + off, v);
+      continue;
+    }
+    if (part == 1) Vec8<T>::store(sink_k_raw + off, v);
+    rotate8(v, ch, 0, 0, m / a.grid_w, m % a.grid_w, a);
+    Vec8<T>::store(part == 0 ? q_rope + off : k_rope + off, v);
+  }
+}
+
+template <typename T>
+__global__ void k_in_identity(const float* __restrict__ x, float* __restrict__ h32, T* __restrict__ hop, long long n) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float v = x[i];
+    h32[i] = v;
+    if (hop) hop[i] = static_cast<T>(v);
+  }
+}
+
+__global__ void k_cvt_bf16(const float* __restrict__ x, __nv_bfloat16* __restrict__ xb, long long n) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    xb[i] = __float2bfloat16_rn(x[i]);
+}
+
+struct EulerArgs {
+  float dt[LA_MAX_STEPS];
+  int active[LA_MAX_STEPS];
+};
+
+// x += dt * v, float4 vectors; C % 4 == 0.
+__global__ void __launch_bounds__(256) k_euler(float* __restrict__ x, const float* __restrict__ v, long long n4,
+                                               long long C4, long long rows_per_group,
+                                               const __grid_constant__ EulerArgs e, float* __restrict__ vtap) {
+  float4* x4 = reinterpret_cast<float4*>(x);
+  const float4* v4 = reinterpret_cast<const float4*>(v);
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int g = static_cast<int>((i / C4) / rows_per_group);
+    if (!e.active[g]) continue;
+    const float dt = e.dt[g];
+    const float4 vv = v4[i];
+    float4 xx = x4[i];
+    xx.x += dt * vv.x;
+    xx.y += dt * vv.y;
+    xx.z += dt * vv.z;
+    xx.w += dt * vv.w;
+    x4[i] = xx;
+    if (vtap) reinterpret_cast<float4*>(vtap)[i] = vv;
+  }
+}
+
+int grid_for(long long n, int per_block = 256) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  long long blocks = (n + per_block - 1) / per_block;
+  const long long cap = static_cast<long long>(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return static_cast<int>(blocks);
+}
+
+}  // namespace
+
+cudaError_t launch_rope_ttab(const PassDesc& pd, int fpb, int pt, const double* omega_t, float* tcos, float* tsin,
+                             cudaStream_t st) {
+  if (pt <= 0 || pd.nactive <= 0) return cudaSuccess;
+  k_rope_ttab<<<1, 256, 0, st>>>(pd, fpb, pt, omega_t, tcos, tsin);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_append(int bf16, const PassDesc& pd, const RopeArgs& a, cudaStream_t st) {
+  const long long chunks = a.d / 8;
+  const long long n_main = static_cast<long long>(pd.nactive) * a.T * 3 * a.H * chunks;
+  const long long n_sink = a.sink_k ? static_cast<long long>(pd.nactive) * a.F * a.H * chunks : 0;
+  const int grid = grid_for(n_main + n_sink);
+  if (bf16)
+    k_rope_append<__nv_bfloat16><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
+  else
+    k_rope_append<float><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sink_qkv(int bf16, const RopeArgs& a, void* sink_k_raw, void* sink_v, void* q_rope, void* k_rope,
+                            cudaStream_t st) {
+  const long long n = static_cast<long long>(a.F) * 3 * a.H * (a.d / 8);
+  const int grid = grid_for(n);
+  if (bf16)
+    k_sink_qkv<__nv_bfloat16><<<grid, 256, 0, st>>>(a, static_cast<__nv_bfloat16*>(sink_k_raw),
+                                                     static_cast<__nv_bfloat16*>(sink_v),
+                                                     static_cast<__nv_bfloat16*>(q_rope),
+                                                     static_cast<__nv_bfloat16*>(k_rope));
+  else
+    k_sink_qkv<float><<<grid, 256, 0, st>>>(a, static_cast<float*>(sink_k_raw), static_cast<float*>(sink_v),
+                                            static_cast<float*>(q_rope), static_cast<float*>(k_rope));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_in_identity(int bf16, const float* x, float* h32, void* hop, long long n, cudaStream_t st) {
+  const int grid = grid_for(n);
+  if (bf16)
+    k_in_identity<__nv_bfloat16><<<grid, 256, 0, st>>>(x, h32, static_cast<__nv_bfloat16*>(hop), n);
+  else
+    k_in_identity<float><<<grid, 256, 0, st>>>(x, h32, hop == h32 ? nullptr : static_cast<float*>(hop), n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cvt_bf16(const float* x, void* xb, long long n, cudaStream_t st) {
+  k_cvt_bf16<<<grid_for(n), 256, 0, st>>>(x, static_cast<__nv_bfloat16*>(xb), n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_euler(float* x, const float* v, long long rows, long long C, int rows_per_group, const float* dt,
+                         const int* active, float* vtap, cudaStream_t st) {
+  EulerArgs e;
+  for (int i = 0; i < LA_MAX_STEPS; ++i) {
+    e.dt[i] = dt ? dt[i] : 0.f;
+    e.active[i] = active ? active[i] : 1;
+  }
+  const long long n4 = rows * C / 4;
+  k_euler<<<grid_for(n4), 256, 0, st>>>(x, v, n4, C / 4, rows_per_group, e, vtap);
+  return cudaGetLastError();
+}

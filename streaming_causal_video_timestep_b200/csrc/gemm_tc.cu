@@ -1,0 +1,285 @@
+// C = A W^T on the 5th-generation tensor cores (tcgen05, accumulators in TMEM).
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0      TMA producer: A [128 x 64] and W [BN x 64] bf16 tiles per k-block,
+//               128-byte swizzle, into a STAGES-deep shared-memory ring;
+//   warp 1      allocates TMEM (2 accumulators of BN fp32 columns) and, with one
+//               thread, issues tcgen05.mma 128 x BN x 16 into the accumulator;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//               32*(w%4) .. +31 = tile rows), fused epilogue, global stores.
+// The two accumulators let the epilogue of tile n overlap the main loop of n+1.
+// Tiles are visited in bands of GROUP_M row-blocks so the A band and the W
+// tiles in flight stay L2-resident.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int GROUP_M = 16;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr size_t SMEM = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
+  const int per_group = GROUP_M * num_n;
+  const int group = tile / per_group;
+  const int first_m = group * GROUP_M;
+  const int gm = min(GROUP_M, num_m - first_m);
+  const int local = tile - group * per_group;
+  m_blk = first_m + local % gm;
+  n_blk = local / gm;
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+    w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+    w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+    w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+    d4[i] = w;
+  }
+}
+
+__device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, long long row, long long col,
+                                               float (&acc)[32]) {
+  const long long off = row * ep.ld + col;
+  switch (ep.kind) {
+    case EPI_STORE:
+      store_bf16x32(reinterpret_cast<__nv_bfloat16*>(ep.out) + off, acc);
+      break;
+    case EPI_RESID: {
+      float4* h4 = reinterpret_cast<float4*>(ep.h32 + off);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 h = h4[i];
+        h.x += acc[4 * i + 0];
+        h.y += acc[4 * i + 1];
+        h.z += acc[4 * i + 2];
+        h.w += acc[4 * i + 3];
+        h4[i] = h;
+        acc[4 * i + 0] = h.x;
+        acc[4 * i + 1] = h.y;
+        acc[4 * i + 2] = h.z;
+        acc[4 * i + 3] = h.w;
+      }
+      store_bf16x32(reinterpret_cast<__nv_bfloat16*>(ep.out) + off, acc);
+      break;
+    }
+    case EPI_SET32: {
+      float4* h4 = reinterpret_cast<float4*>(ep.h32 + off);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) h4[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+      if (ep.out) store_bf16x32(reinterpret_cast<__nv_bfloat16*>(ep.out) + off, acc);
+      break;
+    }
+    case EPI_EULER: {
+      const int g = static_cast<int>(row / ep.rows_per_group);
+      if (!ep.active[g]) break;
+      const float dt = ep.dt[g];
+      float4* x4 = reinterpret_cast<float4*>(ep.h32 + off);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 x = x4[i];
+        x.x += dt * acc[4 * i + 0];
+        x.y += dt * acc[4 * i + 1];
+        x.z += dt * acc[4 * i + 2];
+        x.w += dt * acc[4 * i + 3];
+        x4[i] = x;
+      }
+      if (ep.vtap) {
+        float4* v4 = reinterpret_cast<float4*>(ep.vtap + off);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v4[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+      }
+      break;
+    }
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+          const GemmEpiParams ep, int M, int N, int K, int* err) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);   // one arrive per epilogue warp
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    tma_prefetch_map(&tmA);
+    tma_prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int num_m = (M + BM - 1) / BM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int kblocks = (K + BK - 1) / BK;
+  constexpr uint32_t idesc = idesc_bf16(BM, BN, false, false);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[C::STAGES];
+      for (int i = 0; i < C::STAGES; ++i) last_parity[i] = -1;
+      for (int tile = blockIdx.x; tile < num_tiles && !abort_flag; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, mb, nb);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, err)) { abort_flag = 1; break; }
+          mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * BK, mb * BM);
+          tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * BK, nb * BN);
+          last_parity[stage] = static_cast<int>(phase);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // Every issued load must have landed before the CTA exits: the phase a
+      // load completes has already been observed by the MMA thread on the
+      // normal path (this returns at once); after an abort it bounds the wait.
+      for (int i = 0; i < C::STAGES; ++i)
+        if (last_parity[i] >= 0) mbar_wait(&full[i], static_cast<uint32_t>(last_parity[i]), err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        if (abort_flag) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, err)) { abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            umma_bf16_ss(d_tmem, sdesc_kmajor(a0 + kk * 32), sdesc_kmajor(b0 + kk * 32), idesc,
+                         (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) { abort_flag = 1; break; }
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      // all issued MMAs complete before TMEM is released
+      umma_commit(drain);
+      mbar_wait(drain, 0, err);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int rit = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      if (abort_flag) break;
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, mb, nb);
+      if (!mbar_wait(&tfull[acc], acc_phase, err)) { abort_flag = 1; break; }
+      tc_fence_after();
+      const long long row = static_cast<long long>(mb) * BM + rit;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tbase + c0, r);
+        tmem_ld_wait();
+        const long long col = static_cast<long long>(nb) * BN + c0;
+        if (row < M && col < N) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          epilogue_row32(ep, row, col, v);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M, int N,
+                      int K, int* err, int num_sms, cudaStream_t st) {
+  using C = GemmCfg<BN>;
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::SMEM));
+  if (e != cudaSuccess) return e;
+  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  k_gemm_tc<BN><<<grid, 192, C::SMEM, st>>>(tmA, tmB, ep, M, N, K, err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int gemm_tc_pick_bn(int N) {
+  if (N % 256 == 0 && N >= 1024) return 256;
+  if (N % 128 == 0) return 128;
+  return 64;
+}
+
+cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M, int N,
+                           int K, int bn, int* err, int num_sms, cudaStream_t st) {
+  switch (bn) {
+    case 256: return launch_bn<256>(tmA, tmB, ep, M, N, K, err, num_sms, st);
+    case 128: return launch_bn<128>(tmA, tmB, ep, M, N, K, err, num_sms, st);
+    default: return launch_bn<64>(tmA, tmB, ep, M, N, K, err, num_sms, st);
+  }
+}

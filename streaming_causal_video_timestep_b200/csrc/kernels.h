@@ -1,0 +1,61 @@
+// Host-side launchers of the library's kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+// ---- tcgen05 (bf16) ----------------------------------------------------------------
+int gemm_tc_pick_bn(int N);
+cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M, int N,
+                           int K, int bn, int* err, int num_sms, cudaStream_t st);
+
+// Tensor maps of an attention launch: q (d, Tq, H, q slices) and k[m]/v[m]
+// (d, rows_m, H, slices), bf16, 128-byte swizzle, box (64, 128, 1, 1).
+struct AttnMaps {
+  CUtensorMap q;
+  CUtensorMap k[LA_MAX_SEG];
+  CUtensorMap v[LA_MAX_SEG];
+};
+cudaError_t launch_attn_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);
+
+// ---- SIMT fp32 -----------------------------------------------------------------------
+cudaError_t launch_gemm_f32(const float* A, const float* W, const GemmEpiParams& ep, int M, int N, int K,
+                            cudaStream_t st);
+cudaError_t launch_attn_f32(const AttnParams& p, cudaStream_t st);
+
+// ---- bandwidth kernels (templated on the activation type) -----------------------------
+// Temporal RoPE table of a pass: cos/sin of (pos * omega_t[j]) for every active
+// buffer and each of frames_per_block frames plus the sink row (index fpb).
+cudaError_t launch_rope_ttab(const PassDesc& pd, int fpb, int pt, const double* omega_t, float* tcos, float* tsin,
+                             cudaStream_t st);
+
+struct RopeArgs {
+  int T, F, H, d, D, grid_w, fpb;
+  int pt, ph, pw;
+  const float* tcos;  const float* tsin;       // [LA_MAX_STEPS][LA_TROWS][LA_MAX_PT]
+  const float* rcos;  const float* rsin;       // [grid_h][ph]
+  const float* ccos;  const float* csin;       // [grid_w][pw]
+  const void* qkv;                             // [nbuf*T, 3D]
+  void* q_rope;                                // [nbuf][H][T][d]
+  void* ring_k; void* ring_v;                  // [L][S][E][H][T][d]
+  long long ring_slice0;                       // (layer*S) * E: slice of (layer, slot 0, entry 0)
+  int E;
+  const void* sink_k;                          // un-roped [H][F][d] of this layer
+  void* sink_k_rope;                           // [nbuf][H][F][d]
+};
+cudaError_t launch_rope_append(int bf16, const PassDesc& pd, const RopeArgs& a, cudaStream_t st);
+
+// Sink pass: split qkv [F, 3D] into un-roped K and V of the layer, and roped
+// q / k (temporal row 0 of buffer 0 of the table) for the sink's self-attention.
+cudaError_t launch_sink_qkv(int bf16, const RopeArgs& a, void* sink_k_raw, void* sink_v, void* q_rope,
+                            void* k_rope, cudaStream_t st);
+
+// x (fp32 [rows, C]) -> h32 (fp32) and hop (dtype) when C == D (identity in-proj),
+// or -> xop (bf16) for the in-projection GEMM.
+cudaError_t launch_in_identity(int bf16, const float* x, float* h32, void* hop, long long n, cudaStream_t st);
+cudaError_t launch_cvt_bf16(const float* x, void* xb, long long n, cudaStream_t st);
+// x[r, :] += dt[g] * v[r, :], g = r / rows_per_group, for active groups.
+cudaError_t launch_euler(float* x, const float* v, long long rows, long long C, int rows_per_group,
+                         const float* dt, const int* active, float* vtap, cudaStream_t st);

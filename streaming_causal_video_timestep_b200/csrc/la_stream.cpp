@@ -1,0 +1,959 @@
+// Host side of the streaming step: configuration checks, device buffers, the
+// tick state machine, kernel sequencing and the C ABI declared in la_stream.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "kernels.h"
+#include "la_stream.h"
+#include "tmap.h"
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Tick state machine.
+//
+// Pipelined schedule (the timestep-forcing pipeline of the pages): slot i holds
+// the block slot i-1 held in the previous call; slot 0 takes the new block.
+// Ring of each (layer, slot): window+1 entries; block b writes entry b mod
+// (window+1), evicting block b - window - 1; block b reads b-window .. b-1.
+// ---------------------------------------------------------------------------
+struct SlotRecord {
+  int active_block = -1, write_entry = -1, evicted = -1, sink_tpos = 0, frame_tpos = 0, sink_gen = 0;
+};
+
+struct Scheduler {
+  int S = 0, E = 0, W = 0, fpb = 0, offset = 0, rolling = 1, pipelined = 1, aas = 0;
+  long long tick = -1, blocks_in = 0, blocks_out = 0;
+  int sink_gen = 0;
+  std::vector<long long> held;                  // block held by each slot after the last call
+  std::vector<std::vector<long long>> tag_blk;  // [S][E]
+  std::vector<std::vector<int>> tag_step;       // [S][E]
+  std::vector<SlotRecord> rec;
+
+  void init(const la_config& c) {
+    S = c.num_steps;
+    E = c.window_blocks + 1;
+    W = c.window_blocks;
+    fpb = c.frames_per_block;
+    offset = c.sink_offset_frames;
+    rolling = c.rolling_rope;
+    pipelined = c.schedule == LA_SCHED_PIPELINED;
+    aas = c.sink_mode == LA_SINK_AAS;
+    held.assign(S, -1);
+    tag_blk.assign(S, std::vector<long long>(E, -1));
+    tag_step.assign(S, std::vector<int>(E, -1));
+    rec.assign(S, SlotRecord());
+  }
+  int sink_tpos_of(long long b) const {
+    return rolling ? static_cast<int>(fpb * b - offset) : -offset;
+  }
+  // Which (slot, block) pairs run in the next call, and which block finishes.
+  void plan(bool has_new, std::vector<std::pair<int, long long>>& run, long long& finished,
+            std::vector<long long>& next_held) const {
+    run.clear();
+    if (pipelined) {
+      next_held.assign(S, -1);
+      next_held[0] = has_new ? blocks_in : -1;
+      for (int i = 1; i < S; ++i) next_held[i] = held[i - 1];
+      for (int i = 0; i < S; ++i)
+        if (next_held[i] >= 0) run.emplace_back(i, next_held[i]);
+      finished = next_held[S - 1];
+    } else {
+      next_held.assign(S, -1);
+      for (int i = 0; i < S; ++i) run.emplace_back(i, blocks_in);
+      finished = blocks_in;
+    }
+  }
+  void begin(bool has_new, const std::vector<long long>& next_held) {
+    ++tick;
+    if (has_new) ++blocks_in;
+    if (pipelined) held = next_held;
+    for (auto& r : rec) r = SlotRecord();
+  }
+  int append(int i, long long b) {
+    const int e = static_cast<int>(b % E);
+    SlotRecord& r = rec[i];
+    r.active_block = static_cast<int>(b);
+    r.write_entry = e;
+    r.evicted = static_cast<int>(tag_blk[i][e]);
+    r.sink_tpos = sink_tpos_of(b);
+    r.frame_tpos = static_cast<int>(fpb * b);
+    r.sink_gen = sink_gen;
+    tag_blk[i][e] = b;
+    tag_step[i][e] = i;
+    return e;
+  }
+  bool finish(long long finished) {
+    if (finished >= 0) ++blocks_out;
+    if (finished == 0 && aas && sink_gen == 0) {
+      sink_gen = 1;
+      return true;
+    }
+    return false;
+  }
+  long long state_size() const { return 4 + static_cast<long long>(S) * (8 + 3 * E); }
+  void export_state(int32_t* out) const {
+    out[0] = static_cast<int32_t>(tick);
+    out[1] = static_cast<int32_t>(blocks_in);
+    out[2] = static_cast<int32_t>(blocks_out);
+    out[3] = sink_gen;
+    int32_t* p = out + 4;
+    for (int i = 0; i < S; ++i) {
+      const SlotRecord& r = rec[i];
+      std::vector<long long> res;
+      for (int e = 0; e < E; ++e)
+        if (tag_blk[i][e] >= 0) res.push_back(tag_blk[i][e]);
+      std::sort(res.begin(), res.end());
+      *p++ = r.active_block;
+      *p++ = r.write_entry;
+      *p++ = r.evicted;
+      *p++ = r.active_block >= 0 ? r.sink_tpos : 0;
+      *p++ = r.active_block >= 0 ? r.frame_tpos : 0;
+      *p++ = r.active_block >= 0 ? r.sink_gen : 0;
+      *p++ = i;
+      *p++ = static_cast<int32_t>(res.size());
+      for (int e = 0; e < E; ++e) *p++ = e < static_cast<int>(res.size()) ? static_cast<int32_t>(res[e]) : -1;
+      for (int e = 0; e < E; ++e) {
+        *p++ = static_cast<int32_t>(tag_blk[i][e]);
+        *p++ = tag_step[i][e];
+      }
+    }
+  }
+};
+
+struct ProfEvent {
+  int kind;
+  cudaEvent_t a, b;
+};
+
+}  // namespace
+
+struct la_stream {
+  la_config cfg{};
+  float ts[LA_MAX_STEPS + 1] = {};
+  int S = 0, E = 0, F = 0, T = 0, D = 0, C = 0, H = 0, d = 0, L = 0, fpb = 0, nbuf = 0;
+  int pt = 0, ph = 0, pw = 0;
+  bool bf16 = true, id_in = true, id_head = true;
+  size_t es = 2;
+  int device = 0, num_sms = 148;
+  cudaStream_t st = nullptr;
+
+  const void* w_in = nullptr;
+  const void* w_head = nullptr;
+  std::vector<const void*> w_qkv, w_out;
+
+  std::vector<void*> allocs;
+  float* xs = nullptr;      // [nbuf][T][C]
+  float* h32 = nullptr;     // [nbuf*T][D]
+  void* hop = nullptr;      // [nbuf*T][D] dtype (fp32: == h32)
+  void* xop = nullptr;      // [nbuf*T][C] bf16 (bf16 with an in-projection)
+  void* qkv = nullptr;      // [nbuf*T][3D]
+  void* q_rope = nullptr;   // [nbuf][H][T][d]
+  void* sk_rope = nullptr;  // [nbuf][H][F][d]
+  void* attn_o = nullptr;   // [nbuf*T][D]
+  void* ring_k = nullptr;   // [L][S][E][H][T][d]
+  void* ring_v = nullptr;
+  void* sink_k = nullptr;   // [L][H][F][d] un-roped
+  void* sink_v = nullptr;
+  float* sink_x = nullptr;  // [F][C]
+  float* s_h32 = nullptr;   // [F][D]
+  void* s_hop = nullptr;
+  void* s_xop = nullptr;
+  void* s_qkv = nullptr;
+  void* s_q = nullptr;      // [H][F][d]
+  void* s_k = nullptr;
+  void* s_o = nullptr;      // [F][D]
+  double* omega_t = nullptr;
+  float* tcos = nullptr;
+  float* tsin = nullptr;
+  float *rcos = nullptr, *rsin = nullptr, *ccos = nullptr, *csin = nullptr;
+  int* dev_err = nullptr;
+
+  CUtensorMap tm_hop{}, tm_xop{}, tm_o{}, tm_win{}, tm_whead{};
+  std::vector<CUtensorMap> tm_wqkv, tm_wout;
+  CUtensorMap tm_s_hop{}, tm_s_xop{}, tm_s_o{};
+  AttnMaps maps_stream{};   // q = q_rope; k[0]/v[0] = ring; k[1] = sink K roped per buffer; v[1] = sink V
+  AttnMaps maps_sink{};     // q = s_q; k[0] = s_k; v[0] = sink V
+
+  Scheduler sched;
+  bool sink_set = false;
+  bool started = false;
+  long long launches = 0;
+  std::string err;
+
+  // debug capture (per slot)
+  bool capture = false;
+  float* cap_xin = nullptr;   // [S][T][C]
+  float* cap_xout = nullptr;  // [S][T][C]
+  float* cap_v = nullptr;     // [S][T][C]
+  float* cap_vall = nullptr;  // [nbuf*T][C]
+  float* cap_h = nullptr;     // [S][L+1][T][D]
+  void* cap_q = nullptr;      // [S][L][H][T][d]
+  void* cap_o = nullptr;      // [S][L][T][D]
+  void* cap_sk = nullptr;     // [S][L][H][F][d]
+  std::vector<int> cap_valid;  // per slot: captured in the last call
+
+  bool prof = false;
+  std::vector<ProfEvent> prof_events;
+  std::vector<cudaEvent_t> ev_pool;
+  size_t ev_next = 0;
+};
+
+namespace {
+
+const char* kStatus[] = {"ok", "invalid argument", "invalid state", "out of device memory", "CUDA error",
+                         "device error"};
+
+int fail(la_stream* s, int code, const std::string& msg) {
+  if (s) s->err = msg;
+  return code;
+}
+
+#define CU(call)                                                                                \
+  do {                                                                                          \
+    cudaError_t e_ = (call);                                                                    \
+    if (e_ != cudaSuccess)                                                                      \
+      return fail(s, LA_ECUDA, std::string(#call) + ": " + cudaGetErrorString(e_));            \
+  } while (0)
+
+cudaEvent_t next_event(la_stream* s) {
+  if (s->ev_next >= s->ev_pool.size()) {
+    cudaEvent_t e;
+    cudaEventCreate(&e);
+    s->ev_pool.push_back(e);
+  }
+  return s->ev_pool[s->ev_next++];
+}
+
+// Launch wrapper: counts launches and, when profiling, brackets with events.
+template <typename Fn>
+int launch(la_stream* s, int kind, Fn&& fn) {
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (s->prof) {
+    a = next_event(s);
+    b = next_event(s);
+    cudaEventRecord(a, s->st);
+  }
+  const cudaError_t e = fn();
+  if (e != cudaSuccess) return fail(s, LA_ECUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
+  ++s->launches;
+  if (s->prof) {
+    cudaEventRecord(b, s->st);
+    s->prof_events.push_back({kind, a, b});
+  }
+  return LA_OK;
+}
+
+int dalloc(la_stream* s, void** p, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  const cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) return fail(s, LA_ENOMEM, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+  s->allocs.push_back(*p);
+  const cudaError_t z = cudaMemsetAsync(*p, 0, bytes, s->st);
+  if (z != cudaSuccess) return fail(s, LA_ECUDA, std::string("cudaMemsetAsync: ") + cudaGetErrorString(z));
+  return LA_OK;
+}
+
+#define DALLOC(ptr, bytes)                                                              \
+  do {                                                                                  \
+    void* p_ = nullptr;                                                                 \
+    int r_ = dalloc(s, &p_, (bytes));                                                   \
+    if (r_ != LA_OK) return r_;                                                         \
+    ptr = reinterpret_cast<decltype(ptr)>(p_);                                          \
+  } while (0)
+
+int validate(const la_config* c, const la_weights* w, std::string& msg) {
+  if (!c || !w) { msg = "NULL config or weights"; return LA_EINVAL; }
+  if (c->num_layers < 1 || c->hidden < 1 || c->heads < 1 || c->head_dim < 2 || c->latent_ch < 1 ||
+      c->grid_h < 1 || c->grid_w < 1) { msg = "sizes must be positive"; return LA_EINVAL; }
+  if (static_cast<long long>(c->heads) * c->head_dim != c->hidden) { msg = "hidden != heads*head_dim"; return LA_EINVAL; }
+  if (c->head_dim % 8 != 0 || c->head_dim > 128) { msg = "head_dim must be a multiple of 8 and <= 128"; return LA_EINVAL; }
+  if (c->dtype == LA_BF16 && c->head_dim != 128) { msg = "the bf16 path needs head_dim == 128"; return LA_EINVAL; }
+  if (c->dtype != LA_BF16 && c->dtype != LA_FP32) { msg = "dtype must be LA_BF16 or LA_FP32"; return LA_EINVAL; }
+  if (c->frames_per_block < 1 || c->frames_per_block > LA_MAX_FPB) { msg = "frames_per_block out of range"; return LA_EINVAL; }
+  if (c->sink_frames != 1) { msg = "sink_frames must be 1"; return LA_EINVAL; }
+  if (c->window_blocks < 0 || c->window_blocks > LA_MAX_WINDOW) { msg = "window_blocks out of range"; return LA_EINVAL; }
+  if (c->num_steps < 1 || c->num_steps > LA_MAX_STEPS) { msg = "num_steps out of range"; return LA_EINVAL; }
+  if (!c->timesteps) { msg = "NULL timesteps"; return LA_EINVAL; }
+  for (int i = 0; i <= c->num_steps; ++i)
+    if (!std::isfinite(c->timesteps[i])) { msg = "timesteps must be finite"; return LA_EINVAL; }
+  for (int i = 0; i < c->num_steps; ++i)
+    if (!(c->timesteps[i + 1] < c->timesteps[i])) { msg = "timesteps must be strictly descending"; return LA_EINVAL; }
+  const int P = c->head_dim / 2;
+  if (c->rope_split[0] < 0 || c->rope_split[1] < 0 || c->rope_split[2] < 0 ||
+      c->rope_split[0] + c->rope_split[1] + c->rope_split[2] != P) { msg = "rope_split must sum to head_dim/2"; return LA_EINVAL; }
+  if (c->rope_split[0] > LA_MAX_PT) { msg = "too many temporal rotary pairs"; return LA_EINVAL; }
+  if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) { msg = "rope_theta must be positive"; return LA_EINVAL; }
+  if (c->sink_mode != LA_SINK_FIXED && c->sink_mode != LA_SINK_AAS) { msg = "bad sink_mode"; return LA_EINVAL; }
+  if (c->schedule != LA_SCHED_PIPELINED && c->schedule != LA_SCHED_SEQUENTIAL) { msg = "bad schedule"; return LA_EINVAL; }
+  if (c->rolling_rope != 0 && c->rolling_rope != 1) { msg = "rolling_rope must be 0 or 1"; return LA_EINVAL; }
+  if (c->sink_offset_frames < 0) { msg = "sink_offset_frames must be >= 0"; return LA_EINVAL; }
+  if ((w->w_in == nullptr) != (w->w_head == nullptr)) { msg = "w_in and w_head must both be set or both NULL"; return LA_EINVAL; }
+  if (w->w_in == nullptr && c->latent_ch != c->hidden) { msg = "identity projections need latent_ch == hidden"; return LA_EINVAL; }
+  if (!w->w_qkv || !w->w_out) { msg = "NULL layer weight arrays"; return LA_EINVAL; }
+  for (int l = 0; l < c->num_layers; ++l)
+    if (!w->w_qkv[l] || !w->w_out[l]) { msg = "NULL layer weight"; return LA_EINVAL; }
+  if (c->dtype == LA_BF16) {
+    if (c->hidden % 64 != 0) { msg = "bf16 path needs hidden % 64 == 0"; return LA_EINVAL; }
+    if (w->w_in && (c->latent_ch % 32 != 0)) { msg = "bf16 path needs latent_ch % 32 == 0"; return LA_EINVAL; }
+  }
+  if (c->latent_ch % 4 != 0) { msg = "latent_ch must be a multiple of 4"; return LA_EINVAL; }
+  const long long T = static_cast<long long>(c->frames_per_block) * c->grid_h * c->grid_w;
+  if (T * c->num_steps > (1LL << 30)) { msg = "block too large"; return LA_EINVAL; }
+  return LA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Pass execution
+// ---------------------------------------------------------------------------
+RopeArgs rope_args(la_stream* s) {
+  RopeArgs a{};
+  a.T = s->T; a.F = s->F; a.H = s->H; a.d = s->d; a.D = s->D; a.grid_w = s->cfg.grid_w; a.fpb = s->fpb;
+  a.pt = s->pt; a.ph = s->ph; a.pw = s->pw;
+  a.tcos = s->tcos; a.tsin = s->tsin; a.rcos = s->rcos; a.rsin = s->rsin; a.ccos = s->ccos; a.csin = s->csin;
+  a.E = s->E;
+  return a;
+}
+
+int gemm(la_stream* s, int kind, const CUtensorMap* tmA, const CUtensorMap* tmB, const void* A32, const void* W32,
+         const GemmEpiParams& ep, int M, int N, int K) {
+  if (s->bf16) {
+    const int bn = gemm_tc_pick_bn(N);
+    return launch(s, kind, [&] { return launch_gemm_tc(*tmA, *tmB, ep, M, N, K, bn, s->dev_err, s->num_sms, s->st); });
+  }
+  return launch(s, kind, [&] {
+    return launch_gemm_f32(static_cast<const float*>(A32), static_cast<const float*>(W32), ep, M, N, K, s->st);
+  });
+}
+
+GemmEpiParams epi(int kind, void* out, float* h32, long long ld) {
+  GemmEpiParams e{};
+  e.kind = kind;
+  e.out = out;
+  e.h32 = h32;
+  e.ld = ld;
+  e.rows_per_group = 1 << 30;
+  for (int i = 0; i < LA_MAX_STEPS; ++i) e.active[i] = 1;
+  return e;
+}
+
+char* elem(void* base, long long idx, size_t es) { return static_cast<char*>(base) + idx * static_cast<long long>(es); }
+
+int capture_pass(la_stream* s, const PassDesc& pd, int layer) {
+  // copy the intermediates of every active buffer into its slot's capture area
+  const size_t es = s->es;
+  const long long T = s->T, D = s->D, H = s->H, d = s->d, F = s->F, L = s->L;
+  for (int ai = 0; ai < pd.nactive; ++ai) {
+    const int buf = pd.active_buf[ai];
+    const int slot = pd.slot[buf];
+    if (layer < 0) {
+      CU(cudaMemcpyAsync(s->cap_h + (static_cast<long long>(slot) * (L + 1)) * T * D, s->h32 + buf * T * D,
+                         T * D * 4, cudaMemcpyDeviceToDevice, s->st));
+      continue;
+    }
+    CU(cudaMemcpyAsync(s->cap_h + (static_cast<long long>(slot) * (L + 1) + layer + 1) * T * D, s->h32 + buf * T * D,
+                       T * D * 4, cudaMemcpyDeviceToDevice, s->st));
+    CU(cudaMemcpyAsync(elem(s->cap_q, (static_cast<long long>(slot) * L + layer) * H * T * d, es),
+                       elem(s->q_rope, buf * H * T * d, es), H * T * d * es, cudaMemcpyDeviceToDevice, s->st));
+    CU(cudaMemcpyAsync(elem(s->cap_o, (static_cast<long long>(slot) * L + layer) * T * D, es),
+                       elem(s->attn_o, buf * T * D, es), T * D * es, cudaMemcpyDeviceToDevice, s->st));
+    CU(cudaMemcpyAsync(elem(s->cap_sk, (static_cast<long long>(slot) * L + layer) * H * F * d, es),
+                       elem(s->sk_rope, buf * H * F * d, es), H * F * d * es, cudaMemcpyDeviceToDevice, s->st));
+  }
+  return LA_OK;
+}
+
+// One grouped pass over nbuf buffers (rows = nbuf*T) with the active ones in pd.
+int run_pass(la_stream* s, const PassDesc& pd) {
+  const int T = s->T, D = s->D, C = s->C, H = s->H, d = s->d, F = s->F, S = s->S, E = s->E;
+  const int rows = pd.nbuf * T;
+  int r;
+  if (s->capture) {
+    for (int ai = 0; ai < pd.nactive; ++ai) {
+      const int buf = pd.active_buf[ai];
+      CU(cudaMemcpyAsync(s->cap_xin + static_cast<long long>(pd.slot[buf]) * T * C,
+                         s->xs + static_cast<long long>(buf) * T * C, static_cast<size_t>(T) * C * 4,
+                         cudaMemcpyDeviceToDevice, s->st));
+    }
+  }
+  if ((r = launch(s, LA_KIND_OTHER, [&] {
+         return launch_rope_ttab(pd, s->fpb, s->pt, s->omega_t, s->tcos, s->tsin, s->st);
+       })) != LA_OK)
+    return r;
+
+  // in-projection
+  if (s->id_in) {
+    if ((r = launch(s, LA_KIND_IN_PROJ, [&] {
+           return launch_in_identity(s->bf16, s->xs, s->h32, s->hop, static_cast<long long>(rows) * D, s->st);
+         })) != LA_OK)
+      return r;
+  } else {
+    if (s->bf16 &&
+        (r = launch(s, LA_KIND_IN_PROJ, [&] {
+           return launch_cvt_bf16(s->xs, s->xop, static_cast<long long>(rows) * C, s->st);
+         })) != LA_OK)
+      return r;
+    GemmEpiParams e = epi(EPI_SET32, s->bf16 ? s->hop : nullptr, s->h32, D);
+    if ((r = gemm(s, LA_KIND_IN_PROJ, &s->tm_xop, &s->tm_win, s->xs, s->w_in, e, rows, D, C)) != LA_OK) return r;
+  }
+  if (s->capture && (r = capture_pass(s, pd, -1)) != LA_OK) return r;
+
+  RopeArgs ra = rope_args(s);
+  AttnParams ap{};
+  ap.Tq = T; ap.H = H; ap.d = d;
+  ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  ap.out = s->attn_o; ap.out_ld = D; ap.err = s->dev_err;
+  ap.qbase = s->q_rope;
+  ap.kbase[0] = s->ring_k; ap.vbase[0] = s->ring_v; ap.krows[0] = T; ap.vrows[0] = T;
+  ap.kbase[1] = s->sk_rope; ap.vbase[1] = s->sink_v; ap.krows[1] = F; ap.vrows[1] = F;
+  ap.ngroups = pd.nactive;
+
+  for (int l = 0; l < s->L; ++l) {
+    // QKV projection
+    GemmEpiParams eq = epi(EPI_STORE, s->qkv, nullptr, 3LL * D);
+    if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_hop, &s->tm_wqkv[l], s->bf16 ? s->hop : s->h32, s->w_qkv[l], eq, rows,
+                  3 * D, D)) != LA_OK)
+      return r;
+    // Rolling RoPE + ring append + sink re-rope
+    ra.qkv = s->qkv; ra.q_rope = s->q_rope; ra.ring_k = s->ring_k; ra.ring_v = s->ring_v;
+    ra.ring_slice0 = static_cast<long long>(l) * S * E;
+    ra.sink_k = elem(s->sink_k, static_cast<long long>(l) * H * F * d, s->es);
+    ra.sink_k_rope = s->sk_rope;
+    if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(s->bf16, pd, ra, s->st); })) != LA_OK) return r;
+    // block-causal attention: [sink | window oldest first | self]
+    for (int ai = 0; ai < pd.nactive; ++ai) {
+      const int buf = pd.active_buf[ai];
+      AttnGroup& g = ap.g[ai];
+      g.q_slice = buf;
+      g.out_row0 = buf * T;
+      int ns = 0;
+      g.seg[ns++] = AttnSeg{1, 1, buf, l, F};
+      const long long base = static_cast<long long>(l) * S * E + static_cast<long long>(pd.slot[buf]) * E;
+      for (int w = 0; w < pd.nwin[buf]; ++w)
+        g.seg[ns++] = AttnSeg{0, 0, static_cast<int>(base + pd.win_entry[buf][w]),
+                              static_cast<int>(base + pd.win_entry[buf][w]), T};
+      g.seg[ns++] = AttnSeg{0, 0, static_cast<int>(base + pd.write_entry[buf]),
+                            static_cast<int>(base + pd.write_entry[buf]), T};
+      g.nseg = ns;
+    }
+    if (s->bf16) {
+      if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_tc(s->maps_stream, ap, s->st); })) != LA_OK) return r;
+    } else {
+      if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) return r;
+    }
+    // output projection + residual
+    GemmEpiParams eo = epi(EPI_RESID, s->hop, s->h32, D);
+    if ((r = gemm(s, LA_KIND_OUT_GEMM, &s->tm_o, &s->tm_wout[l], s->attn_o, s->w_out[l], eo, rows, D, D)) != LA_OK)
+      return r;
+    if (s->capture && (r = capture_pass(s, pd, l)) != LA_OK) return r;
+  }
+
+  // velocity head + Euler update x += (t_{i+1} - t_i) v, per buffer
+  float* vtap = s->capture ? s->cap_vall : nullptr;
+  if (s->id_head) {
+    if ((r = launch(s, LA_KIND_HEAD, [&] {
+           return launch_euler(s->xs, s->h32, rows, C, T, pd.dt, pd.active, vtap, s->st);
+         })) != LA_OK)
+      return r;
+  } else {
+    GemmEpiParams e = epi(EPI_EULER, nullptr, s->xs, C);
+    e.rows_per_group = T;
+    for (int i = 0; i < LA_MAX_STEPS; ++i) {
+      e.dt[i] = pd.dt[i];
+      e.active[i] = pd.active[i];
+    }
+    e.vtap = vtap;
+    if ((r = gemm(s, LA_KIND_HEAD, &s->tm_hop, &s->tm_whead, s->bf16 ? s->hop : s->h32, s->w_head, e, rows, C, D)) !=
+        LA_OK)
+      return r;
+  }
+  if (s->capture) {
+    for (int ai = 0; ai < pd.nactive; ++ai) {
+      const int buf = pd.active_buf[ai];
+      const long long so = static_cast<long long>(pd.slot[buf]) * T * C, bo = static_cast<long long>(buf) * T * C;
+      CU(cudaMemcpyAsync(s->cap_xout + so, s->xs + bo, static_cast<size_t>(T) * C * 4, cudaMemcpyDeviceToDevice, s->st));
+      CU(cudaMemcpyAsync(s->cap_v + so, s->cap_vall + bo, static_cast<size_t>(T) * C * 4, cudaMemcpyDeviceToDevice, s->st));
+      s->cap_valid[pd.slot[buf]] = 1;
+    }
+  }
+  return LA_OK;
+}
+
+// The sink frame through the layers: stores per-layer un-roped K and V.
+int run_sink(la_stream* s) {
+  const int F = s->F, D = s->D, C = s->C, H = s->H, d = s->d;
+  int r;
+  PassDesc pd{};
+  pd.nbuf = 1;
+  pd.nactive = 1;
+  pd.active_buf[0] = 0;
+  pd.active[0] = 1;
+  pd.frame_tpos[0] = -s->cfg.sink_offset_frames;
+  pd.sink_tpos[0] = -s->cfg.sink_offset_frames;
+  if ((r = launch(s, LA_KIND_OTHER, [&] {
+         return launch_rope_ttab(pd, s->fpb, s->pt, s->omega_t, s->tcos, s->tsin, s->st);
+       })) != LA_OK)
+    return r;
+  if (s->id_in) {
+    if ((r = launch(s, LA_KIND_IN_PROJ, [&] {
+           return launch_in_identity(s->bf16, s->sink_x, s->s_h32, s->s_hop, static_cast<long long>(F) * D, s->st);
+         })) != LA_OK)
+      return r;
+  } else {
+    if (s->bf16 && (r = launch(s, LA_KIND_IN_PROJ, [&] {
+                      return launch_cvt_bf16(s->sink_x, s->s_xop, static_cast<long long>(F) * C, s->st);
+                    })) != LA_OK)
+      return r;
+    GemmEpiParams e = epi(EPI_SET32, s->bf16 ? s->s_hop : nullptr, s->s_h32, D);
+    if ((r = gemm(s, LA_KIND_IN_PROJ, &s->tm_s_xop, &s->tm_win, s->sink_x, s->w_in, e, F, D, C)) != LA_OK) return r;
+  }
+  RopeArgs ra = rope_args(s);
+  ra.T = F;
+  AttnParams ap{};
+  ap.Tq = F; ap.H = H; ap.d = d;
+  ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  ap.out = s->s_o; ap.out_ld = D; ap.err = s->dev_err;
+  ap.qbase = s->s_q;
+  ap.kbase[0] = s->s_k; ap.krows[0] = F;
+  ap.vbase[0] = s->sink_v; ap.vrows[0] = F;
+  ap.ngroups = 1;
+  for (int l = 0; l < s->L; ++l) {
+    GemmEpiParams eq = epi(EPI_STORE, s->s_qkv, nullptr, 3LL * D);
+    if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_s_hop, &s->tm_wqkv[l], s->bf16 ? s->s_hop : s->s_h32, s->w_qkv[l], eq,
+                  F, 3 * D, D)) != LA_OK)
+      return r;
+    ra.qkv = s->s_qkv;
+    void* kraw = elem(s->sink_k, static_cast<long long>(l) * H * F * d, s->es);
+    void* vraw = elem(s->sink_v, static_cast<long long>(l) * H * F * d, s->es);
+    if ((r = launch(s, LA_KIND_ROPE, [&] {
+           return launch_sink_qkv(s->bf16, ra, kraw, vraw, s->s_q, s->s_k, s->st);
+         })) != LA_OK)
+      return r;
+    if (l == s->L - 1) break;   // the last layer's sink output feeds nothing
+    AttnGroup& g = ap.g[0];
+    g.q_slice = 0;
+    g.out_row0 = 0;
+    g.nseg = 1;
+    g.seg[0] = AttnSeg{0, 0, 0, l, F};
+    if (s->bf16) {
+      if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_tc(s->maps_sink, ap, s->st); })) != LA_OK) return r;
+    } else {
+      if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) return r;
+    }
+    GemmEpiParams eo = epi(EPI_RESID, s->s_hop, s->s_h32, D);
+    if ((r = gemm(s, LA_KIND_OUT_GEMM, &s->tm_s_o, &s->tm_wout[l], s->s_o, s->w_out[l], eo, F, D, D)) != LA_OK)
+      return r;
+  }
+  return LA_OK;
+}
+
+void fill_pass_slot(la_stream* s, PassDesc& pd, int buf, int slot, long long b, int write_entry) {
+  const int W = s->cfg.window_blocks;
+  pd.active[buf] = 1;
+  pd.active_buf[pd.nactive++] = buf;
+  pd.slot[buf] = slot;
+  pd.block[buf] = static_cast<int>(b);
+  pd.write_entry[buf] = write_entry;
+  const int nw = static_cast<int>(std::min<long long>(b, W));
+  pd.nwin[buf] = nw;
+  for (int w = 0; w < nw; ++w) pd.win_entry[buf][w] = static_cast<int>((b - nw + w) % s->E);
+  pd.frame_tpos[buf] = static_cast<int>(s->fpb * b);
+  pd.sink_tpos[buf] = s->sched.sink_tpos_of(b);
+  pd.dt[buf] = s->ts[slot + 1] - s->ts[slot];
+}
+
+int step_impl(la_stream* s, const float* x_new, float* x_out, int64_t* finished_block, cudaMemcpyKind in_kind,
+              cudaMemcpyKind out_kind) {
+  if (!s) return LA_EINVAL;
+  if (!finished_block || !x_out) return fail(s, LA_EINVAL, "NULL x_out or finished_block");
+  if (!s->sink_set) return fail(s, LA_ESTATE, "la_set_sink must be called first");
+  const bool has_new = x_new != nullptr;
+  const bool pipelined = s->cfg.schedule == LA_SCHED_PIPELINED;
+  if (!pipelined && !has_new) return fail(s, LA_EINVAL, "the sequential schedule needs x_new");
+  if (has_new && (s->sched.blocks_in + 1) * static_cast<long long>(s->fpb) > 0x7FFFFFF0LL)
+    return fail(s, LA_ESTATE, "block index exceeds the int32 RoPE position range");
+  std::vector<std::pair<int, long long>> run;
+  std::vector<long long> next_held;
+  long long finished = -1;
+  s->sched.plan(has_new, run, finished, next_held);
+  const long long TC = static_cast<long long>(s->T) * s->C;
+  const long long new_block = s->sched.blocks_in;
+  s->sched.begin(has_new, next_held);
+  s->started = true;
+  if (s->capture) std::fill(s->cap_valid.begin(), s->cap_valid.end(), 0);
+  int r;
+  if (pipelined) {
+    if (has_new)
+      CU(cudaMemcpyAsync(s->xs + (new_block % s->S) * TC, x_new, TC * 4, in_kind, s->st));
+    PassDesc pd{};
+    pd.nbuf = s->S;
+    for (auto& [slot, b] : run) {
+      const int e = s->sched.append(slot, b);
+      fill_pass_slot(s, pd, static_cast<int>(b % s->S), slot, b, e);
+    }
+    if (pd.nactive > 0 && (r = run_pass(s, pd)) != LA_OK) return r;
+    if (finished >= 0)
+      CU(cudaMemcpyAsync(x_out, s->xs + (finished % s->S) * TC, TC * 4, out_kind, s->st));
+  } else {
+    CU(cudaMemcpyAsync(s->xs, x_new, TC * 4, in_kind, s->st));
+    for (auto& [slot, b] : run) {
+      PassDesc pd{};
+      pd.nbuf = 1;
+      const int e = s->sched.append(slot, b);
+      fill_pass_slot(s, pd, 0, slot, b, e);
+      if ((r = run_pass(s, pd)) != LA_OK) return r;
+    }
+    CU(cudaMemcpyAsync(x_out, s->xs, TC * 4, out_kind, s->st));
+  }
+  if (s->sched.finish(finished)) {
+    // Adaptive Attention Sink: frame 0 of finished block 0 becomes the sink
+    const float* src = s->xs + (pipelined ? (finished % s->S) * TC : 0);
+    CU(cudaMemcpyAsync(s->sink_x, src, static_cast<size_t>(s->F) * s->C * 4, cudaMemcpyDeviceToDevice, s->st));
+    if ((r = run_sink(s)) != LA_OK) return r;
+  }
+  *finished_block = finished;
+  return LA_OK;
+}
+
+int alloc_capture(la_stream* s) {
+  if (s->cap_xin) return LA_OK;
+  const long long S = s->S, T = s->T, C = s->C, D = s->D, L = s->L, H = s->H, d = s->d, F = s->F;
+  const size_t es = s->es;
+  DALLOC(s->cap_xin, S * T * C * 4);
+  DALLOC(s->cap_xout, S * T * C * 4);
+  DALLOC(s->cap_v, S * T * C * 4);
+  DALLOC(s->cap_vall, static_cast<long long>(s->nbuf) * T * C * 4);
+  DALLOC(s->cap_h, S * (L + 1) * T * D * 4);
+  DALLOC(s->cap_q, S * L * H * T * d * es);
+  DALLOC(s->cap_o, S * L * T * D * es);
+  DALLOC(s->cap_sk, S * L * H * F * d * es);
+  s->cap_valid.assign(s->S, 0);
+  return LA_OK;
+}
+
+void free_all(la_stream* s) {
+  for (void* p : s->allocs) cudaFree(p);
+  s->allocs.clear();
+  for (auto e : s->ev_pool) cudaEventDestroy(e);
+  s->ev_pool.clear();
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* la_status_string(int status) {
+  if (status > 0 || status < -5) return "unknown status";
+  return kStatus[-status];
+}
+
+const char* la_last_error(const la_stream* s) {
+  if (!s) return "no stream";
+  return s->err.c_str();
+}
+
+int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_stream, la_stream** out) {
+  if (!out) return LA_EINVAL;
+  *out = nullptr;
+  std::string msg;
+  int v = validate(cfg, w, msg);
+  if (v != LA_OK) {
+    std::fprintf(stderr, "la_stream_create: %s\n", msg.c_str());
+    return v;
+  }
+  la_stream* s = new (std::nothrow) la_stream();
+  if (!s) return LA_ENOMEM;
+  auto bail = [&](int code) {
+    if (!s->err.empty()) std::fprintf(stderr, "la_stream_create: %s\n", s->err.c_str());
+    free_all(s);
+    delete s;
+    return code;
+  };
+  s->cfg = *cfg;
+  for (int i = 0; i <= cfg->num_steps; ++i) s->ts[i] = cfg->timesteps[i];
+  s->cfg.timesteps = s->ts;
+  s->S = cfg->num_steps; s->E = cfg->window_blocks + 1; s->F = cfg->grid_h * cfg->grid_w;
+  s->fpb = cfg->frames_per_block; s->T = s->fpb * s->F; s->D = cfg->hidden; s->C = cfg->latent_ch;
+  s->H = cfg->heads; s->d = cfg->head_dim; s->L = cfg->num_layers;
+  s->pt = cfg->rope_split[0]; s->ph = cfg->rope_split[1]; s->pw = cfg->rope_split[2];
+  s->bf16 = cfg->dtype == LA_BF16; s->es = s->bf16 ? 2 : 4;
+  s->id_in = w->w_in == nullptr; s->id_head = w->w_head == nullptr;
+  s->nbuf = cfg->schedule == LA_SCHED_PIPELINED ? s->S : 1;
+  s->st = static_cast<cudaStream_t>(cuda_stream);
+  s->w_in = w->w_in; s->w_head = w->w_head;
+  s->w_qkv.assign(w->w_qkv, w->w_qkv + s->L);
+  s->w_out.assign(w->w_out, w->w_out + s->L);
+  s->sched.init(s->cfg);
+
+  cudaError_t e = cudaGetDevice(&s->device);
+  if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
+  cudaDeviceProp prop{};
+  e = cudaGetDeviceProperties(&prop, s->device);
+  if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
+  if (prop.major != 10) { s->err = "this library is built for sm_100 (B200) devices"; return bail(LA_ECUDA); }
+  s->num_sms = prop.multiProcessorCount;
+  if (s->bf16 && !tmap_init(s->err)) return bail(LA_ECUDA);
+
+  // memory plan, checked before allocating
+  const long long T = s->T, D = s->D, C = s->C, F = s->F, H = s->H, d = s->d, L = s->L, S = s->S, E = s->E;
+  const long long NB = s->nbuf;
+  const size_t es = s->es;
+  const long long need = NB * T * C * 4 + NB * T * D * 4 + (s->bf16 ? NB * T * D * es : 0) +
+                         (s->bf16 && !s->id_in ? NB * T * C * 2 : 0) + NB * T * 3 * D * es + NB * T * D * es * 2 +
+                         NB * H * F * d * es + 2 * L * S * E * H * T * d * es + 2 * L * H * F * d * es +
+                         F * C * 4 + F * D * 4 + F * D * es * 2 + F * C * 2 + F * 3 * D * es + 2 * H * F * d * es +
+                         (64 << 20);
+  size_t free_b = 0, total_b = 0;
+  e = cudaMemGetInfo(&free_b, &total_b);
+  if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
+  if (static_cast<long long>(free_b) < need) {
+    s->err = "stream needs " + std::to_string(need >> 20) + " MiB, " + std::to_string(free_b >> 20) + " MiB free";
+    return bail(LA_ENOMEM);
+  }
+  int r;
+#define ALLOC_OR_BAIL(ptr, bytes)                  \
+  do {                                             \
+    void* p_ = nullptr;                            \
+    r = dalloc(s, &p_, (bytes));                   \
+    if (r != LA_OK) return bail(r);                \
+    ptr = reinterpret_cast<decltype(ptr)>(p_);     \
+  } while (0)
+  ALLOC_OR_BAIL(s->xs, NB * T * C * 4);
+  ALLOC_OR_BAIL(s->h32, NB * T * D * 4);
+  if (s->bf16) ALLOC_OR_BAIL(s->hop, NB * T * D * es); else s->hop = s->h32;
+  if (s->bf16 && !s->id_in) ALLOC_OR_BAIL(s->xop, NB * T * C * 2);
+  ALLOC_OR_BAIL(s->qkv, NB * T * 3 * D * es);
+  ALLOC_OR_BAIL(s->q_rope, NB * T * D * es);
+  ALLOC_OR_BAIL(s->attn_o, NB * T * D * es);
+  ALLOC_OR_BAIL(s->sk_rope, NB * H * F * d * es);
+  ALLOC_OR_BAIL(s->ring_k, L * S * E * H * T * d * es);
+  ALLOC_OR_BAIL(s->ring_v, L * S * E * H * T * d * es);
+  ALLOC_OR_BAIL(s->sink_k, L * H * F * d * es);
+  ALLOC_OR_BAIL(s->sink_v, L * H * F * d * es);
+  ALLOC_OR_BAIL(s->sink_x, F * C * 4);
+  ALLOC_OR_BAIL(s->s_h32, F * D * 4);
+  if (s->bf16) ALLOC_OR_BAIL(s->s_hop, F * D * es); else s->s_hop = s->s_h32;
+  if (s->bf16 && !s->id_in) ALLOC_OR_BAIL(s->s_xop, F * C * 2);
+  ALLOC_OR_BAIL(s->s_qkv, F * 3 * D * es);
+  ALLOC_OR_BAIL(s->s_q, H * F * d * es);
+  ALLOC_OR_BAIL(s->s_k, H * F * d * es);
+  ALLOC_OR_BAIL(s->s_o, F * D * es);
+  ALLOC_OR_BAIL(s->omega_t, std::max(1, s->pt) * 8);
+  ALLOC_OR_BAIL(s->tcos, LA_MAX_STEPS * LA_TROWS * LA_MAX_PT * 4);
+  ALLOC_OR_BAIL(s->tsin, LA_MAX_STEPS * LA_TROWS * LA_MAX_PT * 4);
+  ALLOC_OR_BAIL(s->rcos, std::max(1, cfg->grid_h * s->ph) * 4);
+  ALLOC_OR_BAIL(s->rsin, std::max(1, cfg->grid_h * s->ph) * 4);
+  ALLOC_OR_BAIL(s->ccos, std::max(1, cfg->grid_w * s->pw) * 4);
+  ALLOC_OR_BAIL(s->csin, std::max(1, cfg->grid_w * s->pw) * 4);
+  ALLOC_OR_BAIL(s->dev_err, 64);
+
+  // RoPE frequencies and spatial tables, fp64 on the host
+  {
+    const double theta = cfg->rope_theta;
+    std::vector<double> om(std::max(1, s->pt));
+    for (int j = 0; j < s->pt; ++j) om[j] = std::pow(theta, -static_cast<double>(j) / s->pt);
+    std::vector<float> rc(std::max(1, cfg->grid_h * s->ph)), rs(rc.size()), cc(std::max(1, cfg->grid_w * s->pw)),
+        cs(cc.size());
+    for (int rr = 0; rr < cfg->grid_h; ++rr)
+      for (int j = 0; j < s->ph; ++j) {
+        const double a = rr * std::pow(theta, -static_cast<double>(j) / s->ph);
+        rc[rr * s->ph + j] = static_cast<float>(std::cos(a));
+        rs[rr * s->ph + j] = static_cast<float>(std::sin(a));
+      }
+    for (int c = 0; c < cfg->grid_w; ++c)
+      for (int j = 0; j < s->pw; ++j) {
+        const double a = c * std::pow(theta, -static_cast<double>(j) / s->pw);
+        cc[c * s->pw + j] = static_cast<float>(std::cos(a));
+        cs[c * s->pw + j] = static_cast<float>(std::sin(a));
+      }
+    e = cudaMemcpy(s->omega_t, om.data(), om.size() * 8, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(s->rcos, rc.data(), rc.size() * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(s->rsin, rs.data(), rs.size() * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(s->ccos, cc.data(), cc.size() * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(s->csin, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
+  }
+
+  if (s->bf16) {
+    bool ok = true;
+    const int bn_qkv = gemm_tc_pick_bn(3 * s->D), bn_d = gemm_tc_pick_bn(s->D), bn_c = gemm_tc_pick_bn(s->C);
+    ok = ok && tmap_2d_bf16(&s->tm_hop, s->hop, NB * T, D, D, 128, s->err);
+    ok = ok && tmap_2d_bf16(&s->tm_o, s->attn_o, NB * T, D, D, 128, s->err);
+    ok = ok && tmap_2d_bf16(&s->tm_s_hop, s->s_hop, F, D, D, 128, s->err);
+    ok = ok && tmap_2d_bf16(&s->tm_s_o, s->s_o, F, D, D, 128, s->err);
+    s->tm_wqkv.resize(L);
+    s->tm_wout.resize(L);
+    for (int l = 0; l < L && ok; ++l) {
+      ok = ok && tmap_2d_bf16(&s->tm_wqkv[l], s->w_qkv[l], 3 * D, D, D, bn_qkv, s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_wout[l], s->w_out[l], D, D, D, bn_d, s->err);
+    }
+    if (!s->id_in) {
+      ok = ok && tmap_2d_bf16(&s->tm_xop, s->xop, NB * T, C, C, 128, s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_s_xop, s->s_xop, F, C, C, 128, s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_win, s->w_in, D, C, C, bn_d, s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_whead, s->w_head, C, D, D, bn_c, s->err);
+    }
+    ok = ok && tmap_planes_bf16(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_stream.v[1], s->sink_v, d, F, H, L, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_sink.q, s->s_q, d, F, H, 1, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_sink.k[0], s->s_k, d, F, H, 1, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_sink.v[0], s->sink_v, d, F, H, L, s->err);
+    if (!ok) return bail(LA_ECUDA);
+  }
+  e = cudaStreamSynchronize(s->st);
+  if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
+  *out = s;
+  return LA_OK;
+}
+
+int la_set_sink(la_stream* s, const float* sink_latent) {
+  if (!s) return LA_EINVAL;
+  if (!sink_latent) return fail(s, LA_EINVAL, "NULL sink latent");
+  if (s->started) return fail(s, LA_ESTATE, "the sink can only be set before the first step");
+  CU(cudaMemcpyAsync(s->sink_x, sink_latent, static_cast<size_t>(s->F) * s->C * 4, cudaMemcpyDeviceToDevice, s->st));
+  int r = run_sink(s);
+  if (r != LA_OK) return r;
+  s->sink_set = true;
+  return LA_OK;
+}
+
+int la_denoise_step(la_stream* s, const float* x_new, float* x_out, int64_t* finished_block) {
+  return step_impl(s, x_new, x_out, finished_block, cudaMemcpyDeviceToDevice, cudaMemcpyDeviceToDevice);
+}
+
+int la_denoise_step_host(la_stream* s, const float* x_new_host, float* x_out_host, int64_t* finished_block) {
+  return step_impl(s, x_new_host, x_out_host, finished_block, cudaMemcpyHostToDevice, cudaMemcpyDeviceToHost);
+}
+
+int la_synchronize(la_stream* s) {
+  if (!s) return LA_EINVAL;
+  CU(cudaStreamSynchronize(s->st));
+  int code = 0;
+  CU(cudaMemcpy(&code, s->dev_err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (code != 0) {
+    cudaMemset(s->dev_err, 0, sizeof(int));
+    return fail(s, LA_EDEVICE, "kernel raised device error " + std::to_string(code) +
+                                   (code == LA_DEVERR_WAIT_TIMEOUT ? " (bounded wait timed out)" : ""));
+  }
+  return LA_OK;
+}
+
+int la_stream_destroy(la_stream* s) {
+  if (!s) return LA_OK;
+  cudaStreamSynchronize(s->st);
+  free_all(s);
+  delete s;
+  return LA_OK;
+}
+
+int64_t la_index_state_size(const la_stream* s) { return s ? s->sched.state_size() : 0; }
+
+int la_get_index_state(const la_stream* s, int32_t* host_buf, int64_t n) {
+  if (!s || !host_buf || n < s->sched.state_size()) return LA_EINVAL;
+  s->sched.export_state(host_buf);
+  return LA_OK;
+}
+
+int la_debug_capture(la_stream* s, int32_t enable) {
+  if (!s) return LA_EINVAL;
+  if (enable) {
+    int r = alloc_capture(s);
+    if (r != LA_OK) return r;
+  }
+  s->capture = enable != 0;
+  return LA_OK;
+}
+
+int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* dst, int64_t dst_bytes) {
+  if (!s || !dst) return LA_EINVAL;
+  const long long T = s->T, C = s->C, D = s->D, H = s->H, d = s->d, F = s->F, L = s->L, E = s->E, S = s->S;
+  const size_t es = s->es;
+  const bool per_layer = what == LA_TAP_H || what == LA_TAP_Q || what == LA_TAP_O || what == LA_TAP_RING_K ||
+                         what == LA_TAP_RING_V || what == LA_TAP_SINK_K || what == LA_TAP_SINK_V ||
+                         what == LA_TAP_SINK_KROPE;
+  if (per_layer && (layer < (what == LA_TAP_H ? -1 : 0) || layer >= L)) return fail(s, LA_EINVAL, "bad layer");
+  if (slot < 0 || slot >= S) return fail(s, LA_EINVAL, "bad slot");
+  const void* src = nullptr;
+  long long bytes = 0;
+  const bool needs_capture = what <= LA_TAP_V || what == LA_TAP_SINK_KROPE;
+  if (needs_capture && (!s->cap_xin || s->cap_valid.empty() || !s->cap_valid[slot]))
+    return fail(s, LA_ESTATE, "no capture of that slot in the last call");
+  switch (what) {
+    case LA_TAP_X_IN: src = s->cap_xin + slot * T * C; bytes = T * C * 4; break;
+    case LA_TAP_X_OUT: src = s->cap_xout + slot * T * C; bytes = T * C * 4; break;
+    case LA_TAP_V: src = s->cap_v + slot * T * C; bytes = T * C * 4; break;
+    case LA_TAP_H: src = s->cap_h + (slot * (L + 1) + layer + 1) * T * D; bytes = T * D * 4; break;
+    case LA_TAP_Q: src = elem(s->cap_q, (slot * L + layer) * H * T * d, es); bytes = H * T * d * es; break;
+    case LA_TAP_O: src = elem(s->cap_o, (slot * L + layer) * T * D, es); bytes = T * D * es; break;
+    case LA_TAP_SINK_KROPE: src = elem(s->cap_sk, (slot * L + layer) * H * F * d, es); bytes = H * F * d * es; break;
+    case LA_TAP_RING_K:
+    case LA_TAP_RING_V:
+      src = elem(what == LA_TAP_RING_K ? s->ring_k : s->ring_v, (static_cast<long long>(layer) * S + slot) * E * H * T * d, es);
+      bytes = E * H * T * d * es;
+      break;
+    case LA_TAP_SINK_K:
+    case LA_TAP_SINK_V:
+      src = elem(what == LA_TAP_SINK_K ? s->sink_k : s->sink_v, static_cast<long long>(layer) * H * F * d, es);
+      bytes = H * F * d * es;
+      break;
+    default: return fail(s, LA_EINVAL, "bad tap");
+  }
+  if (dst_bytes < bytes) return fail(s, LA_EINVAL, "tap destination too small");
+  CU(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s->st));
+  return LA_OK;
+}
+
+int la_debug_set_slot_input(la_stream* s, int32_t slot, const float* x) {
+  if (!s || !x) return LA_EINVAL;
+  if (slot < 0 || slot >= s->S) return fail(s, LA_EINVAL, "bad slot");
+  if (s->cfg.schedule != LA_SCHED_PIPELINED) return fail(s, LA_ESTATE, "only the pipelined schedule has slot inputs");
+  if (slot == 0) return fail(s, LA_ESTATE, "slot 0 is fed by x_new");
+  const long long b = s->sched.held[slot - 1];
+  if (b < 0) return fail(s, LA_ESTATE, "slot will be idle in the next tick");
+  const long long TC = static_cast<long long>(s->T) * s->C;
+  CU(cudaMemcpyAsync(s->xs + (b % s->S) * TC, x, TC * 4, cudaMemcpyDeviceToDevice, s->st));
+  return LA_OK;
+}
+
+int la_profile_enable(la_stream* s, int32_t enable) {
+  if (!s) return LA_EINVAL;
+  CU(cudaStreamSynchronize(s->st));
+  s->prof_events.clear();
+  s->ev_next = 0;
+  s->prof = enable != 0;
+  return LA_OK;
+}
+
+int la_profile_read(la_stream* s, int32_t kind, int64_t* launches, double* total_ms) {
+  if (!s || kind < 0 || kind >= LA_NUM_KINDS) return LA_EINVAL;
+  CU(cudaStreamSynchronize(s->st));
+  int64_t n = 0;
+  double ms = 0.0;
+  for (const ProfEvent& pe : s->prof_events) {
+    if (pe.kind != kind) continue;
+    float t = 0.f;
+    CU(cudaEventElapsedTime(&t, pe.a, pe.b));
+    ms += t;
+    ++n;
+  }
+  if (launches) *launches = n;
+  if (total_ms) *total_ms = ms;
+  return LA_OK;
+}
+
+int64_t la_launch_count(const la_stream* s) { return s ? s->launches : 0; }
+
+}  // extern "C"

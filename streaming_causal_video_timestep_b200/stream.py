@@ -1,0 +1,206 @@
+"""Python binding of the streaming step: marshals torch CUDA tensors into the C ABI.
+
+Every computation runs in libla.so's kernels; torch only provides device
+memory and the CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+from ctypes import c_double, c_float, c_int32, c_int64, c_void_p
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import LaConfig, LaWeights, check, load
+
+
+def _dtype_code(dtype):
+    return _lib.LA_BF16 if dtype in (_lib.LA_BF16, "bf16", torch.bfloat16) else _lib.LA_FP32
+
+
+def torch_dtype(code):
+    return torch.bfloat16 if code == _lib.LA_BF16 else torch.float32
+
+
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return c_void_p(s.cuda_stream)
+
+
+def _require(t, dtype, shape, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+class LaStream:
+    """One avatar stream.  `cfg` is any object with the la_config fields
+    (num_layers, hidden, heads, head_dim, latent_ch, grid_h, grid_w,
+    frames_per_block, sink_frames, window_blocks, timesteps, rope_split or
+    pairs, rope_theta, sink_mode, rolling_rope, sink_offset_frames, schedule,
+    dtype).  `weights` holds CUDA tensors in the config dtype:
+    w_qkv / w_out (lists), w_in / w_head (or None)."""
+
+    def __init__(self, cfg, weights, stream=None):
+        self.lib = load()
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        self.dtype = _dtype_code(cfg.dtype)
+        self.tdtype = torch_dtype(self.dtype)
+        ts = [float(t) for t in cfg.timesteps]
+        self._ts = (c_float * len(ts))(*ts)
+        pairs = getattr(cfg, "pairs", None) or cfg.rope_split
+        c = LaConfig()
+        c.num_layers, c.hidden, c.heads, c.head_dim = cfg.num_layers, cfg.hidden, cfg.heads, cfg.head_dim
+        c.latent_ch, c.grid_h, c.grid_w = cfg.latent_ch, cfg.grid_h, cfg.grid_w
+        c.frames_per_block, c.sink_frames, c.window_blocks = cfg.frames_per_block, cfg.sink_frames, cfg.window_blocks
+        c.num_steps = len(ts) - 1
+        c.timesteps = ctypes.cast(self._ts, ctypes.POINTER(c_float))
+        c.rope_split = (c_int32 * 3)(*pairs)
+        c.rope_theta = float(cfg.rope_theta)
+        c.sink_mode, c.rolling_rope, c.sink_offset_frames = cfg.sink_mode, cfg.rolling_rope, cfg.sink_offset_frames
+        c.schedule, c.dtype = cfg.schedule, self.dtype
+        self.cfg = cfg
+        self.c = c
+        self.T = cfg.frames_per_block * cfg.grid_h * cfg.grid_w
+        self.F = cfg.grid_h * cfg.grid_w
+        self.C, self.D = cfg.latent_ch, cfg.hidden
+        self.S = c.num_steps
+        # keep the weight tensors alive for the stream's lifetime (they are borrowed)
+        self._weights = weights
+        L = cfg.num_layers
+        self._wq = (c_void_p * L)(*[w.data_ptr() for w in weights["w_qkv"]])
+        self._wo = (c_void_p * L)(*[w.data_ptr() for w in weights["w_out"]])
+        w = LaWeights()
+        w.w_in = None if weights.get("w_in") is None else weights["w_in"].data_ptr()
+        w.w_head = None if weights.get("w_head") is None else weights["w_head"].data_ptr()
+        w.w_qkv = ctypes.cast(self._wq, ctypes.POINTER(c_void_p))
+        w.w_out = ctypes.cast(self._wo, ctypes.POINTER(c_void_p))
+        self.w = w
+        h = c_void_p()
+        code = self.lib.la_stream_create(ctypes.byref(c), ctypes.byref(w), _stream_handle(self.stream), ctypes.byref(h))
+        check(code)
+        self.h = h
+
+    # -- lifecycle ----------------------------------------------------------------
+    def close(self):
+        if getattr(self, "h", None):
+            self.lib.la_stream_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, code):
+        check(code, self.h)
+
+    # -- the four calls -------------------------------------------------------------
+    def set_sink(self, latent: torch.Tensor):
+        _require(latent, torch.float32, (self.F, self.C), "sink latent")
+        self._check(self.lib.la_set_sink(self.h, _ptr(latent)))
+
+    def step(self, x_new, x_out):
+        """One call of la_denoise_step; returns the finished block id or -1."""
+        if x_new is not None:
+            _require(x_new, torch.float32, (self.T, self.C), "x_new")
+        _require(x_out, torch.float32, (self.T, self.C), "x_out")
+        fin = c_int64(-1)
+        self._check(self.lib.la_denoise_step(self.h, _ptr(x_new), _ptr(x_out), ctypes.byref(fin)))
+        return fin.value
+
+    def step_host(self, x_new_host, x_out_host):
+        """la_denoise_step_host with (pinned) CPU tensors."""
+        for t, nm in ((x_new_host, "x_new"), (x_out_host, "x_out")):
+            if t is not None and (t.is_cuda or t.dtype != torch.float32 or tuple(t.shape) != (self.T, self.C)):
+                raise ValueError(f"{nm} must be a CPU float32 ({self.T}, {self.C}) tensor")
+        fin = c_int64(-1)
+        self._check(self.lib.la_denoise_step_host(self.h, _ptr(x_new_host), _ptr(x_out_host), ctypes.byref(fin)))
+        return fin.value
+
+    def synchronize(self):
+        self._check(self.lib.la_synchronize(self.h))
+
+    # -- debug / test ------------------------------------------------------------------
+    def index_state(self) -> np.ndarray:
+        n = self.lib.la_index_state_size(self.h)
+        buf = (c_int32 * n)()
+        self._check(self.lib.la_get_index_state(self.h, buf, n))
+        return np.frombuffer(buf, dtype=np.int32).copy()
+
+    def capture(self, enable=True):
+        self._check(self.lib.la_debug_capture(self.h, 1 if enable else 0))
+
+    def tap(self, what, layer=0, slot=0):
+        T, C, D, F = self.T, self.C, self.D, self.F
+        H, d, E = self.cfg.heads, self.cfg.head_dim, self.cfg.window_blocks + 1
+        dt = self.tdtype
+        shapes = {
+            "x_in": ((T, C), torch.float32), "x_out": ((T, C), torch.float32), "v": ((T, C), torch.float32),
+            "h": ((T, D), torch.float32), "q": ((H, T, d), dt), "o": ((T, D), dt),
+            "ring_k": ((E, H, T, d), dt), "ring_v": ((E, H, T, d), dt), "sink_k": ((H, F, d), dt),
+            "sink_v": ((H, F, d), dt), "sink_k_rope": ((H, F, d), dt),
+        }
+        shape, tdt = shapes[what]
+        out = torch.empty(shape, dtype=tdt, device="cuda")
+        self._check(self.lib.la_debug_tap(self.h, _lib.TAP[what], layer, slot, _ptr(out),
+                                          out.numel() * out.element_size()))
+        return out
+
+    def set_slot_input(self, slot, x):
+        _require(x, torch.float32, (self.T, self.C), "slot input")
+        self._check(self.lib.la_debug_set_slot_input(self.h, slot, _ptr(x)))
+
+    def profile(self, enable=True):
+        self._check(self.lib.la_profile_enable(self.h, 1 if enable else 0))
+
+    def profile_read(self, kind):
+        n, ms = c_int64(0), c_double(0.0)
+        self._check(self.lib.la_profile_read(self.h, _lib.KIND[kind], ctypes.byref(n), ctypes.byref(ms)))
+        return n.value, ms.value
+
+    def launch_count(self):
+        return self.lib.la_launch_count(self.h)
+
+
+# ---- op-level wrappers -------------------------------------------------------------------
+def op_gemm(A, W, epilogue="store", out=None, h32=None, dt=None, rows_per_group=0, stream=None):
+    lib = load()
+    dtype = _dtype_code(A.dtype)
+    M, K = A.shape
+    N = W.shape[0]
+    epi = dict(store=_lib.LA_EPI_STORE, resid=_lib.LA_EPI_RESID, set32=_lib.LA_EPI_SET32,
+               euler=_lib.LA_EPI_EULER)[epilogue]
+    dtp = None
+    if dt is not None:
+        dtp = (c_float * len(dt))(*[float(x) for x in dt])
+    code = lib.la_op_gemm(dtype, epi, _ptr(A), _ptr(W), _ptr(out), _ptr(h32), M, N, K, dtp, rows_per_group,
+                          _stream_handle(stream))
+    check(code)
+
+
+def op_attention(q, ks, vs, out, stream=None):
+    """q [H, Tq, d]; ks / vs lists of [H, len, d]; out [Tq, H*d]."""
+    lib = load()
+    dtype = _dtype_code(q.dtype)
+    H, Tq, d = q.shape
+    n = len(ks)
+    kp = (c_void_p * n)(*[k.data_ptr() for k in ks])
+    vp = (c_void_p * n)(*[v.data_ptr() for v in vs])
+    ln = (c_int64 * n)(*[k.shape[1] for k in ks])
+    code = lib.la_op_attention(dtype, _ptr(q), Tq, H, d, n, kp, vp, ln, _ptr(out), _stream_handle(stream))
+    check(code)
+
+
+def op_euler(x, v, dt, rows_per_group, stream=None):
+    lib = load()
+    rows, C = x.shape
+    dtp = (c_float * len(dt))(*[float(t) for t in dt])
+    check(lib.la_op_euler(_ptr(x), _ptr(v), rows, C, dtp, rows_per_group, _stream_handle(stream)))

@@ -1,0 +1,51 @@
+"""Test helpers: build streams from workloads, tolerance checks."""
+import numpy as np
+
+from workloads import DTYPE_BF16, Workload, make_weights
+
+# Tolerances stated for this path: bf16 inputs with fp32 accumulation:
+# max|d| <= 1e-2 * max|ref| and sum|d| / sum|ref| <= 2e-3; fp32 configs: 1e-5 for both.
+TOL = {DTYPE_BF16: (1e-2, 2e-3), 1: (1e-5, 1e-5)}
+
+
+def errors(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    diff = np.abs(got - ref)
+    max_rel = diff.max() / max(np.abs(ref).max(), 1e-300)
+    mean_rel = diff.sum() / max(np.abs(ref).sum(), 1e-300)
+    return max_rel, mean_rel
+
+
+def assert_close(got, ref, dtype, what=""):
+    tmax, tmean = TOL[dtype]
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, f"{what}: shape {got.shape} vs {ref.shape}"
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    max_rel, mean_rel = errors(got, ref)
+    assert max_rel <= tmax and mean_rel <= tmean, (
+        f"{what}: max|d|/max|ref| = {max_rel:.3e} (tol {tmax}), sum|d|/sum|ref| = {mean_rel:.3e} (tol {tmean})")
+    return max_rel, mean_rel
+
+
+def torch_weights(W, cfg, device="cuda"):
+    import torch
+    dt = torch.bfloat16 if cfg.dtype == DTYPE_BF16 else torch.float32
+    conv = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device=device, dtype=dt)
+    return dict(w_qkv=[conv(w) for w in W.w_qkv], w_out=[conv(w) for w in W.w_out],
+                w_in=conv(W.w_in), w_head=conv(W.w_head))
+
+
+def make_stream(wl: Workload, W=None, cfg=None):
+    import torch
+    from streaming_causal_video_timestep_b200 import LaStream
+    cfg = cfg or wl.cfg
+    W = W if W is not None else make_weights(wl)
+    s = LaStream(cfg, torch_weights(W, cfg))
+    s.set_sink(torch.from_numpy(W.sink).cuda())
+    return s, W
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy()

@@ -1,0 +1,159 @@
+"""Kernel-level parity on the GPU: tcgen05 GEMM epilogues, block attention over
+segments (tcgen05 bf16 and SIMT fp32), the Euler update -- each against the
+oracle's definition on the same seeded inputs."""
+import numpy as np
+import pytest
+
+from oracle import block_causal_attention, euler_step
+from workloads import DTYPE_BF16, DTYPE_FP32, bf16_round, random_array
+
+from _helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from streaming_causal_video_timestep_b200 import build
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+
+
+def _dev(a, dtype):
+    tdt = torch.bfloat16 if dtype == DTYPE_BF16 else torch.float32
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to("cuda").to(tdt)
+
+
+def _np(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+GEMM_SHAPES = [(300, 256, 320), (130, 64, 64), (1000, 1536, 512), (4680 + 37, 192, 64), (17, 512, 1024)]
+
+
+@pytest.mark.parametrize("dtype", [DTYPE_BF16, DTYPE_FP32])
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_store_and_resid(dtype, M, N, K):
+    from streaming_causal_video_timestep_b200 import op_gemm
+    rnd = bf16_round if dtype == DTYPE_BF16 else (lambda a: a.astype(np.float32))
+    A = rnd(random_array(M * 7 + N, (M, K)))
+    W = rnd(random_array(K * 3 + 1, (N, K), scale=1.0 / np.sqrt(K)))
+    ref = A.astype(np.float64) @ W.astype(np.float64).T
+    tA, tW = _dev(A, dtype), _dev(W, dtype)
+    out = torch.empty((M, N), dtype=tA.dtype, device="cuda")
+    op_gemm(tA, tW, "store", out=out)
+    torch.cuda.synchronize()
+    assert_close(_np(out), ref, dtype, "gemm store")
+    # residual: h32 += acc, out = h32 (rounded to dtype)
+    h0 = random_array(5, (M, N))
+    h32 = torch.from_numpy(h0).cuda()
+    out2 = torch.empty((M, N), dtype=tA.dtype, device="cuda")
+    op_gemm(tA, tW, "resid", out=out2, h32=h32)
+    torch.cuda.synchronize()
+    assert_close(_np(h32), h0 + ref, DTYPE_FP32 if dtype == DTYPE_FP32 else dtype, "gemm resid h32")
+    if dtype == DTYPE_BF16:
+        # the fp32 residual itself carries only fp32 accumulation error
+        err = np.abs(_np(h32) - (h0 + ref)).max() / np.abs(h0 + ref).max()
+        assert err < 1e-4, err
+    assert_close(_np(out2), h0 + ref, dtype, "gemm resid out")
+
+
+@pytest.mark.parametrize("dtype", [DTYPE_BF16, DTYPE_FP32])
+def test_gemm_set32_and_euler_epilogues(dtype):
+    from streaming_causal_video_timestep_b200 import op_gemm
+    rnd = bf16_round if dtype == DTYPE_BF16 else (lambda a: a.astype(np.float32))
+    M, N, K, G = 4 * 180, 64, 256, 4
+    A = rnd(random_array(1, (M, K)))
+    W = rnd(random_array(2, (N, K), scale=0.05))
+    ref = A.astype(np.float64) @ W.astype(np.float64).T
+    tA, tW = _dev(A, dtype), _dev(W, dtype)
+    h32 = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    op_gemm(tA, tW, "set32", out=None, h32=h32)
+    torch.cuda.synchronize()
+    assert_close(_np(h32), ref, DTYPE_FP32 if dtype == DTYPE_FP32 else dtype, "set32")
+    x0 = random_array(3, (M, N))
+    x = torch.from_numpy(x0).cuda()
+    ts = [1.0, 0.75, 0.5, 0.25, 0.0]
+    dts = [ts[i + 1] - ts[i] for i in range(G)]
+    op_gemm(tA, tW, "euler", h32=x, dt=dts, rows_per_group=M // G)
+    torch.cuda.synchronize()
+    want = np.concatenate([euler_step(x0[g * 180:(g + 1) * 180], ref[g * 180:(g + 1) * 180], ts[g], ts[g + 1])
+                           for g in range(G)])
+    assert_close(_np(x), want, DTYPE_FP32 if dtype == DTYPE_FP32 else dtype, "euler epilogue")
+
+
+def _attn_case(seed, H, d, F, T, nwin, scale=1.0, dtype=DTYPE_BF16, Tq=None):
+    rnd = bf16_round if dtype == DTYPE_BF16 else (lambda a: a.astype(np.float32))
+    Tq = Tq or T
+    q = rnd(random_array(seed, (Tq, H, d), scale))
+    sink = (rnd(random_array(seed + 1, (F, H, d), scale)), rnd(random_array(seed + 2, (F, H, d))))
+    b = 5
+    blocks = {b - nwin + w: (rnd(random_array(seed + 10 + w, (T, H, d), scale)),
+                             rnd(random_array(seed + 30 + w, (T, H, d)))) for w in range(nwin + 1)}
+    return q, sink, blocks, b
+
+
+def _run_op_attention(q, sink, blocks, dtype):
+    from streaming_causal_video_timestep_b200 import op_attention
+    to_planes = lambda a: _dev(np.ascontiguousarray(np.transpose(a, (1, 0, 2))), dtype)
+    ks = [to_planes(sink[0])] + [to_planes(blocks[k][0]) for k in sorted(blocks)]
+    vs = [to_planes(sink[1])] + [to_planes(blocks[k][1]) for k in sorted(blocks)]
+    Tq, H, d = q.shape
+    out = torch.empty((Tq, H * d), dtype=ks[0].dtype, device="cuda")
+    op_attention(to_planes(q), ks, vs, out)
+    torch.cuda.synchronize()
+    return _np(out)
+
+
+@pytest.mark.parametrize("F,T,nwin,scale,Tq", [
+    (60, 180, 2, 1.0, None),      # ragged: 180 = 128 + 52, 60 < 128
+    (16, 48, 0, 1.0, None),       # no window (block 0)
+    (130, 300, 2, 1.0, None),     # several q tiles and key tiles, ragged
+    (60, 180, 2, 3.0, None),      # peaked softmax: exercises the lazy O rescale
+    (1560, 256, 1, 1.0, 256),     # full-width sink frame
+])
+def test_attention_bf16_matches_oracle(F, T, nwin, scale, Tq):
+    H, d = 2, 128
+    q, sink, blocks, b = _attn_case(11, H, d, F, T, nwin, scale, Tq=Tq)
+    got = _run_op_attention(q, sink, blocks, DTYPE_BF16)
+    want = block_causal_attention(q, blocks, sink, qblock=b, window=nwin).reshape(q.shape[0], H * d)
+    assert_close(got, want, DTYPE_BF16, "attention bf16")
+
+
+def test_attention_bf16_single_key_passthrough():
+    from streaming_causal_video_timestep_b200 import op_attention
+    H, d = 3, 128
+    q = _dev(random_array(1, (H, 200, d), 5.0), DTYPE_BF16)
+    k = _dev(random_array(2, (H, 1, d)), DTYPE_BF16)
+    v = _dev(random_array(3, (H, 1, d)), DTYPE_BF16)
+    out = torch.empty((200, H * d), dtype=torch.bfloat16, device="cuda")
+    op_attention(q, [k], [v], out)
+    torch.cuda.synchronize()
+    want = np.broadcast_to(_np(v).transpose(1, 0, 2).reshape(1, H * d), (200, H * d))
+    np.testing.assert_array_equal(_np(out), want)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_attention_fp32_matches_oracle(d):
+    H, F, T, nwin = 2, 16, 48, 2
+    q, sink, blocks, b = _attn_case(21, H, d, F, T, nwin, dtype=DTYPE_FP32)
+    got = _run_op_attention(q, sink, blocks, DTYPE_FP32)
+    want = block_causal_attention(q, blocks, sink, qblock=b, window=nwin).reshape(T, H * d)
+    assert_close(got, want, DTYPE_FP32, "attention fp32")
+
+
+def test_euler_standalone_matches_oracle():
+    from streaming_causal_video_timestep_b200 import op_euler
+    rows, C, G = 4 * 4680, 64, 4
+    x0 = random_array(7, (rows, C))
+    v = random_array(8, (rows, C))
+    ts = [1.0, 0.75, 0.5, 0.25, 0.0]
+    x = torch.from_numpy(x0).cuda()
+    op_euler(x, torch.from_numpy(v).cuda(), [ts[i + 1] - ts[i] for i in range(G)], rows // G)
+    torch.cuda.synchronize()
+    want = np.concatenate([euler_step(x0[g * 4680:(g + 1) * 4680], v[g * 4680:(g + 1) * 4680], ts[g], ts[g + 1])
+                           for g in range(G)])
+    assert_close(_np(x), want, DTYPE_FP32, "euler")

@@ -1,0 +1,205 @@
+"""Stream-level parity on the GPU through the C ABI: every tick's integer state
+bit-exact against the oracle's scheduler, and every float intermediate
+(q, appended K/V, sink re-rope, attention output, residual after each layer,
+velocity, latent) within the stated tolerance, teacher-forced per step."""
+import numpy as np
+import pytest
+
+from oracle import OracleStream, TickScheduler
+from workloads import (DTYPE_BF16, DTYPE_FP32, SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_AAS, SINK_FIXED, TINY,
+                       StreamConfig, Workload, block_noise, make_weights)
+
+from _helpers import assert_close, errors, make_stream, to_np
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from streaming_causal_video_timestep_b200 import build
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+
+
+SMALL_BF16 = Workload(
+    name="small-bf16",
+    cfg=StreamConfig(num_layers=2, hidden=256, heads=2, head_dim=128, latent_ch=32, grid_h=6, grid_w=10,
+                     window_blocks=2, sink_mode=SINK_AAS, dtype=DTYPE_BF16),
+    seed=5, num_blocks=8, w_std=1.5 / 16.0, head_std=0.1)
+
+SMALL_BF16_ID = Workload(
+    name="small-bf16-identity",
+    cfg=StreamConfig(num_layers=1, hidden=256, heads=2, head_dim=128, latent_ch=256, grid_h=5, grid_w=9,
+                     window_blocks=1, sink_mode=SINK_FIXED, timesteps=(0.5, 0.25), dtype=DTYPE_BF16),
+    seed=6, num_blocks=4, w_std=1.5 / 16.0)
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+
+def _check_tick(s, orc, cfg, dtype, ran, tag=""):
+    """Compare every captured intermediate of this tick with the oracle trace."""
+    T, D, H, d = cfg.block_tokens, cfg.hidden, cfg.heads, cfg.head_dim
+    worst = 0.0
+    for (b, i) in ran:
+        tr = orc.trace[(b, i)]
+        assert_close(to_np(s.tap("h", -1, i)), tr["h_in"], dtype, f"{tag} h_in b{b} s{i}")
+        for l in range(cfg.num_layers):
+            lt = tr[("layer", l)]
+            assert_close(to_np(s.tap("q", l, i)), lt["q"].transpose(1, 0, 2), dtype, f"{tag} q b{b} s{i} l{l}")
+            ring_k = to_np(s.tap("ring_k", l, i))[b % cfg.ring_entries]
+            ring_v = to_np(s.tap("ring_v", l, i))[b % cfg.ring_entries]
+            assert_close(ring_k, lt["k"].transpose(1, 0, 2), dtype, f"{tag} ring K b{b} s{i} l{l}")
+            assert_close(ring_v, lt["v"].transpose(1, 0, 2), dtype, f"{tag} ring V b{b} s{i} l{l}")
+            assert_close(to_np(s.tap("sink_k_rope", l, i)), lt["sink_k"].transpose(1, 0, 2), dtype,
+                         f"{tag} sink K rope b{b} s{i} l{l}")
+            _, mean_rel = assert_close(to_np(s.tap("o", l, i)), lt["o"].reshape(T, D), dtype,
+                                       f"{tag} attn O b{b} s{i} l{l}")
+            worst = max(worst, mean_rel)
+            assert_close(to_np(s.tap("h", l, i)), lt["h"], dtype, f"{tag} h b{b} s{i} l{l}")
+        assert_close(to_np(s.tap("v", 0, i)), tr["v"], dtype, f"{tag} v b{b} s{i}")
+        assert_close(to_np(s.tap("x_out", 0, i)), tr["x_out"], dtype, f"{tag} x b{b} s{i}")
+    return worst
+
+
+def _run_teacher_forced(wl, check_every_tick=True):
+    cfg = wl.cfg
+    s, W = make_stream(wl)
+    s.capture(True)
+    orc = OracleStream(cfg, W, trace=True)
+    orc.set_sink(W.sink)
+    T, C = cfg.block_tokens, cfg.latent_ch
+    x_out = torch.empty((T, C), dtype=torch.float32, device="cuda")
+    nb = wl.num_blocks
+    S = cfg.num_steps
+    finished_gpu = {}
+    for k in range(nb + S - 1):
+        xn = block_noise(wl, k) if k < nb else None
+        fin = s.step(_dev(xn) if xn is not None else None, x_out)
+        st = s.index_state()
+        per = 8 + 3 * cfg.ring_entries
+        ran = [(int(st[4 + i * per]), i) for i in range(S) if st[4 + i * per] >= 0]
+        inputs = {(b, i): to_np(s.tap("x_in", 0, i)) for (b, i) in ran}
+        aas = to_np(x_out) if fin == 0 else None
+        out, fin_o = orc.denoise_step(xn, inputs=inputs, aas_latent=aas)
+        assert fin == fin_o
+        np.testing.assert_array_equal(st, orc.index_state())
+        if check_every_tick or k >= nb + S - 2:
+            _check_tick(s, orc, cfg, cfg.dtype, ran, tag=f"tick {k}")
+        if fin >= 0:
+            finished_gpu[fin] = to_np(x_out).copy()
+            assert_close(finished_gpu[fin], out, cfg.dtype, f"finished block {fin}")
+    s.synchronize()
+    # sink was replaced exactly once (AAS) and the GPU sink K/V match the oracle's
+    if cfg.sink_mode == SINK_AAS:
+        for l in range(cfg.num_layers):
+            assert_close(to_np(s.tap("sink_k", l)), orc.sink_k[l].transpose(1, 0, 2), cfg.dtype, "sink K")
+            assert_close(to_np(s.tap("sink_v", l)), orc.sink_v[l].transpose(1, 0, 2), cfg.dtype, "sink V")
+    s.close()
+    return finished_gpu
+
+
+def test_tiny_fp32_stream_every_tick_matches_oracle():
+    _run_teacher_forced(TINY)
+
+
+def test_tiny_fp32_stream_free_running_trajectory():
+    """No teacher forcing: the fp32 trajectory itself stays within 1e-5."""
+    wl = TINY
+    cfg = wl.cfg
+    s, W = make_stream(wl)
+    orc = OracleStream(cfg, W)
+    orc.set_sink(W.sink)
+    x_out = torch.empty((cfg.block_tokens, cfg.latent_ch), dtype=torch.float32, device="cuda")
+    for k in range(wl.num_blocks + 3):
+        xn = block_noise(wl, k) if k < wl.num_blocks else None
+        fin = s.step(_dev(xn) if xn is not None else None, x_out)
+        out, fin_o = orc.denoise_step(xn)
+        assert fin == fin_o
+        if fin >= 0:
+            assert_close(to_np(x_out), out, DTYPE_FP32, f"block {fin}")
+    s.close()
+
+
+def test_small_bf16_stream_teacher_forced():
+    _run_teacher_forced(SMALL_BF16)
+
+
+def test_small_bf16_identity_projection_one_slot():
+    _run_teacher_forced(SMALL_BF16_ID)
+
+
+@pytest.mark.parametrize("dtype", [DTYPE_FP32, DTYPE_BF16])
+def test_pipelined_equals_sequential_on_gpu_with_fixed_sink(dtype):
+    base = TINY if dtype == DTYPE_FP32 else SMALL_BF16
+    cfg0 = base.cfg.replace(sink_mode=SINK_FIXED)
+    wl = Workload("cmp", cfg0, base.seed, 6, base.w_std, base.head_std)
+    W = make_weights(wl)
+    outs = {}
+    for sched in (SCHED_PIPELINED, SCHED_SEQUENTIAL):
+        cfg = cfg0.replace(schedule=sched)
+        s, _ = make_stream(wl, W, cfg)
+        x_out = torch.empty((cfg.block_tokens, cfg.latent_ch), dtype=torch.float32, device="cuda")
+        res = {}
+        for k in range(wl.num_blocks + (3 if sched == SCHED_PIPELINED else 0)):
+            xn = block_noise(wl, k) if k < wl.num_blocks else None
+            fin = s.step(_dev(xn) if xn is not None else None, x_out)
+            if fin >= 0:
+                res[fin] = to_np(x_out).copy()
+        s.close()
+        outs[sched] = res
+    for b in range(wl.num_blocks):
+        # the same kernels on the same rows: identical up to bitwise equality
+        np.testing.assert_array_equal(outs[SCHED_PIPELINED][b], outs[SCHED_SEQUENTIAL][b])
+
+
+def test_index_state_bit_exact_over_long_stream_with_bubbles():
+    wl = Workload("idx", TINY.cfg.replace(window_blocks=3), 0, 0, 0.125)
+    s, W = make_stream(wl)
+    ref = TickScheduler(wl.cfg)
+    x = _dev(block_noise(wl, 0))
+    x_out = torch.empty_like(x)
+    rng = np.random.default_rng(0)
+    for k in range(300):
+        has_new = bool(rng.random() < 0.85) or k < 5
+        fin = s.step(x if has_new else None, x_out)
+        run, fin_o = ref.begin_tick(has_new)
+        for i, b in run:
+            ref.append(i, b)
+        ref.end_tick(fin_o)
+        assert fin == fin_o
+        np.testing.assert_array_equal(s.index_state(), ref.index_state())
+    s.synchronize()
+    s.close()
+
+
+def test_state_errors():
+    from streaming_causal_video_timestep_b200 import LaError, LaStream
+    from _helpers import torch_weights
+    wl = TINY
+    W = make_weights(wl)
+    s = LaStream(wl.cfg, torch_weights(W, wl.cfg))
+    x = _dev(block_noise(wl, 0))
+    x_out = torch.empty_like(x)
+    with pytest.raises(LaError) as e:
+        s.step(x, x_out)
+    assert e.value.code == -2
+    s.set_sink(_dev(W.sink))
+    s.step(x, x_out)
+    with pytest.raises(LaError) as e:
+        s.set_sink(_dev(W.sink))
+    assert e.value.code == -2
+    with pytest.raises(LaError) as e:
+        s.set_slot_input(0, x)
+    assert e.value.code == -2
+    s.synchronize()
+    s.close()
+    seq = LaStream(wl.cfg.replace(schedule=SCHED_SEQUENTIAL), torch_weights(W, wl.cfg))
+    seq.set_sink(_dev(W.sink))
+    with pytest.raises(LaError) as e:
+        seq.step(None, x_out)
+    assert e.value.code == -1
+    seq.close()
