@@ -1,0 +1,362 @@
+"""Benchmark of the timestep-forced streaming step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step is one tick of the 4-slot grouped stream in steady state: 4 in-flight
+blocks (one per timestep slot, every window full) through 8 attention
+sublayers, the velocity head and the Euler update; each tick finishes one
+3-latent-frame block.  value = latent frames/s over all ranks (each rank runs
+an independent stream: replicas, weak scaling).  Inputs (weights 1.7 GB, ring
+caches 9.2 GB) are larger than L2.  Prints one JSON line on rank 0.
+
+--impl reference times the fp64 CPU oracle on bounded query-row samples of
+the same workload (rank 0 only) and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "latent frames/s (4-step stream, 1 B200); attention % of bf16 tensor-core peak"
+UNIT = "latent frames/s"
+WORKLOAD = dict(
+    workload="4-step timestep-forced stream: 4 in-flight blocks x 8 attention sublayers, grouped launch",
+    hidden=5120, heads=40, head_dim=128, latent_ch=64, grid="30x52", tokens_per_block=4680, sink_tokens=1560,
+    window_blocks=2, keys_per_query=15600, timesteps=[1.0, 0.75, 0.5, 0.25, 0.0], layers=8,
+    dtype="bf16 weights/activations, fp16 attention operands, fp32 accumulate and latent",
+    l2="inputs larger than L2: 1.68 GB weights + 9.2 GB ring caches read per tick",
+    data="synthetic: N(0,1) latents, N(0,0.02) weights, seeded")
+
+
+def _attn_flops_per_slot(T, F, nw, H, d):
+    nk = F + nw * T + T
+    return 4.0 * T * nk * d * H
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(tflops=j["bf16_tflops"], tflops_sust=j["bf16_tflops_sustained"], hbm=j["hbm_gbs"],
+                    src="measured")
+    return dict(tflops=1590.0, tflops_sust=1400.0, hbm=6650.0, src="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    from streaming_causal_video_timestep_b200 import LaStream
+    from workloads import STREAM
+
+    torch.cuda.set_device(local_rank)
+    wl = STREAM
+    cfg = wl.cfg
+    T, C, D, F, H, d = cfg.block_tokens, cfg.latent_ch, cfg.hidden, cfg.frame_tokens, cfg.heads, cfg.head_dim
+    S, nw, L = cfg.num_steps, cfg.window_blocks, cfg.num_layers
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 + rank)
+    bf = torch.bfloat16
+
+    def rnd(shape, std):
+        return (torch.randn(shape, generator=g, device="cuda") * std).to(bf)
+
+    weights = dict(w_qkv=[rnd((3 * D, D), wl.w_std) for _ in range(L)],
+                   w_out=[rnd((D, D), wl.w_std) for _ in range(L)],
+                   w_in=rnd((D, C), 1.0 / C ** 0.5), w_head=rnd((C, D), wl.head_std))
+    s = LaStream(cfg, weights)
+    s.set_sink(torch.randn((F, C), generator=g, device="cuda"))
+    xs = [torch.randn((T, C), generator=g, device="cuda") for _ in range(4)]
+    x_out = torch.empty((T, C), device="cuda")
+    fill = (S - 1) + nw + 1          # every slot active with a full window from here on
+    k = 0
+    for _ in range(fill + args.warmup):
+        s.step(xs[k % 4], x_out)
+        k += 1
+    s.synchronize()
+    st = s.index_state()
+    per = 8 + 3 * cfg.ring_entries
+    assert all(st[4 + i * per] >= nw for i in range(S)), "not in steady state"
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+        tdist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream()
+    launches0 = s.launch_count()
+    s.profile(True)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        s.step(xs[k % 4], x_out)
+        k += 1
+    ev1.record(stream)
+    s.synchronize()
+    torch.cuda.synchronize()
+    launches = s.launch_count() - launches0
+    ms = ev0.elapsed_time(ev1)
+    kinds = {kind: s.profile_read(kind) for kind in ("in_proj", "qkv_gemm", "rope", "attn", "out_gemm", "head",
+                                                     "other")}
+    s.profile(False)
+    clk = clocks.stop()
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+        tdist.barrier()
+
+    # end to end through the public host-buffer call: H2D of the new block and
+    # D2H of the finished block inside the timed region, waited every tick
+    xh = [torch.randn((T, C)).pin_memory() for _ in range(2)]
+    oh = torch.empty((T, C)).pin_memory()
+    for _ in range(2):
+        s.step_host(xh[0], oh)
+    s.synchronize()
+    if dist:
+        tdist.barrier()
+    e2e_steps = max(3, min(args.steps, 10))
+    t0 = time.perf_counter()
+    for i in range(e2e_steps):
+        fin = s.step_host(xh[i % 2], oh)
+        s.synchronize()
+        assert fin >= 0
+    e2e_s = time.perf_counter() - t0
+    if dist:
+        t = torch.tensor([e2e_s], device="cuda")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    s.close()
+
+    frames_per_tick = cfg.frames_per_block
+    value = frames_per_tick * args.steps * world / (ms / 1000.0)
+    e2e_value = frames_per_tick * e2e_steps * world / e2e_s
+    pk = _peaks()
+    n_attn, ms_attn = kinds["attn"]
+    attn_flops_launch = S * _attn_flops_per_slot(T, F, nw, H, d)
+    attn_ms_avg = ms_attn / max(n_attn, 1)
+    achieved = attn_flops_launch / (attn_ms_avg / 1000.0) / 1e12
+    peak = pk["tflops_sust"]
+    gemm_flops = {"qkv_gemm": 2.0 * S * T * D * 3 * D, "out_gemm": 2.0 * S * T * D * D,
+                  "in_proj": 2.0 * S * T * C * D, "head": 2.0 * S * T * D * C}
+    kernels = {}
+    for kind, (n, tot) in kinds.items():
+        if n == 0:
+            continue
+        avg = tot / n
+        e = {"launches": n, "ms_avg": round(avg, 4), "ms_per_step": round(tot / args.steps, 3)}
+        if kind == "attn":
+            e["tflops"] = round(achieved, 1)
+        elif kind in gemm_flops and n >= args.steps * (L if kind in ("qkv_gemm", "out_gemm") else 1):
+            e["tflops"] = round(gemm_flops[kind] / (avg / 1000.0) / 1e12, 1)
+        kernels[kind] = e
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(WORKLOAD, parallelism=f"replicas x{world} (independent streams, no collective)"),
+        "roofline": {"bound": "tensor", "kernel": "block-causal attention (tcgen05)", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{pk['src']} bf16 sustained (fp16 dense rate = bf16 dense rate)",
+                     "algorithmic_flops_per_launch": attn_flops_launch},
+        "kernels": kernels,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": T * C * 4,
+                "d2h_bytes_per_step": T * C * 4, "steps": e2e_steps},
+    }
+    return line
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host: bounded query-row samples of one slot's sublayer
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """One attention sublayer of one slot in steady state (window full), for a
+    sample of the block's query rows, with the oracle's own functions: QKV
+    projection, 3D Rolling RoPE, block-causal attention over sink + 2 window
+    blocks + the block (15,600 keys), output projection.  Per-row work is the
+    same for every row, so time x (rows of a block / sampled rows) x (slots x
+    layers) estimates one tick."""
+
+    def __init__(self, rows):
+        import numpy as np
+        from oracle.rope import block_positions, sink_positions
+        from workloads import STREAM
+        self.np = np
+        c = STREAM.cfg
+        self.c = c
+        self.rows = rows
+        T, D, H, d, F = c.block_tokens, c.hidden, c.heads, c.head_dim, c.frame_tokens
+        rng = np.random.default_rng(7)
+        self.w_qkv = rng.standard_normal((3 * D, D)) * 0.02
+        self.w_out = rng.standard_normal((D, D)) * 0.02
+        self.h = rng.standard_normal((rows, D))
+        self.b = 2
+        self.blocks = {b: (rng.standard_normal((T, H, d)), rng.standard_normal((T, H, d))) for b in (0, 1)}
+        self.self_v = rng.standard_normal((T, H, d))
+        self.self_k = rng.standard_normal((T, H, d))
+        self.sink = (rng.standard_normal((F, H, d)), rng.standard_normal((F, H, d)))
+        self.pos = block_positions(c, self.b)
+        self.spos = sink_positions(c, 3 * self.b - 3)
+
+    def step(self):
+        from oracle import block_causal_attention, rope_rotate
+        c, r = self.c, self.rows
+        D, H, d = c.hidden, c.heads, c.head_dim
+        qkv = self.h @ self.w_qkv.T
+        q = qkv[:, :D].reshape(r, H, d)
+        k = qkv[:, D:2 * D].reshape(r, H, d)
+        pt, ph, pw = (p[:r] for p in self.pos)
+        qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
+        kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
+        self.self_k[:r] = kr
+        blocks = dict(self.blocks)
+        blocks[self.b] = (self.self_k, self.self_v)
+        sk = rope_rotate(self.sink[0], *self.spos, c.pairs, c.rope_theta)
+        o = block_causal_attention(qr, blocks, (sk, self.sink[1]), qblock=self.b, window=c.window_blocks)
+        return self.h + o.reshape(r, D) @ self.w_out.T
+
+    def frames_per_s(self, seconds_per_step):
+        c = self.c
+        tick_s = seconds_per_step * (c.block_tokens / self.rows) * c.num_steps * c.num_layers
+        return c.frames_per_block / tick_s
+
+
+def cpu_baseline(rows=468, reps=1):
+    smp = OracleSample(rows)
+    smp.step()
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        smp.step()
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(smp.frames_per_s(dt), 6), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": (f"fp64 numpy oracle, one attention sublayer of one slot, {rows} of 4680 query rows over "
+                       f"15,600 keys ({dt:.1f} s), scaled x{4680 / rows:.0f} rows x 4 slots x 8 layers per tick")}
+
+
+def run_reference(args):
+    smp = OracleSample(rows=234)
+    for _ in range(args.warmup):
+        smp.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        smp.step()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = smp.frames_per_s(dt)
+    sample = (f"fp64 numpy oracle, per step one attention sublayer of one slot for 234 of 4680 query rows "
+              f"({dt:.2f} s), scaled to a tick (x20 rows x 4 slots x 8 layers)")
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1000.0, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(WORKLOAD),
+            "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    line = run_gpu(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+        tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -57,8 +57,10 @@ extern "C" {
 #define LA_SINK_AAS          1  /* sink replaced once by frame 0 of finished block 0  */
 #define LA_SCHED_PIPELINED   0  /* one call = one tick: slot i runs step i of block k-i */
 #define LA_SCHED_SEQUENTIAL  1  /* one call = one block through all steps in order     */
-#define LA_BF16              0  /* bf16 weights/activations, fp32 accumulate, fp32 x   */
+#define LA_BF16              0  /* bf16 weights/activations, fp32 accumulate, fp32 x;
+                                   attention operands (q, K, V, P) in fp16            */
 #define LA_FP32              1  /* fp32 everywhere (SIMT path, no TF32)                */
+#define LA_FP16              2  /* op-level attention only: fp16 q/K/V, tcgen05        */
 
 /* Limits of this build. */
 #define LA_MAX_STEPS     8
@@ -187,14 +189,17 @@ int la_debug_capture(la_stream* s, int32_t enable);
 #define LA_TAP_X_IN      0  /* fp32 [T_b, C]   latent the slot's last step started from        */
 #define LA_TAP_X_OUT     1  /* fp32 [T_b, C]   latent after the slot's last step               */
 #define LA_TAP_H         2  /* fp32 [T_b, D]   residual after layer `layer` (-1: after in-proj) */
-#define LA_TAP_Q         3  /* dtype [H, T_b, d] roped queries of layer                          */
-#define LA_TAP_O         4  /* dtype [T_b, D]   attention output of layer                        */
+/* "attn" = the attention operand type: fp16 for LA_BF16 streams, fp32 for LA_FP32. */
+#define LA_TAP_Q         3  /* attn [H, T_b, d] roped queries of layer                           */
+#define LA_TAP_O         4  /* fp32 [T_b, D]   attention output of layer, before rounding        */
 #define LA_TAP_V         5  /* fp32 [T_b, C]    velocity of the slot's last step                 */
-#define LA_TAP_RING_K    6  /* dtype [E, H, T_b, d] ring K of (layer, slot), by entry            */
-#define LA_TAP_RING_V    7  /* dtype [E, H, T_b, d] ring V of (layer, slot)                      */
-#define LA_TAP_SINK_K    8  /* dtype [H, F, d] un-roped sink K of layer (slot ignored)           */
-#define LA_TAP_SINK_V    9  /* dtype [H, F, d] sink V of layer (slot ignored)                    */
-#define LA_TAP_SINK_KROPE 10 /* dtype [H, F, d] sink K as roped for the slot's last step         */
+#define LA_TAP_RING_K    6  /* attn [E, H, T_b, d] ring K of (layer, slot), by entry             */
+#define LA_TAP_RING_V    7  /* attn [E, H, T_b, d] ring V of (layer, slot)                       */
+#define LA_TAP_SINK_K    8  /* fp32 [H, F, d] un-roped sink K of layer (slot ignored)            */
+#define LA_TAP_SINK_V    9  /* attn [H, F, d] sink V of layer (slot ignored)                     */
+#define LA_TAP_SINK_KROPE 10 /* attn [H, F, d] sink K as roped for the slot's last step          */
+#define LA_TAP_SINK_H    11 /* fp32 [F, D] sink residual entering layer `layer` in the last sink
+                               pass (la_set_sink or the AAS replacement; slot ignored)           */
 
 /* Copy one tapped tensor into dst (DEVICE, dst_bytes >= the tensor's size),
  * ordered on the stream.  Taps other than ring / sink need capture enabled
@@ -229,19 +234,21 @@ int64_t la_launch_count(const la_stream* s);
 
 /*
  * C = A W^T with an epilogue.  A: DEVICE [M, K] row-major, W: DEVICE [N, K]
- * row-major, both of `dtype` (bf16 path: tcgen05 tensor cores, fp32
- * accumulate; fp32 path: SIMT fp32).  K % 8 == 0 for bf16.
+ * row-major, both of `dtype` (LA_BF16: tcgen05 tensor cores, fp32
+ * accumulate, N % 32 == 0, K % 8 == 0; LA_FP32: SIMT fp32).
  *   LA_EPI_STORE:   out (dtype [M, N]) = acc
+ *   LA_EPI_STORE32: out (fp32 [M, N]) = acc
  *   LA_EPI_RESID:   h32 (fp32 [M, N]) += acc; out (dtype [M, N]) = h32
  *   LA_EPI_SET32:   h32 = acc; out (dtype [M, N]) = acc   (out may be NULL)
  *   LA_EPI_EULER:   h32[m, n] += dt[m / rows_per_group] * acc (the Euler update;
  *                   dt: HOST array of ceil(M/rows_per_group) floats, <= LA_MAX_STEPS)
  * For LA_FP32 "out" of RESID/SET32 may alias h32.
  */
-#define LA_EPI_STORE  0
-#define LA_EPI_RESID  1
-#define LA_EPI_SET32  2
-#define LA_EPI_EULER  3
+#define LA_EPI_STORE    0
+#define LA_EPI_RESID    1
+#define LA_EPI_SET32    2
+#define LA_EPI_EULER    3
+#define LA_EPI_STORE32  4
 int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, void* out,
                float* h32, int64_t M, int64_t N, int64_t K, const float* dt,
                int64_t rows_per_group, void* cuda_stream);
@@ -252,12 +259,14 @@ int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, vo
  * concatenation of the segments (every key visible; the block-causal mask is
  * expressed by which segments are passed).  q: DEVICE [H, Tq, d]; segment s:
  * k_seg[s], v_seg[s] DEVICE [H, seg_len[s], d] (HOST arrays of nseg pointers /
- * lengths, 1 <= nseg <= LA_MAX_WINDOW + 2, seg_len >= 1); out DEVICE [Tq, H*d].
- * dtype LA_BF16 needs d == 128 (tcgen05), LA_FP32 any even d <= 128.
+ * lengths, 1 <= nseg <= LA_MAX_WINDOW + 2, seg_len >= 1).
+ * dtype LA_FP16: q/K/V fp16, d == 128, tcgen05; out DEVICE bf16 [Tq, H*d] and,
+ *   if out32 != NULL, an fp32 copy [Tq, H*d] (the value before rounding).
+ * dtype LA_FP32: q/K/V/out fp32, d % 8 == 0, d <= 128, SIMT; out32 ignored.
  */
 int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t d,
                     int32_t nseg, const void* const* k_seg, const void* const* v_seg,
-                    const int64_t* seg_len, void* out, void* cuda_stream);
+                    const int64_t* seg_len, void* out, float* out32, void* cuda_stream);
 
 /*
  * Standalone Euler update x[r, :] += dt[r / rows_per_group] * v[r, :] over

@@ -11,11 +11,11 @@ LIB_PATH = os.path.join(_HERE, "libla.so")
 LA_OK, LA_EINVAL, LA_ESTATE, LA_ENOMEM, LA_ECUDA, LA_EDEVICE = 0, -1, -2, -3, -4, -5
 LA_SINK_FIXED, LA_SINK_AAS = 0, 1
 LA_SCHED_PIPELINED, LA_SCHED_SEQUENTIAL = 0, 1
-LA_BF16, LA_FP32 = 0, 1
+LA_BF16, LA_FP32, LA_FP16 = 0, 1, 2
 LA_MAX_STEPS, LA_MAX_WINDOW, LA_MAX_FPB = 8, 14, 7
-LA_EPI_STORE, LA_EPI_RESID, LA_EPI_SET32, LA_EPI_EULER = 0, 1, 2, 3
+LA_EPI_STORE, LA_EPI_RESID, LA_EPI_SET32, LA_EPI_EULER, LA_EPI_STORE32 = 0, 1, 2, 3, 4
 
-TAP = dict(x_in=0, x_out=1, h=2, q=3, o=4, v=5, ring_k=6, ring_v=7, sink_k=8, sink_v=9, sink_k_rope=10)
+TAP = dict(x_in=0, x_out=1, h=2, q=3, o=4, v=5, ring_k=6, ring_v=7, sink_k=8, sink_v=9, sink_k_rope=10, sink_h=11)
 KIND = dict(in_proj=0, qkv_gemm=1, rope=2, attn=3, out_gemm=4, head=5, other=6)
 
 
@@ -72,7 +72,7 @@ def load():
         "la_op_gemm": (c_int, [c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64,
                                c_int64, POINTER(c_float), c_int64, c_void_p]),
         "la_op_attention": (c_int, [c_int32, c_void_p, c_int64, c_int32, c_int32, c_int32, POINTER(c_void_p),
-                                    POINTER(c_void_p), POINTER(c_int64), c_void_p, c_void_p]),
+                                    POINTER(c_void_p), POINTER(c_int64), c_void_p, c_void_p, c_void_p]),
         "la_op_euler": (c_int, [c_void_p, c_void_p, c_int64, c_int64, POINTER(c_float), c_int64, c_void_p]),
     }
     for name, (res, args) in sig.items():

@@ -1,4 +1,5 @@
-// Block-causal attention on tcgen05 tensor cores, head_dim 128, bf16 in / fp32 softmax.
+// Block-causal attention on tcgen05 tensor cores, head_dim 128: fp16 q/K/V/P
+// operands, fp32 scores, softmax and accumulation, bf16 output.
 //
 // One CTA = 128 queries of one (group, head); the keys are the group's list of
 // segments [sink | window blocks oldest first | the block itself], walked in
@@ -13,8 +14,11 @@
 //   warps 2..5  softmax: thread = query row = TMEM lane.  tcgen05.ld of the S
 //               row, masked row max, exp2, row sum, lazy rescale of O in TMEM
 //               (only when the running max grows by more than 2^8), P written
-//               to shared memory as bf16 in the swizzled K-major layout, then
-//               the final 1/l normalisation and bf16 store.
+//               to shared memory as fp16 in the swizzled K-major layout, then
+//               the final 1/l normalisation and bf16 store (plus an optional
+//               fp32 copy).
+// fp16 rather than bf16 for q, K, V and P: same bytes and tensor-core rate,
+// 3 more mantissa bits; P <= 2^8 by construction and q/K/V saturate at 65504.
 // S_{t+1} is computed on the tensor cores while the softmax warps work on S_t.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -128,8 +132,8 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(BQ, BKV, false, false);
-      constexpr uint32_t idPV = idesc_bf16(BQ, 128, false, true);
+      constexpr uint32_t idS = idesc_fp16(BQ, BKV, false, false);
+      constexpr uint32_t idPV = idesc_fp16(BQ, 128, false, true);
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t p_addr = smem_u32(sP);
       bool ok = mbar_wait(q_full, 0, err);
@@ -223,7 +227,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
         const float p0 = c < valid ? fast_exp2(fmaf(__uint_as_float(s[c]), sc, -m_new)) : 0.f;
         const float p1 = c + 1 < valid ? fast_exp2(fmaf(__uint_as_float(s[c + 1]), sc, -m_new)) : 0.f;
         rs += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+        pk[c / 2] = pack_f16x2(p0, p1);
       }
       l = l * alpha + rs;
       m_ref = m_new;
@@ -264,23 +268,32 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       tc_fence_after();
       const float inv = 1.0f / l;
       const bool store = q0 + r < p.Tq;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                            (static_cast<long long>(g.out_row0) + q0 + r) * p.out_ld + static_cast<long long>(h) * 128;
+      const long long orow_idx = static_cast<long long>(g.out_row0) + q0 + r;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + orow_idx * p.out_ld + static_cast<long long>(h) * 128;
+      float* orow32 = p.out32 ? p.out32 + orow_idx * p.out_ld + static_cast<long long>(h) * 128 : nullptr;
 #pragma unroll 1
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_off + O_COL + c4 * 32, o);
         tmem_ld_wait();
         if (store) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o[i]) * inv;
           uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+            w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+            w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+            w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+            w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
             dst[i] = w;
+          }
+          if (orow32) {
+            float4* d32 = reinterpret_cast<float4*>(orow32 + c4 * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) d32[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
         }
       }

@@ -55,7 +55,8 @@ struct AttnParams {
   int Tq;               // queries per group
   int H, d;
   float scale_log2;     // log2(e) / sqrt(d)
-  void* out;            // [rows, H*d] dtype
+  void* out;            // [rows, H*d] bf16 (tcgen05 path) / fp32 (SIMT path)
+  float* out32;         // optional fp32 copy of the output (tcgen05 path)
   long long out_ld;     // elements per output row
   int* err;
   // raw pointers for the SIMT path: element offset of (slice, h, n, e) is
@@ -67,7 +68,24 @@ struct AttnParams {
   int vrows[LA_MAX_SEG];
 };
 
-enum GemmEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SET32 = 2, EPI_EULER = 3 };
+enum GemmEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SET32 = 2, EPI_EULER = 3, EPI_STORE32 = 4, EPI_QKV_ROPE = 5 };
+
+// QKV projection epilogue: rotate q and k (Rolling 3D RoPE) on the fp32
+// accumulators and append K/V to the ring, rounding once to the attention
+// operand type (fp16).  Rows of inactive buffers are not written.
+struct QkvRopeParams {
+  int T, F, H, d, D, E, grid_w;
+  int pt, ph;
+  int active[LA_MAX_STEPS];
+  int slot[LA_MAX_STEPS];
+  int write_entry[LA_MAX_STEPS];
+  long long ring_slice0;     // slice of (layer, slot 0, entry 0)
+  const float* tcos; const float* tsin;   // [LA_MAX_STEPS][LA_TROWS][LA_MAX_PT]
+  const float* rcos; const float* rsin;   // [grid_h][ph]
+  const float* ccos; const float* csin;   // [grid_w][pw]
+  void* q_rope;              // [nbuf][H][T][d]
+  void* ring_k; void* ring_v;// [L][S][E][H][T][d]
+};
 
 struct GemmEpiParams {
   int kind;
@@ -79,5 +97,8 @@ struct GemmEpiParams {
   int active[LA_MAX_STEPS];   // EULER: only active groups update
   float* vtap;          // optional fp32 [M, N] copy of acc (velocity capture)
 };
+
+// Largest finite fp16 magnitude; attention operands saturate there.
+#define LA_F16_MAX 65504.0f
 
 static inline int ceil_div_i(long long a, long long b) { return (int)((a + b - 1) / b); }

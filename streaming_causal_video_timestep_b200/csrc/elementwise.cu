@@ -1,5 +1,7 @@
 // Bandwidth-bound kernels: RoPE tables, fused Rolling RoPE + ring append +
 // sink re-rope, the sink's K/V split, in-projection helpers and the Euler update.
+#include <cuda_fp16.h>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -23,6 +25,19 @@ template <> struct Vec8<__nv_bfloat16> {
     w.y = pack_bf16x2(v[2], v[3]);
     w.z = pack_bf16x2(v[4], v[5]);
     w.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = w;
+  }
+};
+template <> struct Vec8<__half> {
+  static __device__ __forceinline__ void store(__half* p, const float (&v)[8]) {
+    float c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = fminf(fmaxf(v[i], -LA_F16_MAX), LA_F16_MAX);
+    uint4 w;
+    w.x = pack_f16x2(c[0], c[1]);
+    w.y = pack_f16x2(c[2], c[3]);
+    w.z = pack_f16x2(c[4], c[5]);
+    w.w = pack_f16x2(c[6], c[7]);
     *reinterpret_cast<uint4*>(p) = w;
   }
 };
@@ -82,12 +97,15 @@ __global__ void k_rope_ttab(const __grid_constant__ PassDesc pd, int fpb, int pt
   }
 }
 
-template <typename T>
+// Rolling RoPE + ring append from an fp32 [q | k | v] projection (fp32
+// streams), and the per-block re-rope of the fp32 un-roped sink K for every
+// active buffer (both streams).  Outputs are rounded once to TO.
+template <typename TO>
 __global__ void __launch_bounds__(256) k_rope_append(const __grid_constant__ PassDesc pd,
                                                      const __grid_constant__ RopeArgs a, long long n_main,
                                                      long long n_sink) {
   const int chunks = a.d / 8;
-  const T* qkv = reinterpret_cast<const T*>(a.qkv);
+  const float* qkv = reinterpret_cast<const float*>(a.qkv);
   const long long total = n_main + n_sink;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -100,21 +118,21 @@ __global__ void __launch_bounds__(256) k_rope_append(const __grid_constant__ Pas
       const int buf = pd.active_buf[rest];
       const long long row = static_cast<long long>(buf) * a.T + n;
       float v[8];
-      Vec8<T>::load(qkv + row * 3 * a.D + part * a.D + h * a.d + ch * 8, v);
+      Vec8<float>::load(qkv + row * 3 * a.D + part * a.D + h * a.d + ch * 8, v);
       if (part < 2) {
         const int f = n / a.F, rem = n % a.F;
         rotate8(v, ch, buf, f, rem / a.grid_w, rem % a.grid_w, a);
       }
-      T* dst;
+      TO* dst;
       const long long tok = static_cast<long long>(n) * a.d + ch * 8;
       if (part == 0) {
-        dst = reinterpret_cast<T*>(a.q_rope) + (static_cast<long long>(buf) * a.H + h) * a.T * a.d + tok;
+        dst = reinterpret_cast<TO*>(a.q_rope) + (static_cast<long long>(buf) * a.H + h) * a.T * a.d + tok;
       } else {
         const long long slice = a.ring_slice0 + static_cast<long long>(pd.slot[buf]) * a.E + pd.write_entry[buf];
-        T* base = reinterpret_cast<T*>(part == 1 ? a.ring_k : a.ring_v);
+        TO* base = reinterpret_cast<TO*>(part == 1 ? a.ring_k : a.ring_v);
         dst = base + (slice * a.H + h) * a.T * a.d + tok;
       }
-      Vec8<T>::store(dst, v);
+      Vec8<TO>::store(dst, v);
     } else {
       long long rest = idx - n_main;
       const int ch = static_cast<int>(rest % chunks); rest /= chunks;
@@ -123,19 +141,22 @@ __global__ void __launch_bounds__(256) k_rope_append(const __grid_constant__ Pas
       const int buf = pd.active_buf[rest];
       const long long off = (static_cast<long long>(h) * a.F + m) * a.d + ch * 8;
       float v[8];
-      Vec8<T>::load(reinterpret_cast<const T*>(a.sink_k) + off, v);
+      Vec8<float>::load(reinterpret_cast<const float*>(a.sink_k) + off, v);
       rotate8(v, ch, buf, a.fpb, m / a.grid_w, m % a.grid_w, a);
-      Vec8<T>::store(reinterpret_cast<T*>(a.sink_k_rope) + static_cast<long long>(buf) * a.H * a.F * a.d + off, v);
+      Vec8<TO>::store(reinterpret_cast<TO*>(a.sink_k_rope) + static_cast<long long>(buf) * a.H * a.F * a.d + off, v);
     }
   }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(256) k_sink_qkv(const __grid_constant__ RopeArgs a, T* sink_k_raw, T* sink_v,
-                                                  T* q_rope, T* k_rope) {
+// Sink pass: split the fp32 projection [F, 3D] into the layer's un-roped K
+// (fp32, kept for re-roping), V (TO), and roped q / k (TO) for the sink's
+// self-attention (temporal row 0 of buffer 0 of the table).
+template <typename TO>
+__global__ void __launch_bounds__(256) k_sink_qkv(const __grid_constant__ RopeArgs a, float* sink_k_raw, TO* sink_v,
+                                                  TO* q_rope, TO* k_rope) {
   const int chunks = a.d / 8;
   const long long total = static_cast<long long>(a.F) * 3 * a.H * chunks;
-  const T* qkv = reinterpret_cast<const T*>(a.qkv);
+  const float* qkv = reinterpret_cast<const float*>(a.qkv);
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
     long long rest = idx;
@@ -144,15 +165,15 @@ __global__ void __launch_bounds__(256) k_sink_qkv(const __grid_constant__ RopeAr
     const int part = static_cast<int>(rest % 3); rest /= 3;
     const int m = static_cast<int>(rest);
     float v[8];
-    Vec8<T>::load(qkv + static_cast<long long>(m) * 3 * a.D + part * a.D + h * a.d + ch * 8, v);
+    Vec8<float>::load(qkv + static_cast<long long>(m) * 3 * a.D + part * a.D + h * a.d + ch * 8, v);
     const long long off = (static_cast<long long>(h) * a.F + m) * a.d + ch * 8;
     if (part == 2) {
-      Vec8<T>::store(sink_v + off, v);
+      Vec8<TO>::store(sink_v + off, v);
       continue;
     }
-    if (part == 1) Vec8<T>::store(sink_k_raw + off, v);
+    if (part == 1) Vec8<float>::store(sink_k_raw + off, v);
     rotate8(v, ch, 0, 0, m / a.grid_w, m % a.grid_w, a);
-    Vec8<T>::store(part == 0 ? q_rope + off : k_rope + off, v);
+    Vec8<TO>::store(part == 0 ? q_rope + off : k_rope + off, v);
   }
 }
 
@@ -219,30 +240,30 @@ cudaError_t launch_rope_ttab(const PassDesc& pd, int fpb, int pt, const double* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_rope_append(int bf16, const PassDesc& pd, const RopeArgs& a, cudaStream_t st) {
+cudaError_t launch_rope_append(int f16_out, const PassDesc& pd, const RopeArgs& a, bool main_part,
+                               cudaStream_t st) {
   const long long chunks = a.d / 8;
-  const long long n_main = static_cast<long long>(pd.nactive) * a.T * 3 * a.H * chunks;
+  const long long n_main = main_part ? static_cast<long long>(pd.nactive) * a.T * 3 * a.H * chunks : 0;
   const long long n_sink = a.sink_k ? static_cast<long long>(pd.nactive) * a.F * a.H * chunks : 0;
+  if (n_main + n_sink == 0) return cudaSuccess;
   const int grid = grid_for(n_main + n_sink);
-  if (bf16)
-    k_rope_append<__nv_bfloat16><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
+  if (f16_out)
+    k_rope_append<__half><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
   else
     k_rope_append<float><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
   return cudaGetLastError();
 }
 
-cudaError_t launch_sink_qkv(int bf16, const RopeArgs& a, void* sink_k_raw, void* sink_v, void* q_rope, void* k_rope,
-                            cudaStream_t st) {
+cudaError_t launch_sink_qkv(int f16_out, const RopeArgs& a, float* sink_k_raw, void* sink_v, void* q_rope,
+                            void* k_rope, cudaStream_t st) {
   const long long n = static_cast<long long>(a.F) * 3 * a.H * (a.d / 8);
   const int grid = grid_for(n);
-  if (bf16)
-    k_sink_qkv<__nv_bfloat16><<<grid, 256, 0, st>>>(a, static_cast<__nv_bfloat16*>(sink_k_raw),
-                                                     static_cast<__nv_bfloat16*>(sink_v),
-                                                     static_cast<__nv_bfloat16*>(q_rope),
-                                                     static_cast<__nv_bfloat16*>(k_rope));
+  if (f16_out)
+    k_sink_qkv<__half><<<grid, 256, 0, st>>>(a, sink_k_raw, static_cast<__half*>(sink_v),
+                                              static_cast<__half*>(q_rope), static_cast<__half*>(k_rope));
   else
-    k_sink_qkv<float><<<grid, 256, 0, st>>>(a, static_cast<float*>(sink_k_raw), static_cast<float*>(sink_v),
-                                            static_cast<float*>(q_rope), static_cast<float*>(k_rope));
+    k_sink_qkv<float><<<grid, 256, 0, st>>>(a, sink_k_raw, static_cast<float*>(sink_v), static_cast<float*>(q_rope),
+                                            static_cast<float*>(k_rope));
   return cudaGetLastError();
 }
 

@@ -10,6 +10,8 @@
 // The two accumulators let the epilogue of tile n overlap the main loop of n+1.
 // Tiles are visited in bands of GROUP_M row-blocks so the A band and the W
 // tiles in flight stay L2-resident.
+#include <cuda_fp16.h>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -52,10 +54,80 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
   }
 }
 
-__device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, long long row, long long col,
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+  lo = fminf(fmaxf(lo, -LA_F16_MAX), LA_F16_MAX);
+  hi = fminf(fmaxf(hi, -LA_F16_MAX), LA_F16_MAX);
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 32 consecutive columns of one head of the [q | k | v] projection of one token:
+// rotate the pairs of q and k, then write fp16 to q_rope / the ring entry.
+__device__ __forceinline__ void qkv_rope_row32(const QkvRopeParams& qp, long long row, long long col,
                                                float (&acc)[32]) {
+  const int buf = static_cast<int>(row / qp.T);
+  const int n = static_cast<int>(row - static_cast<long long>(buf) * qp.T);
+  if (!qp.active[buf]) return;
+  const int part = static_cast<int>(col / qp.D);
+  const int cc = static_cast<int>(col - static_cast<long long>(part) * qp.D);
+  const int h = cc / qp.d, e0 = cc - h * qp.d;
+  if (part < 2) {
+    const int f = n / qp.F, rem = n - f * qp.F;
+    const int rr = rem / qp.grid_w, ccol = rem - rr * qp.grid_w;
+    const int pw_base = qp.pt + qp.ph;
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const int j = (e0 >> 1) + jj;
+      float c, sn;
+      if (j < qp.pt) {
+        const int idx = (buf * LA_TROWS + f) * LA_MAX_PT + j;
+        c = qp.tcos[idx]; sn = qp.tsin[idx];
+      } else if (j < pw_base) {
+        const int idx = rr * qp.ph + (j - qp.pt);
+        c = qp.rcos[idx]; sn = qp.rsin[idx];
+      } else {
+        const int pw = qp.d / 2 - pw_base;
+        const int idx = ccol * pw + (j - pw_base);
+        c = qp.ccos[idx]; sn = qp.csin[idx];
+      }
+      const float x0 = acc[2 * jj], x1 = acc[2 * jj + 1];
+      acc[2 * jj] = x0 * c - x1 * sn;
+      acc[2 * jj + 1] = x0 * sn + x1 * c;
+    }
+  }
+  __half* dst;
+  const long long tok = static_cast<long long>(n) * qp.d + e0;
+  if (part == 0) {
+    dst = reinterpret_cast<__half*>(qp.q_rope) + (static_cast<long long>(buf) * qp.H + h) * qp.T * qp.d + tok;
+  } else {
+    const long long slice = qp.ring_slice0 + static_cast<long long>(qp.slot[buf]) * qp.E + qp.write_entry[buf];
+    dst = reinterpret_cast<__half*>(part == 1 ? qp.ring_k : qp.ring_v) + (slice * qp.H + h) * qp.T * qp.d + tok;
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 w;
+    w.x = pack_f16x2_sat(acc[8 * i + 0], acc[8 * i + 1]);
+    w.y = pack_f16x2_sat(acc[8 * i + 2], acc[8 * i + 3]);
+    w.z = pack_f16x2_sat(acc[8 * i + 4], acc[8 * i + 5]);
+    w.w = pack_f16x2_sat(acc[8 * i + 6], acc[8 * i + 7]);
+    d4[i] = w;
+  }
+}
+
+__device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, const QkvRopeParams& qp, long long row,
+                                               long long col, float (&acc)[32]) {
   const long long off = row * ep.ld + col;
   switch (ep.kind) {
+    case EPI_QKV_ROPE:
+      qkv_rope_row32(qp, row, col, acc);
+      break;
+    case EPI_STORE32: {
+      float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + off);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o4[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+      break;
+    }
     case EPI_STORE:
       store_bf16x32(reinterpret_cast<__nv_bfloat16*>(ep.out) + off, acc);
       break;
@@ -111,7 +183,8 @@ __device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, long lon
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const GemmEpiParams ep, int M, int N, int K, int* err) {
+          const __grid_constant__ GemmEpiParams ep, const __grid_constant__ QkvRopeParams qp, int M, int N, int K,
+          int* err) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -236,7 +309,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          epilogue_row32(ep, row, col, v);
+          epilogue_row32(ep, qp, row, col, v);
         }
       }
       tc_fence_before();
@@ -255,15 +328,15 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 }
 
 template <int BN>
-cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M, int N,
-                      int K, int* err, int num_sms, cudaStream_t st) {
+cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep,
+                      const QkvRopeParams& qp, int M, int N, int K, int* err, int num_sms, cudaStream_t st) {
   using C = GemmCfg<BN>;
   cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::SMEM));
   if (e != cudaSuccess) return e;
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  k_gemm_tc<BN><<<grid, 192, C::SMEM, st>>>(tmA, tmB, ep, M, N, K, err);
+  k_gemm_tc<BN><<<grid, 192, C::SMEM, st>>>(tmA, tmB, ep, qp, M, N, K, err);
   return cudaGetLastError();
 }
 
@@ -276,10 +349,12 @@ int gemm_tc_pick_bn(int N) {
 }
 
 cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M, int N,
-                           int K, int bn, int* err, int num_sms, cudaStream_t st) {
+                           int K, int bn, int* err, int num_sms, cudaStream_t st, const QkvRopeParams* qp) {
+  QkvRopeParams none{};
+  const QkvRopeParams& q = qp ? *qp : none;
   switch (bn) {
-    case 256: return launch_bn<256>(tmA, tmB, ep, M, N, K, err, num_sms, st);
-    case 128: return launch_bn<128>(tmA, tmB, ep, M, N, K, err, num_sms, st);
-    default: return launch_bn<64>(tmA, tmB, ep, M, N, K, err, num_sms, st);
+    case 256: return launch_bn<256>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
+    case 128: return launch_bn<128>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
+    default: return launch_bn<64>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
   }
 }

@@ -8,11 +8,12 @@
 
 // ---- tcgen05 (bf16) ----------------------------------------------------------------
 int gemm_tc_pick_bn(int N);
+// qp: parameters of the EPI_QKV_ROPE epilogue (NULL for the others).
 cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M, int N,
-                           int K, int bn, int* err, int num_sms, cudaStream_t st);
+                           int K, int bn, int* err, int num_sms, cudaStream_t st, const QkvRopeParams* qp = nullptr);
 
 // Tensor maps of an attention launch: q (d, Tq, H, q slices) and k[m]/v[m]
-// (d, rows_m, H, slices), bf16, 128-byte swizzle, box (64, 128, 1, 1).
+// (d, rows_m, H, slices), fp16, 128-byte swizzle, box (64, 128, 1, 1).
 struct AttnMaps {
   CUtensorMap q;
   CUtensorMap k[LA_MAX_SEG];
@@ -37,19 +38,22 @@ struct RopeArgs {
   const float* tcos;  const float* tsin;       // [LA_MAX_STEPS][LA_TROWS][LA_MAX_PT]
   const float* rcos;  const float* rsin;       // [grid_h][ph]
   const float* ccos;  const float* csin;       // [grid_w][pw]
-  const void* qkv;                             // [nbuf*T, 3D]
+  const void* qkv;                             // fp32 [nbuf*T, 3D]
   void* q_rope;                                // [nbuf][H][T][d]
   void* ring_k; void* ring_v;                  // [L][S][E][H][T][d]
   long long ring_slice0;                       // (layer*S) * E: slice of (layer, slot 0, entry 0)
   int E;
-  const void* sink_k;                          // un-roped [H][F][d] of this layer
+  const void* sink_k;                          // fp32 un-roped [H][F][d] of this layer (NULL: no sink part)
   void* sink_k_rope;                           // [nbuf][H][F][d]
 };
-cudaError_t launch_rope_append(int bf16, const PassDesc& pd, const RopeArgs& a, cudaStream_t st);
+// Outputs are fp16 (f16_out) or fp32.  main_part: also rope/append the block
+// from qkv (fp32 streams; bf16 streams do that in the QKV GEMM epilogue).
+cudaError_t launch_rope_append(int f16_out, const PassDesc& pd, const RopeArgs& a, bool main_part,
+                               cudaStream_t st);
 
-// Sink pass: split qkv [F, 3D] into un-roped K and V of the layer, and roped
-// q / k (temporal row 0 of buffer 0 of the table) for the sink's self-attention.
-cudaError_t launch_sink_qkv(int bf16, const RopeArgs& a, void* sink_k_raw, void* sink_v, void* q_rope,
+// Sink pass: split the fp32 qkv [F, 3D] into the layer's fp32 un-roped K, its
+// V, and roped q / k (temporal row 0 of buffer 0 of the table).
+cudaError_t launch_sink_qkv(int f16_out, const RopeArgs& a, float* sink_k_raw, void* sink_v, void* q_rope,
                             void* k_rope, cudaStream_t st);
 
 // x (fp32 [rows, C]) -> h32 (fp32) and hop (dtype) when C == D (identity in-proj),

@@ -24,8 +24,8 @@ extern "C" {
 int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, void* out, float* h32, int64_t M,
                int64_t N, int64_t K, const float* dt, int64_t rows_per_group, void* cuda_stream) {
   if (!A || !W || M < 1 || N < 1 || K < 1 || M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return LA_EINVAL;
-  if (epilogue < LA_EPI_STORE || epilogue > LA_EPI_EULER) return LA_EINVAL;
-  if (epilogue == LA_EPI_STORE && !out) return LA_EINVAL;
+  if (epilogue < LA_EPI_STORE || epilogue > LA_EPI_STORE32) return LA_EINVAL;
+  if ((epilogue == LA_EPI_STORE || epilogue == LA_EPI_STORE32) && !out) return LA_EINVAL;
   if (epilogue == LA_EPI_RESID && (!out || !h32)) return LA_EINVAL;
   if ((epilogue == LA_EPI_SET32 || epilogue == LA_EPI_EULER) && !h32) return LA_EINVAL;
   GemmEpiParams ep{};
@@ -58,7 +58,7 @@ int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, vo
 
 int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t d, int32_t nseg,
                     const void* const* k_seg, const void* const* v_seg, const int64_t* seg_len, void* out,
-                    void* cuda_stream) {
+                    float* out32, void* cuda_stream) {
   if (!q || !out || !k_seg || !v_seg || !seg_len || Tq < 1 || Tq > (1 << 30) || H < 1 || H > 65535) return LA_EINVAL;
   if (nseg < 1 || nseg > LA_MAX_SEG || d < 8 || d > 128 || d % 8 != 0) return LA_EINVAL;
   for (int s = 0; s < nseg; ++s)
@@ -70,6 +70,7 @@ int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t
   p.d = d;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   p.out = out;
+  p.out32 = dtype == LA_FP16 ? out32 : nullptr;
   p.out_ld = static_cast<long long>(H) * d;
   p.err = nullptr;
   p.qbase = q;
@@ -85,15 +86,15 @@ int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t
     p.vrows[s] = static_cast<int>(seg_len[s]);
   }
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  if (dtype == LA_BF16) {
+  if (dtype == LA_FP16) {
     if (d != 128) return LA_EINVAL;
     std::string err;
     if (!tmap_init(err)) return LA_ECUDA;
     AttnMaps maps;
-    if (!tmap_planes_bf16(&maps.q, q, d, Tq, H, 1, err)) return LA_ECUDA;
+    if (!tmap_planes_f16(&maps.q, q, d, Tq, H, 1, err)) return LA_ECUDA;
     for (int s = 0; s < nseg; ++s) {
-      if (!tmap_planes_bf16(&maps.k[s], k_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
-      if (!tmap_planes_bf16(&maps.v[s], v_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
+      if (!tmap_planes_f16(&maps.k[s], k_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
+      if (!tmap_planes_f16(&maps.v[s], v_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
     }
     return ret(launch_attn_tc(maps, p, st));
   }

@@ -141,7 +141,8 @@ struct la_stream {
   int S = 0, E = 0, F = 0, T = 0, D = 0, C = 0, H = 0, d = 0, L = 0, fpb = 0, nbuf = 0;
   int pt = 0, ph = 0, pw = 0;
   bool bf16 = true, id_in = true, id_head = true;
-  size_t es = 2;
+  size_t es = 2;            // activation / weight element (bf16 or fp32)
+  size_t ea = 2;            // attention operand element (fp16 or fp32)
   int device = 0, num_sms = 148;
   cudaStream_t st = nullptr;
 
@@ -154,20 +155,20 @@ struct la_stream {
   float* h32 = nullptr;     // [nbuf*T][D]
   void* hop = nullptr;      // [nbuf*T][D] dtype (fp32: == h32)
   void* xop = nullptr;      // [nbuf*T][C] bf16 (bf16 with an in-projection)
-  void* qkv = nullptr;      // [nbuf*T][3D]
-  void* q_rope = nullptr;   // [nbuf][H][T][d]
-  void* sk_rope = nullptr;  // [nbuf][H][F][d]
-  void* attn_o = nullptr;   // [nbuf*T][D]
-  void* ring_k = nullptr;   // [L][S][E][H][T][d]
+  float* qkv = nullptr;     // fp32 [nbuf*T][3D] (fp32 streams; bf16 fuses it into the GEMM)
+  void* q_rope = nullptr;   // attn type [nbuf][H][T][d]
+  void* sk_rope = nullptr;  // attn type [nbuf][H][F][d]
+  void* attn_o = nullptr;   // dtype [nbuf*T][D]
+  void* ring_k = nullptr;   // attn type [L][S][E][H][T][d]
   void* ring_v = nullptr;
-  void* sink_k = nullptr;   // [L][H][F][d] un-roped
-  void* sink_v = nullptr;
+  float* sink_k = nullptr;  // fp32 [L][H][F][d] un-roped
+  void* sink_v = nullptr;   // attn type [L][H][F][d]
   float* sink_x = nullptr;  // [F][C]
   float* s_h32 = nullptr;   // [F][D]
   void* s_hop = nullptr;
   void* s_xop = nullptr;
-  void* s_qkv = nullptr;
-  void* s_q = nullptr;      // [H][F][d]
+  float* s_qkv = nullptr;   // fp32 [F][3D]
+  void* s_q = nullptr;      // attn type [H][F][d]
   void* s_k = nullptr;
   void* s_o = nullptr;      // [F][D]
   double* omega_t = nullptr;
@@ -194,10 +195,13 @@ struct la_stream {
   float* cap_xout = nullptr;  // [S][T][C]
   float* cap_v = nullptr;     // [S][T][C]
   float* cap_vall = nullptr;  // [nbuf*T][C]
+  float* cap_oall = nullptr;  // fp32 [nbuf*T][D] (attention output before rounding)
   float* cap_h = nullptr;     // [S][L+1][T][D]
-  void* cap_q = nullptr;      // [S][L][H][T][d]
-  void* cap_o = nullptr;      // [S][L][T][D]
-  void* cap_sk = nullptr;     // [S][L][H][F][d]
+  void* cap_q = nullptr;      // attn type [S][L][H][T][d]
+  float* cap_o = nullptr;     // fp32 [S][L][T][D]
+  void* cap_sk = nullptr;     // attn type [S][L][H][F][d]
+  float* cap_sink_h = nullptr;  // fp32 [L][F][D] sink residual entering each layer
+  bool cap_sink_valid = false;
   std::vector<int> cap_valid;  // per slot: captured in the last call
 
   bool prof = false;
@@ -348,8 +352,9 @@ char* elem(void* base, long long idx, size_t es) { return static_cast<char*>(bas
 
 int capture_pass(la_stream* s, const PassDesc& pd, int layer) {
   // copy the intermediates of every active buffer into its slot's capture area
-  const size_t es = s->es;
+  const size_t ea = s->ea;
   const long long T = s->T, D = s->D, H = s->H, d = s->d, F = s->F, L = s->L;
+  const float* o32 = s->bf16 ? s->cap_oall : static_cast<const float*>(s->attn_o);
   for (int ai = 0; ai < pd.nactive; ++ai) {
     const int buf = pd.active_buf[ai];
     const int slot = pd.slot[buf];
@@ -360,12 +365,12 @@ int capture_pass(la_stream* s, const PassDesc& pd, int layer) {
     }
     CU(cudaMemcpyAsync(s->cap_h + (static_cast<long long>(slot) * (L + 1) + layer + 1) * T * D, s->h32 + buf * T * D,
                        T * D * 4, cudaMemcpyDeviceToDevice, s->st));
-    CU(cudaMemcpyAsync(elem(s->cap_q, (static_cast<long long>(slot) * L + layer) * H * T * d, es),
-                       elem(s->q_rope, buf * H * T * d, es), H * T * d * es, cudaMemcpyDeviceToDevice, s->st));
-    CU(cudaMemcpyAsync(elem(s->cap_o, (static_cast<long long>(slot) * L + layer) * T * D, es),
-                       elem(s->attn_o, buf * T * D, es), T * D * es, cudaMemcpyDeviceToDevice, s->st));
-    CU(cudaMemcpyAsync(elem(s->cap_sk, (static_cast<long long>(slot) * L + layer) * H * F * d, es),
-                       elem(s->sk_rope, buf * H * F * d, es), H * F * d * es, cudaMemcpyDeviceToDevice, s->st));
+    CU(cudaMemcpyAsync(elem(s->cap_q, (static_cast<long long>(slot) * L + layer) * H * T * d, ea),
+                       elem(s->q_rope, buf * H * T * d, ea), H * T * d * ea, cudaMemcpyDeviceToDevice, s->st));
+    CU(cudaMemcpyAsync(s->cap_o + (static_cast<long long>(slot) * L + layer) * T * D, o32 + buf * T * D, T * D * 4,
+                       cudaMemcpyDeviceToDevice, s->st));
+    CU(cudaMemcpyAsync(elem(s->cap_sk, (static_cast<long long>(slot) * L + layer) * H * F * d, ea),
+                       elem(s->sk_rope, buf * H * F * d, ea), H * F * d * ea, cudaMemcpyDeviceToDevice, s->st));
   }
   return LA_OK;
 }
@@ -415,18 +420,44 @@ int run_pass(la_stream* s, const PassDesc& pd) {
   ap.kbase[1] = s->sk_rope; ap.vbase[1] = s->sink_v; ap.krows[1] = F; ap.vrows[1] = F;
   ap.ngroups = pd.nactive;
 
+  QkvRopeParams qp{};
+  qp.T = T; qp.F = F; qp.H = H; qp.d = d; qp.D = D; qp.E = E; qp.grid_w = s->cfg.grid_w;
+  qp.pt = s->pt; qp.ph = s->ph;
+  for (int i = 0; i < LA_MAX_STEPS; ++i) {
+    qp.active[i] = pd.active[i];
+    qp.slot[i] = pd.slot[i];
+    qp.write_entry[i] = pd.write_entry[i];
+  }
+  qp.tcos = s->tcos; qp.tsin = s->tsin; qp.rcos = s->rcos; qp.rsin = s->rsin; qp.ccos = s->ccos; qp.csin = s->csin;
+  qp.q_rope = s->q_rope; qp.ring_k = s->ring_k; qp.ring_v = s->ring_v;
+  ap.out32 = (s->bf16 && s->capture) ? s->cap_oall : nullptr;
+
   for (int l = 0; l < s->L; ++l) {
-    // QKV projection
-    GemmEpiParams eq = epi(EPI_STORE, s->qkv, nullptr, 3LL * D);
-    if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_hop, &s->tm_wqkv[l], s->bf16 ? s->hop : s->h32, s->w_qkv[l], eq, rows,
-                  3 * D, D)) != LA_OK)
-      return r;
-    // Rolling RoPE + ring append + sink re-rope
     ra.qkv = s->qkv; ra.q_rope = s->q_rope; ra.ring_k = s->ring_k; ra.ring_v = s->ring_v;
     ra.ring_slice0 = static_cast<long long>(l) * S * E;
-    ra.sink_k = elem(s->sink_k, static_cast<long long>(l) * H * F * d, s->es);
+    ra.sink_k = s->sink_k + static_cast<long long>(l) * H * F * d;
     ra.sink_k_rope = s->sk_rope;
-    if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(s->bf16, pd, ra, s->st); })) != LA_OK) return r;
+    if (s->bf16) {
+      // QKV projection with Rolling RoPE + ring append fused into the epilogue
+      qp.ring_slice0 = ra.ring_slice0;
+      GemmEpiParams eq = epi(EPI_QKV_ROPE, nullptr, nullptr, 3LL * D);
+      const int bn = gemm_tc_pick_bn(3 * D);
+      if ((r = launch(s, LA_KIND_QKV_GEMM, [&] {
+             return launch_gemm_tc(s->tm_hop, s->tm_wqkv[l], eq, rows, 3 * D, D, bn, s->dev_err, s->num_sms, s->st,
+                                   &qp);
+           })) != LA_OK)
+        return r;
+      // per-block re-rope of the sink K (fp32 -> fp16, once per active buffer)
+      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(1, pd, ra, false, s->st); })) != LA_OK)
+        return r;
+    } else {
+      GemmEpiParams eq = epi(EPI_STORE, s->qkv, nullptr, 3LL * D);
+      if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_hop, &s->tm_wqkv[l], s->h32, s->w_qkv[l], eq, rows, 3 * D, D)) !=
+          LA_OK)
+        return r;
+      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(0, pd, ra, true, s->st); })) != LA_OK)
+        return r;
+    }
     // block-causal attention: [sink | window oldest first | self]
     for (int ai = 0; ai < pd.nactive; ++ai) {
       const int buf = pd.active_buf[ai];
@@ -525,13 +556,18 @@ int run_sink(la_stream* s) {
   ap.vbase[0] = s->sink_v; ap.vrows[0] = F;
   ap.ngroups = 1;
   for (int l = 0; l < s->L; ++l) {
-    GemmEpiParams eq = epi(EPI_STORE, s->s_qkv, nullptr, 3LL * D);
+    if (s->capture) {
+      CU(cudaMemcpyAsync(s->cap_sink_h + static_cast<long long>(l) * F * D, s->s_h32,
+                         static_cast<size_t>(F) * D * 4, cudaMemcpyDeviceToDevice, s->st));
+      s->cap_sink_valid = true;
+    }
+    GemmEpiParams eq = epi(s->bf16 ? EPI_STORE32 : EPI_STORE, s->s_qkv, nullptr, 3LL * D);
     if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_s_hop, &s->tm_wqkv[l], s->bf16 ? s->s_hop : s->s_h32, s->w_qkv[l], eq,
                   F, 3 * D, D)) != LA_OK)
       return r;
     ra.qkv = s->s_qkv;
-    void* kraw = elem(s->sink_k, static_cast<long long>(l) * H * F * d, s->es);
-    void* vraw = elem(s->sink_v, static_cast<long long>(l) * H * F * d, s->es);
+    float* kraw = s->sink_k + static_cast<long long>(l) * H * F * d;
+    void* vraw = elem(s->sink_v, static_cast<long long>(l) * H * F * d, s->ea);
     if ((r = launch(s, LA_KIND_ROPE, [&] {
            return launch_sink_qkv(s->bf16, ra, kraw, vraw, s->s_q, s->s_k, s->st);
          })) != LA_OK)
@@ -625,15 +661,16 @@ int step_impl(la_stream* s, const float* x_new, float* x_out, int64_t* finished_
 int alloc_capture(la_stream* s) {
   if (s->cap_xin) return LA_OK;
   const long long S = s->S, T = s->T, C = s->C, D = s->D, L = s->L, H = s->H, d = s->d, F = s->F;
-  const size_t es = s->es;
   DALLOC(s->cap_xin, S * T * C * 4);
   DALLOC(s->cap_xout, S * T * C * 4);
   DALLOC(s->cap_v, S * T * C * 4);
   DALLOC(s->cap_vall, static_cast<long long>(s->nbuf) * T * C * 4);
+  DALLOC(s->cap_oall, static_cast<long long>(s->nbuf) * T * D * 4);
   DALLOC(s->cap_h, S * (L + 1) * T * D * 4);
-  DALLOC(s->cap_q, S * L * H * T * d * es);
-  DALLOC(s->cap_o, S * L * T * D * es);
-  DALLOC(s->cap_sk, S * L * H * F * d * es);
+  DALLOC(s->cap_q, S * L * H * T * d * s->ea);
+  DALLOC(s->cap_o, S * L * T * D * 4);
+  DALLOC(s->cap_sk, S * L * H * F * d * s->ea);
+  DALLOC(s->cap_sink_h, L * F * D * 4);
   s->cap_valid.assign(s->S, 0);
   return LA_OK;
 }
@@ -686,7 +723,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   s->fpb = cfg->frames_per_block; s->T = s->fpb * s->F; s->D = cfg->hidden; s->C = cfg->latent_ch;
   s->H = cfg->heads; s->d = cfg->head_dim; s->L = cfg->num_layers;
   s->pt = cfg->rope_split[0]; s->ph = cfg->rope_split[1]; s->pw = cfg->rope_split[2];
-  s->bf16 = cfg->dtype == LA_BF16; s->es = s->bf16 ? 2 : 4;
+  s->bf16 = cfg->dtype == LA_BF16; s->es = s->bf16 ? 2 : 4; s->ea = s->es;
   s->id_in = w->w_in == nullptr; s->id_head = w->w_head == nullptr;
   s->nbuf = cfg->schedule == LA_SCHED_PIPELINED ? s->S : 1;
   s->st = static_cast<cudaStream_t>(cuda_stream);
@@ -707,12 +744,12 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   // memory plan, checked before allocating
   const long long T = s->T, D = s->D, C = s->C, F = s->F, H = s->H, d = s->d, L = s->L, S = s->S, E = s->E;
   const long long NB = s->nbuf;
-  const size_t es = s->es;
+  const size_t es = s->es, ea = s->ea;
   const long long need = NB * T * C * 4 + NB * T * D * 4 + (s->bf16 ? NB * T * D * es : 0) +
-                         (s->bf16 && !s->id_in ? NB * T * C * 2 : 0) + NB * T * 3 * D * es + NB * T * D * es * 2 +
-                         NB * H * F * d * es + 2 * L * S * E * H * T * d * es + 2 * L * H * F * d * es +
-                         F * C * 4 + F * D * 4 + F * D * es * 2 + F * C * 2 + F * 3 * D * es + 2 * H * F * d * es +
-                         (64 << 20);
+                         (s->bf16 && !s->id_in ? NB * T * C * 2 : 0) + (s->bf16 ? 0 : NB * T * 3 * D * 4) +
+                         NB * T * D * ea + NB * T * D * es + NB * H * F * d * ea + 2 * L * S * E * H * T * d * ea +
+                         L * H * F * d * (4 + ea) + F * C * 4 + F * D * 4 + F * D * es * 2 + F * C * 2 +
+                         F * 3 * D * 4 + 2 * H * F * d * ea + (64 << 20);
   size_t free_b = 0, total_b = 0;
   e = cudaMemGetInfo(&free_b, &total_b);
   if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
@@ -732,21 +769,21 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   ALLOC_OR_BAIL(s->h32, NB * T * D * 4);
   if (s->bf16) ALLOC_OR_BAIL(s->hop, NB * T * D * es); else s->hop = s->h32;
   if (s->bf16 && !s->id_in) ALLOC_OR_BAIL(s->xop, NB * T * C * 2);
-  ALLOC_OR_BAIL(s->qkv, NB * T * 3 * D * es);
-  ALLOC_OR_BAIL(s->q_rope, NB * T * D * es);
+  if (!s->bf16) ALLOC_OR_BAIL(s->qkv, NB * T * 3 * D * 4);
+  ALLOC_OR_BAIL(s->q_rope, NB * T * D * ea);
   ALLOC_OR_BAIL(s->attn_o, NB * T * D * es);
-  ALLOC_OR_BAIL(s->sk_rope, NB * H * F * d * es);
-  ALLOC_OR_BAIL(s->ring_k, L * S * E * H * T * d * es);
-  ALLOC_OR_BAIL(s->ring_v, L * S * E * H * T * d * es);
-  ALLOC_OR_BAIL(s->sink_k, L * H * F * d * es);
-  ALLOC_OR_BAIL(s->sink_v, L * H * F * d * es);
+  ALLOC_OR_BAIL(s->sk_rope, NB * H * F * d * ea);
+  ALLOC_OR_BAIL(s->ring_k, L * S * E * H * T * d * ea);
+  ALLOC_OR_BAIL(s->ring_v, L * S * E * H * T * d * ea);
+  ALLOC_OR_BAIL(s->sink_k, L * H * F * d * 4);
+  ALLOC_OR_BAIL(s->sink_v, L * H * F * d * ea);
   ALLOC_OR_BAIL(s->sink_x, F * C * 4);
   ALLOC_OR_BAIL(s->s_h32, F * D * 4);
   if (s->bf16) ALLOC_OR_BAIL(s->s_hop, F * D * es); else s->s_hop = s->s_h32;
   if (s->bf16 && !s->id_in) ALLOC_OR_BAIL(s->s_xop, F * C * 2);
-  ALLOC_OR_BAIL(s->s_qkv, F * 3 * D * es);
-  ALLOC_OR_BAIL(s->s_q, H * F * d * es);
-  ALLOC_OR_BAIL(s->s_k, H * F * d * es);
+  ALLOC_OR_BAIL(s->s_qkv, F * 3 * D * 4);
+  ALLOC_OR_BAIL(s->s_q, H * F * d * ea);
+  ALLOC_OR_BAIL(s->s_k, H * F * d * ea);
   ALLOC_OR_BAIL(s->s_o, F * D * es);
   ALLOC_OR_BAIL(s->omega_t, std::max(1, s->pt) * 8);
   ALLOC_OR_BAIL(s->tcos, LA_MAX_STEPS * LA_TROWS * LA_MAX_PT * 4);
@@ -803,14 +840,14 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
       ok = ok && tmap_2d_bf16(&s->tm_win, s->w_in, D, C, C, bn_d, s->err);
       ok = ok && tmap_2d_bf16(&s->tm_whead, s->w_head, C, D, D, bn_c, s->err);
     }
-    ok = ok && tmap_planes_bf16(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_stream.v[1], s->sink_v, d, F, H, L, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_sink.q, s->s_q, d, F, H, 1, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_sink.k[0], s->s_k, d, F, H, 1, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_sink.v[0], s->sink_v, d, F, H, L, s->err);
+    ok = ok && tmap_planes_f16(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
+    ok = ok && tmap_planes_f16(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
+    ok = ok && tmap_planes_f16(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
+    ok = ok && tmap_planes_f16(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
+    ok = ok && tmap_planes_f16(&s->maps_stream.v[1], s->sink_v, d, F, H, L, s->err);
+    ok = ok && tmap_planes_f16(&s->maps_sink.q, s->s_q, d, F, H, 1, s->err);
+    ok = ok && tmap_planes_f16(&s->maps_sink.k[0], s->s_k, d, F, H, 1, s->err);
+    ok = ok && tmap_planes_f16(&s->maps_sink.v[0], s->sink_v, d, F, H, L, s->err);
     if (!ok) return bail(LA_ECUDA);
   }
   e = cudaStreamSynchronize(s->st);
@@ -880,10 +917,10 @@ int la_debug_capture(la_stream* s, int32_t enable) {
 int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* dst, int64_t dst_bytes) {
   if (!s || !dst) return LA_EINVAL;
   const long long T = s->T, C = s->C, D = s->D, H = s->H, d = s->d, F = s->F, L = s->L, E = s->E, S = s->S;
-  const size_t es = s->es;
+  const size_t ea = s->ea;
   const bool per_layer = what == LA_TAP_H || what == LA_TAP_Q || what == LA_TAP_O || what == LA_TAP_RING_K ||
                          what == LA_TAP_RING_V || what == LA_TAP_SINK_K || what == LA_TAP_SINK_V ||
-                         what == LA_TAP_SINK_KROPE;
+                         what == LA_TAP_SINK_KROPE || what == LA_TAP_SINK_H;
   if (per_layer && (layer < (what == LA_TAP_H ? -1 : 0) || layer >= L)) return fail(s, LA_EINVAL, "bad layer");
   if (slot < 0 || slot >= S) return fail(s, LA_EINVAL, "bad slot");
   const void* src = nullptr;
@@ -896,18 +933,20 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
     case LA_TAP_X_OUT: src = s->cap_xout + slot * T * C; bytes = T * C * 4; break;
     case LA_TAP_V: src = s->cap_v + slot * T * C; bytes = T * C * 4; break;
     case LA_TAP_H: src = s->cap_h + (slot * (L + 1) + layer + 1) * T * D; bytes = T * D * 4; break;
-    case LA_TAP_Q: src = elem(s->cap_q, (slot * L + layer) * H * T * d, es); bytes = H * T * d * es; break;
-    case LA_TAP_O: src = elem(s->cap_o, (slot * L + layer) * T * D, es); bytes = T * D * es; break;
-    case LA_TAP_SINK_KROPE: src = elem(s->cap_sk, (slot * L + layer) * H * F * d, es); bytes = H * F * d * es; break;
+    case LA_TAP_Q: src = elem(s->cap_q, (slot * L + layer) * H * T * d, ea); bytes = H * T * d * ea; break;
+    case LA_TAP_O: src = s->cap_o + (slot * L + layer) * T * D; bytes = T * D * 4; break;
+    case LA_TAP_SINK_KROPE: src = elem(s->cap_sk, (slot * L + layer) * H * F * d, ea); bytes = H * F * d * ea; break;
     case LA_TAP_RING_K:
     case LA_TAP_RING_V:
-      src = elem(what == LA_TAP_RING_K ? s->ring_k : s->ring_v, (static_cast<long long>(layer) * S + slot) * E * H * T * d, es);
-      bytes = E * H * T * d * es;
+      src = elem(what == LA_TAP_RING_K ? s->ring_k : s->ring_v, (static_cast<long long>(layer) * S + slot) * E * H * T * d, ea);
+      bytes = E * H * T * d * ea;
       break;
-    case LA_TAP_SINK_K:
-    case LA_TAP_SINK_V:
-      src = elem(what == LA_TAP_SINK_K ? s->sink_k : s->sink_v, static_cast<long long>(layer) * H * F * d, es);
-      bytes = H * F * d * es;
+    case LA_TAP_SINK_K: src = s->sink_k + static_cast<long long>(layer) * H * F * d; bytes = H * F * d * 4; break;
+    case LA_TAP_SINK_V: src = elem(s->sink_v, static_cast<long long>(layer) * H * F * d, ea); bytes = H * F * d * ea; break;
+    case LA_TAP_SINK_H:
+      if (!s->cap_sink_valid) return fail(s, LA_ESTATE, "no capture of a sink pass");
+      src = s->cap_sink_h + static_cast<long long>(layer) * F * D;
+      bytes = F * D * 4;
       break;
     default: return fail(s, LA_EINVAL, "bad tap");
   }

@@ -11,7 +11,8 @@ __device__ __forceinline__ void epi_scalar(const GemmEpiParams& ep, long long ro
   const long long off = row * ep.ld + col;
   float* out = reinterpret_cast<float*>(ep.out);
   switch (ep.kind) {
-    case EPI_STORE: out[off] = acc; break;
+    case EPI_STORE:
+    case EPI_STORE32: out[off] = acc; break;
     case EPI_RESID: {
       const float h = ep.h32[off] + acc;
       ep.h32[off] = h;

@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -180,20 +181,32 @@ __device__ __forceinline__ uint64_t sdesc_mnmajor(uint32_t saddr, uint32_t lbo_b
   return sdesc_sw128(saddr, lbo_bytes, 1024);
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+// Instruction descriptor, kind::f16 with fp32 D; A and B share one input type
+// (ab_fmt 0 = fp16, 1 = bf16).
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, bool a_mn_major, bool b_mn_major, uint32_t ab_fmt) {
   return (1u << 4)                                     // D format F32
-         | (1u << 7)                                   // A format BF16
-         | (1u << 10)                                  // B format BF16
+         | (ab_fmt << 7)                               // A format
+         | (ab_fmt << 10)                              // B format (same type as A)
          | ((a_mn_major ? 1u : 0u) << 15)              // A major
          | ((b_mn_major ? 1u : 0u) << 16)              // B major
          | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);      // M / 16
 }
 
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_f16kind(M, N, a_mn_major, b_mn_major, 1u);
+}
+__host__ __device__ constexpr uint32_t idesc_fp16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_f16kind(M, N, a_mn_major, b_mn_major, 0u);
+}
+
 // ---- small helpers ---------------------------------------------------------------
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 __device__ __forceinline__ float fast_exp2(float x) {

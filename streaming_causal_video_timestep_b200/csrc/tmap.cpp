@@ -21,14 +21,14 @@ void resolve() {
   g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
 }
 
-bool encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
-            const cuuint32_t* box, std::string& err) {
+bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+            const cuuint64_t* strides_bytes, const cuuint32_t* box, std::string& err) {
   if (!g_encode) {
     err = g_init_err.empty() ? "tensor-map encoder not initialised" : g_init_err;
     return false;
   }
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+  const CUresult r = g_encode(m, dt, static_cast<cuuint32_t>(rank),
                               const_cast<void*>(base), dims, strides_bytes, box, estr,
                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -54,13 +54,13 @@ bool tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {ld * 2};
   const cuuint32_t box[2] = {64, box_rows};
-  return encode(m, 2, base, dims, strides, box, err);
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, err);
 }
 
-bool tmap_planes_bf16(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint64_t H, uint64_t slices,
-                      std::string& err) {
+bool tmap_planes_f16(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint64_t H, uint64_t slices,
+                     std::string& err) {
   const cuuint64_t dims[4] = {d, rows, H, slices};
   const cuuint64_t strides[3] = {d * 2, rows * d * 2, H * rows * d * 2};
   const cuuint32_t box[4] = {64, 128, 1, 1};
-  return encode(m, 4, base, dims, strides, box, err);
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, base, dims, strides, box, err);
 }

@@ -16,11 +16,18 @@ from ._lib import LaConfig, LaWeights, check, load
 
 
 def _dtype_code(dtype):
+    if dtype in (_lib.LA_FP16, "fp16", torch.float16):
+        return _lib.LA_FP16
     return _lib.LA_BF16 if dtype in (_lib.LA_BF16, "bf16", torch.bfloat16) else _lib.LA_FP32
 
 
 def torch_dtype(code):
     return torch.bfloat16 if code == _lib.LA_BF16 else torch.float32
+
+
+def attn_dtype(code):
+    """Element type of the attention operands (q, K, V) of a stream."""
+    return torch.float16 if code == _lib.LA_BF16 else torch.float32
 
 
 def _ptr(t):
@@ -146,9 +153,13 @@ class LaStream:
             "x_in": ((T, C), torch.float32), "x_out": ((T, C), torch.float32), "v": ((T, C), torch.float32),
             "h": ((T, D), torch.float32), "q": ((H, T, d), dt), "o": ((T, D), dt),
             "ring_k": ((E, H, T, d), dt), "ring_v": ((E, H, T, d), dt), "sink_k": ((H, F, d), dt),
-            "sink_v": ((H, F, d), dt), "sink_k_rope": ((H, F, d), dt),
+            "sink_v": ((H, F, d), dt), "sink_k_rope": ((H, F, d), dt), "sink_h": ((F, D), torch.float32),
         }
         shape, tdt = shapes[what]
+        if what in ("q", "ring_k", "ring_v", "sink_v", "sink_k_rope"):
+            tdt = attn_dtype(self.dtype)
+        elif what in ("o", "sink_k"):
+            tdt = torch.float32
         out = torch.empty(shape, dtype=tdt, device="cuda")
         self._check(self.lib.la_debug_tap(self.h, _lib.TAP[what], layer, slot, _ptr(out),
                                           out.numel() * out.element_size()))
@@ -177,7 +188,7 @@ def op_gemm(A, W, epilogue="store", out=None, h32=None, dt=None, rows_per_group=
     M, K = A.shape
     N = W.shape[0]
     epi = dict(store=_lib.LA_EPI_STORE, resid=_lib.LA_EPI_RESID, set32=_lib.LA_EPI_SET32,
-               euler=_lib.LA_EPI_EULER)[epilogue]
+               euler=_lib.LA_EPI_EULER, store32=_lib.LA_EPI_STORE32)[epilogue]
     dtp = None
     if dt is not None:
         dtp = (c_float * len(dt))(*[float(x) for x in dt])
@@ -186,8 +197,9 @@ def op_gemm(A, W, epilogue="store", out=None, h32=None, dt=None, rows_per_group=
     check(code)
 
 
-def op_attention(q, ks, vs, out, stream=None):
-    """q [H, Tq, d]; ks / vs lists of [H, len, d]; out [Tq, H*d]."""
+def op_attention(q, ks, vs, out, out32=None, stream=None):
+    """q [H, Tq, d] fp16 (tcgen05) or fp32 (SIMT); ks / vs lists of [H, len, d];
+    out [Tq, H*d] bf16 (fp16 inputs) or fp32; out32 optional fp32 copy."""
     lib = load()
     dtype = _dtype_code(q.dtype)
     H, Tq, d = q.shape
@@ -195,7 +207,8 @@ def op_attention(q, ks, vs, out, stream=None):
     kp = (c_void_p * n)(*[k.data_ptr() for k in ks])
     vp = (c_void_p * n)(*[v.data_ptr() for v in vs])
     ln = (c_int64 * n)(*[k.shape[1] for k in ks])
-    code = lib.la_op_attention(dtype, _ptr(q), Tq, H, d, n, kp, vp, ln, _ptr(out), _stream_handle(stream))
+    code = lib.la_op_attention(dtype, _ptr(q), Tq, H, d, n, kp, vp, ln, _ptr(out), _ptr(out32),
+                               _stream_handle(stream))
     check(code)
 
 

@@ -37,12 +37,14 @@ def torch_weights(W, cfg, device="cuda"):
                 w_in=conv(W.w_in), w_head=conv(W.w_head))
 
 
-def make_stream(wl: Workload, W=None, cfg=None):
+def make_stream(wl: Workload, W=None, cfg=None, capture=False):
     import torch
     from streaming_causal_video_timestep_b200 import LaStream
     cfg = cfg or wl.cfg
     W = W if W is not None else make_weights(wl)
     s = LaStream(cfg, torch_weights(W, cfg))
+    if capture:
+        s.capture(True)
     s.set_sink(torch.from_numpy(W.sink).cuda())
     return s, W
 

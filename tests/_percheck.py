@@ -1,0 +1,104 @@
+"""Per-op teacher-forced parity of one captured (block, step) of a stream.
+
+Each kernel of the step is checked against the oracle's definition applied to
+the GPU's own inputs to that kernel (the tolerance is stated for bf16 inputs
+with fp32 accumulation): the in-projection from the captured latent, QKV +
+Rolling RoPE + ring append from the captured residual rounded to the GEMM
+operand type, the sink re-rope from the stored un-roped sink K, attention from
+the captured q and the ring / sink tensors, the output projection from the
+attention output as the next GEMM consumes it, and the head + Euler update.
+`rows` restricts the row-wise checks to a sample of query rows (full-size
+streams); attention keys are always complete.
+"""
+import numpy as np
+
+from oracle import block_causal_attention, euler_step, rope_rotate
+from oracle.rope import block_positions, sink_positions
+from workloads import DTYPE_BF16, bf16_round
+
+from _helpers import assert_close, to_np
+
+
+def _operand(a, cfg):
+    """The value a GEMM consumes: bf16-rounded in bf16 streams, as is in fp32 streams."""
+    a = np.asarray(a, np.float32)
+    return bf16_round(a).astype(np.float64) if cfg.dtype == DTYPE_BF16 else a.astype(np.float64)
+
+
+def check_sink(s, cfg, W, latent, rows=None, tag=""):
+    """Per-op check of the last sink pass: in-projection of the sink latent and,
+    per layer, the stored un-roped K (fp32) and V from the captured sink residual."""
+    dt = cfg.dtype
+    F, D, H, d = cfg.sink_tokens, cfg.hidden, cfg.heads, cfg.head_dim
+    R = np.arange(F) if rows is None else np.asarray(rows)
+    h0 = to_np(s.tap("sink_h", 0))
+    lat = np.asarray(latent, np.float64)
+    want = lat[R] if W.w_in is None else _operand(lat[R], cfg) @ np.asarray(W.w_in, np.float64).T
+    assert_close(h0[R], want, dt, f"{tag} sink in-proj")
+    for l in range(cfg.num_layers):
+        hs = to_np(s.tap("sink_h", l))
+        qkv = _operand(hs[R], cfg) @ np.asarray(W.w_qkv[l], np.float64).T
+        k = qkv[:, D:2 * D].reshape(len(R), H, d)
+        v = qkv[:, 2 * D:].reshape(len(R), H, d)
+        assert_close(to_np(s.tap("sink_k", l)).transpose(1, 0, 2)[R], k, dt, f"{tag} sink K l{l}")
+        assert_close(to_np(s.tap("sink_v", l)).transpose(1, 0, 2)[R], v, dt, f"{tag} sink V l{l}")
+
+
+def check_step(s, cfg, W, b, i, rows=None, tag="", report=None):
+    dt = cfg.dtype
+    T, D, H, d, E, L = cfg.block_tokens, cfg.hidden, cfg.heads, cfg.head_dim, cfg.ring_entries, cfg.num_layers
+    R = np.arange(T) if rows is None else np.asarray(rows)
+    f64 = lambda a: None if a is None else np.asarray(a, np.float64)
+    w_in, w_head = f64(W.w_in), f64(W.w_head)
+    pt, ph, pw = block_positions(cfg, b)
+    st = sink_positions(cfg, (cfg.frames_per_block * b - cfg.sink_offset_frames) if cfg.rolling_rope
+                        else -cfg.sink_offset_frames)
+    errs = {}
+
+    def chk(got, want, what):
+        e = assert_close(got, want, dt, f"{tag} {what} b{b} s{i}")
+        errs[what] = max(errs.get(what, (0, 0)), e)
+
+    x_in = to_np(s.tap("x_in", 0, i)).astype(np.float64)
+    h_in = to_np(s.tap("h", -1, i))
+    want = x_in[R] if w_in is None else _operand(x_in[R], cfg) @ w_in.T
+    chk(h_in[R], want, "in-proj h")
+    h_prev = h_in
+    for l in range(L):
+        wqkv = np.asarray(W.w_qkv[l], np.float64)
+        qkv = _operand(h_prev[R], cfg) @ wqkv.T
+        q = qkv[:, :D].reshape(len(R), H, d)
+        k = qkv[:, D:2 * D].reshape(len(R), H, d)
+        v = qkv[:, 2 * D:].reshape(len(R), H, d)
+        qr = rope_rotate(q, pt[R], ph[R], pw[R], cfg.pairs, cfg.rope_theta)
+        kr = rope_rotate(k, pt[R], ph[R], pw[R], cfg.pairs, cfg.rope_theta)
+        q_gpu = to_np(s.tap("q", l, i)).transpose(1, 0, 2)           # [T, H, d]
+        ring_k = to_np(s.tap("ring_k", l, i)).transpose(0, 2, 1, 3)  # [E, T, H, d]
+        ring_v = to_np(s.tap("ring_v", l, i)).transpose(0, 2, 1, 3)
+        e = b % E
+        chk(q_gpu[R], qr, f"q l{l}")
+        chk(ring_k[e][R], kr, f"ring K l{l}")
+        chk(ring_v[e][R], v, f"ring V l{l}")
+        # sink re-rope for this block from the stored fp32 un-roped sink K
+        sk_raw = to_np(s.tap("sink_k", l)).transpose(1, 0, 2)
+        sk_rope = to_np(s.tap("sink_k_rope", l, i)).transpose(1, 0, 2)
+        chk(sk_rope, rope_rotate(sk_raw, *st, cfg.pairs, cfg.rope_theta), f"sink K rope l{l}")
+        sv = to_np(s.tap("sink_v", l)).transpose(1, 0, 2)
+        # attention from the GPU's own q and cache contents
+        blocks = {bb: (ring_k[bb % E], ring_v[bb % E]) for bb in range(max(0, b - cfg.window_blocks), b + 1)}
+        o_want = block_causal_attention(q_gpu[R], blocks, (sk_rope, sv), qblock=b, window=cfg.window_blocks)
+        o_gpu = to_np(s.tap("o", l, i))
+        chk(o_gpu[R], o_want.reshape(len(R), D), f"attn O l{l}")
+        # output projection + residual from the attention output as the GEMM consumes it
+        h_next = to_np(s.tap("h", l, i))
+        want = h_prev[R].astype(np.float64) + _operand(o_gpu[R], cfg) @ np.asarray(W.w_out[l], np.float64).T
+        chk(h_next[R], want, f"h l{l}")
+        h_prev = h_next
+    vel = h_prev[R].astype(np.float64) if w_head is None else _operand(h_prev[R], cfg) @ w_head.T
+    chk(to_np(s.tap("v", 0, i))[R], vel, "velocity")
+    x_want = euler_step(x_in[R], vel, cfg.timesteps[i], cfg.timesteps[i + 1])
+    chk(to_np(s.tap("x_out", 0, i))[R], x_want, "x")
+    if report is not None:
+        for k_, v_ in errs.items():
+            report[k_] = max(report.get(k_, (0, 0)), v_)
+    return errs

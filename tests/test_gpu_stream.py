@@ -10,6 +10,7 @@ from workloads import (DTYPE_BF16, DTYPE_FP32, SCHED_PIPELINED, SCHED_SEQUENTIAL
                        StreamConfig, Workload, block_noise, make_weights)
 
 from _helpers import assert_close, errors, make_stream, to_np
+from _percheck import check_sink, check_step
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -40,66 +41,41 @@ def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
 
 
-def _check_tick(s, orc, cfg, dtype, ran, tag=""):
-    """Compare every captured intermediate of this tick with the oracle trace."""
-    T, D, H, d = cfg.block_tokens, cfg.hidden, cfg.heads, cfg.head_dim
-    worst = 0.0
-    for (b, i) in ran:
-        tr = orc.trace[(b, i)]
-        assert_close(to_np(s.tap("h", -1, i)), tr["h_in"], dtype, f"{tag} h_in b{b} s{i}")
-        for l in range(cfg.num_layers):
-            lt = tr[("layer", l)]
-            assert_close(to_np(s.tap("q", l, i)), lt["q"].transpose(1, 0, 2), dtype, f"{tag} q b{b} s{i} l{l}")
-            ring_k = to_np(s.tap("ring_k", l, i))[b % cfg.ring_entries]
-            ring_v = to_np(s.tap("ring_v", l, i))[b % cfg.ring_entries]
-            assert_close(ring_k, lt["k"].transpose(1, 0, 2), dtype, f"{tag} ring K b{b} s{i} l{l}")
-            assert_close(ring_v, lt["v"].transpose(1, 0, 2), dtype, f"{tag} ring V b{b} s{i} l{l}")
-            assert_close(to_np(s.tap("sink_k_rope", l, i)), lt["sink_k"].transpose(1, 0, 2), dtype,
-                         f"{tag} sink K rope b{b} s{i} l{l}")
-            _, mean_rel = assert_close(to_np(s.tap("o", l, i)), lt["o"].reshape(T, D), dtype,
-                                       f"{tag} attn O b{b} s{i} l{l}")
-            worst = max(worst, mean_rel)
-            assert_close(to_np(s.tap("h", l, i)), lt["h"], dtype, f"{tag} h b{b} s{i} l{l}")
-        assert_close(to_np(s.tap("v", 0, i)), tr["v"], dtype, f"{tag} v b{b} s{i}")
-        assert_close(to_np(s.tap("x_out", 0, i)), tr["x_out"], dtype, f"{tag} x b{b} s{i}")
-    return worst
-
-
 def _run_teacher_forced(wl, check_every_tick=True):
+    """Per-op parity of every (block, step) (tests/_percheck.py) plus the
+    step-level result: the oracle runs each step in fp64 from the GPU's input
+    latent and the GPU's finished block must match it."""
     cfg = wl.cfg
-    s, W = make_stream(wl)
-    s.capture(True)
-    orc = OracleStream(cfg, W, trace=True)
+    s, W = make_stream(wl, capture=True)
+    check_sink(s, cfg, W, W.sink, tag="reference sink")
+    orc = OracleStream(cfg, W)
     orc.set_sink(W.sink)
     T, C = cfg.block_tokens, cfg.latent_ch
     x_out = torch.empty((T, C), dtype=torch.float32, device="cuda")
     nb = wl.num_blocks
     S = cfg.num_steps
-    finished_gpu = {}
+    per = 8 + 3 * cfg.ring_entries
+    report = {}
     for k in range(nb + S - 1):
         xn = block_noise(wl, k) if k < nb else None
         fin = s.step(_dev(xn) if xn is not None else None, x_out)
         st = s.index_state()
-        per = 8 + 3 * cfg.ring_entries
         ran = [(int(st[4 + i * per]), i) for i in range(S) if st[4 + i * per] >= 0]
+        if check_every_tick or k >= nb + S - 2:
+            for (b, i) in ran:
+                check_step(s, cfg, W, b, i, tag=f"tick {k}", report=report)
         inputs = {(b, i): to_np(s.tap("x_in", 0, i)) for (b, i) in ran}
-        aas = to_np(x_out) if fin == 0 else None
-        out, fin_o = orc.denoise_step(xn, inputs=inputs, aas_latent=aas)
+        got = to_np(x_out).copy() if fin >= 0 else None
+        out, fin_o = orc.denoise_step(xn, inputs=inputs, aas_latent=got if fin == 0 else None)
         assert fin == fin_o
         np.testing.assert_array_equal(st, orc.index_state())
-        if check_every_tick or k >= nb + S - 2:
-            _check_tick(s, orc, cfg, cfg.dtype, ran, tag=f"tick {k}")
         if fin >= 0:
-            finished_gpu[fin] = to_np(x_out).copy()
-            assert_close(finished_gpu[fin], out, cfg.dtype, f"finished block {fin}")
+            assert_close(got, out, cfg.dtype, f"finished block {fin} (step-level)")
+        if fin == 0 and cfg.sink_mode == SINK_AAS:
+            check_sink(s, cfg, W, got[:cfg.sink_tokens], tag="AAS sink")
     s.synchronize()
-    # sink was replaced exactly once (AAS) and the GPU sink K/V match the oracle's
-    if cfg.sink_mode == SINK_AAS:
-        for l in range(cfg.num_layers):
-            assert_close(to_np(s.tap("sink_k", l)), orc.sink_k[l].transpose(1, 0, 2), cfg.dtype, "sink K")
-            assert_close(to_np(s.tap("sink_v", l)), orc.sink_v[l].transpose(1, 0, 2), cfg.dtype, "sink V")
     s.close()
-    return finished_gpu
+    return report
 
 
 def test_tiny_fp32_stream_every_tick_matches_oracle():
