@@ -57,10 +57,9 @@ extern "C" {
 #define LA_SINK_AAS          1  /* sink replaced once by frame 0 of finished block 0  */
 #define LA_SCHED_PIPELINED   0  /* one call = one tick: slot i runs step i of block k-i */
 #define LA_SCHED_SEQUENTIAL  1  /* one call = one block through all steps in order     */
-#define LA_BF16              0  /* bf16 weights/activations, fp32 accumulate, fp32 x;
-                                   attention operands (q, K, V, P) in fp16            */
+#define LA_BF16              0  /* bf16 GEMM operands and attention operands, fp32
+                                   accumulation, fp32 residual stream and latent x    */
 #define LA_FP32              1  /* fp32 everywhere (SIMT path, no TF32)                */
-#define LA_FP16              2  /* op-level attention only: fp16 q/K/V, tcgen05        */
 
 /* Limits of this build. */
 #define LA_MAX_STEPS     8
@@ -189,8 +188,9 @@ int la_debug_capture(la_stream* s, int32_t enable);
 #define LA_TAP_X_IN      0  /* fp32 [T_b, C]   latent the slot's last step started from        */
 #define LA_TAP_X_OUT     1  /* fp32 [T_b, C]   latent after the slot's last step               */
 #define LA_TAP_H         2  /* fp32 [T_b, D]   residual after layer `layer` (-1: after in-proj) */
-/* "attn" = the attention operand type: fp16 for LA_BF16 streams, fp32 for LA_FP32. */
-#define LA_TAP_Q         3  /* attn [H, T_b, d] roped queries of layer                           */
+/* "attn" = the attention operand type: bf16 for LA_BF16 streams, fp32 for LA_FP32. */
+#define LA_TAP_Q         3  /* attn [H, T_b, d] roped queries of layer; LA_BF16 streams store
+                               them pre-multiplied by the softmax scale log2(e)/sqrt(d)         */
 #define LA_TAP_O         4  /* fp32 [T_b, D]   attention output of layer, before rounding        */
 #define LA_TAP_V         5  /* fp32 [T_b, C]    velocity of the slot's last step                 */
 #define LA_TAP_RING_K    6  /* attn [E, H, T_b, d] ring K of (layer, slot), by entry             */
@@ -260,7 +260,7 @@ int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, vo
  * expressed by which segments are passed).  q: DEVICE [H, Tq, d]; segment s:
  * k_seg[s], v_seg[s] DEVICE [H, seg_len[s], d] (HOST arrays of nseg pointers /
  * lengths, 1 <= nseg <= LA_MAX_WINDOW + 2, seg_len >= 1).
- * dtype LA_FP16: q/K/V fp16, d == 128, tcgen05; out DEVICE bf16 [Tq, H*d] and,
+ * dtype LA_BF16: q/K/V bf16, d == 128, tcgen05; out DEVICE bf16 [Tq, H*d] and,
  *   if out32 != NULL, an fp32 copy [Tq, H*d] (the value before rounding).
  * dtype LA_FP32: q/K/V/out fp32, d % 8 == 0, d <= 128, SIMT; out32 ignored.
  */

@@ -11,7 +11,7 @@ LIB_PATH = os.path.join(_HERE, "libla.so")
 LA_OK, LA_EINVAL, LA_ESTATE, LA_ENOMEM, LA_ECUDA, LA_EDEVICE = 0, -1, -2, -3, -4, -5
 LA_SINK_FIXED, LA_SINK_AAS = 0, 1
 LA_SCHED_PIPELINED, LA_SCHED_SEQUENTIAL = 0, 1
-LA_BF16, LA_FP32, LA_FP16 = 0, 1, 2
+LA_BF16, LA_FP32 = 0, 1
 LA_MAX_STEPS, LA_MAX_WINDOW, LA_MAX_FPB = 8, 14, 7
 LA_EPI_STORE, LA_EPI_RESID, LA_EPI_SET32, LA_EPI_EULER, LA_EPI_STORE32 = 0, 1, 2, 3, 4
 

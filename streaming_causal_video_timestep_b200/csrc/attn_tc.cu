@@ -1,4 +1,4 @@
-// Block-causal attention on tcgen05 tensor cores, head_dim 128: fp16 q/K/V/P
+// Block-causal attention on tcgen05 tensor cores, head_dim 128: bf16 q/K/V/P
 // operands, fp32 scores, softmax and accumulation, bf16 output.
 //
 // One CTA = 128 queries of one (group, head); the keys are the group's list of
@@ -14,11 +14,13 @@
 //   warps 2..5  softmax: thread = query row = TMEM lane.  tcgen05.ld of the S
 //               row, masked row max, exp2, row sum, lazy rescale of O in TMEM
 //               (only when the running max grows by more than 2^8), P written
-//               to shared memory as fp16 in the swizzled K-major layout, then
+//               to shared memory as bf16 in the swizzled K-major layout, then
 //               the final 1/l normalisation and bf16 store (plus an optional
 //               fp32 copy).
-// fp16 rather than bf16 for q, K, V and P: same bytes and tensor-core rate,
-// 3 more mantissa bits; P <= 2^8 by construction and q/K/V saturate at 65504.
+// Scores are formed in the log2 domain: with q pre-multiplied by log2(e)/sqrt(d)
+// (PRESCALED, the stream's QKV epilogue does it) p = 2^(s - max s); otherwise the
+// scaled score x = s * scale is rounded first.  Either way the row maximum gives
+// exactly 2^0 = 1, so the row sum is >= 1 whatever the magnitude of the logits.
 // S_{t+1} is computed on the tensor cores while the softmax warps work on S_t.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -48,6 +50,7 @@ __device__ __forceinline__ int group_tiles(const AttnGroup& g) {
   return n;
 }
 
+template <bool PRESCALED>
 __global__ void __launch_bounds__(192, 1)
 k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -132,8 +135,8 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_fp16(BQ, BKV, false, false);
-      constexpr uint32_t idPV = idesc_fp16(BQ, 128, false, true);
+      constexpr uint32_t idS = idesc_bf16(BQ, BKV, false, false);
+      constexpr uint32_t idPV = idesc_bf16(BQ, 128, false, true);
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t p_addr = smem_u32(sP);
       bool ok = mbar_wait(q_full, 0, err);
@@ -210,25 +213,49 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
 
-      float mx = -INFINITY;
+      // scores in the log2 domain (rounded once), row max and sum with 8
+      // independent partial accumulators (one warp per scheduler: latency is
+      // hidden by ILP, not by other warps)
+      float x[128];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float v = c < valid ? __uint_as_float(s[c]) : -INFINITY;
-        mx = fmaxf(mx, v);
+      for (int c = 0; c < 128; ++c) x[c] = PRESCALED ? __uint_as_float(s[c]) : __uint_as_float(s[c]) * sc;
+      float mx8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+      if (valid == BKV) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], c < valid ? x[c] : -INFINITY);
       }
-      const float m_tile = mx * sc;
+      const float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const bool need = m_tile > m_ref + 8.0f;
       const float m_new = need ? m_tile : m_ref;
       const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
-      float rs = 0.f;
-      uint32_t pk[64];
+      float rs8[8];
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = c < valid ? fast_exp2(fmaf(__uint_as_float(s[c]), sc, -m_new)) : 0.f;
-        const float p1 = c + 1 < valid ? fast_exp2(fmaf(__uint_as_float(s[c + 1]), sc, -m_new)) : 0.f;
-        rs += p0 + p1;
-        pk[c / 2] = pack_f16x2(p0, p1);
+      for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
+      uint32_t pk[64];
+      if (valid == BKV) {
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float p0 = fast_exp2(x[c] - m_new);
+          const float p1 = fast_exp2(x[c + 1] - m_new);
+          rs8[(c >> 1) & 7] += p0 + p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float p0 = c < valid ? fast_exp2(x[c] - m_new) : 0.f;
+          const float p1 = c + 1 < valid ? fast_exp2(x[c + 1] - m_new) : 0.f;
+          rs8[(c >> 1) & 7] += p0 + p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
       }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l = l * alpha + rs;
       m_ref = m_new;
 
@@ -311,9 +338,10 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
 }  // namespace
 
 cudaError_t launch_attn_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM));
+  auto kern = p.q_prescaled ? k_attn_tc<true> : k_attn_tc<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
   dim3 grid((p.Tq + BQ - 1) / BQ, p.H, p.ngroups);
-  k_attn_tc<<<grid, 192, SMEM, st>>>(maps, p);
+  kern<<<grid, 192, SMEM, st>>>(maps, p);
   return cudaGetLastError();
 }

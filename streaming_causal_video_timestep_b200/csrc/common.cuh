@@ -55,6 +55,7 @@ struct AttnParams {
   int Tq;               // queries per group
   int H, d;
   float scale_log2;     // log2(e) / sqrt(d)
+  int q_prescaled;      // q already multiplied by scale_log2 (tcgen05 path)
   void* out;            // [rows, H*d] bf16 (tcgen05 path) / fp32 (SIMT path)
   float* out32;         // optional fp32 copy of the output (tcgen05 path)
   long long out_ld;     // elements per output row
@@ -71,11 +72,12 @@ struct AttnParams {
 enum GemmEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SET32 = 2, EPI_EULER = 3, EPI_STORE32 = 4, EPI_QKV_ROPE = 5 };
 
 // QKV projection epilogue: rotate q and k (Rolling 3D RoPE) on the fp32
-// accumulators and append K/V to the ring, rounding once to the attention
-// operand type (fp16).  Rows of inactive buffers are not written.
+// accumulators, pre-multiply q by the softmax scale log2(e)/sqrt(d), and append
+// K/V to the ring, rounding once to bf16.  Rows of inactive buffers are not written.
 struct QkvRopeParams {
   int T, F, H, d, D, E, grid_w;
   int pt, ph;
+  float qscale;              // log2(e)/sqrt(d)
   int active[LA_MAX_STEPS];
   int slot[LA_MAX_STEPS];
   int write_entry[LA_MAX_STEPS];
@@ -98,7 +100,5 @@ struct GemmEpiParams {
   float* vtap;          // optional fp32 [M, N] copy of acc (velocity capture)
 };
 
-// Largest finite fp16 magnitude; attention operands saturate there.
-#define LA_F16_MAX 65504.0f
 
 static inline int ceil_div_i(long long a, long long b) { return (int)((a + b - 1) / b); }

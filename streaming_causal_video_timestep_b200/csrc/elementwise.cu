@@ -28,19 +28,6 @@ template <> struct Vec8<__nv_bfloat16> {
     *reinterpret_cast<uint4*>(p) = w;
   }
 };
-template <> struct Vec8<__half> {
-  static __device__ __forceinline__ void store(__half* p, const float (&v)[8]) {
-    float c[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) c[i] = fminf(fmaxf(v[i], -LA_F16_MAX), LA_F16_MAX);
-    uint4 w;
-    w.x = pack_f16x2(c[0], c[1]);
-    w.y = pack_f16x2(c[2], c[3]);
-    w.z = pack_f16x2(c[4], c[5]);
-    w.w = pack_f16x2(c[6], c[7]);
-    *reinterpret_cast<uint4*>(p) = w;
-  }
-};
 template <> struct Vec8<float> {
   static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
     const float4 a = reinterpret_cast<const float4*>(p)[0];
@@ -152,8 +139,8 @@ __global__ void __launch_bounds__(256) k_rope_append(const __grid_constant__ Pas
 // (fp32, kept for re-roping), V (TO), and roped q / k (TO) for the sink's
 // self-attention (temporal row 0 of buffer 0 of the table).
 template <typename TO>
-__global__ void __launch_bounds__(256) k_sink_qkv(const __grid_constant__ RopeArgs a, float* sink_k_raw, TO* sink_v,
-                                                  TO* q_rope, TO* k_rope) {
+__global__ void __launch_bounds__(256) k_sink_qkv(const __grid_constant__ RopeArgs a, float qscale, float* sink_k_raw,
+                                                  TO* sink_v, TO* q_rope, TO* k_rope) {
   const int chunks = a.d / 8;
   const long long total = static_cast<long long>(a.F) * 3 * a.H * chunks;
   const float* qkv = reinterpret_cast<const float*>(a.qkv);
@@ -173,6 +160,10 @@ __global__ void __launch_bounds__(256) k_sink_qkv(const __grid_constant__ RopeAr
     }
     if (part == 1) Vec8<float>::store(sink_k_raw + off, v);
     rotate8(v, ch, 0, 0, m / a.grid_w, m % a.grid_w, a);
+    if (part == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] *= qscale;
+    }
     Vec8<TO>::store(part == 0 ? q_rope + off : k_rope + off, v);
   }
 }
@@ -240,30 +231,31 @@ cudaError_t launch_rope_ttab(const PassDesc& pd, int fpb, int pt, const double* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_rope_append(int f16_out, const PassDesc& pd, const RopeArgs& a, bool main_part,
+cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs& a, bool main_part,
                                cudaStream_t st) {
   const long long chunks = a.d / 8;
   const long long n_main = main_part ? static_cast<long long>(pd.nactive) * a.T * 3 * a.H * chunks : 0;
   const long long n_sink = a.sink_k ? static_cast<long long>(pd.nactive) * a.F * a.H * chunks : 0;
   if (n_main + n_sink == 0) return cudaSuccess;
   const int grid = grid_for(n_main + n_sink);
-  if (f16_out)
-    k_rope_append<__half><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
+  if (bf16_out)
+    k_rope_append<__nv_bfloat16><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
   else
     k_rope_append<float><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
   return cudaGetLastError();
 }
 
-cudaError_t launch_sink_qkv(int f16_out, const RopeArgs& a, float* sink_k_raw, void* sink_v, void* q_rope,
-                            void* k_rope, cudaStream_t st) {
+cudaError_t launch_sink_qkv(int bf16_out, const RopeArgs& a, float qscale, float* sink_k_raw, void* sink_v,
+                            void* q_rope, void* k_rope, cudaStream_t st) {
   const long long n = static_cast<long long>(a.F) * 3 * a.H * (a.d / 8);
   const int grid = grid_for(n);
-  if (f16_out)
-    k_sink_qkv<__half><<<grid, 256, 0, st>>>(a, sink_k_raw, static_cast<__half*>(sink_v),
-                                              static_cast<__half*>(q_rope), static_cast<__half*>(k_rope));
+  if (bf16_out)
+    k_sink_qkv<__nv_bfloat16><<<grid, 256, 0, st>>>(a, qscale, sink_k_raw, static_cast<__nv_bfloat16*>(sink_v),
+                                                     static_cast<__nv_bfloat16*>(q_rope),
+                                                     static_cast<__nv_bfloat16*>(k_rope));
   else
-    k_sink_qkv<float><<<grid, 256, 0, st>>>(a, sink_k_raw, static_cast<float*>(sink_v), static_cast<float*>(q_rope),
-                                            static_cast<float*>(k_rope));
+    k_sink_qkv<float><<<grid, 256, 0, st>>>(a, qscale, sink_k_raw, static_cast<float*>(sink_v),
+                                            static_cast<float*>(q_rope), static_cast<float*>(k_rope));
   return cudaGetLastError();
 }
 

@@ -54,15 +54,9 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
   }
 }
 
-__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
-  lo = fminf(fmaxf(lo, -LA_F16_MAX), LA_F16_MAX);
-  hi = fminf(fmaxf(hi, -LA_F16_MAX), LA_F16_MAX);
-  __half2 v = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
 // 32 consecutive columns of one head of the [q | k | v] projection of one token:
-// rotate the pairs of q and k, then write fp16 to q_rope / the ring entry.
+// rotate the pairs of q and k, scale q by log2(e)/sqrt(d), then write bf16 to
+// q_rope / the ring entry.
 __device__ __forceinline__ void qkv_rope_row32(const QkvRopeParams& qp, long long row, long long col,
                                                float (&acc)[32]) {
   const int buf = static_cast<int>(row / qp.T);
@@ -95,24 +89,18 @@ __device__ __forceinline__ void qkv_rope_row32(const QkvRopeParams& qp, long lon
       acc[2 * jj + 1] = x0 * sn + x1 * c;
     }
   }
-  __half* dst;
+  __nv_bfloat16* dst;
   const long long tok = static_cast<long long>(n) * qp.d + e0;
   if (part == 0) {
-    dst = reinterpret_cast<__half*>(qp.q_rope) + (static_cast<long long>(buf) * qp.H + h) * qp.T * qp.d + tok;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] *= qp.qscale;
+    dst = reinterpret_cast<__nv_bfloat16*>(qp.q_rope) + (static_cast<long long>(buf) * qp.H + h) * qp.T * qp.d + tok;
   } else {
     const long long slice = qp.ring_slice0 + static_cast<long long>(qp.slot[buf]) * qp.E + qp.write_entry[buf];
-    dst = reinterpret_cast<__half*>(part == 1 ? qp.ring_k : qp.ring_v) + (slice * qp.H + h) * qp.T * qp.d + tok;
+    dst = reinterpret_cast<__nv_bfloat16*>(part == 1 ? qp.ring_k : qp.ring_v) + (slice * qp.H + h) * qp.T * qp.d +
+          tok;
   }
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 w;
-    w.x = pack_f16x2_sat(acc[8 * i + 0], acc[8 * i + 1]);
-    w.y = pack_f16x2_sat(acc[8 * i + 2], acc[8 * i + 3]);
-    w.z = pack_f16x2_sat(acc[8 * i + 4], acc[8 * i + 5]);
-    w.w = pack_f16x2_sat(acc[8 * i + 6], acc[8 * i + 7]);
-    d4[i] = w;
-  }
+  store_bf16x32(dst, acc);
 }
 
 __device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, const QkvRopeParams& qp, long long row,

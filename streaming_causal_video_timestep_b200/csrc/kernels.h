@@ -13,13 +13,16 @@ cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const
                            int K, int bn, int* err, int num_sms, cudaStream_t st, const QkvRopeParams* qp = nullptr);
 
 // Tensor maps of an attention launch: q (d, Tq, H, q slices) and k[m]/v[m]
-// (d, rows_m, H, slices), fp16, 128-byte swizzle, box (64, 128, 1, 1).
+// (d, rows_m, H, slices), bf16, 128-byte swizzle, box (64, 128, 1, 1).
 struct AttnMaps {
   CUtensorMap q;
   CUtensorMap k[LA_MAX_SEG];
   CUtensorMap v[LA_MAX_SEG];
 };
-cudaError_t launch_attn_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);
+cudaError_t launch_attn_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);    // 1 query tile / CTA
+cudaError_t launch_attn_tc2(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);   // 2 query tiles / CTA
+// The attention launcher used by the library (LA_ATTN_V1=1 in the environment selects the one-tile kernel).
+cudaError_t launch_attention_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);
 
 // ---- SIMT fp32 -----------------------------------------------------------------------
 cudaError_t launch_gemm_f32(const float* A, const float* W, const GemmEpiParams& ep, int M, int N, int K,
@@ -46,15 +49,16 @@ struct RopeArgs {
   const void* sink_k;                          // fp32 un-roped [H][F][d] of this layer (NULL: no sink part)
   void* sink_k_rope;                           // [nbuf][H][F][d]
 };
-// Outputs are fp16 (f16_out) or fp32.  main_part: also rope/append the block
+// Outputs are bf16 (bf16_out) or fp32.  main_part: also rope/append the block
 // from qkv (fp32 streams; bf16 streams do that in the QKV GEMM epilogue).
-cudaError_t launch_rope_append(int f16_out, const PassDesc& pd, const RopeArgs& a, bool main_part,
+cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs& a, bool main_part,
                                cudaStream_t st);
 
 // Sink pass: split the fp32 qkv [F, 3D] into the layer's fp32 un-roped K, its
-// V, and roped q / k (temporal row 0 of buffer 0 of the table).
-cudaError_t launch_sink_qkv(int f16_out, const RopeArgs& a, float* sink_k_raw, void* sink_v, void* q_rope,
-                            void* k_rope, cudaStream_t st);
+// V, and roped q / k (temporal row 0 of buffer 0 of the table); q is
+// multiplied by qscale (the softmax scale on the bf16 path, 1 on fp32).
+cudaError_t launch_sink_qkv(int bf16_out, const RopeArgs& a, float qscale, float* sink_k_raw, void* sink_v,
+                            void* q_rope, void* k_rope, cudaStream_t st);
 
 // x (fp32 [rows, C]) -> h32 (fp32) and hop (dtype) when C == D (identity in-proj),
 // or -> xop (bf16) for the in-projection GEMM.

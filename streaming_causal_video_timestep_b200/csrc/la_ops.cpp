@@ -70,7 +70,8 @@ int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t
   p.d = d;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   p.out = out;
-  p.out32 = dtype == LA_FP16 ? out32 : nullptr;
+  p.out32 = dtype == LA_BF16 ? out32 : nullptr;
+  p.q_prescaled = 0;
   p.out_ld = static_cast<long long>(H) * d;
   p.err = nullptr;
   p.qbase = q;
@@ -86,17 +87,17 @@ int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t
     p.vrows[s] = static_cast<int>(seg_len[s]);
   }
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  if (dtype == LA_FP16) {
+  if (dtype == LA_BF16) {
     if (d != 128) return LA_EINVAL;
     std::string err;
     if (!tmap_init(err)) return LA_ECUDA;
     AttnMaps maps;
-    if (!tmap_planes_f16(&maps.q, q, d, Tq, H, 1, err)) return LA_ECUDA;
+    if (!tmap_planes_bf16(&maps.q, q, d, Tq, H, 1, err)) return LA_ECUDA;
     for (int s = 0; s < nseg; ++s) {
-      if (!tmap_planes_f16(&maps.k[s], k_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
-      if (!tmap_planes_f16(&maps.v[s], v_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
+      if (!tmap_planes_bf16(&maps.k[s], k_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
+      if (!tmap_planes_bf16(&maps.v[s], v_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
     }
-    return ret(launch_attn_tc(maps, p, st));
+    return ret(launch_attention_tc(maps, p, st));
   }
   if (dtype != LA_FP32) return LA_EINVAL;
   return ret(launch_attn_f32(p, st));

@@ -142,7 +142,7 @@ struct la_stream {
   int pt = 0, ph = 0, pw = 0;
   bool bf16 = true, id_in = true, id_head = true;
   size_t es = 2;            // activation / weight element (bf16 or fp32)
-  size_t ea = 2;            // attention operand element (fp16 or fp32)
+  size_t ea = 2;            // attention operand element (bf16 or fp32)
   int device = 0, num_sms = 148;
   cudaStream_t st = nullptr;
 
@@ -423,6 +423,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
   QkvRopeParams qp{};
   qp.T = T; qp.F = F; qp.H = H; qp.d = d; qp.D = D; qp.E = E; qp.grid_w = s->cfg.grid_w;
   qp.pt = s->pt; qp.ph = s->ph;
+  qp.qscale = ap.scale_log2;
   for (int i = 0; i < LA_MAX_STEPS; ++i) {
     qp.active[i] = pd.active[i];
     qp.slot[i] = pd.slot[i];
@@ -431,6 +432,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
   qp.tcos = s->tcos; qp.tsin = s->tsin; qp.rcos = s->rcos; qp.rsin = s->rsin; qp.ccos = s->ccos; qp.csin = s->csin;
   qp.q_rope = s->q_rope; qp.ring_k = s->ring_k; qp.ring_v = s->ring_v;
   ap.out32 = (s->bf16 && s->capture) ? s->cap_oall : nullptr;
+  ap.q_prescaled = s->bf16 ? 1 : 0;
 
   for (int l = 0; l < s->L; ++l) {
     ra.qkv = s->qkv; ra.q_rope = s->q_rope; ra.ring_k = s->ring_k; ra.ring_v = s->ring_v;
@@ -447,7 +449,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
                                    &qp);
            })) != LA_OK)
         return r;
-      // per-block re-rope of the sink K (fp32 -> fp16, once per active buffer)
+      // per-block re-rope of the sink K (fp32 -> bf16, once per active buffer)
       if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(1, pd, ra, false, s->st); })) != LA_OK)
         return r;
     } else {
@@ -475,7 +477,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
       g.nseg = ns;
     }
     if (s->bf16) {
-      if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_tc(s->maps_stream, ap, s->st); })) != LA_OK) return r;
+      if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attention_tc(s->maps_stream, ap, s->st); })) != LA_OK) return r;
     } else {
       if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) return r;
     }
@@ -552,6 +554,7 @@ int run_sink(la_stream* s) {
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   ap.out = s->s_o; ap.out_ld = D; ap.err = s->dev_err;
   ap.qbase = s->s_q;
+  ap.q_prescaled = s->bf16 ? 1 : 0;
   ap.kbase[0] = s->s_k; ap.krows[0] = F;
   ap.vbase[0] = s->sink_v; ap.vrows[0] = F;
   ap.ngroups = 1;
@@ -569,7 +572,7 @@ int run_sink(la_stream* s) {
     float* kraw = s->sink_k + static_cast<long long>(l) * H * F * d;
     void* vraw = elem(s->sink_v, static_cast<long long>(l) * H * F * d, s->ea);
     if ((r = launch(s, LA_KIND_ROPE, [&] {
-           return launch_sink_qkv(s->bf16, ra, kraw, vraw, s->s_q, s->s_k, s->st);
+           return launch_sink_qkv(s->bf16, ra, s->bf16 ? ap.scale_log2 : 1.0f, kraw, vraw, s->s_q, s->s_k, s->st);
          })) != LA_OK)
       return r;
     if (l == s->L - 1) break;   // the last layer's sink output feeds nothing
@@ -579,7 +582,7 @@ int run_sink(la_stream* s) {
     g.nseg = 1;
     g.seg[0] = AttnSeg{0, 0, 0, l, F};
     if (s->bf16) {
-      if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_tc(s->maps_sink, ap, s->st); })) != LA_OK) return r;
+      if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attention_tc(s->maps_sink, ap, s->st); })) != LA_OK) return r;
     } else {
       if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) return r;
     }
@@ -840,14 +843,14 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
       ok = ok && tmap_2d_bf16(&s->tm_win, s->w_in, D, C, C, bn_d, s->err);
       ok = ok && tmap_2d_bf16(&s->tm_whead, s->w_head, C, D, D, bn_c, s->err);
     }
-    ok = ok && tmap_planes_f16(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
-    ok = ok && tmap_planes_f16(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
-    ok = ok && tmap_planes_f16(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
-    ok = ok && tmap_planes_f16(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
-    ok = ok && tmap_planes_f16(&s->maps_stream.v[1], s->sink_v, d, F, H, L, s->err);
-    ok = ok && tmap_planes_f16(&s->maps_sink.q, s->s_q, d, F, H, 1, s->err);
-    ok = ok && tmap_planes_f16(&s->maps_sink.k[0], s->s_k, d, F, H, 1, s->err);
-    ok = ok && tmap_planes_f16(&s->maps_sink.v[0], s->sink_v, d, F, H, L, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_stream.v[1], s->sink_v, d, F, H, L, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_sink.q, s->s_q, d, F, H, 1, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_sink.k[0], s->s_k, d, F, H, 1, s->err);
+    ok = ok && tmap_planes_bf16(&s->maps_sink.v[0], s->sink_v, d, F, H, L, s->err);
     if (!ok) return bail(LA_ECUDA);
   }
   e = cudaStreamSynchronize(s->st);

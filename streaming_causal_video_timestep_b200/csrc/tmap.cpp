@@ -57,10 +57,10 @@ bool tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, err);
 }
 
-bool tmap_planes_f16(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint64_t H, uint64_t slices,
+bool tmap_planes_bf16(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint64_t H, uint64_t slices,
                      std::string& err) {
   const cuuint64_t dims[4] = {d, rows, H, slices};
   const cuuint64_t strides[3] = {d * 2, rows * d * 2, H * rows * d * 2};
   const cuuint32_t box[4] = {64, 128, 1, 1};
-  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, base, dims, strides, box, err);
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, err);
 }

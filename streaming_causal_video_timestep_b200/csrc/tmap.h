@@ -14,7 +14,7 @@ bool tmap_init(std::string& err);
 bool tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows,
                   std::string& err);
 
-// fp16 stack of [H, rows, d] planes: dims (d, rows, H, slices), dense; box
+// bf16 stack of [H, rows, d] planes: dims (d, rows, H, slices), dense; box
 // (64, 128, 1, 1), 128-byte swizzle; rows beyond `rows` read as zero.
-bool tmap_planes_f16(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint64_t H, uint64_t slices,
+bool tmap_planes_bf16(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint64_t H, uint64_t slices,
                      std::string& err);

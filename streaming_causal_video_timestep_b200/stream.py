@@ -16,8 +16,6 @@ from ._lib import LaConfig, LaWeights, check, load
 
 
 def _dtype_code(dtype):
-    if dtype in (_lib.LA_FP16, "fp16", torch.float16):
-        return _lib.LA_FP16
     return _lib.LA_BF16 if dtype in (_lib.LA_BF16, "bf16", torch.bfloat16) else _lib.LA_FP32
 
 
@@ -27,7 +25,7 @@ def torch_dtype(code):
 
 def attn_dtype(code):
     """Element type of the attention operands (q, K, V) of a stream."""
-    return torch.float16 if code == _lib.LA_BF16 else torch.float32
+    return torch.bfloat16 if code == _lib.LA_BF16 else torch.float32
 
 
 def _ptr(t):
@@ -198,8 +196,8 @@ def op_gemm(A, W, epilogue="store", out=None, h32=None, dt=None, rows_per_group=
 
 
 def op_attention(q, ks, vs, out, out32=None, stream=None):
-    """q [H, Tq, d] fp16 (tcgen05) or fp32 (SIMT); ks / vs lists of [H, len, d];
-    out [Tq, H*d] bf16 (fp16 inputs) or fp32; out32 optional fp32 copy."""
+    """q [H, Tq, d] bf16 (tcgen05) or fp32 (SIMT), unscaled; ks / vs lists of
+    [H, len, d]; out [Tq, H*d] in the input type; out32 optional fp32 copy."""
     lib = load()
     dtype = _dtype_code(q.dtype)
     H, Tq, d = q.shape

@@ -12,6 +12,8 @@ streams); attention keys are always complete.
 """
 import numpy as np
 
+import math
+
 from oracle import block_causal_attention, euler_step, rope_rotate
 from oracle.rope import block_positions, sink_positions
 from workloads import DTYPE_BF16, bf16_round
@@ -44,7 +46,16 @@ def check_sink(s, cfg, W, latent, rows=None, tag=""):
         assert_close(to_np(s.tap("sink_v", l)).transpose(1, 0, 2)[R], v, dt, f"{tag} sink V l{l}")
 
 
-def check_step(s, cfg, W, b, i, rows=None, tag="", report=None):
+def sink_snapshot(s, cfg):
+    """The sink K (un-roped) and V of every layer as they are now: take it before
+    a call whose per-op check follows (the AAS replacement at the end of the
+    call that finishes block 0 changes them)."""
+    return ([to_np(s.tap("sink_k", l)).transpose(1, 0, 2) for l in range(cfg.num_layers)],
+            [to_np(s.tap("sink_v", l)).transpose(1, 0, 2) for l in range(cfg.num_layers)])
+
+
+def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
+    """sink: sink_snapshot() taken before the call (default: the current sink)."""
     dt = cfg.dtype
     T, D, H, d, E, L = cfg.block_tokens, cfg.hidden, cfg.heads, cfg.head_dim, cfg.ring_entries, cfg.num_layers
     R = np.arange(T) if rows is None else np.asarray(rows)
@@ -73,6 +84,13 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None):
         qr = rope_rotate(q, pt[R], ph[R], pw[R], cfg.pairs, cfg.rope_theta)
         kr = rope_rotate(k, pt[R], ph[R], pw[R], cfg.pairs, cfg.rope_theta)
         q_gpu = to_np(s.tap("q", l, i)).transpose(1, 0, 2)           # [T, H, d]
+        if dt == DTYPE_BF16:
+            # bf16 streams store q pre-multiplied by the softmax scale log2(e)/sqrt(d)
+            qscale = float(np.float32(math.log2(math.e) / math.sqrt(d)))
+            qr = qr * qscale
+            q_att = q_gpu / qscale
+        else:
+            q_att = q_gpu
         ring_k = to_np(s.tap("ring_k", l, i)).transpose(0, 2, 1, 3)  # [E, T, H, d]
         ring_v = to_np(s.tap("ring_v", l, i)).transpose(0, 2, 1, 3)
         e = b % E
@@ -80,13 +98,13 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None):
         chk(ring_k[e][R], kr, f"ring K l{l}")
         chk(ring_v[e][R], v, f"ring V l{l}")
         # sink re-rope for this block from the stored fp32 un-roped sink K
-        sk_raw = to_np(s.tap("sink_k", l)).transpose(1, 0, 2)
+        sk_raw = sink[0][l] if sink is not None else to_np(s.tap("sink_k", l)).transpose(1, 0, 2)
         sk_rope = to_np(s.tap("sink_k_rope", l, i)).transpose(1, 0, 2)
         chk(sk_rope, rope_rotate(sk_raw, *st, cfg.pairs, cfg.rope_theta), f"sink K rope l{l}")
-        sv = to_np(s.tap("sink_v", l)).transpose(1, 0, 2)
+        sv = sink[1][l] if sink is not None else to_np(s.tap("sink_v", l)).transpose(1, 0, 2)
         # attention from the GPU's own q and cache contents
         blocks = {bb: (ring_k[bb % E], ring_v[bb % E]) for bb in range(max(0, b - cfg.window_blocks), b + 1)}
-        o_want = block_causal_attention(q_gpu[R], blocks, (sk_rope, sv), qblock=b, window=cfg.window_blocks)
+        o_want = block_causal_attention(q_att[R], blocks, (sk_rope, sv), qblock=b, window=cfg.window_blocks)
         o_gpu = to_np(s.tap("o", l, i))
         chk(o_gpu[R], o_want.reshape(len(R), D), f"attn O l{l}")
         # output projection + residual from the attention output as the GEMM consumes it

@@ -1,0 +1,183 @@
+"""Parity at the full 14B-like shapes, in the launch configuration bench.py
+times (4 slots per grouped launch): every kernel checked per op on sampled
+query rows (the first and last query tiles, the ragged tail and a spread in
+between; attention always over all keys), integer state bit-exact every tick."""
+import numpy as np
+import pytest
+
+from oracle import TickScheduler
+from workloads import (SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_FIXED, SOAK, STREAM, SUBLAYER, Workload,
+                       block_noise, make_weights, step_input, sweep_point)
+
+from _helpers import make_stream, to_np
+from _percheck import check_sink, check_step, sink_snapshot
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from streaming_causal_video_timestep_b200 import build
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+
+
+def sample_rows(T, n=48, seed=0):
+    rng = np.random.default_rng(seed)
+    edge = [0, 1, 127, 128, T - 129, T - 73, T - 72, T - 2, T - 1]
+    mid = rng.choice(np.arange(129, T - 129), size=n - len(edge), replace=False)
+    return np.unique(np.concatenate([edge, mid]))
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+
+def _active(s, cfg):
+    st = s.index_state()
+    per = 8 + 3 * cfg.ring_entries
+    return [(int(st[4 + i * per]), i) for i in range(cfg.num_steps) if st[4 + i * per] >= 0]
+
+
+def test_sublayer_at_14b_shape_one_slot():
+    """One attention sublayer, hidden 5120, 40 x 128, 30x52 grid, window 2, t = 0.5:
+    blocks 0 and 1 fill the window, block 2 is checked in steady state."""
+    wl = SUBLAYER
+    cfg = wl.cfg
+    s, W = make_stream(wl, capture=True)
+    R = sample_rows(cfg.block_tokens)
+    check_sink(s, cfg, W, W.sink, rows=R[R < cfg.sink_tokens], tag="sink")
+    x_out = torch.empty((cfg.block_tokens, cfg.latent_ch), device="cuda")
+    ref = TickScheduler(cfg)
+    for b in range(wl.num_blocks):
+        fin = s.step(_dev(block_noise(wl, b)), x_out)
+        run, fin_o = ref.begin_tick(True)
+        for i, bb in run:
+            ref.append(i, bb)
+        ref.end_tick(fin_o)
+        assert fin == fin_o == b
+        np.testing.assert_array_equal(s.index_state(), ref.index_state())
+        if b == wl.num_blocks - 1:
+            errs = check_step(s, cfg, W, b, 0, rows=R, tag="sublayer")
+            print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in errs.items()})
+    s.synchronize()
+    s.close()
+
+
+def test_eight_layer_stream_four_slots_grouped():
+    """The benchmarked workload: 4 slots x 8 sublayers per grouped launch, head
+    5120 -> 64, AAS.  Per-op checks at the AAS tick, in steady state and in the drain."""
+    wl = Workload(STREAM.name, STREAM.cfg, STREAM.seed, 8, STREAM.w_std, STREAM.head_std)
+    cfg = wl.cfg
+    s, W = make_stream(wl, capture=True)
+    R = sample_rows(cfg.block_tokens, n=24)
+    check_sink(s, cfg, W, W.sink, rows=R[R < cfg.sink_tokens], tag="sink")
+    x_out = torch.empty((cfg.block_tokens, cfg.latent_ch), device="cuda")
+    ref = TickScheduler(cfg)
+    check_ticks = {3, 6, wl.num_blocks + 2}
+    for k in range(wl.num_blocks + 3):
+        sink = sink_snapshot(s, cfg) if k in check_ticks else None
+        fin = s.step(_dev(block_noise(wl, k)) if k < wl.num_blocks else None, x_out)
+        run, fin_o = ref.begin_tick(k < wl.num_blocks)
+        for i, bb in run:
+            ref.append(i, bb)
+        ref.end_tick(fin_o)
+        assert fin == fin_o
+        np.testing.assert_array_equal(s.index_state(), ref.index_state())
+        if k in check_ticks:
+            for (b, i) in _active(s, cfg):
+                check_step(s, cfg, W, b, i, rows=R, tag=f"tick {k}", sink=sink)
+        if fin == 0:
+            check_sink(s, cfg, W, to_np(x_out)[:cfg.sink_tokens], rows=R[R < cfg.sink_tokens], tag="AAS sink")
+    s.synchronize()
+    s.close()
+
+
+def test_full_shape_pipelined_equals_sequential_bitwise():
+    wl = Workload("cmp", STREAM.cfg.replace(num_layers=2, sink_mode=SINK_FIXED), 4, 5, 0.02)
+    W = make_weights(wl)
+    outs = {}
+    for sched in (SCHED_PIPELINED, SCHED_SEQUENTIAL):
+        cfg = wl.cfg.replace(schedule=sched)
+        s, _ = make_stream(wl, W, cfg)
+        x_out = torch.empty((cfg.block_tokens, cfg.latent_ch), device="cuda")
+        res = {}
+        for k in range(wl.num_blocks + (3 if sched == SCHED_PIPELINED else 0)):
+            fin = s.step(_dev(block_noise(wl, k)) if k < wl.num_blocks else None, x_out)
+            if fin >= 0:
+                res[fin] = to_np(x_out).copy()
+        s.close()
+        outs[sched] = res
+    for b in range(wl.num_blocks):
+        np.testing.assert_array_equal(outs[SCHED_PIPELINED][b], outs[SCHED_SEQUENTIAL][b])
+
+
+@pytest.mark.slow
+def test_soak_10000_blocks_rolling_rope_and_ring():
+    """10,000 blocks at the 14B shape with 2 sublayers; every (block, step) input
+    is fresh noise.  Integer state bit-exact every tick; every op checked on
+    sampled rows for blocks 1, 10, 100, 1000 and 9999 (RoPE positions up to 29,999)."""
+    wl = SOAK
+    cfg = wl.cfg
+    S = cfg.num_steps
+    s, W = make_stream(wl, capture=False)
+    R = sample_rows(cfg.block_tokens, n=16)
+    checked = {1, 10, 100, 1000, wl.num_blocks - 1}
+    g = torch.Generator(device="cuda")
+    g.manual_seed(wl.seed)
+    T, C = cfg.block_tokens, cfg.latent_ch
+    x_out = torch.empty((T, C), device="cuda")
+    ref = TickScheduler(cfg)
+    held = [-1] * S
+    n_checked = 0
+    for k in range(wl.num_blocks + S - 1):
+        has_new = k < wl.num_blocks
+        slots = [k if has_new else -1] + held[:-1]
+        want_check = any(b in checked for b in slots if b >= 0)
+        s.capture(want_check)
+        for i in range(1, S):
+            b = slots[i]
+            if b >= 0:
+                x = _dev(step_input(wl, b, i)) if b in checked else torch.randn((T, C), generator=g, device="cuda")
+                s.set_slot_input(i, x)
+        xn = (_dev(step_input(wl, k, 0)) if k in checked else torch.randn((T, C), generator=g, device="cuda")) \
+            if has_new else None
+        sink = sink_snapshot(s, cfg) if want_check else None
+        fin = s.step(xn, x_out)
+        held = slots
+        run, fin_o = ref.begin_tick(has_new)
+        for i, bb in run:
+            ref.append(i, bb)
+        ref.end_tick(fin_o)
+        assert fin == fin_o
+        np.testing.assert_array_equal(s.index_state(), ref.index_state())
+        if want_check:
+            for (b, i) in _active(s, cfg):
+                if b in checked:
+                    check_step(s, cfg, W, b, i, rows=R, tag=f"soak tick {k}", sink=sink)
+                    n_checked += 1
+        if k % 1000 == 0:
+            s.synchronize()
+    s.synchronize()
+    s.close()
+    assert n_checked == len(checked) * S
+
+
+@pytest.mark.slow
+def test_largest_sweep_point_45x80_window_8():
+    wl = sweep_point((45, 80), 8)
+    wl = Workload(wl.name, wl.cfg, wl.seed, 10, wl.w_std, wl.head_std)
+    cfg = wl.cfg
+    s, W = make_stream(wl, capture=False)
+    R = sample_rows(cfg.block_tokens, n=16)
+    x_out = torch.empty((cfg.block_tokens, cfg.latent_ch), device="cuda")
+    last = wl.num_blocks + 2
+    for k in range(last + 1):
+        s.capture(k == last)
+        fin = s.step(_dev(block_noise(wl, k)) if k < wl.num_blocks else None, x_out)
+    for (b, i) in _active(s, cfg):
+        check_step(s, cfg, W, b, i, rows=R, tag="sweep 45x80 w8")
+    s.synchronize()
+    s.close()
