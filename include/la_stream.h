@@ -20,6 +20,12 @@
  *   - each step ends with the flow-matching Euler update
  *     x_{t_{i+1}} = x_{t_i} + (t_{i+1} - t_i) v (papernotes note, 损失函数).
  *
+ * The synthetic stack per step: h = x W_in^T; per sublayer
+ * [q|k|v] = n(h) W_qkv^T, Rolling RoPE on q/k, ring append, block-causal
+ * attention, h += O W_out^T; v = n(h) W_head^T; with n the per-token RMS
+ * normalisation n(h) = h / sqrt(mean(h^2) + LA_RMS_EPS) (the pages give no
+ * layer internals; without it the stacked residual map expands).
+ *
  * Conventions for every function:
  *   - Return value: LA_OK (0) or a negative LA_E* status.  No C++ exception
  *     crosses this boundary.  la_last_error() gives a text for the last
@@ -60,6 +66,8 @@ extern "C" {
 #define LA_BF16              0  /* bf16 GEMM operands and attention operands, fp32
                                    accumulation, fp32 residual stream and latent x    */
 #define LA_FP32              1  /* fp32 everywhere (SIMT path, no TF32)                */
+
+#define LA_RMS_EPS 1e-6
 
 /* Limits of this build. */
 #define LA_MAX_STEPS     8
@@ -262,11 +270,15 @@ int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, vo
  * lengths, 1 <= nseg <= LA_MAX_WINDOW + 2, seg_len >= 1).
  * dtype LA_BF16: q/K/V bf16, d == 128, tcgen05; out DEVICE bf16 [Tq, H*d] and,
  *   if out32 != NULL, an fp32 copy [Tq, H*d] (the value before rounding).
- * dtype LA_FP32: q/K/V/out fp32, d % 8 == 0, d <= 128, SIMT; out32 ignored.
+ *   q_scaled != 0: q is already multiplied by log2(e)/sqrt(d) (the stream's
+ *   layout); 0: plain q.
+ * dtype LA_FP32: q/K/V/out fp32, d % 8 == 0, d <= 128, SIMT; out32 and
+ *   q_scaled ignored.
  */
 int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t d,
                     int32_t nseg, const void* const* k_seg, const void* const* v_seg,
-                    const int64_t* seg_len, void* out, float* out32, void* cuda_stream);
+                    const int64_t* seg_len, void* out, float* out32, int32_t q_scaled,
+                    void* cuda_stream);
 
 /*
  * Standalone Euler update x[r, :] += dt[r / rows_per_group] * v[r, :] over

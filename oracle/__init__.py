@@ -20,6 +20,8 @@ What it computes (Live Avatar, arXiv 2512.04677, as described on the pages):
     admirer.cn article, "滾動位置編碼");
   * Adaptive Attention Sink: the first generated latent replaces the reference
     sink once (papernotes note, 关键设计 3; gitcode blog, question 5);
+  * per-token RMS pre-norm of every sublayer input and of the head input
+    (a reading: the pages give no layer internals; see oracle/norm.py);
   * flow-matching velocity v ~ x1 - x0 and an Euler step between the 4
     distilled timesteps (papernotes note, 损失函数 / L_FM);
   * the timestep-pipelined order of the 4 in-flight blocks (10100.com article,
@@ -41,11 +43,12 @@ worked example.
 from .rope import axis_frequencies, rope_rotate, block_positions, sink_positions
 from .attention import block_causal_attention
 from .flow import euler_step
+from .norm import RMS_EPS, rms_norm
 from .schedule import TickScheduler, index_state_layout
 from .stream import OracleStream
 
 __all__ = [
     "axis_frequencies", "rope_rotate", "block_positions", "sink_positions",
-    "block_causal_attention", "euler_step", "TickScheduler", "index_state_layout",
+    "block_causal_attention", "euler_step", "rms_norm", "RMS_EPS", "TickScheduler", "index_state_layout",
     "OracleStream",
 ]

@@ -4,17 +4,19 @@ One slot pass (block b at step i), per the pages' description of the
 streaming DiT step (papernotes note, 整体框架 and 关键设计 2-4):
     h = x W_in^T                       (identity when latent_ch == hidden)
     for each layer l:
-        [q | k | v] = h W_qkv[l]^T      (heads of width d, q/k/v in that order)
+        [q | k | v] = n(h) W_qkv[l]^T   (n = per-token RMS norm; heads of width d)
         q, k = RoPE at (3b + f, r, c)
         cache[(l, i, b)] = (k, v)       noisy K/V of THIS step: timestep forcing
         drop cache[(l, i, b - window - 1)]
         sink K re-roped at (3b - 3, r, c) (Rolling RoPE), sink V as stored
         o = block-causal attention over [sink | window | block]
         h = h + o W_out[l]^T
-    v = h W_head^T                       (identity when latent_ch == hidden)
+    v = n(h) W_head^T                    (identity map when latent_ch == hidden)
     x <- x + (t_{i+1} - t_i) v
-The synthetic sublayers have no norm, FFN or conditioning (the pages give no
-layer internals; the sublayer is the attention step the pages describe).
+The synthetic sublayers have no FFN or conditioning (the pages give no layer
+internals; the sublayer is the attention step the pages describe); the
+per-token RMS pre-norm keeps the stacked residual map from expanding (see
+oracle/norm.py).
 
 Sink (reading: the sink frame passes through the same stack attending only to
 itself; its un-roped K and its V are kept per layer and shared by all slots).
@@ -28,6 +30,7 @@ import numpy as np
 
 from .attention import block_causal_attention
 from .flow import euler_step
+from .norm import rms_norm
 from .rope import block_positions, rope_rotate, sink_positions
 from .schedule import TickScheduler
 
@@ -63,7 +66,8 @@ class OracleStream:
         return x.copy() if self.w_in is None else x @ self.w_in.T
 
     def project_head(self, h):
-        return h.copy() if self.w_head is None else h @ self.w_head.T
+        n = rms_norm(h)
+        return n if self.w_head is None else n @ self.w_head.T
 
     # -- sink -----------------------------------------------------------------
     def set_sink(self, latent):
@@ -75,7 +79,7 @@ class OracleStream:
         pt, ph, pw = sink_positions(c, t0)
         self.sink_k, self.sink_v = [], []
         for l in range(c.num_layers):
-            q, k, v = self._split_heads(h @ self.w_qkv[l].T)
+            q, k, v = self._split_heads(rms_norm(h) @ self.w_qkv[l].T)
             self.sink_k.append(k.copy())
             self.sink_v.append(v.copy())
             qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
@@ -99,7 +103,7 @@ class OracleStream:
             tr["h_in"] = h.copy()
             tr["record"] = list(rec)
         for l in range(c.num_layers):
-            q, k, v = self._split_heads(h @ self.w_qkv[l].T)
+            q, k, v = self._split_heads(rms_norm(h) @ self.w_qkv[l].T)
             qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
             kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
             self.cache[(l, i, b)] = (kr, v.copy(), (b, i))

@@ -72,7 +72,7 @@ def load():
         "la_op_gemm": (c_int, [c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64,
                                c_int64, POINTER(c_float), c_int64, c_void_p]),
         "la_op_attention": (c_int, [c_int32, c_void_p, c_int64, c_int32, c_int32, c_int32, POINTER(c_void_p),
-                                    POINTER(c_void_p), POINTER(c_int64), c_void_p, c_void_p, c_void_p]),
+                                    POINTER(c_void_p), POINTER(c_int64), c_void_p, c_void_p, c_int32, c_void_p]),
         "la_op_euler": (c_int, [c_void_p, c_void_p, c_int64, c_int64, POINTER(c_float), c_int64, c_void_p]),
     }
     for name, (res, args) in sig.items():

@@ -218,7 +218,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       // hidden by ILP, not by other warps)
       float x[128];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = PRESCALED ? __uint_as_float(s[c]) : __uint_as_float(s[c]) * sc;
+      for (int c = 0; c < 128; ++c) x[c] = PRESCALED ? __uint_as_float(s[c]) : __fmul_rn(__uint_as_float(s[c]), sc);
       float mx8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;

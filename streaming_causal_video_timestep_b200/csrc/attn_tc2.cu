@@ -19,6 +19,7 @@
 // PRESCALED, else scaled and rounded first), so the row maximum contributes
 // exactly 2^0 = 1 and the row sum is >= 1.  The running max is updated lazily:
 // O is rescaled in TMEM only when the max grows by more than 2^8.
+#include <cstdio>
 #include <cstdlib>
 
 #include "kernels.h"
@@ -52,7 +53,7 @@ __device__ __forceinline__ int group_tiles(const AttnGroup& g) {
 }
 
 template <bool PRESCALED>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(320, 1)
 k_attn_tc2(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -209,30 +210,25 @@ k_attn_tc2(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPa
         cur.next(g);
         if (abort_flag || !mbar_wait(&s_full[w], static_cast<uint32_t>(t & 1), err)) { ok = false; break; }
         tc_fence_after();
-        uint32_t s[128];
-        {
-          uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
-          uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-          uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
-          uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
-          tmem_ld32(s_base + 0, s0);
-          tmem_ld32(s_base + 32, s1);
-          tmem_ld32(s_base + 64, s2);
-          tmem_ld32(s_base + 96, s3);
-          tmem_ld_wait();
-        }
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float x = __uint_as_float(s[c]);
-          if (!PRESCALED) x *= sc;
-          if (c >= valid) x = -INFINITY;
-          s[c] = __float_as_uint(x);
-        }
+        // pass 1: row max of the scaled scores, 64 columns at a time
         float mx8[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(s[c]));
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t a[32], b[32];
+          tmem_ld32(s_base + hf * 64, a);
+          tmem_ld32(s_base + hf * 64 + 32, b);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float xa = __uint_as_float(a[i]), xb = __uint_as_float(b[i]);
+            if (!PRESCALED) { xa = __fmul_rn(xa, sc); xb = __fmul_rn(xb, sc); }
+            if (hf * 64 + i >= valid) xa = -INFINITY;
+            if (hf * 64 + 32 + i >= valid) xb = -INFINITY;
+            mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(xa, xb));
+          }
+        }
         const float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const bool need = m_tile > m_ref + 8.0f;
@@ -254,22 +250,34 @@ k_attn_tc2(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPa
             }
           }
         }
-        // P = 2^(x - m) as bf16 into the first 64 columns of this tile's S
+        // pass 2: P = 2^(x - m) as bf16 over the consumed S columns: S columns
+        // [64h, 64h+64) become P columns [32h, 32h+32) (written only after read)
         float rs8[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t a[32], b[32];
+          tmem_ld32(s_base + hf * 64, a);
+          tmem_ld32(s_base + hf * 64 + 32, b);
+          tmem_ld_wait();
+          uint32_t pa[16], pb[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int c = half * 64 + 2 * i;
-            const float p0 = fast_exp2(__uint_as_float(s[c]) - m_new);
-            const float p1 = fast_exp2(__uint_as_float(s[c + 1]) - m_new);
-            rs8[i & 7] += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            float x0 = __uint_as_float(a[2 * i]), x1 = __uint_as_float(a[2 * i + 1]);
+            float y0 = __uint_as_float(b[2 * i]), y1 = __uint_as_float(b[2 * i + 1]);
+            if (!PRESCALED) { x0 = __fmul_rn(x0, sc); x1 = __fmul_rn(x1, sc); y0 = __fmul_rn(y0, sc); y1 = __fmul_rn(y1, sc); }
+            const int c = hf * 64 + 2 * i;
+            const float p0 = c < valid ? fast_exp2(x0 - m_new) : 0.f;
+            const float p1 = c + 1 < valid ? fast_exp2(x1 - m_new) : 0.f;
+            const float p2 = c + 32 < valid ? fast_exp2(y0 - m_new) : 0.f;
+            const float p3 = c + 33 < valid ? fast_exp2(y1 - m_new) : 0.f;
+            rs8[i & 7] += (p0 + p1) + (p2 + p3);
+            pa[i] = pack_bf16x2(p0, p1);
+            pb[i] = pack_bf16x2(p2, p3);
           }
-          tmem_st32(s_base + half * 32, pk);
+          tmem_st16(s_base + hf * 32, pa);
+          tmem_st16(s_base + hf * 32 + 16, pb);
         }
         tmem_st_wait();
         l = l * alpha + (((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7])));
@@ -335,7 +343,17 @@ cudaError_t launch_attn_tc2(const AttnMaps& maps, const AttnParams& p, cudaStrea
   const int qtiles = (p.Tq + BQ - 1) / BQ;
   dim3 grid((qtiles + 1) / 2, p.H, p.ngroups);
   kern<<<grid, 320, SMEM, st>>>(maps, p);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, kern);
+    std::fprintf(stderr,
+                 "k_attn_tc2 launch refused (%s): regs %d, maxThreadsPerBlock %d, static smem %zu, "
+                 "max dynamic smem %d, requested dynamic smem %zu, local %zu, param bytes %zu\n",
+                 cudaGetErrorString(e), fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes,
+                 fa.maxDynamicSharedSizeBytes, SMEM, fa.localSizeBytes, sizeof(AttnMaps) + sizeof(AttnParams));
+  }
+  return e;
 }
 
 cudaError_t launch_attention_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st) {

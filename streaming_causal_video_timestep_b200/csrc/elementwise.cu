@@ -211,6 +211,44 @@ __global__ void __launch_bounds__(256) k_euler(float* __restrict__ x, const floa
   }
 }
 
+// Per-token RMS normalisation: out[r, :] = h[r, :] / sqrt(mean(h[r, :]^2) + eps),
+// one CTA per row, fp32 sum of squares; writes bf16 and / or fp32.  D % 4 == 0.
+__global__ void __launch_bounds__(256) k_rmsnorm(const float* __restrict__ h, long long D, float eps,
+                                                 __nv_bfloat16* __restrict__ out_bf16, float* __restrict__ out_f32) {
+  const long long row = blockIdx.x;
+  const float4* h4 = reinterpret_cast<const float4*>(h + row * D);
+  const int n4 = static_cast<int>(D / 4);
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = h4[i];
+    ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+  }
+  __shared__ float red[8];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  const float scale = rsqrtf(red[0] / static_cast<float>(D) + eps);
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = h4[i];
+    const float4 o = make_float4(v.x * scale, v.y * scale, v.z * scale, v.w * scale);
+    if (out_f32) reinterpret_cast<float4*>(out_f32 + row * D)[i] = o;
+    if (out_bf16) {
+      uint2 w;
+      w.x = pack_bf16x2(o.x, o.y);
+      w.y = pack_bf16x2(o.z, o.w);
+      reinterpret_cast<uint2*>(out_bf16 + row * D)[i] = w;
+    }
+  }
+}
+
 int grid_for(long long n, int per_block = 256) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -282,5 +320,12 @@ cudaError_t launch_euler(float* x, const float* v, long long rows, long long C, 
   }
   const long long n4 = rows * C / 4;
   k_euler<<<grid_for(n4), 256, 0, st>>>(x, v, n4, C / 4, rows_per_group, e, vtap);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const float* h, long long rows, long long D, float eps, void* out_bf16, float* out_f32,
+                           cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  k_rmsnorm<<<static_cast<unsigned>(rows), 256, 0, st>>>(h, D, eps, static_cast<__nv_bfloat16*>(out_bf16), out_f32);
   return cudaGetLastError();
 }

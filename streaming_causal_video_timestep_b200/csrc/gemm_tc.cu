@@ -134,7 +134,7 @@ __device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, const Qk
         acc[4 * i + 2] = h.z;
         acc[4 * i + 3] = h.w;
       }
-      store_bf16x32(reinterpret_cast<__nv_bfloat16*>(ep.out) + off, acc);
+      if (ep.out) store_bf16x32(reinterpret_cast<__nv_bfloat16*>(ep.out) + off, acc);
       break;
     }
     case EPI_SET32: {

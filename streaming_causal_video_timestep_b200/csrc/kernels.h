@@ -67,3 +67,8 @@ cudaError_t launch_cvt_bf16(const float* x, void* xb, long long n, cudaStream_t 
 // x[r, :] += dt[g] * v[r, :], g = r / rows_per_group, for active groups.
 cudaError_t launch_euler(float* x, const float* v, long long rows, long long C, int rows_per_group,
                          const float* dt, const int* active, float* vtap, cudaStream_t st);
+
+// out = h / sqrt(mean(h^2) + eps) per row of D fp32 values (D % 4 == 0), written
+// as bf16 (out_bf16) and / or fp32 (out_f32).
+cudaError_t launch_rmsnorm(const float* h, long long rows, long long D, float eps, void* out_bf16, float* out_f32,
+                           cudaStream_t st);

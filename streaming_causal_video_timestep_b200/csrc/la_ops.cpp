@@ -58,7 +58,7 @@ int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, vo
 
 int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t d, int32_t nseg,
                     const void* const* k_seg, const void* const* v_seg, const int64_t* seg_len, void* out,
-                    float* out32, void* cuda_stream) {
+                    float* out32, int32_t q_scaled, void* cuda_stream) {
   if (!q || !out || !k_seg || !v_seg || !seg_len || Tq < 1 || Tq > (1 << 30) || H < 1 || H > 65535) return LA_EINVAL;
   if (nseg < 1 || nseg > LA_MAX_SEG || d < 8 || d > 128 || d % 8 != 0) return LA_EINVAL;
   for (int s = 0; s < nseg; ++s)
@@ -71,7 +71,7 @@ int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   p.out = out;
   p.out32 = dtype == LA_BF16 ? out32 : nullptr;
-  p.q_prescaled = 0;
+  p.q_prescaled = (dtype == LA_BF16 && q_scaled) ? 1 : 0;
   p.out_ld = static_cast<long long>(H) * d;
   p.err = nullptr;
   p.qbase = q;

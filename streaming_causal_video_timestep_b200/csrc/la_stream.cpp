@@ -152,8 +152,9 @@ struct la_stream {
 
   std::vector<void*> allocs;
   float* xs = nullptr;      // [nbuf][T][C]
-  float* h32 = nullptr;     // [nbuf*T][D]
-  void* hop = nullptr;      // [nbuf*T][D] dtype (fp32: == h32)
+  float* h32 = nullptr;     // [nbuf*T][D] residual stream
+  void* hop = nullptr;      // [nbuf*T][D] normalised GEMM operand, dtype (fp32: == hn32)
+  float* hn32 = nullptr;    // [nbuf*T][D] fp32 normalised residual (fp32 streams, identity head)
   void* xop = nullptr;      // [nbuf*T][C] bf16 (bf16 with an in-projection)
   float* qkv = nullptr;     // fp32 [nbuf*T][3D] (fp32 streams; bf16 fuses it into the GEMM)
   void* q_rope = nullptr;   // attn type [nbuf][H][T][d]
@@ -165,7 +166,8 @@ struct la_stream {
   void* sink_v = nullptr;   // attn type [L][H][F][d]
   float* sink_x = nullptr;  // [F][C]
   float* s_h32 = nullptr;   // [F][D]
-  void* s_hop = nullptr;
+  void* s_hop = nullptr;    // normalised operand (fp32 streams: == s_hn32)
+  float* s_hn32 = nullptr;
   void* s_xop = nullptr;
   float* s_qkv = nullptr;   // fp32 [F][3D]
   void* s_q = nullptr;      // attn type [H][F][d]
@@ -375,6 +377,15 @@ int capture_pass(la_stream* s, const PassDesc& pd, int layer) {
   return LA_OK;
 }
 
+constexpr float kRmsEps = 1e-6f;
+
+// Per-token RMS normalisation of the residual into the next GEMM's operand.
+int normalise(la_stream* s, const float* h, long long rows, void* op_bf16, float* op_f32) {
+  return launch(s, LA_KIND_OTHER, [&] {
+    return launch_rmsnorm(h, rows, s->D, kRmsEps, s->bf16 ? op_bf16 : nullptr, op_f32, s->st);
+  });
+}
+
 // One grouped pass over nbuf buffers (rows = nbuf*T) with the active ones in pd.
 int run_pass(la_stream* s, const PassDesc& pd) {
   const int T = s->T, D = s->D, C = s->C, H = s->H, d = s->d, F = s->F, S = s->S, E = s->E;
@@ -393,10 +404,10 @@ int run_pass(la_stream* s, const PassDesc& pd) {
        })) != LA_OK)
     return r;
 
-  // in-projection
+  // in-projection into the fp32 residual stream, then its normalised operand
   if (s->id_in) {
     if ((r = launch(s, LA_KIND_IN_PROJ, [&] {
-           return launch_in_identity(s->bf16, s->xs, s->h32, s->hop, static_cast<long long>(rows) * D, s->st);
+           return launch_in_identity(s->bf16, s->xs, s->h32, nullptr, static_cast<long long>(rows) * D, s->st);
          })) != LA_OK)
       return r;
   } else {
@@ -405,10 +416,11 @@ int run_pass(la_stream* s, const PassDesc& pd) {
            return launch_cvt_bf16(s->xs, s->xop, static_cast<long long>(rows) * C, s->st);
          })) != LA_OK)
       return r;
-    GemmEpiParams e = epi(EPI_SET32, s->bf16 ? s->hop : nullptr, s->h32, D);
+    GemmEpiParams e = epi(EPI_SET32, nullptr, s->h32, D);
     if ((r = gemm(s, LA_KIND_IN_PROJ, &s->tm_xop, &s->tm_win, s->xs, s->w_in, e, rows, D, C)) != LA_OK) return r;
   }
   if (s->capture && (r = capture_pass(s, pd, -1)) != LA_OK) return r;
+  if ((r = normalise(s, s->h32, rows, s->hop, s->bf16 ? nullptr : s->hn32)) != LA_OK) return r;
 
   RopeArgs ra = rope_args(s);
   AttnParams ap{};
@@ -454,7 +466,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
         return r;
     } else {
       GemmEpiParams eq = epi(EPI_STORE, s->qkv, nullptr, 3LL * D);
-      if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_hop, &s->tm_wqkv[l], s->h32, s->w_qkv[l], eq, rows, 3 * D, D)) !=
+      if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_hop, &s->tm_wqkv[l], s->hn32, s->w_qkv[l], eq, rows, 3 * D, D)) !=
           LA_OK)
         return r;
       if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(0, pd, ra, true, s->st); })) != LA_OK)
@@ -481,18 +493,23 @@ int run_pass(la_stream* s, const PassDesc& pd) {
     } else {
       if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) return r;
     }
-    // output projection + residual
-    GemmEpiParams eo = epi(EPI_RESID, s->hop, s->h32, D);
+    // output projection + residual, then the next operand (next layer or head)
+    GemmEpiParams eo = epi(EPI_RESID, nullptr, s->h32, D);
     if ((r = gemm(s, LA_KIND_OUT_GEMM, &s->tm_o, &s->tm_wout[l], s->attn_o, s->w_out[l], eo, rows, D, D)) != LA_OK)
       return r;
     if (s->capture && (r = capture_pass(s, pd, l)) != LA_OK) return r;
+    const bool last = l == s->L - 1;
+    const bool want_f32 = !s->bf16 || (last && s->id_head);
+    if ((r = normalise(s, s->h32, rows, (s->bf16 && !(last && s->id_head)) ? s->hop : nullptr,
+                       want_f32 ? s->hn32 : nullptr)) != LA_OK)
+      return r;
   }
 
   // velocity head + Euler update x += (t_{i+1} - t_i) v, per buffer
   float* vtap = s->capture ? s->cap_vall : nullptr;
   if (s->id_head) {
     if ((r = launch(s, LA_KIND_HEAD, [&] {
-           return launch_euler(s->xs, s->h32, rows, C, T, pd.dt, pd.active, vtap, s->st);
+           return launch_euler(s->xs, s->hn32, rows, C, T, pd.dt, pd.active, vtap, s->st);
          })) != LA_OK)
       return r;
   } else {
@@ -503,8 +520,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
       e.active[i] = pd.active[i];
     }
     e.vtap = vtap;
-    if ((r = gemm(s, LA_KIND_HEAD, &s->tm_hop, &s->tm_whead, s->bf16 ? s->hop : s->h32, s->w_head, e, rows, C, D)) !=
-        LA_OK)
+    if ((r = gemm(s, LA_KIND_HEAD, &s->tm_hop, &s->tm_whead, s->hn32, s->w_head, e, rows, C, D)) != LA_OK)
       return r;
   }
   if (s->capture) {
@@ -536,7 +552,7 @@ int run_sink(la_stream* s) {
     return r;
   if (s->id_in) {
     if ((r = launch(s, LA_KIND_IN_PROJ, [&] {
-           return launch_in_identity(s->bf16, s->sink_x, s->s_h32, s->s_hop, static_cast<long long>(F) * D, s->st);
+           return launch_in_identity(s->bf16, s->sink_x, s->s_h32, nullptr, static_cast<long long>(F) * D, s->st);
          })) != LA_OK)
       return r;
   } else {
@@ -544,7 +560,7 @@ int run_sink(la_stream* s) {
                       return launch_cvt_bf16(s->sink_x, s->s_xop, static_cast<long long>(F) * C, s->st);
                     })) != LA_OK)
       return r;
-    GemmEpiParams e = epi(EPI_SET32, s->bf16 ? s->s_hop : nullptr, s->s_h32, D);
+    GemmEpiParams e = epi(EPI_SET32, nullptr, s->s_h32, D);
     if ((r = gemm(s, LA_KIND_IN_PROJ, &s->tm_s_xop, &s->tm_win, s->sink_x, s->w_in, e, F, D, C)) != LA_OK) return r;
   }
   RopeArgs ra = rope_args(s);
@@ -564,9 +580,10 @@ int run_sink(la_stream* s) {
                          static_cast<size_t>(F) * D * 4, cudaMemcpyDeviceToDevice, s->st));
       s->cap_sink_valid = true;
     }
+    if ((r = normalise(s, s->s_h32, F, s->s_hop, s->bf16 ? nullptr : s->s_hn32)) != LA_OK) return r;
     GemmEpiParams eq = epi(s->bf16 ? EPI_STORE32 : EPI_STORE, s->s_qkv, nullptr, 3LL * D);
-    if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_s_hop, &s->tm_wqkv[l], s->bf16 ? s->s_hop : s->s_h32, s->w_qkv[l], eq,
-                  F, 3 * D, D)) != LA_OK)
+    if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_s_hop, &s->tm_wqkv[l], s->s_hn32, s->w_qkv[l], eq, F, 3 * D, D)) !=
+        LA_OK)
       return r;
     ra.qkv = s->s_qkv;
     float* kraw = s->sink_k + static_cast<long long>(l) * H * F * d;
@@ -586,7 +603,7 @@ int run_sink(la_stream* s) {
     } else {
       if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) return r;
     }
-    GemmEpiParams eo = epi(EPI_RESID, s->s_hop, s->s_h32, D);
+    GemmEpiParams eo = epi(EPI_RESID, nullptr, s->s_h32, D);
     if ((r = gemm(s, LA_KIND_OUT_GEMM, &s->tm_s_o, &s->tm_wout[l], s->s_o, s->w_out[l], eo, F, D, D)) != LA_OK)
       return r;
   }
@@ -749,6 +766,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   const long long NB = s->nbuf;
   const size_t es = s->es, ea = s->ea;
   const long long need = NB * T * C * 4 + NB * T * D * 4 + (s->bf16 ? NB * T * D * es : 0) +
+                         ((!s->bf16 || s->id_head) ? NB * T * D * 4 : 0) + F * D * 4 +
                          (s->bf16 && !s->id_in ? NB * T * C * 2 : 0) + (s->bf16 ? 0 : NB * T * 3 * D * 4) +
                          NB * T * D * ea + NB * T * D * es + NB * H * F * d * ea + 2 * L * S * E * H * T * d * ea +
                          L * H * F * d * (4 + ea) + F * C * 4 + F * D * 4 + F * D * es * 2 + F * C * 2 +
@@ -770,7 +788,8 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   } while (0)
   ALLOC_OR_BAIL(s->xs, NB * T * C * 4);
   ALLOC_OR_BAIL(s->h32, NB * T * D * 4);
-  if (s->bf16) ALLOC_OR_BAIL(s->hop, NB * T * D * es); else s->hop = s->h32;
+  if (!s->bf16 || s->id_head) ALLOC_OR_BAIL(s->hn32, NB * T * D * 4);
+  if (s->bf16) ALLOC_OR_BAIL(s->hop, NB * T * D * es); else s->hop = s->hn32;
   if (s->bf16 && !s->id_in) ALLOC_OR_BAIL(s->xop, NB * T * C * 2);
   if (!s->bf16) ALLOC_OR_BAIL(s->qkv, NB * T * 3 * D * 4);
   ALLOC_OR_BAIL(s->q_rope, NB * T * D * ea);
@@ -782,7 +801,8 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   ALLOC_OR_BAIL(s->sink_v, L * H * F * d * ea);
   ALLOC_OR_BAIL(s->sink_x, F * C * 4);
   ALLOC_OR_BAIL(s->s_h32, F * D * 4);
-  if (s->bf16) ALLOC_OR_BAIL(s->s_hop, F * D * es); else s->s_hop = s->s_h32;
+  if (s->bf16) ALLOC_OR_BAIL(s->s_hop, F * D * es);
+  else { ALLOC_OR_BAIL(s->s_hn32, F * D * 4); s->s_hop = s->s_hn32; }
   if (s->bf16 && !s->id_in) ALLOC_OR_BAIL(s->s_xop, F * C * 2);
   ALLOC_OR_BAIL(s->s_qkv, F * 3 * D * 4);
   ALLOC_OR_BAIL(s->s_q, H * F * d * ea);

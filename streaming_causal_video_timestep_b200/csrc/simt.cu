@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(128) k_attn_f32(const __grid_constant__ AttnPa
         const float* kr = kb + static_cast<long long>(j) * d;
         float dot = 0.f;
         for (int e = 0; e < d; ++e) dot = fmaf(qs[warp][e], kr[e], dot);
-        sj = dot * p.scale_log2;
+        sj = __fmul_rn(dot, p.scale_log2);   // rounded: the row max then gives exactly 2^0
       }
       float mx = sj;
 #pragma unroll

@@ -195,9 +195,10 @@ def op_gemm(A, W, epilogue="store", out=None, h32=None, dt=None, rows_per_group=
     check(code)
 
 
-def op_attention(q, ks, vs, out, out32=None, stream=None):
-    """q [H, Tq, d] bf16 (tcgen05) or fp32 (SIMT), unscaled; ks / vs lists of
-    [H, len, d]; out [Tq, H*d] in the input type; out32 optional fp32 copy."""
+def op_attention(q, ks, vs, out, out32=None, q_scaled=False, stream=None):
+    """q [H, Tq, d] bf16 (tcgen05) or fp32 (SIMT); ks / vs lists of [H, len, d];
+    out [Tq, H*d] in the input type; out32 optional fp32 copy; q_scaled: q is
+    already multiplied by log2(e)/sqrt(d) (bf16 only)."""
     lib = load()
     dtype = _dtype_code(q.dtype)
     H, Tq, d = q.shape
@@ -206,7 +207,7 @@ def op_attention(q, ks, vs, out, out32=None, stream=None):
     vp = (c_void_p * n)(*[v.data_ptr() for v in vs])
     ln = (c_int64 * n)(*[k.shape[1] for k in ks])
     code = lib.la_op_attention(dtype, _ptr(q), Tq, H, d, n, kp, vp, ln, _ptr(out), _ptr(out32),
-                               _stream_handle(stream))
+                               1 if q_scaled else 0, _stream_handle(stream))
     check(code)
 
 

@@ -17,6 +17,16 @@ def matvec_rows(X, W):
     return out
 
 
+def normalize_rows(X, eps=1e-6):
+    """Each row divided by the square root of (its mean square + eps)."""
+    out = []
+    for row in X:
+        ms = sum(v * v for v in row) / len(row)
+        s = math.sqrt(ms + eps)
+        out.append([v / s for v in row])
+    return out
+
+
 def rotate(vec, t, r, c, pairs, theta):
     pt, ph, pw = pairs
     res = list(vec)
@@ -84,7 +94,7 @@ class BruteStream:
         t0 = -c.sink_offset_frames
         self.sink = []
         for l in range(c.num_layers):
-            qkv = matvec_rows(h, self.wqkv[l])
+            qkv = matvec_rows(normalize_rows(h), self.wqkv[l])
             entries, qrot, krot = [], [], []
             for n, vec in enumerate(qkv):
                 _, r, cc = self._tok_rc(n)
@@ -105,7 +115,7 @@ class BruteStream:
         fpb = c.frames_per_block
         t_sink = fpb * b - c.sink_offset_frames if c.rolling_rope else -c.sink_offset_frames
         for l in range(c.num_layers):
-            qkv = matvec_rows(h, self.wqkv[l])
+            qkv = matvec_rows(normalize_rows(h), self.wqkv[l])
             qrot = []
             for n, vec in enumerate(qkv):
                 f, r, cc = self._tok_rc(n)
@@ -122,7 +132,8 @@ class BruteStream:
             o = self._layer_attend(qrot, visible)
             proj = matvec_rows(o, self.wout[l])
             h = [[a + bq for a, bq in zip(hr, pr)] for hr, pr in zip(h, proj)]
-        v = h if self.whead is None else matvec_rows(h, self.whead)
+        hn = normalize_rows(h)
+        v = hn if self.whead is None else matvec_rows(hn, self.whead)
         dt = c.timesteps[i + 1] - c.timesteps[i]
         return [[xa + dt * va for xa, va in zip(xr, vr)] for xr, vr in zip(x, v)]
 

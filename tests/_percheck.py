@@ -14,7 +14,7 @@ import numpy as np
 
 import math
 
-from oracle import block_causal_attention, euler_step, rope_rotate
+from oracle import block_causal_attention, euler_step, rms_norm, rope_rotate
 from oracle.rope import block_positions, sink_positions
 from workloads import DTYPE_BF16, bf16_round
 
@@ -22,9 +22,14 @@ from _helpers import assert_close, to_np
 
 
 def _operand(a, cfg):
-    """The value a GEMM consumes: bf16-rounded in bf16 streams, as is in fp32 streams."""
+    """The value a GEMM consumes: bf16-rounded in bf16 streams, fp32 in fp32 streams."""
     a = np.asarray(a, np.float32)
     return bf16_round(a).astype(np.float64) if cfg.dtype == DTYPE_BF16 else a.astype(np.float64)
+
+
+def _normed_operand(h, cfg):
+    """The per-token RMS-normalised residual as the next GEMM consumes it."""
+    return _operand(rms_norm(np.asarray(h, np.float64)).astype(np.float32), cfg)
 
 
 def check_sink(s, cfg, W, latent, rows=None, tag=""):
@@ -39,7 +44,7 @@ def check_sink(s, cfg, W, latent, rows=None, tag=""):
     assert_close(h0[R], want, dt, f"{tag} sink in-proj")
     for l in range(cfg.num_layers):
         hs = to_np(s.tap("sink_h", l))
-        qkv = _operand(hs[R], cfg) @ np.asarray(W.w_qkv[l], np.float64).T
+        qkv = _normed_operand(hs[R], cfg) @ np.asarray(W.w_qkv[l], np.float64).T
         k = qkv[:, D:2 * D].reshape(len(R), H, d)
         v = qkv[:, 2 * D:].reshape(len(R), H, d)
         assert_close(to_np(s.tap("sink_k", l)).transpose(1, 0, 2)[R], k, dt, f"{tag} sink K l{l}")
@@ -77,7 +82,7 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
     h_prev = h_in
     for l in range(L):
         wqkv = np.asarray(W.w_qkv[l], np.float64)
-        qkv = _operand(h_prev[R], cfg) @ wqkv.T
+        qkv = _normed_operand(h_prev[R], cfg) @ wqkv.T
         q = qkv[:, :D].reshape(len(R), H, d)
         k = qkv[:, D:2 * D].reshape(len(R), H, d)
         v = qkv[:, 2 * D:].reshape(len(R), H, d)
@@ -112,7 +117,8 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
         want = h_prev[R].astype(np.float64) + _operand(o_gpu[R], cfg) @ np.asarray(W.w_out[l], np.float64).T
         chk(h_next[R], want, f"h l{l}")
         h_prev = h_next
-    vel = h_prev[R].astype(np.float64) if w_head is None else _operand(h_prev[R], cfg) @ w_head.T
+    vel = (rms_norm(h_prev[R].astype(np.float64)) if w_head is None
+           else _normed_operand(h_prev[R], cfg) @ w_head.T)
     chk(to_np(s.tap("v", 0, i))[R], vel, "velocity")
     x_want = euler_step(x_in[R], vel, cfg.timesteps[i], cfg.timesteps[i + 1])
     chk(to_np(s.tap("x_out", 0, i))[R], x_want, "x")

@@ -115,7 +115,7 @@ def test_null_stream_calls_return_einval(lib):
 def test_op_entry_points_reject_bad_sizes(lib):
     assert lib.la_op_gemm(0, 0, None, None, None, None, 0, 0, 0, None, 0, None) == _lib.LA_EINVAL
     assert lib.la_op_euler(None, None, 0, 0, None, 0, None) == _lib.LA_EINVAL
-    assert lib.la_op_attention(0, None, 0, 0, 0, 0, None, None, None, None, None, None) == _lib.LA_EINVAL
+    assert lib.la_op_attention(0, None, 0, 0, 0, 0, None, None, None, None, None, 0, None) == _lib.LA_EINVAL
 
 
 def test_valid_config_without_gpu_fails_loudly(lib):

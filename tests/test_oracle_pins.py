@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import OracleStream, TickScheduler, block_causal_attention, euler_step, rope_rotate
+from oracle import OracleStream, TickScheduler, block_causal_attention, euler_step, rms_norm, rope_rotate
 from oracle.rope import axis_frequencies, block_positions, sink_positions, sink_temporal_position
 from workloads import (SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_AAS, SINK_FIXED, TINY,
                        StreamConfig, Workload, block_noise, make_weights, random_array)
@@ -338,25 +338,37 @@ def _special_weights(cfg, q_scale=0.0, k_scale=0.0, out_scale=1.0, sink=None):
 
 def test_uniform_attention_closed_form_counts_the_visible_tokens():
     """With W_q = W_k = 0, W_v = W_out = I and identity in/head projections the
-    layer adds the mean of the visible tokens' inputs, so one step gives
-    x' = x + dt (x + mean(sink_h, window inputs at this step, x))."""
+    layer adds the mean of the visible tokens' normalised inputs, so one step
+    gives x' = x + dt n(x + mean(n(sink), n(window inputs at this step), n(x)))
+    with n the per-token RMS normalisation."""
     cfg = TINY.cfg.replace(sink_mode=SINK_FIXED, window_blocks=2)
     rng = np.random.default_rng(10)
     sink = rng.standard_normal((cfg.sink_tokens, cfg.hidden)).astype(np.float32)
     W = _special_weights(cfg, sink=sink)
     s = OracleStream(cfg, W, trace=True)
     s.set_sink(sink)
-    # the sink's own layer: uniform over itself, so sink h_1 = sink + mean(sink) (unused later)
-    np.testing.assert_allclose(s.sink_v[0].reshape(cfg.sink_tokens, -1), sink, atol=0)
+    nrm = lambda a: a / np.sqrt((a.astype(np.float64) ** 2).mean(axis=-1, keepdims=True) + 1e-6)
+    # the sink's stored V is its normalised latent
+    np.testing.assert_allclose(s.sink_v[0].reshape(cfg.sink_tokens, -1), nrm(sink), rtol=1e-12, atol=1e-12)
     nb = 6
     for k in range(nb + 3):
         s.denoise_step(block_noise(Workload("n", cfg, 5, nb, 0.1), k) if k < nb else None)
     for (b, i), tr in [(key, v) for key, v in s.trace.items() if isinstance(key[0], int)]:
         x = tr["x_in"]
-        toks = [sink] + [s.trace[(bb, i)]["x_in"] for bb in range(max(0, b - 2), b)] + [x]
+        toks = [nrm(sink)] + [nrm(s.trace[(bb, i)]["x_in"]) for bb in range(max(0, b - 2), b)] + [nrm(x)]
         mean = np.concatenate(toks).mean(axis=0)
         dt = cfg.timesteps[i + 1] - cfg.timesteps[i]
-        np.testing.assert_allclose(tr["x_out"], x + dt * (x + mean[None, :]), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(tr["x_out"], x + dt * nrm(x + mean[None, :]), rtol=1e-12, atol=1e-12)
+
+
+def test_rms_norm_matches_torch_and_is_scale_free():
+    rng = np.random.default_rng(12)
+    h = rng.standard_normal((7, 64)) * rng.uniform(0.01, 1e4, size=(7, 1))
+    want = torch.nn.functional.rms_norm(torch.from_numpy(h), (64,), eps=1e-6).numpy()
+    np.testing.assert_allclose(rms_norm(h), want, rtol=1e-12, atol=1e-12)
+    big = rms_norm(h * 1e3)
+    np.testing.assert_allclose(np.sqrt((big ** 2).mean(axis=-1)), 1.0, rtol=1e-9)
+    np.testing.assert_allclose(big, rms_norm(h), rtol=1e-6)
 
 
 def test_oracle_stream_matches_scalar_brute_force_stream():
