@@ -287,6 +287,33 @@ int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t
 int la_op_euler(float* x, const float* v, int64_t rows, int64_t C, const float* dt,
                 int64_t rows_per_group, void* cuda_stream);
 
+/*
+ * Block attention for callers that cannot allocate device memory (a plugin
+ * whose host application owns all device memory through its own allocator or
+ * a fixed budget, or a real-time path where an allocation and its implicit
+ * synchronisation are not allowed).  No
+ * counterpart on the pages.  It takes a plain bf16 q, writes q times the
+ * softmax scale log2(e)/sqrt(d) (fp32 product, rounded once to bf16: the form
+ * the stream's QKV epilogue writes) to its one scratch buffer, and runs the
+ * la_op_attention kernel with q_scaled = 1 on it; the result equals
+ * la_op_attention(LA_BF16, that scaled q, ..., q_scaled = 1) bit for bit.  The
+ * scratch is a file-scope device array of LA_STATIC_Q_ELEMS bf16 values
+ * (16 MiB) instead of an allocation.  Every GPU that loads the library holds
+ * that array until the process exits.
+ *   - Arguments as la_op_attention with dtype LA_BF16 (q, segments, out, out32),
+ *     d == 128.  H*Tq*d must be <= LA_STATIC_Q_ELEMS, else LA_EINVAL with a
+ *     message on stderr.
+ *   - Calls nothing that allocates.  The first call on a device looks up the
+ *     array's device address (cudaGetSymbolAddress, with that device current);
+ *     make that first call before any stream capture.
+ *   - All calls share the array and overwrite the part they use (nothing needs
+ *     to start at zero); calls that overlap on the GPU race on it.
+ */
+#define LA_STATIC_Q_ELEMS (8LL * 1024 * 1024)
+int la_op_attention_static(const void* q, int64_t Tq, int32_t H, int32_t d, int32_t nseg,
+                           const void* const* k_seg, const void* const* v_seg,
+                           const int64_t* seg_len, void* out, float* out32, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif
