@@ -32,7 +32,7 @@ WORKLOAD = dict(
     workload="4-step timestep-forced stream: 4 in-flight blocks x 8 attention sublayers, grouped launch",
     hidden=5120, heads=40, head_dim=128, latent_ch=64, grid="30x52", tokens_per_block=4680, sink_tokens=1560,
     window_blocks=2, keys_per_query=15600, timesteps=[1.0, 0.75, 0.5, 0.25, 0.0], layers=8,
-    dtype="bf16 weights/activations, fp16 attention operands, fp32 accumulate and latent",
+    dtype="bf16 weights, activations and attention operands (q pre-scaled); fp32 accumulate, residual stream and latent",
     l2="inputs larger than L2: 1.68 GB weights + 9.2 GB ring caches read per tick",
     data="synthetic: N(0,1) latents, N(0,0.02) weights, seeded")
 

@@ -357,9 +357,11 @@ cudaError_t launch_attn_tc2(const AttnMaps& maps, const AttnParams& p, cudaStrea
 }
 
 cudaError_t launch_attention_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st) {
-  static const bool v1 = [] {
-    const char* e = std::getenv("LA_ATTN_V1");
-    return e && e[0] == '1';
+  static const int v = [] {
+    const char* e = std::getenv("LA_ATTN_VERSION");
+    return e ? std::atoi(e) : 3;
   }();
-  return v1 ? launch_attn_tc(maps, p, st) : launch_attn_tc2(maps, p, st);
+  if (v == 1) return launch_attn_tc(maps, p, st);
+  if (v == 2) return launch_attn_tc2(maps, p, st);
+  return launch_attn_tc3(maps, p, st);
 }

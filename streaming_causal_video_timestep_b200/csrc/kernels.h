@@ -21,7 +21,8 @@ struct AttnMaps {
 };
 cudaError_t launch_attn_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);    // 1 query tile / CTA
 cudaError_t launch_attn_tc2(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);   // 2 query tiles / CTA
-// The attention launcher used by the library (LA_ATTN_V1=1 in the environment selects the one-tile kernel).
+cudaError_t launch_attn_tc3(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);   // 2 tiles, scores in regs
+// The attention launcher used by the library (LA_ATTN_VERSION=1 / 2 in the environment selects an older kernel).
 cudaError_t launch_attention_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);
 
 // ---- SIMT fp32 -----------------------------------------------------------------------

@@ -112,5 +112,5 @@ extern "C" int la_op_attention_static(const void* q, int64_t Tq, int32_t H, int3
   k_prescale_q<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(scratch),
                                        n, p.scale_log2);
   if (cudaGetLastError() != cudaSuccess) return LA_ECUDA;
-  return launch_attn_tc2(maps, p, st) == cudaSuccess ? LA_OK : LA_ECUDA;
+  return launch_attention_tc(maps, p, st) == cudaSuccess ? LA_OK : LA_ECUDA;
 }
