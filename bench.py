@@ -37,6 +37,13 @@ WORKLOAD = dict(
     data="synthetic: N(0,1) latents, N(0,0.02) weights, seeded")
 
 
+# DRAM bytes (read + write) of one slot's attention launch (4680 queries x 15,600 keys x 40 heads x 128,
+# bf16 q/K/V and output) from one ncu capture of the one-slot attention microbenchmark: 379.7 MB read +
+# 41.2 MB written, against 415.2 MB of algorithmic bytes.  The grouped launch of the stream reads the
+# disjoint q / K / V of its S slots, so its traffic is S times this.
+ATTN_DRAM_BYTES_PER_SLOT = 420.8e6
+
+
 def _attn_flops_per_slot(T, F, nw, H, d):
     nk = F + nw * T + T
     return 4.0 * T * nk * d * H
@@ -223,7 +230,9 @@ def run_gpu(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(WORKLOAD, parallelism=f"replicas x{world} (independent streams, no collective)"),
         "roofline": {"bound": "tensor", "kernel": "block-causal attention (tcgen05)", "achieved": round(achieved, 1),
-                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": ATTN_DRAM_BYTES_PER_SLOT * S,
+                     "traffic_unit": "bytes per launch (ncu dram read+write, one-slot capture x slots)",
                      "peak_source": f"{pk['src']} bf16 sustained (fp16 dense rate = bf16 dense rate)",
                      "algorithmic_flops_per_launch": attn_flops_launch},
         "kernels": kernels,

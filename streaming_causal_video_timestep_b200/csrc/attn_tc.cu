@@ -1,27 +1,39 @@
-// Block-causal attention on tcgen05 tensor cores, head_dim 128: bf16 q/K/V/P
-// operands, fp32 scores, softmax and accumulation, bf16 output.
+// Block-causal attention, tcgen05, head_dim 128, two query tiles per CTA,
+// softmax with the scores of a row held in registers.
 //
-// One CTA = 128 queries of one (group, head); the keys are the group's list of
-// segments [sink | window blocks oldest first | the block itself], walked in
-// tiles of 128 keys (the last tile of a segment is ragged and masked).
-// 6 warps:
-//   warp 0      TMA producer: Q once, then K_t and V_t tiles (two 64-column
-//               boxes each, 128-byte swizzle) into a 4-deep ring;
-//   warp 1      TMEM owner (512 columns: S0 | S1 | O) and MMA issuer:
-//               S_t = Q K_t^T into S[t%2] (K-major A and B), then
-//               O += P_{t-1} V_{t-1} (P K-major from shared memory, V read
-//               MN-major straight from its [keys, d] tile);
-//   warps 2..5  softmax: thread = query row = TMEM lane.  tcgen05.ld of the S
-//               row, masked row max, exp2, row sum, lazy rescale of O in TMEM
-//               (only when the running max grows by more than 2^8), P written
-//               to shared memory as bf16 in the swizzled K-major layout, then
-//               the final 1/l normalisation and bf16 store (plus an optional
-//               fp32 copy).
-// Scores are formed in the log2 domain: with q pre-multiplied by log2(e)/sqrt(d)
-// (PRESCALED, the stream's QKV epilogue does it) p = 2^(s - max s); otherwise the
-// scaled score x = s * scale is rounded first.  Either way the row maximum gives
-// exactly 2^0 = 1, so the row sum is >= 1 whatever the magnitude of the logits.
-// S_{t+1} is computed on the tensor cores while the softmax warps work on S_t.
+// One CTA = up to 256 queries (two 128-row tiles A and B) of one (group, head),
+// sharing every K/V tile of the group's segments [sink | window | block].
+// 12 warps in three warpgroups:
+//   warpgroup 0  warp 0: TMA producer (Q_A, Q_B once, then K_t / V_t as two
+//                64-column 128-byte-swizzled boxes each, 5-stage ring);
+//                warp 1: TMEM owner (512 columns: S_A | S_B | O_A | O_B) and
+//                MMA issuer; warps 2-3 idle.  Drops to 56 registers a thread.
+//   warpgroup 1  softmax of tile A, warpgroup 2 softmax of tile B: one thread
+//                per query row (= TMEM lane).  Raised to 224 registers a thread
+//                so that a row's 128 scores of a key tile stay in registers
+//                (one tensor-memory read per tile).
+// Per key tile t the tensor core runs, in issue order,
+//   ... PV_A(t-1), S_A(t), PV_B(t-1), S_B(t) ...
+// so while one softmax warpgroup turns S into P the tensor core works on the
+// other tile.  P is written as bf16 into the first 64 columns of its own S
+// tile (tcgen05.st) and read from there as the A operand of O += P V
+// (tcgen05.mma with A in tensor memory); V is read MN-major from its [keys, d]
+// tile.
+// Scores are in the log2 domain (q pre-multiplied by log2(e)/sqrt(d) when
+// PRESCALED, else scaled here first), so the row maximum contributes exactly
+// 2^0 = 1.  The running max is updated lazily: O is rescaled in TMEM only when
+// the max grows by more than 2^8.
+//
+// The exponentials: at 16 ex2 per clock per SM the special-function unit needs
+// as many cycles for the 128 x 128 exponentials of a tile pair as the tensor
+// core needs for its two 128 x 128 x 128 products, so on full key tiles EMU of
+// every 8 column pairs are computed on the FMA pipe instead (exp2_poly2 below:
+// Cody-Waite split into integer and fraction, as in the FlashAttention-4
+// softmax, with a polynomial of our own fit).  Partial tiles (a segment's
+// ragged tail) use ex2 only, so masked keys get exactly 0.
+#include <cstdio>
+#include <cstdlib>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -29,12 +41,19 @@ namespace {
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int NS = 4;
-constexpr uint32_t HALF = 16384;            // one 128-row x 128-byte swizzled box
+constexpr int NS = 5;
+constexpr int THREADS = 384;
+constexpr int LAUNCH_REGS = 168;            // 65536 / 384 rounded down to the allocation unit of 8
+constexpr int REGS_LOW = 56;                // warpgroup 0 after setmaxnreg.dec
+constexpr int REGS_HIGH = 224;              // warpgroups 1-2 after setmaxnreg.inc
+static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * LAUNCH_REGS, "register split exceeds the launch");
+constexpr uint32_t HALF = 16384;            // 128 rows x 128 bytes, one swizzle-128B box
 constexpr uint32_t TILE = 2 * HALF;         // 128 rows x 128 bf16
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t O_COL = 256;
-constexpr size_t SMEM = 1024 + TILE /*Q*/ + NS * TILE /*K,V ring*/ + TILE /*P*/ + 256;
+constexpr size_t SMEM = 1024 + 2 * TILE /*Q_A, Q_B*/ + NS * TILE /*K, V ring*/ + 256;
+
+__device__ __forceinline__ uint32_t s_col(int w) { return static_cast<uint32_t>(w * 128); }
+__device__ __forceinline__ uint32_t o_col(int w) { return static_cast<uint32_t>(256 + w * 128); }
 
 struct SegCursor {
   int seg = 0, start = 0;
@@ -50,29 +69,109 @@ __device__ __forceinline__ int group_tiles(const AttnGroup& g) {
   return n;
 }
 
-template <bool PRESCALED>
-__global__ void __launch_bounds__(192, 1)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+template <int N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
+// 2^x for a pair, x in (-inf, 9): clamp at -125 (2^-125 ~ 2e-38, so the result
+// is a normal float), split x = j + f with j = round(x) by adding and removing
+// 1.5 * 2^23 (|f| <= 1/2, exact), approximate 2^f by
+//   p(f) = 1 + f (c1 + f (c2 + f c3)),
+// the degree-3 polynomial with p(0) = 1 of least maximum relative error on
+// [-1/2, 1/2] (fit by iteratively reweighted least squares; max relative error
+// 1.0e-4 in fp32, 19x below half a bf16 ulp), and add j to its exponent field:
+// the low bits of (x + 1.5 * 2^23) hold j, so (bits << 23) is j << 23 mod 2^32.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+  constexpr float c1 = 0.6932829022407532f, c2 = 0.2422107458114624f, c3 = 0.055008791387081146f;
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+  const float2 j = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(f, make_float2(c3, c3), make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(1.0f, 1.0f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// One row's pass over the 128 scores of a key tile held in s[]: row max (masked
+// beyond `valid` when MASKED), lazy max update, P = 2^(s - m) into P[] (bf16
+// pairs), returns the tile's row sum of the unrounded P; m_ref / alpha / need
+// are updated for the caller.
+template <bool MASKED, int EMU>
+__device__ __forceinline__ float softmax_tile(float (&s)[128], uint32_t (&P)[64], int valid, float& m_ref,
+                                              float& alpha, bool& need) {
+  if (MASKED) {
+#pragma unroll
+    for (int i = 0; i < 128; ++i)
+      if (i >= valid) s[i] = -INFINITY;
+  }
+  float mx[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float a = fmax3(s[32 * c], s[32 * c + 1], s[32 * c + 2]);
+#pragma unroll
+    for (int i = 3; i + 1 < 32; i += 2) a = fmax3(a, s[32 * c + i], s[32 * c + i + 1]);
+    mx[c] = fmaxf(a, s[32 * c + 31]);
+  }
+  const float m_tile = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+  need = m_tile > m_ref + 8.0f;
+  const float m_new = need ? m_tile : m_ref;
+  alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
+  m_ref = m_new;
+  const float2 negm = make_float2(-m_new, -m_new);
+  float2 acc[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const float2 x = __fadd2_rn(make_float2(s[2 * i], s[2 * i + 1]), negm);
+    float2 p;
+    if (!MASKED && (i & 7) >= 8 - EMU) {
+      p = exp2_poly2(x);
+    } else {
+      p.x = fast_exp2(x.x);
+      p.y = fast_exp2(x.y);
+    }
+    acc[i & 3] = __fadd2_rn(acc[i & 3], p);
+    P[i] = pack_bf16x2(p.x, p.y);
+  }
+  const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+  const float2 a = __fadd2_rn(a01, a23);
+  return a.x + a.y;
+}
+
+template <bool PRESCALED, int EMU>
+__global__ void __launch_bounds__(THREADS, 1)
 k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = smem + TILE;
-  uint8_t* sP = sKV + NS * TILE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + TILE);
+  uint8_t* sQ = smem;                       // Q_A at 0, Q_B at TILE
+  uint8_t* sKV = smem + 2 * TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * TILE);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + NS;
-  uint64_t* s_full = kv_empty + NS;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* drain = pv_done + 1;
+  uint64_t* s_full = kv_empty + NS;         // [2]
+  uint64_t* p_full = s_full + 2;            // [2]
+  uint64_t* pv_done = p_full + 2;           // [2]
+  uint64_t* drain = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   __shared__ volatile int abort_flag;
 
   const AttnGroup& g = p.g[blockIdx.z];
   const int h = blockIdx.y;
-  const int q0 = blockIdx.x * BQ;
+  const int q0 = blockIdx.x * 2 * BQ;
+  const int nq = (q0 + BQ < p.Tq) ? 2 : 1;  // query tiles of this CTA
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   int* err = p.err;
 
@@ -83,12 +182,11 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w], 4);
+      mbar_init(&pv_done[w], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -102,13 +200,17 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
   const uint32_t tmem = *tmem_slot;
   const int nt = group_tiles(g);
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < 4) {
+    regs_dec<REGS_LOW>();
+    if (warp == 0 && lane == 0) {
+      // -------------------------------------------------------------- producer
       int last_parity[NS];
       for (int i = 0; i < NS; ++i) last_parity[i] = -1;
-      mbar_expect_tx(q_full, TILE);
-      tma_load_4d(sQ, &maps.q, q_full, 0, q0, h, g.q_slice);
-      tma_load_4d(sQ + HALF, &maps.q, q_full, 64, q0, h, g.q_slice);
+      mbar_expect_tx(q_full, 2 * TILE);
+      for (int w = 0; w < 2; ++w) {
+        tma_load_4d(sQ + w * TILE, &maps.q, q_full, 0, q0 + w * BQ, h, g.q_slice);
+        tma_load_4d(sQ + w * TILE + HALF, &maps.q, q_full, 64, q0 + w * BQ, h, g.q_slice);
+      }
       SegCursor cur;
       int n = 0;
       for (int t = 0; t < nt && !abort_flag; ++t) {
@@ -132,195 +234,162 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       mbar_wait(q_full, 0, err);
       for (int i = 0; i < NS; ++i)
         if (last_parity[i] >= 0) mbar_wait(&kv_full[i], static_cast<uint32_t>(last_parity[i]), err);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // -------------------------------------------------------------- MMA issuer
+      // The tensor core queues only a few MMAs, so the issue loop is kept lean:
+      // descriptors are precomputed and advanced by adding offsets, pv_done is
+      // committed only for the last key tile (the commit of S(t) already covers
+      // PV(t-1), issued before it), and the loop polls no flags.
       constexpr uint32_t idS = idesc_bf16(BQ, BKV, false, false);
       constexpr uint32_t idPV = idesc_bf16(BQ, 128, false, true);
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t p_addr = smem_u32(sP);
-      bool ok = mbar_wait(q_full, 0, err);
-      auto issue_pv = [&](int u) -> bool {
-        const int n = 2 * u + 1;
-        const int vs = n % NS;
-        if (!mbar_wait(p_full, static_cast<uint32_t>(u & 1), err)) return false;
-        if (!mbar_wait(&kv_full[vs], static_cast<uint32_t>((n / NS) & 1), err)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sKV + vs * TILE);
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t a = sdesc_kmajor(p_addr + (kk >> 2) * HALF + (kk & 3) * 32);
-          const uint64_t b = sdesc_mnmajor(v_addr + kk * 2048, HALF);
-          umma_bf16_ss(tmem + O_COL, a, b, idPV, (u > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&kv_empty[vs]);
-        umma_commit(pv_done);
-        return true;
-      };
-      for (int t = 0; t < nt && ok; ++t) {
-        if (abort_flag) { ok = false; break; }
-        const int n = 2 * t;
-        const int ks = n % NS;
-        const int sb = t & 1;
-        if (!mbar_wait(&kv_full[ks], static_cast<uint32_t>((n / NS) & 1), err)) { ok = false; break; }
-        if (!mbar_wait(&s_free[sb], static_cast<uint32_t>(((t >> 1) & 1) ^ 1), err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sKV + ks * TILE);
+      // The start-address field of a descriptor is (address >> 4) in its low 14
+      // bits; every shared address here is below 256 KB, so adding (offset >> 4)
+      // moves a descriptor by `offset` bytes without a carry out of the field.
+      const uint64_t dQ = sdesc_kmajor(smem_u32(sQ));
+      const uint64_t dK = sdesc_kmajor(smem_u32(sKV));
+      const uint64_t dV = sdesc_mnmajor(smem_u32(sKV), HALF);
+      auto issue_s = [&](int w, uint32_t stage) {
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk) {
           const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
-          umma_bf16_ss(tmem + sb * 128, sdesc_kmajor(q_addr + off), sdesc_kmajor(k_addr + off), idS,
+          umma_bf16_ss(tmem + s_col(w), dQ + ((w * TILE + off) >> 4), dK + ((stage * TILE + off) >> 4), idS,
                        kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[sb]);
-        umma_commit(&kv_empty[ks]);
-        if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+        umma_commit(&s_full[w]);
+      };
+      bool ok = mbar_wait(q_full, 0, err) && (nt == 0 || mbar_wait(&kv_full[0], 0, err));
+      if (ok && nt > 0) {
+        tc_fence_after();
+        for (int w = 0; w < nq; ++w) issue_s(w, 0);
+        umma_commit(&kv_empty[0]);
       }
-      if (ok && nt > 0) ok = issue_pv(nt - 1);
+      // V(t) is load 2t+1 and K(t+1) load 2t+2 of the ring: stage n % NS, phase (n / NS) & 1
+      uint32_t vs = 1, ks = 2, vpar = 0, kpar = 0;
+      for (int t = 0; t < nt && ok; ++t) {
+        const bool more = t + 1 < nt;
+        ok = mbar_wait(&kv_full[vs], vpar, err) && (!more || mbar_wait(&kv_full[ks], kpar, err));
+        if (!ok) break;
+        for (int w = 0; w < nq; ++w) {
+          if (!mbar_wait(&p_full[w], static_cast<uint32_t>(t & 1), err)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk)
+            umma_bf16_ts(tmem + o_col(w), tmem + s_col(w) + kk * 8, dV + ((vs * TILE + kk * 2048) >> 4), idPV,
+                         (t > 0 || kk > 0) ? 1u : 0u);
+          if (more)
+            issue_s(w, ks);
+          else
+            umma_commit(&pv_done[w]);
+        }
+        if (!ok) break;
+        umma_commit(&kv_empty[vs]);
+        if (more) umma_commit(&kv_empty[ks]);
+        vs += 2;
+        if (vs >= NS) { vs -= NS; vpar ^= 1u; }
+        ks += 2;
+        if (ks >= NS) { ks -= NS; kpar ^= 1u; }
+      }
       if (!ok) abort_flag = 1;
       umma_commit(drain);
       mbar_wait(drain, 0, err);
     }
   } else {
-    // softmax warps
+    regs_inc<REGS_HIGH>();
+    // ---------------------------------------------------------------- softmax
+    const int w = (warp >> 2) - 1;          // 0: tile A (warps 4..7), 1: tile B (warps 8..11)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const float sc = p.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;
-    SegCursor cur;
-    bool ok = true;
-    for (int t = 0; t < nt; ++t) {
-      const int sb = t & 1;
-      const int valid = min(BKV, g.seg[cur.seg].len - cur.start);
-      cur.next(g);
-      if (abort_flag || !mbar_wait(&s_full[sb], static_cast<uint32_t>((t >> 1) & 1), err)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t s[128];
-      {
-        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
-        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-        uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
-        uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
-        const uint32_t base = tmem + lane_off + static_cast<uint32_t>(sb * 128);
-        tmem_ld32(base + 0, s0);
-        tmem_ld32(base + 32, s1);
-        tmem_ld32(base + 64, s2);
-        tmem_ld32(base + 96, s3);
-        tmem_ld_wait();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-
-      // scores in the log2 domain (rounded once), row max and sum with 8
-      // independent partial accumulators (one warp per scheduler: latency is
-      // hidden by ILP, not by other warps)
-      float x[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = PRESCALED ? __uint_as_float(s[c]) : __fmul_rn(__uint_as_float(s[c]), sc);
-      float mx8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-      if (valid == BKV) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], c < valid ? x[c] : -INFINITY);
-      }
-      const float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const bool need = m_tile > m_ref + 8.0f;
-      const float m_new = need ? m_tile : m_ref;
-      const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
-      float rs8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
-      uint32_t pk[64];
-      if (valid == BKV) {
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = fast_exp2(x[c] - m_new);
-          const float p1 = fast_exp2(x[c + 1] - m_new);
-          rs8[(c >> 1) & 7] += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = c < valid ? fast_exp2(x[c] - m_new) : 0.f;
-          const float p1 = c + 1 < valid ? fast_exp2(x[c + 1] - m_new) : 0.f;
-          rs8[(c >> 1) & 7] += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-        }
-      }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      l = l * alpha + rs;
-      m_ref = m_new;
-
-      if (t >= 1) {
-        if (!mbar_wait(pv_done, static_cast<uint32_t>((t - 1) & 1), err)) { ok = false; break; }
+    const uint32_t s_base = tmem + lane_off + s_col(w);
+    const uint32_t o_base = tmem + lane_off + o_col(w);
+    if (w < nq) {
+      float m_ref = -INFINITY, l = 0.f;
+      SegCursor cur;
+      bool ok = true;
+      for (int t = 0; t < nt; ++t) {
+        const int valid = min(BKV, g.seg[cur.seg].len - cur.start);
+        cur.next(g);
+        if (abort_flag || !mbar_wait(&s_full[w], static_cast<uint32_t>(t & 1), err)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+        float s[128];
+        {
+          uint32_t u[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(s_base + c * 32, u[c]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(u[c][i]);
+        }
+        if (!PRESCALED) {
+          const float2 sc = make_float2(p.scale_log2, p.scale_log2);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const float2 v = __fmul2_rn(make_float2(s[2 * i], s[2 * i + 1]), sc);
+            s[2 * i] = v.x;
+            s[2 * i + 1] = v.y;
+          }
+        }
+        uint32_t P[64];
+        float alpha;
+        bool need;
+        const float rs = valid == BKV ? softmax_tile<false, EMU>(s, P, valid, m_ref, alpha, need)
+                                      : softmax_tile<true, EMU>(s, P, valid, m_ref, alpha, need);
+        if (t >= 1 && __any_sync(0xffffffffu, need)) {
+          // O is stable: the commit that signalled S(t) also covers PV(t-1), issued before it
 #pragma unroll 1
           for (int c4 = 0; c4 < 4; ++c4) {
             uint32_t o[32];
-            const uint32_t addr = tmem + lane_off + O_COL + c4 * 32;
-            tmem_ld32(addr, o);
+            tmem_ld32(o_base + c4 * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(addr, o);
+            tmem_st32(o_base + c4 * 32, o);
           }
-          tmem_st_wait();
         }
+        tmem_st32(s_base, *reinterpret_cast<uint32_t(*)[32]>(P));
+        tmem_st32(s_base + 32, *reinterpret_cast<uint32_t(*)[32]>(P + 32));
+        tmem_st_wait();
+        l = l * alpha + rs;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[w]);
       }
-      // P row r, swizzled K-major: 16-byte chunk c of 64-key atom a at
-      // a*HALF + r*128 + ((c ^ (r & 7)) * 16)
-      uint8_t* prow = sP + r * 128;
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int atom = ch >> 3, c = ch & 7;
-        uint4 w = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(prow + atom * HALF + ((c ^ (r & 7)) << 4)) = w;
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    if (!ok) abort_flag = 1;
-    if (ok && nt > 0 && mbar_wait(pv_done, static_cast<uint32_t>((nt - 1) & 1), err)) {
-      tc_fence_after();
-      const float inv = 1.0f / l;
-      const bool store = q0 + r < p.Tq;
-      const long long orow_idx = static_cast<long long>(g.out_row0) + q0 + r;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + orow_idx * p.out_ld + static_cast<long long>(h) * 128;
-      float* orow32 = p.out32 ? p.out32 + orow_idx * p.out_ld + static_cast<long long>(h) * 128 : nullptr;
+      if (!ok) abort_flag = 1;
+      if (ok && nt > 0 && mbar_wait(&pv_done[w], 0, err)) {   // committed once, after the last PV
+        tc_fence_after();
+        const float inv = 1.0f / l;
+        const int qrow = q0 + w * BQ + r;
+        const bool store = qrow < p.Tq;
+        const long long orow_idx = static_cast<long long>(g.out_row0) + qrow;
+        __nv_bfloat16* orow =
+            reinterpret_cast<__nv_bfloat16*>(p.out) + orow_idx * p.out_ld + static_cast<long long>(h) * 128;
+        float* orow32 = p.out32 ? p.out32 + orow_idx * p.out_ld + static_cast<long long>(h) * 128 : nullptr;
 #pragma unroll 1
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_off + O_COL + c4 * 32, o);
-        tmem_ld_wait();
-        if (store) {
-          float v[32];
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t o[32];
+          tmem_ld32(o_base + c4 * 32, o);
+          tmem_ld_wait();
+          if (store) {
+            float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o[i]) * inv;
-          uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o[i]) * inv;
+            uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 w;
-            w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
-            w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
-            w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
-            w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
-            dst[i] = w;
-          }
-          if (orow32) {
-            float4* d32 = reinterpret_cast<float4*>(orow32 + c4 * 32);
+            for (int i = 0; i < 4; ++i) {
+              uint4 wv;
+              wv.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+              wv.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+              wv.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+              wv.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+              dst[i] = wv;
+            }
+            if (orow32) {
+              float4* d32 = reinterpret_cast<float4*>(orow32 + c4 * 32);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) d32[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+              for (int i = 0; i < 8; ++i) d32[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
           }
         }
       }
@@ -335,13 +404,45 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
   }
 }
 
-}  // namespace
-
-cudaError_t launch_attn_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st) {
-  auto kern = p.q_prescaled ? k_attn_tc<true> : k_attn_tc<false>;
+template <bool PRESCALED, int EMU>
+cudaError_t launch_variant(const AttnMaps& maps, const AttnParams& p, cudaStream_t st) {
+  auto kern = k_attn_tc<PRESCALED, EMU>;
+  // The register split above assumes the kernel launches with exactly
+  // LAUNCH_REGS registers a thread; with fewer, setmaxnreg.inc could not be
+  // satisfied, so refuse to launch.
+  static const int regs = [&] {
+    cudaFuncAttributes fa{};
+    return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1;
+  }();
+  if (regs != LAUNCH_REGS) {
+    std::fprintf(stderr, "k_attn_tc: compiled with %d registers a thread, the register split needs %d\n", regs,
+                 LAUNCH_REGS);
+    return cudaErrorInvalidConfiguration;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
-  dim3 grid((p.Tq + BQ - 1) / BQ, p.H, p.ngroups);
-  kern<<<grid, 192, SMEM, st>>>(maps, p);
+  const int qtiles = (p.Tq + BQ - 1) / BQ;
+  dim3 grid((qtiles + 1) / 2, p.H, p.ngroups);
+  kern<<<grid, THREADS, SMEM, st>>>(maps, p);
   return cudaGetLastError();
+}
+
+int emu_setting() {
+  static const int v = [] {
+    const char* e = std::getenv("LA_ATTN_EMU");
+    return e ? std::atoi(e) : 0;
+  }();
+  return v;
+}
+
+}  // namespace
+
+cudaError_t launch_attention_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st) {
+  const bool pre = p.q_prescaled != 0;
+  switch (emu_setting()) {
+    case 0: return pre ? launch_variant<true, 0>(maps, p, st) : launch_variant<false, 0>(maps, p, st);
+    case 2: return pre ? launch_variant<true, 2>(maps, p, st) : launch_variant<false, 2>(maps, p, st);
+    case 4: return pre ? launch_variant<true, 4>(maps, p, st) : launch_variant<false, 4>(maps, p, st);
+    default: return pre ? launch_variant<true, 3>(maps, p, st) : launch_variant<false, 3>(maps, p, st);
+  }
 }

@@ -19,10 +19,9 @@ struct AttnMaps {
   CUtensorMap k[LA_MAX_SEG];
   CUtensorMap v[LA_MAX_SEG];
 };
-cudaError_t launch_attn_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);    // 1 query tile / CTA
-cudaError_t launch_attn_tc2(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);   // 2 query tiles / CTA
-cudaError_t launch_attn_tc3(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);   // 2 tiles, scores in regs
-// The attention launcher used by the library (LA_ATTN_VERSION=1 / 2 in the environment selects an older kernel).
+// Block-causal attention over the segments of each group (two 128-query tiles
+// per CTA).  LA_ATTN_EMU=k in the environment (k in {0, 2, 3, 4}; default 0)
+// computes k of every 8 exponential pairs of full key tiles on the FMA pipe.
 cudaError_t launch_attention_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);
 
 // ---- SIMT fp32 -----------------------------------------------------------------------

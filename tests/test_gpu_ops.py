@@ -165,3 +165,31 @@ def test_euler_standalone_matches_oracle():
     want = np.concatenate([euler_step(x0[g * 4680:(g + 1) * 4680], v[g * 4680:(g + 1) * 4680], ts[g], ts[g + 1])
                            for g in range(G)])
     assert_close(_np(x), want, DTYPE_FP32, "euler")
+
+
+@pytest.mark.parametrize("emu", [3, 4])
+def test_attention_with_polynomial_exp2_share_matches_oracle(emu, tmp_path):
+    """LA_ATTN_EMU=k computes k of every 8 exponential pairs of full key tiles
+    with the FMA-pipe polynomial; the setting is read once per process, so the
+    case runs in a child process and the parity check runs here."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    out = tmp_path / "attn.npz"
+    code = (
+        "import sys, numpy as np\n"
+        f"sys.path[:0] = [{here!r}, {os.path.dirname(here)!r}]\n"
+        "import test_gpu_ops as t\n"
+        "from workloads import DTYPE_BF16\n"
+        "q, sink, blocks, b = t._attn_case(11, 2, 128, 130, 300, 2)\n"
+        "got, got32 = t._run_op_attention(q, sink, blocks, DTYPE_BF16)\n"
+        f"np.savez({str(out)!r}, got=got, got32=got32)\n")
+    env = dict(os.environ, LA_ATTN_EMU=str(emu))
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    res = np.load(out)
+    q, sink, blocks, b = _attn_case(11, 2, 128, 130, 300, 2)
+    want = block_causal_attention(q, blocks, sink, qblock=b, window=2).reshape(q.shape[0], 2 * 128)
+    assert_close(res["got32"], want, DTYPE_BF16, f"attention fp32 result, polynomial share {emu}/8")
+    np.testing.assert_array_equal(res["got"], bf16_round(res["got32"].astype(np.float32)))

@@ -1,7 +1,7 @@
 """Host-side checks of the arithmetic the attention kernel uses in place of ex2.
 
 The softmax of the tcgen05 attention kernel computes part of its
-exponentials 2^x on the FMA pipe (exp2_poly2 in csrc/attn_tc3.cu): clamp at
+exponentials 2^x on the FMA pipe (exp2_poly2 in csrc/attn_tc.cu): clamp at
 -125, split x = j + f with j = round(x) through the 1.5 * 2^23 shifter, a
 degree-3 polynomial p(f) with p(0) = 1 for 2^f on [-1/2, 1/2], and j added to
 the exponent field.  These tests replay those steps in numpy float32 with the
@@ -15,7 +15,7 @@ import re
 
 import numpy as np
 
-SRC = os.path.join(os.path.dirname(__file__), "..", "streaming_causal_video_timestep_b200", "csrc", "attn_tc3.cu")
+SRC = os.path.join(os.path.dirname(__file__), "..", "streaming_causal_video_timestep_b200", "csrc", "attn_tc.cu")
 REL_BOUND = 1.02e-4          # the fit's maximum relative error on [-1/2, 1/2]
 BF16_HALF_ULP = 2.0 ** -9    # relative rounding bound of bf16 (8 significant bits)
 
