@@ -1,6 +1,6 @@
 """Benchmark of the timestep-forced streaming step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sweep]
 
 A step is one tick of the 4-slot grouped stream in steady state: 4 in-flight
 blocks (one per timestep slot, every window full) through 8 attention
@@ -221,6 +221,13 @@ def run_gpu(args, rank, world, local_rank):
         e = {"launches": n, "ms_avg": round(avg, 4), "ms_per_step": round(tot / args.steps, 3)}
         if kind == "attn":
             e["tflops"] = round(achieved, 1)
+        elif kind == "rope":
+            # sink re-rope of every active slot: read the layer's fp32 un-roped sink K once,
+            # write S bf16 roped copies (the block's RoPE + append is fused into the QKV GEMM)
+            nbytes = F * D * 4 + S * F * D * 2
+            e["gbs"] = round(nbytes / (avg / 1000.0) / 1e9, 1)
+            e["frac_hbm"] = round(e["gbs"] / pk["hbm"], 3)
+            e["bytes_per_launch"] = nbytes
         elif kind in gemm_flops and n >= args.steps * (L if kind in ("qkv_gemm", "out_gemm") else 1):
             e["tflops"] = round(gemm_flops[kind] / (avg / 1000.0) / 1e12, 1)
         kernels[kind] = e
@@ -311,6 +318,84 @@ def cpu_baseline(rows=468, reps=1):
                        f"15,600 keys ({dt:.1f} s), scaled x{4680 / rows:.0f} rows x 4 slots x 8 layers per tick")}
 
 
+def run_sweep(args):
+    """One JSON line per shape-sweep point (two token grids x cache windows 1, 2, 4, 8; one attention
+    sublayer; 4 slots as one grouped launch) and one for the standalone Euler update.  Not the
+    headline metric: each point reports the attention kernel's TFLOP/s and the sink re-rope's GB/s
+    against the measured peaks."""
+    import torch
+    from streaming_causal_video_timestep_b200 import LaStream, op_euler
+    from workloads import SWEEP
+
+    torch.cuda.set_device(0)
+    pk = _peaks()
+    bf = torch.bfloat16
+    for wl in SWEEP:
+        cfg = wl.cfg
+        T, C, D, F, H, d = cfg.block_tokens, cfg.latent_ch, cfg.hidden, cfg.frame_tokens, cfg.heads, cfg.head_dim
+        S, nw, L = cfg.num_steps, cfg.window_blocks, cfg.num_layers
+        g = torch.Generator(device="cuda")
+        g.manual_seed(wl.seed)
+        rnd = lambda shape, std: (torch.randn(shape, generator=g, device="cuda") * std).to(bf)
+        weights = dict(w_qkv=[rnd((3 * D, D), wl.w_std) for _ in range(L)],
+                       w_out=[rnd((D, D), wl.w_std) for _ in range(L)],
+                       w_in=rnd((D, C), 1.0 / C ** 0.5), w_head=rnd((C, D), wl.head_std))
+        s = LaStream(cfg, weights)
+        s.set_sink(torch.randn((F, C), generator=g, device="cuda"))
+        xs = [torch.randn((T, C), generator=g, device="cuda") for _ in range(2)]
+        x_out = torch.empty((T, C), device="cuda")
+        for k in range((S - 1) + nw + 1 + args.warmup):
+            s.step(xs[k % 2], x_out)
+        s.synchronize()
+        s.profile(True)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for k in range(args.steps):
+            s.step(xs[k % 2], x_out)
+        ev1.record()
+        s.synchronize()
+        torch.cuda.synchronize()
+        ms = ev0.elapsed_time(ev1) / args.steps
+        n_a, t_a = s.profile_read("attn")
+        n_r, t_r = s.profile_read("rope")
+        s.profile(False)
+        attn_flops = S * _attn_flops_per_slot(T, F, nw, H, d)
+        attn_tf = attn_flops / (t_a / n_a / 1000.0) / 1e12
+        rope_bytes = F * D * 4 + S * F * D * 2
+        rope_gbs = rope_bytes / (t_r / n_r / 1000.0) / 1e9
+        print(json.dumps({"sweep": wl.name, "grid": f"{cfg.grid_h}x{cfg.grid_w}", "window_blocks": nw,
+                          "keys_per_query": F + nw * T + T, "ms_per_tick": round(ms, 3),
+                          "latent_frames_per_s": round(cfg.frames_per_block / (ms / 1000.0), 2),
+                          "attn": {"tflops": round(attn_tf, 1), "flops_per_launch": attn_flops,
+                                   "frac_sustained": round(attn_tf / pk["tflops_sust"], 3),
+                                   "frac_burst": round(attn_tf / pk["tflops"], 3),
+                                   "frac_spec_2250": round(attn_tf / 2250.0, 3)},
+                          "sink_rerope": {"gbs": round(rope_gbs, 1), "bytes_per_launch": rope_bytes,
+                                          "frac_hbm": round(rope_gbs / pk["hbm"], 3)},
+                          "peaks": pk["src"]}), flush=True)
+        s.close()
+        del s, weights
+        torch.cuda.empty_cache()
+    rows, C, G = 1 << 20, 64, 4   # 256 MB per tensor, larger than L2
+    x = torch.randn(rows, C, device="cuda")
+    v = torch.randn(rows, C, device="cuda")
+    for _ in range(args.warmup):
+        op_euler(x, v, [-0.25] * G, rows // G)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        op_euler(x, v, [-0.25] * G, rows // G)
+    ev1.record()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    gbs = 3 * rows * C * 4 / (ms / 1000.0) / 1e9
+    print(json.dumps({"sweep": "euler_standalone", "shape": f"{rows}x{C} fp32, {G} timestep groups",
+                      "ms": round(ms, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 3),
+                      "note": "in the stream the Euler update is fused into the velocity-head GEMM epilogue"}),
+          flush=True)
+
+
 def run_reference(args):
     smp = OracleSample(rows=234)
     for _ in range(args.warmup):
@@ -338,6 +423,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="shape sweep lines instead of the headline line")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -348,6 +434,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args)
         return
 
     if world > 1:

@@ -85,52 +85,110 @@ __global__ void k_rope_ttab(const __grid_constant__ PassDesc pd, int fpb, int pt
 }
 
 // Rolling RoPE + ring append from an fp32 [q | k | v] projection (fp32
-// streams), and the per-block re-rope of the fp32 un-roped sink K for every
-// active buffer (both streams).  Outputs are rounded once to TO.
+// streams; bf16 streams do this in the QKV GEMM epilogue).  Outputs are
+// rounded once to TO.
 template <typename TO>
 __global__ void __launch_bounds__(256) k_rope_append(const __grid_constant__ PassDesc pd,
-                                                     const __grid_constant__ RopeArgs a, long long n_main,
-                                                     long long n_sink) {
+                                                     const __grid_constant__ RopeArgs a, long long n_main) {
   const int chunks = a.d / 8;
   const float* qkv = reinterpret_cast<const float*>(a.qkv);
-  const long long total = n_main + n_sink;
-  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n_main;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    if (idx < n_main) {
-      long long rest = idx;
-      const int ch = static_cast<int>(rest % chunks); rest /= chunks;
-      const int h = static_cast<int>(rest % a.H); rest /= a.H;
-      const int part = static_cast<int>(rest % 3); rest /= 3;
-      const int n = static_cast<int>(rest % a.T); rest /= a.T;
-      const int buf = pd.active_buf[rest];
-      const long long row = static_cast<long long>(buf) * a.T + n;
-      float v[8];
-      Vec8<float>::load(qkv + row * 3 * a.D + part * a.D + h * a.d + ch * 8, v);
-      if (part < 2) {
-        const int f = n / a.F, rem = n % a.F;
-        rotate8(v, ch, buf, f, rem / a.grid_w, rem % a.grid_w, a);
-      }
-      TO* dst;
-      const long long tok = static_cast<long long>(n) * a.d + ch * 8;
-      if (part == 0) {
-        dst = reinterpret_cast<TO*>(a.q_rope) + (static_cast<long long>(buf) * a.H + h) * a.T * a.d + tok;
-      } else {
-        const long long slice = a.ring_slice0 + static_cast<long long>(pd.slot[buf]) * a.E + pd.write_entry[buf];
-        TO* base = reinterpret_cast<TO*>(part == 1 ? a.ring_k : a.ring_v);
-        dst = base + (slice * a.H + h) * a.T * a.d + tok;
-      }
-      Vec8<TO>::store(dst, v);
+    long long rest = idx;
+    const int ch = static_cast<int>(rest % chunks); rest /= chunks;
+    const int h = static_cast<int>(rest % a.H); rest /= a.H;
+    const int part = static_cast<int>(rest % 3); rest /= 3;
+    const int n = static_cast<int>(rest % a.T); rest /= a.T;
+    const int buf = pd.active_buf[rest];
+    const long long row = static_cast<long long>(buf) * a.T + n;
+    float v[8];
+    Vec8<float>::load(qkv + row * 3 * a.D + part * a.D + h * a.d + ch * 8, v);
+    if (part < 2) {
+      const int f = n / a.F, rem = n % a.F;
+      rotate8(v, ch, buf, f, rem / a.grid_w, rem % a.grid_w, a);
+    }
+    TO* dst;
+    const long long tok = static_cast<long long>(n) * a.d + ch * 8;
+    if (part == 0) {
+      dst = reinterpret_cast<TO*>(a.q_rope) + (static_cast<long long>(buf) * a.H + h) * a.T * a.d + tok;
     } else {
-      long long rest = idx - n_main;
-      const int ch = static_cast<int>(rest % chunks); rest /= chunks;
-      const int m = static_cast<int>(rest % a.F); rest /= a.F;
-      const int h = static_cast<int>(rest % a.H); rest /= a.H;
-      const int buf = pd.active_buf[rest];
-      const long long off = (static_cast<long long>(h) * a.F + m) * a.d + ch * 8;
-      float v[8];
-      Vec8<float>::load(reinterpret_cast<const float*>(a.sink_k) + off, v);
-      rotate8(v, ch, buf, a.fpb, m / a.grid_w, m % a.grid_w, a);
-      Vec8<TO>::store(reinterpret_cast<TO*>(a.sink_k_rope) + static_cast<long long>(buf) * a.H * a.F * a.d + off, v);
+      const long long slice = a.ring_slice0 + static_cast<long long>(pd.slot[buf]) * a.E + pd.write_entry[buf];
+      TO* base = reinterpret_cast<TO*>(part == 1 ? a.ring_k : a.ring_v);
+      dst = base + (slice * a.H + h) * a.T * a.d + tok;
+    }
+    Vec8<TO>::store(dst, v);
+  }
+}
+
+// Per-block re-rope of the fp32 un-roped sink K for every active buffer.  The
+// spatial rotation factors depend only on (token, pair) and the temporal ones
+// only on (buffer, pair), so one thread takes one (token, 8-element chunk) for
+// SINK_HEADS heads: it loads their chunks and the factors once and writes each
+// chunk roped, rounded once to TO, for every active buffer.  Reads F*H*d*4
+// bytes once and writes nactive*F*H*d*sizeof(TO).
+constexpr int SINK_HEADS = 8;
+
+template <typename TO>
+__global__ void __launch_bounds__(256) k_sink_rerope(const __grid_constant__ PassDesc pd,
+                                                     const __grid_constant__ RopeArgs a, long long n) {
+  const int chunks = a.d / 8;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int ch = static_cast<int>(idx % chunks);
+    const long long rest = idx / chunks;
+    const int m = static_cast<int>(rest % a.F);
+    const int h0 = static_cast<int>(rest / a.F) * SINK_HEADS;
+    const int nh = min(SINK_HEADS, a.H - h0);
+    float v[SINK_HEADS][8];
+#pragma unroll
+    for (int k = 0; k < SINK_HEADS; ++k)
+      if (k < nh)
+        Vec8<float>::load(reinterpret_cast<const float*>(a.sink_k) +
+                              (static_cast<long long>(h0 + k) * a.F + m) * a.d + ch * 8, v[k]);
+    const int rr = m / a.grid_w, cc = m % a.grid_w;
+    float c[4], sn[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = 4 * ch + jj;
+      if (j >= a.pt && j < a.pt + a.ph) {
+        c[jj] = a.rcos[rr * a.ph + (j - a.pt)];
+        sn[jj] = a.rsin[rr * a.ph + (j - a.pt)];
+      } else if (j >= a.pt) {
+        c[jj] = a.ccos[cc * a.pw + (j - a.pt - a.ph)];
+        sn[jj] = a.csin[cc * a.pw + (j - a.pt - a.ph)];
+      } else {
+        c[jj] = 1.f;
+        sn[jj] = 0.f;
+      }
+    }
+    for (int ai = 0; ai < pd.nactive; ++ai) {
+      const int buf = pd.active_buf[ai];
+      float cb[4], sb[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int j = 4 * ch + jj;
+        if (j < a.pt) {
+          const int t = (buf * LA_TROWS + a.fpb) * LA_MAX_PT + j;
+          cb[jj] = a.tcos[t];
+          sb[jj] = a.tsin[t];
+        } else {
+          cb[jj] = c[jj];
+          sb[jj] = sn[jj];
+        }
+      }
+      TO* out = reinterpret_cast<TO*>(a.sink_k_rope) + static_cast<long long>(buf) * a.H * a.F * a.d;
+#pragma unroll
+      for (int k = 0; k < SINK_HEADS; ++k) {
+        if (k >= nh) break;
+        float w[8];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float x0 = v[k][2 * jj], x1 = v[k][2 * jj + 1];
+          w[2 * jj] = x0 * cb[jj] - x1 * sb[jj];
+          w[2 * jj + 1] = x0 * sb[jj] + x1 * cb[jj];
+        }
+        Vec8<TO>::store(out + (static_cast<long long>(h0 + k) * a.F + m) * a.d + ch * 8, w);
+      }
     }
   }
 }
@@ -187,26 +245,30 @@ __global__ void k_cvt_bf16(const float* __restrict__ x, __nv_bfloat16* __restric
 struct EulerArgs {
   float dt[LA_MAX_STEPS];
   int active[LA_MAX_STEPS];
+  long long start[LA_MAX_STEPS];   // first float4 index of group g (groups past the last start at n4)
 };
 
-// x += dt * v, float4 vectors; C % 4 == 0.
+// x += dt[g] * v over float4 vectors, g = the timestep group of the row; C % 4 == 0.
+// The group is found by comparing the index against the group starts (no division).
 __global__ void __launch_bounds__(256) k_euler(float* __restrict__ x, const float* __restrict__ v, long long n4,
-                                               long long C4, long long rows_per_group,
                                                const __grid_constant__ EulerArgs e, float* __restrict__ vtap) {
   float4* x4 = reinterpret_cast<float4*>(x);
   const float4* v4 = reinterpret_cast<const float4*>(v);
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int g = static_cast<int>((i / C4) / rows_per_group);
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+#pragma unroll 4
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
+    int g = 0;
+#pragma unroll
+    for (int k = 1; k < LA_MAX_STEPS; ++k) g += i >= e.start[k] ? 1 : 0;
     if (!e.active[g]) continue;
     const float dt = e.dt[g];
-    const float4 vv = v4[i];
-    float4 xx = x4[i];
-    xx.x += dt * vv.x;
-    xx.y += dt * vv.y;
-    xx.z += dt * vv.z;
-    xx.w += dt * vv.w;
-    x4[i] = xx;
+    const float4 vv = __ldcs(v4 + i);
+    float4 xx = __ldcs(x4 + i);
+    xx.x = __fmaf_rn(dt, vv.x, xx.x);
+    xx.y = __fmaf_rn(dt, vv.y, xx.y);
+    xx.z = __fmaf_rn(dt, vv.z, xx.z);
+    xx.w = __fmaf_rn(dt, vv.w, xx.w);
+    __stcs(x4 + i, xx);
     if (vtap) reinterpret_cast<float4*>(vtap)[i] = vv;
   }
 }
@@ -269,17 +331,25 @@ cudaError_t launch_rope_ttab(const PassDesc& pd, int fpb, int pt, const double* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs& a, bool main_part,
-                               cudaStream_t st) {
-  const long long chunks = a.d / 8;
-  const long long n_main = main_part ? static_cast<long long>(pd.nactive) * a.T * 3 * a.H * chunks : 0;
-  const long long n_sink = a.sink_k ? static_cast<long long>(pd.nactive) * a.F * a.H * chunks : 0;
-  if (n_main + n_sink == 0) return cudaSuccess;
-  const int grid = grid_for(n_main + n_sink);
+cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs& a, cudaStream_t st) {
+  const long long n_main = static_cast<long long>(pd.nactive) * a.T * 3 * a.H * (a.d / 8);
+  if (n_main == 0) return cudaSuccess;
+  const int grid = grid_for(n_main);
   if (bf16_out)
-    k_rope_append<__nv_bfloat16><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
+    k_rope_append<__nv_bfloat16><<<grid, 256, 0, st>>>(pd, a, n_main);
   else
-    k_rope_append<float><<<grid, 256, 0, st>>>(pd, a, n_main, n_sink);
+    k_rope_append<float><<<grid, 256, 0, st>>>(pd, a, n_main);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sink_rerope(int bf16_out, const PassDesc& pd, const RopeArgs& a, cudaStream_t st) {
+  if (!a.sink_k || pd.nactive == 0) return cudaSuccess;
+  const long long n = static_cast<long long>(a.F) * ((a.H + SINK_HEADS - 1) / SINK_HEADS) * (a.d / 8);
+  const int grid = grid_for(n);
+  if (bf16_out)
+    k_sink_rerope<__nv_bfloat16><<<grid, 256, 0, st>>>(pd, a, n);
+  else
+    k_sink_rerope<float><<<grid, 256, 0, st>>>(pd, a, n);
   return cudaGetLastError();
 }
 
@@ -314,12 +384,14 @@ cudaError_t launch_cvt_bf16(const float* x, void* xb, long long n, cudaStream_t 
 cudaError_t launch_euler(float* x, const float* v, long long rows, long long C, int rows_per_group, const float* dt,
                          const int* active, float* vtap, cudaStream_t st) {
   EulerArgs e;
+  const long long n4 = rows * C / 4;
   for (int i = 0; i < LA_MAX_STEPS; ++i) {
     e.dt[i] = dt ? dt[i] : 0.f;
     e.active[i] = active ? active[i] : 1;
+    const long long start = static_cast<long long>(i) * rows_per_group * (C / 4);
+    e.start[i] = start < n4 ? start : n4;
   }
-  const long long n4 = rows * C / 4;
-  k_euler<<<grid_for(n4), 256, 0, st>>>(x, v, n4, C / 4, rows_per_group, e, vtap);
+  k_euler<<<grid_for(n4), 256, 0, st>>>(x, v, n4, e, vtap);
   return cudaGetLastError();
 }
 

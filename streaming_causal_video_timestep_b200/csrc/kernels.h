@@ -49,10 +49,13 @@ struct RopeArgs {
   const void* sink_k;                          // fp32 un-roped [H][F][d] of this layer (NULL: no sink part)
   void* sink_k_rope;                           // [nbuf][H][F][d]
 };
-// Outputs are bf16 (bf16_out) or fp32.  main_part: also rope/append the block
-// from qkv (fp32 streams; bf16 streams do that in the QKV GEMM epilogue).
-cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs& a, bool main_part,
-                               cudaStream_t st);
+// Rolling RoPE + ring append of every active buffer's block from the fp32 qkv
+// (fp32 streams; bf16 streams do it in the QKV GEMM epilogue).  Outputs are
+// bf16 (bf16_out) or fp32.
+cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs& a, cudaStream_t st);
+// Re-rope of the layer's fp32 un-roped sink K at every active buffer's sink
+// position (a.sink_k -> a.sink_k_rope[buf]).
+cudaError_t launch_sink_rerope(int bf16_out, const PassDesc& pd, const RopeArgs& a, cudaStream_t st);
 
 // Sink pass: split the fp32 qkv [F, 3D] into the layer's fp32 un-roped K, its
 // V, and roped q / k (temporal row 0 of buffer 0 of the table); q is

@@ -462,15 +462,14 @@ int run_pass(la_stream* s, const PassDesc& pd) {
            })) != LA_OK)
         return r;
       // per-block re-rope of the sink K (fp32 -> bf16, once per active buffer)
-      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(1, pd, ra, false, s->st); })) != LA_OK)
-        return r;
+      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_sink_rerope(1, pd, ra, s->st); })) != LA_OK) return r;
     } else {
       GemmEpiParams eq = epi(EPI_STORE, s->qkv, nullptr, 3LL * D);
       if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_hop, &s->tm_wqkv[l], s->hn32, s->w_qkv[l], eq, rows, 3 * D, D)) !=
           LA_OK)
         return r;
-      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(0, pd, ra, true, s->st); })) != LA_OK)
-        return r;
+      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(0, pd, ra, s->st); })) != LA_OK) return r;
+      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_sink_rerope(0, pd, ra, s->st); })) != LA_OK) return r;
     }
     // block-causal attention: [sink | window oldest first | self]
     for (int ai = 0; ai < pd.nactive; ++ai) {
