@@ -44,6 +44,22 @@ WORKLOAD = dict(
 ATTN_DRAM_BYTES_PER_SLOT = 420.8e6
 
 
+def max_over_ranks(x, device):
+    """The largest of every rank's x (the job's time is its slowest rank's); x itself on one rank."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(frames_per_tick, ticks, world, seconds):
+    """Whole-job latent frames/s: every rank runs `ticks` ticks of its own stream (weak scaling)."""
+    return frames_per_tick * ticks * world / seconds
+
+
 def _attn_flops_per_slot(T, F, nw, H, d):
     nk = F + nw * T + T
     return 4.0 * T * nk * d * H
@@ -140,10 +156,19 @@ def run_gpu(args, rank, world, local_rank):
     x_out = torch.empty((T, C), device="cuda")
     fill = (S - 1) + nw + 1          # every slot active with a full window from here on
     k = 0
+    ph = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ph[0].record()
     for _ in range(fill + args.warmup):
-        s.step(xs[k % 4], x_out)
+        fin = s.step(xs[k % 4], x_out)
         k += 1
+        if k == S:                   # block 0 leaves the last slot at tick S - 1
+            ph[1].record()
+            assert fin == 0
+        if k == fill:
+            ph[2].record()
     s.synchronize()
+    torch.cuda.synchronize()
+    first_block_ms, fill_ms = ph[0].elapsed_time(ph[1]), ph[0].elapsed_time(ph[2])
     st = s.index_state()
     per = 8 + 3 * cfg.ring_entries
     assert all(st[4 + i * per] >= nw for i in range(S)), "not in steady state"
@@ -174,10 +199,8 @@ def run_gpu(args, rank, world, local_rank):
                                                      "other")}
     s.profile(False)
     clk = clocks.stop()
+    ms = max_over_ranks(ms, "cuda")
     if dist:
-        t = torch.tensor([ms], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
         tdist.barrier()
 
     # end to end through the public host-buffer call: H2D of the new block and
@@ -196,15 +219,20 @@ def run_gpu(args, rank, world, local_rank):
         s.synchronize()
         assert fin >= 0
     e2e_s = time.perf_counter() - t0
-    if dist:
-        t = torch.tensor([e2e_s], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks(e2e_s, "cuda")
+    # drain: S - 1 ticks without new blocks finish the blocks still in flight
+    dr = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    dr[0].record()
+    for _ in range(S - 1):
+        assert s.step(None, x_out) >= 0
+    dr[1].record()
+    torch.cuda.synchronize()
+    drain_ms = dr[0].elapsed_time(dr[1])
     s.close()
 
     frames_per_tick = cfg.frames_per_block
-    value = frames_per_tick * args.steps * world / (ms / 1000.0)
-    e2e_value = frames_per_tick * e2e_steps * world / e2e_s
+    value = job_throughput(frames_per_tick, args.steps, world, ms / 1000.0)
+    e2e_value = job_throughput(frames_per_tick, e2e_steps, world, e2e_s)
     pk = _peaks()
     n_attn, ms_attn = kinds["attn"]
     attn_flops_launch = S * _attn_flops_per_slot(T, F, nw, H, d)
@@ -244,6 +272,9 @@ def run_gpu(args, rank, world, local_rank):
                      "algorithmic_flops_per_launch": attn_flops_launch},
         "kernels": kernels,
         "gpu_launches": int(launches),
+        "phases": {"first_finished_block_ms": round(first_block_ms, 3), "fill_ticks": fill,
+                   "fill_ms": round(fill_ms, 3), "drain_ticks": S - 1, "drain_ms": round(drain_ms, 3),
+                   "note": "rank 0; fill = ticks until every slot is active with a full window (untimed by value)"},
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": T * C * 4,
                 "d2h_bytes_per_step": T * C * 4, "steps": e2e_steps},
