@@ -186,3 +186,19 @@ def test_state_errors():
         seq.step(None, x_out)
     assert e.value.code == -1
     seq.close()
+
+
+@pytest.mark.parametrize("rolling,sink_mode", [(0, SINK_AAS), (0, SINK_FIXED), (1, SINK_FIXED)])
+def test_tiny_fp32_ablations_match_oracle(rolling, sink_mode):
+    """Ablation schedules on the same kernels: Rolling RoPE off (the sink keeps the
+    temporal position of block 0, -3) and / or AAS off (the reference sink for the
+    whole stream); integer state bit-exact and every op within 1e-5 every tick."""
+    cfg = TINY.cfg.replace(rolling_rope=rolling, sink_mode=sink_mode)
+    _run_teacher_forced(Workload(f"tiny-rolling{rolling}-sink{sink_mode}", cfg, TINY.seed, TINY.num_blocks,
+                                 TINY.w_std, TINY.head_std))
+
+
+def test_small_bf16_rolling_rope_off_teacher_forced():
+    cfg = SMALL_BF16.cfg.replace(rolling_rope=0)
+    _run_teacher_forced(Workload("small-bf16-rolling0", cfg, SMALL_BF16.seed, 6, SMALL_BF16.w_std,
+                                 SMALL_BF16.head_std))
