@@ -235,6 +235,21 @@ int la_profile_read(la_stream* s, int32_t kind, int64_t* launches, double* total
 /* Kernels launched by this stream since creation. */
 int64_t la_launch_count(const la_stream* s);
 
+/*
+ * Failure-detection check (the pages have no counterpart; it tests the
+ * library's own error path without faulting the GPU).  Launches one CTA on the
+ * current device whose thread waits on an mbarrier phase with a limit of
+ * limit_ns nanoseconds (0 <= limit_ns <= 1e10), as every pipelined kernel of
+ * the library waits.  complete != 0: the phase is completed before the wait;
+ * 0: nothing completes it, the wait gives up after the limit, raises the
+ * device error word and the kernel returns.  Synchronises the device.
+ * *device_error receives the word (0, or LA_DEVERR_WAIT_TIMEOUT = 1).
+ * Returns LA_OK, LA_EDEVICE when the word was raised, LA_EINVAL, LA_ENOMEM
+ * (the 4-byte word could not be allocated) or LA_ECUDA.  The CUDA context
+ * stays usable after LA_EDEVICE.
+ */
+int la_debug_wait_timeout(int64_t limit_ns, int32_t complete, int32_t* device_error);
+
 /* ---- op-level entry points (unit tests, microbenchmarks) ------------------
  * Each enqueues one kernel on cuda_stream (a cudaStream_t, NULL = default).
  * They allocate nothing except where stated.
