@@ -21,12 +21,19 @@ Index-state record (int32), identical to the C-ABI's debug export:
 active_block, write_entry and evicted_block are -1 and sink_tpos, frame_tpos,
 sink_generation_used are 0 for a slot idle this tick; step_index is the slot
 index; n_resident, resident and tags always describe the ring contents.
+
+Clean-cache refresh (the ablation the method removes; papernotes note, 关键设计 2
+and the NFE row of its Table 2; gitcode blog, question 4 table): one cache of
+clean K/V serves every step, so all slots share ring 0 (their records describe
+it); after the last step of block b one more pass runs the stack on the
+finished latent and overwrites block b's entry, tagged (b, num_steps).  Only
+in the sequential schedule.
 """
 from __future__ import annotations
 
 import numpy as np
 
-from workloads import SCHED_PIPELINED, SINK_AAS
+from workloads import CACHE_CLEAN_REFRESH, SCHED_PIPELINED, SINK_AAS
 
 
 def index_state_layout(cfg):
@@ -37,7 +44,10 @@ def index_state_layout(cfg):
 
 class TickScheduler:
     def __init__(self, cfg):
+        if cfg.cache_mode == CACHE_CLEAN_REFRESH and cfg.schedule == SCHED_PIPELINED:
+            raise ValueError("the clean-cache refresh runs in the sequential schedule")
         self.cfg = cfg
+        self.clean = cfg.cache_mode == CACHE_CLEAN_REFRESH
         S, E = cfg.num_steps, cfg.ring_entries
         self.S, self.E = S, E
         self.slots = [-1] * S          # block held by each slot after the last tick
@@ -82,26 +92,37 @@ class TickScheduler:
             return True
         return False
 
+    def ring_of(self, i: int) -> int:
+        """The cache slot i reads and writes: its own, or the one clean cache."""
+        return 0 if self.clean else i
+
     def append(self, i: int, b: int):
-        """Ring append of block b in slot i; returns the slot's record."""
+        """Ring append of block b at step i; returns the slot's record."""
         cfg, E = self.cfg, self.E
+        ring = self.ring_of(i)
         e = b % E
-        evicted = self.tags[i][e][0]
-        self.tags[i][e] = (b, i)
-        resident = self.resident(i)
+        evicted = self.tags[ring][e][0]
+        self.tags[ring][e] = (b, i)
+        resident = self.resident(ring)
         rec = [b, e, evicted, self.sink_tpos(b), cfg.frames_per_block * b,
                self.sink_generation, i, len(resident)]
-        rec = rec + self._pad(resident) + [v for tag in self.tags[i] for v in tag]
+        rec = rec + self._pad(resident) + [v for tag in self.tags[ring] for v in tag]
         self._records[i] = rec
         return rec
 
+    def append_refresh(self, b: int) -> int:
+        """The refresh pass of block b rewrites its entry of the clean cache; returns the entry."""
+        e = b % self.E
+        self.tags[0][e] = (b, self.S)
+        return e
+
     # -- queries ------------------------------------------------------------
-    def resident(self, i):
-        return sorted(t[0] for t in self.tags[i] if t[0] >= 0)
+    def resident(self, ring):
+        return sorted(t[0] for t in self.tags[ring] if t[0] >= 0)
 
     def window_blocks(self, i, b):
-        """Prior blocks block b reads in slot i, oldest first."""
-        return [x for x in self.resident(i) if b - self.cfg.window_blocks <= x < b]
+        """Prior blocks block b reads at step i, oldest first."""
+        return [x for x in self.resident(self.ring_of(i)) if b - self.cfg.window_blocks <= x < b]
 
     def sink_tpos(self, b: int) -> int:
         cfg = self.cfg
@@ -115,9 +136,10 @@ class TickScheduler:
         for i in range(self.S):
             rec = list(self._records[i])
             # ring-content fields always reflect the current ring
-            rec[7] = len(self.resident(i))
-            rec[8:8 + self.E] = self._pad(self.resident(i))
-            rec[8 + self.E:] = [v for tag in self.tags[i] for v in tag]
+            ring = self.ring_of(i)
+            rec[7] = len(self.resident(ring))
+            rec[8:8 + self.E] = self._pad(self.resident(ring))
+            rec[8 + self.E:] = [v for tag in self.tags[ring] for v in tag]
             body += rec
         return np.asarray(head + body, dtype=np.int32)
 

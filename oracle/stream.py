@@ -23,6 +23,15 @@ itself; its un-roped K and its V are kept per layer and shared by all slots).
 Adaptive Attention Sink (papernotes note, 关键设计 3; gitcode blog, question 5):
 once block 0 is finished, frame 0 of its final latent replaces the sink and the
 sink is never replaced again.
+
+Clean-cache refresh (the baseline the pages remove, papernotes note 关键设计 2
+and the "DMD 4-step" row of its Table 2: 4 denoising steps plus 1 clean
+forward refresh, NFE 5; gitcode blog question 4: the cache holds the clean x0's
+K/V, written by one extra forward per block): one cache per layer; every step
+of block b reads the clean K/V of blocks b-window .. b-1 and its own current
+K/V; after the last step the finished latent goes through the stack once more
+(no Euler update) and its K/V replace block b's entry.  Reading: with AAS the
+refresh of block 0 uses the reference sink, and the sink is replaced after it.
 """
 from __future__ import annotations
 
@@ -44,7 +53,7 @@ class OracleStream:
         self.w_in = f64(weights.w_in)
         self.w_head = f64(weights.w_head)
         self.sched = TickScheduler(cfg)
-        self.cache = {}            # (layer, slot, block) -> (k_roped, v, (block, step))
+        self.cache = {}            # (layer, ring, block) -> (k_roped, v, (block, step))
         self.sink_k = None         # per layer, un-roped [F, H, d]
         self.sink_v = None
         self.sink_latent = None
@@ -90,9 +99,16 @@ class OracleStream:
                 self.trace[("sink", l)] = dict(k=k.copy(), v=v.copy(), o=o, h=h.copy())
 
     # -- one step of one block --------------------------------------------------
-    def slot_pass(self, x, b: int, i: int):
+    def slot_pass(self, x, b: int, i: int, refresh: bool = False):
+        """Block b at step i (refresh: the clean-cache refresh of finished block b,
+        which writes its K/V and leaves x unchanged)."""
         c = self.cfg
-        rec = self.sched.append(i, b)
+        ring = self.sched.ring_of(i)
+        if refresh:
+            self.sched.append_refresh(b)
+            rec = None
+        else:
+            rec = self.sched.append(i, b)
         x = np.asarray(x, np.float64)
         h = self.project_in(x)
         pt, ph, pw = block_positions(c, b)
@@ -101,21 +117,25 @@ class OracleStream:
         if tr is not None:
             tr["x_in"] = x.copy()
             tr["h_in"] = h.copy()
-            tr["record"] = list(rec)
+            tr["record"] = list(rec) if rec is not None else None
         for l in range(c.num_layers):
             q, k, v = self._split_heads(rms_norm(h) @ self.w_qkv[l].T)
             qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
             kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
-            self.cache[(l, i, b)] = (kr, v.copy(), (b, i))
-            self.cache.pop((l, i, b - c.window_blocks - 1), None)
+            self.cache[(l, ring, b)] = (kr, v.copy(), (b, c.num_steps if refresh else i))
+            self.cache.pop((l, ring, b - c.window_blocks - 1), None)
             sk = rope_rotate(self.sink_k[l], st, sh, sw, c.pairs, c.rope_theta)
-            blocks = {bb: (kk, vv) for (ll, ii, bb), (kk, vv, _) in self.cache.items()
-                      if ll == l and ii == i}
+            blocks = {bb: (kk, vv) for (ll, rr, bb), (kk, vv, _) in self.cache.items()
+                      if ll == l and rr == ring}
             o = block_causal_attention(qr, blocks, (sk, self.sink_v[l]), qblock=b,
                                        window=c.window_blocks)
             h = h + o.reshape(h.shape[0], -1) @ self.w_out[l].T
             if tr is not None:
                 tr[("layer", l)] = dict(q=qr, k=kr, v=v.copy(), sink_k=sk, o=o, h=h.copy())
+        if refresh:
+            if tr is not None:
+                self.trace[(b, "refresh")] = tr
+            return x
         vel = self.project_head(h)
         x_next = euler_step(x, vel, c.timesteps[i], c.timesteps[i + 1])
         if tr is not None:
@@ -144,6 +164,8 @@ class OracleStream:
         out = None
         if finished >= 0:
             out = self.latents.pop(finished)
+            if self.sched.clean:
+                self.slot_pass(out, finished, self.cfg.num_steps, refresh=True)
         if self.sched.end_tick(finished):
             src = out if aas_latent is None else np.asarray(aas_latent, np.float64)
             self.set_sink(src[: self.cfg.sink_tokens])

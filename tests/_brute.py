@@ -55,6 +55,7 @@ class BruteStream:
         self.sink = None      # per layer: list of (r, c, k_heads (unroped), v_heads)
         self.replaced = False
         self.lat = {}
+        self.clean = []       # clean-cache entries (layer, block, k_rot, v)
 
     def _heads(self, vec, part):
         c = self.c
@@ -155,4 +156,59 @@ class BruteStream:
                 if fin == 0 and c.sink_mode == 1 and not self.replaced:
                     self.replaced = True
                     self.set_sink(done[0][: c.sink_tokens])
+        return done
+
+    # -- clean-cache refresh (NFE num_steps + 1), sequential -------------------------
+    def _forward_clean(self, x, b):
+        """One pass of block b over the clean cache: every layer attends to the
+        sink, the clean K/V of blocks b - window .. b - 1 and the pass's own K/V.
+        Returns (final residual, [(layer, [(k_rot, v) per token])])."""
+        c = self.c
+        h = [list(map(float, r)) for r in x]
+        if self.win is not None:
+            h = matvec_rows(h, self.win)
+        fpb = c.frames_per_block
+        t_sink = fpb * b - c.sink_offset_frames if c.rolling_rope else -c.sink_offset_frames
+        own_all = []
+        for l in range(c.num_layers):
+            qkv = matvec_rows(normalize_rows(h), self.wqkv[l])
+            qrot, own = [], []
+            for n, vec in enumerate(qkv):
+                f, r, cc = self._tok_rc(n)
+                t = fpb * b + f
+                qrot.append([rotate(x_, t, r, cc, c.pairs, c.rope_theta) for x_ in self._heads(vec, 0)])
+                own.append(([rotate(x_, t, r, cc, c.pairs, c.rope_theta) for x_ in self._heads(vec, 1)],
+                            self._heads(vec, 2)))
+            visible = [([rotate(x_, t_sink, r, cc, c.pairs, c.rope_theta) for x_ in kh], vh)
+                       for (r, cc, kh, vh) in self.sink[l]]
+            visible += [(kr, vh) for (ll, bb, kr, vh) in self.clean if ll == l and b - c.window_blocks <= bb < b]
+            visible += own
+            o = self._layer_attend(qrot, visible)
+            proj = matvec_rows(o, self.wout[l])
+            h = [[a + bq for a, bq in zip(hr, pr)] for hr, pr in zip(h, proj)]
+            own_all.append((l, own))
+        return h, own_all
+
+    def run_sequential_clean(self, noises):
+        """Each block: num_steps Euler steps over the clean cache, then one more
+        pass of the finished latent whose K/V become that block's clean entry."""
+        c = self.c
+        self.clean = []       # (layer, block, k_rot, v)
+        done = {}
+        for b, noise in enumerate(noises):
+            x = [list(map(float, r)) for r in noise]
+            for i in range(c.num_steps):
+                h, _ = self._forward_clean(x, b)
+                hn = normalize_rows(h)
+                v = hn if self.whead is None else matvec_rows(hn, self.whead)
+                dt = c.timesteps[i + 1] - c.timesteps[i]
+                x = [[xa + dt * va for xa, va in zip(xr, vr)] for xr, vr in zip(x, v)]
+            _, own_all = self._forward_clean(x, b)
+            for l, own in own_all:
+                for kr, vh in own:
+                    self.clean.append((l, b, kr, vh))
+            done[b] = x
+            if b == 0 and c.sink_mode == 1 and not self.replaced:
+                self.replaced = True
+                self.set_sink(x[: c.sink_tokens])
         return done

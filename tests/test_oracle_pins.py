@@ -13,8 +13,8 @@ import torch
 
 from oracle import OracleStream, TickScheduler, block_causal_attention, euler_step, rms_norm, rope_rotate
 from oracle.rope import axis_frequencies, block_positions, sink_positions, sink_temporal_position
-from workloads import (SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_AAS, SINK_FIXED, TINY,
-                       StreamConfig, Workload, block_noise, make_weights, random_array)
+from workloads import (CACHE_CLEAN_REFRESH, CACHE_TIMESTEP, SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_AAS,
+                       SINK_FIXED, TINY, StreamConfig, Workload, block_noise, make_weights, random_array)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pages_facts.json")
 
@@ -407,3 +407,73 @@ def test_oracle_stream_matches_brute_force_with_projections_and_no_rolling():
         out, fin = s.denoise_step(noises[k] if k < wl.num_blocks else None)
         if fin >= 0:
             np.testing.assert_allclose(out, np.array(want[fin]), rtol=1e-11, atol=1e-11)
+
+
+# -- the clean-cache refresh ablation (NFE num_steps + 1) ---------------------------------------
+def _clean_cfg(**kw):
+    base = dict(num_layers=2, hidden=16, heads=2, head_dim=8, latent_ch=16, grid_h=2, grid_w=2, window_blocks=1,
+                rope_split=(2, 1, 1), sink_mode=SINK_AAS, dtype=1, schedule=SCHED_SEQUENTIAL,
+                cache_mode=CACHE_CLEAN_REFRESH)
+    base.update(kw)
+    return StreamConfig(**base)
+
+
+@pytest.mark.parametrize("window,sink_mode,rolling", [(1, SINK_AAS, 1), (2, SINK_FIXED, 0)])
+def test_clean_refresh_oracle_matches_scalar_brute_force(window, sink_mode, rolling):
+    cfg = _clean_cfg(window_blocks=window, sink_mode=sink_mode, rolling_rope=rolling)
+    wl = Workload("brute-clean", cfg, 13, 5, 0.25)
+    W = make_weights(wl)
+    noises = [block_noise(wl, b) for b in range(wl.num_blocks)]
+    from _brute import BruteStream
+    bs = BruteStream(cfg, W)
+    bs.set_sink(W.sink)
+    want = bs.run_sequential_clean(noises)
+    s = OracleStream(cfg, W)
+    s.set_sink(W.sink)
+    for b in range(wl.num_blocks):
+        out, fin = s.denoise_step(noises[b])
+        assert fin == b
+        np.testing.assert_allclose(out, np.array(want[b]), rtol=1e-11, atol=1e-11)
+
+
+def test_clean_refresh_equals_timestep_forcing_without_a_window():
+    """Window 0: no step reads a cache entry of another block, so the two cache
+    modes compute the same latents (the refresh leaves x unchanged)."""
+    outs = {}
+    for mode in (CACHE_TIMESTEP, CACHE_CLEAN_REFRESH):
+        cfg = _clean_cfg(window_blocks=0, cache_mode=mode)
+        wl = Workload("w0", cfg, 14, 4, 0.25)
+        W = make_weights(wl)
+        s = OracleStream(cfg, W)
+        s.set_sink(W.sink)
+        outs[mode] = [s.denoise_step(block_noise(wl, b))[0] for b in range(wl.num_blocks)]
+    for a, b in zip(outs[CACHE_TIMESTEP], outs[CACHE_CLEAN_REFRESH]):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_clean_refresh_ring_tags_closed_form():
+    """One shared ring: after block b, entry b mod (window+1) holds (b, S) (the
+    refresh), the resident blocks are b-window .. b, and every step's record
+    shows that ring."""
+    cfg = _clean_cfg(window_blocks=2)
+    wl = Workload("tags", cfg, 15, 6, 0.25)
+    W = make_weights(wl)
+    s = OracleStream(cfg, W)
+    s.set_sink(W.sink)
+    S, E = cfg.num_steps, cfg.ring_entries
+    _, per, _ = __import__("oracle").index_state_layout(cfg)
+    for b in range(wl.num_blocks):
+        s.denoise_step(block_noise(wl, b))
+        st = s.index_state()
+        tags = {(b2 % E): (b2, S) for b2 in range(max(0, b - 2), b + 1)}
+        for i in range(S):
+            rec = st[4 + i * per: 4 + (i + 1) * per]
+            assert rec[0] == b and rec[1] == b % E and rec[6] == i
+            assert list(rec[8:8 + E]) == list(range(max(0, b - 2), b + 1)) + [-1] * (E - min(b + 1, E))
+            got = {e: (rec[8 + E + 2 * e], rec[8 + E + 2 * e + 1]) for e in range(E) if rec[8 + E + 2 * e] >= 0}
+            assert got == tags
+
+
+def test_clean_refresh_needs_the_sequential_schedule():
+    with pytest.raises(ValueError):
+        TickScheduler(_clean_cfg(schedule=SCHED_PIPELINED))

@@ -27,6 +27,8 @@ SCHED_PIPELINED = 0
 SCHED_SEQUENTIAL = 1
 DTYPE_BF16 = 0
 DTYPE_FP32 = 1
+CACHE_TIMESTEP = 0         # noisy K/V of each step in that step's own cache (timestep forcing)
+CACHE_CLEAN_REFRESH = 1    # one cache of clean K/V, refreshed by an extra forward of x0 per block (NFE S+1)
 
 
 def default_rope_split(head_dim: int) -> tuple:
@@ -57,6 +59,7 @@ class StreamConfig:
     sink_offset_frames: int = 3
     schedule: int = SCHED_PIPELINED
     dtype: int = DTYPE_BF16
+    cache_mode: int = CACHE_TIMESTEP
 
     @property
     def num_steps(self) -> int:
