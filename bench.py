@@ -1,6 +1,6 @@
 """Benchmark of the timestep-forced streaming step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sweep]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sweep | --ablation]
 
 A step is one tick of the 4-slot grouped stream in steady state: 4 in-flight
 blocks (one per timestep slot, every window full) through 8 attention
@@ -427,6 +427,55 @@ def run_sweep(args):
           flush=True)
 
 
+def run_ablation(args):
+    """Seconds per block at the headline shape (8 sublayers, 14B-like, window 2) for the
+    schedules the pages compare (papernotes note, Table 2): the grouped timestep-forced stream
+    (4 blocks in flight, NFE 4), the same cache sequentially (one block through its 4 steps per
+    call, NFE 4), and the clean-cache refresh the method removes (4 steps + 1 refresh forward,
+    NFE 5).  One JSON line each."""
+    import torch
+    from streaming_causal_video_timestep_b200 import LaStream
+    from workloads import CACHE_CLEAN_REFRESH, CACHE_TIMESTEP, SCHED_PIPELINED, SCHED_SEQUENTIAL, STREAM
+
+    torch.cuda.set_device(0)
+    bf = torch.bfloat16
+    for name, sched, mode, nfe in (("timestep-forced, grouped pipeline", SCHED_PIPELINED, CACHE_TIMESTEP, 4),
+                                   ("timestep-forced, sequential", SCHED_SEQUENTIAL, CACHE_TIMESTEP, 4),
+                                   ("clean-cache refresh, sequential", SCHED_SEQUENTIAL, CACHE_CLEAN_REFRESH, 5)):
+        cfg = STREAM.cfg.replace(schedule=sched, cache_mode=mode)
+        T, C, D, F = cfg.block_tokens, cfg.latent_ch, cfg.hidden, cfg.frame_tokens
+        S, nw, L = cfg.num_steps, cfg.window_blocks, cfg.num_layers
+        g = torch.Generator(device="cuda")
+        g.manual_seed(7)
+        rnd = lambda shape, std: (torch.randn(shape, generator=g, device="cuda") * std).to(bf)
+        weights = dict(w_qkv=[rnd((3 * D, D), STREAM.w_std) for _ in range(L)],
+                       w_out=[rnd((D, D), STREAM.w_std) for _ in range(L)],
+                       w_in=rnd((D, C), 1.0 / C ** 0.5), w_head=rnd((C, D), STREAM.head_std))
+        s = LaStream(cfg, weights)
+        s.set_sink(torch.randn((F, C), generator=g, device="cuda"))
+        xs = [torch.randn((T, C), generator=g, device="cuda") for _ in range(2)]
+        x_out = torch.empty((T, C), device="cuda")
+        fill = ((S - 1) if sched == SCHED_PIPELINED else 0) + nw + 1 + args.warmup
+        for k in range(fill):
+            s.step(xs[k % 2], x_out)
+        s.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for k in range(args.steps):
+            assert s.step(xs[k % 2], x_out) >= 0
+        ev1.record()
+        s.synchronize()
+        torch.cuda.synchronize()
+        ms = ev0.elapsed_time(ev1) / args.steps
+        print(json.dumps({"ablation": name, "nfe_per_block": nfe, "ms_per_block": round(ms, 3),
+                          "latent_frames_per_s": round(cfg.frames_per_block / (ms / 1000.0), 3),
+                          "config": "8 sublayers, hidden 5120, 40x128 heads, 30x52 grid, window 2, bf16"}),
+              flush=True)
+        s.close()
+        del s, weights
+        torch.cuda.empty_cache()
+
+
 def run_reference(args):
     smp = OracleSample(rows=234)
     for _ in range(args.warmup):
@@ -455,6 +504,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="shape sweep lines instead of the headline line")
+    ap.add_argument("--ablation", action="store_true",
+                    help="seconds per block: grouped pipeline vs sequential vs clean-cache refresh")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -469,6 +520,10 @@ def main():
     if args.sweep:
         if rank == 0:
             run_sweep(args)
+        return
+    if args.ablation:
+        if rank == 0:
+            run_ablation(args)
         return
 
     if world > 1:

@@ -66,6 +66,14 @@ extern "C" {
 #define LA_BF16              0  /* bf16 GEMM operands and attention operands, fp32
                                    accumulation, fp32 residual stream and latent x    */
 #define LA_FP32              1  /* fp32 everywhere (SIMT path, no TF32)                */
+#define LA_CACHE_TIMESTEP    0  /* each step keeps the noisy K/V it computed in its own
+                                   cache (timestep forcing; papernotes note, key design
+                                   4; gitcode blog, question 6)                         */
+#define LA_CACHE_CLEAN_REFRESH 1 /* the ablation the method removes: one cache of clean
+                                   K/V; after a block's last step one more pass of the
+                                   finished latent rewrites its entry (NFE num_steps+1;
+                                   papernotes note, key design 2 and Table 2; gitcode
+                                   blog, question 4).  Sequential schedule only.       */
 
 #define LA_RMS_EPS 1e-6
 
@@ -100,6 +108,7 @@ typedef struct la_config {
   int32_t sink_offset_frames;  /* 3                                                      */
   int32_t schedule;            /* LA_SCHED_PIPELINED | LA_SCHED_SEQUENTIAL               */
   int32_t dtype;               /* LA_BF16 | LA_FP32                                      */
+  int32_t cache_mode;          /* LA_CACHE_TIMESTEP | LA_CACHE_CLEAN_REFRESH              */
 } la_config;
 
 /*
@@ -201,7 +210,8 @@ int la_debug_capture(la_stream* s, int32_t enable);
                                them pre-multiplied by the softmax scale log2(e)/sqrt(d)         */
 #define LA_TAP_O         4  /* fp32 [T_b, D]   attention output of layer, before rounding        */
 #define LA_TAP_V         5  /* fp32 [T_b, C]    velocity of the slot's last step                 */
-#define LA_TAP_RING_K    6  /* attn [E, H, T_b, d] ring K of (layer, slot), by entry             */
+#define LA_TAP_RING_K    6  /* attn [E, H, T_b, d] ring K of (layer, slot), by entry (the one
+                               clean cache for every slot under LA_CACHE_CLEAN_REFRESH)          */
 #define LA_TAP_RING_V    7  /* attn [E, H, T_b, d] ring V of (layer, slot)                       */
 #define LA_TAP_SINK_K    8  /* fp32 [H, F, d] un-roped sink K of layer (slot ignored)            */
 #define LA_TAP_SINK_V    9  /* attn [H, F, d] sink V of layer (slot ignored)                     */

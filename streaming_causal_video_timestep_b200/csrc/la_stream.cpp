@@ -29,7 +29,7 @@ struct SlotRecord {
 };
 
 struct Scheduler {
-  int S = 0, E = 0, W = 0, fpb = 0, offset = 0, rolling = 1, pipelined = 1, aas = 0;
+  int S = 0, E = 0, W = 0, fpb = 0, offset = 0, rolling = 1, pipelined = 1, aas = 0, clean = 0;
   long long tick = -1, blocks_in = 0, blocks_out = 0;
   int sink_gen = 0;
   std::vector<long long> held;                  // block held by each slot after the last call
@@ -46,11 +46,14 @@ struct Scheduler {
     rolling = c.rolling_rope;
     pipelined = c.schedule == LA_SCHED_PIPELINED;
     aas = c.sink_mode == LA_SINK_AAS;
+    clean = c.cache_mode == LA_CACHE_CLEAN_REFRESH;
     held.assign(S, -1);
     tag_blk.assign(S, std::vector<long long>(E, -1));
     tag_step.assign(S, std::vector<int>(E, -1));
     rec.assign(S, SlotRecord());
   }
+  // The cache step i reads and writes: its own, or the one clean cache.
+  int ring_of(int i) const { return clean ? 0 : i; }
   int sink_tpos_of(long long b) const {
     return rolling ? static_cast<int>(fpb * b - offset) : -offset;
   }
@@ -79,15 +82,23 @@ struct Scheduler {
   }
   int append(int i, long long b) {
     const int e = static_cast<int>(b % E);
+    const int ring = ring_of(i);
     SlotRecord& r = rec[i];
     r.active_block = static_cast<int>(b);
     r.write_entry = e;
-    r.evicted = static_cast<int>(tag_blk[i][e]);
+    r.evicted = static_cast<int>(tag_blk[ring][e]);
     r.sink_tpos = sink_tpos_of(b);
     r.frame_tpos = static_cast<int>(fpb * b);
     r.sink_gen = sink_gen;
-    tag_blk[i][e] = b;
-    tag_step[i][e] = i;
+    tag_blk[ring][e] = b;
+    tag_step[ring][e] = i;
+    return e;
+  }
+  // The clean-cache refresh of finished block b rewrites its entry, tagged (b, S).
+  int append_refresh(long long b) {
+    const int e = static_cast<int>(b % E);
+    tag_blk[0][e] = b;
+    tag_step[0][e] = S;
     return e;
   }
   bool finish(long long finished) {
@@ -107,9 +118,10 @@ struct Scheduler {
     int32_t* p = out + 4;
     for (int i = 0; i < S; ++i) {
       const SlotRecord& r = rec[i];
+      const int ring = ring_of(i);
       std::vector<long long> res;
       for (int e = 0; e < E; ++e)
-        if (tag_blk[i][e] >= 0) res.push_back(tag_blk[i][e]);
+        if (tag_blk[ring][e] >= 0) res.push_back(tag_blk[ring][e]);
       std::sort(res.begin(), res.end());
       *p++ = r.active_block;
       *p++ = r.write_entry;
@@ -121,8 +133,8 @@ struct Scheduler {
       *p++ = static_cast<int32_t>(res.size());
       for (int e = 0; e < E; ++e) *p++ = e < static_cast<int>(res.size()) ? static_cast<int32_t>(res[e]) : -1;
       for (int e = 0; e < E; ++e) {
-        *p++ = static_cast<int32_t>(tag_blk[i][e]);
-        *p++ = tag_step[i][e];
+        *p++ = static_cast<int32_t>(tag_blk[ring][e]);
+        *p++ = tag_step[ring][e];
       }
     }
   }
@@ -299,6 +311,11 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
   if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) { msg = "rope_theta must be positive"; return LA_EINVAL; }
   if (c->sink_mode != LA_SINK_FIXED && c->sink_mode != LA_SINK_AAS) { msg = "bad sink_mode"; return LA_EINVAL; }
   if (c->schedule != LA_SCHED_PIPELINED && c->schedule != LA_SCHED_SEQUENTIAL) { msg = "bad schedule"; return LA_EINVAL; }
+  if (c->cache_mode != LA_CACHE_TIMESTEP && c->cache_mode != LA_CACHE_CLEAN_REFRESH) { msg = "bad cache_mode"; return LA_EINVAL; }
+  if (c->cache_mode == LA_CACHE_CLEAN_REFRESH && c->schedule != LA_SCHED_SEQUENTIAL) {
+    msg = "the clean-cache refresh needs the sequential schedule";
+    return LA_EINVAL;
+  }
   if (c->rolling_rope != 0 && c->rolling_rope != 1) { msg = "rolling_rope must be 0 or 1"; return LA_EINVAL; }
   if (c->sink_offset_frames < 0) { msg = "sink_offset_frames must be >= 0"; return LA_EINVAL; }
   if ((w->w_in == nullptr) != (w->w_head == nullptr)) { msg = "w_in and w_head must both be set or both NULL"; return LA_EINVAL; }
@@ -359,7 +376,8 @@ int capture_pass(la_stream* s, const PassDesc& pd, int layer) {
   const float* o32 = s->bf16 ? s->cap_oall : static_cast<const float*>(s->attn_o);
   for (int ai = 0; ai < pd.nactive; ++ai) {
     const int buf = pd.active_buf[ai];
-    const int slot = pd.slot[buf];
+    const int slot = pd.step[buf];   // capture areas are per denoising step
+    if (slot >= s->S) continue;      // the clean-cache refresh is not captured
     if (layer < 0) {
       CU(cudaMemcpyAsync(s->cap_h + (static_cast<long long>(slot) * (L + 1)) * T * D, s->h32 + buf * T * D,
                          T * D * 4, cudaMemcpyDeviceToDevice, s->st));
@@ -394,7 +412,8 @@ int run_pass(la_stream* s, const PassDesc& pd) {
   if (s->capture) {
     for (int ai = 0; ai < pd.nactive; ++ai) {
       const int buf = pd.active_buf[ai];
-      CU(cudaMemcpyAsync(s->cap_xin + static_cast<long long>(pd.slot[buf]) * T * C,
+      if (pd.step[buf] >= S) continue;
+      CU(cudaMemcpyAsync(s->cap_xin + static_cast<long long>(pd.step[buf]) * T * C,
                          s->xs + static_cast<long long>(buf) * T * C, static_cast<size_t>(T) * C * 4,
                          cudaMemcpyDeviceToDevice, s->st));
     }
@@ -525,10 +544,11 @@ int run_pass(la_stream* s, const PassDesc& pd) {
   if (s->capture) {
     for (int ai = 0; ai < pd.nactive; ++ai) {
       const int buf = pd.active_buf[ai];
-      const long long so = static_cast<long long>(pd.slot[buf]) * T * C, bo = static_cast<long long>(buf) * T * C;
+      if (pd.step[buf] >= S) continue;
+      const long long so = static_cast<long long>(pd.step[buf]) * T * C, bo = static_cast<long long>(buf) * T * C;
       CU(cudaMemcpyAsync(s->cap_xout + so, s->xs + bo, static_cast<size_t>(T) * C * 4, cudaMemcpyDeviceToDevice, s->st));
       CU(cudaMemcpyAsync(s->cap_v + so, s->cap_vall + bo, static_cast<size_t>(T) * C * 4, cudaMemcpyDeviceToDevice, s->st));
-      s->cap_valid[pd.slot[buf]] = 1;
+      s->cap_valid[pd.step[buf]] = 1;
     }
   }
   return LA_OK;
@@ -609,11 +629,14 @@ int run_sink(la_stream* s) {
   return LA_OK;
 }
 
-void fill_pass_slot(la_stream* s, PassDesc& pd, int buf, int slot, long long b, int write_entry) {
+// Buffer buf runs block b at step `step` (num_steps: a clean-cache refresh, dt 0)
+// reading and writing ring `ring`.
+void fill_pass_slot(la_stream* s, PassDesc& pd, int buf, int ring, int step, long long b, int write_entry) {
   const int W = s->cfg.window_blocks;
   pd.active[buf] = 1;
   pd.active_buf[pd.nactive++] = buf;
-  pd.slot[buf] = slot;
+  pd.slot[buf] = ring;
+  pd.step[buf] = step;
   pd.block[buf] = static_cast<int>(b);
   pd.write_entry[buf] = write_entry;
   const int nw = static_cast<int>(std::min<long long>(b, W));
@@ -621,7 +644,7 @@ void fill_pass_slot(la_stream* s, PassDesc& pd, int buf, int slot, long long b, 
   for (int w = 0; w < nw; ++w) pd.win_entry[buf][w] = static_cast<int>((b - nw + w) % s->E);
   pd.frame_tpos[buf] = static_cast<int>(s->fpb * b);
   pd.sink_tpos[buf] = s->sched.sink_tpos_of(b);
-  pd.dt[buf] = s->ts[slot + 1] - s->ts[slot];
+  pd.dt[buf] = step < s->S ? s->ts[step + 1] - s->ts[step] : 0.0f;
 }
 
 int step_impl(la_stream* s, const float* x_new, float* x_out, int64_t* finished_block, cudaMemcpyKind in_kind,
@@ -651,7 +674,7 @@ int step_impl(la_stream* s, const float* x_new, float* x_out, int64_t* finished_
     pd.nbuf = s->S;
     for (auto& [slot, b] : run) {
       const int e = s->sched.append(slot, b);
-      fill_pass_slot(s, pd, static_cast<int>(b % s->S), slot, b, e);
+      fill_pass_slot(s, pd, static_cast<int>(b % s->S), slot, slot, b, e);
     }
     if (pd.nactive > 0 && (r = run_pass(s, pd)) != LA_OK) return r;
     if (finished >= 0)
@@ -662,7 +685,16 @@ int step_impl(la_stream* s, const float* x_new, float* x_out, int64_t* finished_
       PassDesc pd{};
       pd.nbuf = 1;
       const int e = s->sched.append(slot, b);
-      fill_pass_slot(s, pd, 0, slot, b, e);
+      fill_pass_slot(s, pd, 0, s->sched.ring_of(slot), slot, b, e);
+      if ((r = run_pass(s, pd)) != LA_OK) return r;
+    }
+    if (s->sched.clean) {
+      // clean-cache refresh: the finished latent through the stack once more
+      // (dt 0 leaves it unchanged); its K/V replace the block's cache entry
+      PassDesc pd{};
+      pd.nbuf = 1;
+      const int e = s->sched.append_refresh(finished);
+      fill_pass_slot(s, pd, 0, 0, s->S, finished, e);
       if ((r = run_pass(s, pd)) != LA_OK) return r;
     }
     CU(cudaMemcpyAsync(x_out, s->xs, TC * 4, out_kind, s->st));
@@ -960,7 +992,8 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
     case LA_TAP_SINK_KROPE: src = elem(s->cap_sk, (slot * L + layer) * H * F * d, ea); bytes = H * F * d * ea; break;
     case LA_TAP_RING_K:
     case LA_TAP_RING_V:
-      src = elem(what == LA_TAP_RING_K ? s->ring_k : s->ring_v, (static_cast<long long>(layer) * S + slot) * E * H * T * d, ea);
+      src = elem(what == LA_TAP_RING_K ? s->ring_k : s->ring_v,
+                 (static_cast<long long>(layer) * S + s->sched.ring_of(slot)) * E * H * T * d, ea);
       bytes = E * H * T * d * ea;
       break;
     case LA_TAP_SINK_K: src = s->sink_k + static_cast<long long>(layer) * H * F * d; bytes = H * F * d * 4; break;

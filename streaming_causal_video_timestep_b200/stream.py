@@ -49,7 +49,7 @@ class LaStream:
     (num_layers, hidden, heads, head_dim, latent_ch, grid_h, grid_w,
     frames_per_block, sink_frames, window_blocks, timesteps, rope_split or
     pairs, rope_theta, sink_mode, rolling_rope, sink_offset_frames, schedule,
-    dtype).  `weights` holds CUDA tensors in the config dtype:
+    dtype, and optionally cache_mode).  `weights` holds CUDA tensors in the config dtype:
     w_qkv / w_out (lists), w_in / w_head (or None)."""
 
     def __init__(self, cfg, weights, stream=None):
@@ -70,6 +70,7 @@ class LaStream:
         c.rope_theta = float(cfg.rope_theta)
         c.sink_mode, c.rolling_rope, c.sink_offset_frames = cfg.sink_mode, cfg.rolling_rope, cfg.sink_offset_frames
         c.schedule, c.dtype = cfg.schedule, self.dtype
+        c.cache_mode = getattr(cfg, "cache_mode", 0)
         self.cfg = cfg
         self.c = c
         self.T = cfg.frames_per_block * cfg.grid_h * cfg.grid_w

@@ -86,6 +86,8 @@ def _weights(nonnull=True):
     dict(sink_frames=2), dict(num_steps=0, timesteps=(1.0,)), dict(num_steps=9),
     dict(sink_mode=5), dict(schedule=3), dict(rope_theta=0.0), dict(frames_per_block=0),
     dict(latent_ch=32),                               # identity needs latent_ch == hidden
+    dict(cache_mode=2),
+    dict(cache_mode=1, schedule=0),                   # the clean-cache refresh is sequential only
 ])
 def test_invalid_config_returns_einval(lib, over):
     c = _cfg(**over)

@@ -6,8 +6,8 @@ import numpy as np
 import pytest
 
 from oracle import OracleStream, TickScheduler
-from workloads import (DTYPE_BF16, DTYPE_FP32, SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_AAS, SINK_FIXED, TINY,
-                       StreamConfig, Workload, block_noise, make_weights)
+from workloads import (CACHE_CLEAN_REFRESH, DTYPE_BF16, DTYPE_FP32, SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_AAS,
+                       SINK_FIXED, TINY, StreamConfig, Workload, block_noise, make_weights)
 
 from _helpers import assert_close, errors, make_stream, to_np
 from _percheck import check_sink, check_step, sink_snapshot
@@ -202,3 +202,40 @@ def test_small_bf16_rolling_rope_off_teacher_forced():
     cfg = SMALL_BF16.cfg.replace(rolling_rope=0)
     _run_teacher_forced(Workload("small-bf16-rolling0", cfg, SMALL_BF16.seed, 6, SMALL_BF16.w_std,
                                  SMALL_BF16.head_std))
+
+
+
+def _run_clean_refresh(wl):
+    """The clean-cache refresh ablation, free-running: integer state bit-exact and
+    the finished block against the oracle every call; returns the worst errors."""
+    cfg = wl.cfg
+    s, W = make_stream(wl)
+    orc = OracleStream(cfg, W)
+    orc.set_sink(W.sink)
+    x_out = torch.empty((cfg.block_tokens, cfg.latent_ch), dtype=torch.float32, device="cuda")
+    worst = (0.0, 0.0)
+    for b in range(wl.num_blocks):
+        xn = block_noise(wl, b)
+        fin = s.step(_dev(xn), x_out)
+        out, fin_o = orc.denoise_step(xn)
+        assert fin == fin_o == b
+        np.testing.assert_array_equal(s.index_state(), orc.index_state())
+        if cfg.dtype == DTYPE_FP32:
+            assert_close(to_np(x_out), out, DTYPE_FP32, f"clean-refresh block {b}")
+        worst = max(worst, errors(to_np(x_out), out))
+    s.close()
+    return worst
+
+
+@pytest.mark.parametrize("window", [1, 2])
+def test_tiny_fp32_clean_cache_refresh_matches_oracle(window):
+    cfg = TINY.cfg.replace(schedule=SCHED_SEQUENTIAL, cache_mode=CACHE_CLEAN_REFRESH, window_blocks=window)
+    _run_clean_refresh(Workload(f"tiny-clean-w{window}", cfg, TINY.seed, TINY.num_blocks, TINY.w_std,
+                                TINY.head_std))
+
+
+def test_small_bf16_clean_cache_refresh_integer_state_and_drift():
+    cfg = SMALL_BF16.cfg.replace(schedule=SCHED_SEQUENTIAL, cache_mode=CACHE_CLEAN_REFRESH)
+    worst = _run_clean_refresh(Workload("small-bf16-clean", cfg, SMALL_BF16.seed, 5, SMALL_BF16.w_std,
+                                        SMALL_BF16.head_std))
+    print({"free-running drift": (f"{worst[0]:.2e}", f"{worst[1]:.2e}")})
