@@ -3,12 +3,16 @@
     python -m streaming_causal_video_timestep_b200.microbench attn  [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench gemm  [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench euler [--iters N]
+    python -m streaming_causal_video_timestep_b200.microbench rerope [--iters N]
 
 attn : one block's attention in steady state at the 14B-like shape: 4680
        queries x 40 heads x 128 over [sink 1560 | 2 window blocks | block]
        = 15,600 keys (the per-slot launch of the stream), q pre-scaled.
 gemm : the QKV projection of one block, [4680, 5120] x [15360, 5120]^T.
 euler: x += dt * v over 2^20 rows x 64 fp32 (256 MB per tensor), 4 groups.
+rerope: the per-block sink re-rope of a one-sublayer stream (30x52 grid, 40x128
+       heads, 4 slots): reads the fp32 un-roped sink K (32 MB) once and writes
+       4 bf16 roped copies (64 MB); timed by the stream's profiling counters.
 Inputs exceed L2 (126 MB) except the per-slot attention keys (160 MB K/V +
 48 MB q).  Prints one JSON line per mode.
 """
@@ -74,14 +78,46 @@ def bench_euler(iters):
             "bytes": nbytes}
 
 
+def bench_rerope(iters):
+    from types import SimpleNamespace
+    from .stream import LaStream
+    cfg = SimpleNamespace(num_layers=1, hidden=5120, heads=40, head_dim=128, latent_ch=64, grid_h=30, grid_w=52,
+                          frames_per_block=3, sink_frames=1, window_blocks=1, timesteps=(1.0, 0.75, 0.5, 0.25, 0.0),
+                          rope_split=(22, 21, 21), pairs=(22, 21, 21), rope_theta=10000.0, sink_mode=0, rolling_rope=1,
+                          sink_offset_frames=3, schedule=0, dtype=0)
+    D, C, F, T = cfg.hidden, cfg.latent_ch, cfg.grid_h * cfg.grid_w, 3 * cfg.grid_h * cfg.grid_w
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    rnd = lambda *sh: (torch.randn(*sh, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    w = dict(w_qkv=[rnd(3 * D, D)], w_out=[rnd(D, D)], w_in=rnd(D, C), w_head=rnd(C, D))
+    s = LaStream(cfg, w)
+    s.set_sink(torch.randn(F, C, generator=g, device="cuda"))
+    x = torch.randn(T, C, generator=g, device="cuda")
+    out = torch.empty(T, C, device="cuda")
+    for _ in range(3 + 2 + 3):          # fill: every slot active
+        s.step(x, out)
+    s.synchronize()
+    s.profile(True)
+    for _ in range(iters):
+        s.step(x, out)
+    s.synchronize()
+    n, tot = s.profile_read("rope")
+    s.profile(False)
+    s.close()
+    ms = tot / n
+    nbytes = F * D * 4 + 4 * F * D * 2
+    return {"mode": "rerope", "shape": f"sink {F} tokens x {D}, 4 slots", "ms": round(ms, 4),
+            "gbs": round(nbytes / ms / 1e6, 1), "bytes": nbytes}
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("mode", choices=["attn", "gemm", "euler", "all"])
+    ap.add_argument("mode", choices=["attn", "gemm", "euler", "rerope", "all"])
     ap.add_argument("--iters", type=int, default=10)
     args = ap.parse_args()
-    modes = ["attn", "gemm", "euler"] if args.mode == "all" else [args.mode]
+    modes = ["attn", "gemm", "euler", "rerope"] if args.mode == "all" else [args.mode]
     for m in modes:
-        r = {"attn": bench_attn, "gemm": bench_gemm, "euler": bench_euler}[m](args.iters)
+        r = {"attn": bench_attn, "gemm": bench_gemm, "euler": bench_euler, "rerope": bench_rerope}[m](args.iters)
         print(json.dumps(r), flush=True)
 
 
