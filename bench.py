@@ -429,7 +429,7 @@ def run_sweep(args):
 
 def run_ablation(args):
     """Seconds per block at the headline shape (8 sublayers, 14B-like, window 2) for the
-    schedules the pages compare (papernotes note, Table 2): the grouped timestep-forced stream
+    schedules the pages compare (papernotes note, inference-efficiency ablation, the paper's Table 3): the grouped timestep-forced stream
     (4 blocks in flight, NFE 4), the same cache sequentially (one block through its 4 steps per
     call, NFE 4), and the clean-cache refresh the method removes (4 steps + 1 refresh forward,
     NFE 5).  One JSON line each."""

@@ -72,7 +72,7 @@ extern "C" {
 #define LA_CACHE_CLEAN_REFRESH 1 /* the ablation the method removes: one cache of clean
                                    K/V; after a block's last step one more pass of the
                                    finished latent rewrites its entry (NFE num_steps+1;
-                                   papernotes note, key design 2 and Table 2; gitcode
+                                   papernotes note, key design 2 and the paper's Table 3; gitcode
                                    blog, question 4).  Sequential schedule only.       */
 
 #define LA_RMS_EPS 1e-6

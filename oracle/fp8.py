@@ -1,0 +1,82 @@
+"""FP8 (e4m3) quantization and the FP8 GEMM, fp64 (the operator-optimisation row).
+
+TEST INFRASTRUCTURE ONLY (see oracle/__init__.py).
+
+The pages' largest single speed-up is operator-level optimisation (papernotes
+note, inference-efficiency ablation = the paper's Table 3, last row: FP8
+quantisation + FlashAttention-3 + fused kernels).  The pages give no FP8
+scheme; the reading taken for the projections is per-row scaling: each row of
+an operand is quantized to e4m3 with its own fp32 scale, the tensor core
+multiplies the 8-bit codes exactly and accumulates, and the result is rescaled
+by the row's and the column's scales:
+    scale_r = amax_r / 448            (fp32; 1 for an all-zero row)
+    q[r, k] = e4m3(x[r, k] / scale_r) (fp32 division, round to nearest even,
+                                        saturating at +-448)
+    C[m, n] = (sum_k dec(qa[m, k]) dec(qw[n, k])) * scale_a[m] * scale_w[n]
+
+e4m3 here is the OCP 8-bit floating point format E4M3 ("FN": no infinities):
+1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 is
+subnormal (m/8 * 2^-6); the code with all exponent and mantissa bits set is NaN,
+so the largest finite magnitude is 1.75 * 2^8 = 448.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode_table() -> np.ndarray:
+    """Value of each of the 256 codes (float64; NaN for the two NaN codes)."""
+    vals = np.empty(256, np.float64)
+    for code in range(256):
+        sign = -1.0 if code & 0x80 else 1.0
+        e = (code >> 3) & 0xF
+        m = code & 0x7
+        if e == 0xF and m == 0x7:
+            vals[code] = np.nan
+        elif e == 0:
+            vals[code] = sign * (m / 8.0) * 2.0 ** -6
+        else:
+            vals[code] = sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return vals
+
+
+_TABLE = e4m3_decode_table()
+_POS_CODES = np.arange(0x00, 0x7F)              # 0 .. 126: the non-negative finite values, increasing
+_POS_VALS = _TABLE[_POS_CODES]
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    return _TABLE[np.asarray(codes, np.uint8)]
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Round float32 values to the nearest e4m3 value, ties to the even code,
+    saturating to +-448; NaN is not expected here.  Returns uint8 codes."""
+    x = np.asarray(x, np.float32).astype(np.float64)
+    mag = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.searchsorted(_POS_VALS, mag, side="left")          # first value >= mag
+    hi = np.clip(hi, 0, len(_POS_VALS) - 1)
+    lo = np.clip(hi - 1, 0, len(_POS_VALS) - 1)
+    d_hi = _POS_VALS[hi] - mag
+    d_lo = mag - _POS_VALS[lo]
+    pick_lo = (d_lo < d_hi) | ((d_lo == d_hi) & (_POS_CODES[lo] % 2 == 0))
+    code = np.where(pick_lo, _POS_CODES[lo], _POS_CODES[hi]).astype(np.uint8)
+    neg = (x < 0) & (code != 0)
+    return np.where(neg, code | 0x80, code).astype(np.uint8)
+
+
+def quantize_rows(x):
+    """Per-row e4m3 quantization: (codes uint8 [R, K], scales float32 [R])."""
+    x = np.asarray(x, np.float32)
+    amax = np.max(np.abs(x), axis=1).astype(np.float32)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    return e4m3_encode((x / scale[:, None]).astype(np.float32)), scale
+
+
+def gemm_fp8(a_codes, a_scale, w_codes, w_scale) -> np.ndarray:
+    """C = (dec(A) dec(W)^T) * a_scale[:, None] * w_scale[None, :], fp64."""
+    a = e4m3_decode(a_codes)
+    w = e4m3_decode(w_codes)
+    return (a @ w.T) * np.asarray(a_scale, np.float64)[:, None] * np.asarray(w_scale, np.float64)[None, :]

@@ -23,7 +23,7 @@ sink_generation_used are 0 for a slot idle this tick; step_index is the slot
 index; n_resident, resident and tags always describe the ring contents.
 
 Clean-cache refresh (the ablation the method removes; papernotes note, 关键设计 2
-and the NFE row of its Table 2; gitcode blog, question 4 table): one cache of
+and the NFE column of its inference-efficiency ablation, the paper's Table 3; gitcode blog, question 4 table): one cache of
 clean K/V serves every step, so all slots share ring 0 (their records describe
 it); after the last step of block b one more pass runs the stack on the
 finished latent and overwrites block b's entry, tagged (b, num_steps).  Only

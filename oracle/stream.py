@@ -25,7 +25,7 @@ once block 0 is finished, frame 0 of its final latent replaces the sink and the
 sink is never replaced again.
 
 Clean-cache refresh (the baseline the pages remove, papernotes note 关键设计 2
-and the "DMD 4-step" row of its Table 2: 4 denoising steps plus 1 clean
+and the "DMD 4-step" row of its inference-efficiency ablation (the paper's Table 3): 4 denoising steps plus 1 clean
 forward refresh, NFE 5; gitcode blog question 4: the cache holds the clean x0's
 K/V, written by one extra forward per block): one cache per layer; every step
 of block b reads the clean K/V of blocks b-window .. b-1 and its own current
