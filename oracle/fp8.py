@@ -53,7 +53,9 @@ def e4m3_decode(codes) -> np.ndarray:
 
 def e4m3_encode(x) -> np.ndarray:
     """Round float32 values to the nearest e4m3 value, ties to the even code,
-    saturating to +-448; NaN is not expected here.  Returns uint8 codes."""
+    saturating to +-448; the sign is kept, so a negative value that rounds to
+    zero gives -0 (code 0x80), as IEEE rounding does.  NaN is not expected
+    here.  Returns uint8 codes."""
     x = np.asarray(x, np.float32).astype(np.float64)
     mag = np.minimum(np.abs(x), E4M3_MAX)
     hi = np.searchsorted(_POS_VALS, mag, side="left")          # first value >= mag
@@ -63,8 +65,7 @@ def e4m3_encode(x) -> np.ndarray:
     d_lo = mag - _POS_VALS[lo]
     pick_lo = (d_lo < d_hi) | ((d_lo == d_hi) & (_POS_CODES[lo] % 2 == 0))
     code = np.where(pick_lo, _POS_CODES[lo], _POS_CODES[hi]).astype(np.uint8)
-    neg = (x < 0) & (code != 0)
-    return np.where(neg, code | 0x80, code).astype(np.uint8)
+    return np.where(np.signbit(x), code | 0x80, code).astype(np.uint8)
 
 
 def quantize_rows(x):
