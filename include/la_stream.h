@@ -313,6 +313,30 @@ int la_op_euler(float* x, const float* v, int64_t rows, int64_t C, const float* 
                 int64_t rows_per_group, void* cuda_stream);
 
 /*
+ * FP8 (e4m3) operands for the projections: the pages' operator-level
+ * optimisation row (papernotes note, inference-efficiency ablation = the
+ * paper's Table 3: FP8 quantisation + FlashAttention-3 + fused kernels; the
+ * pages give no scheme, per-row scaling is the reading taken).
+ *
+ * la_op_quantize_e4m3: per-row quantization of x (DEVICE, in_dtype LA_BF16 or
+ * LA_FP32, [rows, cols] dense, cols even): scales[r] = amax_r / 448 (fp32;
+ * 1 for an all-zero row), codes[r, c] = e4m3(x[r, c] / scales[r]) with IEEE
+ * fp32 division, rounding to nearest even and saturation at +-448 (OCP E4M3,
+ * no infinities).  codes: DEVICE uint8 [rows, cols]; scales: DEVICE fp32 [rows].
+ *
+ * la_op_gemm_fp8: out[m, n] = (sum_k a[m, k] w[n, k]) * a_scales[m] *
+ * w_scales[n] on the tensor cores (tcgen05 kind::f8f6f4, fp32 accumulate):
+ * a_codes DEVICE uint8 [M, K], w_codes [N, K] (both dense, K % 16 == 0),
+ * scales DEVICE fp32 [M] / [N]; out DEVICE [M, N], out_dtype LA_BF16 (rounded
+ * once) or LA_FP32.  N % 32 == 0.  LA_EINVAL on bad sizes or NULL pointers.
+ */
+int la_op_quantize_e4m3(int32_t in_dtype, const void* x, int64_t rows, int64_t cols,
+                        void* codes, float* scales, void* cuda_stream);
+int la_op_gemm_fp8(const void* a_codes, const float* a_scales, const void* w_codes,
+                   const float* w_scales, void* out, int32_t out_dtype, int64_t M, int64_t N,
+                   int64_t K, void* cuda_stream);
+
+/*
  * Block attention for callers that cannot allocate device memory (a plugin
  * whose host application owns all device memory through its own allocator or
  * a fixed budget, or a real-time path where an allocation and its implicit

@@ -99,6 +99,8 @@ struct GemmEpiParams {
   float dt[LA_MAX_STEPS];
   int active[LA_MAX_STEPS];   // EULER: only active groups update
   float* vtap;          // optional fp32 [M, N] copy of acc (velocity capture)
+  const float* row_scale;   // optional [M]: acc *= row_scale[row] * col_scale[col] first (FP8 operands)
+  const float* col_scale;   // [N], set together with row_scale
 };
 
 

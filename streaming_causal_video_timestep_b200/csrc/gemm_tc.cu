@@ -1,10 +1,13 @@
 // C = A W^T on the 5th-generation tensor cores (tcgen05, accumulators in TMEM).
 //
 // Persistent kernel, one CTA per SM, 6 warps:
-//   warp 0      TMA producer: A [128 x 64] and W [BN x 64] bf16 tiles per k-block,
-//               128-byte swizzle, into a STAGES-deep shared-memory ring;
+//   warp 0      TMA producer: A [128 x 128 B] and W [BN x 128 B] tiles per k-block
+//               (64 bf16 or 128 e4m3 values a row), 128-byte swizzle, into a
+//               STAGES-deep shared-memory ring;
 //   warp 1      allocates TMEM (2 accumulators of BN fp32 columns) and, with one
-//               thread, issues tcgen05.mma 128 x BN x 16 into the accumulator;
+//               thread, issues tcgen05.mma into the accumulator: kind::f16
+//               128 x BN x 16 (bf16) or kind::f8f6f4 128 x BN x 32 (e4m3), four
+//               per k-block (32 bytes of K each);
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //               32*(w%4) .. +31 = tile rows), fused epilogue, global stores.
 // The two accumulators let the epilogue of tile n overlap the main loop of n+1.
@@ -18,14 +21,14 @@
 namespace {
 
 constexpr int BM = 128;
-constexpr int BK = 64;
+constexpr int BK_BYTES = 128;   // K bytes per k-block: one 128-byte swizzle row
 constexpr int GROUP_M = 16;
 
 template <int BN>
 struct GemmCfg {
   static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
-  static constexpr uint32_t A_BYTES = BM * BK * 2;
-  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t A_BYTES = BM * BK_BYTES;
+  static constexpr uint32_t B_BYTES = BN * BK_BYTES;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
   static constexpr size_t SMEM = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
@@ -168,7 +171,7 @@ __device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, const Qk
   }
 }
 
-template <int BN>
+template <int BN, bool FP8>
 __global__ void __launch_bounds__(192, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ GemmEpiParams ep, const __grid_constant__ QkvRopeParams qp, int M, int N, int K,
@@ -214,8 +217,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   const int num_m = (M + BM - 1) / BM;
   const int num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
+  constexpr int BK = FP8 ? 128 : 64;   // K elements per k-block
   const int kblocks = (K + BK - 1) / BK;
-  constexpr uint32_t idesc = idesc_bf16(BM, BN, false, false);
+  constexpr uint32_t idesc = FP8 ? idesc_e4m3(BM, BN) : idesc_bf16(BM, BN, false, false);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -259,9 +263,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            umma_bf16_ss(d_tmem, sdesc_kmajor(a0 + kk * 32), sdesc_kmajor(b0 + kk * 32), idesc,
-                         (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK_BYTES / 32; ++kk) {
+            if (FP8)
+              umma_e4m3_ss(d_tmem, sdesc_kmajor(a0 + kk * 32), sdesc_kmajor(b0 + kk * 32), idesc,
+                           (kb | kk) != 0 ? 1u : 0u);
+            else
+              umma_bf16_ss(d_tmem, sdesc_kmajor(a0 + kk * 32), sdesc_kmajor(b0 + kk * 32), idesc,
+                           (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -297,6 +305,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          if (ep.row_scale) {
+            const float rs = ep.row_scale[row];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= rs * ep.col_scale[col + i];
+          }
           epilogue_row32(ep, qp, row, col, v);
         }
       }
@@ -315,16 +328,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   }
 }
 
-template <int BN>
+template <int BN, bool FP8>
 cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep,
                       const QkvRopeParams& qp, int M, int N, int K, int* err, int num_sms, cudaStream_t st) {
   using C = GemmCfg<BN>;
-  cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::SMEM));
   if (e != cudaSuccess) return e;
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  k_gemm_tc<BN><<<grid, 192, C::SMEM, st>>>(tmA, tmB, ep, qp, M, N, K, err);
+  k_gemm_tc<BN, FP8><<<grid, 192, C::SMEM, st>>>(tmA, tmB, ep, qp, M, N, K, err);
   return cudaGetLastError();
 }
 
@@ -341,8 +354,19 @@ cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const
   QkvRopeParams none{};
   const QkvRopeParams& q = qp ? *qp : none;
   switch (bn) {
-    case 256: return launch_bn<256>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
-    case 128: return launch_bn<128>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
-    default: return launch_bn<64>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
+    case 256: return launch_bn<256, false>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
+    case 128: return launch_bn<128, false>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
+    default: return launch_bn<64, false>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
+  }
+}
+
+cudaError_t launch_gemm_tc_fp8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M,
+                               int N, int K, int bn, int* err, int num_sms, cudaStream_t st) {
+  if (!ep.row_scale || !ep.col_scale) return cudaErrorInvalidValue;
+  QkvRopeParams none{};
+  switch (bn) {
+    case 256: return launch_bn<256, true>(tmA, tmB, ep, none, M, N, K, err, num_sms, st);
+    case 128: return launch_bn<128, true>(tmA, tmB, ep, none, M, N, K, err, num_sms, st);
+    default: return launch_bn<64, true>(tmA, tmB, ep, none, M, N, K, err, num_sms, st);
   }
 }

@@ -12,6 +12,16 @@ int gemm_tc_pick_bn(int N);
 cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M, int N,
                            int K, int bn, int* err, int num_sms, cudaStream_t st, const QkvRopeParams* qp = nullptr);
 
+// The same GEMM on e4m3 operands (kind::f8f6f4; tmA / tmB from tmap_2d_u8 with
+// box rows 128 / bn); ep.row_scale / ep.col_scale are required and multiply the
+// fp32 accumulator before the epilogue.
+cudaError_t launch_gemm_tc_fp8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M,
+                               int N, int K, int bn, int* err, int num_sms, cudaStream_t st);
+// Per-row e4m3 quantization of x (bf16 if bf16_in, else fp32) [rows, cols]:
+// q uint8 [rows, cols], scale fp32 [rows] = amax / 448 (1 for a zero row).
+cudaError_t launch_quant_rows_e4m3(int bf16_in, const void* x, long long rows, long long cols, void* q,
+                                   float* scale, cudaStream_t st);
+
 // Tensor maps of an attention launch: q (d, Tq, H, q slices) and k[m]/v[m]
 // (d, rows_m, H, slices), bf16, 128-byte swizzle, box (64, 128, 1, 1).
 struct AttnMaps {

@@ -103,6 +103,37 @@ int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t
   return ret(launch_attn_f32(p, st));
 }
 
+int la_op_quantize_e4m3(int32_t in_dtype, const void* x, int64_t rows, int64_t cols, void* codes, float* scales,
+                        void* cuda_stream) {
+  if (!x || !codes || !scales || rows < 1 || rows > (1LL << 31) - 1 || cols < 2 || cols % 2 != 0) return LA_EINVAL;
+  if (in_dtype != LA_BF16 && in_dtype != LA_FP32) return LA_EINVAL;
+  return ret(launch_quant_rows_e4m3(in_dtype == LA_BF16, x, rows, cols, codes, scales,
+                                    static_cast<cudaStream_t>(cuda_stream)));
+}
+
+int la_op_gemm_fp8(const void* a_codes, const float* a_scales, const void* w_codes, const float* w_scales, void* out,
+                   int32_t out_dtype, int64_t M, int64_t N, int64_t K, void* cuda_stream) {
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !out) return LA_EINVAL;
+  if (M < 1 || N < 32 || K < 16 || M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return LA_EINVAL;
+  if (N % 32 != 0 || K % 16 != 0) return LA_EINVAL;
+  if (out_dtype != LA_BF16 && out_dtype != LA_FP32) return LA_EINVAL;
+  std::string err;
+  if (!tmap_init(err)) return LA_ECUDA;
+  const int bn = gemm_tc_pick_bn(static_cast<int>(N));
+  CUtensorMap ta, tb;
+  if (!tmap_2d_u8(&ta, a_codes, M, K, K, 128, err) || !tmap_2d_u8(&tb, w_codes, N, K, K, bn, err)) return LA_ECUDA;
+  GemmEpiParams ep{};
+  ep.kind = out_dtype == LA_BF16 ? LA_EPI_STORE : LA_EPI_STORE32;
+  ep.out = out;
+  ep.ld = N;
+  ep.rows_per_group = 1 << 30;
+  for (int i = 0; i < LA_MAX_STEPS; ++i) ep.active[i] = 1;
+  ep.row_scale = a_scales;
+  ep.col_scale = w_scales;
+  return ret(launch_gemm_tc_fp8(ta, tb, ep, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), bn,
+                                nullptr, num_sms_current(), static_cast<cudaStream_t>(cuda_stream)));
+}
+
 int la_op_euler(float* x, const float* v, int64_t rows, int64_t C, const float* dt, int64_t rows_per_group,
                 void* cuda_stream) {
   if (!x || !v || !dt || rows < 1 || C < 4 || C % 4 != 0 || rows_per_group < 1) return LA_EINVAL;

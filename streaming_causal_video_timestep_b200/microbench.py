@@ -4,12 +4,15 @@
     python -m streaming_causal_video_timestep_b200.microbench gemm  [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench euler [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench rerope [--iters N]
+    python -m streaming_causal_video_timestep_b200.microbench gemm_fp8 [--iters N]
 
 attn : one block's attention in steady state at the 14B-like shape: 4680
        queries x 40 heads x 128 over [sink 1560 | 2 window blocks | block]
        = 15,600 keys (the per-slot launch of the stream), q pre-scaled.
 gemm : the QKV projection of one block, [4680, 5120] x [15360, 5120]^T.
 euler: x += dt * v over 2^20 rows x 64 fp32 (256 MB per tensor), 4 groups.
+gemm_fp8: the QKV projection shape on e4m3 operands (kind::f8f6f4, per-row
+       scales, bf16 output), and the per-row quantization of its activation.
 rerope: the per-block sink re-rope of a one-sublayer stream (30x52 grid, 40x128
        heads, 4 slots): reads the fp32 un-roped sink K (32 MB) once and writes
        4 bf16 roped copies (64 MB); timed by the stream's profiling counters.
@@ -23,7 +26,7 @@ import json
 
 import torch
 
-from .stream import op_attention, op_euler, op_gemm
+from .stream import op_attention, op_euler, op_gemm, op_gemm_fp8, op_quantize_e4m3
 
 
 def _time(fn, iters, warmup=3):
@@ -65,6 +68,27 @@ def bench_gemm(iters):
     flops = 2.0 * M * N * K
     return {"mode": "gemm", "shape": f"{M}x{N}x{K}", "ms": round(ms, 4), "tflops": round(flops / ms / 1e9, 1),
             "flops": flops}
+
+
+def bench_gemm_fp8(iters):
+    M, N, K = 4680, 15360, 5120
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    x = torch.randn(M, K, generator=g, device="cuda").to(torch.bfloat16)
+    wt = (torch.randn(N, K, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    qa = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    sa = torch.empty(M, device="cuda")
+    qw = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    sw = torch.empty(N, device="cuda")
+    op_quantize_e4m3(wt, qw, sw)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ms_q = _time(lambda: op_quantize_e4m3(x, qa, sa), iters)
+    ms = _time(lambda: op_gemm_fp8(qa, sa, qw, sw, out), iters)
+    flops = 2.0 * M * N * K
+    qbytes = M * K * 2 + M * K + M * 4
+    return {"mode": "gemm_fp8", "shape": f"{M}x{N}x{K} e4m3", "ms": round(ms, 4),
+            "tflops": round(flops / ms / 1e9, 1), "flops": flops,
+            "quantize": {"ms": round(ms_q, 4), "gbs": round(qbytes / ms_q / 1e6, 1), "bytes": qbytes}}
 
 
 def bench_euler(iters):
@@ -112,12 +136,13 @@ def bench_rerope(iters):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("mode", choices=["attn", "gemm", "euler", "rerope", "all"])
+    ap.add_argument("mode", choices=["attn", "gemm", "euler", "rerope", "gemm_fp8", "all"])
     ap.add_argument("--iters", type=int, default=10)
     args = ap.parse_args()
-    modes = ["attn", "gemm", "euler", "rerope"] if args.mode == "all" else [args.mode]
+    modes = ["attn", "gemm", "gemm_fp8", "euler", "rerope"] if args.mode == "all" else [args.mode]
     for m in modes:
-        r = {"attn": bench_attn, "gemm": bench_gemm, "euler": bench_euler, "rerope": bench_rerope}[m](args.iters)
+        r = {"attn": bench_attn, "gemm": bench_gemm, "euler": bench_euler, "rerope": bench_rerope,
+             "gemm_fp8": bench_gemm_fp8}[m](args.iters)
         print(json.dumps(r), flush=True)
 
 

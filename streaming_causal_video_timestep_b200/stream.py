@@ -217,3 +217,22 @@ def op_euler(x, v, dt, rows_per_group, stream=None):
     rows, C = x.shape
     dtp = (c_float * len(dt))(*[float(t) for t in dt])
     check(lib.la_op_euler(_ptr(x), _ptr(v), rows, C, dtp, rows_per_group, _stream_handle(stream)))
+
+
+def op_quantize_e4m3(x, codes, scales, stream=None):
+    """Per-row e4m3 quantization: x [rows, cols] bf16 or fp32 CUDA tensor ->
+    codes uint8 [rows, cols], scales fp32 [rows] (amax / 448)."""
+    lib = load()
+    rows, cols = x.shape
+    check(lib.la_op_quantize_e4m3(_dtype_code(x.dtype), _ptr(x), rows, cols, _ptr(codes), _ptr(scales),
+                                  _stream_handle(stream)))
+
+
+def op_gemm_fp8(a_codes, a_scales, w_codes, w_scales, out, stream=None):
+    """out [M, N] (bf16 or fp32) = (A W^T) * a_scales[:, None] * w_scales[None, :] from
+    uint8 e4m3 codes A [M, K], W [N, K] on the tensor cores."""
+    lib = load()
+    M, K = a_codes.shape
+    N = w_codes.shape[0]
+    check(lib.la_op_gemm_fp8(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes), _ptr(w_scales), _ptr(out),
+                             _dtype_code(out.dtype), M, N, K, _stream_handle(stream)))
