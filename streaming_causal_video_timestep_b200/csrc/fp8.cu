@@ -44,11 +44,82 @@ __global__ void __launch_bounds__(256) k_quant_rows_e4m3(const TI* __restrict__ 
     q2[c >> 1] = e4m3x2(__fdiv_rn(load_as_float(xr, c), s), __fdiv_rn(load_as_float(xr, c + 1), s));
 }
 
+// 8 consecutive values as fp32.
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+// Rows of up to 256 * 8 * QV values, cols % 8 == 0: each thread keeps its
+// vectors in registers between the max and the quantization (one read of x).
+constexpr int QV = 4;
+
+template <typename TI>
+__global__ void __launch_bounds__(256) k_quant_rows_e4m3_vec(const TI* __restrict__ x, long long cols,
+                                                             uint8_t* __restrict__ q, float* __restrict__ scale) {
+  __shared__ float red[8];
+  const long long row = blockIdx.x;
+  const int nvec = static_cast<int>(cols / 8);
+  const TI* xr = x + row * cols;
+  float v[QV][8];
+  float m = 0.f;
+#pragma unroll
+  for (int j = 0; j < QV; ++j) {
+    const int idx = threadIdx.x + j * 256;
+    if (idx < nvec) {
+      load8(xr + static_cast<long long>(idx) * 8, v[j]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[j][i]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float amax = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  const float s = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  if (threadIdx.x == 0) scale[row] = s;
+  uint2* q8 = reinterpret_cast<uint2*>(q + row * cols);
+#pragma unroll
+  for (int j = 0; j < QV; ++j) {
+    const int idx = threadIdx.x + j * 256;
+    if (idx < nvec) {
+      uint32_t lo = e4m3x2(__fdiv_rn(v[j][0], s), __fdiv_rn(v[j][1], s)) |
+                    (static_cast<uint32_t>(e4m3x2(__fdiv_rn(v[j][2], s), __fdiv_rn(v[j][3], s))) << 16);
+      uint32_t hi = e4m3x2(__fdiv_rn(v[j][4], s), __fdiv_rn(v[j][5], s)) |
+                    (static_cast<uint32_t>(e4m3x2(__fdiv_rn(v[j][6], s), __fdiv_rn(v[j][7], s))) << 16);
+      q8[idx] = make_uint2(lo, hi);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_quant_rows_e4m3(int bf16_in, const void* x, long long rows, long long cols, void* q,
                                    float* scale, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
+  const uintptr_t align = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(q);
+  if (cols % 8 == 0 && cols <= 256LL * 8 * QV && align % 16 == 0) {
+    if (bf16_in)
+      k_quant_rows_e4m3_vec<__nv_bfloat16><<<static_cast<unsigned>(rows), 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), cols, static_cast<uint8_t*>(q), scale);
+    else
+      k_quant_rows_e4m3_vec<float><<<static_cast<unsigned>(rows), 256, 0, st>>>(
+          static_cast<const float*>(x), cols, static_cast<uint8_t*>(q), scale);
+    return cudaGetLastError();
+  }
   if (bf16_in)
     k_quant_rows_e4m3<__nv_bfloat16><<<static_cast<unsigned>(rows), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), cols, static_cast<uint8_t*>(q), scale);
