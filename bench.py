@@ -439,10 +439,12 @@ def run_ablation(args):
 
     torch.cuda.set_device(0)
     bf = torch.bfloat16
-    for name, sched, mode, nfe in (("timestep-forced, grouped pipeline", SCHED_PIPELINED, CACHE_TIMESTEP, 4),
-                                   ("timestep-forced, sequential", SCHED_SEQUENTIAL, CACHE_TIMESTEP, 4),
-                                   ("clean-cache refresh, sequential", SCHED_SEQUENTIAL, CACHE_CLEAN_REFRESH, 5)):
-        cfg = STREAM.cfg.replace(schedule=sched, cache_mode=mode)
+    for name, sched, mode, nfe, fp8 in (
+            ("timestep-forced, grouped pipeline", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0),
+            ("timestep-forced, sequential", SCHED_SEQUENTIAL, CACHE_TIMESTEP, 4, 0),
+            ("clean-cache refresh, sequential", SCHED_SEQUENTIAL, CACHE_CLEAN_REFRESH, 5, 0),
+            ("timestep-forced, grouped pipeline, e4m3 projections", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 1)):
+        cfg = STREAM.cfg.replace(schedule=sched, cache_mode=mode, proj_fp8=fp8)
         T, C, D, F = cfg.block_tokens, cfg.latent_ch, cfg.hidden, cfg.frame_tokens
         S, nw, L = cfg.num_steps, cfg.window_blocks, cfg.num_layers
         g = torch.Generator(device="cuda")
@@ -459,6 +461,7 @@ def run_ablation(args):
         for k in range(fill):
             s.step(xs[k % 2], x_out)
         s.synchronize()
+        s.profile(True)
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record()
         for k in range(args.steps):
@@ -467,9 +470,13 @@ def run_ablation(args):
         s.synchronize()
         torch.cuda.synchronize()
         ms = ev0.elapsed_time(ev1) / args.steps
+        kinds = {kd: round(s.profile_read(kd)[1] / args.steps, 3) for kd in ("qkv_gemm", "attn", "out_gemm", "other")}
+        s.profile(False)
         print(json.dumps({"ablation": name, "nfe_per_block": nfe, "ms_per_block": round(ms, 3),
                           "latent_frames_per_s": round(cfg.frames_per_block / (ms / 1000.0), 3),
-                          "config": "8 sublayers, hidden 5120, 40x128 heads, 30x52 grid, window 2, bf16"}),
+                          "ms_per_block_by_kind": kinds,
+                          "config": "8 sublayers, hidden 5120, 40x128 heads, 30x52 grid, window 2, "
+                                    + ("e4m3 QKV/output projections, bf16 elsewhere" if fp8 else "bf16")}),
               flush=True)
         s.close()
         del s, weights

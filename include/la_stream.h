@@ -109,6 +109,13 @@ typedef struct la_config {
   int32_t schedule;            /* LA_SCHED_PIPELINED | LA_SCHED_SEQUENTIAL               */
   int32_t dtype;               /* LA_BF16 | LA_FP32                                      */
   int32_t cache_mode;          /* LA_CACHE_TIMESTEP | LA_CACHE_CLEAN_REFRESH              */
+  int32_t proj_fp8;            /* 1 (LA_BF16 only): the QKV and output projections run on
+                                  e4m3 operands: weights quantized per output row at
+                                  creation, the bf16 GEMM operand per token before each
+                                  projection (la_op_quantize_e4m3's definition), fp32
+                                  accumulate, scales applied before the epilogue.  The
+                                  pages' FP8 row (papernotes note, the paper's Table 3).
+                                  0: bf16 projections.                                   */
 } la_config;
 
 /*
@@ -218,6 +225,9 @@ int la_debug_capture(la_stream* s, int32_t enable);
 #define LA_TAP_SINK_KROPE 10 /* attn [H, F, d] sink K as roped for the slot's last step          */
 #define LA_TAP_SINK_H    11 /* fp32 [F, D] sink residual entering layer `layer` in the last sink
                                pass (la_set_sink or the AAS replacement; slot ignored)           */
+#define LA_TAP_HOP       12 /* bf16 [T_b, D] normalised residual as the QKV projection of layer
+                               `layer` consumed it at the slot's step (bf16 streams)             */
+#define LA_TAP_SINK_HOP  13 /* bf16 [F, D] the same in the last sink pass (slot ignored)         */
 
 /* Copy one tapped tensor into dst (DEVICE, dst_bytes >= the tensor's size),
  * ordered on the stream.  Taps other than ring / sink need capture enabled

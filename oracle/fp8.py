@@ -68,6 +68,21 @@ def e4m3_encode(x) -> np.ndarray:
     return np.where(np.signbit(x), code | 0x80, code).astype(np.uint8)
 
 
+def bf16_round_f32(x) -> np.ndarray:
+    """float32 values rounded to the nearest bfloat16 (8 significant bits, ties
+    to even), returned as float32: the operand a bf16 GEMM consumes."""
+    u = np.asarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return (r & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
+
+
+def project(a, w_codes, w_scales):
+    """A projection on e4m3 operands: a (the bf16 operand, as float64 or
+    float32 values) quantized per row, times the weight codes."""
+    qa, sa = quantize_rows(bf16_round_f32(np.asarray(a, np.float64).astype(np.float32)))
+    return gemm_fp8(qa, sa, w_codes, w_scales)
+
+
 def quantize_rows(x):
     """Per-row e4m3 quantization: (codes uint8 [R, K], scales float32 [R])."""
     x = np.asarray(x, np.float32)

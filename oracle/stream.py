@@ -32,6 +32,11 @@ of block b reads the clean K/V of blocks b-window .. b-1 and its own current
 K/V; after the last step the finished latent goes through the stack once more
 (no Euler update) and its K/V replace block b's entry.  Reading: with AAS the
 refresh of block 0 uses the reference sink, and the sink is replaced after it.
+
+e4m3 projections (cfg.proj_fp8; the pages' FP8 row, papernotes note, the
+paper's Table 3): the QKV and output projections take their operand as the
+bf16 stream's GEMM consumes it (bf16), quantize it per token and multiply
+e4m3 codes (oracle/fp8.py); everything else is unchanged.
 """
 from __future__ import annotations
 
@@ -39,6 +44,7 @@ import numpy as np
 
 from .attention import block_causal_attention
 from .flow import euler_step
+from .fp8 import project, quantize_rows
 from .norm import rms_norm
 from .rope import block_positions, rope_rotate, sink_positions
 from .schedule import TickScheduler
@@ -52,6 +58,10 @@ class OracleStream:
         self.w_out = [f64(w) for w in weights.w_out]
         self.w_in = f64(weights.w_in)
         self.w_head = f64(weights.w_head)
+        # e4m3 projections (cfg.proj_fp8): weights quantized per output row, once
+        fp8 = getattr(cfg, "proj_fp8", 0)
+        self.wq8 = [quantize_rows(np.asarray(w, np.float32)) for w in weights.w_qkv] if fp8 else None
+        self.wo8 = [quantize_rows(np.asarray(w, np.float32)) for w in weights.w_out] if fp8 else None
         self.sched = TickScheduler(cfg)
         self.cache = {}            # (layer, ring, block) -> (k_roped, v, (block, step))
         self.sink_k = None         # per layer, un-roped [F, H, d]
@@ -69,6 +79,14 @@ class OracleStream:
         k = qkv[:, D:2 * D].reshape(T, H, d)
         v = qkv[:, 2 * D:3 * D].reshape(T, H, d)
         return q, k, v
+
+    def _proj_qkv(self, l, n):
+        """[q | k | v] of the normalised residual n; e4m3 projections quantize the
+        bf16 operand per token (oracle/fp8.py)."""
+        return n @ self.w_qkv[l].T if self.wq8 is None else project(n, *self.wq8[l])
+
+    def _proj_out(self, l, o):
+        return o @ self.w_out[l].T if self.wo8 is None else project(o, *self.wo8[l])
 
     def project_in(self, x):
         x = np.asarray(x, np.float64)
@@ -88,13 +106,13 @@ class OracleStream:
         pt, ph, pw = sink_positions(c, t0)
         self.sink_k, self.sink_v = [], []
         for l in range(c.num_layers):
-            q, k, v = self._split_heads(rms_norm(h) @ self.w_qkv[l].T)
+            q, k, v = self._split_heads(self._proj_qkv(l, rms_norm(h)))
             self.sink_k.append(k.copy())
             self.sink_v.append(v.copy())
             qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
             kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
             o = block_causal_attention(qr, {}, (kr, v), qblock=0, window=c.window_blocks)
-            h = h + o.reshape(h.shape[0], -1) @ self.w_out[l].T
+            h = h + self._proj_out(l, o.reshape(h.shape[0], -1))
             if self.trace is not None:
                 self.trace[("sink", l)] = dict(k=k.copy(), v=v.copy(), o=o, h=h.copy())
 
@@ -119,7 +137,7 @@ class OracleStream:
             tr["h_in"] = h.copy()
             tr["record"] = list(rec) if rec is not None else None
         for l in range(c.num_layers):
-            q, k, v = self._split_heads(rms_norm(h) @ self.w_qkv[l].T)
+            q, k, v = self._split_heads(self._proj_qkv(l, rms_norm(h)))
             qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
             kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
             self.cache[(l, ring, b)] = (kr, v.copy(), (b, c.num_steps if refresh else i))
@@ -129,7 +147,7 @@ class OracleStream:
                       if ll == l and rr == ring}
             o = block_causal_attention(qr, blocks, (sk, self.sink_v[l]), qblock=b,
                                        window=c.window_blocks)
-            h = h + o.reshape(h.shape[0], -1) @ self.w_out[l].T
+            h = h + self._proj_out(l, o.reshape(h.shape[0], -1))
             if tr is not None:
                 tr[("layer", l)] = dict(q=qr, k=kr, v=v.copy(), sink_k=sk, o=o, h=h.copy())
         if refresh:

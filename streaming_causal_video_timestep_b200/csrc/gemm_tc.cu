@@ -361,12 +361,13 @@ cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const
 }
 
 cudaError_t launch_gemm_tc_fp8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M,
-                               int N, int K, int bn, int* err, int num_sms, cudaStream_t st) {
+                               int N, int K, int bn, int* err, int num_sms, cudaStream_t st, const QkvRopeParams* qp) {
   if (!ep.row_scale || !ep.col_scale) return cudaErrorInvalidValue;
   QkvRopeParams none{};
+  const QkvRopeParams& q = qp ? *qp : none;
   switch (bn) {
-    case 256: return launch_bn<256, true>(tmA, tmB, ep, none, M, N, K, err, num_sms, st);
-    case 128: return launch_bn<128, true>(tmA, tmB, ep, none, M, N, K, err, num_sms, st);
-    default: return launch_bn<64, true>(tmA, tmB, ep, none, M, N, K, err, num_sms, st);
+    case 256: return launch_bn<256, true>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
+    case 128: return launch_bn<128, true>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
+    default: return launch_bn<64, true>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
   }
 }

@@ -16,7 +16,8 @@ cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const
 // box rows 128 / bn); ep.row_scale / ep.col_scale are required and multiply the
 // fp32 accumulator before the epilogue.
 cudaError_t launch_gemm_tc_fp8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M,
-                               int N, int K, int bn, int* err, int num_sms, cudaStream_t st);
+                               int N, int K, int bn, int* err, int num_sms, cudaStream_t st,
+                               const QkvRopeParams* qp = nullptr);
 // Per-row e4m3 quantization of x (bf16 if bf16_in, else fp32) [rows, cols]:
 // q uint8 [rows, cols], scale fp32 [rows] = amax / 448 (1 for a zero row).
 cudaError_t launch_quant_rows_e4m3(int bf16_in, const void* x, long long rows, long long cols, void* q,

@@ -153,6 +153,7 @@ struct la_stream {
   int S = 0, E = 0, F = 0, T = 0, D = 0, C = 0, H = 0, d = 0, L = 0, fpb = 0, nbuf = 0;
   int pt = 0, ph = 0, pw = 0;
   bool bf16 = true, id_in = true, id_head = true;
+  bool fp8 = false;         // e4m3 QKV / output projections (bf16 streams)
   size_t es = 2;            // activation / weight element (bf16 or fp32)
   size_t ea = 2;            // attention operand element (bf16 or fp32)
   int device = 0, num_sms = 148;
@@ -194,6 +195,14 @@ struct la_stream {
   CUtensorMap tm_hop{}, tm_xop{}, tm_o{}, tm_win{}, tm_whead{};
   std::vector<CUtensorMap> tm_wqkv, tm_wout;
   CUtensorMap tm_s_hop{}, tm_s_xop{}, tm_s_o{};
+  // e4m3 projections: weight codes [rows, D] with per-row scales, and the
+  // codes / scales of the operand quantized before each projection
+  std::vector<void*> wq8, wo8;
+  std::vector<float*> wq8s, wo8s;
+  void* a8 = nullptr;       // uint8 [max(nbuf*T, F)][D]
+  float* a8s = nullptr;     // [max(nbuf*T, F)]
+  CUtensorMap tm_a8{}, tm_s_a8{};
+  std::vector<CUtensorMap> tm_wq8, tm_wo8;
   AttnMaps maps_stream{};   // q = q_rope; k[0]/v[0] = ring; k[1] = sink K roped per buffer; v[1] = sink V
   AttnMaps maps_sink{};     // q = s_q; k[0] = s_k; v[0] = sink V
 
@@ -215,6 +224,8 @@ struct la_stream {
   float* cap_o = nullptr;     // fp32 [S][L][T][D]
   void* cap_sk = nullptr;     // attn type [S][L][H][F][d]
   float* cap_sink_h = nullptr;  // fp32 [L][F][D] sink residual entering each layer
+  void* cap_hop = nullptr;      // bf16 [S][L][T][D] normalised residual entering each QKV projection
+  void* cap_sink_hop = nullptr; // bf16 [L][F][D] the same in the last sink pass
   bool cap_sink_valid = false;
   std::vector<int> cap_valid;  // per slot: captured in the last call
 
@@ -312,6 +323,8 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
   if (c->sink_mode != LA_SINK_FIXED && c->sink_mode != LA_SINK_AAS) { msg = "bad sink_mode"; return LA_EINVAL; }
   if (c->schedule != LA_SCHED_PIPELINED && c->schedule != LA_SCHED_SEQUENTIAL) { msg = "bad schedule"; return LA_EINVAL; }
   if (c->cache_mode != LA_CACHE_TIMESTEP && c->cache_mode != LA_CACHE_CLEAN_REFRESH) { msg = "bad cache_mode"; return LA_EINVAL; }
+  if (c->proj_fp8 != 0 && c->proj_fp8 != 1) { msg = "proj_fp8 must be 0 or 1"; return LA_EINVAL; }
+  if (c->proj_fp8 && c->dtype != LA_BF16) { msg = "e4m3 projections need the bf16 stream"; return LA_EINVAL; }
   if (c->cache_mode == LA_CACHE_CLEAN_REFRESH && c->schedule != LA_SCHED_SEQUENTIAL) {
     msg = "the clean-cache refresh needs the sequential schedule";
     return LA_EINVAL;
@@ -365,6 +378,21 @@ GemmEpiParams epi(int kind, void* out, float* h32, long long ld) {
   e.rows_per_group = 1 << 30;
   for (int i = 0; i < LA_MAX_STEPS; ++i) e.active[i] = 1;
   return e;
+}
+
+// A projection on e4m3 operands: the bf16 operand a [M, K] is quantized per
+// row into a8 / a8s, then the GEMM runs on its codes and the layer's weight
+// codes (tmW, per-row scales wscale) with the scales ahead of the epilogue.
+int proj_fp8(la_stream* s, int kind, const void* a, const CUtensorMap& tmA8, const CUtensorMap& tmW,
+             const float* wscale, GemmEpiParams ep, int M, int N, int K, const QkvRopeParams* qp = nullptr) {
+  int r = launch(s, LA_KIND_OTHER, [&] { return launch_quant_rows_e4m3(1, a, M, K, s->a8, s->a8s, s->st); });
+  if (r != LA_OK) return r;
+  ep.row_scale = s->a8s;
+  ep.col_scale = wscale;
+  const int bn = gemm_tc_pick_bn(N);
+  return launch(s, kind, [&] {
+    return launch_gemm_tc_fp8(tmA8, tmW, ep, M, N, K, bn, s->dev_err, s->num_sms, s->st, qp);
+  });
 }
 
 char* elem(void* base, long long idx, size_t es) { return static_cast<char*>(base) + idx * static_cast<long long>(es); }
@@ -466,6 +494,16 @@ int run_pass(la_stream* s, const PassDesc& pd) {
   ap.q_prescaled = s->bf16 ? 1 : 0;
 
   for (int l = 0; l < s->L; ++l) {
+    if (s->capture && s->bf16) {
+      // the normalised residual as the QKV projection consumes it (bf16)
+      for (int ai = 0; ai < pd.nactive; ++ai) {
+        const int buf = pd.active_buf[ai];
+        if (pd.step[buf] >= S) continue;
+        CU(cudaMemcpyAsync(elem(s->cap_hop, (static_cast<long long>(pd.step[buf]) * s->L + l) * T * D, s->es),
+                           elem(s->hop, static_cast<long long>(buf) * T * D, s->es), static_cast<size_t>(T) * D * s->es,
+                           cudaMemcpyDeviceToDevice, s->st));
+      }
+    }
     ra.qkv = s->qkv; ra.q_rope = s->q_rope; ra.ring_k = s->ring_k; ra.ring_v = s->ring_v;
     ra.ring_slice0 = static_cast<long long>(l) * S * E;
     ra.sink_k = s->sink_k + static_cast<long long>(l) * H * F * d;
@@ -475,11 +513,16 @@ int run_pass(la_stream* s, const PassDesc& pd) {
       qp.ring_slice0 = ra.ring_slice0;
       GemmEpiParams eq = epi(EPI_QKV_ROPE, nullptr, nullptr, 3LL * D);
       const int bn = gemm_tc_pick_bn(3 * D);
-      if ((r = launch(s, LA_KIND_QKV_GEMM, [&] {
-             return launch_gemm_tc(s->tm_hop, s->tm_wqkv[l], eq, rows, 3 * D, D, bn, s->dev_err, s->num_sms, s->st,
-                                   &qp);
-           })) != LA_OK)
+      if (s->fp8) {
+        if ((r = proj_fp8(s, LA_KIND_QKV_GEMM, s->hop, s->tm_a8, s->tm_wq8[l], s->wq8s[l], eq, rows, 3 * D, D, &qp)) !=
+            LA_OK)
+          return r;
+      } else if ((r = launch(s, LA_KIND_QKV_GEMM, [&] {
+                    return launch_gemm_tc(s->tm_hop, s->tm_wqkv[l], eq, rows, 3 * D, D, bn, s->dev_err, s->num_sms,
+                                          s->st, &qp);
+                  })) != LA_OK) {
         return r;
+      }
       // per-block re-rope of the sink K (fp32 -> bf16, once per active buffer)
       if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_sink_rerope(1, pd, ra, s->st); })) != LA_OK) return r;
     } else {
@@ -513,7 +556,11 @@ int run_pass(la_stream* s, const PassDesc& pd) {
     }
     // output projection + residual, then the next operand (next layer or head)
     GemmEpiParams eo = epi(EPI_RESID, nullptr, s->h32, D);
-    if ((r = gemm(s, LA_KIND_OUT_GEMM, &s->tm_o, &s->tm_wout[l], s->attn_o, s->w_out[l], eo, rows, D, D)) != LA_OK)
+    if (s->fp8) {
+      if ((r = proj_fp8(s, LA_KIND_OUT_GEMM, s->attn_o, s->tm_a8, s->tm_wo8[l], s->wo8s[l], eo, rows, D, D)) != LA_OK)
+        return r;
+    } else if ((r = gemm(s, LA_KIND_OUT_GEMM, &s->tm_o, &s->tm_wout[l], s->attn_o, s->w_out[l], eo, rows, D, D)) !=
+               LA_OK)
       return r;
     if (s->capture && (r = capture_pass(s, pd, l)) != LA_OK) return r;
     const bool last = l == s->L - 1;
@@ -600,10 +647,18 @@ int run_sink(la_stream* s) {
       s->cap_sink_valid = true;
     }
     if ((r = normalise(s, s->s_h32, F, s->s_hop, s->bf16 ? nullptr : s->s_hn32)) != LA_OK) return r;
+    if (s->capture && s->bf16)
+      CU(cudaMemcpyAsync(elem(s->cap_sink_hop, static_cast<long long>(l) * F * D, s->es), s->s_hop,
+                         static_cast<size_t>(F) * D * s->es, cudaMemcpyDeviceToDevice, s->st));
     GemmEpiParams eq = epi(s->bf16 ? EPI_STORE32 : EPI_STORE, s->s_qkv, nullptr, 3LL * D);
-    if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_s_hop, &s->tm_wqkv[l], s->s_hn32, s->w_qkv[l], eq, F, 3 * D, D)) !=
-        LA_OK)
+    if (s->fp8) {
+      if ((r = proj_fp8(s, LA_KIND_QKV_GEMM, s->s_hop, s->tm_s_a8, s->tm_wq8[l], s->wq8s[l], eq, F, 3 * D, D)) !=
+          LA_OK)
+        return r;
+    } else if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_s_hop, &s->tm_wqkv[l], s->s_hn32, s->w_qkv[l], eq, F, 3 * D,
+                         D)) != LA_OK) {
       return r;
+    }
     ra.qkv = s->s_qkv;
     float* kraw = s->sink_k + static_cast<long long>(l) * H * F * d;
     void* vraw = elem(s->sink_v, static_cast<long long>(l) * H * F * d, s->ea);
@@ -623,8 +678,13 @@ int run_sink(la_stream* s) {
       if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) return r;
     }
     GemmEpiParams eo = epi(EPI_RESID, nullptr, s->s_h32, D);
-    if ((r = gemm(s, LA_KIND_OUT_GEMM, &s->tm_s_o, &s->tm_wout[l], s->s_o, s->w_out[l], eo, F, D, D)) != LA_OK)
+    if (s->fp8) {
+      if ((r = proj_fp8(s, LA_KIND_OUT_GEMM, s->s_o, s->tm_s_a8, s->tm_wo8[l], s->wo8s[l], eo, F, D, D)) != LA_OK)
+        return r;
+    } else if ((r = gemm(s, LA_KIND_OUT_GEMM, &s->tm_s_o, &s->tm_wout[l], s->s_o, s->w_out[l], eo, F, D, D)) !=
+               LA_OK) {
       return r;
+    }
   }
   return LA_OK;
 }
@@ -722,6 +782,10 @@ int alloc_capture(la_stream* s) {
   DALLOC(s->cap_o, S * L * T * D * 4);
   DALLOC(s->cap_sk, S * L * H * F * d * s->ea);
   DALLOC(s->cap_sink_h, L * F * D * 4);
+  if (s->bf16) {
+    DALLOC(s->cap_hop, S * L * T * D * s->es);
+    DALLOC(s->cap_sink_hop, L * F * D * s->es);
+  }
   s->cap_valid.assign(s->S, 0);
   return LA_OK;
 }
@@ -775,6 +839,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   s->H = cfg->heads; s->d = cfg->head_dim; s->L = cfg->num_layers;
   s->pt = cfg->rope_split[0]; s->ph = cfg->rope_split[1]; s->pw = cfg->rope_split[2];
   s->bf16 = cfg->dtype == LA_BF16; s->es = s->bf16 ? 2 : 4; s->ea = s->es;
+  s->fp8 = s->bf16 && cfg->proj_fp8;
   s->id_in = w->w_in == nullptr; s->id_head = w->w_head == nullptr;
   s->nbuf = cfg->schedule == LA_SCHED_PIPELINED ? s->S : 1;
   s->st = static_cast<cudaStream_t>(cuda_stream);
@@ -904,6 +969,29 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
     ok = ok && tmap_planes_bf16(&s->maps_sink.v[0], s->sink_v, d, F, H, L, s->err);
     if (!ok) return bail(LA_ECUDA);
   }
+  if (s->fp8) {
+    // weights quantized once per output row; operand buffers for the projections
+    const long long rows_max = std::max(NB * T, F);
+    ALLOC_OR_BAIL(s->a8, rows_max * D);
+    ALLOC_OR_BAIL(s->a8s, rows_max * 4);
+    s->wq8.resize(L); s->wo8.resize(L); s->wq8s.resize(L); s->wo8s.resize(L);
+    s->tm_wq8.resize(L); s->tm_wo8.resize(L);
+    const int bn_qkv = gemm_tc_pick_bn(3 * s->D), bn_d = gemm_tc_pick_bn(s->D);
+    bool ok = tmap_2d_u8(&s->tm_a8, s->a8, NB * T, D, D, 128, s->err) &&
+              tmap_2d_u8(&s->tm_s_a8, s->a8, F, D, D, 128, s->err);
+    for (int l = 0; l < L && ok; ++l) {
+      ALLOC_OR_BAIL(s->wq8[l], 3 * D * D);
+      ALLOC_OR_BAIL(s->wq8s[l], 3 * D * 4);
+      ALLOC_OR_BAIL(s->wo8[l], D * D);
+      ALLOC_OR_BAIL(s->wo8s[l], D * 4);
+      e = launch_quant_rows_e4m3(1, s->w_qkv[l], 3 * D, D, s->wq8[l], s->wq8s[l], s->st);
+      if (e == cudaSuccess) e = launch_quant_rows_e4m3(1, s->w_out[l], D, D, s->wo8[l], s->wo8s[l], s->st);
+      if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
+      ok = tmap_2d_u8(&s->tm_wq8[l], s->wq8[l], 3 * D, D, D, bn_qkv, s->err) &&
+           tmap_2d_u8(&s->tm_wo8[l], s->wo8[l], D, D, D, bn_d, s->err);
+    }
+    if (!ok) return bail(LA_ECUDA);
+  }
   e = cudaStreamSynchronize(s->st);
   if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
   *out = s;
@@ -974,12 +1062,15 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
   const size_t ea = s->ea;
   const bool per_layer = what == LA_TAP_H || what == LA_TAP_Q || what == LA_TAP_O || what == LA_TAP_RING_K ||
                          what == LA_TAP_RING_V || what == LA_TAP_SINK_K || what == LA_TAP_SINK_V ||
-                         what == LA_TAP_SINK_KROPE || what == LA_TAP_SINK_H;
+                         what == LA_TAP_SINK_KROPE || what == LA_TAP_SINK_H || what == LA_TAP_HOP ||
+                         what == LA_TAP_SINK_HOP;
   if (per_layer && (layer < (what == LA_TAP_H ? -1 : 0) || layer >= L)) return fail(s, LA_EINVAL, "bad layer");
   if (slot < 0 || slot >= S) return fail(s, LA_EINVAL, "bad slot");
   const void* src = nullptr;
   long long bytes = 0;
-  const bool needs_capture = what <= LA_TAP_V || what == LA_TAP_SINK_KROPE;
+  const bool needs_capture = what <= LA_TAP_V || what == LA_TAP_SINK_KROPE || what == LA_TAP_HOP;
+  if ((what == LA_TAP_HOP || what == LA_TAP_SINK_HOP) && !s->bf16)
+    return fail(s, LA_EINVAL, "the GEMM-operand taps exist in bf16 streams only");
   if (needs_capture && (!s->cap_xin || s->cap_valid.empty() || !s->cap_valid[slot]))
     return fail(s, LA_ESTATE, "no capture of that slot in the last call");
   switch (what) {
@@ -1002,6 +1093,15 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
       if (!s->cap_sink_valid) return fail(s, LA_ESTATE, "no capture of a sink pass");
       src = s->cap_sink_h + static_cast<long long>(layer) * F * D;
       bytes = F * D * 4;
+      break;
+    case LA_TAP_HOP:
+      src = elem(s->cap_hop, (static_cast<long long>(slot) * L + layer) * T * D, s->es);
+      bytes = T * D * s->es;
+      break;
+    case LA_TAP_SINK_HOP:
+      if (!s->cap_sink_valid) return fail(s, LA_ESTATE, "no capture of a sink pass");
+      src = elem(s->cap_sink_hop, static_cast<long long>(layer) * F * D, s->es);
+      bytes = F * D * s->es;
       break;
     default: return fail(s, LA_EINVAL, "bad tap");
   }

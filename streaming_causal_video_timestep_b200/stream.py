@@ -71,6 +71,7 @@ class LaStream:
         c.sink_mode, c.rolling_rope, c.sink_offset_frames = cfg.sink_mode, cfg.rolling_rope, cfg.sink_offset_frames
         c.schedule, c.dtype = cfg.schedule, self.dtype
         c.cache_mode = getattr(cfg, "cache_mode", 0)
+        c.proj_fp8 = getattr(cfg, "proj_fp8", 0)
         self.cfg = cfg
         self.c = c
         self.T = cfg.frames_per_block * cfg.grid_h * cfg.grid_w
@@ -153,6 +154,7 @@ class LaStream:
             "h": ((T, D), torch.float32), "q": ((H, T, d), dt), "o": ((T, D), dt),
             "ring_k": ((E, H, T, d), dt), "ring_v": ((E, H, T, d), dt), "sink_k": ((H, F, d), dt),
             "sink_v": ((H, F, d), dt), "sink_k_rope": ((H, F, d), dt), "sink_h": ((F, D), torch.float32),
+            "hop": ((T, D), dt), "sink_hop": ((F, D), dt),
         }
         shape, tdt = shapes[what]
         if what in ("q", "ring_k", "ring_v", "sink_v", "sink_k_rope"):

@@ -15,6 +15,7 @@ import numpy as np
 import math
 
 from oracle import block_causal_attention, euler_step, rms_norm, rope_rotate
+from oracle.fp8 import project, quantize_rows
 from oracle.rope import block_positions, sink_positions
 from workloads import DTYPE_BF16, bf16_round
 
@@ -32,6 +33,22 @@ def _normed_operand(h, cfg):
     return _operand(rms_norm(np.asarray(h, np.float64)).astype(np.float32), cfg)
 
 
+_W8 = {}
+
+
+def _proj(a, w, cfg):
+    """A QKV / output projection of the operand a (as the GEMM consumes it): bf16
+    or fp32 GEMM, or with e4m3 projections (cfg.proj_fp8) the quantized operand
+    times the per-row-quantized weights (oracle/fp8.py)."""
+    if not getattr(cfg, "proj_fp8", 0):
+        return a @ np.asarray(w, np.float64).T
+    hit = _W8.get(id(w))
+    if hit is None or hit[0] is not w:
+        hit = (w, quantize_rows(np.asarray(w, np.float32)))
+        _W8[id(w)] = hit
+    return project(a, *hit[1])
+
+
 def check_sink(s, cfg, W, latent, rows=None, tag=""):
     """Per-op check of the last sink pass: in-projection of the sink latent and,
     per layer, the stored un-roped K (fp32) and V from the captured sink residual."""
@@ -44,7 +61,15 @@ def check_sink(s, cfg, W, latent, rows=None, tag=""):
     assert_close(h0[R], want, dt, f"{tag} sink in-proj")
     for l in range(cfg.num_layers):
         hs = to_np(s.tap("sink_h", l))
-        qkv = _normed_operand(hs[R], cfg) @ np.asarray(W.w_qkv[l], np.float64).T
+        op = _normed_operand(hs[R], cfg)
+        if getattr(cfg, "proj_fp8", 0):
+            # e4m3 projections: the normalisation on its own, then the projection
+            # from the operand the GPU quantized (a one-ulp difference there can move
+            # a code, or a row's scale, by a whole e4m3 step)
+            op_gpu = to_np(s.tap("sink_hop", l))[R].astype(np.float64)
+            assert_close(op_gpu, op, dt, f"{tag} sink norm operand l{l}")
+            op = op_gpu
+        qkv = _proj(op, W.w_qkv[l], cfg)
         k = qkv[:, D:2 * D].reshape(len(R), H, d)
         v = qkv[:, 2 * D:].reshape(len(R), H, d)
         assert_close(to_np(s.tap("sink_k", l)).transpose(1, 0, 2)[R], k, dt, f"{tag} sink K l{l}")
@@ -81,8 +106,12 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
     chk(h_in[R], want, "in-proj h")
     h_prev = h_in
     for l in range(L):
-        wqkv = np.asarray(W.w_qkv[l], np.float64)
-        qkv = _normed_operand(h_prev[R], cfg) @ wqkv.T
+        op = _normed_operand(h_prev[R], cfg)
+        if getattr(cfg, "proj_fp8", 0):
+            op_gpu = to_np(s.tap("hop", l, i))[R].astype(np.float64)
+            chk(op_gpu, op, f"norm operand l{l}")
+            op = op_gpu
+        qkv = _proj(op, W.w_qkv[l], cfg)
         q = qkv[:, :D].reshape(len(R), H, d)
         k = qkv[:, D:2 * D].reshape(len(R), H, d)
         v = qkv[:, 2 * D:].reshape(len(R), H, d)
@@ -114,7 +143,7 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
         chk(o_gpu[R], o_want.reshape(len(R), D), f"attn O l{l}")
         # output projection + residual from the attention output as the GEMM consumes it
         h_next = to_np(s.tap("h", l, i))
-        want = h_prev[R].astype(np.float64) + _operand(o_gpu[R], cfg) @ np.asarray(W.w_out[l], np.float64).T
+        want = h_prev[R].astype(np.float64) + _proj(_operand(o_gpu[R], cfg), W.w_out[l], cfg)
         chk(h_next[R], want, f"h l{l}")
         h_prev = h_next
     vel = (rms_norm(h_prev[R].astype(np.float64)) if w_head is None

@@ -239,3 +239,18 @@ def test_small_bf16_clean_cache_refresh_integer_state_and_drift():
     worst = _run_clean_refresh(Workload("small-bf16-clean", cfg, SMALL_BF16.seed, 5, SMALL_BF16.w_std,
                                         SMALL_BF16.head_std))
     print({"free-running drift": (f"{worst[0]:.2e}", f"{worst[1]:.2e}")})
+
+
+def test_small_bf16_stream_with_e4m3_projections_teacher_forced():
+    """e4m3 QKV / output projections: every op of every (block, step) against the
+    oracle's quantize-then-multiply definition, integer state bit-exact."""
+    cfg = SMALL_BF16.cfg.replace(proj_fp8=1)
+    report = _run_teacher_forced(Workload("small-bf16-fp8", cfg, SMALL_BF16.seed, 6, SMALL_BF16.w_std,
+                                          SMALL_BF16.head_std))
+    print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in report.items()})
+
+
+def test_tiny_fp32_stream_rejects_e4m3_projections():
+    from streaming_causal_video_timestep_b200 import LaError
+    with pytest.raises(LaError):
+        make_stream(Workload("tiny-fp8", TINY.cfg.replace(proj_fp8=1), TINY.seed, 2, TINY.w_std, TINY.head_std))

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle.fp8 import E4M3_MAX, e4m3_decode, e4m3_decode_table, e4m3_encode, gemm_fp8, quantize_rows
+from oracle.fp8 import E4M3_MAX, bf16_round_f32, e4m3_decode, e4m3_decode_table, e4m3_encode, gemm_fp8, quantize_rows
 
 
 def _torch_decode(codes):
@@ -82,3 +82,11 @@ def test_gemm_fp8_equals_product_of_torch_decoded_operands():
     ref = (_torch_decode(a).astype(np.float64) @ _torch_decode(w).astype(np.float64).T) \
         * sa[:, None].astype(np.float64) * sw[None, :].astype(np.float64)
     np.testing.assert_allclose(gemm_fp8(a, sa, w, sw), ref, rtol=1e-13, atol=0)
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(6)
+    x = np.concatenate([rng.standard_normal(200000) * 10, rng.standard_normal(1000) * 1e-30,
+                        np.float32([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -0.0, 3.0e38])]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(bf16_round_f32(x), ref)

@@ -60,6 +60,7 @@ class StreamConfig:
     schedule: int = SCHED_PIPELINED
     dtype: int = DTYPE_BF16
     cache_mode: int = CACHE_TIMESTEP
+    proj_fp8: int = 0        # 1: QKV / output projections on per-row-quantized e4m3 operands (bf16 streams)
 
     @property
     def num_steps(self) -> int:
