@@ -26,9 +26,10 @@ What it computes (Live Avatar, arXiv 2512.04677, as described on the pages):
     distilled timesteps (papernotes note, 损失函数 / L_FM);
   * the timestep-pipelined order of the 4 in-flight blocks (10100.com article,
     TPP figure caption; gitcode blog, question 6);
-  * the clean-cache refresh ablation (oracle/schedule.py, oracle/stream.py) and
-    per-row e4m3 quantization with the FP8 GEMM (oracle/fp8.py) for the
-    operator-optimisation row (papernotes note, the paper's Table 3).
+  * the clean-cache refresh ablation (oracle/schedule.py, oracle/stream.py),
+    and per-row e4m3 quantization with the FP8 GEMM plus FP8 attention
+    (oracle/fp8.py) for the operator-optimisation row (papernotes note, the
+    paper's Table 3).
 
 Everything is fp64 numpy with a dict-indexed cache, an explicit mask matrix and
 a naive softmax.  The readings taken where the pages are silent are listed in

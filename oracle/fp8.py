@@ -1,4 +1,4 @@
-"""FP8 (e4m3) quantization and the FP8 GEMM, fp64 (the operator-optimisation row).
+"""FP8 (e4m3) quantization, the FP8 GEMM and FP8 attention, fp64 (the operator-optimisation row).
 
 TEST INFRASTRUCTURE ONLY (see oracle/__init__.py).
 
@@ -96,3 +96,45 @@ def gemm_fp8(a_codes, a_scale, w_codes, w_scale) -> np.ndarray:
     a = e4m3_decode(a_codes)
     w = e4m3_decode(w_codes)
     return (a @ w.T) * np.asarray(a_scale, np.float64)[:, None] * np.asarray(w_scale, np.float64)[None, :]
+
+
+# ---- FP8 attention ---------------------------------------------------------------------
+# P is formed as 2^(s - M + P_BIAS) with s the score in the log2 domain and M the
+# row's largest score rounded UP to an integer, so the row's largest P lies in
+# (2^(P_BIAS-1), 2^P_BIAS]: well inside e4m3's normal range, and far above its
+# subnormal floor (2^-6).  Because M is an integer, scaling P by any power of two
+# (another integer M) scales its e4m3 codes by the same power exactly, as long as
+# the values stay normal and below 448.
+P_BIAS = 5
+
+
+def attention_fp8(q_codes, k_codes, v_codes, q_scale, k_scale, v_scale):
+    """Softmax attention on e4m3 operands with an e4m3 probability matrix, fp64.
+
+    The pages give no FP8 attention scheme beyond naming FP8 quantisation and
+    FlashAttention-3 (papernotes note, the paper's Table 3, last row).  The
+    reading taken, in FlashAttention-3's FP8 form:
+      q = dec(q_codes) * q_scale[h], k and v likewise with their per-head scales;
+      s[i, j] = (q_i . k_j) / sqrt(d) * log2(e)     (the log2 domain)
+      M_i = ceil(max_j s[i, j])
+      p[i, j] = 2^(s[i, j] - M_i + P_BIAS), rounded to float32
+      O_i = sum_j dec(e4m3(p[i, j])) v_j / sum_j p[i, j]
+    i.e. the product P V takes P rounded to e4m3, the normaliser takes the
+    unrounded P.  Every key passed is visible (the block-causal mask is the
+    choice of keys).
+
+    q_codes: uint8 [T, H, d]; k_codes, v_codes: uint8 [N, H, d] (the visible
+    keys, concatenated); scales: [H].  Returns O float64 [T, H, d]."""
+    q_codes = np.asarray(q_codes, np.uint8)
+    T, H, d = q_codes.shape
+    out = np.empty((T, H, d), np.float64)
+    for h in range(H):
+        q = e4m3_decode(q_codes[:, h, :]) * float(q_scale[h])
+        k = e4m3_decode(np.asarray(k_codes, np.uint8)[:, h, :]) * float(k_scale[h])
+        v = e4m3_decode(np.asarray(v_codes, np.uint8)[:, h, :]) * float(v_scale[h])
+        s = (q @ k.T) / np.sqrt(d) * np.log2(np.e)
+        M = np.ceil(s.max(axis=1, keepdims=True))
+        p = np.exp2(s - M + P_BIAS).astype(np.float32)
+        pq = e4m3_decode(e4m3_encode(p))
+        out[:, h, :] = (pq @ v) / p.astype(np.float64).sum(axis=1, keepdims=True)
+    return out

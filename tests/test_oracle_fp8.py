@@ -90,3 +90,105 @@ def test_bf16_rounding_matches_torch():
                         np.float32([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -0.0, 3.0e38])]).astype(np.float32)
     ref = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
     np.testing.assert_array_equal(bf16_round_f32(x), ref)
+
+
+# ---- FP8 attention ---------------------------------------------------------------------
+from oracle.attention import block_causal_attention
+from oracle.fp8 import P_BIAS, attention_fp8
+
+LOG2E = float(np.log2(np.e))
+
+
+def _exact_attention(q_codes, k_codes, v_codes, sq, sk, sv):
+    """Softmax attention of the dequantized operands (the plain oracle, fp64)."""
+    q = e4m3_decode(q_codes) * np.asarray(sq, np.float64)[None, :, None]
+    k = e4m3_decode(k_codes) * np.asarray(sk, np.float64)[None, :, None]
+    v = e4m3_decode(v_codes) * np.asarray(sv, np.float64)[None, :, None]
+    return block_causal_attention(q, {0: (k, v)}, None, qblock=0, window=0)
+
+
+def _gauss_codes(rng, shape, sigma=1.0):
+    return e4m3_encode((rng.standard_normal(shape) * sigma).astype(np.float32))
+
+
+def test_attention_fp8_is_exact_softmax_attention_when_p_is_a_power_of_two():
+    """Scores that are whole numbers in the log2 domain make every P = 2^(s - M + bias) a
+    power of two within e4m3's normal range, so its rounding is exact and the FP8 result
+    must equal plain softmax attention of the dequantized operands."""
+    rng = np.random.default_rng(11)
+    T, N, H, d = 6, 40, 2, 16
+    q = np.zeros((T, H, d), np.uint8)
+    k = np.zeros((N, H, d), np.uint8)
+    q[:, :, 0] = e4m3_encode(rng.choice([1.0, 2.0], size=(T, H)).astype(np.float32))
+    k[:, :, 0] = e4m3_encode(rng.integers(-4, 3, size=(N, H)).astype(np.float32))
+    v = _gauss_codes(rng, (N, H, d))
+    sq = np.float32([1.0, 0.5])
+    # q_scale * k_scale * log2(e) / sqrt(d) = 1 up to the float32 rounding of k_scale
+    sk = (np.float32(np.sqrt(d) / LOG2E) / sq).astype(np.float32)
+    sv = np.float32([0.25, 3.0])
+    got = attention_fp8(q, k, v, sq, sk, sv)
+    ref = _exact_attention(q, k, v, sq, sk, sv)
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-7 * np.abs(ref).max())
+
+
+def test_attention_fp8_single_key_returns_its_value():
+    rng = np.random.default_rng(12)
+    q = _gauss_codes(rng, (5, 1, 32))
+    k = _gauss_codes(rng, (1, 1, 32))
+    v = _gauss_codes(rng, (1, 1, 32))
+    # P of the lone key is 2^(s - ceil(s) + bias), rounded to e4m3 in the product but not
+    # in the normaliser: the output is v times that rounding ratio, within 2^-4 of 1
+    got = attention_fp8(q, k, v, [1.0], [1.0], [2.0])
+    s = (e4m3_decode(q[:, 0]) @ e4m3_decode(k[:, 0]).T) / np.sqrt(32) * LOG2E
+    p = np.exp2(s - np.ceil(s) + P_BIAS).astype(np.float32)
+    ratio = e4m3_decode(e4m3_encode(p)) / p.astype(np.float64)
+    np.testing.assert_allclose(got[:, 0, :], ratio * 2.0 * e4m3_decode(v[0, 0])[None, :], rtol=1e-12)
+    assert np.all(np.abs(ratio - 1) <= 2.0 ** -4)
+
+
+def test_attention_fp8_is_unchanged_by_a_whole_number_shift_of_all_scores():
+    """Adding the same whole number to every score of a row moves M by it and scales
+    every P by a power of two, which e4m3 represents exactly in its normal range."""
+    rng = np.random.default_rng(13)
+    T, N, H, d = 8, 64, 1, 16
+    q = _gauss_codes(rng, (T, H, d), 0.5)
+    k = _gauss_codes(rng, (N, H, d), 0.5)
+    v = _gauss_codes(rng, (N, H, d))
+    q[:, :, d - 1] = e4m3_encode([1.0])[0]
+    sq = np.float32([1.0])
+    sk = np.float32([np.sqrt(d) / LOG2E])
+    outs = []
+    for shift in (0.0, 3.0, -5.0):
+        kk = k.copy()
+        kk[:, :, d - 1] = e4m3_encode([shift])[0]
+        outs.append(attention_fp8(q, kk, v, sq, sk, [1.0]))
+    np.testing.assert_allclose(outs[1], outs[0], rtol=1e-5, atol=1e-9)
+    np.testing.assert_allclose(outs[2], outs[0], rtol=1e-5, atol=1e-9)
+
+
+def test_attention_fp8_error_is_within_the_rounding_bound_of_p():
+    """Against softmax attention of the dequantized operands, the only rounding is P's:
+    at most half an e4m3 unit (2^-4 relative) for normal values, and half the
+    subnormal step (2^-10) below 2^-6, against a normaliser of at least 2^(bias-1)."""
+    rng = np.random.default_rng(14)
+    T, N, H, d = 40, 300, 2, 64
+    q = _gauss_codes(rng, (T, H, d))
+    k = _gauss_codes(rng, (N, H, d))
+    v = _gauss_codes(rng, (N, H, d))
+    for i in range(8):                          # rows dominated by one key
+        j = int(rng.integers(N))
+        q[i] = e4m3_encode(e4m3_decode(k[j]).astype(np.float32) * 2.0)
+    sq, sk, sv = np.float32([1.0, 0.5]), np.float32([0.5, 1.0]), np.float32([1.0, 2.0])
+    got = attention_fp8(q, k, v, sq, sk, sv)
+    ref = _exact_attention(q, k, v, sq, sk, sv)
+    qd = e4m3_decode(q) * sq[None, :, None]
+    kd = e4m3_decode(k) * sk[None, :, None]
+    vd = np.abs(e4m3_decode(v) * sv[None, :, None])
+    for h in range(H):
+        s = qd[:, h] @ kd[:, h].T / np.sqrt(d)
+        w = np.exp(s - s.max(axis=1, keepdims=True))
+        w /= w.sum(axis=1, keepdims=True)
+        bound = np.maximum(2.0 ** -4 * w, 2.0 ** -10 / 2.0 ** (P_BIAS - 1)) @ vd[:, h]
+        assert np.all(np.abs(got[:, h] - ref[:, h]) <= bound * (1 + 1e-6) + 1e-12)
+    # the rounding of P is visible: the result is not the unquantized one
+    assert np.abs(got - ref).max() > 1e-4 * np.abs(ref).max()
