@@ -347,6 +347,34 @@ int la_op_gemm_fp8(const void* a_codes, const float* a_scales, const void* w_cod
                    int64_t K, void* cuda_stream);
 
 /*
+ * FP8 (e4m3) attention, the attention half of the same operator-optimisation
+ * row ("FP8 quantisation + FlashAttention-3"; the pages give no scheme).  The
+ * reading taken is FlashAttention-3's FP8 form: e4m3 q, K, V with one fp32
+ * scale per head each, and an e4m3 probability matrix in P V:
+ *   s[t, j] = (q_code[t] . k_code[j]) * q_scale[h] * k_scale[h] * log2(e)/sqrt(d)
+ *   M[t]    = ceil(max_j s[t, j])            (a whole number)
+ *   p[t, j] = 2^(s[t, j] - M[t] + 5)         (fp32; the row max lies in (16, 32])
+ *   O[t, h*d + e] = v_scale[h] * sum_j e4m3(p[t, j]) v_code[j][e] / sum_j p[t, j]
+ * over the concatenation of the segments (every key visible).  The kernel
+ * keeps M as a running whole number that is raised only when a key tile's
+ * max exceeds it by more than 3; a raise rescales O by an exact power of two,
+ * so the codes of P equal those formed against the final M wherever they are
+ * normal e4m3 values (keys weighing >= 2^-11 of the row's largest).
+ *   q_codes DEVICE uint8 [H, Tq, d]; segment s: k_seg[s], v_seg[s] DEVICE uint8
+ *   [H, seg_len[s], d] (HOST arrays of nseg pointers / lengths, 1 <= nseg <=
+ *   LA_MAX_WINDOW + 2, seg_len >= 1), 16-byte aligned; d == 128.
+ *   q_scale, k_scale, v_scale: DEVICE fp32 [H], positive.
+ *   out DEVICE bf16 [Tq, H*d] (rounded once) and, if out32 != NULL, the fp32
+ *   value [Tq, H*d].
+ * Codes are the caller's (no NaN codes expected).  LA_EINVAL on bad sizes or
+ * NULL pointers; LA_ECUDA if the launch fails.
+ */
+int la_op_attention_fp8(const void* q_codes, int64_t Tq, int32_t H, int32_t d, int32_t nseg,
+                        const void* const* k_seg, const void* const* v_seg,
+                        const int64_t* seg_len, const float* q_scale, const float* k_scale,
+                        const float* v_scale, void* out, float* out32, void* cuda_stream);
+
+/*
  * Block attention for callers that cannot allocate device memory (a plugin
  * whose host application owns all device memory through its own allocator or
  * a fixed budget, or a real-time path where an allocation and its implicit

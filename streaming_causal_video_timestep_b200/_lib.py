@@ -81,6 +81,9 @@ def load():
         "la_op_quantize_e4m3": (c_int, [c_int32, c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
         "la_op_gemm_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int64, c_int64,
                                    c_int64, c_void_p]),
+        "la_op_attention_fp8": (c_int, [c_void_p, c_int64, c_int32, c_int32, c_int32, POINTER(c_void_p),
+                                        POINTER(c_void_p), POINTER(c_int64), c_void_p, c_void_p, c_void_p,
+                                        c_void_p, c_void_p, c_void_p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -97,7 +100,7 @@ def exported_symbols():
         "la_stream_destroy", "la_last_error", "la_status_string", "la_index_state_size", "la_get_index_state",
         "la_debug_capture", "la_debug_tap", "la_debug_set_slot_input", "la_profile_enable", "la_profile_read",
         "la_launch_count", "la_op_gemm", "la_op_attention", "la_op_euler", "la_op_attention_static",
-        "la_debug_wait_timeout", "la_op_quantize_e4m3", "la_op_gemm_fp8",
+        "la_debug_wait_timeout", "la_op_quantize_e4m3", "la_op_gemm_fp8", "la_op_attention_fp8",
     ]
 
 

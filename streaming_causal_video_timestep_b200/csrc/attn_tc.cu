@@ -31,6 +31,18 @@
 // Cody-Waite split into integer and fraction, as in the FlashAttention-4
 // softmax, with a polynomial of our own fit).  Partial tiles (a segment's
 // ragged tail) use ex2 only, so masked keys get exactly 0.
+//
+// FP8 variant (the FP8 template argument): q, K and V are e4m3 codes with one
+// scale per head each, S = Q K^T and O += P V run as kind::f8f6f4 (32 keys or
+// dims a tensor-core step; one 128-byte box per 128 x 128 tile), and P is
+// written to tensor memory as e4m3 (32 columns).  The scores enter the softmax
+// as acc * (sq * sk * log2(e)/sqrt(d)); the running max M is kept as a whole
+// number (the tile max rounded up) and P = 2^(s - M + FP8_P_BIAS), so a row's
+// largest P lies in (16, 32] when M is set and P stays below 2^(FP8_TAU +
+// FP8_P_BIAS) = 256 < 448 until the max grows by more than FP8_TAU.  With M a
+// whole number, a later rescale of O multiplies earlier P codes by an exact
+// power of two, so the codes are those of P formed against the final row max
+// wherever they are normal e4m3 values.  The normaliser sums the unrounded P.
 #include <cstdio>
 #include <cstdlib>
 
@@ -41,16 +53,23 @@ namespace {
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int NS = 5;
 constexpr int THREADS = 384;
 constexpr int LAUNCH_REGS = 168;            // 65536 / 384 rounded down to the allocation unit of 8
 constexpr int REGS_LOW = 56;                // warpgroup 0 after setmaxnreg.dec
 constexpr int REGS_HIGH = 224;              // warpgroups 1-2 after setmaxnreg.inc
 static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * LAUNCH_REGS, "register split exceeds the launch");
 constexpr uint32_t HALF = 16384;            // 128 rows x 128 bytes, one swizzle-128B box
-constexpr uint32_t TILE = 2 * HALF;         // 128 rows x 128 bf16
 constexpr uint32_t TMEM_COLS = 512;
-constexpr size_t SMEM = 1024 + 2 * TILE /*Q_A, Q_B*/ + NS * TILE /*K, V ring*/ + 256;
+constexpr float FP8_P_BIAS = 5.0f;
+constexpr float FP8_TAU = 3.0f;
+
+// A 128 x 128 tile: two boxes of 64 bf16 columns, or one box of 128 e4m3 columns.
+template <bool FP8> __host__ __device__ constexpr uint32_t tile_bytes() { return FP8 ? HALF : 2 * HALF; }
+// Stages of the K/V ring.
+template <bool FP8> __host__ __device__ constexpr int kv_stages() { return FP8 ? 8 : 5; }
+template <bool FP8> __host__ __device__ constexpr size_t smem_bytes() {
+  return 1024 + 2 * tile_bytes<FP8>() /*Q_A, Q_B*/ + kv_stages<FP8>() * tile_bytes<FP8>() /*K, V ring*/ + 256;
+}
 
 __device__ __forceinline__ uint32_t s_col(int w) { return static_cast<uint32_t>(w * 128); }
 __device__ __forceinline__ uint32_t o_col(int w) { return static_cast<uint32_t>(256 + w * 128); }
@@ -150,9 +169,56 @@ __device__ __forceinline__ float softmax_tile(float (&s)[128], uint32_t (&P)[64]
   return a.x + a.y;
 }
 
-template <bool PRESCALED, int EMU>
+// The FP8 form: s[] holds the raw accumulators q_code . k_code; c = sq * sk *
+// log2(e)/sqrt(d) maps them to the log2 domain.  M (m_ref) is a whole number;
+// P = 2^(s c - M + FP8_P_BIAS) as e4m3 codes, four to a 32-bit word (key 4i+b
+// in byte b of P[i]); returns the tile's row sum of the unrounded P.
+template <bool MASKED>
+__device__ __forceinline__ float softmax_tile_fp8(float (&s)[128], uint32_t (&P)[32], int valid, float c,
+                                                  float& m_ref, float& alpha, bool& need) {
+  if (MASKED) {
+#pragma unroll
+    for (int i = 0; i < 128; ++i)
+      if (i >= valid) s[i] = -INFINITY;
+  }
+  float mx[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float a = fmax3(s[32 * q], s[32 * q + 1], s[32 * q + 2]);
+#pragma unroll
+    for (int i = 3; i + 1 < 32; i += 2) a = fmax3(a, s[32 * q + i], s[32 * q + i + 1]);
+    mx[q] = fmaxf(a, s[32 * q + 31]);
+  }
+  const float m_tile = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * c;
+  need = m_tile > m_ref + FP8_TAU;
+  const float m_new = need ? ceilf(m_tile) : m_ref;
+  alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
+  m_ref = m_new;
+  const float2 cc = make_float2(c, c);
+  const float2 off = make_float2(FP8_P_BIAS - m_new, FP8_P_BIAS - m_new);
+  float2 acc[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 x0 = __ffma2_rn(make_float2(s[4 * i], s[4 * i + 1]), cc, off);
+    const float2 x1 = __ffma2_rn(make_float2(s[4 * i + 2], s[4 * i + 3]), cc, off);
+    const float2 p0 = make_float2(fast_exp2(x0.x), fast_exp2(x0.y));
+    const float2 p1 = make_float2(fast_exp2(x1.x), fast_exp2(x1.y));
+    acc[(2 * i) & 3] = __fadd2_rn(acc[(2 * i) & 3], p0);
+    acc[(2 * i + 1) & 3] = __fadd2_rn(acc[(2 * i + 1) & 3], p1);
+    P[i] = pack_e4m3x2(p0.x, p0.y) | (pack_e4m3x2(p1.x, p1.y) << 16);
+  }
+  const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+  const float2 a = __fadd2_rn(a01, a23);
+  return a.x + a.y;
+}
+
+template <bool PRESCALED, int EMU, bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
 k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnParams p) {
+  constexpr uint32_t TILE = tile_bytes<FP8>();
+  constexpr int NS = kv_stages<FP8>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                       // Q_A at 0, Q_B at TILE
@@ -209,7 +275,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       mbar_expect_tx(q_full, 2 * TILE);
       for (int w = 0; w < 2; ++w) {
         tma_load_4d(sQ + w * TILE, &maps.q, q_full, 0, q0 + w * BQ, h, g.q_slice);
-        tma_load_4d(sQ + w * TILE + HALF, &maps.q, q_full, 64, q0 + w * BQ, h, g.q_slice);
+        if (!FP8) tma_load_4d(sQ + w * TILE + HALF, &maps.q, q_full, 64, q0 + w * BQ, h, g.q_slice);
       }
       SegCursor cur;
       int n = 0;
@@ -225,7 +291,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
           uint8_t* dst = sKV + stage * TILE;
           mbar_expect_tx(&kv_full[stage], TILE);
           tma_load_4d(dst, m, &kv_full[stage], 0, cur.start, h, slice);
-          tma_load_4d(dst + HALF, m, &kv_full[stage], 64, cur.start, h, slice);
+          if (!FP8) tma_load_4d(dst + HALF, m, &kv_full[stage], 64, cur.start, h, slice);
           last_parity[stage] = static_cast<int>(par);
           ++n;
         }
@@ -240,20 +306,30 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       // descriptors are precomputed and advanced by adding offsets, pv_done is
       // committed only for the last key tile (the commit of S(t) already covers
       // PV(t-1), issued before it), and the loop polls no flags.
-      constexpr uint32_t idS = idesc_bf16(BQ, BKV, false, false);
-      constexpr uint32_t idPV = idesc_bf16(BQ, 128, false, true);
+      constexpr uint32_t idS = FP8 ? idesc_e4m3(BQ, BKV) : idesc_bf16(BQ, BKV, false, false);
+      constexpr uint32_t idPV = FP8 ? idesc_e4m3(BQ, 128, true) : idesc_bf16(BQ, 128, false, true);
       // The start-address field of a descriptor is (address >> 4) in its low 14
       // bits; every shared address here is below 256 KB, so adding (offset >> 4)
       // moves a descriptor by `offset` bytes without a carry out of the field.
       const uint64_t dQ = sdesc_kmajor(smem_u32(sQ));
       const uint64_t dK = sdesc_kmajor(smem_u32(sKV));
       const uint64_t dV = sdesc_mnmajor(smem_u32(sKV), HALF);
+      // One K step is 32 bytes of a 128-byte row: 16 bf16 or 32 e4m3 head dims.
       auto issue_s = [&](int w, uint32_t stage) {
+        if (FP8) {
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
-          umma_bf16_ss(tmem + s_col(w), dQ + ((w * TILE + off) >> 4), dK + ((stage * TILE + off) >> 4), idS,
-                       kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t off = kk * 32;
+            umma_e4m3_ss(tmem + s_col(w), dQ + ((w * TILE + off) >> 4), dK + ((stage * TILE + off) >> 4), idS,
+                         kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+            umma_bf16_ss(tmem + s_col(w), dQ + ((w * TILE + off) >> 4), dK + ((stage * TILE + off) >> 4), idS,
+                         kk > 0 ? 1u : 0u);
+          }
         }
         umma_commit(&s_full[w]);
       };
@@ -272,10 +348,19 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
         for (int w = 0; w < nq; ++w) {
           if (!mbar_wait(&p_full[w], static_cast<uint32_t>(t & 1), err)) { ok = false; break; }
           tc_fence_after();
+          // One K step is 8 tensor-memory columns of P (16 bf16 or 32 e4m3 keys)
+          // and 16 or 32 key rows of the V tile (128 bytes each).
+          if (FP8) {
 #pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk)
-            umma_bf16_ts(tmem + o_col(w), tmem + s_col(w) + kk * 8, dV + ((vs * TILE + kk * 2048) >> 4), idPV,
-                         (t > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BKV / 32; ++kk)
+              umma_e4m3_ts(tmem + o_col(w), tmem + s_col(w) + kk * 8, dV + ((vs * TILE + kk * 4096) >> 4), idPV,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BKV / 16; ++kk)
+              umma_bf16_ts(tmem + o_col(w), tmem + s_col(w) + kk * 8, dV + ((vs * TILE + kk * 2048) >> 4), idPV,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+          }
           if (more)
             issue_s(w, ks);
           else
@@ -304,6 +389,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
     const uint32_t o_base = tmem + lane_off + o_col(w);
     if (w < nq) {
       float m_ref = -INFINITY, l = 0.f;
+      const float c8 = FP8 ? p.sq[h] * p.sk[h] * p.scale_log2 : 0.f;
       SegCursor cur;
       bool ok = true;
       for (int t = 0; t < nt; ++t) {
@@ -322,7 +408,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
 #pragma unroll
             for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(u[c][i]);
         }
-        if (!PRESCALED) {
+        if (!PRESCALED && !FP8) {
           const float2 sc = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
@@ -331,11 +417,16 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
             s[2 * i + 1] = v.y;
           }
         }
-        uint32_t P[64];
+        uint32_t P[FP8 ? 32 : 64];
         float alpha;
         bool need;
-        const float rs = valid == BKV ? softmax_tile<false, EMU>(s, P, valid, m_ref, alpha, need)
-                                      : softmax_tile<true, EMU>(s, P, valid, m_ref, alpha, need);
+        float rs;
+        if constexpr (FP8)
+          rs = valid == BKV ? softmax_tile_fp8<false>(s, P, valid, c8, m_ref, alpha, need)
+                            : softmax_tile_fp8<true>(s, P, valid, c8, m_ref, alpha, need);
+        else
+          rs = valid == BKV ? softmax_tile<false, EMU>(s, P, valid, m_ref, alpha, need)
+                            : softmax_tile<true, EMU>(s, P, valid, m_ref, alpha, need);
         if (t >= 1 && __any_sync(0xffffffffu, need)) {
           // O is stable: the commit that signalled S(t) also covers PV(t-1), issued before it
 #pragma unroll 1
@@ -349,7 +440,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
           }
         }
         tmem_st32(s_base, *reinterpret_cast<uint32_t(*)[32]>(P));
-        tmem_st32(s_base + 32, *reinterpret_cast<uint32_t(*)[32]>(P + 32));
+        if constexpr (!FP8) tmem_st32(s_base + 32, *reinterpret_cast<uint32_t(*)[32]>(P + 32));
         tmem_st_wait();
         l = l * alpha + rs;
         tc_fence_before();
@@ -359,7 +450,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       if (!ok) abort_flag = 1;
       if (ok && nt > 0 && mbar_wait(&pv_done[w], 0, err)) {   // committed once, after the last PV
         tc_fence_after();
-        const float inv = 1.0f / l;
+        const float inv = FP8 ? p.sv[h] / l : 1.0f / l;
         const int qrow = q0 + w * BQ + r;
         const bool store = qrow < p.Tq;
         const long long orow_idx = static_cast<long long>(g.out_row0) + qrow;
@@ -404,9 +495,10 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
   }
 }
 
-template <bool PRESCALED, int EMU>
+template <bool PRESCALED, int EMU, bool FP8 = false>
 cudaError_t launch_variant(const AttnMaps& maps, const AttnParams& p, cudaStream_t st) {
-  auto kern = k_attn_tc<PRESCALED, EMU>;
+  auto kern = k_attn_tc<PRESCALED, EMU, FP8>;
+  constexpr size_t SMEM = smem_bytes<FP8>();
   // The register split above assumes the kernel launches with exactly
   // LAUNCH_REGS registers a thread; with fewer, setmaxnreg.inc could not be
   // satisfied, so refuse to launch.
@@ -438,6 +530,10 @@ int emu_setting() {
 }  // namespace
 
 cudaError_t launch_attention_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st) {
+  if (p.fp8) {
+    if (!p.sq || !p.sk || !p.sv) return cudaErrorInvalidValue;
+    return launch_variant<false, 0, true>(maps, p, st);
+  }
   const bool pre = p.q_prescaled != 0;
   switch (emu_setting()) {
     case 0: return pre ? launch_variant<true, 0>(maps, p, st) : launch_variant<false, 0>(maps, p, st);

@@ -57,6 +57,10 @@ struct AttnParams {
   int H, d;
   float scale_log2;     // log2(e) / sqrt(d)
   int q_prescaled;      // q already multiplied by scale_log2 (tcgen05 path)
+  int fp8;              // q/K/V are e4m3 codes (tcgen05 path): value = code * scale of its head
+  const float* sq;      // fp8: DEVICE [H] scales of q, K, V
+  const float* sk;
+  const float* sv;
   void* out;            // [rows, H*d] bf16 (tcgen05 path) / fp32 (SIMT path)
   float* out32;         // optional fp32 copy of the output (tcgen05 path)
   long long out_ld;     // elements per output row

@@ -24,7 +24,8 @@ cudaError_t launch_quant_rows_e4m3(int bf16_in, const void* x, long long rows, l
                                    float* scale, cudaStream_t st);
 
 // Tensor maps of an attention launch: q (d, Tq, H, q slices) and k[m]/v[m]
-// (d, rows_m, H, slices), bf16, 128-byte swizzle, box (64, 128, 1, 1).
+// (d, rows_m, H, slices), 128-byte swizzle: bf16 with box (64, 128, 1, 1), or
+// e4m3 codes (p.fp8) with box (128, 128, 1, 1).
 struct AttnMaps {
   CUtensorMap q;
   CUtensorMap k[LA_MAX_SEG];
@@ -33,6 +34,7 @@ struct AttnMaps {
 // Block-causal attention over the segments of each group (two 128-query tiles
 // per CTA).  LA_ATTN_EMU=k in the environment (k in {0, 2, 3, 4}; default 0)
 // computes k of every 8 exponential pairs of full key tiles on the FMA pipe.
+// p.fp8: e4m3 q/K/V with per-head scales p.sq / p.sk / p.sv (kind::f8f6f4).
 cudaError_t launch_attention_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st);
 
 // ---- SIMT fp32 -----------------------------------------------------------------------

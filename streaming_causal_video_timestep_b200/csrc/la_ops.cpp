@@ -103,6 +103,41 @@ int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t
   return ret(launch_attn_f32(p, st));
 }
 
+int la_op_attention_fp8(const void* q_codes, int64_t Tq, int32_t H, int32_t d, int32_t nseg,
+                        const void* const* k_seg, const void* const* v_seg, const int64_t* seg_len,
+                        const float* q_scale, const float* k_scale, const float* v_scale, void* out, float* out32,
+                        void* cuda_stream) {
+  if (!q_codes || !out || !k_seg || !v_seg || !seg_len || !q_scale || !k_scale || !v_scale) return LA_EINVAL;
+  if (Tq < 1 || Tq > (1 << 30) || H < 1 || H > 65535 || d != 128 || nseg < 1 || nseg > LA_MAX_SEG) return LA_EINVAL;
+  for (int s = 0; s < nseg; ++s)
+    if (!k_seg[s] || !v_seg[s] || seg_len[s] < 1 || seg_len[s] > (1 << 30)) return LA_EINVAL;
+  AttnParams p{};
+  p.ngroups = 1;
+  p.Tq = static_cast<int>(Tq);
+  p.H = H;
+  p.d = d;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  p.fp8 = 1;
+  p.sq = q_scale;
+  p.sk = k_scale;
+  p.sv = v_scale;
+  p.out = out;
+  p.out32 = out32;
+  p.out_ld = static_cast<long long>(H) * d;
+  AttnGroup& g = p.g[0];
+  g.nseg = nseg;
+  for (int s = 0; s < nseg; ++s) g.seg[s] = AttnSeg{s, s, 0, 0, static_cast<int>(seg_len[s])};
+  std::string err;
+  if (!tmap_init(err)) return LA_ECUDA;
+  AttnMaps maps;
+  if (!tmap_planes_u8(&maps.q, q_codes, d, Tq, H, 1, err)) return LA_ECUDA;
+  for (int s = 0; s < nseg; ++s) {
+    if (!tmap_planes_u8(&maps.k[s], k_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
+    if (!tmap_planes_u8(&maps.v[s], v_seg[s], d, seg_len[s], H, 1, err)) return LA_ECUDA;
+  }
+  return ret(launch_attention_tc(maps, p, static_cast<cudaStream_t>(cuda_stream)));
+}
+
 int la_op_quantize_e4m3(int32_t in_dtype, const void* x, int64_t rows, int64_t cols, void* codes, float* scales,
                         void* cuda_stream) {
   if (!x || !codes || !scales || rows < 1 || rows > (1LL << 31) - 1 || cols < 2 || cols % 2 != 0) return LA_EINVAL;

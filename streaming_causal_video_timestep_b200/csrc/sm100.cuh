@@ -147,6 +147,18 @@ __device__ __forceinline__ void umma_e4m3_ss(uint32_t d_tmem, uint64_t a_desc, u
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f8f6f4: A (K-major, e4m3) read from
+// tensor memory, row m in lane m, four 8-bit elements per 32-bit column
+// (element k in byte k % 4 of column k / 4).
+__device__ __forceinline__ void umma_e4m3_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive on an mbarrier once all previously issued tcgen05 ops of this thread completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -230,9 +242,11 @@ __host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, bool a_mn_maj
 
 // Instruction descriptor, kind::f8f6f4 with fp32 D and both operands e4m3
 // (format code 0 in the A and B fields; same field layout as kind::f16).
-__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+// b_mn_major: B stored MN-major (valid for 8-bit formats as for 16-bit ones).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major = false) {
   return (1u << 4)                                     // D format F32
          | (0u << 7) | (0u << 10)                      // A, B format E4M3
+         | ((b_mn_major ? 1u : 0u) << 16)              // B major
          | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);      // M / 16
 }
@@ -252,6 +266,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+// Two fp32 values to a pair of e4m3 codes (OCP E4M3, round to nearest even,
+// saturating at +-448): lo in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

@@ -72,3 +72,11 @@ bool tmap_planes_bf16(CUtensorMap* m, const void* base, uint64_t d, uint64_t row
   const cuuint32_t box[4] = {64, 128, 1, 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, err);
 }
+
+bool tmap_planes_u8(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint64_t H, uint64_t slices,
+                    std::string& err) {
+  const cuuint64_t dims[4] = {d, rows, H, slices};
+  const cuuint64_t strides[3] = {d, rows * d, H * rows * d};
+  const cuuint32_t box[4] = {128, 128, 1, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, err);
+}

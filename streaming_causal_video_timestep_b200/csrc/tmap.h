@@ -24,3 +24,8 @@ bool tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, 
 // (64, 128, 1, 1), 128-byte swizzle; rows beyond `rows` read as zero.
 bool tmap_planes_bf16(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint64_t H, uint64_t slices,
                      std::string& err);
+// 8-bit (e4m3 codes) stack of [H, rows, d] planes, d = 128: dims (d, rows, H,
+// slices), dense; box (128, 128, 1, 1), 128-byte swizzle; rows beyond `rows`
+// read as zero.
+bool tmap_planes_u8(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint64_t H, uint64_t slices,
+                    std::string& err);

@@ -5,10 +5,12 @@
     python -m streaming_causal_video_timestep_b200.microbench euler [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench rerope [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench gemm_fp8 [--iters N]
+    python -m streaming_causal_video_timestep_b200.microbench attn_fp8 [--iters N]
 
 attn : one block's attention in steady state at the 14B-like shape: 4680
        queries x 40 heads x 128 over [sink 1560 | 2 window blocks | block]
        = 15,600 keys (the per-slot launch of the stream), q pre-scaled.
+attn_fp8: the same attention on e4m3 q/K/V (per-head scales, e4m3 P).
 gemm : the QKV projection of one block, [4680, 5120] x [15360, 5120]^T.
 euler: x += dt * v over 2^20 rows x 64 fp32 (256 MB per tensor), 4 groups.
 gemm_fp8: the QKV projection shape on e4m3 operands (kind::f8f6f4, per-row
@@ -26,7 +28,7 @@ import json
 
 import torch
 
-from .stream import op_attention, op_euler, op_gemm, op_gemm_fp8, op_quantize_e4m3
+from .stream import op_attention, op_attention_fp8, op_euler, op_gemm, op_gemm_fp8, op_quantize_e4m3
 
 
 def _time(fn, iters, warmup=3):
@@ -54,6 +56,24 @@ def bench_attn(iters):
     ms = _time(lambda: op_attention(q, ks, vs, out, q_scaled=True), iters)
     flops = 4.0 * T * (F + (nw + 1) * T) * d * H
     return {"mode": "attn", "shape": f"{T} q x {F + (nw + 1) * T} keys x {H}x{d}", "ms": round(ms, 4),
+            "tflops": round(flops / ms / 1e9, 1), "flops": flops}
+
+
+def bench_attn_fp8(iters):
+    H, d, T, F, nw = 40, 128, 4680, 1560, 2
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    rnd = lambda *s: torch.randn(*s, generator=g, device="cuda").to(torch.float8_e4m3fn).view(torch.uint8)
+    q = rnd(H, T, d)
+    ks = [rnd(H, F, d)] + [rnd(H, T, d) for _ in range(nw + 1)]
+    vs = [rnd(H, F, d)] + [rnd(H, T, d) for _ in range(nw + 1)]
+    sq = torch.ones(H, device="cuda")
+    sk = torch.ones(H, device="cuda")
+    sv = torch.ones(H, device="cuda")
+    out = torch.empty((T, H * d), dtype=torch.bfloat16, device="cuda")
+    ms = _time(lambda: op_attention_fp8(q, ks, vs, sq, sk, sv, out), iters)
+    flops = 4.0 * T * (F + (nw + 1) * T) * d * H
+    return {"mode": "attn_fp8", "shape": f"{T} q x {F + (nw + 1) * T} keys x {H}x{d} e4m3", "ms": round(ms, 4),
             "tflops": round(flops / ms / 1e9, 1), "flops": flops}
 
 
@@ -136,12 +156,12 @@ def bench_rerope(iters):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("mode", choices=["attn", "gemm", "euler", "rerope", "gemm_fp8", "all"])
+    ap.add_argument("mode", choices=["attn", "attn_fp8", "gemm", "euler", "rerope", "gemm_fp8", "all"])
     ap.add_argument("--iters", type=int, default=10)
     args = ap.parse_args()
-    modes = ["attn", "gemm", "gemm_fp8", "euler", "rerope"] if args.mode == "all" else [args.mode]
+    modes = ["attn", "attn_fp8", "gemm", "gemm_fp8", "euler", "rerope"] if args.mode == "all" else [args.mode]
     for m in modes:
-        r = {"attn": bench_attn, "gemm": bench_gemm, "euler": bench_euler, "rerope": bench_rerope,
+        r = {"attn": bench_attn, "attn_fp8": bench_attn_fp8, "gemm": bench_gemm, "euler": bench_euler, "rerope": bench_rerope,
              "gemm_fp8": bench_gemm_fp8}[m](args.iters)
         print(json.dumps(r), flush=True)
 

@@ -238,3 +238,17 @@ def op_gemm_fp8(a_codes, a_scales, w_codes, w_scales, out, stream=None):
     N = w_codes.shape[0]
     check(lib.la_op_gemm_fp8(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes), _ptr(w_scales), _ptr(out),
                              _dtype_code(out.dtype), M, N, K, _stream_handle(stream)))
+
+
+def op_attention_fp8(q_codes, ks, vs, q_scale, k_scale, v_scale, out, out32=None, stream=None):
+    """FP8 attention: q_codes [H, Tq, 128] uint8 e4m3; ks / vs lists of uint8 [H, len, 128];
+    q_scale / k_scale / v_scale fp32 [H] CUDA tensors; out bf16 [Tq, H*128], out32 optional
+    fp32 copy."""
+    lib = load()
+    H, Tq, d = q_codes.shape
+    n = len(ks)
+    kp = (c_void_p * n)(*[k.data_ptr() for k in ks])
+    vp = (c_void_p * n)(*[v.data_ptr() for v in vs])
+    ln = (c_int64 * n)(*[k.shape[1] for k in ks])
+    check(lib.la_op_attention_fp8(_ptr(q_codes), Tq, H, d, n, kp, vp, ln, _ptr(q_scale), _ptr(k_scale),
+                                  _ptr(v_scale), _ptr(out), _ptr(out32), _stream_handle(stream)))

@@ -120,6 +120,17 @@ def test_op_entry_points_reject_bad_sizes(lib):
     assert lib.la_op_gemm(0, 0, None, None, None, None, 0, 0, 0, None, 0, None) == _lib.LA_EINVAL
     assert lib.la_op_euler(None, None, 0, 0, None, 0, None) == _lib.LA_EINVAL
     assert lib.la_op_attention(0, None, 0, 0, 0, 0, None, None, None, None, None, 0, None) == _lib.LA_EINVAL
+    # FP8 attention: NULL pointers, and head_dim other than 128 with every pointer set
+    assert lib.la_op_attention_fp8(None, 0, 0, 0, 0, None, None, None, None, None, None, None, None,
+                                   None) == _lib.LA_EINVAL
+    buf = ctypes.c_void_p(16)
+    ptrs = (ctypes.c_void_p * 1)(16)
+    lens = (ctypes.c_int64 * 1)(128)
+    assert lib.la_op_attention_fp8(buf, 128, 1, 64, 1, ptrs, ptrs, lens, buf, buf, buf, buf, None,
+                                   None) == _lib.LA_EINVAL
+    lens0 = (ctypes.c_int64 * 1)(0)
+    assert lib.la_op_attention_fp8(buf, 128, 1, 128, 1, ptrs, ptrs, lens0, buf, buf, buf, buf, None,
+                                   None) == _lib.LA_EINVAL
 
 
 def test_valid_config_without_gpu_fails_loudly(lib):
