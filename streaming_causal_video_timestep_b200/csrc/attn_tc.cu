@@ -169,11 +169,24 @@ __device__ __forceinline__ float softmax_tile(float (&s)[128], uint32_t (&P)[64]
   return a.x + a.y;
 }
 
+// Four fp32 values to four e4m3 codes in one 32-bit word, value b in byte b.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float2 lo, float2 hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\t"
+      "mov.b32 %0, {l, h};\n\t}"
+      : "=r"(r)
+      : "f"(lo.x), "f"(lo.y), "f"(hi.x), "f"(hi.y));
+  return r;
+}
+
 // The FP8 form: s[] holds the raw accumulators q_code . k_code; c = sq * sk *
 // log2(e)/sqrt(d) maps them to the log2 domain.  M (m_ref) is a whole number;
 // P = 2^(s c - M + FP8_P_BIAS) as e4m3 codes, four to a 32-bit word (key 4i+b
-// in byte b of P[i]); returns the tile's row sum of the unrounded P.
-template <bool MASKED>
+// in byte b of P[i]); returns the tile's row sum of the unrounded P.  On full
+// tiles EMU of every 8 pairs take the polynomial exp2 on the FMA pipe.
+template <bool MASKED, int EMU>
 __device__ __forceinline__ float softmax_tile_fp8(float (&s)[128], uint32_t (&P)[32], int valid, float c,
                                                   float& m_ref, float& alpha, bool& need) {
   if (MASKED) {
@@ -201,13 +214,19 @@ __device__ __forceinline__ float softmax_tile_fp8(float (&s)[128], uint32_t (&P)
   for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    const float2 x0 = __ffma2_rn(make_float2(s[4 * i], s[4 * i + 1]), cc, off);
-    const float2 x1 = __ffma2_rn(make_float2(s[4 * i + 2], s[4 * i + 3]), cc, off);
-    const float2 p0 = make_float2(fast_exp2(x0.x), fast_exp2(x0.y));
-    const float2 p1 = make_float2(fast_exp2(x1.x), fast_exp2(x1.y));
-    acc[(2 * i) & 3] = __fadd2_rn(acc[(2 * i) & 3], p0);
-    acc[(2 * i + 1) & 3] = __fadd2_rn(acc[(2 * i + 1) & 3], p1);
-    P[i] = pack_e4m3x2(p0.x, p0.y) | (pack_e4m3x2(p1.x, p1.y) << 16);
+    float2 pp[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int j = 2 * i + h2;              // pair index 0..63
+      const float2 x = __ffma2_rn(make_float2(s[2 * j], s[2 * j + 1]), cc, off);
+      if (!MASKED && (j & 7) >= 8 - EMU) {
+        pp[h2] = exp2_poly2(x);
+      } else {
+        pp[h2] = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+      }
+      acc[j & 3] = __fadd2_rn(acc[j & 3], pp[h2]);
+    }
+    P[i] = pack_e4m3x4(pp[0], pp[1]);
   }
   const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
   const float2 a = __fadd2_rn(a01, a23);
@@ -422,8 +441,8 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
         bool need;
         float rs;
         if constexpr (FP8)
-          rs = valid == BKV ? softmax_tile_fp8<false>(s, P, valid, c8, m_ref, alpha, need)
-                            : softmax_tile_fp8<true>(s, P, valid, c8, m_ref, alpha, need);
+          rs = valid == BKV ? softmax_tile_fp8<false, EMU>(s, P, valid, c8, m_ref, alpha, need)
+                            : softmax_tile_fp8<true, EMU>(s, P, valid, c8, m_ref, alpha, need);
         else
           rs = valid == BKV ? softmax_tile<false, EMU>(s, P, valid, m_ref, alpha, need)
                             : softmax_tile<true, EMU>(s, P, valid, m_ref, alpha, need);
@@ -532,7 +551,12 @@ int emu_setting() {
 cudaError_t launch_attention_tc(const AttnMaps& maps, const AttnParams& p, cudaStream_t st) {
   if (p.fp8) {
     if (!p.sq || !p.sk || !p.sv) return cudaErrorInvalidValue;
-    return launch_variant<false, 0, true>(maps, p, st);
+    switch (emu_setting()) {
+      case 0: return launch_variant<false, 0, true>(maps, p, st);
+      case 2: return launch_variant<false, 2, true>(maps, p, st);
+      case 4: return launch_variant<false, 4, true>(maps, p, st);
+      default: return launch_variant<false, 3, true>(maps, p, st);
+    }
   }
   const bool pre = p.q_prescaled != 0;
   switch (emu_setting()) {
