@@ -116,6 +116,18 @@ typedef struct la_config {
                                   accumulate, scales applied before the epilogue.  The
                                   pages' FP8 row (papernotes note, the paper's Table 3).
                                   0: bf16 projections.                                   */
+  int32_t attn_fp8;            /* 1 (LA_BF16, head_dim 128 only): the denoising passes'
+                                  attention runs on e4m3 q / K / V (la_op_attention_fp8's
+                                  definition): the QKV epilogue, the sink re-rope and the
+                                  sink V store e4m3 codes of value / scale, with one
+                                  power-of-two scale per (layer, q|K|V, head) fixed at
+                                  creation: the smallest 2^k >= bound / 448, where bound =
+                                  1.07 sqrt(hidden) times the largest norm of the head's
+                                  QKV weight rows (of a rotary pair of rows for q and K),
+                                  a bound on |value| for any RMS-normalised input (the
+                                  1.07 covers the rounding of the GEMM operand).  The
+                                  sink's own pass keeps bf16 attention.  Same row as
+                                  proj_fp8.  0: bf16 attention.                          */
 } la_config;
 
 /*
@@ -228,6 +240,10 @@ int la_debug_capture(la_stream* s, int32_t enable);
 #define LA_TAP_HOP       12 /* bf16 [T_b, D] normalised residual as the QKV projection of layer
                                `layer` consumed it at the slot's step (bf16 streams)             */
 #define LA_TAP_SINK_HOP  13 /* bf16 [F, D] the same in the last sink pass (slot ignored)         */
+/* With attn_fp8 the Q, RING_K, RING_V and SINK_KROPE taps hold uint8 e4m3 codes
+ * (value = code * scale of its layer, part and head; Q not pre-scaled), and: */
+#define LA_TAP_SINK_V8   14 /* uint8 [H, F, d] e4m3 codes of the sink V of layer (slot ignored) */
+#define LA_TAP_ATTN_SCALES 15 /* fp32 [3, H] scales of q, K, V of layer (slot ignored)          */
 
 /* Copy one tapped tensor into dst (DEVICE, dst_bytes >= the tensor's size),
  * ordered on the stream.  Taps other than ring / sink need capture enabled

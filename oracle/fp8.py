@@ -138,3 +138,49 @@ def attention_fp8(q_codes, k_codes, v_codes, q_scale, k_scale, v_scale):
         pq = e4m3_decode(e4m3_encode(p))
         out[:, h, :] = (pq @ v) / p.astype(np.float64).sum(axis=1, keepdims=True)
     return out
+
+
+# ---- e4m3 attention operands of the stream -------------------------------------------------
+ATTN_ACT_BOUND = 1.07
+
+
+def pow2_at_least(x: float) -> float:
+    """The smallest power of two >= x > 0."""
+    mant, ex = np.frexp(x)                  # x = mant * 2^ex, mant in [1/2, 1)
+    return float(np.ldexp(1.0, int(ex) - 1 if mant == 0.5 else int(ex)))
+
+
+def attn_fp8_scales(w_qkv, D: int, H: int, d: int) -> np.ndarray:
+    """Per-head power-of-two scales [3, H] (q, K, V) of the stream's e4m3 attention
+    operands (a reading: the pages give no FP8 scheme).  An RMS-normalised row has
+    norm <= sqrt(D); its rounding to the GEMM operand grows each element by less
+    than 7 % (bf16: 2^-8; per-row e4m3: 2^-4 plus the subnormal floor), so
+        |value of output row j| <= 1.07 sqrt(D) ||w_j||
+    by Cauchy-Schwarz, and a rotary pair (2m, 2m+1) of q or K, which RoPE mixes, is
+    bounded by 1.07 sqrt(D) ||(w_2m, w_2m+1)||.  The head's scale is the smallest
+    power of two with (largest bound) / scale <= 448, e4m3's largest value.
+    w_qkv: the weight as the projection uses it, [3D, D] values."""
+    w = np.asarray(w_qkv, np.float64)
+    n2 = np.einsum("ij,ij->i", w, w)
+    out = np.ones((3, H), np.float64)
+    for part in range(3):
+        for h in range(H):
+            rows = n2[part * D + h * d: part * D + (h + 1) * d]
+            m = (rows[0::2] + rows[1::2]).max() if part < 2 else rows.max()
+            bound = ATTN_ACT_BOUND * np.sqrt(D) * np.sqrt(m)
+            if bound > 0:
+                out[part, h] = pow2_at_least(bound / E4M3_MAX)
+    return out.astype(np.float32)
+
+
+def quantize_heads(x, scales) -> np.ndarray:
+    """e4m3 codes of x [N, H, d] over its head's scale: e4m3(float32(x) / scale[h])
+    (the division by a power of two is exact)."""
+    x = np.asarray(x, np.float64).astype(np.float32)
+    return e4m3_encode(x / np.asarray(scales, np.float32)[None, :, None])
+
+
+def dequantize_weight(codes_scales):
+    """The weight a per-row e4m3 projection multiplies by: dec(codes) * row scale."""
+    codes, scales = codes_scales
+    return e4m3_decode(codes) * np.asarray(scales, np.float64)[:, None]

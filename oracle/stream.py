@@ -37,6 +37,13 @@ e4m3 projections (cfg.proj_fp8; the pages' FP8 row, papernotes note, the
 paper's Table 3): the QKV and output projections take their operand as the
 bf16 stream's GEMM consumes it (bf16), quantize it per token and multiply
 e4m3 codes (oracle/fp8.py); everything else is unchanged.
+
+e4m3 attention (cfg.attn_fp8, the same row): in the denoising passes, q, the
+roped K and V of every block, the re-roped sink K and the sink V are held as
+e4m3 codes over one power-of-two scale per (layer, q|K|V, head) fixed from the
+weights (oracle/fp8.py attn_fp8_scales), and the attention is
+oracle/fp8.py attention_fp8 over [sink | window oldest first | block].  The
+sink's own pass keeps the plain attention.
 """
 from __future__ import annotations
 
@@ -44,7 +51,7 @@ import numpy as np
 
 from .attention import block_causal_attention
 from .flow import euler_step
-from .fp8 import project, quantize_rows
+from .fp8 import attention_fp8, attn_fp8_scales, dequantize_weight, project, quantize_heads, quantize_rows
 from .norm import rms_norm
 from .rope import block_positions, rope_rotate, sink_positions
 from .schedule import TickScheduler
@@ -62,6 +69,11 @@ class OracleStream:
         fp8 = getattr(cfg, "proj_fp8", 0)
         self.wq8 = [quantize_rows(np.asarray(w, np.float32)) for w in weights.w_qkv] if fp8 else None
         self.wo8 = [quantize_rows(np.asarray(w, np.float32)) for w in weights.w_out] if fp8 else None
+        # e4m3 attention (cfg.attn_fp8): per-head scales from the weights the QKV projection uses
+        self.attn_sc = None
+        if getattr(cfg, "attn_fp8", 0):
+            used = [dequantize_weight(q) for q in self.wq8] if fp8 else self.w_qkv
+            self.attn_sc = [attn_fp8_scales(w, cfg.hidden, cfg.heads, cfg.head_dim) for w in used]
         self.sched = TickScheduler(cfg)
         self.cache = {}            # (layer, ring, block) -> (k_roped, v, (block, step))
         self.sink_k = None         # per layer, un-roped [F, H, d]
@@ -140,13 +152,25 @@ class OracleStream:
             q, k, v = self._split_heads(self._proj_qkv(l, rms_norm(h)))
             qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
             kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
-            self.cache[(l, ring, b)] = (kr, v.copy(), (b, c.num_steps if refresh else i))
+            sc = self.attn_sc[l] if self.attn_sc is not None else None
+            if sc is not None:                 # the cache holds e4m3 codes
+                self.cache[(l, ring, b)] = (quantize_heads(kr, sc[1]), quantize_heads(v, sc[2]),
+                                            (b, c.num_steps if refresh else i))
+            else:
+                self.cache[(l, ring, b)] = (kr, v.copy(), (b, c.num_steps if refresh else i))
             self.cache.pop((l, ring, b - c.window_blocks - 1), None)
             sk = rope_rotate(self.sink_k[l], st, sh, sw, c.pairs, c.rope_theta)
             blocks = {bb: (kk, vv) for (ll, rr, bb), (kk, vv, _) in self.cache.items()
                       if ll == l and rr == ring}
-            o = block_causal_attention(qr, blocks, (sk, self.sink_v[l]), qblock=b,
-                                       window=c.window_blocks)
+            if sc is not None:
+                # [sink | window oldest first | block]: every assembled key is visible
+                order = sorted(bb for bb in blocks if b - c.window_blocks <= bb <= b)
+                keys = np.concatenate([quantize_heads(sk, sc[1])] + [blocks[bb][0] for bb in order])
+                vals = np.concatenate([quantize_heads(self.sink_v[l], sc[2])] + [blocks[bb][1] for bb in order])
+                o = attention_fp8(quantize_heads(qr, sc[0]), keys, vals, sc[0], sc[1], sc[2])
+            else:
+                o = block_causal_attention(qr, blocks, (sk, self.sink_v[l]), qblock=b,
+                                           window=c.window_blocks)
             h = h + self._proj_out(l, o.reshape(h.shape[0], -1))
             if tr is not None:
                 tr[("layer", l)] = dict(q=qr, k=kr, v=v.copy(), sink_k=sk, o=o, h=h.copy())

@@ -169,18 +169,6 @@ __device__ __forceinline__ float softmax_tile(float (&s)[128], uint32_t (&P)[64]
   return a.x + a.y;
 }
 
-// Four fp32 values to four e4m3 codes in one 32-bit word, value b in byte b.
-__device__ __forceinline__ uint32_t pack_e4m3x4(float2 lo, float2 hi) {
-  uint32_t r;
-  asm("{\n\t.reg .b16 l, h;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\t"
-      "mov.b32 %0, {l, h};\n\t}"
-      : "=r"(r)
-      : "f"(lo.x), "f"(lo.y), "f"(hi.x), "f"(hi.y));
-  return r;
-}
-
 // The FP8 form: s[] holds the raw accumulators q_code . k_code; c = sq * sk *
 // log2(e)/sqrt(d) maps them to the log2 domain.  M (m_ref) is a whole number;
 // P = 2^(s c - M + FP8_P_BIAS) as e4m3 codes, four to a 32-bit word (key 4i+b

@@ -92,6 +92,8 @@ struct QkvRopeParams {
   const float* ccos; const float* csin;   // [grid_w][pw]
   void* q_rope;              // [nbuf][H][T][d]
   void* ring_k; void* ring_v;// [L][S][E][H][T][d]
+  const float* fp8_inv;      // NULL, or [3][H] inverse scales of q, K, V: write e4m3 codes of
+                             // (roped) value * inverse scale instead of bf16 (q not pre-scaled)
 };
 
 struct GemmEpiParams {

@@ -187,7 +187,11 @@ __global__ void __launch_bounds__(256) k_sink_rerope(const __grid_constant__ Pas
           w[2 * jj] = x0 * cb[jj] - x1 * sb[jj];
           w[2 * jj + 1] = x0 * sb[jj] + x1 * cb[jj];
         }
-        Vec8<TO>::store(out + (static_cast<long long>(h0 + k) * a.F + m) * a.d + ch * 8, w);
+        TO* dst = out + (static_cast<long long>(h0 + k) * a.F + m) * a.d + ch * 8;
+        if constexpr (sizeof(TO) == 1)
+          store_e4m3x8(reinterpret_cast<uint8_t*>(dst), w, a.fp8_inv[a.H + h0 + k]);
+        else
+          Vec8<TO>::store(dst, w);
       }
     }
   }
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(256) k_sink_rerope(const __grid_constant__ Pas
 // self-attention (temporal row 0 of buffer 0 of the table).
 template <typename TO>
 __global__ void __launch_bounds__(256) k_sink_qkv(const __grid_constant__ RopeArgs a, float qscale, float* sink_k_raw,
-                                                  TO* sink_v, TO* q_rope, TO* k_rope) {
+                                                  TO* sink_v, TO* q_rope, TO* k_rope, uint8_t* sink_v8) {
   const int chunks = a.d / 8;
   const long long total = static_cast<long long>(a.F) * 3 * a.H * chunks;
   const float* qkv = reinterpret_cast<const float*>(a.qkv);
@@ -214,6 +218,7 @@ __global__ void __launch_bounds__(256) k_sink_qkv(const __grid_constant__ RopeAr
     const long long off = (static_cast<long long>(h) * a.F + m) * a.d + ch * 8;
     if (part == 2) {
       Vec8<TO>::store(sink_v + off, v);
+      if (sink_v8) store_e4m3x8(sink_v8 + off, v, a.fp8_inv[2 * a.H + h]);
       continue;
     }
     if (part == 1) Vec8<float>::store(sink_k_raw + off, v);
@@ -342,11 +347,14 @@ cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs&
   return cudaGetLastError();
 }
 
-cudaError_t launch_sink_rerope(int bf16_out, const PassDesc& pd, const RopeArgs& a, cudaStream_t st) {
+cudaError_t launch_sink_rerope(int out_kind, const PassDesc& pd, const RopeArgs& a, cudaStream_t st) {
   if (!a.sink_k || pd.nactive == 0) return cudaSuccess;
+  if (out_kind == 2 && !a.fp8_inv) return cudaErrorInvalidValue;
   const long long n = static_cast<long long>(a.F) * ((a.H + SINK_HEADS - 1) / SINK_HEADS) * (a.d / 8);
   const int grid = grid_for(n);
-  if (bf16_out)
+  if (out_kind == 2)
+    k_sink_rerope<uint8_t><<<grid, 256, 0, st>>>(pd, a, n);
+  else if (out_kind == 1)
     k_sink_rerope<__nv_bfloat16><<<grid, 256, 0, st>>>(pd, a, n);
   else
     k_sink_rerope<float><<<grid, 256, 0, st>>>(pd, a, n);
@@ -354,16 +362,17 @@ cudaError_t launch_sink_rerope(int bf16_out, const PassDesc& pd, const RopeArgs&
 }
 
 cudaError_t launch_sink_qkv(int bf16_out, const RopeArgs& a, float qscale, float* sink_k_raw, void* sink_v,
-                            void* q_rope, void* k_rope, cudaStream_t st) {
+                            void* q_rope, void* k_rope, cudaStream_t st, uint8_t* sink_v8) {
+  if (sink_v8 && !a.fp8_inv) return cudaErrorInvalidValue;
   const long long n = static_cast<long long>(a.F) * 3 * a.H * (a.d / 8);
   const int grid = grid_for(n);
   if (bf16_out)
     k_sink_qkv<__nv_bfloat16><<<grid, 256, 0, st>>>(a, qscale, sink_k_raw, static_cast<__nv_bfloat16*>(sink_v),
                                                      static_cast<__nv_bfloat16*>(q_rope),
-                                                     static_cast<__nv_bfloat16*>(k_rope));
+                                                     static_cast<__nv_bfloat16*>(k_rope), sink_v8);
   else
     k_sink_qkv<float><<<grid, 256, 0, st>>>(a, qscale, sink_k_raw, static_cast<float*>(sink_v),
-                                            static_cast<float*>(q_rope), static_cast<float*>(k_rope));
+                                            static_cast<float*>(q_rope), static_cast<float*>(k_rope), sink_v8);
   return cudaGetLastError();
 }
 

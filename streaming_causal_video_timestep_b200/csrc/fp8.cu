@@ -7,6 +7,7 @@
 // saturating at +-448 (cvt.rn.satfinite), so the codes are a pure function of
 // the fp32 inputs.  One CTA per row; cols must be even.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -105,7 +106,74 @@ __global__ void __launch_bounds__(256) k_quant_rows_e4m3_vec(const TI* __restric
   }
 }
 
+// One e4m3 code to fp32 (exact: every e4m3 value is an fp16 value).
+__device__ __forceinline__ float e4m3_to_float(uint8_t c) {
+  uint32_t h2;
+  const uint16_t c2 = c;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c2));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// One CTA per (head, part) of one layer's QKV weight: the squared norms of the
+// head's d output rows, then the head's power-of-two scale.
+__global__ void __launch_bounds__(256) k_attn_fp8_scales(const void* w, int w_fp8, const float* w_rowscale, int D,
+                                                         int H, int d, float act_bound, float* scale, float* inv) {
+  __shared__ float n2[128];
+  const int h = blockIdx.x, part = blockIdx.y;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int r = warp; r < d; r += 8) {
+    const long long row = static_cast<long long>(part) * D + static_cast<long long>(h) * d + r;
+    float acc = 0.f;
+    if (w_fp8) {
+      const uint8_t* wr = static_cast<const uint8_t*>(w) + row * D;
+      for (int c = lane; c < D; c += 32) {
+        const float x = e4m3_to_float(wr[c]);
+        acc = fmaf(x, x, acc);
+      }
+    } else {
+      const __nv_bfloat16* wr = static_cast<const __nv_bfloat16*>(w) + row * D;
+      for (int c = lane; c < D; c += 32) {
+        const float x = __bfloat162float(wr[c]);
+        acc = fmaf(x, x, acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      const float rs = w_fp8 ? w_rowscale[row] : 1.0f;
+      n2[r] = acc * rs * rs;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    if (part < 2) {
+      for (int j = 0; j + 1 < d; j += 2) m = fmaxf(m, n2[j] + n2[j + 1]);
+    } else {
+      for (int j = 0; j < d; ++j) m = fmaxf(m, n2[j]);
+    }
+    const float bound = act_bound * sqrtf(m);
+    float sc = 1.0f, iv = 1.0f;
+    if (bound > 0.f) {
+      int ex = 0;
+      const float mant = frexpf(bound / 448.0f, &ex);   // bound / 448 = mant * 2^ex, mant in [1/2, 1)
+      const int e = mant == 0.5f ? ex - 1 : ex;
+      sc = ldexpf(1.0f, e);
+      iv = ldexpf(1.0f, -e);
+    }
+    scale[part * H + h] = sc;
+    inv[part * H + h] = iv;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_attn_fp8_scales(const void* w, int w_fp8, const float* w_rowscale, int D, int H, int d,
+                                   float act_bound, float* scale, float* inv, cudaStream_t st) {
+  if (!w || d > 128 || d % 2 != 0 || (w_fp8 && !w_rowscale)) return cudaErrorInvalidValue;
+  k_attn_fp8_scales<<<dim3(H, 3), 256, 0, st>>>(w, w_fp8, w_rowscale, D, H, d, act_bound, scale, inv);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quant_rows_e4m3(int bf16_in, const void* x, long long rows, long long cols, void* q,
                                    float* scale, cudaStream_t st) {

@@ -59,7 +59,8 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
 
 // 32 consecutive columns of one head of the [q | k | v] projection of one token:
 // rotate the pairs of q and k, scale q by log2(e)/sqrt(d), then write bf16 to
-// q_rope / the ring entry.
+// q_rope / the ring entry (or, with qp.fp8_inv, e4m3 codes of the unscaled
+// values over the head's scale).
 __device__ __forceinline__ void qkv_rope_row32(const QkvRopeParams& qp, long long row, long long col,
                                                float (&acc)[32]) {
   const int buf = static_cast<int>(row / qp.T);
@@ -92,8 +93,29 @@ __device__ __forceinline__ void qkv_rope_row32(const QkvRopeParams& qp, long lon
       acc[2 * jj + 1] = x0 * sn + x1 * c;
     }
   }
-  __nv_bfloat16* dst;
   const long long tok = static_cast<long long>(n) * qp.d + e0;
+  if (qp.fp8_inv) {
+    // e4m3 attention operands: codes of value / (the head's power-of-two scale)
+    const float inv = qp.fp8_inv[part * qp.H + h];
+    long long base;
+    if (part == 0) {
+      base = (static_cast<long long>(buf) * qp.H + h) * qp.T * qp.d;
+    } else {
+      const long long slice = qp.ring_slice0 + static_cast<long long>(qp.slot[buf]) * qp.E + qp.write_entry[buf];
+      base = (slice * qp.H + h) * qp.T * qp.d;
+    }
+    uint8_t* dst8 = static_cast<uint8_t*>(part == 0 ? qp.q_rope : (part == 1 ? qp.ring_k : qp.ring_v)) + base + tok;
+    uint32_t wv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      wv[k] = pack_e4m3x4(make_float2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
+                          make_float2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
+    uint4* d4 = reinterpret_cast<uint4*>(dst8);
+    d4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    d4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+    return;
+  }
+  __nv_bfloat16* dst;
   if (part == 0) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] *= qp.qscale;

@@ -22,6 +22,15 @@ cudaError_t launch_gemm_tc_fp8(const CUtensorMap& tmA, const CUtensorMap& tmB, c
 // q uint8 [rows, cols], scale fp32 [rows] = amax / 448 (1 for a zero row).
 cudaError_t launch_quant_rows_e4m3(int bf16_in, const void* x, long long rows, long long cols, void* q,
                                    float* scale, cudaStream_t st);
+// Per-head power-of-two scales of the e4m3 attention operands of one layer.
+// For output row j of the QKV weight w ([3D, D], bf16, or e4m3 codes with
+// per-row scales w_rowscale when w_fp8) the bound on |value| is
+//   act_bound * ||w_j||              (V rows),
+//   act_bound * ||(w_2m, w_2m+1)||   (q / K rows of rotary pair m: RoPE mixes the pair),
+// and scale[part][h] = 2^ceil(log2(max over the head's rows of the bound / 448))
+// (1 when the bound is 0); inv = 1 / scale.  Row norms are fp32 sums.
+cudaError_t launch_attn_fp8_scales(const void* w, int w_fp8, const float* w_rowscale, int D, int H, int d,
+                                   float act_bound, float* scale, float* inv, cudaStream_t st);
 
 // Tensor maps of an attention launch: q (d, Tq, H, q slices) and k[m]/v[m]
 // (d, rows_m, H, slices), 128-byte swizzle: bf16 with box (64, 128, 1, 1), or
@@ -61,20 +70,24 @@ struct RopeArgs {
   int E;
   const void* sink_k;                          // fp32 un-roped [H][F][d] of this layer (NULL: no sink part)
   void* sink_k_rope;                           // [nbuf][H][F][d]
+  const float* fp8_inv;                        // [3][H] inverse e4m3 scales of q, K, V (e4m3 outputs)
 };
 // Rolling RoPE + ring append of every active buffer's block from the fp32 qkv
 // (fp32 streams; bf16 streams do it in the QKV GEMM epilogue).  Outputs are
 // bf16 (bf16_out) or fp32.
 cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs& a, cudaStream_t st);
 // Re-rope of the layer's fp32 un-roped sink K at every active buffer's sink
-// position (a.sink_k -> a.sink_k_rope[buf]).
-cudaError_t launch_sink_rerope(int bf16_out, const PassDesc& pd, const RopeArgs& a, cudaStream_t st);
+// position (a.sink_k -> a.sink_k_rope[buf]).  out_kind: 0 fp32, 1 bf16,
+// 2 e4m3 codes of value * a.fp8_inv[H + head].
+cudaError_t launch_sink_rerope(int out_kind, const PassDesc& pd, const RopeArgs& a, cudaStream_t st);
 
 // Sink pass: split the fp32 qkv [F, 3D] into the layer's fp32 un-roped K, its
 // V, and roped q / k (temporal row 0 of buffer 0 of the table); q is
 // multiplied by qscale (the softmax scale on the bf16 path, 1 on fp32).
+// sink_v8 (optional, [H][F][d] uint8): e4m3 codes of V * a.fp8_inv[2H + head]
+// from the fp32 projection, for e4m3 attention.
 cudaError_t launch_sink_qkv(int bf16_out, const RopeArgs& a, float qscale, float* sink_k_raw, void* sink_v,
-                            void* q_rope, void* k_rope, cudaStream_t st);
+                            void* q_rope, void* k_rope, cudaStream_t st, uint8_t* sink_v8 = nullptr);
 
 // x (fp32 [rows, C]) -> h32 (fp32) and hop (dtype) when C == D (identity in-proj),
 // or -> xop (bf16) for the in-projection GEMM.

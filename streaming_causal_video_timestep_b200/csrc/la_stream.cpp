@@ -154,6 +154,8 @@ struct la_stream {
   int pt = 0, ph = 0, pw = 0;
   bool bf16 = true, id_in = true, id_head = true;
   bool fp8 = false;         // e4m3 QKV / output projections (bf16 streams)
+  bool afp8 = false;        // e4m3 attention operands in the denoising passes (bf16 streams)
+  size_t eq = 2;            // element of q_rope / sk_rope / the rings (1 with afp8, else ea)
   size_t es = 2;            // activation / weight element (bf16 or fp32)
   size_t ea = 2;            // attention operand element (bf16 or fp32)
   int device = 0, num_sms = 148;
@@ -177,6 +179,9 @@ struct la_stream {
   void* ring_v = nullptr;
   float* sink_k = nullptr;  // fp32 [L][H][F][d] un-roped
   void* sink_v = nullptr;   // attn type [L][H][F][d]
+  uint8_t* sink_v8 = nullptr;  // afp8: e4m3 codes of the sink V [L][H][F][d]
+  float* attn_sc = nullptr;    // afp8: [L][3][H] power-of-two scales of q, K, V
+  float* attn_inv = nullptr;   // afp8: their inverses
   float* sink_x = nullptr;  // [F][C]
   float* s_h32 = nullptr;   // [F][D]
   void* s_hop = nullptr;    // normalised operand (fp32 streams: == s_hn32)
@@ -325,6 +330,11 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
   if (c->cache_mode != LA_CACHE_TIMESTEP && c->cache_mode != LA_CACHE_CLEAN_REFRESH) { msg = "bad cache_mode"; return LA_EINVAL; }
   if (c->proj_fp8 != 0 && c->proj_fp8 != 1) { msg = "proj_fp8 must be 0 or 1"; return LA_EINVAL; }
   if (c->proj_fp8 && c->dtype != LA_BF16) { msg = "e4m3 projections need the bf16 stream"; return LA_EINVAL; }
+  if (c->attn_fp8 != 0 && c->attn_fp8 != 1) { msg = "attn_fp8 must be 0 or 1"; return LA_EINVAL; }
+  if (c->attn_fp8 && (c->dtype != LA_BF16 || c->head_dim != 128)) {
+    msg = "e4m3 attention needs the bf16 stream and head_dim 128";
+    return LA_EINVAL;
+  }
   if (c->cache_mode == LA_CACHE_CLEAN_REFRESH && c->schedule != LA_SCHED_SEQUENTIAL) {
     msg = "the clean-cache refresh needs the sequential schedule";
     return LA_EINVAL;
@@ -399,7 +409,7 @@ char* elem(void* base, long long idx, size_t es) { return static_cast<char*>(bas
 
 int capture_pass(la_stream* s, const PassDesc& pd, int layer) {
   // copy the intermediates of every active buffer into its slot's capture area
-  const size_t ea = s->ea;
+  const size_t eq = s->eq;
   const long long T = s->T, D = s->D, H = s->H, d = s->d, F = s->F, L = s->L;
   const float* o32 = s->bf16 ? s->cap_oall : static_cast<const float*>(s->attn_o);
   for (int ai = 0; ai < pd.nactive; ++ai) {
@@ -413,17 +423,22 @@ int capture_pass(la_stream* s, const PassDesc& pd, int layer) {
     }
     CU(cudaMemcpyAsync(s->cap_h + (static_cast<long long>(slot) * (L + 1) + layer + 1) * T * D, s->h32 + buf * T * D,
                        T * D * 4, cudaMemcpyDeviceToDevice, s->st));
-    CU(cudaMemcpyAsync(elem(s->cap_q, (static_cast<long long>(slot) * L + layer) * H * T * d, ea),
-                       elem(s->q_rope, buf * H * T * d, ea), H * T * d * ea, cudaMemcpyDeviceToDevice, s->st));
+    CU(cudaMemcpyAsync(elem(s->cap_q, (static_cast<long long>(slot) * L + layer) * H * T * d, eq),
+                       elem(s->q_rope, buf * H * T * d, eq), H * T * d * eq, cudaMemcpyDeviceToDevice, s->st));
     CU(cudaMemcpyAsync(s->cap_o + (static_cast<long long>(slot) * L + layer) * T * D, o32 + buf * T * D, T * D * 4,
                        cudaMemcpyDeviceToDevice, s->st));
-    CU(cudaMemcpyAsync(elem(s->cap_sk, (static_cast<long long>(slot) * L + layer) * H * F * d, ea),
-                       elem(s->sk_rope, buf * H * F * d, ea), H * F * d * ea, cudaMemcpyDeviceToDevice, s->st));
+    CU(cudaMemcpyAsync(elem(s->cap_sk, (static_cast<long long>(slot) * L + layer) * H * F * d, eq),
+                       elem(s->sk_rope, buf * H * F * d, eq), H * F * d * eq, cudaMemcpyDeviceToDevice, s->st));
   }
   return LA_OK;
 }
 
 constexpr float kRmsEps = 1e-6f;
+// |value| of an e4m3 attention operand <= kAttnActBound * sqrt(D) * the norm of its
+// weight row (or rotary pair of rows): an RMS-normalised row has norm <= sqrt(D),
+// and rounding it to the GEMM operand (bf16, or per-row e4m3) grows each element by
+// at most a factor 1 + 2^-4 plus e4m3's subnormal floor; 1.07 covers both.
+constexpr double kAttnActBound = 1.07;
 
 // Per-token RMS normalisation of the residual into the next GEMM's operand.
 int normalise(la_stream* s, const float* h, long long rows, void* op_bf16, float* op_f32) {
@@ -508,6 +523,14 @@ int run_pass(la_stream* s, const PassDesc& pd) {
     ra.ring_slice0 = static_cast<long long>(l) * S * E;
     ra.sink_k = s->sink_k + static_cast<long long>(l) * H * F * d;
     ra.sink_k_rope = s->sk_rope;
+    if (s->afp8) {
+      const long long so = static_cast<long long>(l) * 3 * H;
+      ra.fp8_inv = qp.fp8_inv = s->attn_inv + so;
+      ap.fp8 = 1;
+      ap.sq = s->attn_sc + so;
+      ap.sk = s->attn_sc + so + H;
+      ap.sv = s->attn_sc + so + 2 * H;
+    }
     if (s->bf16) {
       // QKV projection with Rolling RoPE + ring append fused into the epilogue
       qp.ring_slice0 = ra.ring_slice0;
@@ -523,8 +546,9 @@ int run_pass(la_stream* s, const PassDesc& pd) {
                   })) != LA_OK) {
         return r;
       }
-      // per-block re-rope of the sink K (fp32 -> bf16, once per active buffer)
-      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_sink_rerope(1, pd, ra, s->st); })) != LA_OK) return r;
+      // per-block re-rope of the sink K (fp32 -> bf16 or e4m3, once per active buffer)
+      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_sink_rerope(s->afp8 ? 2 : 1, pd, ra, s->st); })) != LA_OK)
+        return r;
     } else {
       GemmEpiParams eq = epi(EPI_STORE, s->qkv, nullptr, 3LL * D);
       if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_hop, &s->tm_wqkv[l], s->hn32, s->w_qkv[l], eq, rows, 3 * D, D)) !=
@@ -662,8 +686,11 @@ int run_sink(la_stream* s) {
     ra.qkv = s->s_qkv;
     float* kraw = s->sink_k + static_cast<long long>(l) * H * F * d;
     void* vraw = elem(s->sink_v, static_cast<long long>(l) * H * F * d, s->ea);
+    uint8_t* v8 = s->afp8 ? s->sink_v8 + static_cast<long long>(l) * H * F * d : nullptr;
+    ra.fp8_inv = s->afp8 ? s->attn_inv + static_cast<long long>(l) * 3 * H : nullptr;
     if ((r = launch(s, LA_KIND_ROPE, [&] {
-           return launch_sink_qkv(s->bf16, ra, s->bf16 ? ap.scale_log2 : 1.0f, kraw, vraw, s->s_q, s->s_k, s->st);
+           return launch_sink_qkv(s->bf16, ra, s->bf16 ? ap.scale_log2 : 1.0f, kraw, vraw, s->s_q, s->s_k, s->st,
+                                  v8);
          })) != LA_OK)
       return r;
     if (l == s->L - 1) break;   // the last layer's sink output feeds nothing
@@ -778,9 +805,9 @@ int alloc_capture(la_stream* s) {
   DALLOC(s->cap_vall, static_cast<long long>(s->nbuf) * T * C * 4);
   DALLOC(s->cap_oall, static_cast<long long>(s->nbuf) * T * D * 4);
   DALLOC(s->cap_h, S * (L + 1) * T * D * 4);
-  DALLOC(s->cap_q, S * L * H * T * d * s->ea);
+  DALLOC(s->cap_q, S * L * H * T * d * s->eq);
   DALLOC(s->cap_o, S * L * T * D * 4);
-  DALLOC(s->cap_sk, S * L * H * F * d * s->ea);
+  DALLOC(s->cap_sk, S * L * H * F * d * s->eq);
   DALLOC(s->cap_sink_h, L * F * D * 4);
   if (s->bf16) {
     DALLOC(s->cap_hop, S * L * T * D * s->es);
@@ -840,6 +867,8 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   s->pt = cfg->rope_split[0]; s->ph = cfg->rope_split[1]; s->pw = cfg->rope_split[2];
   s->bf16 = cfg->dtype == LA_BF16; s->es = s->bf16 ? 2 : 4; s->ea = s->es;
   s->fp8 = s->bf16 && cfg->proj_fp8;
+  s->afp8 = s->bf16 && cfg->attn_fp8;
+  s->eq = s->afp8 ? 1 : s->ea;
   s->id_in = w->w_in == nullptr; s->id_head = w->w_head == nullptr;
   s->nbuf = cfg->schedule == LA_SCHED_PIPELINED ? s->S : 1;
   s->st = static_cast<cudaStream_t>(cuda_stream);
@@ -860,13 +889,14 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   // memory plan, checked before allocating
   const long long T = s->T, D = s->D, C = s->C, F = s->F, H = s->H, d = s->d, L = s->L, S = s->S, E = s->E;
   const long long NB = s->nbuf;
-  const size_t es = s->es, ea = s->ea;
+  const size_t es = s->es, ea = s->ea, eq = s->eq;
   const long long need = NB * T * C * 4 + NB * T * D * 4 + (s->bf16 ? NB * T * D * es : 0) +
                          ((!s->bf16 || s->id_head) ? NB * T * D * 4 : 0) + F * D * 4 +
                          (s->bf16 && !s->id_in ? NB * T * C * 2 : 0) + (s->bf16 ? 0 : NB * T * 3 * D * 4) +
-                         NB * T * D * ea + NB * T * D * es + NB * H * F * d * ea + 2 * L * S * E * H * T * d * ea +
+                         NB * T * D * eq + NB * T * D * es + NB * H * F * d * eq + 2 * L * S * E * H * T * d * eq +
                          L * H * F * d * (4 + ea) + F * C * 4 + F * D * 4 + F * D * es * 2 + F * C * 2 +
-                         F * 3 * D * 4 + 2 * H * F * d * ea + (64 << 20);
+                         F * 3 * D * 4 + 2 * H * F * d * ea + (s->afp8 ? L * H * F * d + L * 3 * H * 8 : 0) +
+                         (64 << 20);
   size_t free_b = 0, total_b = 0;
   e = cudaMemGetInfo(&free_b, &total_b);
   if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
@@ -888,13 +918,18 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   if (s->bf16) ALLOC_OR_BAIL(s->hop, NB * T * D * es); else s->hop = s->hn32;
   if (s->bf16 && !s->id_in) ALLOC_OR_BAIL(s->xop, NB * T * C * 2);
   if (!s->bf16) ALLOC_OR_BAIL(s->qkv, NB * T * 3 * D * 4);
-  ALLOC_OR_BAIL(s->q_rope, NB * T * D * ea);
+  ALLOC_OR_BAIL(s->q_rope, NB * T * D * eq);
   ALLOC_OR_BAIL(s->attn_o, NB * T * D * es);
-  ALLOC_OR_BAIL(s->sk_rope, NB * H * F * d * ea);
-  ALLOC_OR_BAIL(s->ring_k, L * S * E * H * T * d * ea);
-  ALLOC_OR_BAIL(s->ring_v, L * S * E * H * T * d * ea);
+  ALLOC_OR_BAIL(s->sk_rope, NB * H * F * d * eq);
+  ALLOC_OR_BAIL(s->ring_k, L * S * E * H * T * d * eq);
+  ALLOC_OR_BAIL(s->ring_v, L * S * E * H * T * d * eq);
   ALLOC_OR_BAIL(s->sink_k, L * H * F * d * 4);
   ALLOC_OR_BAIL(s->sink_v, L * H * F * d * ea);
+  if (s->afp8) {
+    ALLOC_OR_BAIL(s->sink_v8, L * H * F * d);
+    ALLOC_OR_BAIL(s->attn_sc, L * 3 * H * 4);
+    ALLOC_OR_BAIL(s->attn_inv, L * 3 * H * 4);
+  }
   ALLOC_OR_BAIL(s->sink_x, F * C * 4);
   ALLOC_OR_BAIL(s->s_h32, F * D * 4);
   if (s->bf16) ALLOC_OR_BAIL(s->s_hop, F * D * es);
@@ -959,11 +994,19 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
       ok = ok && tmap_2d_bf16(&s->tm_win, s->w_in, D, C, C, bn_d, s->err);
       ok = ok && tmap_2d_bf16(&s->tm_whead, s->w_head, C, D, D, bn_c, s->err);
     }
-    ok = ok && tmap_planes_bf16(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
-    ok = ok && tmap_planes_bf16(&s->maps_stream.v[1], s->sink_v, d, F, H, L, s->err);
+    if (s->afp8) {
+      ok = ok && tmap_planes_u8(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
+      ok = ok && tmap_planes_u8(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
+      ok = ok && tmap_planes_u8(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
+      ok = ok && tmap_planes_u8(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
+      ok = ok && tmap_planes_u8(&s->maps_stream.v[1], s->sink_v8, d, F, H, L, s->err);
+    } else {
+      ok = ok && tmap_planes_bf16(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
+      ok = ok && tmap_planes_bf16(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
+      ok = ok && tmap_planes_bf16(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
+      ok = ok && tmap_planes_bf16(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
+      ok = ok && tmap_planes_bf16(&s->maps_stream.v[1], s->sink_v, d, F, H, L, s->err);
+    }
     ok = ok && tmap_planes_bf16(&s->maps_sink.q, s->s_q, d, F, H, 1, s->err);
     ok = ok && tmap_planes_bf16(&s->maps_sink.k[0], s->s_k, d, F, H, 1, s->err);
     ok = ok && tmap_planes_bf16(&s->maps_sink.v[0], s->sink_v, d, F, H, L, s->err);
@@ -991,6 +1034,16 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
            tmap_2d_u8(&s->tm_wo8[l], s->wo8[l], D, D, D, bn_d, s->err);
     }
     if (!ok) return bail(LA_ECUDA);
+  }
+  if (s->afp8) {
+    // per-head e4m3 scales from the QKV weights as the projection uses them
+    const float act_bound = static_cast<float>(kAttnActBound * std::sqrt(static_cast<double>(D)));
+    for (int l = 0; l < L; ++l) {
+      e = launch_attn_fp8_scales(s->fp8 ? s->wq8[l] : s->w_qkv[l], s->fp8 ? 1 : 0, s->fp8 ? s->wq8s[l] : nullptr,
+                                 s->D, s->H, s->d, act_bound, s->attn_sc + static_cast<long long>(l) * 3 * H,
+                                 s->attn_inv + static_cast<long long>(l) * 3 * H, s->st);
+      if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
+    }
   }
   e = cudaStreamSynchronize(s->st);
   if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
@@ -1059,11 +1112,11 @@ int la_debug_capture(la_stream* s, int32_t enable) {
 int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* dst, int64_t dst_bytes) {
   if (!s || !dst) return LA_EINVAL;
   const long long T = s->T, C = s->C, D = s->D, H = s->H, d = s->d, F = s->F, L = s->L, E = s->E, S = s->S;
-  const size_t ea = s->ea;
+  const size_t ea = s->ea, eq = s->eq;
   const bool per_layer = what == LA_TAP_H || what == LA_TAP_Q || what == LA_TAP_O || what == LA_TAP_RING_K ||
                          what == LA_TAP_RING_V || what == LA_TAP_SINK_K || what == LA_TAP_SINK_V ||
                          what == LA_TAP_SINK_KROPE || what == LA_TAP_SINK_H || what == LA_TAP_HOP ||
-                         what == LA_TAP_SINK_HOP;
+                         what == LA_TAP_SINK_HOP || what == LA_TAP_SINK_V8 || what == LA_TAP_ATTN_SCALES;
   if (per_layer && (layer < (what == LA_TAP_H ? -1 : 0) || layer >= L)) return fail(s, LA_EINVAL, "bad layer");
   if (slot < 0 || slot >= S) return fail(s, LA_EINVAL, "bad slot");
   const void* src = nullptr;
@@ -1071,6 +1124,8 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
   const bool needs_capture = what <= LA_TAP_V || what == LA_TAP_SINK_KROPE || what == LA_TAP_HOP;
   if ((what == LA_TAP_HOP || what == LA_TAP_SINK_HOP) && !s->bf16)
     return fail(s, LA_EINVAL, "the GEMM-operand taps exist in bf16 streams only");
+  if ((what == LA_TAP_SINK_V8 || what == LA_TAP_ATTN_SCALES) && !s->afp8)
+    return fail(s, LA_EINVAL, "the e4m3 attention taps exist with attn_fp8 only");
   if (needs_capture && (!s->cap_xin || s->cap_valid.empty() || !s->cap_valid[slot]))
     return fail(s, LA_ESTATE, "no capture of that slot in the last call");
   switch (what) {
@@ -1078,17 +1133,19 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
     case LA_TAP_X_OUT: src = s->cap_xout + slot * T * C; bytes = T * C * 4; break;
     case LA_TAP_V: src = s->cap_v + slot * T * C; bytes = T * C * 4; break;
     case LA_TAP_H: src = s->cap_h + (slot * (L + 1) + layer + 1) * T * D; bytes = T * D * 4; break;
-    case LA_TAP_Q: src = elem(s->cap_q, (slot * L + layer) * H * T * d, ea); bytes = H * T * d * ea; break;
+    case LA_TAP_Q: src = elem(s->cap_q, (slot * L + layer) * H * T * d, eq); bytes = H * T * d * eq; break;
     case LA_TAP_O: src = s->cap_o + (slot * L + layer) * T * D; bytes = T * D * 4; break;
-    case LA_TAP_SINK_KROPE: src = elem(s->cap_sk, (slot * L + layer) * H * F * d, ea); bytes = H * F * d * ea; break;
+    case LA_TAP_SINK_KROPE: src = elem(s->cap_sk, (slot * L + layer) * H * F * d, eq); bytes = H * F * d * eq; break;
     case LA_TAP_RING_K:
     case LA_TAP_RING_V:
       src = elem(what == LA_TAP_RING_K ? s->ring_k : s->ring_v,
-                 (static_cast<long long>(layer) * S + s->sched.ring_of(slot)) * E * H * T * d, ea);
-      bytes = E * H * T * d * ea;
+                 (static_cast<long long>(layer) * S + s->sched.ring_of(slot)) * E * H * T * d, eq);
+      bytes = E * H * T * d * eq;
       break;
     case LA_TAP_SINK_K: src = s->sink_k + static_cast<long long>(layer) * H * F * d; bytes = H * F * d * 4; break;
     case LA_TAP_SINK_V: src = elem(s->sink_v, static_cast<long long>(layer) * H * F * d, ea); bytes = H * F * d * ea; break;
+    case LA_TAP_SINK_V8: src = s->sink_v8 + static_cast<long long>(layer) * H * F * d; bytes = H * F * d; break;
+    case LA_TAP_ATTN_SCALES: src = s->attn_sc + static_cast<long long>(layer) * 3 * H; bytes = 3 * H * 4; break;
     case LA_TAP_SINK_H:
       if (!s->cap_sink_valid) return fail(s, LA_ESTATE, "no capture of a sink pass");
       src = s->cap_sink_h + static_cast<long long>(layer) * F * D;

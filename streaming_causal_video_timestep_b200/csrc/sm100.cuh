@@ -274,6 +274,23 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// Four fp32 values to four e4m3 codes in one 32-bit word, value b in byte b.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float2 lo, float2 hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\t"
+      "mov.b32 %0, {l, h};\n\t}"
+      : "=r"(r)
+      : "f"(lo.x), "f"(lo.y), "f"(hi.x), "f"(hi.y));
+  return r;
+}
+// e4m3 codes of v[i] * inv for 8 values, one 8-byte store (p 8-byte aligned).
+__device__ __forceinline__ void store_e4m3x8(uint8_t* p, const float (&v)[8], float inv) {
+  const uint32_t lo = pack_e4m3x4(make_float2(v[0] * inv, v[1] * inv), make_float2(v[2] * inv, v[3] * inv));
+  const uint32_t hi = pack_e4m3x4(make_float2(v[4] * inv, v[5] * inv), make_float2(v[6] * inv, v[7] * inv));
+  *reinterpret_cast<uint2*>(p) = make_uint2(lo, hi);
+}
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

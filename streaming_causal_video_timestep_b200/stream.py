@@ -72,6 +72,7 @@ class LaStream:
         c.schedule, c.dtype = cfg.schedule, self.dtype
         c.cache_mode = getattr(cfg, "cache_mode", 0)
         c.proj_fp8 = getattr(cfg, "proj_fp8", 0)
+        c.attn_fp8 = getattr(cfg, "attn_fp8", 0)
         self.cfg = cfg
         self.c = c
         self.T = cfg.frames_per_block * cfg.grid_h * cfg.grid_w
@@ -155,9 +156,12 @@ class LaStream:
             "ring_k": ((E, H, T, d), dt), "ring_v": ((E, H, T, d), dt), "sink_k": ((H, F, d), dt),
             "sink_v": ((H, F, d), dt), "sink_k_rope": ((H, F, d), dt), "sink_h": ((F, D), torch.float32),
             "hop": ((T, D), dt), "sink_hop": ((F, D), dt),
+            "sink_v8": ((H, F, d), torch.uint8), "attn_scales": ((3, H), torch.float32),
         }
         shape, tdt = shapes[what]
-        if what in ("q", "ring_k", "ring_v", "sink_v", "sink_k_rope"):
+        if what in ("q", "ring_k", "ring_v", "sink_k_rope") and getattr(self.cfg, "attn_fp8", 0):
+            tdt = torch.uint8          # e4m3 codes
+        elif what in ("q", "ring_k", "ring_v", "sink_v", "sink_k_rope"):
             tdt = attn_dtype(self.dtype)
         elif what in ("o", "sink_k"):
             tdt = torch.float32

@@ -15,7 +15,8 @@ import numpy as np
 import math
 
 from oracle import block_causal_attention, euler_step, rms_norm, rope_rotate
-from oracle.fp8 import project, quantize_rows
+from oracle.fp8 import (attention_fp8, attn_fp8_scales, dequantize_weight, project, quantize_heads,
+                        quantize_rows)
 from oracle.rope import block_positions, sink_positions
 from workloads import DTYPE_BF16, bf16_round
 
@@ -49,6 +50,47 @@ def _proj(a, w, cfg):
     return project(a, *hit[1])
 
 
+def _qkv_weight_used(w, cfg):
+    """The QKV weight as the projection multiplies it (dequantized e4m3 with proj_fp8)."""
+    if not getattr(cfg, "proj_fp8", 0):
+        return np.asarray(w, np.float64)
+    _proj(np.zeros((1, w.shape[1])), w, cfg)            # fills the quantized-weight cache
+    return dequantize_weight(_W8[id(w)][1])
+
+
+_SC = {}
+
+
+def attn_scales(s, cfg, W, l):
+    """The GPU's per-head e4m3 scales of layer l, checked equal to the oracle's rule."""
+    sc = to_np(s.tap("attn_scales", l)).astype(np.float32)
+    key = (id(W.w_qkv[l]), getattr(cfg, "proj_fp8", 0))
+    if key not in _SC:
+        _SC[key] = attn_fp8_scales(_qkv_weight_used(W.w_qkv[l], cfg), cfg.hidden, cfg.heads, cfg.head_dim)
+    np.testing.assert_array_equal(sc, _SC[key])
+    return sc
+
+
+def check_codes(codes, x, scales, what):
+    """e4m3 codes of the GPU against the oracle's quantization of its own value x
+    [N, H, d] (quantize_heads).  The GPU quantizes its fp32 result, which differs from
+    the oracle's by the GEMM's accumulation rounding, so a value at a rounding tie may
+    take the neighbouring code: every difference must be to an adjacent code of the
+    same sign, and at most 1 % of the codes may differ.  Returns the fraction."""
+    want = quantize_heads(x, scales)
+    codes = np.asarray(codes, np.uint8)
+    diff = codes != want
+    frac = float(diff.mean())
+    if diff.any():
+        g, w_ = codes[diff].astype(np.int32), want[diff].astype(np.int32)
+        mag_g, mag_w = g & 0x7F, w_ & 0x7F
+        same_sign = ((g & 0x80) == (w_ & 0x80)) | ((mag_g == 0) & (mag_w == 0)) | (np.maximum(mag_g, mag_w) <= 1)
+        adjacent = np.abs(mag_g - mag_w) <= 1
+        assert np.all(same_sign & adjacent), f"{what}: non-adjacent e4m3 code"
+    assert frac <= 1e-2, f"{what}: {frac:.2e} of the codes differ"
+    return frac
+
+
 def check_sink(s, cfg, W, latent, rows=None, tag=""):
     """Per-op check of the last sink pass: in-projection of the sink latent and,
     per layer, the stored un-roped K (fp32) and V from the captured sink residual."""
@@ -62,9 +104,9 @@ def check_sink(s, cfg, W, latent, rows=None, tag=""):
     for l in range(cfg.num_layers):
         hs = to_np(s.tap("sink_h", l))
         op = _normed_operand(hs[R], cfg)
-        if getattr(cfg, "proj_fp8", 0):
-            # e4m3 projections: the normalisation on its own, then the projection
-            # from the operand the GPU quantized (a one-ulp difference there can move
+        if getattr(cfg, "proj_fp8", 0) or getattr(cfg, "attn_fp8", 0):
+            # e4m3 operands downstream: the normalisation on its own, then the projection
+            # from the operand the GPU consumed (a one-ulp difference there can move
             # a code, or a row's scale, by a whole e4m3 step)
             op_gpu = to_np(s.tap("sink_hop", l))[R].astype(np.float64)
             assert_close(op_gpu, op, dt, f"{tag} sink norm operand l{l}")
@@ -74,14 +116,20 @@ def check_sink(s, cfg, W, latent, rows=None, tag=""):
         v = qkv[:, 2 * D:].reshape(len(R), H, d)
         assert_close(to_np(s.tap("sink_k", l)).transpose(1, 0, 2)[R], k, dt, f"{tag} sink K l{l}")
         assert_close(to_np(s.tap("sink_v", l)).transpose(1, 0, 2)[R], v, dt, f"{tag} sink V l{l}")
+        if getattr(cfg, "attn_fp8", 0):
+            sc = attn_scales(s, cfg, W, l)
+            check_codes(to_np(s.tap("sink_v8", l)).transpose(1, 0, 2)[R], v, sc[2], f"{tag} sink V codes l{l}")
 
 
 def sink_snapshot(s, cfg):
     """The sink K (un-roped) and V of every layer as they are now: take it before
     a call whose per-op check follows (the AAS replacement at the end of the
     call that finishes block 0 changes them)."""
-    return ([to_np(s.tap("sink_k", l)).transpose(1, 0, 2) for l in range(cfg.num_layers)],
+    snap = ([to_np(s.tap("sink_k", l)).transpose(1, 0, 2) for l in range(cfg.num_layers)],
             [to_np(s.tap("sink_v", l)).transpose(1, 0, 2) for l in range(cfg.num_layers)])
+    if getattr(cfg, "attn_fp8", 0):
+        snap += ([to_np(s.tap("sink_v8", l)).transpose(1, 0, 2) for l in range(cfg.num_layers)],)
+    return snap
 
 
 def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
@@ -107,7 +155,10 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
     h_prev = h_in
     for l in range(L):
         op = _normed_operand(h_prev[R], cfg)
-        if getattr(cfg, "proj_fp8", 0):
+        if getattr(cfg, "proj_fp8", 0) or getattr(cfg, "attn_fp8", 0):
+            # e4m3 operands downstream: check the normalisation on its own, then go on
+            # from the operand the GPU consumed (a one-ulp bf16 difference there moves
+            # a product by more than the rounding an e4m3 code check can absorb)
             op_gpu = to_np(s.tap("hop", l, i))[R].astype(np.float64)
             chk(op_gpu, op, f"norm operand l{l}")
             op = op_gpu
@@ -117,6 +168,14 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
         v = qkv[:, 2 * D:].reshape(len(R), H, d)
         qr = rope_rotate(q, pt[R], ph[R], pw[R], cfg.pairs, cfg.rope_theta)
         kr = rope_rotate(k, pt[R], ph[R], pw[R], cfg.pairs, cfg.rope_theta)
+        if getattr(cfg, "attn_fp8", 0):
+            _check_attn_fp8(s, cfg, W, b, i, l, R, qr, kr, v, sink, st, chk, errs, tag)
+            o_gpu = to_np(s.tap("o", l, i))
+            h_next = to_np(s.tap("h", l, i))
+            want = h_prev[R].astype(np.float64) + _proj(_operand(o_gpu[R], cfg), W.w_out[l], cfg)
+            chk(h_next[R], want, f"h l{l}")
+            h_prev = h_next
+            continue
         q_gpu = to_np(s.tap("q", l, i)).transpose(1, 0, 2)           # [T, H, d]
         if dt == DTYPE_BF16:
             # bf16 streams store q pre-multiplied by the softmax scale log2(e)/sqrt(d)
@@ -155,3 +214,31 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
         for k_, v_ in errs.items():
             report[k_] = max(report.get(k_, (0, 0)), v_)
     return errs
+
+
+def _check_attn_fp8(s, cfg, W, b, i, l, R, qr, kr, v, sink, st, chk, errs, tag):
+    """e4m3 attention of one layer: scales, the codes of q / the ring entry / the
+    re-roped sink K against the oracle's values, then the attention from the GPU's
+    own codes (oracle.fp8.attention_fp8)."""
+    E, D = cfg.ring_entries, cfg.hidden
+    sc = attn_scales(s, cfg, W, l)
+    q8 = to_np(s.tap("q", l, i)).transpose(1, 0, 2)                  # [T, H, d] codes
+    rk8 = to_np(s.tap("ring_k", l, i)).transpose(0, 2, 1, 3)         # [E, T, H, d]
+    rv8 = to_np(s.tap("ring_v", l, i)).transpose(0, 2, 1, 3)
+    e = b % E
+    fr = {}
+    fr["q codes"] = check_codes(q8[R], qr, sc[0], f"{tag} q codes l{l} b{b} s{i}")
+    fr["ring K codes"] = check_codes(rk8[e][R], kr, sc[1], f"{tag} ring K codes l{l} b{b} s{i}")
+    fr["ring V codes"] = check_codes(rv8[e][R], v, sc[2], f"{tag} ring V codes l{l} b{b} s{i}")
+    sk_raw = sink[0][l] if sink is not None else to_np(s.tap("sink_k", l)).transpose(1, 0, 2)
+    sk8 = to_np(s.tap("sink_k_rope", l, i)).transpose(1, 0, 2)
+    fr["sink K codes"] = check_codes(sk8, rope_rotate(sk_raw, *st, cfg.pairs, cfg.rope_theta), sc[1],
+                                     f"{tag} sink K codes l{l} b{b} s{i}")
+    sv8 = sink[2][l] if sink is not None and len(sink) > 2 else to_np(s.tap("sink_v8", l)).transpose(1, 0, 2)
+    order = range(max(0, b - cfg.window_blocks), b + 1)
+    keys = np.concatenate([sk8] + [rk8[bb % E] for bb in order])
+    vals = np.concatenate([sv8] + [rv8[bb % E] for bb in order])
+    o_want = attention_fp8(q8[R], keys, vals, sc[0], sc[1], sc[2])
+    chk(to_np(s.tap("o", l, i))[R], o_want.reshape(len(R), D), f"attn O (e4m3) l{l}")
+    for k_, f_ in fr.items():
+        errs[k_] = max(errs.get(k_, (0, 0)), (f_, 0.0))

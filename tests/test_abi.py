@@ -90,6 +90,8 @@ def _weights(nonnull=True):
     dict(cache_mode=1, schedule=0),                   # the clean-cache refresh is sequential only
     dict(proj_fp8=1),                                 # e4m3 projections need the bf16 stream (dtype 1 = fp32)
     dict(proj_fp8=2, dtype=0, head_dim=128, hidden=128, latent_ch=128, rope_split=(22, 21, 21)),
+    dict(attn_fp8=1),                                 # e4m3 attention needs the bf16 stream
+    dict(attn_fp8=2, dtype=0, head_dim=128, hidden=128, latent_ch=128, rope_split=(22, 21, 21)),
 ])
 def test_invalid_config_returns_einval(lib, over):
     c = _cfg(**over)

@@ -250,6 +250,30 @@ def test_small_bf16_stream_with_e4m3_projections_teacher_forced():
     print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in report.items()})
 
 
+def test_small_bf16_stream_with_e4m3_attention_teacher_forced():
+    """e4m3 attention in the denoising passes: per-head scales equal to the oracle's
+    rule, the codes of q / ring K, V / re-roped sink K / sink V against the oracle's
+    quantization of its own values, the attention from the GPU's codes, integer state
+    bit-exact."""
+    cfg = SMALL_BF16.cfg.replace(attn_fp8=1)
+    report = _run_teacher_forced(Workload("small-bf16-afp8", cfg, SMALL_BF16.seed, 6, SMALL_BF16.w_std,
+                                          SMALL_BF16.head_std))
+    print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in report.items()})
+
+
+def test_small_bf16_stream_with_e4m3_projections_and_attention_teacher_forced():
+    cfg = SMALL_BF16.cfg.replace(proj_fp8=1, attn_fp8=1)
+    report = _run_teacher_forced(Workload("small-bf16-fp8-all", cfg, SMALL_BF16.seed, 5, SMALL_BF16.w_std,
+                                          SMALL_BF16.head_std))
+    print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in report.items()})
+
+
+def test_tiny_fp32_stream_rejects_e4m3_attention():
+    from streaming_causal_video_timestep_b200 import LaError
+    with pytest.raises(LaError):
+        make_stream(Workload("tiny-afp8", TINY.cfg.replace(attn_fp8=1), TINY.seed, 2, TINY.w_std, TINY.head_std))
+
+
 def test_tiny_fp32_stream_rejects_e4m3_projections():
     from streaming_causal_video_timestep_b200 import LaError
     with pytest.raises(LaError):

@@ -192,3 +192,103 @@ def test_attention_fp8_error_is_within_the_rounding_bound_of_p():
         assert np.all(np.abs(got[:, h] - ref[:, h]) <= bound * (1 + 1e-6) + 1e-12)
     # the rounding of P is visible: the result is not the unquantized one
     assert np.abs(got - ref).max() > 1e-4 * np.abs(ref).max()
+
+
+# ---- e4m3 attention operands of the stream ---------------------------------------------------
+from oracle.fp8 import ATTN_ACT_BOUND, attn_fp8_scales, pow2_at_least, quantize_heads  # noqa: E402
+from oracle.norm import rms_norm  # noqa: E402
+from oracle.rope import rope_rotate  # noqa: E402
+
+
+def test_pow2_at_least():
+    assert [pow2_at_least(x) for x in (1.0, 1.5, 0.75, 2.0 ** -10, 3 * 2.0 ** -10, 448.0)] == \
+        [1.0, 2.0, 1.0, 2.0 ** -10, 2.0 ** -8, 512.0]
+
+
+def test_quantize_heads_is_torch_e4m3_of_value_over_scale():
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((50, 3, 16)) * 20
+    sc = np.float32([0.5, 1.0, 0.125])
+    got = quantize_heads(x, sc)
+    ref = (torch.from_numpy(x.astype(np.float32)) / torch.from_numpy(sc)[None, :, None]) \
+        .clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(got, ref)
+
+
+def _adversarial_inputs(w, D, rows):
+    """Unit-RMS rows aligned with weight rows (or sums of a rotary pair of rows), the
+    inputs that come closest to the Cauchy-Schwarz bound."""
+    xs = []
+    for r in rows:
+        x = w[r] if r % 2 else w[r] + w[r + 1]
+        xs.append(x / np.sqrt(np.mean(x ** 2)))
+    return np.stack(xs)
+
+
+def test_attn_fp8_scales_never_saturate_and_are_tight():
+    rng = np.random.default_rng(22)
+    D, H, d = 256, 4, 64
+    w = (rng.standard_normal((3 * D, D)) * rng.uniform(0.2, 3.0, (3 * D, 1)) * 0.02)
+    sc = attn_fp8_scales(w, D, H, d).astype(np.float64)
+    assert np.all(np.log2(sc) == np.round(np.log2(sc)))          # powers of two
+    # random and adversarial unit-RMS rows, rounded up by the largest operand rounding (6.25 %)
+    x = np.concatenate([rms_norm(rng.standard_normal((200, D))),
+                        _adversarial_inputs(w, D, rng.integers(0, 3 * D - 1, 300))]) * (1 + 2.0 ** -4)
+    qkv = x @ w.T
+    pairs = (d // 2 - 2 * (d // 6), d // 6, d // 6)
+    pos = [rng.integers(-50, 50, len(x)) for _ in range(3)]
+    for part in range(3):
+        vals = qkv[:, part * D:(part + 1) * D].reshape(len(x), H, d)
+        if part < 2:
+            vals = rope_rotate(vals, *pos, pairs, 10000.0)
+        ratio = np.abs(vals).max(axis=(0, 2)) / sc[part]
+        assert np.all(ratio <= 448.0), (part, ratio)
+    # the bound itself lands in (224, 448] of each head's scale
+    n2 = (w ** 2).sum(axis=1)
+    for part in range(3):
+        for h in range(H):
+            rows = n2[part * D + h * d: part * D + (h + 1) * d]
+            m = (rows[0::2] + rows[1::2]).max() if part < 2 else rows.max()
+            b = ATTN_ACT_BOUND * np.sqrt(D * m) / sc[part, h]
+            assert 224.0 < b <= 448.0
+
+
+def test_attn_fp8_scales_pair_bound_is_needed_for_rotated_rows():
+    """A rotation by 45 degrees of a pair whose rows both read the input puts sqrt(2)
+    times a row's bound into one component: the pair norm is what bounds it."""
+    D, H, d = 16, 1, 16
+    w = np.zeros((3 * D, D))
+    w[0, 0] = w[1, 0] = 1.0                      # q rows 0 and 1 (rotary pair 0) read input 0
+    w[D:, :] = 0.01
+    x = np.zeros((1, D))
+    x[0, 0] = np.sqrt(D)                         # unit RMS
+    q = (x @ w[:D].T).reshape(1, H, d)
+    # pair 0 is temporal with frequency 1: angle = position = pi/4
+    qr = rope_rotate(q, np.array([np.pi / 4]), np.array([0]), np.array([0]), (d // 2, 0, 0), 10000.0)
+    v = abs(qr[0, 0, 1])
+    assert v == pytest.approx(np.sqrt(2) * np.sqrt(D))
+    assert v > ATTN_ACT_BOUND * np.sqrt(D) * 1.0                 # above the bound of a single row
+    assert v <= ATTN_ACT_BOUND * np.sqrt(D) * np.sqrt(2.0)       # within the pair's bound
+    assert v / attn_fp8_scales(w, D, H, d)[0, 0] <= 448.0
+
+
+def test_oracle_stream_with_e4m3_attention_stays_near_the_exact_stream():
+    """The e4m3 attention changes the finished latents only by the format's rounding
+    (a few per cent on this flat-attention synthetic stack), block by block."""
+    from oracle import OracleStream
+    from workloads import DTYPE_BF16, SINK_AAS, StreamConfig, Workload, block_noise, make_weights
+    cfg = StreamConfig(num_layers=2, hidden=256, heads=2, head_dim=128, latent_ch=32, grid_h=4, grid_w=6,
+                       window_blocks=2, sink_mode=SINK_AAS, dtype=DTYPE_BF16, attn_fp8=1)
+    wl = Workload("afp8", cfg, 5, 4, 1.5 / 16.0, 0.1)
+    W = make_weights(wl)
+    o8, o = OracleStream(cfg, W), OracleStream(cfg.replace(attn_fp8=0), W)
+    o8.set_sink(W.sink)
+    o.set_sink(W.sink)
+    for k in range(wl.num_blocks + 3):
+        xn = block_noise(wl, k) if k < wl.num_blocks else None
+        a, fa = o8.denoise_step(xn)
+        b, fb = o.denoise_step(xn)
+        assert fa == fb
+        if fa >= 0:
+            rel = np.abs(a - b).sum() / np.abs(b).sum()
+            assert 1e-3 < rel < 0.08, (fa, rel)

@@ -61,6 +61,7 @@ class StreamConfig:
     dtype: int = DTYPE_BF16
     cache_mode: int = CACHE_TIMESTEP
     proj_fp8: int = 0        # 1: QKV / output projections on per-row-quantized e4m3 operands (bf16 streams)
+    attn_fp8: int = 0        # 1: the denoising passes' attention on e4m3 q / K / V (bf16 streams, head_dim 128)
 
     @property
     def num_steps(self) -> int:
