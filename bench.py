@@ -439,12 +439,18 @@ def run_ablation(args):
 
     torch.cuda.set_device(0)
     bf = torch.bfloat16
-    for name, sched, mode, nfe, fp8 in (
-            ("timestep-forced, grouped pipeline", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0),
-            ("timestep-forced, sequential", SCHED_SEQUENTIAL, CACHE_TIMESTEP, 4, 0),
-            ("clean-cache refresh, sequential", SCHED_SEQUENTIAL, CACHE_CLEAN_REFRESH, 5, 0),
-            ("timestep-forced, grouped pipeline, e4m3 projections", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 1)):
-        cfg = STREAM.cfg.replace(schedule=sched, cache_mode=mode, proj_fp8=fp8)
+    only = set(args.ablation_rows.split(",")) if args.ablation_rows else None
+    rows = (("timestep-forced, grouped pipeline", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0, 0),
+            ("timestep-forced, sequential", SCHED_SEQUENTIAL, CACHE_TIMESTEP, 4, 0, 0),
+            ("clean-cache refresh, sequential", SCHED_SEQUENTIAL, CACHE_CLEAN_REFRESH, 5, 0, 0),
+            ("timestep-forced, grouped pipeline, e4m3 projections", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 1, 0),
+            ("timestep-forced, grouped pipeline, e4m3 attention", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0, 1),
+            ("timestep-forced, grouped pipeline, e4m3 projections and attention", SCHED_PIPELINED,
+             CACHE_TIMESTEP, 4, 1, 1))
+    for idx, (name, sched, mode, nfe, fp8, afp8) in enumerate(rows):
+        if only is not None and str(idx) not in only:
+            continue
+        cfg = STREAM.cfg.replace(schedule=sched, cache_mode=mode, proj_fp8=fp8, attn_fp8=afp8)
         T, C, D, F = cfg.block_tokens, cfg.latent_ch, cfg.hidden, cfg.frame_tokens
         S, nw, L = cfg.num_steps, cfg.window_blocks, cfg.num_layers
         g = torch.Generator(device="cuda")
@@ -476,7 +482,9 @@ def run_ablation(args):
                           "latent_frames_per_s": round(cfg.frames_per_block / (ms / 1000.0), 3),
                           "ms_per_block_by_kind": kinds,
                           "config": "8 sublayers, hidden 5120, 40x128 heads, 30x52 grid, window 2, "
-                                    + ("e4m3 QKV/output projections, bf16 elsewhere" if fp8 else "bf16")}),
+                                    + ", ".join([x for x in ("e4m3 QKV/output projections" if fp8 else "",
+                                                             "e4m3 attention" if afp8 else "") if x]
+                                                or ["bf16"])}),
               flush=True)
         s.close()
         del s, weights
@@ -513,6 +521,8 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="shape sweep lines instead of the headline line")
     ap.add_argument("--ablation", action="store_true",
                     help="seconds per block: grouped pipeline vs sequential vs clean-cache refresh")
+    ap.add_argument("--ablation-rows", default="",
+                    help="comma-separated row indices of --ablation to run (default: all)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
