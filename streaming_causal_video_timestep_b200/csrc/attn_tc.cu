@@ -65,10 +65,11 @@ constexpr float FP8_TAU = 3.0f;
 
 // A 128 x 128 tile: two boxes of 64 bf16 columns, or one box of 128 e4m3 columns.
 template <bool FP8> __host__ __device__ constexpr uint32_t tile_bytes() { return FP8 ? HALF : 2 * HALF; }
-// Stages of the K/V ring.
-template <bool FP8> __host__ __device__ constexpr int kv_stages() { return FP8 ? 8 : 5; }
+// The K/V ring holds one key-tile step per stage: stage of step p = [V(p-1) | K(p)]
+// (step 0: K(0) only; step nt: V(nt-1) only), under one full and one empty barrier.
+template <bool FP8> __host__ __device__ constexpr int kv_stages() { return FP8 ? 4 : 2; }
 template <bool FP8> __host__ __device__ constexpr size_t smem_bytes() {
-  return 1024 + 2 * tile_bytes<FP8>() /*Q_A, Q_B*/ + kv_stages<FP8>() * tile_bytes<FP8>() /*K, V ring*/ + 256;
+  return 1024 + 2 * tile_bytes<FP8>() /*Q_A, Q_B*/ + kv_stages<FP8>() * 2 * tile_bytes<FP8>() /*ring*/ + 256;
 }
 
 __device__ __forceinline__ uint32_t s_col(int w) { return static_cast<uint32_t>(w * 128); }
@@ -230,7 +231,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                       // Q_A at 0, Q_B at TILE
   uint8_t* sKV = smem + 2 * TILE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * TILE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * 2 * TILE);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + NS;
@@ -284,25 +285,28 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
         tma_load_4d(sQ + w * TILE, &maps.q, q_full, 0, q0 + w * BQ, h, g.q_slice);
         if (!FP8) tma_load_4d(sQ + w * TILE + HALF, &maps.q, q_full, 64, q0 + w * BQ, h, g.q_slice);
       }
-      SegCursor cur;
-      int n = 0;
-      for (int t = 0; t < nt && !abort_flag; ++t) {
-        const AttnSeg& sg = g.seg[cur.seg];
-#pragma unroll
-        for (int kv = 0; kv < 2; ++kv) {
-          const int stage = n % NS;
-          const uint32_t par = static_cast<uint32_t>((n / NS) & 1);
-          if (!mbar_wait(&kv_empty[stage], par ^ 1, err)) { abort_flag = 1; break; }
-          const CUtensorMap* m = kv == 0 ? &maps.k[sg.kmap] : &maps.v[sg.vmap];
-          const int slice = kv == 0 ? sg.kslice : sg.vslice;
-          uint8_t* dst = sKV + stage * TILE;
-          mbar_expect_tx(&kv_full[stage], TILE);
-          tma_load_4d(dst, m, &kv_full[stage], 0, cur.start, h, slice);
-          if (!FP8) tma_load_4d(dst + HALF, m, &kv_full[stage], 64, cur.start, h, slice);
-          last_parity[stage] = static_cast<int>(par);
-          ++n;
+      // step p of the ring: V(p-1) at the stage's start, K(p) one tile further
+      SegCursor ck, cv;
+      for (int p = 0; p <= nt && !abort_flag; ++p) {
+        const int stage = p % NS;
+        const uint32_t par = static_cast<uint32_t>((p / NS) & 1);
+        if (!mbar_wait(&kv_empty[stage], par ^ 1, err)) { abort_flag = 1; break; }
+        const bool has_v = p >= 1, has_k = p < nt;
+        uint8_t* dst = sKV + stage * 2 * TILE;
+        mbar_expect_tx(&kv_full[stage], (has_v ? TILE : 0u) + (has_k ? TILE : 0u));
+        if (has_v) {
+          const AttnSeg& sg = g.seg[cv.seg];
+          tma_load_4d(dst, &maps.v[sg.vmap], &kv_full[stage], 0, cv.start, h, sg.vslice);
+          if (!FP8) tma_load_4d(dst + HALF, &maps.v[sg.vmap], &kv_full[stage], 64, cv.start, h, sg.vslice);
+          cv.next(g);
         }
-        cur.next(g);
+        if (has_k) {
+          const AttnSeg& sg = g.seg[ck.seg];
+          tma_load_4d(dst + TILE, &maps.k[sg.kmap], &kv_full[stage], 0, ck.start, h, sg.kslice);
+          if (!FP8) tma_load_4d(dst + TILE + HALF, &maps.k[sg.kmap], &kv_full[stage], 64, ck.start, h, sg.kslice);
+          ck.next(g);
+        }
+        last_parity[stage] = static_cast<int>(par);
       }
       mbar_wait(q_full, 0, err);
       for (int i = 0; i < NS; ++i)
@@ -319,7 +323,7 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       // bits; every shared address here is below 256 KB, so adding (offset >> 4)
       // moves a descriptor by `offset` bytes without a carry out of the field.
       const uint64_t dQ = sdesc_kmajor(smem_u32(sQ));
-      const uint64_t dK = sdesc_kmajor(smem_u32(sKV));
+      const uint64_t dK = sdesc_kmajor(smem_u32(sKV + TILE));
       const uint64_t dV = sdesc_mnmajor(smem_u32(sKV), HALF);
       // One K step is 32 bytes of a 128-byte row: 16 bf16 or 32 e4m3 head dims.
       auto issue_s = [&](int w, uint32_t stage) {
@@ -327,14 +331,14 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t off = kk * 32;
-            umma_e4m3_ss(tmem + s_col(w), dQ + ((w * TILE + off) >> 4), dK + ((stage * TILE + off) >> 4), idS,
+            umma_e4m3_ss(tmem + s_col(w), dQ + ((w * TILE + off) >> 4), dK + ((stage * 2 * TILE + off) >> 4), idS,
                          kk > 0 ? 1u : 0u);
           }
         } else {
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk) {
             const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
-            umma_bf16_ss(tmem + s_col(w), dQ + ((w * TILE + off) >> 4), dK + ((stage * TILE + off) >> 4), idS,
+            umma_bf16_ss(tmem + s_col(w), dQ + ((w * TILE + off) >> 4), dK + ((stage * 2 * TILE + off) >> 4), idS,
                          kk > 0 ? 1u : 0u);
           }
         }
@@ -346,11 +350,11 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
         for (int w = 0; w < nq; ++w) issue_s(w, 0);
         umma_commit(&kv_empty[0]);
       }
-      // V(t) is load 2t+1 and K(t+1) load 2t+2 of the ring: stage n % NS, phase (n / NS) & 1
-      uint32_t vs = 1, ks = 2, vpar = 0, kpar = 0;
+      // step t reads ring step t+1 = [V(t) | K(t+1)]: stage (t+1) % NS, phase ((t+1) / NS) & 1
+      uint32_t vs = 1 % NS, vpar = (1 / NS) & 1;
       for (int t = 0; t < nt && ok; ++t) {
         const bool more = t + 1 < nt;
-        ok = mbar_wait(&kv_full[vs], vpar, err) && (!more || mbar_wait(&kv_full[ks], kpar, err));
+        ok = mbar_wait(&kv_full[vs], vpar, err);
         if (!ok) break;
         for (int w = 0; w < nq; ++w) {
           if (!mbar_wait(&p_full[w], static_cast<uint32_t>(t & 1), err)) { ok = false; break; }
@@ -360,26 +364,22 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
           if (FP8) {
 #pragma unroll
             for (int kk = 0; kk < BKV / 32; ++kk)
-              umma_e4m3_ts(tmem + o_col(w), tmem + s_col(w) + kk * 8, dV + ((vs * TILE + kk * 4096) >> 4), idPV,
+              umma_e4m3_ts(tmem + o_col(w), tmem + s_col(w) + kk * 8, dV + ((vs * 2 * TILE + kk * 4096) >> 4), idPV,
                            (t > 0 || kk > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int kk = 0; kk < BKV / 16; ++kk)
-              umma_bf16_ts(tmem + o_col(w), tmem + s_col(w) + kk * 8, dV + ((vs * TILE + kk * 2048) >> 4), idPV,
+              umma_bf16_ts(tmem + o_col(w), tmem + s_col(w) + kk * 8, dV + ((vs * 2 * TILE + kk * 2048) >> 4), idPV,
                            (t > 0 || kk > 0) ? 1u : 0u);
           }
           if (more)
-            issue_s(w, ks);
+            issue_s(w, vs);
           else
             umma_commit(&pv_done[w]);
         }
         if (!ok) break;
         umma_commit(&kv_empty[vs]);
-        if (more) umma_commit(&kv_empty[ks]);
-        vs += 2;
-        if (vs >= NS) { vs -= NS; vpar ^= 1u; }
-        ks += 2;
-        if (ks >= NS) { ks -= NS; kpar ^= 1u; }
+        if (++vs == NS) { vs = 0; vpar ^= 1u; }
       }
       if (!ok) abort_flag = 1;
       umma_commit(drain);
