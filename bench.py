@@ -38,10 +38,10 @@ WORKLOAD = dict(
 
 
 # DRAM bytes (read + write) of one slot's attention launch (4680 queries x 15,600 keys x 40 heads x 128,
-# bf16 q/K/V and output) from one ncu capture of the one-slot attention microbenchmark: 379.7 MB read +
-# 41.2 MB written, against 415.2 MB of algorithmic bytes.  The grouped launch of the stream reads the
+# bf16 q/K/V and output) from one ncu capture of the one-slot attention microbenchmark: 386.0 MB read +
+# 41.3 MB written, against 415.2 MB of algorithmic bytes.  The grouped launch of the stream reads the
 # disjoint q / K / V of its S slots, so its traffic is S times this.
-ATTN_DRAM_BYTES_PER_SLOT = 420.8e6
+ATTN_DRAM_BYTES_PER_SLOT = 427.3e6
 
 
 def max_over_ranks(x, device):
