@@ -28,12 +28,21 @@ clean K/V serves every step, so all slots share ring 0 (their records describe
 it); after the last step of block b one more pass runs the stack on the
 finished latent and overwrites block b's entry, tagged (b, num_steps).  Only
 in the sequential schedule.
+
+Fixed-noise cache (the other alternative to timestep forcing that the
+papernotes note's key findings compare, the paper's Table 6: "fixed noise or
+clean cache"; admirer.cn article: same-step memory against clean memory):
+reading: the prior blocks a step reads come from the cache of one fixed step
+j = cache_step, whatever the current step; every step still writes its own
+cache and attends to its own block's current K/V.  Only in the sequential
+schedule (in the grouped pipeline step j's pass of a later block would evict
+an entry that another slot of the same launch reads).
 """
 from __future__ import annotations
 
 import numpy as np
 
-from workloads import CACHE_CLEAN_REFRESH, SCHED_PIPELINED, SINK_AAS
+from workloads import CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, SCHED_PIPELINED, SINK_AAS
 
 
 def index_state_layout(cfg):
@@ -44,10 +53,13 @@ def index_state_layout(cfg):
 
 class TickScheduler:
     def __init__(self, cfg):
-        if cfg.cache_mode == CACHE_CLEAN_REFRESH and cfg.schedule == SCHED_PIPELINED:
-            raise ValueError("the clean-cache refresh runs in the sequential schedule")
+        if cfg.cache_mode in (CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP) and cfg.schedule == SCHED_PIPELINED:
+            raise ValueError("the clean-cache refresh and the fixed-noise cache run in the sequential schedule")
+        if cfg.cache_mode == CACHE_FIXED_STEP and not 0 <= cfg.cache_step < cfg.num_steps:
+            raise ValueError("cache_step must name one of the steps")
         self.cfg = cfg
         self.clean = cfg.cache_mode == CACHE_CLEAN_REFRESH
+        self.fixed = cfg.cache_step if cfg.cache_mode == CACHE_FIXED_STEP else None
         S, E = cfg.num_steps, cfg.ring_entries
         self.S, self.E = S, E
         self.slots = [-1] * S          # block held by each slot after the last tick
@@ -93,8 +105,12 @@ class TickScheduler:
         return False
 
     def ring_of(self, i: int) -> int:
-        """The cache slot i reads and writes: its own, or the one clean cache."""
+        """The cache slot i writes (and reads its own block from): its own, or the one clean cache."""
         return 0 if self.clean else i
+
+    def window_ring(self, i: int) -> int:
+        """The cache slot i reads the prior blocks from: its own, the clean one, or step cache_step's."""
+        return self.fixed if self.fixed is not None else self.ring_of(i)
 
     def append(self, i: int, b: int):
         """Ring append of block b at step i; returns the slot's record."""
@@ -122,7 +138,7 @@ class TickScheduler:
 
     def window_blocks(self, i, b):
         """Prior blocks block b reads at step i, oldest first."""
-        return [x for x in self.resident(self.ring_of(i)) if b - self.cfg.window_blocks <= x < b]
+        return [x for x in self.resident(self.window_ring(i)) if b - self.cfg.window_blocks <= x < b]
 
     def sink_tpos(self, b: int) -> int:
         cfg = self.cfg

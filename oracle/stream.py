@@ -44,6 +44,10 @@ e4m3 codes over one power-of-two scale per (layer, q|K|V, head) fixed from the
 weights (oracle/fp8.py attn_fp8_scales), and the attention is
 oracle/fp8.py attention_fp8 over [sink | window oldest first | block].  The
 sink's own pass keeps the plain attention.
+
+Fixed-noise cache (cfg.cache_mode == CACHE_FIXED_STEP; oracle/schedule.py):
+the window blocks come from the cache written at step cfg.cache_step, the
+block itself from the current step's K/V.
 """
 from __future__ import annotations
 
@@ -160,8 +164,11 @@ class OracleStream:
                 self.cache[(l, ring, b)] = (kr, v.copy(), (b, c.num_steps if refresh else i))
             self.cache.pop((l, ring, b - c.window_blocks - 1), None)
             sk = rope_rotate(self.sink_k[l], st, sh, sw, c.pairs, c.rope_theta)
+            # prior blocks from the window's cache, the block itself from this pass
+            wring = ring if refresh else self.sched.window_ring(i)
             blocks = {bb: (kk, vv) for (ll, rr, bb), (kk, vv, _) in self.cache.items()
-                      if ll == l and rr == ring}
+                      if ll == l and rr == wring and bb < b}
+            blocks[b] = self.cache[(l, ring, b)][:2]
             if sc is not None:
                 # [sink | window oldest first | block]: every assembled key is visible
                 order = sorted(bb for bb in blocks if b - c.window_blocks <= bb <= b)

@@ -108,8 +108,11 @@ class BruteStream:
             proj = matvec_rows(o, self.wout[l])
             h = [[a + b for a, b in zip(hr, pr)] for hr, pr in zip(h, proj)]
 
-    def step(self, x, b, i):
+    def step(self, x, b, i, win_step=None):
+        """Block b at step i; the prior blocks' K/V come from step win_step's entries
+        (default: step i's own, timestep forcing)."""
         c = self.c
+        ws = i if win_step is None else win_step
         h = [list(map(float, r)) for r in x]
         if self.win is not None:
             h = matvec_rows(h, self.win)
@@ -128,7 +131,7 @@ class BruteStream:
             for (r, cc, kh, vh) in self.sink[l]:
                 visible.append(([rotate(x_, t_sink, r, cc, c.pairs, c.rope_theta) for x_ in kh], vh))
             for (ll, ii, bb, kr, vh) in self.keys:
-                if ll == l and ii == i and b - c.window_blocks <= bb <= b:
+                if ll == l and ((ii == ws and b - c.window_blocks <= bb < b) or (ii == i and bb == b)):
                     visible.append((kr, vh))
             o = self._layer_attend(qrot, visible)
             proj = matvec_rows(o, self.wout[l])
@@ -137,6 +140,21 @@ class BruteStream:
         v = hn if self.whead is None else matvec_rows(hn, self.whead)
         dt = c.timesteps[i + 1] - c.timesteps[i]
         return [[xa + dt * va for xa, va in zip(xr, vr)] for xr, vr in zip(x, v)]
+
+    def run_sequential_fixed(self, noises, win_step):
+        """Each block through its num_steps Euler steps in order; every step reads the
+        prior blocks' K/V written at step win_step (the fixed-noise cache)."""
+        c = self.c
+        done = {}
+        for b, nz in enumerate(noises):
+            x = [list(map(float, r)) for r in nz]
+            for i in range(c.num_steps):
+                x = self.step(x, b, i, win_step=win_step)
+            done[b] = x
+            if b == 0 and c.sink_mode == 1 and not self.replaced:
+                self.replaced = True
+                self.set_sink(x[: c.sink_tokens])
+        return done
 
     def run_pipelined(self, noises):
         """Tick k: slot i runs block k - i.  Returns {block: final latent}."""

@@ -13,8 +13,8 @@ import torch
 
 from oracle import OracleStream, TickScheduler, block_causal_attention, euler_step, rms_norm, rope_rotate
 from oracle.rope import axis_frequencies, block_positions, sink_positions, sink_temporal_position
-from workloads import (CACHE_CLEAN_REFRESH, CACHE_TIMESTEP, SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_AAS,
-                       SINK_FIXED, TINY, StreamConfig, Workload, block_noise, make_weights, random_array)
+from workloads import (CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, CACHE_TIMESTEP, SCHED_PIPELINED, SCHED_SEQUENTIAL,
+                       SINK_AAS, SINK_FIXED, TINY, StreamConfig, Workload, block_noise, make_weights, random_array)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pages_facts.json")
 
@@ -477,3 +477,59 @@ def test_clean_refresh_ring_tags_closed_form():
 def test_clean_refresh_needs_the_sequential_schedule():
     with pytest.raises(ValueError):
         TickScheduler(_clean_cfg(schedule=SCHED_PIPELINED))
+
+
+# -- the fixed-noise cache (every step reads the prior blocks of one step) ------------------------
+@pytest.mark.parametrize("window,j,sink_mode", [(1, 0, SINK_AAS), (2, 3, SINK_AAS), (2, 1, SINK_FIXED)])
+def test_fixed_noise_cache_oracle_matches_scalar_brute_force(window, j, sink_mode):
+    cfg = _clean_cfg(window_blocks=window, sink_mode=sink_mode, cache_mode=CACHE_FIXED_STEP, cache_step=j)
+    wl = Workload("brute-fixed", cfg, 16, 5, 0.25)
+    W = make_weights(wl)
+    noises = [block_noise(wl, b) for b in range(wl.num_blocks)]
+    from _brute import BruteStream
+    bs = BruteStream(cfg, W)
+    bs.set_sink(W.sink)
+    want = bs.run_sequential_fixed(noises, j)
+    s = OracleStream(cfg, W)
+    s.set_sink(W.sink)
+    for b in range(wl.num_blocks):
+        out, fin = s.denoise_step(noises[b])
+        assert fin == b
+        np.testing.assert_allclose(out, np.array(want[b]), rtol=1e-11, atol=1e-11)
+
+
+def test_fixed_noise_cache_is_timestep_forcing_without_a_window_and_differs_with_one():
+    """Window 0: no step reads another block, so the fixed-noise cache computes the
+    timestep-forced latents exactly; with a window the prior blocks come from another
+    step's K/V and the latents differ."""
+    for window, same in ((0, True), (1, False)):
+        outs = {}
+        for mode in (CACHE_TIMESTEP, CACHE_FIXED_STEP):
+            cfg = _clean_cfg(window_blocks=window, cache_mode=mode, cache_step=2)
+            wl = Workload("fx", cfg, 17, 4, 0.25)
+            W = make_weights(wl)
+            s = OracleStream(cfg, W)
+            s.set_sink(W.sink)
+            outs[mode] = [s.denoise_step(block_noise(wl, b))[0] for b in range(wl.num_blocks)]
+        for b, (a, c) in enumerate(zip(outs[CACHE_TIMESTEP], outs[CACHE_FIXED_STEP])):
+            if same or b == 0:
+                # equal up to summation order (a masked key of weight 0 can join the product)
+                np.testing.assert_allclose(a, c, rtol=1e-12, atol=1e-12)
+            else:
+                assert np.abs(a - c).max() > 1e-6
+
+
+def test_fixed_noise_cache_window_reads_the_fixed_step_ring():
+    cfg = _clean_cfg(window_blocks=2, cache_mode=CACHE_FIXED_STEP, cache_step=1)
+    ts = TickScheduler(cfg)
+    for b in range(5):
+        run, fin = ts.begin_tick(True)
+        for i, bb in run:
+            assert ts.window_blocks(i, bb) == list(range(max(0, bb - 2), bb))
+            assert ts.window_ring(i) == 1 and ts.ring_of(i) == i
+            ts.append(i, bb)
+        ts.end_tick(fin)
+    with pytest.raises(ValueError):
+        TickScheduler(_clean_cfg(cache_mode=CACHE_FIXED_STEP, cache_step=4))
+    with pytest.raises(ValueError):
+        TickScheduler(_clean_cfg(cache_mode=CACHE_FIXED_STEP, schedule=SCHED_PIPELINED))

@@ -29,6 +29,7 @@ DTYPE_BF16 = 0
 DTYPE_FP32 = 1
 CACHE_TIMESTEP = 0         # noisy K/V of each step in that step's own cache (timestep forcing)
 CACHE_CLEAN_REFRESH = 1    # one cache of clean K/V, refreshed by an extra forward of x0 per block (NFE S+1)
+CACHE_FIXED_STEP = 2       # every step reads the prior blocks' K/V of one fixed step (cache_step): fixed noise
 
 
 def default_rope_split(head_dim: int) -> tuple:
@@ -62,6 +63,7 @@ class StreamConfig:
     cache_mode: int = CACHE_TIMESTEP
     proj_fp8: int = 0        # 1: QKV / output projections on per-row-quantized e4m3 operands (bf16 streams)
     attn_fp8: int = 0        # 1: the denoising passes' attention on e4m3 q / K / V (bf16 streams, head_dim 128)
+    cache_step: int = 0      # CACHE_FIXED_STEP: the step whose K/V every step reads for the prior blocks
 
     @property
     def num_steps(self) -> int:
