@@ -432,10 +432,12 @@ def run_ablation(args):
     schedules the pages compare (papernotes note, inference-efficiency ablation, the paper's Table 3): the grouped timestep-forced stream
     (4 blocks in flight, NFE 4), the same cache sequentially (one block through its 4 steps per
     call, NFE 4), and the clean-cache refresh the method removes (4 steps + 1 refresh forward,
-    NFE 5).  One JSON line each."""
+    NFE 5); the e4m3 rows of the operator-optimisation row; and the fixed-noise cache the
+    key findings compare (the paper's Table 6; same kernels and NFE as the sequential row).
+    One JSON line each."""
     import torch
     from streaming_causal_video_timestep_b200 import LaStream
-    from workloads import CACHE_CLEAN_REFRESH, CACHE_TIMESTEP, SCHED_PIPELINED, SCHED_SEQUENTIAL, STREAM
+    from workloads import CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, CACHE_TIMESTEP, SCHED_PIPELINED, SCHED_SEQUENTIAL, STREAM
 
     torch.cuda.set_device(0)
     bf = torch.bfloat16
@@ -446,11 +448,14 @@ def run_ablation(args):
             ("timestep-forced, grouped pipeline, e4m3 projections", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 1, 0),
             ("timestep-forced, grouped pipeline, e4m3 attention", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0, 1),
             ("timestep-forced, grouped pipeline, e4m3 projections and attention", SCHED_PIPELINED,
-             CACHE_TIMESTEP, 4, 1, 1))
+             CACHE_TIMESTEP, 4, 1, 1),
+            ("fixed-noise cache (prior blocks at the last step's noise), sequential", SCHED_SEQUENTIAL,
+             CACHE_FIXED_STEP, 4, 0, 0))
     for idx, (name, sched, mode, nfe, fp8, afp8) in enumerate(rows):
         if only is not None and str(idx) not in only:
             continue
-        cfg = STREAM.cfg.replace(schedule=sched, cache_mode=mode, proj_fp8=fp8, attn_fp8=afp8)
+        cfg = STREAM.cfg.replace(schedule=sched, cache_mode=mode, proj_fp8=fp8, attn_fp8=afp8,
+                                 cache_step=STREAM.cfg.num_steps - 1)
         T, C, D, F = cfg.block_tokens, cfg.latent_ch, cfg.hidden, cfg.frame_tokens
         S, nw, L = cfg.num_steps, cfg.window_blocks, cfg.num_layers
         g = torch.Generator(device="cuda")

@@ -74,6 +74,13 @@ extern "C" {
                                    finished latent rewrites its entry (NFE num_steps+1;
                                    papernotes note, key design 2 and the paper's Table 3; gitcode
                                    blog, question 4).  Sequential schedule only.       */
+#define LA_CACHE_FIXED_STEP  2  /* the other alternative the pages compare ("fixed noise or
+                                   clean cache", papernotes note, key findings = the
+                                   paper's Table 6): every step reads the prior blocks'
+                                   K/V written at one fixed step (cache_step); each step
+                                   still writes its own cache and attends to its own
+                                   block's current K/V.  NFE num_steps.  Sequential
+                                   schedule only.                                      */
 
 #define LA_RMS_EPS 1e-6
 
@@ -108,7 +115,7 @@ typedef struct la_config {
   int32_t sink_offset_frames;  /* 3                                                      */
   int32_t schedule;            /* LA_SCHED_PIPELINED | LA_SCHED_SEQUENTIAL               */
   int32_t dtype;               /* LA_BF16 | LA_FP32                                      */
-  int32_t cache_mode;          /* LA_CACHE_TIMESTEP | LA_CACHE_CLEAN_REFRESH              */
+  int32_t cache_mode;          /* LA_CACHE_TIMESTEP | LA_CACHE_CLEAN_REFRESH | LA_CACHE_FIXED_STEP */
   int32_t proj_fp8;            /* 1 (LA_BF16 only): the QKV and output projections run on
                                   e4m3 operands: weights quantized per output row at
                                   creation, the bf16 GEMM operand per token before each
@@ -128,6 +135,9 @@ typedef struct la_config {
                                   1.07 covers the rounding of the GEMM operand).  The
                                   sink's own pass keeps bf16 attention.  Same row as
                                   proj_fp8.  0: bf16 attention.                          */
+  int32_t cache_step;          /* LA_CACHE_FIXED_STEP: the step (0 .. num_steps-1) whose
+                                  K/V of the prior blocks every step reads; ignored by
+                                  the other cache modes.                                */
 } la_config;
 
 /*

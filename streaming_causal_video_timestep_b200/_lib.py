@@ -28,7 +28,7 @@ class LaConfig(ctypes.Structure):
         ("timesteps", POINTER(c_float)), ("rope_split", c_int32 * 3), ("rope_theta", c_double),
         ("sink_mode", c_int32), ("rolling_rope", c_int32), ("sink_offset_frames", c_int32),
         ("schedule", c_int32), ("dtype", c_int32), ("cache_mode", c_int32), ("proj_fp8", c_int32),
-        ("attn_fp8", c_int32),
+        ("attn_fp8", c_int32), ("cache_step", c_int32),
     ]
 
 

@@ -22,7 +22,8 @@ struct PassDesc {
   int nactive;                       // active buffers, listed in active_buf
   int active_buf[LA_MAX_STEPS];
   int active[LA_MAX_STEPS];          // per buffer: 1 if it runs a step this pass
-  int slot[LA_MAX_STEPS];            // cache (ring slice) the buffer's block reads and writes
+  int slot[LA_MAX_STEPS];            // cache (ring slice) the buffer's block writes and reads itself from
+  int win_slot[LA_MAX_STEPS];        // cache the buffer's prior (window) blocks are read from
   int step[LA_MAX_STEPS];            // denoising step of the pass (num_steps: a clean-cache refresh)
   int block[LA_MAX_STEPS];
   int write_entry[LA_MAX_STEPS];     // ring entry the block's K/V go to

@@ -30,6 +30,7 @@ struct SlotRecord {
 
 struct Scheduler {
   int S = 0, E = 0, W = 0, fpb = 0, offset = 0, rolling = 1, pipelined = 1, aas = 0, clean = 0;
+  int fixed_step = -1;      // LA_CACHE_FIXED_STEP: the step whose cache every step reads the window from
   long long tick = -1, blocks_in = 0, blocks_out = 0;
   int sink_gen = 0;
   std::vector<long long> held;                  // block held by each slot after the last call
@@ -47,13 +48,16 @@ struct Scheduler {
     pipelined = c.schedule == LA_SCHED_PIPELINED;
     aas = c.sink_mode == LA_SINK_AAS;
     clean = c.cache_mode == LA_CACHE_CLEAN_REFRESH;
+    fixed_step = c.cache_mode == LA_CACHE_FIXED_STEP ? c.cache_step : -1;
     held.assign(S, -1);
     tag_blk.assign(S, std::vector<long long>(E, -1));
     tag_step.assign(S, std::vector<int>(E, -1));
     rec.assign(S, SlotRecord());
   }
-  // The cache step i reads and writes: its own, or the one clean cache.
+  // The cache step i writes (and reads its own block from): its own, or the one clean cache.
   int ring_of(int i) const { return clean ? 0 : i; }
+  // The cache step i reads the prior blocks from: its own, the clean one, or step fixed_step's.
+  int window_ring(int i) const { return fixed_step >= 0 ? fixed_step : ring_of(i); }
   int sink_tpos_of(long long b) const {
     return rolling ? static_cast<int>(fpb * b - offset) : -offset;
   }
@@ -327,7 +331,15 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
   if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) { msg = "rope_theta must be positive"; return LA_EINVAL; }
   if (c->sink_mode != LA_SINK_FIXED && c->sink_mode != LA_SINK_AAS) { msg = "bad sink_mode"; return LA_EINVAL; }
   if (c->schedule != LA_SCHED_PIPELINED && c->schedule != LA_SCHED_SEQUENTIAL) { msg = "bad schedule"; return LA_EINVAL; }
-  if (c->cache_mode != LA_CACHE_TIMESTEP && c->cache_mode != LA_CACHE_CLEAN_REFRESH) { msg = "bad cache_mode"; return LA_EINVAL; }
+  if (c->cache_mode != LA_CACHE_TIMESTEP && c->cache_mode != LA_CACHE_CLEAN_REFRESH &&
+      c->cache_mode != LA_CACHE_FIXED_STEP) {
+    msg = "bad cache_mode";
+    return LA_EINVAL;
+  }
+  if (c->cache_mode == LA_CACHE_FIXED_STEP) {
+    if (c->schedule != LA_SCHED_SEQUENTIAL) { msg = "the fixed-noise cache runs in the sequential schedule"; return LA_EINVAL; }
+    if (c->cache_step < 0 || c->cache_step >= c->num_steps) { msg = "cache_step must name one of the steps"; return LA_EINVAL; }
+  }
   if (c->proj_fp8 != 0 && c->proj_fp8 != 1) { msg = "proj_fp8 must be 0 or 1"; return LA_EINVAL; }
   if (c->proj_fp8 && c->dtype != LA_BF16) { msg = "e4m3 projections need the bf16 stream"; return LA_EINVAL; }
   if (c->attn_fp8 != 0 && c->attn_fp8 != 1) { msg = "attn_fp8 must be 0 or 1"; return LA_EINVAL; }
@@ -566,9 +578,10 @@ int run_pass(la_stream* s, const PassDesc& pd) {
       int ns = 0;
       g.seg[ns++] = AttnSeg{1, 1, buf, l, F};
       const long long base = static_cast<long long>(l) * S * E + static_cast<long long>(pd.slot[buf]) * E;
+      const long long wbase = static_cast<long long>(l) * S * E + static_cast<long long>(pd.win_slot[buf]) * E;
       for (int w = 0; w < pd.nwin[buf]; ++w)
-        g.seg[ns++] = AttnSeg{0, 0, static_cast<int>(base + pd.win_entry[buf][w]),
-                              static_cast<int>(base + pd.win_entry[buf][w]), T};
+        g.seg[ns++] = AttnSeg{0, 0, static_cast<int>(wbase + pd.win_entry[buf][w]),
+                              static_cast<int>(wbase + pd.win_entry[buf][w]), T};
       g.seg[ns++] = AttnSeg{0, 0, static_cast<int>(base + pd.write_entry[buf]),
                             static_cast<int>(base + pd.write_entry[buf]), T};
       g.nseg = ns;
@@ -723,6 +736,7 @@ void fill_pass_slot(la_stream* s, PassDesc& pd, int buf, int ring, int step, lon
   pd.active[buf] = 1;
   pd.active_buf[pd.nactive++] = buf;
   pd.slot[buf] = ring;
+  pd.win_slot[buf] = step < s->S ? s->sched.window_ring(step) : ring;
   pd.step[buf] = step;
   pd.block[buf] = static_cast<int>(b);
   pd.write_entry[buf] = write_entry;

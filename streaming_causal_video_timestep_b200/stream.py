@@ -73,6 +73,7 @@ class LaStream:
         c.cache_mode = getattr(cfg, "cache_mode", 0)
         c.proj_fp8 = getattr(cfg, "proj_fp8", 0)
         c.attn_fp8 = getattr(cfg, "attn_fp8", 0)
+        c.cache_step = getattr(cfg, "cache_step", 0)
         self.cfg = cfg
         self.c = c
         self.T = cfg.frames_per_block * cfg.grid_h * cfg.grid_w

@@ -18,7 +18,7 @@ from oracle import block_causal_attention, euler_step, rms_norm, rope_rotate
 from oracle.fp8 import (attention_fp8, attn_fp8_scales, dequantize_weight, project, quantize_heads,
                         quantize_rows)
 from oracle.rope import block_positions, sink_positions
-from workloads import DTYPE_BF16, bf16_round
+from workloads import CACHE_FIXED_STEP, DTYPE_BF16, bf16_round
 
 from _helpers import assert_close, to_np
 
@@ -89,6 +89,15 @@ def check_codes(codes, x, scales, what):
         assert np.all(same_sign & adjacent), f"{what}: non-adjacent e4m3 code"
     assert frac <= 1e-2, f"{what}: {frac:.2e} of the codes differ"
     return frac
+
+
+def _window_rings(s, cfg, l, i, ring_k, ring_v):
+    """The rings step i reads its prior blocks from: its own, or with the fixed-noise
+    cache step cache_step's ([E, T, H, d] each)."""
+    if getattr(cfg, "cache_mode", 0) != CACHE_FIXED_STEP or cfg.cache_step == i:
+        return ring_k, ring_v
+    j = cfg.cache_step
+    return (to_np(s.tap("ring_k", l, j)).transpose(0, 2, 1, 3), to_np(s.tap("ring_v", l, j)).transpose(0, 2, 1, 3))
 
 
 def check_sink(s, cfg, W, latent, rows=None, tag=""):
@@ -186,6 +195,7 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
             q_att = q_gpu
         ring_k = to_np(s.tap("ring_k", l, i)).transpose(0, 2, 1, 3)  # [E, T, H, d]
         ring_v = to_np(s.tap("ring_v", l, i)).transpose(0, 2, 1, 3)
+        win_k, win_v = _window_rings(s, cfg, l, i, ring_k, ring_v)
         e = b % E
         chk(q_gpu[R], qr, f"q l{l}")
         chk(ring_k[e][R], kr, f"ring K l{l}")
@@ -196,7 +206,8 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
         chk(sk_rope, rope_rotate(sk_raw, *st, cfg.pairs, cfg.rope_theta), f"sink K rope l{l}")
         sv = sink[1][l] if sink is not None else to_np(s.tap("sink_v", l)).transpose(1, 0, 2)
         # attention from the GPU's own q and cache contents
-        blocks = {bb: (ring_k[bb % E], ring_v[bb % E]) for bb in range(max(0, b - cfg.window_blocks), b + 1)}
+        blocks = {bb: (win_k[bb % E], win_v[bb % E]) for bb in range(max(0, b - cfg.window_blocks), b)}
+        blocks[b] = (ring_k[e], ring_v[e])
         o_want = block_causal_attention(q_att[R], blocks, (sk_rope, sv), qblock=b, window=cfg.window_blocks)
         o_gpu = to_np(s.tap("o", l, i))
         chk(o_gpu[R], o_want.reshape(len(R), D), f"attn O l{l}")
@@ -235,9 +246,10 @@ def _check_attn_fp8(s, cfg, W, b, i, l, R, qr, kr, v, sink, st, chk, errs, tag):
     fr["sink K codes"] = check_codes(sk8, rope_rotate(sk_raw, *st, cfg.pairs, cfg.rope_theta), sc[1],
                                      f"{tag} sink K codes l{l} b{b} s{i}")
     sv8 = sink[2][l] if sink is not None and len(sink) > 2 else to_np(s.tap("sink_v8", l)).transpose(1, 0, 2)
-    order = range(max(0, b - cfg.window_blocks), b + 1)
-    keys = np.concatenate([sk8] + [rk8[bb % E] for bb in order])
-    vals = np.concatenate([sv8] + [rv8[bb % E] for bb in order])
+    wk8, wv8 = _window_rings(s, cfg, l, i, rk8, rv8)
+    order = range(max(0, b - cfg.window_blocks), b)
+    keys = np.concatenate([sk8] + [wk8[bb % E] for bb in order] + [rk8[e]])
+    vals = np.concatenate([sv8] + [wv8[bb % E] for bb in order] + [rv8[e]])
     o_want = attention_fp8(q8[R], keys, vals, sc[0], sc[1], sc[2])
     chk(to_np(s.tap("o", l, i))[R], o_want.reshape(len(R), D), f"attn O (e4m3) l{l}")
     for k_, f_ in fr.items():

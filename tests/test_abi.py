@@ -91,6 +91,9 @@ def _weights(nonnull=True):
     dict(proj_fp8=1),                                 # e4m3 projections need the bf16 stream (dtype 1 = fp32)
     dict(proj_fp8=2, dtype=0, head_dim=128, hidden=128, latent_ch=128, rope_split=(22, 21, 21)),
     dict(attn_fp8=1),                                 # e4m3 attention needs the bf16 stream
+    dict(cache_mode=2, schedule=0),                   # the fixed-noise cache is sequential only
+    dict(cache_mode=2, schedule=1, cache_step=4),     # cache_step names a step
+    dict(cache_mode=3),
     dict(attn_fp8=2, dtype=0, head_dim=128, hidden=128, latent_ch=128, rope_split=(22, 21, 21)),
 ])
 def test_invalid_config_returns_einval(lib, over):

@@ -6,8 +6,8 @@ import numpy as np
 import pytest
 
 from oracle import OracleStream, TickScheduler
-from workloads import (CACHE_CLEAN_REFRESH, DTYPE_BF16, DTYPE_FP32, SCHED_PIPELINED, SCHED_SEQUENTIAL, SINK_AAS,
-                       SINK_FIXED, TINY, StreamConfig, Workload, block_noise, make_weights)
+from workloads import (CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, DTYPE_BF16, DTYPE_FP32, SCHED_PIPELINED,
+                       SCHED_SEQUENTIAL, SINK_AAS, SINK_FIXED, TINY, StreamConfig, Workload, block_noise, make_weights)
 
 from _helpers import assert_close, errors, make_stream, to_np
 from _percheck import check_sink, check_step, sink_snapshot
@@ -56,13 +56,14 @@ def _run_teacher_forced(wl, check_every_tick=True):
     S = cfg.num_steps
     per = 8 + 3 * cfg.ring_entries
     report = {}
-    for k in range(nb + S - 1):
+    drain = S - 1 if cfg.schedule == SCHED_PIPELINED else 0     # the sequential schedule has no pipeline
+    for k in range(nb + drain):
         xn = block_noise(wl, k) if k < nb else None
         sink = sink_snapshot(s, cfg)
         fin = s.step(_dev(xn) if xn is not None else None, x_out)
         st = s.index_state()
         ran = [(int(st[4 + i * per]), i) for i in range(S) if st[4 + i * per] >= 0]
-        if check_every_tick or k >= nb + S - 2:
+        if check_every_tick or k >= nb + drain - 1:
             for (b, i) in ran:
                 check_step(s, cfg, W, b, i, tag=f"tick {k}", report=report, sink=sink)
         inputs = {(b, i): to_np(s.tap("x_in", 0, i)) for (b, i) in ran}
@@ -239,6 +240,23 @@ def test_small_bf16_clean_cache_refresh_integer_state_and_drift():
     worst = _run_clean_refresh(Workload("small-bf16-clean", cfg, SMALL_BF16.seed, 5, SMALL_BF16.w_std,
                                         SMALL_BF16.head_std))
     print({"free-running drift": (f"{worst[0]:.2e}", f"{worst[1]:.2e}")})
+
+
+@pytest.mark.parametrize("window,j", [(1, 0), (2, 3), (2, 1)])
+def test_tiny_fp32_fixed_noise_cache_matches_oracle(window, j):
+    """The fixed-noise cache: every step reads the prior blocks of step j; fp32
+    free-running within 1e-5 and the integer state bit-exact every call."""
+    cfg = TINY.cfg.replace(schedule=SCHED_SEQUENTIAL, cache_mode=CACHE_FIXED_STEP, cache_step=j,
+                           window_blocks=window)
+    _run_clean_refresh(Workload(f"tiny-fixed-w{window}-j{j}", cfg, TINY.seed, TINY.num_blocks, TINY.w_std,
+                                TINY.head_std))
+
+
+def test_small_bf16_fixed_noise_cache_teacher_forced():
+    cfg = SMALL_BF16.cfg.replace(schedule=SCHED_SEQUENTIAL, cache_mode=CACHE_FIXED_STEP, cache_step=3)
+    report = _run_teacher_forced(Workload("small-bf16-fixed", cfg, SMALL_BF16.seed, 5, SMALL_BF16.w_std,
+                                          SMALL_BF16.head_std))
+    print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in report.items()})
 
 
 def test_small_bf16_stream_with_e4m3_projections_teacher_forced():
