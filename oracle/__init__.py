@@ -29,7 +29,10 @@ What it computes (Live Avatar, arXiv 2512.04677, as described on the pages):
   * the clean-cache refresh ablation (oracle/schedule.py, oracle/stream.py),
     and per-row e4m3 quantization with the FP8 GEMM plus FP8 attention
     (oracle/fp8.py) for the operator-optimisation row (papernotes note, the
-    paper's Table 3).
+    paper's Table 3);
+  * the full synthetic DiT block (oracle/dit.py): AdaLN-modulated attention
+    and tanh-GELU FFN sub-blocks with gated residuals (a reading after the
+    Wan-style block the model is built on; the pages give no internals).
 
 Everything is fp64 numpy with a dict-indexed cache, an explicit mask matrix and
 a naive softmax.  The readings taken where the pages are silent are listed in

@@ -48,12 +48,18 @@ sink's own pass keeps the plain attention.
 Fixed-noise cache (cfg.cache_mode == CACHE_FIXED_STEP; oracle/schedule.py):
 the window blocks come from the cache written at step cfg.cache_step, the
 block itself from the current step's K/V.
+
+Full DiT block (cfg.block_kind == BLOCK_DIT; oracle/dit.py): each layer is
+the AdaLN-modulated attention sublayer (gated residual) followed by the
+AdaLN-modulated GELU FFN (gated residual), with the AdaLN vectors of the
+step's timestep (the t = 0 set for the sink pass and the clean refresh).
 """
 from __future__ import annotations
 
 import numpy as np
 
 from .attention import block_causal_attention
+from .dit import ffn, modulate
 from .flow import euler_step
 from .fp8 import attention_fp8, attn_fp8_scales, dequantize_weight, project, quantize_heads, quantize_rows
 from .norm import rms_norm
@@ -78,6 +84,14 @@ class OracleStream:
         if getattr(cfg, "attn_fp8", 0):
             used = [dequantize_weight(q) for q in self.wq8] if fp8 else self.w_qkv
             self.attn_sc = [attn_fp8_scales(w, cfg.hidden, cfg.heads, cfg.head_dim) for w in used]
+        # full DiT block (cfg.block_kind == 1): FFN weights and the AdaLN table [L][S+1][6][D]
+        self.dit = getattr(cfg, "block_kind", 0) == 1
+        if self.dit:
+            if fp8 or getattr(cfg, "attn_fp8", 0):
+                raise ValueError("the DiT block runs without the e4m3 modes")
+            self.w1 = [f64(w) for w in weights.w_ffn1]
+            self.w2 = [f64(w) for w in weights.w_ffn2]
+            self.ada = np.asarray(weights.ada, np.float64)
         self.sched = TickScheduler(cfg)
         self.cache = {}            # (layer, ring, block) -> (k_roped, v, (block, step))
         self.sink_k = None         # per layer, un-roped [F, H, d]
@@ -104,6 +118,21 @@ class OracleStream:
     def _proj_out(self, l, o):
         return o @ self.w_out[l].T if self.wo8 is None else project(o, *self.wo8[l])
 
+    def _attn_operand(self, l, h, t_idx):
+        """The QKV projection's operand: n(h), or with the DiT block its AdaLN modulation."""
+        if not self.dit:
+            return rms_norm(h)
+        a = self.ada[l, t_idx]
+        return modulate(h, a[0], a[1])
+
+    def _attn_residual(self, l, h, proj, t_idx):
+        """h + the attention sublayer's output (gated in the DiT block), then the DiT's FFN sub-block."""
+        if not self.dit:
+            return h + proj
+        a = self.ada[l, t_idx]
+        h = h + a[2] * proj
+        return h + a[5] * ffn(modulate(h, a[3], a[4]), self.w1[l], self.w2[l])
+
     def project_in(self, x):
         x = np.asarray(x, np.float64)
         return x.copy() if self.w_in is None else x @ self.w_in.T
@@ -122,13 +151,13 @@ class OracleStream:
         pt, ph, pw = sink_positions(c, t0)
         self.sink_k, self.sink_v = [], []
         for l in range(c.num_layers):
-            q, k, v = self._split_heads(self._proj_qkv(l, rms_norm(h)))
+            q, k, v = self._split_heads(self._proj_qkv(l, self._attn_operand(l, h, c.num_steps)))
             self.sink_k.append(k.copy())
             self.sink_v.append(v.copy())
             qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
             kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
             o = block_causal_attention(qr, {}, (kr, v), qblock=0, window=c.window_blocks)
-            h = h + self._proj_out(l, o.reshape(h.shape[0], -1))
+            h = self._attn_residual(l, h, self._proj_out(l, o.reshape(h.shape[0], -1)), c.num_steps)
             if self.trace is not None:
                 self.trace[("sink", l)] = dict(k=k.copy(), v=v.copy(), o=o, h=h.copy())
 
@@ -152,8 +181,9 @@ class OracleStream:
             tr["x_in"] = x.copy()
             tr["h_in"] = h.copy()
             tr["record"] = list(rec) if rec is not None else None
+        t_idx = c.num_steps if refresh else i
         for l in range(c.num_layers):
-            q, k, v = self._split_heads(self._proj_qkv(l, rms_norm(h)))
+            q, k, v = self._split_heads(self._proj_qkv(l, self._attn_operand(l, h, t_idx)))
             qr = rope_rotate(q, pt, ph, pw, c.pairs, c.rope_theta)
             kr = rope_rotate(k, pt, ph, pw, c.pairs, c.rope_theta)
             sc = self.attn_sc[l] if self.attn_sc is not None else None
@@ -178,7 +208,7 @@ class OracleStream:
             else:
                 o = block_causal_attention(qr, blocks, (sk, self.sink_v[l]), qblock=b,
                                            window=c.window_blocks)
-            h = h + self._proj_out(l, o.reshape(h.shape[0], -1))
+            h = self._attn_residual(l, h, self._proj_out(l, o.reshape(h.shape[0], -1)), t_idx)
             if tr is not None:
                 tr[("layer", l)] = dict(q=qr, k=kr, v=v.copy(), sink_k=sk, o=o, h=h.copy())
         if refresh:

@@ -56,6 +56,34 @@ class BruteStream:
         self.replaced = False
         self.lat = {}
         self.clean = []       # clean-cache entries (layer, block, k_rot, v)
+        self.dit = getattr(cfg, "block_kind", 0) == 1
+        if self.dit:
+            self.w1 = [tolist(w) for w in W.w_ffn1]
+            self.w2 = [tolist(w) for w in W.w_ffn2]
+            self.ada = [[[[float(v) for v in vec] for vec in st] for st in lay] for lay in W.ada]
+
+    # -- the DiT block's pieces, scalar ------------------------------------------------------------
+    def _operand(self, h, l, t_idx):
+        """Per-token RMS norm, AdaLN-modulated in the DiT block."""
+        n = normalize_rows(h)
+        if not self.dit:
+            return n
+        sh, sc = self.ada[l][t_idx][0], self.ada[l][t_idx][1]
+        return [[v * (1.0 + sc[j]) + sh[j] for j, v in enumerate(row)] for row in n]
+
+    def _residual(self, h, proj, l, t_idx):
+        """h + attention output; in the DiT block gated, then + gated tanh-GELU FFN."""
+        if not self.dit:
+            return [[a + b for a, b in zip(hr, pr)] for hr, pr in zip(h, proj)]
+        a = self.ada[l][t_idx]
+        h = [[x + a[2][j] * p for j, (x, p) in enumerate(zip(hr, pr))] for hr, pr in zip(h, proj)]
+        n = normalize_rows(h)
+        m = [[v * (1.0 + a[4][j]) + a[3][j] for j, v in enumerate(row)] for row in n]
+        u = matvec_rows(m, self.w1[l])
+        g = [[0.5 * z * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (z + 0.044715 * z * z * z))) for z in row]
+             for row in u]
+        f = matvec_rows(g, self.w2[l])
+        return [[x + a[5][j] * y for j, (x, y) in enumerate(zip(hr, fr))] for hr, fr in zip(h, f)]
 
     def _heads(self, vec, part):
         c = self.c
@@ -95,7 +123,7 @@ class BruteStream:
         t0 = -c.sink_offset_frames
         self.sink = []
         for l in range(c.num_layers):
-            qkv = matvec_rows(normalize_rows(h), self.wqkv[l])
+            qkv = matvec_rows(self._operand(h, l, c.num_steps), self.wqkv[l])
             entries, qrot, krot = [], [], []
             for n, vec in enumerate(qkv):
                 _, r, cc = self._tok_rc(n)
@@ -106,7 +134,7 @@ class BruteStream:
             self.sink.append(entries)
             o = self._layer_attend(qrot, krot)
             proj = matvec_rows(o, self.wout[l])
-            h = [[a + b for a, b in zip(hr, pr)] for hr, pr in zip(h, proj)]
+            h = self._residual(h, proj, l, c.num_steps)
 
     def step(self, x, b, i, win_step=None):
         """Block b at step i; the prior blocks' K/V come from step win_step's entries
@@ -119,7 +147,7 @@ class BruteStream:
         fpb = c.frames_per_block
         t_sink = fpb * b - c.sink_offset_frames if c.rolling_rope else -c.sink_offset_frames
         for l in range(c.num_layers):
-            qkv = matvec_rows(normalize_rows(h), self.wqkv[l])
+            qkv = matvec_rows(self._operand(h, l, i), self.wqkv[l])
             qrot = []
             for n, vec in enumerate(qkv):
                 f, r, cc = self._tok_rc(n)
@@ -135,7 +163,7 @@ class BruteStream:
                     visible.append((kr, vh))
             o = self._layer_attend(qrot, visible)
             proj = matvec_rows(o, self.wout[l])
-            h = [[a + bq for a, bq in zip(hr, pr)] for hr, pr in zip(h, proj)]
+            h = self._residual(h, proj, l, i)
         hn = normalize_rows(h)
         v = hn if self.whead is None else matvec_rows(hn, self.whead)
         dt = c.timesteps[i + 1] - c.timesteps[i]

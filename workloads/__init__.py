@@ -30,6 +30,8 @@ DTYPE_FP32 = 1
 CACHE_TIMESTEP = 0         # noisy K/V of each step in that step's own cache (timestep forcing)
 CACHE_CLEAN_REFRESH = 1    # one cache of clean K/V, refreshed by an extra forward of x0 per block (NFE S+1)
 CACHE_FIXED_STEP = 2       # every step reads the prior blocks' K/V of one fixed step (cache_step): fixed noise
+BLOCK_ATTN = 0             # each layer: the attention sublayer of the step
+BLOCK_DIT = 1              # each layer: a full DiT block (AdaLN-modulated attention and GELU FFN sub-blocks)
 
 
 def default_rope_split(head_dim: int) -> tuple:
@@ -64,6 +66,8 @@ class StreamConfig:
     proj_fp8: int = 0        # 1: QKV / output projections on per-row-quantized e4m3 operands (bf16 streams)
     attn_fp8: int = 0        # 1: the denoising passes' attention on e4m3 q / K / V (bf16 streams, head_dim 128)
     cache_step: int = 0      # CACHE_FIXED_STEP: the step whose K/V every step reads for the prior blocks
+    block_kind: int = BLOCK_ATTN
+    ffn_dim: int = 0         # BLOCK_DIT: hidden width of the FFN
 
     @property
     def num_steps(self) -> int:
@@ -184,10 +188,16 @@ class Weights:
     w_in: Optional[np.ndarray]
     w_head: Optional[np.ndarray]
     sink: np.ndarray            # [sink_tokens, latent_ch] float32 reference sink latent
+    w_ffn1: Optional[list] = None   # BLOCK_DIT: per layer [ffn_dim, hidden]
+    w_ffn2: Optional[list] = None   # BLOCK_DIT: per layer [hidden, ffn_dim]
+    ada: Optional[np.ndarray] = None  # BLOCK_DIT: float32 [L][num_steps + 1][6][hidden]
 
 
 def make_weights(wl: Workload) -> Weights:
-    """Draw order: per layer W_qkv then W_out, then W_in, W_head, then the sink."""
+    """Draw order: per layer W_qkv then W_out, then W_in, W_head, then the sink; for
+    BLOCK_DIT then per layer W_ffn1, W_ffn2, then the AdaLN table.  The AdaLN vectors
+    of a (layer, timestep) are [shift1, scale1, gate1, shift2, scale2, gate2]: shifts
+    and scales N(0, 0.1^2), gates N(1, 0.1^2); timestep index num_steps is t = 0."""
     c = wl.cfg
     D, C = c.hidden, c.latent_ch
     rng = np.random.default_rng(wl.seed)
@@ -200,7 +210,16 @@ def make_weights(wl: Workload) -> Weights:
         w_in = _to_dtype(rng.standard_normal((D, C)) / np.sqrt(C), c.dtype)
         w_head = _to_dtype(rng.standard_normal((C, D)) * wl.head_std, c.dtype)
     sink = rng.standard_normal((c.sink_tokens, C)).astype(np.float32)
-    return Weights(w_qkv, w_out, w_in, w_head, sink)
+    if c.block_kind != BLOCK_DIT:
+        return Weights(w_qkv, w_out, w_in, w_head, sink)
+    w1, w2 = [], []
+    for _ in range(c.num_layers):
+        w1.append(_to_dtype(rng.standard_normal((c.ffn_dim, D)) * wl.w_std, c.dtype))
+        w2.append(_to_dtype(rng.standard_normal((D, c.ffn_dim)) * wl.w_std, c.dtype))
+    ada = rng.standard_normal((c.num_layers, c.num_steps + 1, 6, D)) * 0.1
+    ada[:, :, 2] += 1.0
+    ada[:, :, 5] += 1.0
+    return Weights(w_qkv, w_out, w_in, w_head, sink, w1, w2, ada.astype(np.float32))
 
 
 def block_noise(wl: Workload, b: int) -> np.ndarray:
