@@ -42,6 +42,8 @@ WORKLOAD = dict(
 # 41.3 MB written, against 415.2 MB of algorithmic bytes.  The grouped launch of the stream reads the
 # disjoint q / K / V of its S slots, so its traffic is S times this.
 ATTN_DRAM_BYTES_PER_SLOT = 427.3e6
+# FFN width of the full DiT block in the ablation: the 14B Wan-style DiT's 13824 (2.7 x 5120)
+DIT_FFN = 13824
 
 
 def max_over_ranks(x, device):
@@ -437,25 +439,29 @@ def run_ablation(args):
     One JSON line each."""
     import torch
     from streaming_causal_video_timestep_b200 import LaStream
-    from workloads import CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, CACHE_TIMESTEP, SCHED_PIPELINED, SCHED_SEQUENTIAL, STREAM
+    from workloads import (BLOCK_ATTN, BLOCK_DIT, CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, CACHE_TIMESTEP,
+                           SCHED_PIPELINED, SCHED_SEQUENTIAL, STREAM)
 
     torch.cuda.set_device(0)
     bf = torch.bfloat16
     only = set(args.ablation_rows.split(",")) if args.ablation_rows else None
-    rows = (("timestep-forced, grouped pipeline", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0, 0),
-            ("timestep-forced, sequential", SCHED_SEQUENTIAL, CACHE_TIMESTEP, 4, 0, 0),
-            ("clean-cache refresh, sequential", SCHED_SEQUENTIAL, CACHE_CLEAN_REFRESH, 5, 0, 0),
-            ("timestep-forced, grouped pipeline, e4m3 projections", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 1, 0),
-            ("timestep-forced, grouped pipeline, e4m3 attention", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0, 1),
+    rows = (("timestep-forced, grouped pipeline", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0, 0, 0),
+            ("timestep-forced, sequential", SCHED_SEQUENTIAL, CACHE_TIMESTEP, 4, 0, 0, 0),
+            ("clean-cache refresh, sequential", SCHED_SEQUENTIAL, CACHE_CLEAN_REFRESH, 5, 0, 0, 0),
+            ("timestep-forced, grouped pipeline, e4m3 projections", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 1, 0, 0),
+            ("timestep-forced, grouped pipeline, e4m3 attention", SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0, 1, 0),
             ("timestep-forced, grouped pipeline, e4m3 projections and attention", SCHED_PIPELINED,
-             CACHE_TIMESTEP, 4, 1, 1),
+             CACHE_TIMESTEP, 4, 1, 1, 0),
             ("fixed-noise cache (prior blocks at the last step's noise), sequential", SCHED_SEQUENTIAL,
-             CACHE_FIXED_STEP, 4, 0, 0))
-    for idx, (name, sched, mode, nfe, fp8, afp8) in enumerate(rows):
+             CACHE_FIXED_STEP, 4, 0, 0, 0),
+            ("timestep-forced, grouped pipeline, full DiT block (AdaLN, GELU FFN 13824)", SCHED_PIPELINED,
+             CACHE_TIMESTEP, 4, 0, 0, DIT_FFN))
+    for idx, (name, sched, mode, nfe, fp8, afp8, ffn) in enumerate(rows):
         if only is not None and str(idx) not in only:
             continue
         cfg = STREAM.cfg.replace(schedule=sched, cache_mode=mode, proj_fp8=fp8, attn_fp8=afp8,
-                                 cache_step=STREAM.cfg.num_steps - 1)
+                                 cache_step=STREAM.cfg.num_steps - 1,
+                                 block_kind=BLOCK_DIT if ffn else BLOCK_ATTN, ffn_dim=ffn)
         T, C, D, F = cfg.block_tokens, cfg.latent_ch, cfg.hidden, cfg.frame_tokens
         S, nw, L = cfg.num_steps, cfg.window_blocks, cfg.num_layers
         g = torch.Generator(device="cuda")
@@ -464,6 +470,14 @@ def run_ablation(args):
         weights = dict(w_qkv=[rnd((3 * D, D), STREAM.w_std) for _ in range(L)],
                        w_out=[rnd((D, D), STREAM.w_std) for _ in range(L)],
                        w_in=rnd((D, C), 1.0 / C ** 0.5), w_head=rnd((C, D), STREAM.head_std))
+        if ffn:
+            # the DiT block: FFN weights and the AdaLN table (shifts, scales ~ N(0, 0.1^2), gates ~ N(1, 0.1^2))
+            weights["w_ffn1"] = [rnd((ffn, D), STREAM.w_std) for _ in range(L)]
+            weights["w_ffn2"] = [rnd((D, ffn), STREAM.w_std) for _ in range(L)]
+            ada = torch.randn((L, S + 1, 6, D), generator=g, device="cuda") * 0.1
+            ada[:, :, 2] += 1.0
+            ada[:, :, 5] += 1.0
+            weights["ada"] = ada.contiguous()
         s = LaStream(cfg, weights)
         s.set_sink(torch.randn((F, C), generator=g, device="cuda"))
         xs = [torch.randn((T, C), generator=g, device="cuda") for _ in range(2)]
@@ -481,12 +495,19 @@ def run_ablation(args):
         s.synchronize()
         torch.cuda.synchronize()
         ms = ev0.elapsed_time(ev1) / args.steps
-        kinds = {kd: round(s.profile_read(kd)[1] / args.steps, 3) for kd in ("qkv_gemm", "attn", "out_gemm", "other")}
+        kinds = {kd: round(s.profile_read(kd)[1] / args.steps, 3)
+                 for kd in ("qkv_gemm", "attn", "out_gemm", "other") + (("ffn",) if ffn else ())}
+        extra = {}
+        if ffn:
+            # per call (a tick, or a block's S steps): S passes x L layers x two GEMMs of 2 T D F flops
+            ffn_flops = 4.0 * T * D * ffn * L * S
+            extra["ffn_tflops"] = round(ffn_flops / (kinds["ffn"] / 1000.0) / 1e12, 1)
         s.profile(False)
         print(json.dumps({"ablation": name, "nfe_per_block": nfe, "ms_per_block": round(ms, 3),
                           "latent_frames_per_s": round(cfg.frames_per_block / (ms / 1000.0), 3),
-                          "ms_per_block_by_kind": kinds,
-                          "config": "8 sublayers, hidden 5120, 40x128 heads, 30x52 grid, window 2, "
+                          "ms_per_block_by_kind": kinds, **extra,
+                          "config": ("8 DiT blocks (AdaLN, GELU FFN %d)" % ffn if ffn else "8 sublayers")
+                                    + ", hidden 5120, 40x128 heads, 30x52 grid, window 2, "
                                     + ", ".join([x for x in ("e4m3 QKV/output projections" if fp8 else "",
                                                              "e4m3 attention" if afp8 else "") if x]
                                                 or ["bf16"])}),

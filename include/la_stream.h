@@ -138,7 +138,21 @@ typedef struct la_config {
   int32_t cache_step;          /* LA_CACHE_FIXED_STEP: the step (0 .. num_steps-1) whose
                                   K/V of the prior blocks every step reads; ignored by
                                   the other cache modes.                                */
+  int32_t block_kind;          /* LA_BLOCK_ATTN | LA_BLOCK_DIT                           */
+  int32_t ffn_dim;             /* LA_BLOCK_DIT: FFN hidden width F (multiple of 32)       */
 } la_config;
+
+/* Layer kinds.  The pages give the model's base (a 14B DiT with timestep
+ * conditioning; papernotes note, overall framework and FM loss) but no layer
+ * internals; LA_BLOCK_DIT is the Wan-style block the model is built on:
+ *   h += gate1 * Attn(n(h) * (1 + scale1) + shift1)
+ *   h += gate2 * (gelu_tanh(m W_ffn1^T) W_ffn2^T),  m = n(h) * (1 + scale2) + shift2
+ * with n the per-token RMS norm, Attn the attention sublayer (QKV, Rolling
+ * RoPE, cache, block-causal attention, output projection) and the AdaLN
+ * vectors of the layer at the step's timestep (la_weights.ada).  Needs
+ * proj_fp8 = attn_fp8 = 0.  The FFN runs on the same GEMM kernels. */
+#define LA_BLOCK_ATTN        0  /* each layer: the attention sublayer               */
+#define LA_BLOCK_DIT         1  /* each layer: the full DiT block                   */
 
 /*
  * Weights: DEVICE pointers, BORROWED (they must outlive the stream and must
@@ -152,6 +166,13 @@ typedef struct la_weights {
                                     rows 0..D-1 give q, D..2D-1 k, 2D..3D-1 v; head h
                                     owns rows h*d .. h*d+d-1 of each part        */
   const void* const* w_out;      /* HOST array of num_layers DEVICE pointers, each [D, D] */
+  /* LA_BLOCK_DIT only (ignored otherwise): */
+  const void* const* w_ffn1;     /* HOST array of num_layers DEVICE pointers, each [F, D] */
+  const void* const* w_ffn2;     /* HOST array of num_layers DEVICE pointers, each [D, F] */
+  const float* ada;              /* DEVICE fp32 [num_layers][num_steps + 1][6][D]: the AdaLN
+                                    vectors shift1, scale1, gate1, shift2, scale2, gate2 of
+                                    each layer at timesteps[0 .. num_steps-1], and at t = 0
+                                    (index num_steps: the sink pass and the clean refresh) */
 } la_weights;
 
 typedef struct la_stream la_stream;
@@ -254,6 +275,10 @@ int la_debug_capture(la_stream* s, int32_t enable);
  * (value = code * scale of its layer, part and head; Q not pre-scaled), and: */
 #define LA_TAP_SINK_V8   14 /* uint8 [H, F, d] e4m3 codes of the sink V of layer (slot ignored) */
 #define LA_TAP_ATTN_SCALES 15 /* fp32 [3, H] scales of q, K, V of layer (slot ignored)          */
+/* LA_BLOCK_DIT only: */
+#define LA_TAP_H_MID     16 /* fp32 [T_b, D] residual of layer after the attention sub-block   */
+#define LA_TAP_FFN_U     17 /* dtype [T_b, F] GELU output of layer's FFN (the second GEMM's
+                               operand)                                                       */
 
 /* Copy one tapped tensor into dst (DEVICE, dst_bytes >= the tensor's size),
  * ordered on the stream.  Taps other than ring / sink need capture enabled
@@ -275,7 +300,8 @@ int la_debug_set_slot_input(la_stream* s, int32_t slot, const float* x);
 #define LA_KIND_OUT_GEMM  4
 #define LA_KIND_HEAD      5
 #define LA_KIND_OTHER     6
-#define LA_NUM_KINDS      7
+#define LA_KIND_FFN       7  /* LA_BLOCK_DIT: the two FFN GEMMs                   */
+#define LA_NUM_KINDS      8
 int la_profile_enable(la_stream* s, int32_t enable);   /* resets the counters */
 int la_profile_read(la_stream* s, int32_t kind, int64_t* launches, double* total_ms);
 /* Kernels launched by this stream since creation. */

@@ -16,8 +16,8 @@ LA_MAX_STEPS, LA_MAX_WINDOW, LA_MAX_FPB = 8, 14, 7
 LA_EPI_STORE, LA_EPI_RESID, LA_EPI_SET32, LA_EPI_EULER, LA_EPI_STORE32 = 0, 1, 2, 3, 4
 
 TAP = dict(x_in=0, x_out=1, h=2, q=3, o=4, v=5, ring_k=6, ring_v=7, sink_k=8, sink_v=9, sink_k_rope=10, sink_h=11,
-           hop=12, sink_hop=13, sink_v8=14, attn_scales=15)
-KIND = dict(in_proj=0, qkv_gemm=1, rope=2, attn=3, out_gemm=4, head=5, other=6)
+           hop=12, sink_hop=13, sink_v8=14, attn_scales=15, h_mid=16, ffn_u=17)
+KIND = dict(in_proj=0, qkv_gemm=1, rope=2, attn=3, out_gemm=4, head=5, other=6, ffn=7)
 
 
 class LaConfig(ctypes.Structure):
@@ -28,13 +28,14 @@ class LaConfig(ctypes.Structure):
         ("timesteps", POINTER(c_float)), ("rope_split", c_int32 * 3), ("rope_theta", c_double),
         ("sink_mode", c_int32), ("rolling_rope", c_int32), ("sink_offset_frames", c_int32),
         ("schedule", c_int32), ("dtype", c_int32), ("cache_mode", c_int32), ("proj_fp8", c_int32),
-        ("attn_fp8", c_int32), ("cache_step", c_int32),
+        ("attn_fp8", c_int32), ("cache_step", c_int32), ("block_kind", c_int32), ("ffn_dim", c_int32),
     ]
 
 
 class LaWeights(ctypes.Structure):
     _fields_ = [("w_in", c_void_p), ("w_head", c_void_p), ("w_qkv", POINTER(c_void_p)),
-                ("w_out", POINTER(c_void_p))]
+                ("w_out", POINTER(c_void_p)), ("w_ffn1", POINTER(c_void_p)), ("w_ffn2", POINTER(c_void_p)),
+                ("ada", c_void_p)]
 
 
 class LaError(RuntimeError):

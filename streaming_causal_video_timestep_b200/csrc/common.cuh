@@ -75,7 +75,11 @@ struct AttnParams {
   int vrows[LA_MAX_SEG];
 };
 
-enum GemmEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SET32 = 2, EPI_EULER = 3, EPI_STORE32 = 4, EPI_QKV_ROPE = 5 };
+enum GemmEpi {
+  EPI_STORE = 0, EPI_RESID = 1, EPI_SET32 = 2, EPI_EULER = 3, EPI_STORE32 = 4, EPI_QKV_ROPE = 5,
+  EPI_RESID_GATED = 6,   // h32 += gate[row / rows_per_group][col] * acc; out (optional) = h32
+  EPI_GELU = 7           // out = gelu_tanh(acc)
+};
 
 // QKV projection epilogue: rotate q and k (Rolling 3D RoPE) on the fp32
 // accumulators, pre-multiply q by the softmax scale log2(e)/sqrt(d), and append
@@ -108,7 +112,13 @@ struct GemmEpiParams {
   float* vtap;          // optional fp32 [M, N] copy of acc (velocity capture)
   const float* row_scale;   // optional [M]: acc *= row_scale[row] * col_scale[col] first (FP8 operands)
   const float* col_scale;   // [N], set together with row_scale
+  const float* gate[LA_MAX_STEPS];   // RESID_GATED: per row group, [N]
 };
+
+// tanh-approximated GELU: u/2 (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))).
+__device__ __forceinline__ float gelu_tanh(float u) {
+  return 0.5f * u * (1.0f + tanhf(0.7978845608028654f * fmaf(0.044715f * u, u * u, u)));
+}
 
 
 static inline int ceil_div_i(long long a, long long b) { return (int)((a + b - 1) / b); }

@@ -316,6 +316,49 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const float* __restrict__ h, lo
   }
 }
 
+// AdaLN-modulated RMS normalisation: out = n(h) * (1 + scale_g) + shift_g, with
+// g = row / rows_per_group selecting the vectors of the row's buffer.
+__global__ void __launch_bounds__(256) k_rmsnorm_mod(const float* __restrict__ h, long long D, float eps,
+                                                     const __grid_constant__ ModArgs m,
+                                                     __nv_bfloat16* __restrict__ out_bf16, float* __restrict__ out_f32) {
+  const long long row = blockIdx.x;
+  const float4* h4 = reinterpret_cast<const float4*>(h + row * D);
+  const int n4 = static_cast<int>(D / 4);
+  const int g = static_cast<int>(row / m.rows_per_group);
+  const float4* sh4 = reinterpret_cast<const float4*>(m.shift[g]);
+  const float4* sc4 = reinterpret_cast<const float4*>(m.scale[g]);
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = h4[i];
+    ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+  }
+  __shared__ float red[8];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  const float scale = rsqrtf(red[0] / static_cast<float>(D) + eps);
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = h4[i], sh = sh4[i], sc = sc4[i];
+    const float4 o = make_float4(fmaf(v.x * scale, 1.f + sc.x, sh.x), fmaf(v.y * scale, 1.f + sc.y, sh.y),
+                                 fmaf(v.z * scale, 1.f + sc.z, sh.z), fmaf(v.w * scale, 1.f + sc.w, sh.w));
+    if (out_f32) reinterpret_cast<float4*>(out_f32 + row * D)[i] = o;
+    if (out_bf16) {
+      uint2 w;
+      w.x = pack_bf16x2(o.x, o.y);
+      w.y = pack_bf16x2(o.z, o.w);
+      reinterpret_cast<uint2*>(out_bf16 + row * D)[i] = w;
+    }
+  }
+}
+
 int grid_for(long long n, int per_block = 256) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -408,5 +451,15 @@ cudaError_t launch_rmsnorm(const float* h, long long rows, long long D, float ep
                            cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   k_rmsnorm<<<static_cast<unsigned>(rows), 256, 0, st>>>(h, D, eps, static_cast<__nv_bfloat16*>(out_bf16), out_f32);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm_mod(const float* h, long long rows, long long D, float eps, const ModArgs& m,
+                               void* out_bf16, float* out_f32, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (m.rows_per_group < 1 || (rows + m.rows_per_group - 1) / m.rows_per_group > LA_MAX_STEPS)
+    return cudaErrorInvalidValue;
+  k_rmsnorm_mod<<<static_cast<unsigned>(rows), 256, 0, st>>>(h, D, eps, m, static_cast<__nv_bfloat16*>(out_bf16),
+                                                             out_f32);
   return cudaGetLastError();
 }

@@ -101,3 +101,13 @@ cudaError_t launch_euler(float* x, const float* v, long long rows, long long C, 
 // as bf16 (out_bf16) and / or fp32 (out_f32).
 cudaError_t launch_rmsnorm(const float* h, long long rows, long long D, float eps, void* out_bf16, float* out_f32,
                            cudaStream_t st);
+
+// AdaLN vectors of each row group (buffer) for the modulated norm.
+struct ModArgs {
+  int rows_per_group;
+  const float* shift[LA_MAX_STEPS];   // [D] each
+  const float* scale[LA_MAX_STEPS];
+};
+// out = rms-normalised h * (1 + scale[row / rows_per_group]) + shift[...], bf16 and / or fp32.
+cudaError_t launch_rmsnorm_mod(const float* h, long long rows, long long D, float eps, const ModArgs& m,
+                               void* out_bf16, float* out_f32, cudaStream_t st);

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <new>
 #include <string>
 #include <vector>
@@ -159,6 +160,8 @@ struct la_stream {
   bool bf16 = true, id_in = true, id_head = true;
   bool fp8 = false;         // e4m3 QKV / output projections (bf16 streams)
   bool afp8 = false;        // e4m3 attention operands in the denoising passes (bf16 streams)
+  bool dit = false;         // LA_BLOCK_DIT: each layer a full DiT block
+  int Fffn = 0;             // its FFN width
   size_t eq = 2;            // element of q_rope / sk_rope / the rings (1 with afp8, else ea)
   size_t es = 2;            // activation / weight element (bf16 or fp32)
   size_t ea = 2;            // attention operand element (bf16 or fp32)
@@ -168,6 +171,11 @@ struct la_stream {
   const void* w_in = nullptr;
   const void* w_head = nullptr;
   std::vector<const void*> w_qkv, w_out;
+  std::vector<const void*> w_ffn1, w_ffn2;   // LA_BLOCK_DIT
+  const float* ada = nullptr;                // LA_BLOCK_DIT: [L][S+1][6][D]
+  void* ffn_u = nullptr;                     // LA_BLOCK_DIT: GELU output [max(nbuf*T, F)][Fffn], dtype
+  CUtensorMap tm_u{}, tm_s_u{};
+  std::vector<CUtensorMap> tm_w1, tm_w2;
 
   std::vector<void*> allocs;
   float* xs = nullptr;      // [nbuf][T][C]
@@ -235,6 +243,8 @@ struct la_stream {
   float* cap_sink_h = nullptr;  // fp32 [L][F][D] sink residual entering each layer
   void* cap_hop = nullptr;      // bf16 [S][L][T][D] normalised residual entering each QKV projection
   void* cap_sink_hop = nullptr; // bf16 [L][F][D] the same in the last sink pass
+  float* cap_hmid = nullptr;    // LA_BLOCK_DIT: fp32 [S][L][T][D] residual after the attention sub-block
+  void* cap_u = nullptr;        // LA_BLOCK_DIT: dtype [S][L][T][Fffn] GELU output
   bool cap_sink_valid = false;
   std::vector<int> cap_valid;  // per slot: captured in the last call
 
@@ -343,6 +353,11 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
   if (c->proj_fp8 != 0 && c->proj_fp8 != 1) { msg = "proj_fp8 must be 0 or 1"; return LA_EINVAL; }
   if (c->proj_fp8 && c->dtype != LA_BF16) { msg = "e4m3 projections need the bf16 stream"; return LA_EINVAL; }
   if (c->attn_fp8 != 0 && c->attn_fp8 != 1) { msg = "attn_fp8 must be 0 or 1"; return LA_EINVAL; }
+  if (c->block_kind != LA_BLOCK_ATTN && c->block_kind != LA_BLOCK_DIT) { msg = "bad block_kind"; return LA_EINVAL; }
+  if (c->block_kind == LA_BLOCK_DIT) {
+    if (c->ffn_dim < 32 || c->ffn_dim % 32 != 0 || c->ffn_dim > (1 << 20)) { msg = "ffn_dim must be a multiple of 32"; return LA_EINVAL; }
+    if (c->proj_fp8 || c->attn_fp8) { msg = "the DiT block runs without the e4m3 modes"; return LA_EINVAL; }
+  }
   if (c->attn_fp8 && (c->dtype != LA_BF16 || c->head_dim != 128)) {
     msg = "e4m3 attention needs the bf16 stream and head_dim 128";
     return LA_EINVAL;
@@ -358,6 +373,11 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
   if (!w->w_qkv || !w->w_out) { msg = "NULL layer weight arrays"; return LA_EINVAL; }
   for (int l = 0; l < c->num_layers; ++l)
     if (!w->w_qkv[l] || !w->w_out[l]) { msg = "NULL layer weight"; return LA_EINVAL; }
+  if (c->block_kind == LA_BLOCK_DIT) {
+    if (!w->w_ffn1 || !w->w_ffn2 || !w->ada) { msg = "the DiT block needs w_ffn1, w_ffn2 and ada"; return LA_EINVAL; }
+    for (int l = 0; l < c->num_layers; ++l)
+      if (!w->w_ffn1[l] || !w->w_ffn2[l]) { msg = "NULL FFN weight"; return LA_EINVAL; }
+  }
   if (c->dtype == LA_BF16) {
     if (c->hidden % 64 != 0) { msg = "bf16 path needs hidden % 64 == 0"; return LA_EINVAL; }
     if (w->w_in && (c->latent_ch % 32 != 0)) { msg = "bf16 path needs latent_ch % 32 == 0"; return LA_EINVAL; }
@@ -459,6 +479,54 @@ int normalise(la_stream* s, const float* h, long long rows, void* op_bf16, float
   });
 }
 
+// LA_BLOCK_DIT: AdaLN vector k (0 shift1, 1 scale1, 2 gate1, 3 shift2, 4 scale2,
+// 5 gate2) of layer l at timestep index t (num_steps: the t = 0 set).
+const float* ada_vec(const la_stream* s, int l, int t, int k) {
+  return s->ada + ((static_cast<long long>(l) * (s->S + 1) + t) * 6 + k) * s->D;
+}
+
+// The AdaLN-modulated norm of each row group g with the vectors (k_shift, k_shift+1)
+// of timestep index tidx[g].
+int normalise_mod(la_stream* s, const float* h, long long rows, int rows_per_group, const int* tidx, int ngroups,
+                  int l, int k_shift, void* op_bf16, float* op_f32) {
+  ModArgs m{};
+  m.rows_per_group = rows_per_group;
+  for (int g = 0; g < LA_MAX_STEPS; ++g) {
+    const int t = g < ngroups ? tidx[g] : 0;
+    m.shift[g] = ada_vec(s, l, t, k_shift);
+    m.scale[g] = ada_vec(s, l, t, k_shift + 1);
+  }
+  return launch(s, LA_KIND_OTHER, [&] {
+    return launch_rmsnorm_mod(h, rows, s->D, kRmsEps, m, s->bf16 ? op_bf16 : nullptr, op_f32, s->st);
+  });
+}
+
+// Turn a residual epilogue into the gated one with AdaLN vector k per row group.
+void set_gates(const la_stream* s, GemmEpiParams& e, int rows_per_group, const int* tidx, int ngroups, int l, int k) {
+  e.kind = EPI_RESID_GATED;
+  e.rows_per_group = rows_per_group;
+  for (int g = 0; g < LA_MAX_STEPS; ++g) e.gate[g] = ada_vec(s, l, g < ngroups ? tidx[g] : 0, k);
+}
+
+// The DiT block's FFN sub-block on h (rows of `rows_per_group` per group):
+// m = modulated norm (shift2, scale2) into the operand buffer, u = gelu(m W1^T),
+// h += gate2 * (u W2^T).  tm_op / op32 / tm_u describe the operand and u buffers.
+int ffn_block(la_stream* s, float* h, long long rows, int rows_per_group, const int* tidx, int ngroups, int l,
+              void* op_bf16, float* op32, const CUtensorMap* tm_op, const CUtensorMap* tm_u,
+              const std::function<void()>& after_gelu) {
+  const int D = s->D, F = s->Fffn;
+  int r;
+  if ((r = normalise_mod(s, h, rows, rows_per_group, tidx, ngroups, l, 3, op_bf16, s->bf16 ? nullptr : op32)) != LA_OK)
+    return r;
+  GemmEpiParams e1 = epi(EPI_GELU, s->ffn_u, nullptr, F);
+  if ((r = gemm(s, LA_KIND_FFN, tm_op, &s->tm_w1[l], op32, s->w_ffn1[l], e1, static_cast<int>(rows), F, D)) != LA_OK)
+    return r;
+  if (after_gelu) after_gelu();
+  GemmEpiParams e2 = epi(EPI_RESID, nullptr, h, D);
+  set_gates(s, e2, rows_per_group, tidx, ngroups, l, 5);
+  return gemm(s, LA_KIND_FFN, tm_u, &s->tm_w2[l], s->ffn_u, s->w_ffn2[l], e2, static_cast<int>(rows), D, F);
+}
+
 // One grouped pass over nbuf buffers (rows = nbuf*T) with the active ones in pd.
 int run_pass(la_stream* s, const PassDesc& pd) {
   const int T = s->T, D = s->D, C = s->C, H = s->H, d = s->d, F = s->F, S = s->S, E = s->E;
@@ -494,7 +562,10 @@ int run_pass(la_stream* s, const PassDesc& pd) {
     if ((r = gemm(s, LA_KIND_IN_PROJ, &s->tm_xop, &s->tm_win, s->xs, s->w_in, e, rows, D, C)) != LA_OK) return r;
   }
   if (s->capture && (r = capture_pass(s, pd, -1)) != LA_OK) return r;
-  if ((r = normalise(s, s->h32, rows, s->hop, s->bf16 ? nullptr : s->hn32)) != LA_OK) return r;
+  // timestep index of each buffer's AdaLN vectors (the DiT block)
+  int tidx[LA_MAX_STEPS] = {};
+  for (int b = 0; b < pd.nbuf; ++b) tidx[b] = pd.active[b] ? std::min(pd.step[b], S) : 0;
+  if (!s->dit && (r = normalise(s, s->h32, rows, s->hop, s->bf16 ? nullptr : s->hn32)) != LA_OK) return r;
 
   RopeArgs ra = rope_args(s);
   AttnParams ap{};
@@ -521,6 +592,9 @@ int run_pass(la_stream* s, const PassDesc& pd) {
   ap.q_prescaled = s->bf16 ? 1 : 0;
 
   for (int l = 0; l < s->L; ++l) {
+    if (s->dit &&
+        (r = normalise_mod(s, s->h32, rows, T, tidx, pd.nbuf, l, 0, s->hop, s->bf16 ? nullptr : s->hn32)) != LA_OK)
+      return r;
     if (s->capture && s->bf16) {
       // the normalised residual as the QKV projection consumes it (bf16)
       for (int ai = 0; ai < pd.nactive; ++ai) {
@@ -593,16 +667,40 @@ int run_pass(la_stream* s, const PassDesc& pd) {
     }
     // output projection + residual, then the next operand (next layer or head)
     GemmEpiParams eo = epi(EPI_RESID, nullptr, s->h32, D);
+    if (s->dit) set_gates(s, eo, T, tidx, pd.nbuf, l, 2);
     if (s->fp8) {
       if ((r = proj_fp8(s, LA_KIND_OUT_GEMM, s->attn_o, s->tm_a8, s->tm_wo8[l], s->wo8s[l], eo, rows, D, D)) != LA_OK)
         return r;
     } else if ((r = gemm(s, LA_KIND_OUT_GEMM, &s->tm_o, &s->tm_wout[l], s->attn_o, s->w_out[l], eo, rows, D, D)) !=
                LA_OK)
       return r;
+    if (s->dit) {
+      // the FFN sub-block (captures: the residual entering it, the GELU output)
+      int cerr = LA_OK;
+      auto cap = [&](bool gelu) {
+        for (int ai = 0; ai < pd.nactive && s->capture; ++ai) {
+          const int buf = pd.active_buf[ai];
+          if (pd.step[buf] >= S) continue;
+          const long long at = static_cast<long long>(pd.step[buf]) * s->L + l;
+          cudaError_t ce = gelu ? cudaMemcpyAsync(elem(s->cap_u, at * T * s->Fffn, s->es),
+                                                  elem(s->ffn_u, static_cast<long long>(buf) * T * s->Fffn, s->es),
+                                                  static_cast<size_t>(T) * s->Fffn * s->es, cudaMemcpyDeviceToDevice, s->st)
+                                : cudaMemcpyAsync(s->cap_hmid + at * T * D, s->h32 + static_cast<long long>(buf) * T * D,
+                                                  static_cast<size_t>(T) * D * 4, cudaMemcpyDeviceToDevice, s->st);
+          if (ce != cudaSuccess) cerr = fail(s, LA_ECUDA, cudaGetErrorString(ce));
+        }
+      };
+      cap(false);
+      if ((r = ffn_block(s, s->h32, rows, T, tidx, pd.nbuf, l, s->hop, s->hn32, &s->tm_hop, &s->tm_u,
+                         [&] { cap(true); })) != LA_OK)
+        return r;
+      if (cerr != LA_OK) return cerr;
+    }
     if (s->capture && (r = capture_pass(s, pd, l)) != LA_OK) return r;
     const bool last = l == s->L - 1;
     const bool want_f32 = !s->bf16 || (last && s->id_head);
-    if ((r = normalise(s, s->h32, rows, (s->bf16 && !(last && s->id_head)) ? s->hop : nullptr,
+    if ((!s->dit || last) &&
+        (r = normalise(s, s->h32, rows, (s->bf16 && !(last && s->id_head)) ? s->hop : nullptr,
                        want_f32 ? s->hn32 : nullptr)) != LA_OK)
       return r;
   }
@@ -683,7 +781,13 @@ int run_sink(la_stream* s) {
                          static_cast<size_t>(F) * D * 4, cudaMemcpyDeviceToDevice, s->st));
       s->cap_sink_valid = true;
     }
-    if ((r = normalise(s, s->s_h32, F, s->s_hop, s->bf16 ? nullptr : s->s_hn32)) != LA_OK) return r;
+    const int tS[1] = {s->S};   // the sink is a clean frame: the DiT block's t = 0 AdaLN set
+    if (s->dit) {
+      if ((r = normalise_mod(s, s->s_h32, F, F, tS, 1, l, 0, s->s_hop, s->bf16 ? nullptr : s->s_hn32)) != LA_OK)
+        return r;
+    } else if ((r = normalise(s, s->s_h32, F, s->s_hop, s->bf16 ? nullptr : s->s_hn32)) != LA_OK) {
+      return r;
+    }
     if (s->capture && s->bf16)
       CU(cudaMemcpyAsync(elem(s->cap_sink_hop, static_cast<long long>(l) * F * D, s->es), s->s_hop,
                          static_cast<size_t>(F) * D * s->es, cudaMemcpyDeviceToDevice, s->st));
@@ -718,6 +822,7 @@ int run_sink(la_stream* s) {
       if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) return r;
     }
     GemmEpiParams eo = epi(EPI_RESID, nullptr, s->s_h32, D);
+    if (s->dit) set_gates(s, eo, F, tS, 1, l, 2);
     if (s->fp8) {
       if ((r = proj_fp8(s, LA_KIND_OUT_GEMM, s->s_o, s->tm_s_a8, s->tm_wo8[l], s->wo8s[l], eo, F, D, D)) != LA_OK)
         return r;
@@ -725,6 +830,9 @@ int run_sink(la_stream* s) {
                LA_OK) {
       return r;
     }
+    if (s->dit && (r = ffn_block(s, s->s_h32, F, F, tS, 1, l, s->s_hop, s->s_hn32, &s->tm_s_hop, &s->tm_s_u,
+                                 nullptr)) != LA_OK)
+      return r;
   }
   return LA_OK;
 }
@@ -827,6 +935,10 @@ int alloc_capture(la_stream* s) {
     DALLOC(s->cap_hop, S * L * T * D * s->es);
     DALLOC(s->cap_sink_hop, L * F * D * s->es);
   }
+  if (s->dit) {
+    DALLOC(s->cap_hmid, S * L * T * D * 4);
+    DALLOC(s->cap_u, S * L * T * s->Fffn * static_cast<long long>(s->es));
+  }
   s->cap_valid.assign(s->S, 0);
   return LA_OK;
 }
@@ -882,6 +994,8 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   s->bf16 = cfg->dtype == LA_BF16; s->es = s->bf16 ? 2 : 4; s->ea = s->es;
   s->fp8 = s->bf16 && cfg->proj_fp8;
   s->afp8 = s->bf16 && cfg->attn_fp8;
+  s->dit = cfg->block_kind == LA_BLOCK_DIT;
+  s->Fffn = s->dit ? cfg->ffn_dim : 0;
   s->eq = s->afp8 ? 1 : s->ea;
   s->id_in = w->w_in == nullptr; s->id_head = w->w_head == nullptr;
   s->nbuf = cfg->schedule == LA_SCHED_PIPELINED ? s->S : 1;
@@ -889,6 +1003,11 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   s->w_in = w->w_in; s->w_head = w->w_head;
   s->w_qkv.assign(w->w_qkv, w->w_qkv + s->L);
   s->w_out.assign(w->w_out, w->w_out + s->L);
+  if (s->dit) {
+    s->w_ffn1.assign(w->w_ffn1, w->w_ffn1 + s->L);
+    s->w_ffn2.assign(w->w_ffn2, w->w_ffn2 + s->L);
+    s->ada = w->ada;
+  }
   s->sched.init(s->cfg);
 
   cudaError_t e = cudaGetDevice(&s->device);
@@ -910,7 +1029,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
                          NB * T * D * eq + NB * T * D * es + NB * H * F * d * eq + 2 * L * S * E * H * T * d * eq +
                          L * H * F * d * (4 + ea) + F * C * 4 + F * D * 4 + F * D * es * 2 + F * C * 2 +
                          F * 3 * D * 4 + 2 * H * F * d * ea + (s->afp8 ? L * H * F * d + L * 3 * H * 8 : 0) +
-                         (64 << 20);
+                         (s->dit ? std::max(NB * T, F) * s->Fffn * static_cast<long long>(es) : 0) + (64 << 20);
   size_t free_b = 0, total_b = 0;
   e = cudaMemGetInfo(&free_b, &total_b);
   if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
@@ -939,6 +1058,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   ALLOC_OR_BAIL(s->ring_v, L * S * E * H * T * d * eq);
   ALLOC_OR_BAIL(s->sink_k, L * H * F * d * 4);
   ALLOC_OR_BAIL(s->sink_v, L * H * F * d * ea);
+  if (s->dit) ALLOC_OR_BAIL(s->ffn_u, std::max(NB * T, F) * s->Fffn * static_cast<long long>(es));
   if (s->afp8) {
     ALLOC_OR_BAIL(s->sink_v8, L * H * F * d);
     ALLOC_OR_BAIL(s->attn_sc, L * 3 * H * 4);
@@ -1001,6 +1121,17 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
     for (int l = 0; l < L && ok; ++l) {
       ok = ok && tmap_2d_bf16(&s->tm_wqkv[l], s->w_qkv[l], 3 * D, D, D, bn_qkv, s->err);
       ok = ok && tmap_2d_bf16(&s->tm_wout[l], s->w_out[l], D, D, D, bn_d, s->err);
+    }
+    if (s->dit) {
+      const long long Ff = s->Fffn;
+      ok = ok && tmap_2d_bf16(&s->tm_u, s->ffn_u, NB * T, Ff, Ff, 128, s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_s_u, s->ffn_u, F, Ff, Ff, 128, s->err);
+      s->tm_w1.resize(L);
+      s->tm_w2.resize(L);
+      for (int l = 0; l < L && ok; ++l) {
+        ok = ok && tmap_2d_bf16(&s->tm_w1[l], s->w_ffn1[l], Ff, D, D, gemm_tc_pick_bn(s->Fffn), s->err);
+        ok = ok && tmap_2d_bf16(&s->tm_w2[l], s->w_ffn2[l], D, Ff, Ff, bn_d, s->err);
+      }
     }
     if (!s->id_in) {
       ok = ok && tmap_2d_bf16(&s->tm_xop, s->xop, NB * T, C, C, 128, s->err);
@@ -1130,12 +1261,16 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
   const bool per_layer = what == LA_TAP_H || what == LA_TAP_Q || what == LA_TAP_O || what == LA_TAP_RING_K ||
                          what == LA_TAP_RING_V || what == LA_TAP_SINK_K || what == LA_TAP_SINK_V ||
                          what == LA_TAP_SINK_KROPE || what == LA_TAP_SINK_H || what == LA_TAP_HOP ||
-                         what == LA_TAP_SINK_HOP || what == LA_TAP_SINK_V8 || what == LA_TAP_ATTN_SCALES;
+                         what == LA_TAP_SINK_HOP || what == LA_TAP_SINK_V8 || what == LA_TAP_ATTN_SCALES ||
+                         what == LA_TAP_H_MID || what == LA_TAP_FFN_U;
   if (per_layer && (layer < (what == LA_TAP_H ? -1 : 0) || layer >= L)) return fail(s, LA_EINVAL, "bad layer");
   if (slot < 0 || slot >= S) return fail(s, LA_EINVAL, "bad slot");
   const void* src = nullptr;
   long long bytes = 0;
-  const bool needs_capture = what <= LA_TAP_V || what == LA_TAP_SINK_KROPE || what == LA_TAP_HOP;
+  const bool needs_capture = what <= LA_TAP_V || what == LA_TAP_SINK_KROPE || what == LA_TAP_HOP ||
+                             what == LA_TAP_H_MID || what == LA_TAP_FFN_U;
+  if ((what == LA_TAP_H_MID || what == LA_TAP_FFN_U) && !s->dit)
+    return fail(s, LA_EINVAL, "the FFN taps exist with the DiT block only");
   if ((what == LA_TAP_HOP || what == LA_TAP_SINK_HOP) && !s->bf16)
     return fail(s, LA_EINVAL, "the GEMM-operand taps exist in bf16 streams only");
   if ((what == LA_TAP_SINK_V8 || what == LA_TAP_ATTN_SCALES) && !s->afp8)
@@ -1159,6 +1294,11 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
     case LA_TAP_SINK_K: src = s->sink_k + static_cast<long long>(layer) * H * F * d; bytes = H * F * d * 4; break;
     case LA_TAP_SINK_V: src = elem(s->sink_v, static_cast<long long>(layer) * H * F * d, ea); bytes = H * F * d * ea; break;
     case LA_TAP_SINK_V8: src = s->sink_v8 + static_cast<long long>(layer) * H * F * d; bytes = H * F * d; break;
+    case LA_TAP_H_MID: src = s->cap_hmid + (slot * L + layer) * T * D; bytes = T * D * 4; break;
+    case LA_TAP_FFN_U:
+      src = elem(s->cap_u, (slot * L + layer) * T * s->Fffn, s->es);
+      bytes = T * s->Fffn * static_cast<long long>(s->es);
+      break;
     case LA_TAP_ATTN_SCALES: src = s->attn_sc + static_cast<long long>(layer) * 3 * H; bytes = 3 * H * 4; break;
     case LA_TAP_SINK_H:
       if (!s->cap_sink_valid) return fail(s, LA_ESTATE, "no capture of a sink pass");

@@ -23,6 +23,13 @@ __device__ __forceinline__ void epi_scalar(const GemmEpiParams& ep, long long ro
       ep.h32[off] = acc;
       if (out && out != ep.h32) out[off] = acc;
       break;
+    case EPI_RESID_GATED: {
+      const float h = fmaf(ep.gate[row / ep.rows_per_group][col], acc, ep.h32[off]);
+      ep.h32[off] = h;
+      if (out && out != ep.h32) out[off] = h;
+      break;
+    }
+    case EPI_GELU: out[off] = gelu_tanh(acc); break;
     case EPI_EULER: {
       const int g = static_cast<int>(row / ep.rows_per_group);
       if (!ep.active[g]) break;

@@ -74,6 +74,8 @@ class LaStream:
         c.proj_fp8 = getattr(cfg, "proj_fp8", 0)
         c.attn_fp8 = getattr(cfg, "attn_fp8", 0)
         c.cache_step = getattr(cfg, "cache_step", 0)
+        c.block_kind = getattr(cfg, "block_kind", 0)
+        c.ffn_dim = getattr(cfg, "ffn_dim", 0)
         self.cfg = cfg
         self.c = c
         self.T = cfg.frames_per_block * cfg.grid_h * cfg.grid_w
@@ -90,6 +92,15 @@ class LaStream:
         w.w_head = None if weights.get("w_head") is None else weights["w_head"].data_ptr()
         w.w_qkv = ctypes.cast(self._wq, ctypes.POINTER(c_void_p))
         w.w_out = ctypes.cast(self._wo, ctypes.POINTER(c_void_p))
+        if weights.get("w_ffn1") is not None:
+            # the full DiT block: FFN weights per layer and the AdaLN table (fp32 [L][S+1][6][D])
+            self._w1 = (c_void_p * L)(*[t.data_ptr() for t in weights["w_ffn1"]])
+            self._w2 = (c_void_p * L)(*[t.data_ptr() for t in weights["w_ffn2"]])
+            S1 = len(cfg.timesteps)          # num_steps + 1 AdaLN sets
+            _require(weights["ada"], torch.float32, (L, S1, 6, cfg.hidden), "ada")
+            w.w_ffn1 = ctypes.cast(self._w1, ctypes.POINTER(c_void_p))
+            w.w_ffn2 = ctypes.cast(self._w2, ctypes.POINTER(c_void_p))
+            w.ada = weights["ada"].data_ptr()
         self.w = w
         h = c_void_p()
         code = self.lib.la_stream_create(ctypes.byref(c), ctypes.byref(w), _stream_handle(self.stream), ctypes.byref(h))
@@ -158,6 +169,7 @@ class LaStream:
             "sink_v": ((H, F, d), dt), "sink_k_rope": ((H, F, d), dt), "sink_h": ((F, D), torch.float32),
             "hop": ((T, D), dt), "sink_hop": ((F, D), dt),
             "sink_v8": ((H, F, d), torch.uint8), "attn_scales": ((3, H), torch.float32),
+            "h_mid": ((T, D), torch.float32), "ffn_u": ((T, max(1, getattr(self.cfg, "ffn_dim", 0))), dt),
         }
         shape, tdt = shapes[what]
         if what in ("q", "ring_k", "ring_v", "sink_k_rope") and getattr(self.cfg, "attn_fp8", 0):

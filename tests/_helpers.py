@@ -33,8 +33,13 @@ def torch_weights(W, cfg, device="cuda"):
     import torch
     dt = torch.bfloat16 if cfg.dtype == DTYPE_BF16 else torch.float32
     conv = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device=device, dtype=dt)
-    return dict(w_qkv=[conv(w) for w in W.w_qkv], w_out=[conv(w) for w in W.w_out],
-                w_in=conv(W.w_in), w_head=conv(W.w_head))
+    out = dict(w_qkv=[conv(w) for w in W.w_qkv], w_out=[conv(w) for w in W.w_out],
+               w_in=conv(W.w_in), w_head=conv(W.w_head))
+    if getattr(W, "w_ffn1", None) is not None:
+        out["w_ffn1"] = [conv(w) for w in W.w_ffn1]
+        out["w_ffn2"] = [conv(w) for w in W.w_ffn2]
+        out["ada"] = torch.from_numpy(np.ascontiguousarray(W.ada, np.float32)).to(device)
+    return out
 
 
 def make_stream(wl: Workload, W=None, cfg=None, capture=False):

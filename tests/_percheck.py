@@ -15,6 +15,7 @@ import numpy as np
 import math
 
 from oracle import block_causal_attention, euler_step, rms_norm, rope_rotate
+from oracle.dit import gelu_tanh, modulate
 from oracle.fp8 import (attention_fp8, attn_fp8_scales, dequantize_weight, project, quantize_heads,
                         quantize_rows)
 from oracle.rope import block_positions, sink_positions
@@ -32,6 +33,18 @@ def _operand(a, cfg):
 def _normed_operand(h, cfg):
     """The per-token RMS-normalised residual as the next GEMM consumes it."""
     return _operand(rms_norm(np.asarray(h, np.float64)).astype(np.float32), cfg)
+
+
+def _dit(cfg):
+    return getattr(cfg, "block_kind", 0) == 1
+
+
+def _attn_operand(h, cfg, W, l, t_idx):
+    """The QKV projection's operand: the normalised residual, AdaLN-modulated in the DiT block."""
+    if not _dit(cfg):
+        return _normed_operand(h, cfg)
+    a = np.asarray(W.ada, np.float64)[l, t_idx]
+    return _operand(modulate(np.asarray(h, np.float64), a[0], a[1]).astype(np.float32), cfg)
 
 
 _W8 = {}
@@ -112,7 +125,7 @@ def check_sink(s, cfg, W, latent, rows=None, tag=""):
     assert_close(h0[R], want, dt, f"{tag} sink in-proj")
     for l in range(cfg.num_layers):
         hs = to_np(s.tap("sink_h", l))
-        op = _normed_operand(hs[R], cfg)
+        op = _attn_operand(hs[R], cfg, W, l, cfg.num_steps)
         if getattr(cfg, "proj_fp8", 0) or getattr(cfg, "attn_fp8", 0):
             # e4m3 operands downstream: the normalisation on its own, then the projection
             # from the operand the GPU consumed (a one-ulp difference there can move
@@ -163,7 +176,7 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
     chk(h_in[R], want, "in-proj h")
     h_prev = h_in
     for l in range(L):
-        op = _normed_operand(h_prev[R], cfg)
+        op = _attn_operand(h_prev[R], cfg, W, l, i)
         if getattr(cfg, "proj_fp8", 0) or getattr(cfg, "attn_fp8", 0):
             # e4m3 operands downstream: check the normalisation on its own, then go on
             # from the operand the GPU consumed (a one-ulp bf16 difference there moves
@@ -213,6 +226,10 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
         chk(o_gpu[R], o_want.reshape(len(R), D), f"attn O l{l}")
         # output projection + residual from the attention output as the GEMM consumes it
         h_next = to_np(s.tap("h", l, i))
+        if _dit(cfg):
+            _check_ffn(s, cfg, W, l, i, R, h_prev, o_gpu, h_next, chk)
+            h_prev = h_next
+            continue
         want = h_prev[R].astype(np.float64) + _proj(_operand(o_gpu[R], cfg), W.w_out[l], cfg)
         chk(h_next[R], want, f"h l{l}")
         h_prev = h_next
@@ -254,3 +271,18 @@ def _check_attn_fp8(s, cfg, W, b, i, l, R, qr, kr, v, sink, st, chk, errs, tag):
     chk(to_np(s.tap("o", l, i))[R], o_want.reshape(len(R), D), f"attn O (e4m3) l{l}")
     for k_, f_ in fr.items():
         errs[k_] = max(errs.get(k_, (0, 0)), (f_, 0.0))
+
+
+def _check_ffn(s, cfg, W, l, i, R, h_prev, o_gpu, h_next, chk):
+    """The DiT block after attention: the gated output projection (h_mid), the
+    AdaLN-modulated FFN operand and its GELU output (u), and the gated FFN residual,
+    each from the GPU's own inputs."""
+    a = np.asarray(W.ada, np.float64)[l, i]
+    h_mid = to_np(s.tap("h_mid", l, i))
+    want = h_prev[R].astype(np.float64) + a[2] * _proj(_operand(o_gpu[R], cfg), W.w_out[l], cfg)
+    chk(h_mid[R], want, f"h mid l{l}")
+    m2 = _operand(modulate(h_mid[R].astype(np.float64), a[3], a[4]).astype(np.float32), cfg)
+    u_gpu = to_np(s.tap("ffn_u", l, i))
+    chk(u_gpu[R], gelu_tanh(m2 @ np.asarray(W.w_ffn1[l], np.float64).T), f"ffn gelu l{l}")
+    want = h_mid[R].astype(np.float64) + a[5] * (_operand(u_gpu[R], cfg) @ np.asarray(W.w_ffn2[l], np.float64).T)
+    chk(h_next[R], want, f"h l{l}")

@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 from oracle import OracleStream, TickScheduler
-from workloads import (CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, DTYPE_BF16, DTYPE_FP32, SCHED_PIPELINED,
+from workloads import (BLOCK_DIT, CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, DTYPE_BF16, DTYPE_FP32, SCHED_PIPELINED,
                        SCHED_SEQUENTIAL, SINK_AAS, SINK_FIXED, TINY, StreamConfig, Workload, block_noise, make_weights)
 
 from _helpers import assert_close, errors, make_stream, to_np
@@ -257,6 +257,50 @@ def test_small_bf16_fixed_noise_cache_teacher_forced():
     report = _run_teacher_forced(Workload("small-bf16-fixed", cfg, SMALL_BF16.seed, 5, SMALL_BF16.w_std,
                                           SMALL_BF16.head_std))
     print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in report.items()})
+
+
+TINY_DIT = Workload("tiny-dit", TINY.cfg.replace(block_kind=BLOCK_DIT, ffn_dim=160), TINY.seed, TINY.num_blocks,
+                    TINY.w_std, TINY.head_std)
+SMALL_DIT = Workload("small-bf16-dit", SMALL_BF16.cfg.replace(block_kind=BLOCK_DIT, ffn_dim=640), SMALL_BF16.seed, 6,
+                     SMALL_BF16.w_std, SMALL_BF16.head_std)
+
+
+def test_tiny_fp32_dit_stream_every_tick_matches_oracle():
+    """The full DiT block (AdaLN, gated residuals, GELU FFN): every op of every tick
+    teacher-forced, and the finished blocks within 1e-5."""
+    _run_teacher_forced(TINY_DIT)
+
+
+def test_tiny_fp32_dit_stream_free_running_and_sequential():
+    """Free-running fp32 DiT stream within 1e-5 of the oracle, grouped pipeline and
+    sequential schedule (the sequential run also checks the integer state every call)."""
+    cfg = TINY_DIT.cfg.replace(schedule=SCHED_SEQUENTIAL)
+    _run_clean_refresh(Workload("tiny-dit-seq", cfg, TINY.seed, 5, TINY.w_std, TINY.head_std))
+    wl = TINY_DIT
+    s, W = make_stream(wl)
+    orc = OracleStream(wl.cfg, W)
+    orc.set_sink(W.sink)
+    x_out = torch.empty((wl.cfg.block_tokens, wl.cfg.latent_ch), dtype=torch.float32, device="cuda")
+    for k in range(wl.num_blocks + 3):
+        xn = block_noise(wl, k) if k < wl.num_blocks else None
+        fin = s.step(_dev(xn) if xn is not None else None, x_out)
+        out, fin_o = orc.denoise_step(xn)
+        assert fin == fin_o
+        if fin >= 0:
+            assert_close(to_np(x_out), out, DTYPE_FP32, f"dit block {fin}")
+    s.close()
+
+
+def test_small_bf16_dit_stream_teacher_forced():
+    report = _run_teacher_forced(SMALL_DIT)
+    print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in report.items()})
+
+
+def test_dit_block_rejects_the_e4m3_modes():
+    from streaming_causal_video_timestep_b200 import LaError
+    with pytest.raises(LaError):
+        make_stream(Workload("dit-fp8", SMALL_DIT.cfg.replace(proj_fp8=1), SMALL_DIT.seed, 2, SMALL_DIT.w_std,
+                             SMALL_DIT.head_std))
 
 
 def test_small_bf16_stream_with_e4m3_projections_teacher_forced():
