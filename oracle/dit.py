@@ -17,6 +17,13 @@ the timestep embedding and its projection are fixed for the 4 distilled
 timesteps, so the library takes the vectors themselves as weights, one set per
 (layer, timestep) plus one for t = 0 (the clean sink frame and the clean-cache
 refresh).
+
+Audio cross-attention (the model is audio-driven; papernotes note, 整体框架;
+reading: Wan's cross-attention sub-block, between the attention and the FFN):
+    h = h + (softmax(q k^T / sqrt(d)) v) W_oc^T,  q = n(h) W_qc^T,
+    [k | v] = audio_b W_kvc^T
+over all audio tokens of the block (no RoPE, no mask; heads as in the
+self-attention).  The sink frame has no audio: its pass skips the sub-block.
 """
 from __future__ import annotations
 
@@ -41,3 +48,18 @@ def modulate(h, shift, scale):
 def ffn(m, w1, w2):
     """gelu(m W1^T) W2^T; w1 [F, D], w2 [D, F]."""
     return gelu_tanh(np.asarray(m, np.float64) @ np.asarray(w1, np.float64).T) @ np.asarray(w2, np.float64).T
+
+
+def cross_attention(h, audio, w_qc, w_kvc, w_oc, heads, head_dim):
+    """The audio cross-attention sub-block's contribution (to be added to h):
+    softmax(q k^T / sqrt(d)) v W_oc^T with q = n(h) W_qc^T and [k | v] = audio W_kvc^T."""
+    from .attention import block_causal_attention
+    h = np.asarray(h, np.float64)
+    T, D = h.shape
+    q = (rms_norm(h) @ np.asarray(w_qc, np.float64).T).reshape(T, heads, head_dim)
+    kv = np.asarray(audio, np.float64) @ np.asarray(w_kvc, np.float64).T
+    A = kv.shape[0]
+    k = kv[:, :D].reshape(A, heads, head_dim)
+    v = kv[:, D:].reshape(A, heads, head_dim)
+    o = block_causal_attention(q, {0: (k, v)}, None, qblock=0, window=0)
+    return o.reshape(T, D) @ np.asarray(w_oc, np.float64).T

@@ -59,7 +59,7 @@ from __future__ import annotations
 import numpy as np
 
 from .attention import block_causal_attention
-from .dit import ffn, modulate
+from .dit import cross_attention, ffn, modulate
 from .flow import euler_step
 from .fp8 import attention_fp8, attn_fp8_scales, dequantize_weight, project, quantize_heads, quantize_rows
 from .norm import rms_norm
@@ -92,6 +92,12 @@ class OracleStream:
             self.w1 = [f64(w) for w in weights.w_ffn1]
             self.w2 = [f64(w) for w in weights.w_ffn2]
             self.ada = np.asarray(weights.ada, np.float64)
+        self.cross = self.dit and getattr(cfg, "audio_tokens", 0) > 0
+        if self.cross:
+            self.w_qc = [f64(w) for w in weights.w_qc]
+            self.w_kvc = [f64(w) for w in weights.w_kvc]
+            self.w_oc = [f64(w) for w in weights.w_oc]
+        self.audio = {}            # block -> its audio features (cross-attention)
         self.sched = TickScheduler(cfg)
         self.cache = {}            # (layer, ring, block) -> (k_roped, v, (block, step))
         self.sink_k = None         # per layer, un-roped [F, H, d]
@@ -125,12 +131,16 @@ class OracleStream:
         a = self.ada[l, t_idx]
         return modulate(h, a[0], a[1])
 
-    def _attn_residual(self, l, h, proj, t_idx):
-        """h + the attention sublayer's output (gated in the DiT block), then the DiT's FFN sub-block."""
+    def _attn_residual(self, l, h, proj, t_idx, audio=None):
+        """h + the attention sublayer's output (gated in the DiT block), then the DiT's
+        audio cross-attention (when the block has audio) and FFN sub-blocks."""
         if not self.dit:
             return h + proj
         a = self.ada[l, t_idx]
         h = h + a[2] * proj
+        if audio is not None:
+            c = self.cfg
+            h = h + cross_attention(h, audio, self.w_qc[l], self.w_kvc[l], self.w_oc[l], c.heads, c.head_dim)
         return h + a[5] * ffn(modulate(h, a[3], a[4]), self.w1[l], self.w2[l])
 
     def project_in(self, x):
@@ -208,7 +218,8 @@ class OracleStream:
             else:
                 o = block_causal_attention(qr, blocks, (sk, self.sink_v[l]), qblock=b,
                                            window=c.window_blocks)
-            h = self._attn_residual(l, h, self._proj_out(l, o.reshape(h.shape[0], -1)), t_idx)
+            h = self._attn_residual(l, h, self._proj_out(l, o.reshape(h.shape[0], -1)), t_idx,
+                                    self.audio.get(b) if self.cross else None)
             if tr is not None:
                 tr[("layer", l)] = dict(q=qr, k=kr, v=v.copy(), sink_k=sk, o=o, h=h.copy())
         if refresh:
@@ -224,17 +235,22 @@ class OracleStream:
         return x_next
 
     # -- one call of the C-ABI's la_denoise_step ---------------------------------
-    def denoise_step(self, x_new=None, inputs=None, aas_latent=None):
-        """x_new: noise of the next block (or None to drain).  inputs: optional
+    def denoise_step(self, x_new=None, inputs=None, aas_latent=None, audio=None):
+        """x_new: noise of the next block (or None to drain); audio: its audio
+        features (the DiT block's cross-attention).  inputs: optional
         {(block, step): latent} overriding the latent a step starts from, and
         aas_latent: optional finished latent of block 0 to take the new sink
         from (teacher forcing).  Returns (finished latent or None, finished id)."""
         if self.sink_k is None:
             raise RuntimeError("set_sink first")
         has_new = x_new is not None
+        if self.cross and has_new and audio is None:
+            raise ValueError("this stream needs the audio of every new block")
         run, finished = self.sched.begin_tick(has_new)
         if has_new:
             self.latents[self.sched.blocks_in - 1] = np.asarray(x_new, np.float64)
+            if self.cross:
+                self.audio[self.sched.blocks_in - 1] = np.asarray(audio, np.float64)
         for i, b in run:
             x = self.latents[b]
             if inputs is not None and (b, i) in inputs:
@@ -245,6 +261,7 @@ class OracleStream:
             out = self.latents.pop(finished)
             if self.sched.clean:
                 self.slot_pass(out, finished, self.cfg.num_steps, refresh=True)
+            self.audio.pop(finished, None)
         if self.sched.end_tick(finished):
             src = out if aas_latent is None else np.asarray(aas_latent, np.float64)
             self.set_sink(src[: self.cfg.sink_tokens])

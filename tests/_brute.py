@@ -61,6 +61,12 @@ class BruteStream:
             self.w1 = [tolist(w) for w in W.w_ffn1]
             self.w2 = [tolist(w) for w in W.w_ffn2]
             self.ada = [[[[float(v) for v in vec] for vec in st] for st in lay] for lay in W.ada]
+        self.cross = self.dit and getattr(cfg, "audio_tokens", 0) > 0
+        if self.cross:
+            self.wqc = [tolist(w) for w in W.w_qc]
+            self.wkvc = [tolist(w) for w in W.w_kvc]
+            self.woc = [tolist(w) for w in W.w_oc]
+        self.audio = {}
 
     # -- the DiT block's pieces, scalar ------------------------------------------------------------
     def _operand(self, h, l, t_idx):
@@ -71,12 +77,27 @@ class BruteStream:
         sh, sc = self.ada[l][t_idx][0], self.ada[l][t_idx][1]
         return [[v * (1.0 + sc[j]) + sh[j] for j, v in enumerate(row)] for row in n]
 
-    def _residual(self, h, proj, l, t_idx):
-        """h + attention output; in the DiT block gated, then + gated tanh-GELU FFN."""
+    def _cross(self, h, l, audio):
+        """The audio cross-attention sub-block's contribution, scalar."""
+        c = self.c
+        D = c.hidden
+        q = matvec_rows(normalize_rows(h), self.wqc[l])
+        kv = matvec_rows([list(map(float, r)) for r in audio], self.wkvc[l])
+        qh = [[row[hh * c.head_dim:(hh + 1) * c.head_dim] for hh in range(c.heads)] for row in q]
+        keys = [([row[hh * c.head_dim:(hh + 1) * c.head_dim] for hh in range(c.heads)],
+                 [row[D + hh * c.head_dim:D + (hh + 1) * c.head_dim] for hh in range(c.heads)]) for row in kv]
+        return matvec_rows(self._layer_attend(qh, keys), self.woc[l])
+
+    def _residual(self, h, proj, l, t_idx, audio=None):
+        """h + attention output; in the DiT block gated, then + the audio cross-attention
+        (when the block has audio), then + gated tanh-GELU FFN."""
         if not self.dit:
             return [[a + b for a, b in zip(hr, pr)] for hr, pr in zip(h, proj)]
         a = self.ada[l][t_idx]
         h = [[x + a[2][j] * p for j, (x, p) in enumerate(zip(hr, pr))] for hr, pr in zip(h, proj)]
+        if audio is not None:
+            cr = self._cross(h, l, audio)
+            h = [[x + y for x, y in zip(hr, cr_)] for hr, cr_ in zip(h, cr)]
         n = normalize_rows(h)
         m = [[v * (1.0 + a[4][j]) + a[3][j] for j, v in enumerate(row)] for row in n]
         u = matvec_rows(m, self.w1[l])
@@ -163,7 +184,7 @@ class BruteStream:
                     visible.append((kr, vh))
             o = self._layer_attend(qrot, visible)
             proj = matvec_rows(o, self.wout[l])
-            h = self._residual(h, proj, l, i)
+            h = self._residual(h, proj, l, i, self.audio.get(b) if self.cross else None)
         hn = normalize_rows(h)
         v = hn if self.whead is None else matvec_rows(hn, self.whead)
         dt = c.timesteps[i + 1] - c.timesteps[i]
@@ -184,9 +205,11 @@ class BruteStream:
                 self.set_sink(x[: c.sink_tokens])
         return done
 
-    def run_pipelined(self, noises):
+    def run_pipelined(self, noises, audios=None):
         """Tick k: slot i runs block k - i.  Returns {block: final latent}."""
         c = self.c
+        if audios is not None:
+            self.audio = dict(enumerate(audios))
         S = c.num_steps
         nb = len(noises)
         done = {}

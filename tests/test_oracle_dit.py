@@ -105,3 +105,62 @@ def test_dit_with_closed_gates_leaves_the_residual_unchanged():
     got = s.slot_pass(x, 0, 0)
     t = cfg.timesteps
     np.testing.assert_allclose(got, x + (t[1] - t[0]) * rms_norm(x), rtol=1e-13, atol=1e-13)
+
+
+# -- the audio cross-attention sub-block --------------------------------------------------------
+def test_cross_attention_single_audio_token_is_its_value_projected():
+    """One audio token: every softmax weight is 1, so the sub-block adds v W_oc^T to every row."""
+    from oracle.dit import cross_attention
+    rng = np.random.default_rng(31)
+    D, H, d, Da = 16, 2, 8, 6
+    h = rng.standard_normal((5, D))
+    audio = rng.standard_normal((1, Da))
+    wqc, wkvc, woc = rng.standard_normal((D, D)), rng.standard_normal((2 * D, Da)), rng.standard_normal((D, D))
+    v = (audio @ wkvc.T)[0, D:]
+    got = cross_attention(h, audio, wqc, wkvc, woc, H, d)
+    np.testing.assert_allclose(got, np.broadcast_to(v @ woc.T, (5, D)), rtol=1e-12, atol=1e-12)
+
+
+def test_cross_attention_matches_torch_sdpa():
+    from oracle.dit import cross_attention
+    rng = np.random.default_rng(32)
+    D, H, d, Da, T, A = 32, 4, 8, 12, 9, 7
+    h = rng.standard_normal((T, D))
+    audio = rng.standard_normal((A, Da))
+    wqc, wkvc, woc = rng.standard_normal((D, D)), rng.standard_normal((2 * D, Da)), rng.standard_normal((D, D))
+    q = (rms_norm(h) @ wqc.T).reshape(T, H, d).transpose(1, 0, 2)
+    kv = audio @ wkvc.T
+    k = kv[:, :D].reshape(A, H, d).transpose(1, 0, 2)
+    v = kv[:, D:].reshape(A, H, d).transpose(1, 0, 2)
+    o = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q), torch.from_numpy(k),
+                                                         torch.from_numpy(v)).numpy()
+    want = o.transpose(1, 0, 2).reshape(T, D) @ woc.T
+    np.testing.assert_allclose(cross_attention(h, audio, wqc, wkvc, woc, H, d), want, rtol=1e-11, atol=1e-11)
+
+
+def test_dit_stream_with_audio_matches_the_scalar_brute_force():
+    from workloads import block_audio
+    cfg = _cfg(audio_tokens=5, audio_dim=8)
+    wl = Workload("brute-dit-audio", cfg, 24, 4, 0.25)
+    W = make_weights(wl)
+    from _brute import BruteStream
+    bs = BruteStream(cfg, W)
+    bs.set_sink(W.sink)
+    noises = [block_noise(wl, b) for b in range(wl.num_blocks)]
+    audios = [block_audio(wl, b) for b in range(wl.num_blocks)]
+    want = bs.run_pipelined(noises, audios)
+    s = OracleStream(cfg, W)
+    s.set_sink(W.sink)
+    got = {}
+    for k in range(wl.num_blocks + cfg.num_steps - 1):
+        nb = k < wl.num_blocks
+        out, fin = s.denoise_step(noises[k] if nb else None, audio=audios[k] if nb else None)
+        if fin >= 0:
+            got[fin] = out
+    for b in range(wl.num_blocks):
+        np.testing.assert_allclose(got[b], np.array(want[b]), rtol=1e-10, atol=1e-10)
+    # the audio matters
+    s2 = OracleStream(cfg.replace(audio_tokens=0), W)
+    s2.set_sink(W.sink)
+    out0 = [s2.denoise_step(noises[k] if k < 4 else None)[0] for k in range(4 + cfg.num_steps - 1)][-1]
+    assert np.abs(out0 - got[3]).max() > 1e-3

@@ -68,6 +68,8 @@ class StreamConfig:
     cache_step: int = 0      # CACHE_FIXED_STEP: the step whose K/V every step reads for the prior blocks
     block_kind: int = BLOCK_ATTN
     ffn_dim: int = 0         # BLOCK_DIT: hidden width of the FFN
+    audio_tokens: int = 0    # BLOCK_DIT: audio tokens per block for the cross-attention (0: none)
+    audio_dim: int = 0       # their feature width
 
     @property
     def num_steps(self) -> int:
@@ -191,11 +193,15 @@ class Weights:
     w_ffn1: Optional[list] = None   # BLOCK_DIT: per layer [ffn_dim, hidden]
     w_ffn2: Optional[list] = None   # BLOCK_DIT: per layer [hidden, ffn_dim]
     ada: Optional[np.ndarray] = None  # BLOCK_DIT: float32 [L][num_steps + 1][6][hidden]
+    w_qc: Optional[list] = None     # audio cross-attention: per layer [hidden, hidden]
+    w_kvc: Optional[list] = None    # per layer [2 hidden, audio_dim] (rows 0..D-1 K, D..2D-1 V)
+    w_oc: Optional[list] = None     # per layer [hidden, hidden]
 
 
 def make_weights(wl: Workload) -> Weights:
     """Draw order: per layer W_qkv then W_out, then W_in, W_head, then the sink; for
-    BLOCK_DIT then per layer W_ffn1, W_ffn2, then the AdaLN table.  The AdaLN vectors
+    BLOCK_DIT then per layer W_ffn1, W_ffn2, then the AdaLN table, then (audio_tokens > 0)
+    per layer W_qc, W_kvc (std 1/sqrt(audio_dim)), W_oc.  The AdaLN vectors
     of a (layer, timestep) are [shift1, scale1, gate1, shift2, scale2, gate2]: shifts
     and scales N(0, 0.1^2), gates N(1, 0.1^2); timestep index num_steps is t = 0."""
     c = wl.cfg
@@ -219,7 +225,14 @@ def make_weights(wl: Workload) -> Weights:
     ada = rng.standard_normal((c.num_layers, c.num_steps + 1, 6, D)) * 0.1
     ada[:, :, 2] += 1.0
     ada[:, :, 5] += 1.0
-    return Weights(w_qkv, w_out, w_in, w_head, sink, w1, w2, ada.astype(np.float32))
+    W = Weights(w_qkv, w_out, w_in, w_head, sink, w1, w2, ada.astype(np.float32))
+    if c.audio_tokens > 0:
+        W.w_qc, W.w_kvc, W.w_oc = [], [], []
+        for _ in range(c.num_layers):
+            W.w_qc.append(_to_dtype(rng.standard_normal((D, D)) * wl.w_std, c.dtype))
+            W.w_kvc.append(_to_dtype(rng.standard_normal((2 * D, c.audio_dim)) / np.sqrt(c.audio_dim), c.dtype))
+            W.w_oc.append(_to_dtype(rng.standard_normal((D, D)) * wl.w_std, c.dtype))
+    return W
 
 
 def block_noise(wl: Workload, b: int) -> np.ndarray:
@@ -227,6 +240,12 @@ def block_noise(wl: Workload, b: int) -> np.ndarray:
     c = wl.cfg
     return np.random.default_rng([wl.seed, b]).standard_normal(
         (c.block_tokens, c.latent_ch)).astype(np.float32)
+
+
+def block_audio(wl: Workload, b: int) -> np.ndarray:
+    """Audio features of block b for the cross-attention: [audio_tokens, audio_dim] float32 N(0, 1)."""
+    c = wl.cfg
+    return np.random.default_rng([wl.seed, b, 7]).standard_normal((c.audio_tokens, c.audio_dim)).astype(np.float32)
 
 
 def step_input(wl: Workload, b: int, i: int) -> np.ndarray:
