@@ -44,6 +44,9 @@ WORKLOAD = dict(
 ATTN_DRAM_BYTES_PER_SLOT = 427.3e6
 # FFN width of the full DiT block in the ablation: the 14B Wan-style DiT's 13824 (2.7 x 5120)
 DIT_FFN = 13824
+# Audio of a block for the DiT block's cross-attention (synthetic sizes; the pages give none):
+# 256 tokens of width 1024
+DIT_AUDIO = (256, 1024)
 
 
 def max_over_ranks(x, device):
@@ -455,13 +458,18 @@ def run_ablation(args):
             ("fixed-noise cache (prior blocks at the last step's noise), sequential", SCHED_SEQUENTIAL,
              CACHE_FIXED_STEP, 4, 0, 0, 0),
             ("timestep-forced, grouped pipeline, full DiT block (AdaLN, GELU FFN 13824)", SCHED_PIPELINED,
-             CACHE_TIMESTEP, 4, 0, 0, DIT_FFN))
+             CACHE_TIMESTEP, 4, 0, 0, DIT_FFN),
+            ("timestep-forced, grouped pipeline, full DiT block with audio cross-attention (256 x 1024)",
+             SCHED_PIPELINED, CACHE_TIMESTEP, 4, 0, 0, -DIT_FFN))
     for idx, (name, sched, mode, nfe, fp8, afp8, ffn) in enumerate(rows):
         if only is not None and str(idx) not in only:
             continue
+        audio = ffn < 0            # a negative FFN width marks the row with the audio cross-attention
+        ffn = abs(ffn)
         cfg = STREAM.cfg.replace(schedule=sched, cache_mode=mode, proj_fp8=fp8, attn_fp8=afp8,
                                  cache_step=STREAM.cfg.num_steps - 1,
-                                 block_kind=BLOCK_DIT if ffn else BLOCK_ATTN, ffn_dim=ffn)
+                                 block_kind=BLOCK_DIT if ffn else BLOCK_ATTN, ffn_dim=ffn,
+                                 audio_tokens=DIT_AUDIO[0] if audio else 0, audio_dim=DIT_AUDIO[1] if audio else 0)
         T, C, D, F = cfg.block_tokens, cfg.latent_ch, cfg.hidden, cfg.frame_tokens
         S, nw, L = cfg.num_steps, cfg.window_blocks, cfg.num_layers
         g = torch.Generator(device="cuda")
@@ -478,25 +486,31 @@ def run_ablation(args):
             ada[:, :, 2] += 1.0
             ada[:, :, 5] += 1.0
             weights["ada"] = ada.contiguous()
+        if audio:
+            weights["w_qc"] = [rnd((D, D), STREAM.w_std) for _ in range(L)]
+            weights["w_kvc"] = [rnd((2 * D, DIT_AUDIO[1]), DIT_AUDIO[1] ** -0.5) for _ in range(L)]
+            weights["w_oc"] = [rnd((D, D), STREAM.w_std) for _ in range(L)]
+        aud = torch.randn(DIT_AUDIO, generator=g, device="cuda") if audio else None
         s = LaStream(cfg, weights)
         s.set_sink(torch.randn((F, C), generator=g, device="cuda"))
         xs = [torch.randn((T, C), generator=g, device="cuda") for _ in range(2)]
         x_out = torch.empty((T, C), device="cuda")
         fill = ((S - 1) if sched == SCHED_PIPELINED else 0) + nw + 1 + args.warmup
         for k in range(fill):
-            s.step(xs[k % 2], x_out)
+            s.step(xs[k % 2], x_out, audio=aud)
         s.synchronize()
         s.profile(True)
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record()
         for k in range(args.steps):
-            assert s.step(xs[k % 2], x_out) >= 0
+            assert s.step(xs[k % 2], x_out, audio=aud) >= 0
         ev1.record()
         s.synchronize()
         torch.cuda.synchronize()
         ms = ev0.elapsed_time(ev1) / args.steps
         kinds = {kd: round(s.profile_read(kd)[1] / args.steps, 3)
-                 for kd in ("qkv_gemm", "attn", "out_gemm", "other") + (("ffn",) if ffn else ())}
+                 for kd in ("qkv_gemm", "attn", "out_gemm", "other") + (("ffn",) if ffn else ())
+                 + (("cross",) if audio else ())}
         extra = {}
         if ffn:
             # per call (a tick, or a block's S steps): S passes x L layers x two GEMMs of 2 T D F flops
@@ -506,7 +520,9 @@ def run_ablation(args):
         print(json.dumps({"ablation": name, "nfe_per_block": nfe, "ms_per_block": round(ms, 3),
                           "latent_frames_per_s": round(cfg.frames_per_block / (ms / 1000.0), 3),
                           "ms_per_block_by_kind": kinds, **extra,
-                          "config": ("8 DiT blocks (AdaLN, GELU FFN %d)" % ffn if ffn else "8 sublayers")
+                          "config": ("8 DiT blocks (AdaLN, GELU FFN %d%s)" % (
+                                         ffn, ", audio cross-attention %d x %d" % DIT_AUDIO if audio else "")
+                                     if ffn else "8 sublayers")
                                     + ", hidden 5120, 40x128 heads, 30x52 grid, window 2, "
                                     + ", ".join([x for x in ("e4m3 QKV/output projections" if fp8 else "",
                                                              "e4m3 attention" if afp8 else "") if x]

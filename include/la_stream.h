@@ -140,6 +140,9 @@ typedef struct la_config {
                                   the other cache modes.                                */
   int32_t block_kind;          /* LA_BLOCK_ATTN | LA_BLOCK_DIT                           */
   int32_t ffn_dim;             /* LA_BLOCK_DIT: FFN hidden width F (multiple of 32)       */
+  int32_t audio_tokens;        /* LA_BLOCK_DIT: audio tokens A per block for the audio
+                                  cross-attention (0: none; then la_denoise_step_av)     */
+  int32_t audio_dim;           /* their feature width D_a (multiple of 8)               */
 } la_config;
 
 /* Layer kinds.  The pages give the model's base (a 14B DiT with timestep
@@ -150,7 +153,14 @@ typedef struct la_config {
  * with n the per-token RMS norm, Attn the attention sublayer (QKV, Rolling
  * RoPE, cache, block-causal attention, output projection) and the AdaLN
  * vectors of the layer at the step's timestep (la_weights.ada).  Needs
- * proj_fp8 = attn_fp8 = 0.  The FFN runs on the same GEMM kernels. */
+ * proj_fp8 = attn_fp8 = 0.  The FFN runs on the same GEMM kernels.
+ * With audio_tokens > 0 the block also has the audio cross-attention (the
+ * model is audio-driven; reading: Wan's cross-attention sub-block), between
+ * the attention and the FFN sub-blocks:
+ *   h += (softmax(q k^T / sqrt(d)) v) W_oc^T,  q = n(h) W_qc^T,  [k | v] = audio_b W_kvc^T
+ * over the A audio tokens of the block (no RoPE, no mask).  A block's audio
+ * K/V are computed once, when the block enters the stream; the sink pass
+ * has no audio and skips the sub-block. */
 #define LA_BLOCK_ATTN        0  /* each layer: the attention sublayer               */
 #define LA_BLOCK_DIT         1  /* each layer: the full DiT block                   */
 
@@ -173,6 +183,10 @@ typedef struct la_weights {
                                     vectors shift1, scale1, gate1, shift2, scale2, gate2 of
                                     each layer at timesteps[0 .. num_steps-1], and at t = 0
                                     (index num_steps: the sink pass and the clean refresh) */
+  /* LA_BLOCK_DIT with audio_tokens > 0 only: */
+  const void* const* w_qc;       /* HOST array of num_layers DEVICE pointers, each [D, D] */
+  const void* const* w_kvc;      /* ... each [2D, D_a]: rows 0..D-1 K, D..2D-1 V          */
+  const void* const* w_oc;       /* ... each [D, D]                                      */
 } la_weights;
 
 typedef struct la_stream la_stream;
@@ -219,6 +233,15 @@ int la_denoise_step(la_stream* s, const float* x_new, float* x_out, int64_t* fin
  * after enqueueing, so read x_out only after la_synchronize(). */
 int la_denoise_step_host(la_stream* s, const float* x_new_host, float* x_out_host,
                          int64_t* finished_block);
+
+/* la_denoise_step for streams with the audio cross-attention (audio_tokens >
+ * 0): audio_new (DEVICE fp32 [audio_tokens, audio_dim]) is the audio of the
+ * new block x_new (both NULL to drain).  Its K/V for every layer are
+ * computed in this call and kept while the block is in flight, so audio_new
+ * may be reused after the call is enqueued.  la_denoise_step and
+ * la_denoise_step_host return LA_EINVAL for a new block of such a stream. */
+int la_denoise_step_av(la_stream* s, const float* x_new, const float* audio_new, float* x_out,
+                       int64_t* finished_block);
 
 /* Wait for all work of the stream; LA_EDEVICE if a kernel raised the device
  * error word (the word is cleared after being reported). */
@@ -279,6 +302,13 @@ int la_debug_capture(la_stream* s, int32_t enable);
 #define LA_TAP_H_MID     16 /* fp32 [T_b, D] residual of layer after the attention sub-block   */
 #define LA_TAP_FFN_U     17 /* dtype [T_b, F] GELU output of layer's FFN (the second GEMM's
                                operand)                                                       */
+/* LA_BLOCK_DIT with audio only: */
+#define LA_TAP_H_CROSS   18 /* fp32 [T_b, D] residual of layer after the cross-attention      */
+#define LA_TAP_XQ        19 /* attn [H, T_b, d] cross-attention q (bf16 streams: times
+                               log2(e)/sqrt(d), like LA_TAP_Q)                                */
+#define LA_TAP_XK        20 /* attn [H, A, d] the block's audio K of layer                    */
+#define LA_TAP_XV        21 /* attn [H, A, d] the block's audio V of layer                    */
+#define LA_TAP_XO        22 /* fp32 [T_b, D] cross-attention output of layer, before rounding */
 
 /* Copy one tapped tensor into dst (DEVICE, dst_bytes >= the tensor's size),
  * ordered on the stream.  Taps other than ring / sink need capture enabled
@@ -301,7 +331,10 @@ int la_debug_set_slot_input(la_stream* s, int32_t slot, const float* x);
 #define LA_KIND_HEAD      5
 #define LA_KIND_OTHER     6
 #define LA_KIND_FFN       7  /* LA_BLOCK_DIT: the two FFN GEMMs                   */
-#define LA_NUM_KINDS      8
+#define LA_KIND_CROSS     8  /* LA_BLOCK_DIT with audio: the cross-attention's q and
+                                output GEMMs, head split and attention, and the
+                                audio K/V of each entering block                 */
+#define LA_NUM_KINDS      9
 int la_profile_enable(la_stream* s, int32_t enable);   /* resets the counters */
 int la_profile_read(la_stream* s, int32_t kind, int64_t* launches, double* total_ms);
 /* Kernels launched by this stream since creation. */

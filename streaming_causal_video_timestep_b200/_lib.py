@@ -16,8 +16,9 @@ LA_MAX_STEPS, LA_MAX_WINDOW, LA_MAX_FPB = 8, 14, 7
 LA_EPI_STORE, LA_EPI_RESID, LA_EPI_SET32, LA_EPI_EULER, LA_EPI_STORE32 = 0, 1, 2, 3, 4
 
 TAP = dict(x_in=0, x_out=1, h=2, q=3, o=4, v=5, ring_k=6, ring_v=7, sink_k=8, sink_v=9, sink_k_rope=10, sink_h=11,
-           hop=12, sink_hop=13, sink_v8=14, attn_scales=15, h_mid=16, ffn_u=17)
-KIND = dict(in_proj=0, qkv_gemm=1, rope=2, attn=3, out_gemm=4, head=5, other=6, ffn=7)
+           hop=12, sink_hop=13, sink_v8=14, attn_scales=15, h_mid=16, ffn_u=17, h_cross=18, xq=19, xk=20, xv=21,
+           xo=22)
+KIND = dict(in_proj=0, qkv_gemm=1, rope=2, attn=3, out_gemm=4, head=5, other=6, ffn=7, cross=8)
 
 
 class LaConfig(ctypes.Structure):
@@ -29,13 +30,15 @@ class LaConfig(ctypes.Structure):
         ("sink_mode", c_int32), ("rolling_rope", c_int32), ("sink_offset_frames", c_int32),
         ("schedule", c_int32), ("dtype", c_int32), ("cache_mode", c_int32), ("proj_fp8", c_int32),
         ("attn_fp8", c_int32), ("cache_step", c_int32), ("block_kind", c_int32), ("ffn_dim", c_int32),
+        ("audio_tokens", c_int32), ("audio_dim", c_int32),
     ]
 
 
 class LaWeights(ctypes.Structure):
     _fields_ = [("w_in", c_void_p), ("w_head", c_void_p), ("w_qkv", POINTER(c_void_p)),
                 ("w_out", POINTER(c_void_p)), ("w_ffn1", POINTER(c_void_p)), ("w_ffn2", POINTER(c_void_p)),
-                ("ada", c_void_p)]
+                ("ada", c_void_p), ("w_qc", POINTER(c_void_p)), ("w_kvc", POINTER(c_void_p)),
+                ("w_oc", POINTER(c_void_p))]
 
 
 class LaError(RuntimeError):
@@ -59,6 +62,7 @@ def load():
         "la_stream_create": (c_int, [POINTER(LaConfig), POINTER(LaWeights), c_void_p, POINTER(c_void_p)]),
         "la_set_sink": (c_int, [c_void_p, c_void_p]),
         "la_denoise_step": (c_int, [c_void_p, c_void_p, c_void_p, POINTER(c_int64)]),
+        "la_denoise_step_av": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(c_int64)]),
         "la_denoise_step_host": (c_int, [c_void_p, c_void_p, c_void_p, POINTER(c_int64)]),
         "la_synchronize": (c_int, [c_void_p]),
         "la_stream_destroy": (c_int, [c_void_p]),
@@ -98,7 +102,8 @@ def load():
 def exported_symbols():
     """Names of the C-ABI functions declared in include/la_stream.h."""
     return [
-        "la_stream_create", "la_set_sink", "la_denoise_step", "la_denoise_step_host", "la_synchronize",
+        "la_stream_create", "la_set_sink", "la_denoise_step", "la_denoise_step_host", "la_denoise_step_av",
+        "la_synchronize",
         "la_stream_destroy", "la_last_error", "la_status_string", "la_index_state_size", "la_get_index_state",
         "la_debug_capture", "la_debug_tap", "la_debug_set_slot_input", "la_profile_enable", "la_profile_read",
         "la_launch_count", "la_op_gemm", "la_op_attention", "la_op_euler", "la_op_attention_static",

@@ -359,6 +359,30 @@ __global__ void __launch_bounds__(256) k_rmsnorm_mod(const float* __restrict__ h
   }
 }
 
+// Token-major fp32 columns col0 .. col0 + H*d of src [rows, src_ld] to head-major
+// planes: dst[((row / rows_per_slice) * H + h) * rows_per_slice + row % rows_per_slice][e],
+// times scale, rounded once to TO.  One thread per 8 consecutive values.
+template <typename TO>
+__global__ void __launch_bounds__(256) k_split_heads(const float* __restrict__ src, long long rows,
+                                                     int rows_per_slice, int H, int d, long long src_ld,
+                                                     long long col0, TO* __restrict__ dst, float scale) {
+  const int chunks = d / 8;
+  const long long n = rows * H * chunks;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int ch = static_cast<int>(idx % chunks);
+    const long long rest = idx / chunks;
+    const int h = static_cast<int>(rest % H);
+    const long long row = rest / H;
+    float v[8];
+    Vec8<float>::load(src + row * src_ld + col0 + static_cast<long long>(h) * d + ch * 8, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= scale;
+    const long long slice = row / rows_per_slice, r = row - slice * rows_per_slice;
+    Vec8<TO>::store(dst + ((slice * H + h) * rows_per_slice + r) * d + ch * 8, v);
+  }
+}
+
 int grid_for(long long n, int per_block = 256) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -461,5 +485,20 @@ cudaError_t launch_rmsnorm_mod(const float* h, long long rows, long long D, floa
     return cudaErrorInvalidValue;
   k_rmsnorm_mod<<<static_cast<unsigned>(rows), 256, 0, st>>>(h, D, eps, m, static_cast<__nv_bfloat16*>(out_bf16),
                                                              out_f32);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_heads(int bf16_out, const float* src, long long rows, int rows_per_slice, int H, int d,
+                               long long src_ld, long long col0, void* dst, float scale, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (d % 8 != 0 || src_ld % 4 != 0 || col0 % 4 != 0 || rows_per_slice < 1) return cudaErrorInvalidValue;
+  const long long n = rows * H * (d / 8);
+  const int grid = grid_for(n);
+  if (bf16_out)
+    k_split_heads<__nv_bfloat16><<<grid, 256, 0, st>>>(src, rows, rows_per_slice, H, d, src_ld, col0,
+                                                        static_cast<__nv_bfloat16*>(dst), scale);
+  else
+    k_split_heads<float><<<grid, 256, 0, st>>>(src, rows, rows_per_slice, H, d, src_ld, col0,
+                                               static_cast<float*>(dst), scale);
   return cudaGetLastError();
 }

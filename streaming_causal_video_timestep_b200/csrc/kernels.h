@@ -102,6 +102,12 @@ cudaError_t launch_euler(float* x, const float* v, long long rows, long long C, 
 cudaError_t launch_rmsnorm(const float* h, long long rows, long long D, float eps, void* out_bf16, float* out_f32,
                            cudaStream_t st);
 
+// Token-major fp32 src [rows, src_ld], columns col0 + h*d + e, to head-major
+// planes dst [rows / rows_per_slice][H][rows_per_slice][d] times scale, bf16
+// (bf16_out) or fp32.  d % 8 == 0, src_ld and col0 multiples of 4.
+cudaError_t launch_split_heads(int bf16_out, const float* src, long long rows, int rows_per_slice, int H, int d,
+                               long long src_ld, long long col0, void* dst, float scale, cudaStream_t st);
+
 // AdaLN vectors of each row group (buffer) for the modulated norm.
 struct ModArgs {
   int rows_per_group;

@@ -162,6 +162,8 @@ struct la_stream {
   bool afp8 = false;        // e4m3 attention operands in the denoising passes (bf16 streams)
   bool dit = false;         // LA_BLOCK_DIT: each layer a full DiT block
   int Fffn = 0;             // its FFN width
+  bool cross = false;       // LA_BLOCK_DIT with audio: the audio cross-attention sub-block
+  int A = 0, Da = 0;        // audio tokens per block, their width
   size_t eq = 2;            // element of q_rope / sk_rope / the rings (1 with afp8, else ea)
   size_t es = 2;            // activation / weight element (bf16 or fp32)
   size_t ea = 2;            // attention operand element (bf16 or fp32)
@@ -176,6 +178,17 @@ struct la_stream {
   void* ffn_u = nullptr;                     // LA_BLOCK_DIT: GELU output [max(nbuf*T, F)][Fffn], dtype
   CUtensorMap tm_u{}, tm_s_u{};
   std::vector<CUtensorMap> tm_w1, tm_w2;
+  std::vector<const void*> w_qc, w_kvc, w_oc;   // audio cross-attention
+  void* audio_op = nullptr;  // bf16 [A][Da]: the GEMM operand of an entering block's audio
+  float* kv32 = nullptr;     // fp32 [A][2D]: one layer's audio K | V before the head split
+  void* audio_k = nullptr;   // attn [L][nbuf][H][A][d]: each in-flight block's audio K
+  void* audio_v = nullptr;
+  float* qc32 = nullptr;     // fp32 [nbuf*T][D]: cross-attention q before the head split
+  void* qc_heads = nullptr;  // attn [nbuf][H][T][d]
+  void* xo_buf = nullptr;    // dtype [nbuf*T][D]: cross-attention output (the self-attention's stays in attn_o)
+  CUtensorMap tm_audio_op{}, tm_xo{};
+  std::vector<CUtensorMap> tm_wqc, tm_wkvc, tm_woc;
+  AttnMaps maps_cross{};     // q = qc_heads; k[0] / v[0] = audio K / V
 
   std::vector<void*> allocs;
   float* xs = nullptr;      // [nbuf][T][C]
@@ -244,6 +257,12 @@ struct la_stream {
   void* cap_hop = nullptr;      // bf16 [S][L][T][D] normalised residual entering each QKV projection
   void* cap_sink_hop = nullptr; // bf16 [L][F][D] the same in the last sink pass
   float* cap_hmid = nullptr;    // LA_BLOCK_DIT: fp32 [S][L][T][D] residual after the attention sub-block
+  float* cap_hx = nullptr;      // audio: fp32 [S][L][T][D] residual after the cross-attention
+  void* cap_xq = nullptr;       // audio: attn [S][L][H][T][d] cross-attention q
+  void* cap_xk = nullptr;       // audio: attn [S][L][H][A][d] the block's audio K / V
+  void* cap_xv = nullptr;
+  float* cap_xo = nullptr;      // audio: fp32 [S][L][T][D] cross-attention output
+  float* cap_xoall = nullptr;   // audio, bf16 streams: fp32 [nbuf*T][D] cross-attention output of a pass
   void* cap_u = nullptr;        // LA_BLOCK_DIT: dtype [S][L][T][Fffn] GELU output
   bool cap_sink_valid = false;
   std::vector<int> cap_valid;  // per slot: captured in the last call
@@ -358,6 +377,11 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
     if (c->ffn_dim < 32 || c->ffn_dim % 32 != 0 || c->ffn_dim > (1 << 20)) { msg = "ffn_dim must be a multiple of 32"; return LA_EINVAL; }
     if (c->proj_fp8 || c->attn_fp8) { msg = "the DiT block runs without the e4m3 modes"; return LA_EINVAL; }
   }
+  if (c->audio_tokens != 0) {
+    if (c->block_kind != LA_BLOCK_DIT) { msg = "the audio cross-attention needs the DiT block"; return LA_EINVAL; }
+    if (c->audio_tokens < 0 || c->audio_tokens > 65536) { msg = "bad audio_tokens"; return LA_EINVAL; }
+    if (c->audio_dim < 8 || c->audio_dim % 8 != 0 || c->audio_dim > 65536) { msg = "audio_dim must be a multiple of 8"; return LA_EINVAL; }
+  }
   if (c->attn_fp8 && (c->dtype != LA_BF16 || c->head_dim != 128)) {
     msg = "e4m3 attention needs the bf16 stream and head_dim 128";
     return LA_EINVAL;
@@ -377,6 +401,11 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
     if (!w->w_ffn1 || !w->w_ffn2 || !w->ada) { msg = "the DiT block needs w_ffn1, w_ffn2 and ada"; return LA_EINVAL; }
     for (int l = 0; l < c->num_layers; ++l)
       if (!w->w_ffn1[l] || !w->w_ffn2[l]) { msg = "NULL FFN weight"; return LA_EINVAL; }
+  }
+  if (c->block_kind == LA_BLOCK_DIT && c->audio_tokens > 0) {
+    if (!w->w_qc || !w->w_kvc || !w->w_oc) { msg = "the audio cross-attention needs w_qc, w_kvc and w_oc"; return LA_EINVAL; }
+    for (int l = 0; l < c->num_layers; ++l)
+      if (!w->w_qc[l] || !w->w_kvc[l] || !w->w_oc[l]) { msg = "NULL cross-attention weight"; return LA_EINVAL; }
   }
   if (c->dtype == LA_BF16) {
     if (c->hidden % 64 != 0) { msg = "bf16 path needs hidden % 64 == 0"; return LA_EINVAL; }
@@ -525,6 +554,94 @@ int ffn_block(la_stream* s, float* h, long long rows, int rows_per_group, const 
   GemmEpiParams e2 = epi(EPI_RESID, nullptr, h, D);
   set_gates(s, e2, rows_per_group, tidx, ngroups, l, 5);
   return gemm(s, LA_KIND_FFN, tm_u, &s->tm_w2[l], s->ffn_u, s->w_ffn2[l], e2, static_cast<int>(rows), D, F);
+}
+
+// The audio K / V of every layer for the block entering buffer buf: [k | v] =
+// audio W_kvc^T (fp32), split into the buffer's head-major planes.
+int audio_kv(la_stream* s, const float* audio, int buf) {
+  const int D = s->D, H = s->H, d = s->d, A = s->A;
+  int r;
+  if (s->bf16 && (r = launch(s, LA_KIND_CROSS, [&] {
+                    return launch_cvt_bf16(audio, s->audio_op, static_cast<long long>(A) * s->Da, s->st);
+                  })) != LA_OK)
+    return r;
+  for (int l = 0; l < s->L; ++l) {
+    GemmEpiParams e = epi(s->bf16 ? EPI_STORE32 : EPI_STORE, s->kv32, nullptr, 2LL * D);
+    if ((r = gemm(s, LA_KIND_CROSS, &s->tm_audio_op, &s->tm_wkvc[l], audio, s->w_kvc[l], e, A, 2 * D, s->Da)) !=
+        LA_OK)
+      return r;
+    const long long plane = (static_cast<long long>(l) * s->nbuf + buf) * H * A * d;
+    for (int part = 0; part < 2; ++part)
+      if ((r = launch(s, LA_KIND_CROSS, [&] {
+             return launch_split_heads(s->bf16, s->kv32, A, A, H, d, 2LL * D, static_cast<long long>(part) * D,
+                                       elem(part ? s->audio_v : s->audio_k, plane, s->ea), 1.0f, s->st);
+           })) != LA_OK)
+        return r;
+  }
+  return LA_OK;
+}
+
+// The DiT block's audio cross-attention sub-block of layer l on the pass's rows:
+// q = n(h) W_qc^T (split into heads; bf16 streams times log2(e)/sqrt(d)),
+// attention over each active buffer's audio K / V, h += O W_oc^T.
+int cross_block(la_stream* s, const PassDesc& pd, int l, int rows) {
+  const int T = s->T, D = s->D, H = s->H, d = s->d, S = s->S;
+  int r;
+  if ((r = normalise(s, s->h32, rows, s->hop, s->bf16 ? nullptr : s->hn32)) != LA_OK) return r;
+  GemmEpiParams eq = epi(s->bf16 ? EPI_STORE32 : EPI_STORE, s->qc32, nullptr, D);
+  if ((r = gemm(s, LA_KIND_CROSS, &s->tm_hop, &s->tm_wqc[l], s->hn32, s->w_qc[l], eq, rows, D, D)) != LA_OK) return r;
+  const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  if ((r = launch(s, LA_KIND_CROSS, [&] {
+         return launch_split_heads(s->bf16, s->qc32, rows, T, H, d, D, 0, s->qc_heads, s->bf16 ? scale_log2 : 1.0f,
+                                   s->st);
+       })) != LA_OK)
+    return r;
+  AttnParams ap{};
+  ap.Tq = T; ap.H = H; ap.d = d;
+  ap.scale_log2 = scale_log2;
+  ap.q_prescaled = s->bf16 ? 1 : 0;
+  ap.out = s->xo_buf; ap.out_ld = D; ap.err = s->dev_err;
+  ap.out32 = (s->bf16 && s->capture) ? s->cap_xoall : nullptr;
+  ap.qbase = s->qc_heads;
+  ap.kbase[0] = s->audio_k; ap.vbase[0] = s->audio_v; ap.krows[0] = s->A; ap.vrows[0] = s->A;
+  ap.ngroups = pd.nactive;
+  for (int ai = 0; ai < pd.nactive; ++ai) {
+    const int buf = pd.active_buf[ai];
+    AttnGroup& g = ap.g[ai];
+    g.q_slice = buf;
+    g.out_row0 = buf * T;
+    g.nseg = 1;
+    const int plane = l * s->nbuf + buf;
+    g.seg[0] = AttnSeg{0, 0, plane, plane, s->A};
+  }
+  if (s->bf16) {
+    if ((r = launch(s, LA_KIND_CROSS, [&] { return launch_attention_tc(s->maps_cross, ap, s->st); })) != LA_OK) return r;
+  } else if ((r = launch(s, LA_KIND_CROSS, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) {
+    return r;
+  }
+  GemmEpiParams eo = epi(EPI_RESID, nullptr, s->h32, D);
+  if ((r = gemm(s, LA_KIND_CROSS, &s->tm_xo, &s->tm_woc[l], s->xo_buf, s->w_oc[l], eo, rows, D, D)) != LA_OK) return r;
+  if (s->capture) {
+    const float* o32 = s->bf16 ? s->cap_xoall : static_cast<const float*>(s->xo_buf);
+    const long long HTd = static_cast<long long>(H) * T * d, HAd = static_cast<long long>(H) * s->A * d;
+    for (int ai = 0; ai < pd.nactive; ++ai) {
+      const int buf = pd.active_buf[ai];
+      if (pd.step[buf] >= S) continue;
+      const long long at = static_cast<long long>(pd.step[buf]) * s->L + l;
+      const long long plane = static_cast<long long>(l) * s->nbuf + buf;
+      CU(cudaMemcpyAsync(s->cap_hx + at * T * D, s->h32 + static_cast<long long>(buf) * T * D,
+                         static_cast<size_t>(T) * D * 4, cudaMemcpyDeviceToDevice, s->st));
+      CU(cudaMemcpyAsync(s->cap_xo + at * T * D, o32 + static_cast<long long>(buf) * T * D,
+                         static_cast<size_t>(T) * D * 4, cudaMemcpyDeviceToDevice, s->st));
+      CU(cudaMemcpyAsync(elem(s->cap_xq, at * HTd, s->ea), elem(s->qc_heads, buf * HTd, s->ea), HTd * s->ea,
+                         cudaMemcpyDeviceToDevice, s->st));
+      CU(cudaMemcpyAsync(elem(s->cap_xk, at * HAd, s->ea), elem(s->audio_k, plane * HAd, s->ea), HAd * s->ea,
+                         cudaMemcpyDeviceToDevice, s->st));
+      CU(cudaMemcpyAsync(elem(s->cap_xv, at * HAd, s->ea), elem(s->audio_v, plane * HAd, s->ea), HAd * s->ea,
+                         cudaMemcpyDeviceToDevice, s->st));
+    }
+  }
+  return LA_OK;
 }
 
 // One grouped pass over nbuf buffers (rows = nbuf*T) with the active ones in pd.
@@ -691,6 +808,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
         }
       };
       cap(false);
+      if (s->cross && (r = cross_block(s, pd, l, rows)) != LA_OK) return r;
       if ((r = ffn_block(s, s->h32, rows, T, tidx, pd.nbuf, l, s->hop, s->hn32, &s->tm_hop, &s->tm_u,
                          [&] { cap(true); })) != LA_OK)
         return r;
@@ -857,9 +975,12 @@ void fill_pass_slot(la_stream* s, PassDesc& pd, int buf, int ring, int step, lon
 }
 
 int step_impl(la_stream* s, const float* x_new, float* x_out, int64_t* finished_block, cudaMemcpyKind in_kind,
-              cudaMemcpyKind out_kind) {
+              cudaMemcpyKind out_kind, const float* audio_new = nullptr) {
   if (!s) return LA_EINVAL;
   if (!finished_block || !x_out) return fail(s, LA_EINVAL, "NULL x_out or finished_block");
+  if (s->cross && x_new && !audio_new)
+    return fail(s, LA_EINVAL, "this stream has the audio cross-attention: la_denoise_step_av with the block's audio");
+  if (!s->cross && audio_new) return fail(s, LA_EINVAL, "this stream has no audio cross-attention");
   if (!s->sink_set) return fail(s, LA_ESTATE, "la_set_sink must be called first");
   const bool has_new = x_new != nullptr;
   const bool pipelined = s->cfg.schedule == LA_SCHED_PIPELINED;
@@ -879,6 +1000,7 @@ int step_impl(la_stream* s, const float* x_new, float* x_out, int64_t* finished_
   if (pipelined) {
     if (has_new)
       CU(cudaMemcpyAsync(s->xs + (new_block % s->S) * TC, x_new, TC * 4, in_kind, s->st));
+    if (has_new && s->cross && (r = audio_kv(s, audio_new, static_cast<int>(new_block % s->S))) != LA_OK) return r;
     PassDesc pd{};
     pd.nbuf = s->S;
     for (auto& [slot, b] : run) {
@@ -890,6 +1012,7 @@ int step_impl(la_stream* s, const float* x_new, float* x_out, int64_t* finished_
       CU(cudaMemcpyAsync(x_out, s->xs + (finished % s->S) * TC, TC * 4, out_kind, s->st));
   } else {
     CU(cudaMemcpyAsync(s->xs, x_new, TC * 4, in_kind, s->st));
+    if (s->cross && (r = audio_kv(s, audio_new, 0)) != LA_OK) return r;
     for (auto& [slot, b] : run) {
       PassDesc pd{};
       pd.nbuf = 1;
@@ -938,6 +1061,14 @@ int alloc_capture(la_stream* s) {
   if (s->dit) {
     DALLOC(s->cap_hmid, S * L * T * D * 4);
     DALLOC(s->cap_u, S * L * T * s->Fffn * static_cast<long long>(s->es));
+  }
+  if (s->cross) {
+    DALLOC(s->cap_hx, S * L * T * D * 4);
+    DALLOC(s->cap_xo, S * L * T * D * 4);
+    DALLOC(s->cap_xq, S * L * H * T * d * s->ea);
+    DALLOC(s->cap_xk, S * L * H * s->A * d * s->ea);
+    DALLOC(s->cap_xv, S * L * H * s->A * d * s->ea);
+    if (s->bf16) DALLOC(s->cap_xoall, static_cast<long long>(s->nbuf) * T * D * 4);
   }
   s->cap_valid.assign(s->S, 0);
   return LA_OK;
@@ -996,6 +1127,9 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   s->afp8 = s->bf16 && cfg->attn_fp8;
   s->dit = cfg->block_kind == LA_BLOCK_DIT;
   s->Fffn = s->dit ? cfg->ffn_dim : 0;
+  s->cross = s->dit && cfg->audio_tokens > 0;
+  s->A = s->cross ? cfg->audio_tokens : 0;
+  s->Da = s->cross ? cfg->audio_dim : 0;
   s->eq = s->afp8 ? 1 : s->ea;
   s->id_in = w->w_in == nullptr; s->id_head = w->w_head == nullptr;
   s->nbuf = cfg->schedule == LA_SCHED_PIPELINED ? s->S : 1;
@@ -1007,6 +1141,11 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
     s->w_ffn1.assign(w->w_ffn1, w->w_ffn1 + s->L);
     s->w_ffn2.assign(w->w_ffn2, w->w_ffn2 + s->L);
     s->ada = w->ada;
+  }
+  if (s->cross) {
+    s->w_qc.assign(w->w_qc, w->w_qc + s->L);
+    s->w_kvc.assign(w->w_kvc, w->w_kvc + s->L);
+    s->w_oc.assign(w->w_oc, w->w_oc + s->L);
   }
   s->sched.init(s->cfg);
 
@@ -1029,7 +1168,11 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
                          NB * T * D * eq + NB * T * D * es + NB * H * F * d * eq + 2 * L * S * E * H * T * d * eq +
                          L * H * F * d * (4 + ea) + F * C * 4 + F * D * 4 + F * D * es * 2 + F * C * 2 +
                          F * 3 * D * 4 + 2 * H * F * d * ea + (s->afp8 ? L * H * F * d + L * 3 * H * 8 : 0) +
-                         (s->dit ? std::max(NB * T, F) * s->Fffn * static_cast<long long>(es) : 0) + (64 << 20);
+                         (s->dit ? std::max(NB * T, F) * s->Fffn * static_cast<long long>(es) : 0) +
+                         (s->cross ? static_cast<long long>(s->A) * (s->Da * 2 + 2 * D * 4) + 2 * L * NB * s->A * D * ea +
+                                         NB * T * D * (4 + ea + es)
+                                   : 0) +
+                         (64 << 20);
   size_t free_b = 0, total_b = 0;
   e = cudaMemGetInfo(&free_b, &total_b);
   if (e != cudaSuccess) { s->err = cudaGetErrorString(e); return bail(LA_ECUDA); }
@@ -1059,6 +1202,16 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   ALLOC_OR_BAIL(s->sink_k, L * H * F * d * 4);
   ALLOC_OR_BAIL(s->sink_v, L * H * F * d * ea);
   if (s->dit) ALLOC_OR_BAIL(s->ffn_u, std::max(NB * T, F) * s->Fffn * static_cast<long long>(es));
+  if (s->cross) {
+    const long long Aa = s->A;
+    if (s->bf16) ALLOC_OR_BAIL(s->audio_op, Aa * s->Da * 2);
+    ALLOC_OR_BAIL(s->kv32, Aa * 2 * D * 4);
+    ALLOC_OR_BAIL(s->audio_k, L * NB * Aa * D * ea);
+    ALLOC_OR_BAIL(s->audio_v, L * NB * Aa * D * ea);
+    ALLOC_OR_BAIL(s->qc32, NB * T * D * 4);
+    ALLOC_OR_BAIL(s->qc_heads, NB * T * D * ea);
+    ALLOC_OR_BAIL(s->xo_buf, NB * T * D * es);
+  }
   if (s->afp8) {
     ALLOC_OR_BAIL(s->sink_v8, L * H * F * d);
     ALLOC_OR_BAIL(s->attn_sc, L * 3 * H * 4);
@@ -1132,6 +1285,22 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
         ok = ok && tmap_2d_bf16(&s->tm_w1[l], s->w_ffn1[l], Ff, D, D, gemm_tc_pick_bn(s->Fffn), s->err);
         ok = ok && tmap_2d_bf16(&s->tm_w2[l], s->w_ffn2[l], D, Ff, Ff, bn_d, s->err);
       }
+    }
+    if (s->cross) {
+      const long long Aa = s->A;
+      ok = ok && tmap_2d_bf16(&s->tm_audio_op, s->audio_op, Aa, s->Da, s->Da, 128, s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_xo, s->xo_buf, NB * T, D, D, 128, s->err);
+      s->tm_wqc.resize(L);
+      s->tm_wkvc.resize(L);
+      s->tm_woc.resize(L);
+      for (int l = 0; l < L && ok; ++l) {
+        ok = ok && tmap_2d_bf16(&s->tm_wqc[l], s->w_qc[l], D, D, D, bn_d, s->err);
+        ok = ok && tmap_2d_bf16(&s->tm_wkvc[l], s->w_kvc[l], 2 * D, s->Da, s->Da, gemm_tc_pick_bn(2 * s->D), s->err);
+        ok = ok && tmap_2d_bf16(&s->tm_woc[l], s->w_oc[l], D, D, D, bn_d, s->err);
+      }
+      ok = ok && tmap_planes_bf16(&s->maps_cross.q, s->qc_heads, d, T, H, NB, s->err);
+      ok = ok && tmap_planes_bf16(&s->maps_cross.k[0], s->audio_k, d, Aa, H, L * NB, s->err);
+      ok = ok && tmap_planes_bf16(&s->maps_cross.v[0], s->audio_v, d, Aa, H, L * NB, s->err);
     }
     if (!s->id_in) {
       ok = ok && tmap_2d_bf16(&s->tm_xop, s->xop, NB * T, C, C, 128, s->err);
@@ -1215,6 +1384,13 @@ int la_denoise_step_host(la_stream* s, const float* x_new_host, float* x_out_hos
   return step_impl(s, x_new_host, x_out_host, finished_block, cudaMemcpyHostToDevice, cudaMemcpyDeviceToHost);
 }
 
+int la_denoise_step_av(la_stream* s, const float* x_new, const float* audio_new, float* x_out,
+                       int64_t* finished_block) {
+  if (s && (x_new == nullptr) != (audio_new == nullptr))
+    return fail(s, LA_EINVAL, "x_new and audio_new must both be set or both NULL");
+  return step_impl(s, x_new, x_out, finished_block, cudaMemcpyDeviceToDevice, cudaMemcpyDeviceToDevice, audio_new);
+}
+
 int la_synchronize(la_stream* s) {
   if (!s) return LA_EINVAL;
   CU(cudaStreamSynchronize(s->st));
@@ -1262,13 +1438,15 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
                          what == LA_TAP_RING_V || what == LA_TAP_SINK_K || what == LA_TAP_SINK_V ||
                          what == LA_TAP_SINK_KROPE || what == LA_TAP_SINK_H || what == LA_TAP_HOP ||
                          what == LA_TAP_SINK_HOP || what == LA_TAP_SINK_V8 || what == LA_TAP_ATTN_SCALES ||
-                         what == LA_TAP_H_MID || what == LA_TAP_FFN_U;
+                         what == LA_TAP_H_MID || what == LA_TAP_FFN_U || (what >= LA_TAP_H_CROSS && what <= LA_TAP_XO);
   if (per_layer && (layer < (what == LA_TAP_H ? -1 : 0) || layer >= L)) return fail(s, LA_EINVAL, "bad layer");
   if (slot < 0 || slot >= S) return fail(s, LA_EINVAL, "bad slot");
   const void* src = nullptr;
   long long bytes = 0;
+  const bool xtap = what >= LA_TAP_H_CROSS && what <= LA_TAP_XO;
   const bool needs_capture = what <= LA_TAP_V || what == LA_TAP_SINK_KROPE || what == LA_TAP_HOP ||
-                             what == LA_TAP_H_MID || what == LA_TAP_FFN_U;
+                             what == LA_TAP_H_MID || what == LA_TAP_FFN_U || xtap;
+  if (xtap && !s->cross) return fail(s, LA_EINVAL, "the cross-attention taps exist with audio only");
   if ((what == LA_TAP_H_MID || what == LA_TAP_FFN_U) && !s->dit)
     return fail(s, LA_EINVAL, "the FFN taps exist with the DiT block only");
   if ((what == LA_TAP_HOP || what == LA_TAP_SINK_HOP) && !s->bf16)
@@ -1295,6 +1473,14 @@ int la_debug_tap(la_stream* s, int32_t what, int32_t layer, int32_t slot, void* 
     case LA_TAP_SINK_V: src = elem(s->sink_v, static_cast<long long>(layer) * H * F * d, ea); bytes = H * F * d * ea; break;
     case LA_TAP_SINK_V8: src = s->sink_v8 + static_cast<long long>(layer) * H * F * d; bytes = H * F * d; break;
     case LA_TAP_H_MID: src = s->cap_hmid + (slot * L + layer) * T * D; bytes = T * D * 4; break;
+    case LA_TAP_H_CROSS: src = s->cap_hx + (slot * L + layer) * T * D; bytes = T * D * 4; break;
+    case LA_TAP_XO: src = s->cap_xo + (slot * L + layer) * T * D; bytes = T * D * 4; break;
+    case LA_TAP_XQ: src = elem(s->cap_xq, (slot * L + layer) * H * T * d, ea); bytes = H * T * d * ea; break;
+    case LA_TAP_XK:
+    case LA_TAP_XV:
+      src = elem(what == LA_TAP_XK ? s->cap_xk : s->cap_xv, (slot * L + layer) * H * s->A * d, ea);
+      bytes = H * s->A * d * ea;
+      break;
     case LA_TAP_FFN_U:
       src = elem(s->cap_u, (slot * L + layer) * T * s->Fffn, s->es);
       bytes = T * s->Fffn * static_cast<long long>(s->es);

@@ -76,6 +76,8 @@ class LaStream:
         c.cache_step = getattr(cfg, "cache_step", 0)
         c.block_kind = getattr(cfg, "block_kind", 0)
         c.ffn_dim = getattr(cfg, "ffn_dim", 0)
+        c.audio_tokens = getattr(cfg, "audio_tokens", 0)
+        c.audio_dim = getattr(cfg, "audio_dim", 0)
         self.cfg = cfg
         self.c = c
         self.T = cfg.frames_per_block * cfg.grid_h * cfg.grid_w
@@ -101,6 +103,14 @@ class LaStream:
             w.w_ffn1 = ctypes.cast(self._w1, ctypes.POINTER(c_void_p))
             w.w_ffn2 = ctypes.cast(self._w2, ctypes.POINTER(c_void_p))
             w.ada = weights["ada"].data_ptr()
+        if weights.get("w_qc") is not None:
+            # the audio cross-attention: per layer [D, D], [2D, D_a], [D, D]
+            self._wqc = (c_void_p * L)(*[t.data_ptr() for t in weights["w_qc"]])
+            self._wkvc = (c_void_p * L)(*[t.data_ptr() for t in weights["w_kvc"]])
+            self._woc = (c_void_p * L)(*[t.data_ptr() for t in weights["w_oc"]])
+            w.w_qc = ctypes.cast(self._wqc, ctypes.POINTER(c_void_p))
+            w.w_kvc = ctypes.cast(self._wkvc, ctypes.POINTER(c_void_p))
+            w.w_oc = ctypes.cast(self._woc, ctypes.POINTER(c_void_p))
         self.w = w
         h = c_void_p()
         code = self.lib.la_stream_create(ctypes.byref(c), ctypes.byref(w), _stream_handle(self.stream), ctypes.byref(h))
@@ -127,13 +137,22 @@ class LaStream:
         _require(latent, torch.float32, (self.F, self.C), "sink latent")
         self._check(self.lib.la_set_sink(self.h, _ptr(latent)))
 
-    def step(self, x_new, x_out):
-        """One call of la_denoise_step; returns the finished block id or -1."""
+    def step(self, x_new, x_out, audio=None):
+        """One call of la_denoise_step (la_denoise_step_av when the stream has the audio
+        cross-attention; audio: the new block's fp32 [audio_tokens, audio_dim]); returns
+        the finished block id or -1."""
         if x_new is not None:
             _require(x_new, torch.float32, (self.T, self.C), "x_new")
         _require(x_out, torch.float32, (self.T, self.C), "x_out")
         fin = c_int64(-1)
-        self._check(self.lib.la_denoise_step(self.h, _ptr(x_new), _ptr(x_out), ctypes.byref(fin)))
+        A = getattr(self.cfg, "audio_tokens", 0)
+        if A > 0:
+            if audio is not None:
+                _require(audio, torch.float32, (A, self.cfg.audio_dim), "audio")
+            self._check(self.lib.la_denoise_step_av(self.h, _ptr(x_new), _ptr(audio), _ptr(x_out),
+                                                    ctypes.byref(fin)))
+        else:
+            self._check(self.lib.la_denoise_step(self.h, _ptr(x_new), _ptr(x_out), ctypes.byref(fin)))
         return fin.value
 
     def step_host(self, x_new_host, x_out_host):
@@ -170,9 +189,14 @@ class LaStream:
             "hop": ((T, D), dt), "sink_hop": ((F, D), dt),
             "sink_v8": ((H, F, d), torch.uint8), "attn_scales": ((3, H), torch.float32),
             "h_mid": ((T, D), torch.float32), "ffn_u": ((T, max(1, getattr(self.cfg, "ffn_dim", 0))), dt),
+            "h_cross": ((T, D), torch.float32), "xo": ((T, D), torch.float32), "xq": ((H, T, d), dt),
+            "xk": ((H, max(1, getattr(self.cfg, "audio_tokens", 0)), d), dt),
+            "xv": ((H, max(1, getattr(self.cfg, "audio_tokens", 0)), d), dt),
         }
         shape, tdt = shapes[what]
-        if what in ("q", "ring_k", "ring_v", "sink_k_rope") and getattr(self.cfg, "attn_fp8", 0):
+        if what in ("xq", "xk", "xv"):
+            tdt = attn_dtype(self.dtype)
+        elif what in ("q", "ring_k", "ring_v", "sink_k_rope") and getattr(self.cfg, "attn_fp8", 0):
             tdt = torch.uint8          # e4m3 codes
         elif what in ("q", "ring_k", "ring_v", "sink_v", "sink_k_rope"):
             tdt = attn_dtype(self.dtype)

@@ -39,6 +39,10 @@ def torch_weights(W, cfg, device="cuda"):
         out["w_ffn1"] = [conv(w) for w in W.w_ffn1]
         out["w_ffn2"] = [conv(w) for w in W.w_ffn2]
         out["ada"] = torch.from_numpy(np.ascontiguousarray(W.ada, np.float32)).to(device)
+    if getattr(W, "w_qc", None) is not None:
+        out["w_qc"] = [conv(w) for w in W.w_qc]
+        out["w_kvc"] = [conv(w) for w in W.w_kvc]
+        out["w_oc"] = [conv(w) for w in W.w_oc]
     return out
 
 

@@ -154,8 +154,9 @@ def sink_snapshot(s, cfg):
     return snap
 
 
-def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
-    """sink: sink_snapshot() taken before the call (default: the current sink)."""
+def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None, audio=None):
+    """sink: sink_snapshot() taken before the call (default: the current sink); audio:
+    block b's audio features (streams with the audio cross-attention)."""
     dt = cfg.dtype
     T, D, H, d, E, L = cfg.block_tokens, cfg.hidden, cfg.heads, cfg.head_dim, cfg.ring_entries, cfg.num_layers
     R = np.arange(T) if rows is None else np.asarray(rows)
@@ -227,7 +228,7 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None):
         # output projection + residual from the attention output as the GEMM consumes it
         h_next = to_np(s.tap("h", l, i))
         if _dit(cfg):
-            _check_ffn(s, cfg, W, l, i, R, h_prev, o_gpu, h_next, chk)
+            _check_ffn(s, cfg, W, l, i, R, h_prev, o_gpu, h_next, chk, audio)
             h_prev = h_next
             continue
         want = h_prev[R].astype(np.float64) + _proj(_operand(o_gpu[R], cfg), W.w_out[l], cfg)
@@ -273,16 +274,42 @@ def _check_attn_fp8(s, cfg, W, b, i, l, R, qr, kr, v, sink, st, chk, errs, tag):
         errs[k_] = max(errs.get(k_, (0, 0)), (f_, 0.0))
 
 
-def _check_ffn(s, cfg, W, l, i, R, h_prev, o_gpu, h_next, chk):
-    """The DiT block after attention: the gated output projection (h_mid), the
-    AdaLN-modulated FFN operand and its GELU output (u), and the gated FFN residual,
-    each from the GPU's own inputs."""
+def _check_ffn(s, cfg, W, l, i, R, h_prev, o_gpu, h_next, chk, audio=None):
+    """The DiT block after attention: the gated output projection (h_mid), the audio
+    cross-attention (when the stream has audio), the AdaLN-modulated FFN operand and
+    its GELU output (u), and the gated FFN residual, each from the GPU's own inputs."""
     a = np.asarray(W.ada, np.float64)[l, i]
     h_mid = to_np(s.tap("h_mid", l, i))
     want = h_prev[R].astype(np.float64) + a[2] * _proj(_operand(o_gpu[R], cfg), W.w_out[l], cfg)
     chk(h_mid[R], want, f"h mid l{l}")
+    if getattr(cfg, "audio_tokens", 0) > 0:
+        h_mid = _check_cross(s, cfg, W, l, i, R, h_mid, audio, chk)
     m2 = _operand(modulate(h_mid[R].astype(np.float64), a[3], a[4]).astype(np.float32), cfg)
     u_gpu = to_np(s.tap("ffn_u", l, i))
     chk(u_gpu[R], gelu_tanh(m2 @ np.asarray(W.w_ffn1[l], np.float64).T), f"ffn gelu l{l}")
     want = h_mid[R].astype(np.float64) + a[5] * (_operand(u_gpu[R], cfg) @ np.asarray(W.w_ffn2[l], np.float64).T)
     chk(h_next[R], want, f"h l{l}")
+
+
+def _check_cross(s, cfg, W, l, i, R, h_mid, audio, chk):
+    """The audio cross-attention sub-block from the GPU's inputs: its q from the
+    residual, the block's audio K / V, the attention from the GPU's q / K / V, and
+    the residual after the output projection.  Returns the GPU's residual after it."""
+    D, H, d = cfg.hidden, cfg.heads, cfg.head_dim
+    q_want = (_normed_operand(h_mid[R], cfg) @ np.asarray(W.w_qc[l], np.float64).T).reshape(len(R), H, d)
+    xq = to_np(s.tap("xq", l, i)).transpose(1, 0, 2)                 # [T, H, d]
+    qs = float(np.float32(math.log2(math.e) / math.sqrt(d))) if cfg.dtype == DTYPE_BF16 else 1.0
+    chk(xq[R] / qs, q_want, f"cross q l{l}")
+    kv = _operand(np.asarray(audio, np.float32), cfg) @ np.asarray(W.w_kvc[l], np.float64).T
+    A = kv.shape[0]
+    xk = to_np(s.tap("xk", l, i)).transpose(1, 0, 2)                 # [A, H, d]
+    xv = to_np(s.tap("xv", l, i)).transpose(1, 0, 2)
+    chk(xk, kv[:, :D].reshape(A, H, d), f"cross K l{l}")
+    chk(xv, kv[:, D:].reshape(A, H, d), f"cross V l{l}")
+    o_want = block_causal_attention(xq[R] / qs, {0: (xk, xv)}, None, qblock=0, window=0)
+    xo = to_np(s.tap("xo", l, i))
+    chk(xo[R], o_want.reshape(len(R), D), f"cross O l{l}")
+    h_x = to_np(s.tap("h_cross", l, i))
+    want = h_mid[R].astype(np.float64) + _operand(xo[R], cfg) @ np.asarray(W.w_oc[l], np.float64).T
+    chk(h_x[R], want, f"h cross l{l}")
+    return h_x

@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 from oracle import OracleStream, TickScheduler
-from workloads import (BLOCK_DIT, CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, DTYPE_BF16, DTYPE_FP32, SCHED_PIPELINED,
+from workloads import (BLOCK_DIT, CACHE_CLEAN_REFRESH, CACHE_FIXED_STEP, DTYPE_BF16, block_audio, DTYPE_FP32, SCHED_PIPELINED,
                        SCHED_SEQUENTIAL, SINK_AAS, SINK_FIXED, TINY, StreamConfig, Workload, block_noise, make_weights)
 
 from _helpers import assert_close, errors, make_stream, to_np
@@ -57,18 +57,21 @@ def _run_teacher_forced(wl, check_every_tick=True):
     per = 8 + 3 * cfg.ring_entries
     report = {}
     drain = S - 1 if cfg.schedule == SCHED_PIPELINED else 0     # the sequential schedule has no pipeline
+    has_audio = getattr(cfg, "audio_tokens", 0) > 0
     for k in range(nb + drain):
         xn = block_noise(wl, k) if k < nb else None
+        au = block_audio(wl, k) if (k < nb and has_audio) else None
         sink = sink_snapshot(s, cfg)
-        fin = s.step(_dev(xn) if xn is not None else None, x_out)
+        fin = s.step(_dev(xn) if xn is not None else None, x_out, audio=_dev(au) if au is not None else None)
         st = s.index_state()
         ran = [(int(st[4 + i * per]), i) for i in range(S) if st[4 + i * per] >= 0]
         if check_every_tick or k >= nb + drain - 1:
             for (b, i) in ran:
-                check_step(s, cfg, W, b, i, tag=f"tick {k}", report=report, sink=sink)
+                check_step(s, cfg, W, b, i, tag=f"tick {k}", report=report, sink=sink,
+                           audio=block_audio(wl, b) if has_audio else None)
         inputs = {(b, i): to_np(s.tap("x_in", 0, i)) for (b, i) in ran}
         got = to_np(x_out).copy() if fin >= 0 else None
-        out, fin_o = orc.denoise_step(xn, inputs=inputs, aas_latent=got if fin == 0 else None)
+        out, fin_o = orc.denoise_step(xn, inputs=inputs, aas_latent=got if fin == 0 else None, audio=au)
         assert fin == fin_o
         np.testing.assert_array_equal(st, orc.index_state())
         if fin >= 0:
@@ -294,6 +297,33 @@ def test_tiny_fp32_dit_stream_free_running_and_sequential():
 def test_small_bf16_dit_stream_teacher_forced():
     report = _run_teacher_forced(SMALL_DIT)
     print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in report.items()})
+
+
+TINY_DIT_AV = Workload("tiny-dit-av", TINY_DIT.cfg.replace(audio_tokens=20, audio_dim=24), TINY.seed, 5,
+                       TINY.w_std, TINY.head_std)
+SMALL_DIT_AV = Workload("small-bf16-dit-av", SMALL_DIT.cfg.replace(audio_tokens=150, audio_dim=64),
+                        SMALL_BF16.seed, 5, SMALL_BF16.w_std, SMALL_BF16.head_std)
+
+
+def test_tiny_fp32_dit_stream_with_audio_every_tick_matches_oracle():
+    """The audio cross-attention: its q, the block's audio K / V, the attention and the
+    residual after it per op every tick, and the finished blocks within 1e-5."""
+    _run_teacher_forced(TINY_DIT_AV)
+
+
+def test_small_bf16_dit_stream_with_audio_teacher_forced():
+    """150 audio tokens: a full key tile and a ragged one."""
+    report = _run_teacher_forced(SMALL_DIT_AV)
+    print({k: (f"{v[0]:.2e}", f"{v[1]:.2e}") for k, v in report.items()})
+
+
+def test_audio_stream_needs_the_audio():
+    from streaming_causal_video_timestep_b200 import LaError
+    s, W = make_stream(TINY_DIT_AV)
+    x_out = torch.empty((TINY_DIT_AV.cfg.block_tokens, TINY_DIT_AV.cfg.latent_ch), device="cuda")
+    with pytest.raises(LaError):
+        s.step(_dev(block_noise(TINY_DIT_AV, 0)), x_out)          # no audio
+    s.close()
 
 
 def test_dit_block_rejects_the_e4m3_modes():
