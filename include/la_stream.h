@@ -63,6 +63,11 @@ extern "C" {
 #define LA_SINK_AAS          1  /* sink replaced once by frame 0 of finished block 0  */
 #define LA_SCHED_PIPELINED   0  /* one call = one tick: slot i runs step i of block k-i */
 #define LA_SCHED_SEQUENTIAL  1  /* one call = one block through all steps in order     */
+#define LA_SCHED_SLOT        2  /* one rank of the timestep pipeline across GPUs (TPP):
+                                   one call = step slot_index of the next block, with
+                                   that step's own cache; the caller moves the latent
+                                   from rank to rank and replaces the sink on every
+                                   rank (la_replace_sink) when block 0 finishes       */
 #define LA_BF16              0  /* bf16 GEMM operands and attention operands, fp32
                                    accumulation, fp32 residual stream and latent x    */
 #define LA_FP32              1  /* fp32 everywhere (SIMT path, no TF32)                */
@@ -113,7 +118,7 @@ typedef struct la_config {
   int32_t rolling_rope;        /* 1: sink t-pos = frames_per_block*b - sink_offset_frames;
                                   0: fixed at -sink_offset_frames                         */
   int32_t sink_offset_frames;  /* 3                                                      */
-  int32_t schedule;            /* LA_SCHED_PIPELINED | LA_SCHED_SEQUENTIAL               */
+  int32_t schedule;            /* LA_SCHED_PIPELINED | LA_SCHED_SEQUENTIAL | LA_SCHED_SLOT */
   int32_t dtype;               /* LA_BF16 | LA_FP32                                      */
   int32_t cache_mode;          /* LA_CACHE_TIMESTEP | LA_CACHE_CLEAN_REFRESH | LA_CACHE_FIXED_STEP */
   int32_t proj_fp8;            /* 1 (LA_BF16 only): the QKV and output projections run on
@@ -143,6 +148,7 @@ typedef struct la_config {
   int32_t audio_tokens;        /* LA_BLOCK_DIT: audio tokens A per block for the audio
                                   cross-attention (0: none; then la_denoise_step_av)     */
   int32_t audio_dim;           /* their feature width D_a (multiple of 8)               */
+  int32_t slot_index;          /* LA_SCHED_SLOT: the step this stream runs (0 .. num_steps-1) */
 } la_config;
 
 /* Layer kinds.  The pages give the model's base (a 14B DiT with timestep
@@ -242,6 +248,22 @@ int la_denoise_step_host(la_stream* s, const float* x_new_host, float* x_out_hos
  * la_denoise_step_host return LA_EINVAL for a new block of such a stream. */
 int la_denoise_step_av(la_stream* s, const float* x_new, const float* audio_new, float* x_out,
                        int64_t* finished_block);
+
+/* LA_SCHED_SLOT streams (one rank of the timestep pipeline; the papernotes
+ * note's TPP: each GPU pinned to one denoising step with its own cache, the
+ * latent passed on): each call runs step slot_index of the next block (ids
+ * 0, 1, ... in call order).  x_new (DEVICE fp32 [T_b, C], required) is the
+ * block's latent at timesteps[slot_index] (noise for slot 0, the previous
+ * rank's x_out otherwise); x_out receives it after the step and
+ * *finished_block the block's id.  Such a stream never replaces its sink on
+ * its own: with LA_SINK_AAS the caller calls la_replace_sink on every rank
+ * with frame 0 of block 0's finished latent (the last rank's output) before
+ * any rank runs a step of a later tick, which gives the single-GPU pipeline's
+ * timing (the new sink from tick num_steps on).
+ * la_replace_sink: sink_latent DEVICE fp32 [F * sink_frames, C]; reruns the
+ * sink pass and marks the sink generation 1.  LA_ESTATE for other schedules
+ * or a second replacement. */
+int la_replace_sink(la_stream* s, const float* sink_latent);
 
 /* Wait for all work of the stream; LA_EDEVICE if a kernel raised the device
  * error word (the word is cleared after being reported). */

@@ -30,7 +30,7 @@ class LaConfig(ctypes.Structure):
         ("sink_mode", c_int32), ("rolling_rope", c_int32), ("sink_offset_frames", c_int32),
         ("schedule", c_int32), ("dtype", c_int32), ("cache_mode", c_int32), ("proj_fp8", c_int32),
         ("attn_fp8", c_int32), ("cache_step", c_int32), ("block_kind", c_int32), ("ffn_dim", c_int32),
-        ("audio_tokens", c_int32), ("audio_dim", c_int32),
+        ("audio_tokens", c_int32), ("audio_dim", c_int32), ("slot_index", c_int32),
     ]
 
 
@@ -63,6 +63,7 @@ def load():
         "la_set_sink": (c_int, [c_void_p, c_void_p]),
         "la_denoise_step": (c_int, [c_void_p, c_void_p, c_void_p, POINTER(c_int64)]),
         "la_denoise_step_av": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(c_int64)]),
+        "la_replace_sink": (c_int, [c_void_p, c_void_p]),
         "la_denoise_step_host": (c_int, [c_void_p, c_void_p, c_void_p, POINTER(c_int64)]),
         "la_synchronize": (c_int, [c_void_p]),
         "la_stream_destroy": (c_int, [c_void_p]),
@@ -103,6 +104,7 @@ def exported_symbols():
     """Names of the C-ABI functions declared in include/la_stream.h."""
     return [
         "la_stream_create", "la_set_sink", "la_denoise_step", "la_denoise_step_host", "la_denoise_step_av",
+        "la_replace_sink",
         "la_synchronize",
         "la_stream_destroy", "la_last_error", "la_status_string", "la_index_state_size", "la_get_index_state",
         "la_debug_capture", "la_debug_tap", "la_debug_set_slot_input", "la_profile_enable", "la_profile_read",

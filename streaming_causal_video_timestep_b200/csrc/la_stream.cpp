@@ -31,6 +31,7 @@ struct SlotRecord {
 
 struct Scheduler {
   int S = 0, E = 0, W = 0, fpb = 0, offset = 0, rolling = 1, pipelined = 1, aas = 0, clean = 0;
+  int slot_only = -1;       // LA_SCHED_SLOT: the one step this stream runs
   int fixed_step = -1;      // LA_CACHE_FIXED_STEP: the step whose cache every step reads the window from
   long long tick = -1, blocks_in = 0, blocks_out = 0;
   int sink_gen = 0;
@@ -47,7 +48,8 @@ struct Scheduler {
     offset = c.sink_offset_frames;
     rolling = c.rolling_rope;
     pipelined = c.schedule == LA_SCHED_PIPELINED;
-    aas = c.sink_mode == LA_SINK_AAS;
+    slot_only = c.schedule == LA_SCHED_SLOT ? c.slot_index : -1;
+    aas = c.sink_mode == LA_SINK_AAS && slot_only < 0;   // a slot stream's sink is replaced by the caller
     clean = c.cache_mode == LA_CACHE_CLEAN_REFRESH;
     fixed_step = c.cache_mode == LA_CACHE_FIXED_STEP ? c.cache_step : -1;
     held.assign(S, -1);
@@ -73,6 +75,10 @@ struct Scheduler {
       for (int i = 0; i < S; ++i)
         if (next_held[i] >= 0) run.emplace_back(i, next_held[i]);
       finished = next_held[S - 1];
+    } else if (slot_only >= 0) {
+      next_held.assign(S, -1);
+      run.emplace_back(slot_only, blocks_in);
+      finished = blocks_in;
     } else {
       next_held.assign(S, -1);
       for (int i = 0; i < S; ++i) run.emplace_back(i, blocks_in);
@@ -359,7 +365,14 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
   if (c->rope_split[0] > LA_MAX_PT) { msg = "too many temporal rotary pairs"; return LA_EINVAL; }
   if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) { msg = "rope_theta must be positive"; return LA_EINVAL; }
   if (c->sink_mode != LA_SINK_FIXED && c->sink_mode != LA_SINK_AAS) { msg = "bad sink_mode"; return LA_EINVAL; }
-  if (c->schedule != LA_SCHED_PIPELINED && c->schedule != LA_SCHED_SEQUENTIAL) { msg = "bad schedule"; return LA_EINVAL; }
+  if (c->schedule != LA_SCHED_PIPELINED && c->schedule != LA_SCHED_SEQUENTIAL && c->schedule != LA_SCHED_SLOT) {
+    msg = "bad schedule";
+    return LA_EINVAL;
+  }
+  if (c->schedule == LA_SCHED_SLOT) {
+    if (c->slot_index < 0 || c->slot_index >= c->num_steps) { msg = "slot_index must name one of the steps"; return LA_EINVAL; }
+    if (c->cache_mode != LA_CACHE_TIMESTEP) { msg = "a slot stream keeps its own step's cache (timestep forcing)"; return LA_EINVAL; }
+  }
   if (c->cache_mode != LA_CACHE_TIMESTEP && c->cache_mode != LA_CACHE_CLEAN_REFRESH &&
       c->cache_mode != LA_CACHE_FIXED_STEP) {
     msg = "bad cache_mode";
@@ -1373,6 +1386,20 @@ int la_set_sink(la_stream* s, const float* sink_latent) {
   int r = run_sink(s);
   if (r != LA_OK) return r;
   s->sink_set = true;
+  return LA_OK;
+}
+
+int la_replace_sink(la_stream* s, const float* sink_latent) {
+  if (!s) return LA_EINVAL;
+  if (!sink_latent) return fail(s, LA_EINVAL, "NULL sink latent");
+  if (s->cfg.schedule != LA_SCHED_SLOT)
+    return fail(s, LA_ESTATE, "la_replace_sink is for slot streams (the others replace the sink themselves)");
+  if (!s->sink_set) return fail(s, LA_ESTATE, "la_set_sink must be called first");
+  if (s->sched.sink_gen != 0) return fail(s, LA_ESTATE, "the sink is replaced once");
+  CU(cudaMemcpyAsync(s->sink_x, sink_latent, static_cast<size_t>(s->F) * s->C * 4, cudaMemcpyDeviceToDevice, s->st));
+  int r = run_sink(s);
+  if (r != LA_OK) return r;
+  s->sched.sink_gen = 1;
   return LA_OK;
 }
 

@@ -78,6 +78,7 @@ class LaStream:
         c.ffn_dim = getattr(cfg, "ffn_dim", 0)
         c.audio_tokens = getattr(cfg, "audio_tokens", 0)
         c.audio_dim = getattr(cfg, "audio_dim", 0)
+        c.slot_index = getattr(cfg, "slot_index", 0)
         self.cfg = cfg
         self.c = c
         self.T = cfg.frames_per_block * cfg.grid_h * cfg.grid_w
@@ -163,6 +164,12 @@ class LaStream:
         fin = c_int64(-1)
         self._check(self.lib.la_denoise_step_host(self.h, _ptr(x_new_host), _ptr(x_out_host), ctypes.byref(fin)))
         return fin.value
+
+    def replace_sink(self, latent):
+        """Slot streams (one rank of the timestep pipeline): replace the sink with frame 0
+        of block 0's finished latent (device fp32 [F * sink_frames, C])."""
+        _require(latent, torch.float32, (self.F * self.cfg.sink_frames, self.C), "sink latent")
+        self._check(self.lib.la_replace_sink(self.h, _ptr(latent)))
 
     def synchronize(self):
         self._check(self.lib.la_synchronize(self.h))

@@ -94,6 +94,8 @@ def _weights(nonnull=True):
     dict(cache_mode=2, schedule=0),                   # the fixed-noise cache is sequential only
     dict(cache_mode=2, schedule=1, cache_step=4),     # cache_step names a step
     dict(cache_mode=3),
+    dict(schedule=2, slot_index=4),                   # slot_index names a step
+    dict(schedule=2, slot_index=0, cache_mode=1),     # a slot stream keeps its own step's cache
     dict(attn_fp8=2, dtype=0, head_dim=128, hidden=128, latent_ch=128, rope_split=(22, 21, 21)),
 ])
 def test_invalid_config_returns_einval(lib, over):

@@ -44,7 +44,7 @@ def _rank_main(rank, world, port, elapsed, out):
 def test_two_gloo_ranks_agree_on_the_slowest_rank_and_the_job_value():
     world, port = 2, _free_port()
     elapsed = [0.25, 0.4]                 # rank 1 is the slow one
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, port, elapsed, out), nprocs=world, join=True)
     assert out[0] == out[1]               # every rank computes the same job figure
     seconds, value = out[0]

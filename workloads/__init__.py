@@ -25,6 +25,7 @@ SINK_FIXED = 0
 SINK_AAS = 1
 SCHED_PIPELINED = 0
 SCHED_SEQUENTIAL = 1
+SCHED_SLOT = 2             # one rank of the timestep pipeline across GPUs: step slot_index of each block
 DTYPE_BF16 = 0
 DTYPE_FP32 = 1
 CACHE_TIMESTEP = 0         # noisy K/V of each step in that step's own cache (timestep forcing)
@@ -70,6 +71,7 @@ class StreamConfig:
     ffn_dim: int = 0         # BLOCK_DIT: hidden width of the FFN
     audio_tokens: int = 0    # BLOCK_DIT: audio tokens per block for the cross-attention (0: none)
     audio_dim: int = 0       # their feature width
+    slot_index: int = 0      # SCHED_SLOT: the step this rank runs
 
     @property
     def num_steps(self) -> int:
