@@ -10,6 +10,9 @@
 //               per k-block (32 bytes of K each);
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //               32*(w%4) .. +31 = tile rows), fused epilogue, global stores.
+//               The residual epilogues move each 32 x 32 chunk of the fp32
+//               residual through a per-warp shared-memory stage, so that the
+//               global loads and stores cover whole 128-byte row segments.
 // The two accumulators let the epilogue of tile n overlap the main loop of n+1.
 // Tiles are visited in bands of GROUP_M row-blocks so the A band and the W
 // tiles in flight stay L2-resident.
@@ -24,6 +27,10 @@ constexpr int BM = 128;
 constexpr int BK_BYTES = 128;   // K bytes per k-block: one 128-byte swizzle row
 constexpr int GROUP_M = 16;
 
+// Per epilogue warp: a 32 x 32 fp32 chunk (4 KB) and its bf16 copy (2 KB).
+constexpr uint32_t EPI_F32_BYTES = 32 * 32 * 4;
+constexpr uint32_t EPI_WARP_BYTES = EPI_F32_BYTES + 32 * 32 * 2;
+
 template <int BN>
 struct GemmCfg {
   static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
@@ -31,7 +38,8 @@ struct GemmCfg {
   static constexpr uint32_t B_BYTES = BN * BK_BYTES;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
-  static constexpr size_t SMEM = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
+  static constexpr size_t SMEM = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/ + 4 * EPI_WARP_BYTES;
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
@@ -126,6 +134,88 @@ __device__ __forceinline__ void qkv_rope_row32(const QkvRopeParams& qp, long lon
           tok;
   }
   store_bf16x32(dst, acc);
+}
+
+// h32 (+)= [gate *] acc for the 32 rows row0 .. row0+31 of one epilogue warp and
+// the 32 columns col .. col+31 (all in range), plus the bf16 copy to ep.out.
+// Lane t holds row t's values in acc.  The chunk passes through the warp's
+// shared-memory stage: loaded and stored by lanes 8 to a 128-byte row segment
+// (bf16: 4 to a 64-byte segment), combined by lanes one row each.  16-byte
+// slots in the stage are XOR-swizzled by row, so neither access pattern has
+// bank conflicts beyond the 4 wavefronts that 512 bytes take.
+template <bool GATED>
+__device__ __forceinline__ void epilogue_resid_warp(const GemmEpiParams& ep, long long row0, long long col,
+                                                   float (&acc)[32], uint8_t* stage, int lane) {
+  float4* sf = reinterpret_cast<float4*>(stage);
+  uint4* sb = reinterpret_cast<uint4*>(stage + EPI_F32_BYTES);
+  const int sub = lane >> 3, ch = lane & 7;
+  float4 gvs[8];
+  if (GATED) {
+    const float4* g4 = reinterpret_cast<const float4*>(ep.gate[(row0 + lane) / ep.rows_per_group] + col);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) gvs[i] = __ldg(g4 + i);
+  }
+  float4 hv[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = 4 * k + sub;
+    hv[k] = *reinterpret_cast<const float4*>(ep.h32 + (row0 + r) * ep.ld + col + 4 * ch);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = 4 * k + sub;
+    sf[r * 8 + (ch ^ (r & 7))] = hv[k];
+  }
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float4& slot = sf[lane * 8 + (c ^ (lane & 7))];
+    float4 h = slot;
+    if (GATED) {
+      h.x = fmaf(gvs[c].x, acc[4 * c + 0], h.x);
+      h.y = fmaf(gvs[c].y, acc[4 * c + 1], h.y);
+      h.z = fmaf(gvs[c].z, acc[4 * c + 2], h.z);
+      h.w = fmaf(gvs[c].w, acc[4 * c + 3], h.w);
+    } else {
+      h.x += acc[4 * c + 0];
+      h.y += acc[4 * c + 1];
+      h.z += acc[4 * c + 2];
+      h.w += acc[4 * c + 3];
+    }
+    slot = h;
+    acc[4 * c + 0] = h.x;
+    acc[4 * c + 1] = h.y;
+    acc[4 * c + 2] = h.z;
+    acc[4 * c + 3] = h.w;
+  }
+  if (ep.out) {
+    const int sw = (lane >> 1) & 3;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint4 w;
+      w.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
+      w.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
+      w.z = pack_bf16x2(acc[8 * c + 4], acc[8 * c + 5]);
+      w.w = pack_bf16x2(acc[8 * c + 6], acc[8 * c + 7]);
+      sb[lane * 4 + (c ^ sw)] = w;
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = 4 * k + sub;
+    *reinterpret_cast<float4*>(ep.h32 + (row0 + r) * ep.ld + col + 4 * ch) = sf[r * 8 + (ch ^ (r & 7))];
+  }
+  if (ep.out) {
+    const int sub2 = lane >> 2, c2 = lane & 3;
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(ep.out);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int r = 8 * k + sub2;
+      *reinterpret_cast<uint4*>(out + (row0 + r) * ep.ld + col + 8 * c2) = sb[r * 4 + (c2 ^ ((r >> 1) & 3))];
+    }
+  }
+  __syncwarp();   // the next chunk rewrites the stage
 }
 
 __device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, const QkvRopeParams& qp, long long row,
@@ -339,6 +429,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   } else {
     const int quarter = warp & 3;
     const int rit = quarter * 32 + lane;
+    uint8_t* epi_stage = smem + C::STAGES * C::STAGE_BYTES + 256 + (warp - 2) * EPI_WARP_BYTES;
+    // the residual kinds take the staged path when the warp's 32 rows are all in
+    // range and h32 / out rows start on 16-byte boundaries
+    const bool staged_kind = (ep.kind == EPI_RESID || ep.kind == EPI_RESID_GATED) && (ep.ld % 8) == 0 &&
+                             (reinterpret_cast<uintptr_t>(ep.h32) & 15) == 0 &&
+                             (reinterpret_cast<uintptr_t>(ep.out) & 15) == 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -348,6 +444,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       if (!mbar_wait(&tfull[acc], acc_phase, err)) { abort_flag = 1; break; }
       tc_fence_after();
       const long long row = static_cast<long long>(mb) * BM + rit;
+      const long long row0 = static_cast<long long>(mb) * BM + quarter * 32;
+      const bool staged = staged_kind && row0 + 32 <= M;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -355,7 +453,20 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         tmem_ld32(tbase + c0, r);
         tmem_ld_wait();
         const long long col = static_cast<long long>(nb) * BN + c0;
-        if (row < M && col < N) {
+        if (staged && col + 32 <= N) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          if (ep.row_scale) {
+            const float rs = ep.row_scale[row];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= rs * ep.col_scale[col + i];
+          }
+          if (ep.kind == EPI_RESID_GATED)
+            epilogue_resid_warp<true>(ep, row0, col, v, epi_stage, lane);
+          else
+            epilogue_resid_warp<false>(ep, row0, col, v, epi_stage, lane);
+        } else if (row < M && col < N) {
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);

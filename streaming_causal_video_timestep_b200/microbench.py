@@ -2,6 +2,7 @@
 
     python -m streaming_causal_video_timestep_b200.microbench attn  [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench gemm  [--iters N]
+    python -m streaming_causal_video_timestep_b200.microbench gemm_out [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench euler [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench rerope [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench gemm_fp8 [--iters N]
@@ -12,6 +13,8 @@ attn : one block's attention in steady state at the 14B-like shape: 4680
        = 15,600 keys (the per-slot launch of the stream), q pre-scaled.
 attn_fp8: the same attention on e4m3 q/K/V (per-head scales, e4m3 P).
 gemm : the QKV projection of one block, [4680, 5120] x [15360, 5120]^T.
+gemm_out: the output projection of the 4-slot grouped launch, [18720, 5120] x
+       [5120, 5120]^T, with the residual epilogue and with a plain bf16 store.
 euler: x += dt * v over 2^20 rows x 64 fp32 (256 MB per tensor), 4 groups.
 gemm_fp8: the QKV projection shape on e4m3 operands (kind::f8f6f4, per-row
        scales, bf16 output), and the per-row quantization of its activation.
@@ -90,6 +93,25 @@ def bench_gemm(iters):
             "flops": flops}
 
 
+def bench_gemm_out(iters):
+    """The output projection of the grouped 4-slot stream (M = 4 x 4680), with the
+    residual epilogue it runs with there (h32 += A W^T, plus the bf16 copy) and,
+    for comparison, with a plain bf16 store."""
+    M, N, K = 4 * 4680, 5120, 5120
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    A = torch.randn(M, K, generator=g, device="cuda").to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    h32 = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    flops = 2.0 * M * N * K
+    res = {"mode": "gemm_out", "shape": f"{M}x{N}x{K}", "flops": flops}
+    for epi in ("store", "resid"):
+        ms = _time(lambda: op_gemm(A, W, epi, out=out, h32=h32 if epi == "resid" else None), iters)
+        res[epi] = {"ms": round(ms, 4), "tflops": round(flops / ms / 1e9, 1)}
+    return res
+
+
 def bench_gemm_fp8(iters):
     M, N, K = 4680, 15360, 5120
     g = torch.Generator(device="cuda")
@@ -156,13 +178,13 @@ def bench_rerope(iters):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("mode", choices=["attn", "attn_fp8", "gemm", "euler", "rerope", "gemm_fp8", "all"])
+    ap.add_argument("mode", choices=["attn", "attn_fp8", "gemm", "gemm_out", "euler", "rerope", "gemm_fp8", "all"])
     ap.add_argument("--iters", type=int, default=10)
     args = ap.parse_args()
-    modes = ["attn", "attn_fp8", "gemm", "gemm_fp8", "euler", "rerope"] if args.mode == "all" else [args.mode]
+    modes = ["attn", "attn_fp8", "gemm", "gemm_out", "gemm_fp8", "euler", "rerope"] if args.mode == "all" else [args.mode]
     for m in modes:
-        r = {"attn": bench_attn, "attn_fp8": bench_attn_fp8, "gemm": bench_gemm, "euler": bench_euler, "rerope": bench_rerope,
-             "gemm_fp8": bench_gemm_fp8}[m](args.iters)
+        r = {"attn": bench_attn, "attn_fp8": bench_attn_fp8, "gemm": bench_gemm, "gemm_out": bench_gemm_out,
+             "euler": bench_euler, "rerope": bench_rerope, "gemm_fp8": bench_gemm_fp8}[m](args.iters)
         print(json.dumps(r), flush=True)
 
 
