@@ -208,22 +208,34 @@ def run_gpu(args, rank, world, local_rank):
     if dist:
         tdist.barrier()
 
-    # end to end through the public host-buffer call: H2D of the new block and
-    # D2H of the finished block inside the timed region, waited every tick
+    # end to end through the public host-buffer call: every tick copies its new
+    # block from pinned host memory and its finished block back to pinned host
+    # memory inside the timed region.  Two output buffers: the host enqueues tick
+    # i, then waits for tick i - 1 and reads its block, so host work overlaps
+    # the GPU the way a streaming server runs.
     xh = [torch.randn((T, C)).pin_memory() for _ in range(2)]
-    oh = torch.empty((T, C)).pin_memory()
+    oh = [torch.empty((T, C)).pin_memory() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
     for _ in range(2):
-        s.step_host(xh[0], oh)
+        s.step_host(xh[0], oh[0])
     s.synchronize()
     if dist:
         tdist.barrier()
     e2e_steps = max(3, min(args.steps, 10))
+    read_back = 0.0
     t0 = time.perf_counter()
     for i in range(e2e_steps):
-        fin = s.step_host(xh[i % 2], oh)
-        s.synchronize()
+        fin = s.step_host(xh[i % 2], oh[i % 2])
+        done[i % 2].record(s.stream)
         assert fin >= 0
+        if i > 0:
+            done[(i - 1) % 2].synchronize()
+            read_back += float(oh[(i - 1) % 2][0, 0])
+    done[(e2e_steps - 1) % 2].synchronize()
+    read_back += float(oh[(e2e_steps - 1) % 2][0, 0])
+    s.synchronize()
     e2e_s = time.perf_counter() - t0
+    assert read_back == read_back, "NaN in the latents read back"
     e2e_s = max_over_ranks(e2e_s, "cuda")
     # drain: S - 1 ticks without new blocks finish the blocks still in flight
     dr = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
