@@ -65,35 +65,54 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
   }
 }
 
+// Where one token (row) of the grouped QKV projection goes: its buffer, index in
+// the block, frame and grid position.  Computed once per tile for each lane's
+// row; the 32-column chunks of the row reuse it.
+struct QkvRow {
+  int buf, n, f, rr, ccol;
+  bool active;
+};
+
+__device__ __forceinline__ QkvRow qkv_row_info(const QkvRopeParams& qp, long long row) {
+  QkvRow q;
+  const int r32 = static_cast<int>(row);   // rows of one grouped launch fit in int
+  q.buf = r32 / qp.T;
+  q.n = r32 - q.buf * qp.T;
+  q.active = qp.active[q.buf] != 0;
+  q.f = q.n / qp.F;
+  const int rem = q.n - q.f * qp.F;
+  q.rr = rem / qp.grid_w;
+  q.ccol = rem - q.rr * qp.grid_w;
+  return q;
+}
+
 // 32 consecutive columns of one head of the [q | k | v] projection of one token:
-// rotate the pairs of q and k, scale q by log2(e)/sqrt(d), then write bf16 to
+// rotate the pairs of q and k, scale q by log2(e)/sqrt(d), then pack bf16 for
 // q_rope / the ring entry (or, with qp.fp8_inv, e4m3 codes of the unscaled
-// values over the head's scale).
-__device__ __forceinline__ void qkv_rope_row32(const QkvRopeParams& qp, long long row, long long col,
-                                               float (&acc)[32]) {
-  const int buf = static_cast<int>(row / qp.T);
-  const int n = static_cast<int>(row - static_cast<long long>(buf) * qp.T);
-  if (!qp.active[buf]) return;
-  const int part = static_cast<int>(col / qp.D);
-  const int cc = static_cast<int>(col - static_cast<long long>(part) * qp.D);
+// values over the head's scale).  Returns the destination of the packed words
+// (64 bytes of bf16 or 32 of e4m3), nullptr when the row's buffer is inactive.
+__device__ __forceinline__ void* qkv_rope_words(const QkvRopeParams& qp, const QkvRow& qr, long long col,
+                                                float (&acc)[32], uint32_t (&w)[16]) {
+  if (!qr.active) return nullptr;
+  const int c32 = static_cast<int>(col);
+  const int part = c32 / qp.D;
+  const int cc = c32 - part * qp.D;
   const int h = cc / qp.d, e0 = cc - h * qp.d;
   if (part < 2) {
-    const int f = n / qp.F, rem = n - f * qp.F;
-    const int rr = rem / qp.grid_w, ccol = rem - rr * qp.grid_w;
     const int pw_base = qp.pt + qp.ph;
 #pragma unroll
     for (int jj = 0; jj < 16; ++jj) {
       const int j = (e0 >> 1) + jj;
       float c, sn;
       if (j < qp.pt) {
-        const int idx = (buf * LA_TROWS + f) * LA_MAX_PT + j;
+        const int idx = (qr.buf * LA_TROWS + qr.f) * LA_MAX_PT + j;
         c = qp.tcos[idx]; sn = qp.tsin[idx];
       } else if (j < pw_base) {
-        const int idx = rr * qp.ph + (j - qp.pt);
+        const int idx = qr.rr * qp.ph + (j - qp.pt);
         c = qp.rcos[idx]; sn = qp.rsin[idx];
       } else {
         const int pw = qp.d / 2 - pw_base;
-        const int idx = ccol * pw + (j - pw_base);
+        const int idx = qr.ccol * pw + (j - pw_base);
         c = qp.ccos[idx]; sn = qp.csin[idx];
       }
       const float x0 = acc[2 * jj], x1 = acc[2 * jj + 1];
@@ -101,39 +120,80 @@ __device__ __forceinline__ void qkv_rope_row32(const QkvRopeParams& qp, long lon
       acc[2 * jj + 1] = x0 * sn + x1 * c;
     }
   }
-  const long long tok = static_cast<long long>(n) * qp.d + e0;
+  const long long tok = static_cast<long long>(qr.n) * qp.d + e0;
+  long long base;
+  if (part == 0) {
+    base = (static_cast<long long>(qr.buf) * qp.H + h) * qp.T * qp.d;
+  } else {
+    const long long slice = qp.ring_slice0 + static_cast<long long>(qp.slot[qr.buf]) * qp.E + qp.write_entry[qr.buf];
+    base = (slice * qp.H + h) * qp.T * qp.d;
+  }
+  void* plane = part == 0 ? qp.q_rope : (part == 1 ? qp.ring_k : qp.ring_v);
   if (qp.fp8_inv) {
     // e4m3 attention operands: codes of value / (the head's power-of-two scale)
     const float inv = qp.fp8_inv[part * qp.H + h];
-    long long base;
-    if (part == 0) {
-      base = (static_cast<long long>(buf) * qp.H + h) * qp.T * qp.d;
-    } else {
-      const long long slice = qp.ring_slice0 + static_cast<long long>(qp.slot[buf]) * qp.E + qp.write_entry[buf];
-      base = (slice * qp.H + h) * qp.T * qp.d;
-    }
-    uint8_t* dst8 = static_cast<uint8_t*>(part == 0 ? qp.q_rope : (part == 1 ? qp.ring_k : qp.ring_v)) + base + tok;
-    uint32_t wv[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      wv[k] = pack_e4m3x4(make_float2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
-                          make_float2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
-    uint4* d4 = reinterpret_cast<uint4*>(dst8);
-    d4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-    d4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-    return;
+      w[k] = pack_e4m3x4(make_float2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
+                         make_float2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
+    return static_cast<uint8_t*>(plane) + base + tok;
   }
-  __nv_bfloat16* dst;
   if (part == 0) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] *= qp.qscale;
-    dst = reinterpret_cast<__nv_bfloat16*>(qp.q_rope) + (static_cast<long long>(buf) * qp.H + h) * qp.T * qp.d + tok;
-  } else {
-    const long long slice = qp.ring_slice0 + static_cast<long long>(qp.slot[buf]) * qp.E + qp.write_entry[buf];
-    dst = reinterpret_cast<__nv_bfloat16*>(part == 1 ? qp.ring_k : qp.ring_v) + (slice * qp.H + h) * qp.T * qp.d +
-          tok;
   }
-  store_bf16x32(dst, acc);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+  return static_cast<__nv_bfloat16*>(plane) + base + tok;
+}
+
+// One row segment of WORDS 32-bit words per lane (16: 64 bytes, 8: 32 bytes) to
+// dst (16-byte aligned; nullptr: this lane's row stores nothing).
+__device__ __forceinline__ void store_row_words_direct(void* dst, const uint32_t* w, int words) {
+  if (!dst) return;
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  for (int q = 0; q < words / 4; ++q) d4[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+}
+
+// The same for the whole warp through its shared-memory stage: lane t holds row
+// t's words; the segments go out Q = WORDS / 4 lanes to a row (16 bytes each), so
+// one store instruction covers 32 / Q rows with whole 32-byte sectors.  Each
+// row's destination comes from its owner lane by shuffle.  The 16-byte slots are
+// XOR-swizzled by row, so neither the row-wise writes nor the lane-group reads
+// conflict on banks.
+template <int WORDS>
+__device__ __forceinline__ void store_row_words_staged(void* dst, const uint32_t* w, uint8_t* stage, int lane) {
+  constexpr int Q = WORDS / 4;
+  static_assert(Q == 4 || Q == 2, "64- or 32-byte row segments");
+  uint4* sq = reinterpret_cast<uint4*>(stage);
+  auto swz = [](int r) { return Q == 4 ? ((r >> 1) & 3) : ((r >> 2) & 1); };
+  const int sw = swz(lane);
+#pragma unroll
+  for (int q = 0; q < Q; ++q) sq[lane * Q + (q ^ sw)] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  __syncwarp();
+  const unsigned long long d = reinterpret_cast<unsigned long long>(dst);
+#pragma unroll
+  for (int k = 0; k < Q; ++k) {
+    const int r = k * (32 / Q) + lane / Q, q = lane % Q;
+    const unsigned long long dr = __shfl_sync(0xffffffffu, d, r);
+    if (dr) *reinterpret_cast<uint4*>(dr + 16ull * q) = sq[r * Q + (q ^ swz(r))];
+  }
+  __syncwarp();   // the next chunk rewrites the stage
+}
+
+// The epilogues that end in one packed row segment a row (bf16 store, GELU, the
+// QKV RoPE/append): the destination and words of this lane's row, nullptr when
+// it stores nothing.
+__device__ __forceinline__ void* segment_words(const GemmEpiParams& ep, const QkvRopeParams& qp, const QkvRow& qr,
+                                               long long row, long long col, float (&acc)[32], uint32_t (&w)[16]) {
+  if (ep.kind == EPI_QKV_ROPE) return qkv_rope_words(qp, qr, col, acc, w);
+  if (ep.kind == EPI_GELU) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = gelu_tanh(acc[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+  return reinterpret_cast<__nv_bfloat16*>(ep.out) + row * ep.ld + col;
 }
 
 // h32 (+)= [gate *] acc for the 32 rows row0 .. row0+31 of one epilogue warp and
@@ -218,22 +278,18 @@ __device__ __forceinline__ void epilogue_resid_warp(const GemmEpiParams& ep, lon
   __syncwarp();   // the next chunk rewrites the stage
 }
 
-__device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, const QkvRopeParams& qp, long long row,
-                                               long long col, float (&acc)[32]) {
+// The remaining epilogues, one lane per row (residual kinds on partial warps,
+// fp32 stores, set, Euler update).
+__device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, long long row, long long col,
+                                               float (&acc)[32]) {
   const long long off = row * ep.ld + col;
   switch (ep.kind) {
-    case EPI_QKV_ROPE:
-      qkv_rope_row32(qp, row, col, acc);
-      break;
     case EPI_STORE32: {
       float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + off);
 #pragma unroll
       for (int i = 0; i < 8; ++i) o4[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
       break;
     }
-    case EPI_STORE:
-      store_bf16x32(reinterpret_cast<__nv_bfloat16*>(ep.out) + off, acc);
-      break;
     case EPI_RESID: {
       float4* h4 = reinterpret_cast<float4*>(ep.h32 + off);
 #pragma unroll
@@ -276,12 +332,6 @@ __device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, const Qk
         acc[4 * i + 3] = h.w;
       }
       if (ep.out) store_bf16x32(reinterpret_cast<__nv_bfloat16*>(ep.out) + off, acc);
-      break;
-    }
-    case EPI_GELU: {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = gelu_tanh(acc[i]);
-      store_bf16x32(reinterpret_cast<__nv_bfloat16*>(ep.out) + off, acc);
       break;
     }
     case EPI_SET32: {
@@ -435,6 +485,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const bool staged_kind = (ep.kind == EPI_RESID || ep.kind == EPI_RESID_GATED) && (ep.ld % 8) == 0 &&
                              (reinterpret_cast<uintptr_t>(ep.h32) & 15) == 0 &&
                              (reinterpret_cast<uintptr_t>(ep.out) & 15) == 0;
+    // the kinds that end in one packed segment a row (64 bytes of bf16, or 32 of
+    // e4m3 for the QKV epilogue of e4m3 attention) store through the stage
+    const bool segment_kind = ep.kind == EPI_STORE || ep.kind == EPI_GELU || ep.kind == EPI_QKV_ROPE;
+    const bool seg_e4m3 = ep.kind == EPI_QKV_ROPE && qp.fp8_inv != nullptr;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -446,6 +500,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       const long long row = static_cast<long long>(mb) * BM + rit;
       const long long row0 = static_cast<long long>(mb) * BM + quarter * 32;
       const bool staged = staged_kind && row0 + 32 <= M;
+      QkvRow qr{};
+      if (ep.kind == EPI_QKV_ROPE && row < M) qr = qkv_row_info(qp, row);
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -453,7 +509,25 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         tmem_ld32(tbase + c0, r);
         tmem_ld_wait();
         const long long col = static_cast<long long>(nb) * BN + c0;
-        if (staged && col + 32 <= N) {
+        if (segment_kind && col + 32 <= N) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          uint32_t w[16];
+          void* dst = nullptr;
+          if (row < M) {
+            if (ep.row_scale) {
+              const float rs = ep.row_scale[row];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] *= rs * ep.col_scale[col + i];
+            }
+            dst = segment_words(ep, qp, qr, row, col, v, w);
+          }
+          if (seg_e4m3)
+            store_row_words_staged<8>(dst, w, epi_stage, lane);
+          else
+            store_row_words_staged<16>(dst, w, epi_stage, lane);
+        } else if (staged && col + 32 <= N) {
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
@@ -475,7 +549,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] *= rs * ep.col_scale[col + i];
           }
-          epilogue_row32(ep, qp, row, col, v);
+          if (segment_kind) {
+            uint32_t w[16];
+            store_row_words_direct(segment_words(ep, qp, qr, row, col, v, w), w, seg_e4m3 ? 8 : 16);
+          } else {
+            epilogue_row32(ep, row, col, v);
+          }
         }
       }
       tc_fence_before();
