@@ -278,6 +278,29 @@ __device__ __forceinline__ void epilogue_resid_warp(const GemmEpiParams& ep, lon
   __syncwarp();   // the next chunk rewrites the stage
 }
 
+// e4m3 operands: acc *= row_scale[row] * col_scale[col + i].  The 32 column
+// scales of the chunk (the same for every lane) are read as 8 float4 through
+// the read-only path when the array is 16-byte aligned (col is a multiple of
+// 32), else one by one.
+__device__ __forceinline__ void apply_operand_scales(const GemmEpiParams& ep, long long row, long long col,
+                                                     float (&v)[32]) {
+  const float rs = ep.row_scale[row];
+  if ((reinterpret_cast<uintptr_t>(ep.col_scale) & 15) != 0) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= rs * ep.col_scale[col + i];
+    return;
+  }
+  const float4* c4 = reinterpret_cast<const float4*>(ep.col_scale + col);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 c = __ldg(c4 + q);
+    v[4 * q + 0] *= rs * c.x;
+    v[4 * q + 1] *= rs * c.y;
+    v[4 * q + 2] *= rs * c.z;
+    v[4 * q + 3] *= rs * c.w;
+  }
+}
+
 // The remaining epilogues, one lane per row (residual kinds on partial warps,
 // fp32 stores, set, Euler update).
 __device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, long long row, long long col,
@@ -517,9 +540,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           void* dst = nullptr;
           if (row < M) {
             if (ep.row_scale) {
-              const float rs = ep.row_scale[row];
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] *= rs * ep.col_scale[col + i];
+              apply_operand_scales(ep, row, col, v);
             }
             dst = segment_words(ep, qp, qr, row, col, v, w);
           }
@@ -532,9 +553,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
           if (ep.row_scale) {
-            const float rs = ep.row_scale[row];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= rs * ep.col_scale[col + i];
+            apply_operand_scales(ep, row, col, v);
           }
           if (ep.kind == EPI_RESID_GATED)
             epilogue_resid_warp<true>(ep, row0, col, v, epi_stage, lane);
@@ -545,9 +564,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
           if (ep.row_scale) {
-            const float rs = ep.row_scale[row];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= rs * ep.col_scale[col + i];
+            apply_operand_scales(ep, row, col, v);
           }
           if (segment_kind) {
             uint32_t w[16];
