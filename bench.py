@@ -70,6 +70,36 @@ def _attn_flops_per_slot(T, F, nw, H, d):
     return 4.0 * T * nk * d * H
 
 
+def kernel_entries(kinds, steps, L, S, T, D, C, F, attn_tflops, pk):
+    """Per-kernel-kind figures of the timed ticks: kinds maps a kind to (launches,
+    total ms) from the library's profiling counters.  Tensor-core kinds get
+    TFLOP/s and the fraction of the measured sustained bf16 peak; the sink
+    re-rope gets GB/s and the fraction of the measured HBM copy."""
+    gemm_flops = {"qkv_gemm": 2.0 * S * T * D * 3 * D, "out_gemm": 2.0 * S * T * D * D,
+                  "in_proj": 2.0 * S * T * C * D, "head": 2.0 * S * T * D * C}
+    kernels = {}
+    for kind, (n, tot) in kinds.items():
+        if n == 0:
+            continue
+        avg = tot / n
+        e = {"launches": n, "ms_avg": round(avg, 4), "ms_per_step": round(tot / steps, 3)}
+        if kind == "attn":
+            e["tflops"] = round(attn_tflops, 1)
+        elif kind == "rope":
+            # sink re-rope of every active slot: read the layer's fp32 un-roped sink K once,
+            # write S bf16 roped copies (the block's RoPE + append is fused into the QKV GEMM)
+            nbytes = F * D * 4 + S * F * D * 2
+            e["gbs"] = round(nbytes / (avg / 1000.0) / 1e9, 1)
+            e["frac_hbm"] = round(e["gbs"] / pk["hbm"], 3)
+            e["bytes_per_launch"] = nbytes
+        elif kind in gemm_flops and n >= steps * (L if kind in ("qkv_gemm", "out_gemm") else 1):
+            e["tflops"] = round(gemm_flops[kind] / (avg / 1000.0) / 1e12, 1)
+        if "tflops" in e:
+            e["frac_sustained"] = round(e["tflops"] / pk["tflops_sust"], 3)
+        kernels[kind] = e
+    return kernels
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -256,26 +286,7 @@ def run_gpu(args, rank, world, local_rank):
     attn_ms_avg = ms_attn / max(n_attn, 1)
     achieved = attn_flops_launch / (attn_ms_avg / 1000.0) / 1e12
     peak = pk["tflops_sust"]
-    gemm_flops = {"qkv_gemm": 2.0 * S * T * D * 3 * D, "out_gemm": 2.0 * S * T * D * D,
-                  "in_proj": 2.0 * S * T * C * D, "head": 2.0 * S * T * D * C}
-    kernels = {}
-    for kind, (n, tot) in kinds.items():
-        if n == 0:
-            continue
-        avg = tot / n
-        e = {"launches": n, "ms_avg": round(avg, 4), "ms_per_step": round(tot / args.steps, 3)}
-        if kind == "attn":
-            e["tflops"] = round(achieved, 1)
-        elif kind == "rope":
-            # sink re-rope of every active slot: read the layer's fp32 un-roped sink K once,
-            # write S bf16 roped copies (the block's RoPE + append is fused into the QKV GEMM)
-            nbytes = F * D * 4 + S * F * D * 2
-            e["gbs"] = round(nbytes / (avg / 1000.0) / 1e9, 1)
-            e["frac_hbm"] = round(e["gbs"] / pk["hbm"], 3)
-            e["bytes_per_launch"] = nbytes
-        elif kind in gemm_flops and n >= args.steps * (L if kind in ("qkv_gemm", "out_gemm") else 1):
-            e["tflops"] = round(gemm_flops[kind] / (avg / 1000.0) / 1e12, 1)
-        kernels[kind] = e
+    kernels = kernel_entries(kinds, args.steps, L, S, T, D, C, F, achieved, pk)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
