@@ -35,8 +35,10 @@ What it computes (Live Avatar, arXiv 2512.04677, as described on the pages):
     Wan-style block the model is built on; the pages give no internals).
 
 Everything is fp64 numpy with a dict-indexed cache, an explicit mask matrix and
-a naive softmax.  The readings taken where the pages are silent are listed in
-the design doc of this repository.
+a naive softmax.  Where the pages are silent, each module states the reading it
+takes in its own docstring (flow direction and timesteps in flow.py, the RoPE
+pair layout and the sink offset in rope.py, the ring layout and eviction in
+schedule.py, the FP8 scales in fp8.py, the block internals in dit.py).
 
 Pins (tests/test_oracle_*.py): brute force on tiny inputs, SDPA on the visible
 segments, softmax rows summing to 1, single-key passthrough, RoPE norm and
