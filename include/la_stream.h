@@ -89,7 +89,7 @@ extern "C" {
 
 #define LA_RMS_EPS 1e-6
 
-/* Limits of this build. */
+/* Compile-time limits of the library (larger configurations return LA_EINVAL). */
 #define LA_MAX_STEPS     8
 #define LA_MAX_WINDOW   14
 #define LA_MAX_FPB       7
