@@ -296,7 +296,7 @@ def run_gpu(args, rank, world, local_rank):
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": ATTN_DRAM_BYTES_PER_SLOT * S,
                      "traffic_unit": "bytes per launch (ncu dram read+write, one-slot capture x slots)",
-                     "peak_source": f"{pk['src']} bf16 sustained (fp16 dense rate = bf16 dense rate)",
+                     "peak_source": f"{pk['src']} bf16 sustained (the kernel's operands are bf16)",
                      "algorithmic_flops_per_launch": attn_flops_launch},
         "kernels": kernels,
         "gpu_launches": int(launches),

@@ -377,10 +377,31 @@ int64_t la_launch_count(const la_stream* s);
  */
 int la_debug_wait_timeout(int64_t limit_ns, int32_t complete, int32_t* device_error);
 
+/*
+ * The same check for the op-level entry points: enqueues on cuda_stream one
+ * CTA whose wait nothing completes, so that after limit_ns (0..1e10) it raises
+ * the op-level error word (see la_op_status) and returns.  Asynchronous;
+ * allocates nothing.  LA_OK, LA_EINVAL or LA_ECUDA.
+ */
+int la_debug_op_wait_timeout(int64_t limit_ns, void* cuda_stream);
+
 /* ---- op-level entry points (unit tests, microbenchmarks) ------------------
  * Each enqueues one kernel on cuda_stream (a cudaStream_t, NULL = default).
- * They allocate nothing except where stated.
+ * They allocate nothing except where stated.  Their tensor-core kernels wait
+ * on mbarriers with a limit, like the stream's; a wait that gives up raises a
+ * per-device op-level error word (a file-scope device int of the library,
+ * first error wins) and the kernel returns with its output unfinished.
  */
+
+/*
+ * Reports and clears the op-level error word of the current device:
+ * synchronises cuda_stream, then returns LA_EDEVICE (message on stderr) if a
+ * kernel of an la_op_* call raised the word since the last la_op_status on
+ * this device, else LA_OK; LA_ECUDA if the word cannot be read.  Allocates
+ * nothing.  The word is shared by every op-level call on the device, so an
+ * error raised by a call on another stream is reported here too.
+ */
+int la_op_status(void* cuda_stream);
 
 /*
  * C = A W^T with an epilogue.  A: DEVICE [M, K] row-major, W: DEVICE [N, K]
@@ -496,12 +517,19 @@ int la_op_attention_fp8(const void* q_codes, int64_t Tq, int32_t H, int32_t d, i
  * that array until the process exits.
  *   - Arguments as la_op_attention with dtype LA_BF16 (q, segments, out, out32),
  *     d == 128.  H*Tq*d must be <= LA_STATIC_Q_ELEMS, else LA_EINVAL with a
- *     message on stderr.
- *   - Calls nothing that allocates.  The first call on a device looks up the
- *     array's device address (cudaGetSymbolAddress, with that device current);
- *     make that first call before any stream capture.
+ *     message on stderr. *   - Calls no cudaMalloc, cudaFree or allocating library routine.  The first
+ *     call on a device (and the first after the device's context changed, as
+ *     after cudaDeviceReset) looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.  Under CUDA's default lazy module loading the
+ *     first call also loads the library's device code and so reserves the
+ *     array then: it can fail with LA_ECUDA if the device's memory is already
+ *     taken.  Callers with a fixed memory budget make one call (or set
+ *     CUDA_MODULE_LOADING=EAGER) before their allocator takes the budget.
  *   - All calls share the array and overwrite the part they use (nothing needs
  *     to start at zero); calls that overlap on the GPU race on it.
+ *   - A bounded wait that gives up in the kernel raises the op-level error
+ *     word: la_op_status reports it (LA_EDEVICE) and clears it.
  */
 #define LA_STATIC_Q_ELEMS (8LL * 1024 * 1024)
 int la_op_attention_static(const void* q, int64_t Tq, int32_t H, int32_t d, int32_t nseg,

@@ -85,6 +85,8 @@ def load():
         "la_op_attention_static": (c_int, [c_void_p, c_int64, c_int32, c_int32, c_int32, POINTER(c_void_p),
                                            POINTER(c_void_p), POINTER(c_int64), c_void_p, c_void_p, c_void_p]),
         "la_debug_wait_timeout": (c_int, [c_int64, c_int32, POINTER(c_int32)]),
+        "la_debug_op_wait_timeout": (c_int, [c_int64, c_void_p]),
+        "la_op_status": (c_int, [c_void_p]),
         "la_op_quantize_e4m3": (c_int, [c_int32, c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
         "la_op_gemm_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int64, c_int64,
                                    c_int64, c_void_p]),
@@ -110,6 +112,7 @@ def exported_symbols():
         "la_debug_capture", "la_debug_tap", "la_debug_set_slot_input", "la_profile_enable", "la_profile_read",
         "la_launch_count", "la_op_gemm", "la_op_attention", "la_op_euler", "la_op_attention_static",
         "la_debug_wait_timeout", "la_op_quantize_e4m3", "la_op_gemm_fp8", "la_op_attention_fp8",
+        "la_debug_op_wait_timeout", "la_op_status",
     ]
 
 

@@ -4,8 +4,10 @@
 // One CTA = up to 256 queries (two 128-row tiles A and B) of one (group, head),
 // sharing every K/V tile of the group's segments [sink | window | block].
 // 12 warps in three warpgroups:
-//   warpgroup 0  warp 0: TMA producer (Q_A, Q_B once, then K_t / V_t as two
-//                64-column 128-byte-swizzled boxes each, 5-stage ring);
+//   warpgroup 0  warp 0: TMA producer (Q_A, Q_B once, then one ring stage
+//                [V(p-1) | K(p)] per key-tile step p, each tile as two
+//                64-column 128-byte-swizzled boxes: a 2-stage ring for bf16,
+//                4 stages for e4m3, see kv_stages());
 //                warp 1: TMEM owner (512 columns: S_A | S_B | O_A | O_B) and
 //                MMA issuer; warps 2-3 idle.  Drops to 56 registers a thread.
 //   warpgroup 1  softmax of tile A, warpgroup 2 softmax of tile B: one thread

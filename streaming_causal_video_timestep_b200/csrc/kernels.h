@@ -6,6 +6,10 @@
 
 #include "common.cuh"
 
+// Device address of the op-level error word on the current device (la_static.cu;
+// read and cleared by la_op_status).  Returns LA_OK or LA_ECUDA.
+int op_error_word(int** out);
+
 // ---- tcgen05 (bf16) ----------------------------------------------------------------
 int gemm_tc_pick_bn(int N);
 // qp: parameters of the EPI_QKV_ROPE epilogue (NULL for the others).

@@ -1,8 +1,10 @@
-// la_debug_wait_timeout: exercises the failure path of every pipelined kernel
-// (a bounded mbarrier wait that gives up, raises the device error word and
-// returns) without faulting or hanging the GPU.
+// la_debug_wait_timeout / la_debug_op_wait_timeout: exercise the failure path
+// of every pipelined kernel (a bounded mbarrier wait that gives up, raises the
+// device error word and returns) without faulting or hanging the GPU; the
+// second raises the op-level error word that la_op_status reports.
 #include <cuda_runtime.h>
 
+#include "kernels.h"
 #include "la_stream.h"
 #include "sm100.cuh"
 
@@ -40,4 +42,13 @@ extern "C" int la_debug_wait_timeout(int64_t limit_ns, int32_t complete, int32_t
   if (code != LA_OK) return code;
   *device_error = h;
   return h ? LA_EDEVICE : LA_OK;
+}
+
+extern "C" int la_debug_op_wait_timeout(int64_t limit_ns, void* cuda_stream) {
+  if (limit_ns < 0 || limit_ns > 10000000000LL) return LA_EINVAL;
+  int* err = nullptr;
+  if (op_error_word(&err) != LA_OK) return LA_ECUDA;
+  k_wait_probe<<<1, 32, 0, static_cast<cudaStream_t>(cuda_stream)>>>(static_cast<unsigned long long>(limit_ns), 0,
+                                                                      err);
+  return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ECUDA;
 }

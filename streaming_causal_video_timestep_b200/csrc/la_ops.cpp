@@ -48,7 +48,9 @@ int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, vo
     const int bn = gemm_tc_pick_bn(static_cast<int>(N));
     CUtensorMap ta, tb;
     if (!tmap_2d_bf16(&ta, A, M, K, K, 128, err) || !tmap_2d_bf16(&tb, W, N, K, K, bn, err)) return LA_ECUDA;
-    return ret(launch_gemm_tc(ta, tb, ep, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), bn, nullptr,
+    int* dev_err = nullptr;
+    if (op_error_word(&dev_err) != LA_OK) return LA_ECUDA;
+    return ret(launch_gemm_tc(ta, tb, ep, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), bn, dev_err,
                               num_sms_current(), st));
   }
   if (dtype != LA_FP32) return LA_EINVAL;
@@ -73,7 +75,7 @@ int la_op_attention(int32_t dtype, const void* q, int64_t Tq, int32_t H, int32_t
   p.out32 = dtype == LA_BF16 ? out32 : nullptr;
   p.q_prescaled = (dtype == LA_BF16 && q_scaled) ? 1 : 0;
   p.out_ld = static_cast<long long>(H) * d;
-  p.err = nullptr;
+  if (op_error_word(&p.err) != LA_OK) return LA_ECUDA;
   p.qbase = q;
   AttnGroup& g = p.g[0];
   g.nseg = nseg;
@@ -124,6 +126,7 @@ int la_op_attention_fp8(const void* q_codes, int64_t Tq, int32_t H, int32_t d, i
   p.out = out;
   p.out32 = out32;
   p.out_ld = static_cast<long long>(H) * d;
+  if (op_error_word(&p.err) != LA_OK) return LA_ECUDA;
   AttnGroup& g = p.g[0];
   g.nseg = nseg;
   for (int s = 0; s < nseg; ++s) g.seg[s] = AttnSeg{s, s, 0, 0, static_cast<int>(seg_len[s])};
@@ -165,8 +168,10 @@ int la_op_gemm_fp8(const void* a_codes, const float* a_scales, const void* w_cod
   for (int i = 0; i < LA_MAX_STEPS; ++i) ep.active[i] = 1;
   ep.row_scale = a_scales;
   ep.col_scale = w_scales;
+  int* dev_err = nullptr;
+  if (op_error_word(&dev_err) != LA_OK) return LA_ECUDA;
   return ret(launch_gemm_tc_fp8(ta, tb, ep, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), bn,
-                                nullptr, num_sms_current(), static_cast<cudaStream_t>(cuda_stream)));
+                                dev_err, num_sms_current(), static_cast<cudaStream_t>(cuda_stream)));
 }
 
 int la_op_euler(float* x, const float* v, int64_t rows, int64_t C, const float* dt, int64_t rows_per_group,

@@ -66,6 +66,34 @@ def test_sublayer_at_14b_shape_one_slot():
     s.close()
 
 
+@pytest.mark.slow
+def test_sublayer_at_14b_shape_step_level_all_rows():
+    """Step-level parity at the full one-slot sublayer shape: the fp64 oracle runs
+    the whole step (norm, QKV, Rolling RoPE, ring append, attention over sink +
+    window + block, output projection, head, Euler) for blocks 0, 1 and 2 from
+    the same noise, and every row of every finished block matches it at the bf16
+    tolerance (block 2 in steady state: 15,600 keys a query)."""
+    from oracle import OracleStream
+    from _helpers import assert_close
+    from workloads import DTYPE_BF16
+    wl = SUBLAYER
+    cfg = wl.cfg
+    s, W = make_stream(wl)
+    orc = OracleStream(cfg, W)
+    orc.set_sink(W.sink)
+    x_out = torch.empty((cfg.block_tokens, cfg.latent_ch), device="cuda")
+    for b in range(wl.num_blocks):
+        xn = block_noise(wl, b)
+        fin = s.step(_dev(xn), x_out)
+        ref, fin_o = orc.denoise_step(xn)
+        assert fin == fin_o == b
+        np.testing.assert_array_equal(s.index_state(), orc.index_state())
+        e = assert_close(to_np(x_out), ref, DTYPE_BF16, f"sublayer block {b} (step-level, all rows)")
+        print(f"block {b}: max rel {e[0]:.2e}, mean rel {e[1]:.2e}")
+    s.synchronize()
+    s.close()
+
+
 def test_eight_layer_stream_four_slots_grouped():
     """The benchmarked workload: 4 slots x 8 sublayers per grouped launch, head
     5120 -> 64, AAS.  Per-op checks at the AAS tick, in steady state and in the drain."""

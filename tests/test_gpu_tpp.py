@@ -3,14 +3,18 @@ stream per denoising step (rank), chained by the same TppRank code that runs the
 ranks over torch.distributed (streaming_causal_video_timestep_b200/tpp.py), against
 the grouped single-GPU stream.  Each rank's step runs the same kernels on the same
 rows as the grouped launch, so the finished blocks are equal bit for bit, with the
-Adaptive Attention Sink swapped on every rank by the broadcast from the last rank."""
+Adaptive Attention Sink swapped on every rank by the broadcast from the last rank.
+The fp32 chains are also checked against the fp64 oracle's pipelined stream
+within 1e-5, free-running."""
 import numpy as np
 import pytest
 
-from workloads import BLOCK_DIT, DTYPE_BF16, SCHED_SLOT, SINK_AAS, SINK_FIXED, TINY, StreamConfig, Workload, \
+from workloads import BLOCK_DIT, DTYPE_BF16, DTYPE_FP32, SCHED_SLOT, SINK_AAS, SINK_FIXED, TINY, StreamConfig, Workload, \
     block_audio, block_noise, make_weights
 
-from _helpers import make_stream
+from oracle import OracleStream
+
+from _helpers import assert_close, make_stream
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -80,6 +84,19 @@ def test_tpp_ranks_on_one_gpu_equal_the_grouped_stream(wl):
     assert sorted(got) == list(range(wl.num_blocks))
     for b in range(wl.num_blocks):
         np.testing.assert_array_equal(got[b].cpu().numpy(), want[b])
+    if cfg.dtype == DTYPE_FP32:
+        # and against the fp64 oracle's single-process pipelined stream, free-running,
+        # within the fp32 tolerance (no teacher forcing: the whole trajectory)
+        orc = OracleStream(cfg, W)
+        orc.set_sink(W.sink)
+        ref = {}
+        for k in range(wl.num_blocks + S - 1):
+            out, fin = orc.denoise_step(block_noise(wl, k) if k < wl.num_blocks else None)
+            if fin >= 0:
+                ref[fin] = out
+        assert sorted(ref) == list(range(wl.num_blocks))
+        for b in range(wl.num_blocks):
+            assert_close(got[b].cpu().numpy(), ref[b], DTYPE_FP32, f"TPP rank chain, block {b}")
 
 
 def test_slot_stream_rejects_other_cache_modes_and_a_second_sink_swap():

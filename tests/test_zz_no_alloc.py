@@ -4,7 +4,9 @@ Callers that cannot allocate device memory (plugins whose host application
 owns all device memory, real-time paths) use this variant: its scratch -- the scaled queries the attention kernel
 reads -- lives in a static device array inside the library.  This test calls it
 through the C ABI twice in a row, with different inputs and sizes, and checks
-each output against the allocating entry point la_op_attention given the same
+each output against the fp64 oracle's block-causal attention (sink + two
+blocks, all visible) at the bf16 tolerance, and against the allocating entry
+point la_op_attention given the same
 query already scaled (q_scaled=1, q*log2(e)/sqrt(d) rounded once to bf16), with
 the tolerance the other GPU tests use; both run the same attention kernel on the
 same bf16 operands, so the outputs also agree bit for bit.  The file is named so
@@ -15,6 +17,7 @@ import ctypes
 import numpy as np
 import pytest
 
+from oracle import block_causal_attention
 from workloads import DTYPE_BF16, bf16_round, random_array
 
 from _helpers import assert_close
@@ -70,6 +73,12 @@ def test_static_scratch_attention_matches_allocating_entry_point_twice(lib):
                                           ctypes.c_void_p(got.data_ptr()), ctypes.c_void_p(got32.data_ptr()),
                                           _stream()) == 0
         torch.cuda.synchronize()
+        assert lib.la_op_status(_stream()) == 0, f"call {call}: a kernel reported a device error"
+        # against the fp64 oracle's block-causal attention on the unscaled bf16 inputs
+        hm = lambda t: t.float().cpu().numpy().transpose(1, 0, 2)          # [H, n, d] -> [n, H, d]
+        want = block_causal_attention(hm(q), {0: (hm(ks[1]), hm(vs[1])), 1: (hm(ks[2]), hm(vs[2]))},
+                                      (hm(ks[0]), hm(vs[0])), qblock=1, window=1).reshape(Tq, H * d)
+        assert_close(got32.cpu().numpy(), want, DTYPE_BF16, f"call {call}: fp32 output against the oracle")
         assert_close(got32.cpu().numpy(), ref32.cpu().numpy(), DTYPE_BF16, f"call {call}: fp32 output")
         assert_close(got.float().cpu().numpy(), ref.float().cpu().numpy(), DTYPE_BF16, f"call {call}: bf16 output")
         assert torch.equal(got32, ref32) and torch.equal(got, ref), f"call {call}: not bitwise equal"
