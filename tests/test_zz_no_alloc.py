@@ -74,9 +74,12 @@ def test_static_scratch_attention_matches_allocating_entry_point_twice(lib):
                                           _stream()) == 0
         torch.cuda.synchronize()
         assert lib.la_op_status(_stream()) == 0, f"call {call}: a kernel reported a device error"
-        # against the fp64 oracle's block-causal attention on the unscaled bf16 inputs
-        hm = lambda t: t.float().cpu().numpy().transpose(1, 0, 2)          # [H, n, d] -> [n, H, d]
-        want = block_causal_attention(hm(q), {0: (hm(ks[1]), hm(vs[1])), 1: (hm(ks[2]), hm(vs[2]))},
+        # against the fp64 oracle's block-causal attention on the operands the kernel
+        # reads: the query it consumes is q * log2(e)/sqrt(d) rounded once to bf16,
+        # i.e. the query q_scaled / (log2(e)/sqrt(d)) in the oracle's natural-log form
+        hm = lambda t: t.double().cpu().numpy().transpose(1, 0, 2)         # [H, n, d] -> [n, H, d]
+        want = block_causal_attention(hm(q_scaled) / SCALE_LOG2, {0: (hm(ks[1]), hm(vs[1])),
+                                                                   1: (hm(ks[2]), hm(vs[2]))},
                                       (hm(ks[0]), hm(vs[0])), qblock=1, window=1).reshape(Tq, H * d)
         assert_close(got32.cpu().numpy(), want, DTYPE_BF16, f"call {call}: fp32 output against the oracle")
         assert_close(got32.cpu().numpy(), ref32.cpu().numpy(), DTYPE_BF16, f"call {call}: fp32 output")
