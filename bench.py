@@ -1,6 +1,6 @@
 """Benchmark of the timestep-forced streaming step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sweep | --ablation]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sweep | --ablation] [--no-tpp]
 
 A step is one tick of the 4-slot grouped stream in steady state: 4 in-flight
 blocks (one per timestep slot, every window full) through 8 attention
@@ -17,14 +17,13 @@ from __future__ import annotations
 import argparse
 import json
 import os
-import statistics
-import subprocess
 import sys
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
+
+from streaming_causal_video_timestep_b200.clocks import ClockSampler  # noqa: E402
 
 METRIC = "latent frames/s (4-step stream, 1 B200); attention % of bf16 tensor-core peak"
 UNIT = "latent frames/s"
@@ -86,9 +85,11 @@ def kernel_entries(kinds, steps, L, S, T, D, C, F, attn_tflops, pk):
         if kind == "attn":
             e["tflops"] = round(attn_tflops, 1)
         elif kind == "rope":
-            # sink re-rope of every active slot: read the layer's fp32 un-roped sink K once,
-            # write S bf16 roped copies (the block's RoPE + append is fused into the QKV GEMM)
-            nbytes = F * D * 4 + S * F * D * 2
+            # sink re-rope of every active slot: read each layer's fp32 un-roped sink K once,
+            # write S bf16 roped copies (the block's RoPE + append is fused into the QKV GEMM);
+            # one launch covers all L layers of a pass (L steps / n layers a launch)
+            layers = max(1, round(L * steps / n))
+            nbytes = layers * (F * D * 4 + S * F * D * 2)
             e["gbs"] = round(nbytes / (avg / 1000.0) / 1e9, 1)
             e["frac_hbm"] = round(e["gbs"] / pk["hbm"], 3)
             e["bytes_per_launch"] = nbytes
@@ -110,61 +111,52 @@ def _peaks():
     return dict(tflops=1590.0, tflops_sust=1400.0, hbm=6650.0, src="fallback")
 
 
-class ClockSampler:
-    """nvidia-smi clocks and throttle reasons during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-
-    def __init__(self, gpu_index):
-        self.idx = gpu_index
-        self.proc = None
-        self.lines = []
-
-    def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except OSError:
-            self.proc = None
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.t.join(timeout=2)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
-
-
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
+def append_marginal(qkv_kind, S, T, D, iters=20):
+    """The Rolling RoPE + ring append runs as the epilogue of the QKV GEMM.  Its
+    cost is the difference between that GEMM, as the stream times it (all S
+    slots' rows, M = S T, N = 3D, K = D), and a plain bf16 store of the same GEMM
+    shape timed here in the same run; against it stand the bytes a separate
+    RoPE + append kernel would move (read qkv, write q, K and V: 2 x M x 3D x 2 B)."""
+    import torch
+    from streaming_causal_video_timestep_b200 import op_gemm
+
+    n, tot = qkv_kind
+    ms_epi = tot / max(n, 1)
+    M, N, K = S * T, 3 * D, D
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    A = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
+    W = (torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    for _ in range(3):
+        op_gemm(A, W, "store", out=out)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(iters):
+        op_gemm(A, W, "store", out=out)
+    ev1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms_plain = ev0.elapsed_time(ev1) / iters
+    standalone = 2 * M * N * 2
+    marginal = ms_epi - ms_plain
+    del A, W, out
+    torch.cuda.empty_cache()
+    return {"qkv_gemm_with_rope_append_ms": round(ms_epi, 4), "qkv_gemm_plain_store_ms": round(ms_plain, 4),
+            "marginal_ms": round(marginal, 4), "marginal_frac_of_gemm": round(marginal / ms_epi, 4),
+            "standalone_bytes": standalone,
+            "standalone_ms_at_measured_hbm": round(standalone / (_peaks()["hbm"] * 1e9) * 1e3, 4),
+            "shape": f"{M}x{N}x{K}", "clocks_plain_store": clk,
+            "note": "the epilogue writes the same number of bytes as the plain store (q, K, V vs qkv); a separate "
+                    "RoPE + append kernel would move standalone_bytes"}
+
+
 def run_gpu(args, rank, world, local_rank):
     import torch
     from streaming_causal_video_timestep_b200 import LaStream
@@ -276,6 +268,9 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     drain_ms = dr[0].elapsed_time(dr[1])
     s.close()
+    del s, weights
+    torch.cuda.empty_cache()
+    append = append_marginal(kinds["qkv_gemm"], S, T, D)
 
     frames_per_tick = cfg.frames_per_block
     value = job_throughput(frames_per_tick, args.steps, world, ms / 1000.0)
@@ -304,10 +299,116 @@ def run_gpu(args, rank, world, local_rank):
                    "fill_ms": round(fill_ms, 3), "drain_ticks": S - 1, "drain_ms": round(drain_ms, 3),
                    "note": "rank 0; fill = ticks until every slot is active with a full window (untimed by value)"},
         "clocks": clk,
+        "append": append,
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": T * C * 4,
                 "d2h_bytes_per_step": T * C * 4, "steps": e2e_steps},
     }
     return line
+
+
+def run_tpp(args, rank, world, local_rank):
+    """The timestep pipeline across GPUs (the pages' TPP): world / num_steps
+    pipelines of num_steps consecutive ranks; rank r of a pipeline owns denoising
+    step r of every block with its own cache (an LA_SCHED_SLOT stream of the
+    headline workload) and hands the latent to rank r + 1 by NCCL send/recv (no
+    other data path; the Adaptive Attention Sink is broadcast once).  Every rank
+    runs this; rank 0 returns the record.  Timed on the device: K ticks between
+    CUDA events on each rank, max over all ranks."""
+    import torch
+    import torch.distributed as tdist
+    from streaming_causal_video_timestep_b200 import LaStream
+    from streaming_causal_video_timestep_b200.tpp import DistTransport, TppRank
+    from workloads import SCHED_SLOT, SINK_AAS, STREAM
+
+    wl = STREAM
+    S = wl.cfg.num_steps
+    G = world // S
+    groups = [tdist.new_group(list(range(p * S, (p + 1) * S))) for p in range(G)]
+    pid, r = rank // S, rank % S
+    cfg = wl.cfg.replace(schedule=SCHED_SLOT, slot_index=r)
+    T, C, D, F = cfg.block_tokens, cfg.latent_ch, cfg.hidden, cfg.frame_tokens
+    L = cfg.num_layers
+    dev = torch.device("cuda", local_rank)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2000 + pid)               # the ranks of a pipeline hold the same model and sink
+    bf = torch.bfloat16
+    rnd = lambda shape, std: (torch.randn(shape, generator=g, device="cuda") * std).to(bf)
+    weights = dict(w_qkv=[rnd((3 * D, D), wl.w_std) for _ in range(L)],
+                   w_out=[rnd((D, D), wl.w_std) for _ in range(L)],
+                   w_in=rnd((D, C), 1.0 / C ** 0.5), w_head=rnd((C, D), wl.head_std))
+    s = LaStream(cfg, weights)
+    s.set_sink(torch.randn((F, C), generator=g, device="cuda"))
+    xs = [torch.randn((T, C), generator=g, device="cuda") for _ in range(4)]
+    tr = DistTransport(r, S, dev, group=groups[pid], base=pid * S)
+    me = TppRank(s, r, S, tr, dev, S, cfg.sink_tokens, cfg.sink_mode == SINK_AAS)
+    k = 0
+
+    def tick():
+        nonlocal k
+        fin = me.tick(xs[k % 4] if r == 0 else None)
+        k += 1
+        return fin[0]
+
+    tdist.barrier()
+    torch.cuda.synchronize()
+    ev_first = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev_first[0].record()
+    first_ms = 0.0
+    for _ in range(S - 1 + args.warmup):     # fill: block 0 leaves the last rank at tick S - 1
+        if tick() == 0:
+            ev_first[1].record()
+    torch.cuda.synchronize()
+    if r == S - 1:
+        first_ms = ev_first[0].elapsed_time(ev_first[1])
+    tdist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(args.steps):
+        tick()
+    ev[1].record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(ev[0].elapsed_time(ev[1]), "cuda")
+    first_ms = max_over_ranks(first_ms, "cuda")
+    me.close()                               # the last tick's hand-off is received before the next test
+    # the hand-off alone: the message a rank sends each tick (block id + T x C fp32),
+    # rank r -> r + 1 of every pipeline at once, timed on each rank, max over ranks
+    msg = [torch.zeros(1, dtype=torch.int64, device=dev), torch.zeros((T, C), dtype=torch.float32, device=dev)]
+    inbox = [torch.empty_like(t) for t in msg]
+    tdist.barrier()
+    torch.cuda.synchronize()
+    hev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    reps = 20
+    hev[0].record()
+    for _ in range(reps):
+        works = []
+        if r < S - 1:
+            works += [tdist.isend(t, pid * S + r + 1, group=groups[pid]) for t in msg]
+        if r > 0:
+            works += [tdist.irecv(t, pid * S + r - 1, group=groups[pid]) for t in inbox]
+        for w in works:
+            w.wait()
+    hev[1].record()
+    torch.cuda.synchronize()
+    hand_ms = max_over_ranks(hev[0].elapsed_time(hev[1]) / reps, "cuda")
+    tdist.barrier()
+    s.close()
+    del s, weights
+    torch.cuda.empty_cache()
+    for grp in groups:
+        tdist.destroy_process_group(grp)
+    return {"pipelines": G, "ranks_per_pipeline": S,
+            "latent_frames_per_s": round(job_throughput(cfg.frames_per_block, args.steps, G, ms / 1000.0), 3),
+            "ms_per_tick": round(ms / args.steps, 3), "steps": args.steps,
+            "first_finished_block_ms": round(first_ms, 3),
+            "handoff_bytes_per_tick_per_link": 8 + T * C * 4, "handoff_ms": round(hand_ms, 4),
+            "clocks": clk,
+            "note": "rank r of each pipeline owns step r with its own cache (LA_SCHED_SLOT stream); NCCL "
+                    "send/recv of the latent between consecutive ranks; the AAS sink broadcast once"}
 
 
 # ---------------------------------------------------------------------------
@@ -405,6 +506,8 @@ def run_sweep(args):
         s.set_sink(torch.randn((F, C), generator=g, device="cuda"))
         xs = [torch.randn((T, C), generator=g, device="cuda") for _ in range(2)]
         x_out = torch.empty((T, C), device="cuda")
+        clocks = ClockSampler(0)
+        clocks.start()
         for k in range((S - 1) + nw + 1 + args.warmup):
             s.step(xs[k % 2], x_out)
         s.synchronize()
@@ -417,6 +520,7 @@ def run_sweep(args):
         s.synchronize()
         torch.cuda.synchronize()
         ms = ev0.elapsed_time(ev1) / args.steps
+        clk = clocks.stop()
         n_a, t_a = s.profile_read("attn")
         n_r, t_r = s.profile_read("rope")
         s.profile(False)
@@ -433,27 +537,32 @@ def run_sweep(args):
                                    "frac_spec_2250": round(attn_tf / 2250.0, 3)},
                           "sink_rerope": {"gbs": round(rope_gbs, 1), "bytes_per_launch": rope_bytes,
                                           "frac_hbm": round(rope_gbs / pk["hbm"], 3)},
-                          "peaks": pk["src"]}), flush=True)
+                          "peaks": pk["src"], "clocks": clk}), flush=True)
         s.close()
         del s, weights
         torch.cuda.empty_cache()
     rows, C, G = 1 << 20, 64, 4   # 256 MB per tensor, larger than L2
     x = torch.randn(rows, C, device="cuda")
     v = torch.randn(rows, C, device="cuda")
+    clocks = ClockSampler(0)
+    clocks.start()
     for _ in range(args.warmup):
         op_euler(x, v, [-0.25] * G, rows // G)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_euler = max(args.steps, 2000)     # ~0.25 ms a launch: enough launches to cover clock samples
     ev0.record()
-    for _ in range(args.steps):
+    for _ in range(n_euler):
         op_euler(x, v, [-0.25] * G, rows // G)
     ev1.record()
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1) / args.steps
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / n_euler
     gbs = 3 * rows * C * 4 / (ms / 1000.0) / 1e9
     print(json.dumps({"sweep": "euler_standalone", "shape": f"{rows}x{C} fp32, {G} timestep groups",
                       "ms": round(ms, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 3),
-                      "note": "in the stream the Euler update is fused into the velocity-head GEMM epilogue"}),
+                      "note": "in the stream the Euler update is fused into the velocity-head GEMM epilogue",
+                      "clocks": clk}),
           flush=True)
 
 
@@ -521,6 +630,8 @@ def run_ablation(args):
         xs = [torch.randn((T, C), generator=g, device="cuda") for _ in range(2)]
         x_out = torch.empty((T, C), device="cuda")
         fill = ((S - 1) if sched == SCHED_PIPELINED else 0) + nw + 1 + args.warmup
+        clocks = ClockSampler(0)
+        clocks.start()
         for k in range(fill):
             s.step(xs[k % 2], x_out, audio=aud)
         s.synchronize()
@@ -533,6 +644,7 @@ def run_ablation(args):
         s.synchronize()
         torch.cuda.synchronize()
         ms = ev0.elapsed_time(ev1) / args.steps
+        clk = clocks.stop()
         kinds = {kd: round(s.profile_read(kd)[1] / args.steps, 3)
                  for kd in ("qkv_gemm", "attn", "out_gemm", "other") + (("ffn",) if ffn else ())
                  + (("cross",) if audio else ())}
@@ -551,7 +663,8 @@ def run_ablation(args):
                                     + ", hidden 5120, 40x128 heads, 30x52 grid, window 2, "
                                     + ", ".join([x for x in ("e4m3 QKV/output projections" if fp8 else "",
                                                              "e4m3 attention" if afp8 else "") if x]
-                                                or ["bf16"])}),
+                                                or ["bf16"]),
+                          "clocks": clk}),
               flush=True)
         s.close()
         del s, weights
@@ -590,6 +703,8 @@ def main():
                     help="seconds per block: grouped pipeline vs sequential vs clean-cache refresh")
     ap.add_argument("--ablation-rows", default="",
                     help="comma-separated row indices of --ablation to run (default: all)")
+    ap.add_argument("--no-tpp", action="store_true",
+                    help="with N a multiple of the step count, skip the timestep-pipeline sub-record")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -617,6 +732,11 @@ def main():
         torch.cuda.set_device(local_rank)
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     line = run_gpu(args, rank, world, local_rank)
+    from workloads import STREAM
+    if world > 1 and world % STREAM.cfg.num_steps == 0 and not args.no_tpp:
+        tpp = run_tpp(args, rank, world, local_rank)
+        if rank == 0:
+            line["tpp"] = tpp
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()

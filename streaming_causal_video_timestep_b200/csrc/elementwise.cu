@@ -120,12 +120,14 @@ __global__ void __launch_bounds__(256) k_rope_append(const __grid_constant__ Pas
   }
 }
 
-// Per-block re-rope of the fp32 un-roped sink K for every active buffer.  The
-// spatial rotation factors depend only on (token, pair) and the temporal ones
-// only on (buffer, pair), so one thread takes one (token, 8-element chunk) for
-// SINK_HEADS heads: it loads their chunks and the factors once and writes each
-// chunk roped, rounded once to TO, for every active buffer.  Reads F*H*d*4
-// bytes once and writes nactive*F*H*d*sizeof(TO).
+// Per-block re-rope of the fp32 un-roped sink K of every layer for every active
+// buffer, in one launch (the sink positions depend on the buffer's block, not
+// on the layer).  The spatial rotation factors depend only on (token, pair) and
+// the temporal ones only on (buffer, pair), so one thread takes one (layer,
+// token, 8-element chunk) for SINK_HEADS heads: it loads their chunks and the
+// factors once and writes each chunk roped, rounded once to TO, for every
+// active buffer.  Reads nl*F*H*d*4 bytes once and writes
+// nl*nactive*F*H*d*sizeof(TO).
 constexpr int SINK_HEADS = 8;
 
 template <typename TO>
@@ -135,15 +137,19 @@ __global__ void __launch_bounds__(256) k_sink_rerope(const __grid_constant__ Pas
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int ch = static_cast<int>(idx % chunks);
-    const long long rest = idx / chunks;
+    long long rest = idx / chunks;
     const int m = static_cast<int>(rest % a.F);
-    const int h0 = static_cast<int>(rest / a.F) * SINK_HEADS;
+    rest /= a.F;
+    const int hgroups = (a.H + SINK_HEADS - 1) / SINK_HEADS;
+    const int h0 = static_cast<int>(rest % hgroups) * SINK_HEADS;
+    const int l = static_cast<int>(rest / hgroups);
     const int nh = min(SINK_HEADS, a.H - h0);
+    const long long plane = static_cast<long long>(a.H) * a.F * a.d;
     float v[SINK_HEADS][8];
 #pragma unroll
     for (int k = 0; k < SINK_HEADS; ++k)
       if (k < nh)
-        Vec8<float>::load(reinterpret_cast<const float*>(a.sink_k) +
+        Vec8<float>::load(reinterpret_cast<const float*>(a.sink_k) + l * plane +
                               (static_cast<long long>(h0 + k) * a.F + m) * a.d + ch * 8, v[k]);
     const int rr = m / a.grid_w, cc = m % a.grid_w;
     float c[4], sn[4];
@@ -176,7 +182,7 @@ __global__ void __launch_bounds__(256) k_sink_rerope(const __grid_constant__ Pas
           sb[jj] = sn[jj];
         }
       }
-      TO* out = reinterpret_cast<TO*>(a.sink_k_rope) + static_cast<long long>(buf) * a.H * a.F * a.d;
+      TO* out = reinterpret_cast<TO*>(a.sink_k_rope) + (static_cast<long long>(l) * a.nb + buf) * plane;
 #pragma unroll
       for (int k = 0; k < SINK_HEADS; ++k) {
         if (k >= nh) break;
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(256) k_sink_rerope(const __grid_constant__ Pas
         }
         TO* dst = out + (static_cast<long long>(h0 + k) * a.F + m) * a.d + ch * 8;
         if constexpr (sizeof(TO) == 1)
-          store_e4m3x8(reinterpret_cast<uint8_t*>(dst), w, a.fp8_inv[a.H + h0 + k]);
+          store_e4m3x8(reinterpret_cast<uint8_t*>(dst), w, a.fp8_inv[l * 3 * a.H + a.H + h0 + k]);
         else
           Vec8<TO>::store(dst, w);
       }
@@ -417,7 +423,10 @@ cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs&
 cudaError_t launch_sink_rerope(int out_kind, const PassDesc& pd, const RopeArgs& a, cudaStream_t st) {
   if (!a.sink_k || pd.nactive == 0) return cudaSuccess;
   if (out_kind == 2 && !a.fp8_inv) return cudaErrorInvalidValue;
-  const long long n = static_cast<long long>(a.F) * ((a.H + SINK_HEADS - 1) / SINK_HEADS) * (a.d / 8);
+  if (a.nl < 1 || a.nb < 1) return cudaErrorInvalidValue;
+  for (int ai = 0; ai < pd.nactive; ++ai)
+    if (pd.active_buf[ai] < 0 || pd.active_buf[ai] >= a.nb) return cudaErrorInvalidValue;
+  const long long n = static_cast<long long>(a.nl) * a.F * ((a.H + SINK_HEADS - 1) / SINK_HEADS) * (a.d / 8);
   const int grid = grid_for(n);
   if (out_kind == 2)
     k_sink_rerope<uint8_t><<<grid, 256, 0, st>>>(pd, a, n);

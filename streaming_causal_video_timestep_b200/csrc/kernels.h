@@ -72,17 +72,19 @@ struct RopeArgs {
   void* ring_k; void* ring_v;                  // [L][S][E][H][T][d]
   long long ring_slice0;                       // (layer*S) * E: slice of (layer, slot 0, entry 0)
   int E;
-  const void* sink_k;                          // fp32 un-roped [H][F][d] of this layer (NULL: no sink part)
-  void* sink_k_rope;                           // [nbuf][H][F][d]
-  const float* fp8_inv;                        // [3][H] inverse e4m3 scales of q, K, V (e4m3 outputs)
+  const void* sink_k;                          // fp32 un-roped [nl][H][F][d] from the first layer (NULL: no sink part)
+  void* sink_k_rope;                           // [nl][nb][H][F][d]
+  const float* fp8_inv;                        // [nl][3][H] inverse e4m3 scales of q, K, V (e4m3 outputs)
+  int nl = 1;                                  // layers of one sink re-rope launch
+  int nb = 1;                                  // buffers of sink_k_rope a layer
 };
 // Rolling RoPE + ring append of every active buffer's block from the fp32 qkv
 // (fp32 streams; bf16 streams do it in the QKV GEMM epilogue).  Outputs are
 // bf16 (bf16_out) or fp32.
 cudaError_t launch_rope_append(int bf16_out, const PassDesc& pd, const RopeArgs& a, cudaStream_t st);
-// Re-rope of the layer's fp32 un-roped sink K at every active buffer's sink
-// position (a.sink_k -> a.sink_k_rope[buf]).  out_kind: 0 fp32, 1 bf16,
-// 2 e4m3 codes of value * a.fp8_inv[H + head].
+// Re-rope of the fp32 un-roped sink K of a.nl layers at every active buffer's
+// sink position (a.sink_k[l] -> a.sink_k_rope[l][buf]), one launch.  out_kind:
+// 0 fp32, 1 bf16, 2 e4m3 codes of value * a.fp8_inv[l][H + head].
 cudaError_t launch_sink_rerope(int out_kind, const PassDesc& pd, const RopeArgs& a, cudaStream_t st);
 
 // Sink pass: split the fp32 qkv [F, 3D] into the layer's fp32 un-roped K, its

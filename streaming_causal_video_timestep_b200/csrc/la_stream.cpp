@@ -204,7 +204,7 @@ struct la_stream {
   void* xop = nullptr;      // [nbuf*T][C] bf16 (bf16 with an in-projection)
   float* qkv = nullptr;     // fp32 [nbuf*T][3D] (fp32 streams; bf16 fuses it into the GEMM)
   void* q_rope = nullptr;   // attn type [nbuf][H][T][d]
-  void* sk_rope = nullptr;  // attn type [nbuf][H][F][d]
+  void* sk_rope = nullptr;  // attn type [L][nbuf][H][F][d]
   void* attn_o = nullptr;   // dtype [nbuf*T][D]
   void* ring_k = nullptr;   // attn type [L][S][E][H][T][d]
   void* ring_v = nullptr;
@@ -502,7 +502,8 @@ int capture_pass(la_stream* s, const PassDesc& pd, int layer) {
     CU(cudaMemcpyAsync(s->cap_o + (static_cast<long long>(slot) * L + layer) * T * D, o32 + buf * T * D, T * D * 4,
                        cudaMemcpyDeviceToDevice, s->st));
     CU(cudaMemcpyAsync(elem(s->cap_sk, (static_cast<long long>(slot) * L + layer) * H * F * d, eq),
-                       elem(s->sk_rope, buf * H * F * d, eq), H * F * d * eq, cudaMemcpyDeviceToDevice, s->st));
+                       elem(s->sk_rope, (static_cast<long long>(layer) * s->nbuf + buf) * H * F * d, eq), H * F * d * eq,
+                       cudaMemcpyDeviceToDevice, s->st));
   }
   return LA_OK;
 }
@@ -707,6 +708,18 @@ int run_pass(la_stream* s, const PassDesc& pd) {
   ap.kbase[1] = s->sk_rope; ap.vbase[1] = s->sink_v; ap.krows[1] = F; ap.vrows[1] = F;
   ap.ngroups = pd.nactive;
 
+  // per-block re-rope of every layer's sink K (fp32 -> bf16, e4m3 or fp32), once
+  // per active buffer: the sink's positions depend on the buffer's block only
+  ra.sink_k = s->sink_k;
+  ra.sink_k_rope = s->sk_rope;
+  ra.nl = s->L;
+  ra.nb = s->nbuf;
+  ra.fp8_inv = s->afp8 ? s->attn_inv : nullptr;
+  if ((r = launch(s, LA_KIND_ROPE, [&] {
+         return launch_sink_rerope(s->bf16 ? (s->afp8 ? 2 : 1) : 0, pd, ra, s->st);
+       })) != LA_OK)
+    return r;
+
   QkvRopeParams qp{};
   qp.T = T; qp.F = F; qp.H = H; qp.d = d; qp.D = D; qp.E = E; qp.grid_w = s->cfg.grid_w;
   qp.pt = s->pt; qp.ph = s->ph;
@@ -737,8 +750,6 @@ int run_pass(la_stream* s, const PassDesc& pd) {
     }
     ra.qkv = s->qkv; ra.q_rope = s->q_rope; ra.ring_k = s->ring_k; ra.ring_v = s->ring_v;
     ra.ring_slice0 = static_cast<long long>(l) * S * E;
-    ra.sink_k = s->sink_k + static_cast<long long>(l) * H * F * d;
-    ra.sink_k_rope = s->sk_rope;
     if (s->afp8) {
       const long long so = static_cast<long long>(l) * 3 * H;
       ra.fp8_inv = qp.fp8_inv = s->attn_inv + so;
@@ -762,16 +773,12 @@ int run_pass(la_stream* s, const PassDesc& pd) {
                   })) != LA_OK) {
         return r;
       }
-      // per-block re-rope of the sink K (fp32 -> bf16 or e4m3, once per active buffer)
-      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_sink_rerope(s->afp8 ? 2 : 1, pd, ra, s->st); })) != LA_OK)
-        return r;
     } else {
       GemmEpiParams eq = epi(EPI_STORE, s->qkv, nullptr, 3LL * D);
       if ((r = gemm(s, LA_KIND_QKV_GEMM, &s->tm_hop, &s->tm_wqkv[l], s->hn32, s->w_qkv[l], eq, rows, 3 * D, D)) !=
           LA_OK)
         return r;
       if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_rope_append(0, pd, ra, s->st); })) != LA_OK) return r;
-      if ((r = launch(s, LA_KIND_ROPE, [&] { return launch_sink_rerope(0, pd, ra, s->st); })) != LA_OK) return r;
     }
     // block-causal attention: [sink | window oldest first | self]
     for (int ai = 0; ai < pd.nactive; ++ai) {
@@ -780,7 +787,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
       g.q_slice = buf;
       g.out_row0 = buf * T;
       int ns = 0;
-      g.seg[ns++] = AttnSeg{1, 1, buf, l, F};
+      g.seg[ns++] = AttnSeg{1, 1, l * s->nbuf + buf, l, F};
       const long long base = static_cast<long long>(l) * S * E + static_cast<long long>(pd.slot[buf]) * E;
       const long long wbase = static_cast<long long>(l) * S * E + static_cast<long long>(pd.win_slot[buf]) * E;
       for (int w = 0; w < pd.nwin[buf]; ++w)
@@ -1178,7 +1185,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   const long long need = NB * T * C * 4 + NB * T * D * 4 + (s->bf16 ? NB * T * D * es : 0) +
                          ((!s->bf16 || s->id_head) ? NB * T * D * 4 : 0) + F * D * 4 +
                          (s->bf16 && !s->id_in ? NB * T * C * 2 : 0) + (s->bf16 ? 0 : NB * T * 3 * D * 4) +
-                         NB * T * D * eq + NB * T * D * es + NB * H * F * d * eq + 2 * L * S * E * H * T * d * eq +
+                         NB * T * D * eq + NB * T * D * es + L * NB * H * F * d * eq + 2 * L * S * E * H * T * d * eq +
                          L * H * F * d * (4 + ea) + F * C * 4 + F * D * 4 + F * D * es * 2 + F * C * 2 +
                          F * 3 * D * 4 + 2 * H * F * d * ea + (s->afp8 ? L * H * F * d + L * 3 * H * 8 : 0) +
                          (s->dit ? std::max(NB * T, F) * s->Fffn * static_cast<long long>(es) : 0) +
@@ -1209,7 +1216,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   if (!s->bf16) ALLOC_OR_BAIL(s->qkv, NB * T * 3 * D * 4);
   ALLOC_OR_BAIL(s->q_rope, NB * T * D * eq);
   ALLOC_OR_BAIL(s->attn_o, NB * T * D * es);
-  ALLOC_OR_BAIL(s->sk_rope, NB * H * F * d * eq);
+  ALLOC_OR_BAIL(s->sk_rope, L * NB * H * F * d * eq);
   ALLOC_OR_BAIL(s->ring_k, L * S * E * H * T * d * eq);
   ALLOC_OR_BAIL(s->ring_v, L * S * E * H * T * d * eq);
   ALLOC_OR_BAIL(s->sink_k, L * H * F * d * 4);
@@ -1325,13 +1332,13 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
       ok = ok && tmap_planes_u8(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
       ok = ok && tmap_planes_u8(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
       ok = ok && tmap_planes_u8(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
-      ok = ok && tmap_planes_u8(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
+      ok = ok && tmap_planes_u8(&s->maps_stream.k[1], s->sk_rope, d, F, H, L * NB, s->err);
       ok = ok && tmap_planes_u8(&s->maps_stream.v[1], s->sink_v8, d, F, H, L, s->err);
     } else {
       ok = ok && tmap_planes_bf16(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);
       ok = ok && tmap_planes_bf16(&s->maps_stream.k[0], s->ring_k, d, T, H, L * S * E, s->err);
       ok = ok && tmap_planes_bf16(&s->maps_stream.v[0], s->ring_v, d, T, H, L * S * E, s->err);
-      ok = ok && tmap_planes_bf16(&s->maps_stream.k[1], s->sk_rope, d, F, H, NB, s->err);
+      ok = ok && tmap_planes_bf16(&s->maps_stream.k[1], s->sk_rope, d, F, H, L * NB, s->err);
       ok = ok && tmap_planes_bf16(&s->maps_stream.v[1], s->sink_v, d, F, H, L, s->err);
     }
     ok = ok && tmap_planes_bf16(&s->maps_sink.q, s->s_q, d, F, H, 1, s->err);

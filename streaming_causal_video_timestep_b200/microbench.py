@@ -18,11 +18,13 @@ gemm_out: the output projection of the 4-slot grouped launch, [18720, 5120] x
 euler: x += dt * v over 2^20 rows x 64 fp32 (256 MB per tensor), 4 groups.
 gemm_fp8: the QKV projection shape on e4m3 operands (kind::f8f6f4, per-row
        scales, bf16 output), and the per-row quantization of its activation.
-rerope: the per-block sink re-rope of a one-sublayer stream (30x52 grid, 40x128
-       heads, 4 slots): reads the fp32 un-roped sink K (32 MB) once and writes
-       4 bf16 roped copies (64 MB); timed by the stream's profiling counters.
+rerope: the per-block sink re-rope of the 8-sublayer stream (30x52 grid, 40x128
+       heads, 4 slots), one launch a tick for all layers: reads each layer's
+       fp32 un-roped sink K (32 MB) once and writes 4 bf16 roped copies (64 MB),
+       766 MB a launch; timed by the stream's profiling counters.
 Inputs exceed L2 (126 MB) except the per-slot attention keys (160 MB K/V +
-48 MB q).  Prints one JSON line per mode.
+48 MB q).  Each timed loop spans at least 1.5 s; prints one JSON line per mode
+with the SM clock record (median under load, throttle reasons) taken around it.
 """
 from __future__ import annotations
 
@@ -31,20 +33,29 @@ import json
 
 import torch
 
+from .clocks import ClockSampler
 from .stream import op_attention, op_attention_fp8, op_euler, op_gemm, op_gemm_fp8, op_quantize_e4m3
 
 
-def _time(fn, iters, warmup=3):
+def _time(fn, iters, warmup=3, min_ms=1500.0):
+    """Average ms of fn on the current stream (CUDA events), after warm-up; at
+    least `iters` launches and enough of them to span min_ms, so that the clock
+    sampler running around each mode sees several samples under load."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     ev[0].record()
-    for _ in range(iters):
+    fn()
+    ev[1].record()
+    torch.cuda.synchronize()
+    n = max(iters, int(min_ms / max(ev[0].elapsed_time(ev[1]), 1e-3)) + 1)
+    ev[0].record()
+    for _ in range(n):
         fn()
     ev[1].record()
     torch.cuda.synchronize()
-    return ev[0].elapsed_time(ev[1]) / iters
+    return ev[0].elapsed_time(ev[1]) / n
 
 
 def bench_attn(iters):
@@ -147,7 +158,7 @@ def bench_euler(iters):
 def bench_rerope(iters):
     from types import SimpleNamespace
     from .stream import LaStream
-    cfg = SimpleNamespace(num_layers=1, hidden=5120, heads=40, head_dim=128, latent_ch=64, grid_h=30, grid_w=52,
+    cfg = SimpleNamespace(num_layers=8, hidden=5120, heads=40, head_dim=128, latent_ch=64, grid_h=30, grid_w=52,
                           frames_per_block=3, sink_frames=1, window_blocks=1, timesteps=(1.0, 0.75, 0.5, 0.25, 0.0),
                           rope_split=(22, 21, 21), pairs=(22, 21, 21), rope_theta=10000.0, sink_mode=0, rolling_rope=1,
                           sink_offset_frames=3, schedule=0, dtype=0)
@@ -155,7 +166,9 @@ def bench_rerope(iters):
     g = torch.Generator(device="cuda")
     g.manual_seed(0)
     rnd = lambda *sh: (torch.randn(*sh, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
-    w = dict(w_qkv=[rnd(3 * D, D)], w_out=[rnd(D, D)], w_in=rnd(D, C), w_head=rnd(C, D))
+    L = cfg.num_layers
+    w = dict(w_qkv=[rnd(3 * D, D) for _ in range(L)], w_out=[rnd(D, D) for _ in range(L)], w_in=rnd(D, C),
+             w_head=rnd(C, D))
     s = LaStream(cfg, w)
     s.set_sink(torch.randn(F, C, generator=g, device="cuda"))
     x = torch.randn(T, C, generator=g, device="cuda")
@@ -171,9 +184,9 @@ def bench_rerope(iters):
     s.profile(False)
     s.close()
     ms = tot / n
-    nbytes = F * D * 4 + 4 * F * D * 2
-    return {"mode": "rerope", "shape": f"sink {F} tokens x {D}, 4 slots", "ms": round(ms, 4),
-            "gbs": round(nbytes / ms / 1e6, 1), "bytes": nbytes}
+    nbytes = L * (F * D * 4 + 4 * F * D * 2)
+    return {"mode": "rerope", "shape": f"sink {F} tokens x {D}, {L} layers, 4 slots, one launch a tick",
+            "ms": round(ms, 4), "gbs": round(nbytes / ms / 1e6, 1), "bytes": nbytes}
 
 
 def main():
@@ -183,8 +196,11 @@ def main():
     args = ap.parse_args()
     modes = ["attn", "attn_fp8", "gemm", "gemm_out", "gemm_fp8", "euler", "rerope"] if args.mode == "all" else [args.mode]
     for m in modes:
+        clocks = ClockSampler(torch.cuda.current_device())
+        clocks.start()
         r = {"attn": bench_attn, "attn_fp8": bench_attn_fp8, "gemm": bench_gemm, "gemm_out": bench_gemm_out,
              "euler": bench_euler, "rerope": bench_rerope, "gemm_fp8": bench_gemm_fp8}[m](args.iters)
+        r["clocks"] = clocks.stop()
         print(json.dumps(r), flush=True)
 
 

@@ -29,11 +29,17 @@ import torch
 
 class DistTransport:
     """Point-to-point hand-off and the sink broadcast over torch.distributed (NCCL
-    over NVLink on GPUs, gloo on the host)."""
+    over NVLink on GPUs, gloo on the host).
 
-    def __init__(self, rank: int, world: int, device, group=None):
+    rank / world: the rank's step and the pipeline's length; base: the global
+    rank of the pipeline's step 0 (several pipelines in one job each take a run
+    of num_steps consecutive global ranks and their own process group, since
+    torch.distributed addresses peers by global rank)."""
+
+    def __init__(self, rank: int, world: int, device, group=None, base: int = 0):
         import torch.distributed as dist
         self.dist, self.rank, self.world, self.device, self.group = dist, rank, world, device, group
+        self.base = base
         self._pending = []
 
     def send_next(self, tensors):
@@ -42,16 +48,16 @@ class DistTransport:
         for w in self._pending:
             w.wait()
         self._keep = [t.contiguous().clone() for t in tensors]
-        self._pending = [self.dist.isend(t, self.rank + 1, group=self.group) for t in self._keep]
+        self._pending = [self.dist.isend(t, self.base + self.rank + 1, group=self.group) for t in self._keep]
 
     def recv_prev(self, shapes_dtypes):
         out = [torch.empty(s, dtype=d, device=self.device) for s, d in shapes_dtypes]
-        for w in [self.dist.irecv(t, self.rank - 1, group=self.group) for t in out]:
+        for w in [self.dist.irecv(t, self.base + self.rank - 1, group=self.group) for t in out]:
             w.wait()
         return out
 
     def bcast_from_last(self, t):
-        self.dist.broadcast(t, self.world - 1, group=self.group)
+        self.dist.broadcast(t, self.base + self.world - 1, group=self.group)
         return t
 
     def finish(self):

@@ -64,3 +64,11 @@ def test_other_kinds_and_partial_counts():
     # a GEMM kind with fewer launches than one a layer and tick gets no FLOP rate
     run = dict(RUN, out_gemm=(40, 0.7291, None))
     assert "tflops" not in _table(run)["out_gemm"]
+
+
+def test_rope_launch_covering_every_layer_counts_every_layers_bytes():
+    """One sink re-rope launch a tick for all 8 layers: 8x the bytes of a per-layer launch."""
+    run = dict(RUN, rope=(10, 0.1300, None))
+    e = _table(run)["rope"]
+    assert e["bytes_per_launch"] == 8 * (1560 * 5120 * 4 + 4 * 1560 * 5120 * 2)
+    assert e["gbs"] == pytest.approx(e["bytes_per_launch"] / 0.1300e-3 / 1e9, rel=1e-3)

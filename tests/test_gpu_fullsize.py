@@ -193,19 +193,34 @@ def test_soak_10000_blocks_rolling_rope_and_ring():
     assert n_checked == len(checked) * S
 
 
-@pytest.mark.slow
-def test_largest_sweep_point_45x80_window_8():
-    wl = sweep_point((45, 80), 8)
-    wl = Workload(wl.name, wl.cfg, wl.seed, 10, wl.w_std, wl.head_std)
+@pytest.mark.parametrize("grid,window", [(g, w) for g in ((30, 52), (45, 80)) for w in (1, 2, 4, 8)],
+                         ids=[f"{g[0]}x{g[1]}-w{w}" for g in ((30, 52), (45, 80)) for w in (1, 2, 4, 8)])
+def test_sweep_point_steady_state_all_slots(grid, window):
+    """Every shape-sweep point (token grids 30x52 and 45x80, windows 1, 2, 4, 8; one
+    sublayer; 4 slots in a grouped launch): at the first tick where all 4 slots run
+    blocks with a full window, every op of every slot is checked on sampled rows
+    (attention over all keys), integer state bit-exact every tick."""
+    wl = sweep_point(grid, window)
+    wl = Workload(wl.name, wl.cfg, wl.seed, window + 4, wl.w_std, wl.head_std)
     cfg = wl.cfg
     s, W = make_stream(wl, capture=False)
     R = sample_rows(cfg.block_tokens, n=16)
     x_out = torch.empty((cfg.block_tokens, cfg.latent_ch), device="cuda")
-    last = wl.num_blocks + 2
+    ref = TickScheduler(cfg)
+    last = wl.num_blocks - 1              # slots 0..3 run blocks last .. last-3 >= window
     for k in range(last + 1):
         s.capture(k == last)
-        fin = s.step(_dev(block_noise(wl, k)) if k < wl.num_blocks else None, x_out)
-    for (b, i) in _active(s, cfg):
-        check_step(s, cfg, W, b, i, rows=R, tag="sweep 45x80 w8")
+        sink = sink_snapshot(s, cfg) if k == last else None
+        fin = s.step(_dev(block_noise(wl, k)), x_out)
+        run, fin_o = ref.begin_tick(True)
+        for i, bb in run:
+            ref.append(i, bb)
+        ref.end_tick(fin_o)
+        assert fin == fin_o
+        np.testing.assert_array_equal(s.index_state(), ref.index_state())
+    act = _active(s, cfg)
+    assert len(act) == cfg.num_steps and min(b for b, _ in act) >= window
+    for (b, i) in act:
+        check_step(s, cfg, W, b, i, rows=R, tag=f"sweep {grid[0]}x{grid[1]} w{window}", sink=sink)
     s.synchronize()
     s.close()

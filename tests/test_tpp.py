@@ -29,12 +29,14 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _workload(aas=True, audio=False):
+def _workload(aas=True, audio=False, steps=4, seed=3):
     from workloads import BLOCK_DIT, SINK_AAS, SINK_FIXED, TINY, Workload
     cfg = TINY.cfg.replace(sink_mode=SINK_AAS if aas else SINK_FIXED)
+    if steps == 2:
+        cfg = cfg.replace(timesteps=(1.0, 0.5, 0.0))
     if audio:
         cfg = cfg.replace(block_kind=BLOCK_DIT, ffn_dim=96, audio_tokens=6, audio_dim=8)
-    return Workload("tpp", cfg, 3, 6, TINY.w_std, TINY.head_std)
+    return Workload("tpp", cfg, seed, 6, TINY.w_std, TINY.head_std)
 
 
 class OracleSlot:
@@ -150,3 +152,57 @@ def test_tpp_needs_one_rank_per_step():
         T, C = 4, 2
     with pytest.raises(ValueError):
         TppRank(_B(), 0, 3, LocalTransport(3).endpoint(0), "cpu", 4, 1, False)
+
+
+def _pipelines_main(rank, world, steps, port, out):
+    """world / steps pipelines of `steps` consecutive ranks in one job, each over its
+    own process group (DistTransport's base rank), each with its own workload."""
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    tdist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from streaming_causal_video_timestep_b200.tpp import DistTransport, TppRank
+        from workloads import make_weights
+        groups = [tdist.new_group(list(range(p * steps, (p + 1) * steps))) for p in range(world // steps)]
+        pid, r = rank // steps, rank % steps
+        wl = _workload(True, False, steps=steps, seed=3 + pid)
+        W = make_weights(wl)
+        tr = DistTransport(r, steps, "cpu", group=groups[pid], base=pid * steps)
+        me = TppRank(OracleSlot(wl, W, r), r, steps, tr, "cpu", steps, wl.cfg.sink_tokens, True)
+        done = {}
+        for item in _inputs(wl):
+            x_new = item[0] if (item is not None and r == 0) else None
+            blk, lat = me.tick(x_new)
+            if blk >= 0:
+                done[blk] = lat.numpy().copy()
+        me.close()
+        tdist.barrier()
+        if r == steps - 1:
+            want = _single_process(wl, W)
+            out[pid] = (sorted(done), max(float(np.abs(done[b] - want[b]).max()) for b in want))
+    finally:
+        tdist.destroy_process_group()
+
+
+def test_tpp_two_gloo_ranks_aas_broadcast_matches_the_pipelined_stream():
+    """Two ranks, two denoising steps: block 0 leaves the last rank at tick 1 and its
+    frame 0 is broadcast before tick 2, the single-process pipeline's AAS timing."""
+    port = _free_port()
+    out = mp.get_context("spawn").Manager().dict()
+    mp.spawn(_pipelines_main, args=(2, 2, port, out), nprocs=2, join=True)
+    blocks, err = out[0]
+    assert blocks == list(range(6))
+    assert err < 2e-6
+
+
+def test_tpp_two_pipelines_in_one_job_over_their_own_groups():
+    """Four gloo ranks as two 2-step pipelines (global ranks 0-1 and 2-3), as bench.py
+    runs 8 GPUs as two 4-step pipelines: each matches the oracle on its own workload."""
+    port = _free_port()
+    out = mp.get_context("spawn").Manager().dict()
+    mp.spawn(_pipelines_main, args=(4, 2, port, out), nprocs=4, join=True)
+    for pid in (0, 1):
+        blocks, err = out[pid]
+        assert blocks == list(range(6))
+        assert err < 2e-6
