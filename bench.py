@@ -114,7 +114,7 @@ def _peaks():
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
-def append_marginal(qkv_kind, S, T, D, iters=20):
+def append_marginal(qkv_kind, S, T, D, iters=200):
     """The Rolling RoPE + ring append runs as the epilogue of the QKV GEMM.  Its
     cost is the difference between that GEMM, as the stream times it (all S
     slots' rows, M = S T, N = 3D, K = D), and a plain bf16 store of the same GEMM
