@@ -388,6 +388,75 @@ __device__ __forceinline__ void epilogue_row32(const GemmEpiParams& ep, long lon
   }
 }
 
+// Tensor-memory address of an epilogue warp's lane quarter in accumulator column col0.
+__device__ __forceinline__ uint32_t tbase_of(uint32_t tmem, int quarter, int col0) {
+  return tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(col0);
+}
+
+// The epilogue of one 128 x BN accumulator tile in tensor memory (tbase: this
+// warp's lane quarter, column 0 of the tile) for rows row_base .. row_base+127
+// and column block nb: one epilogue warp takes rows 32*quarter .. +31.
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(const GemmEpiParams& ep, const QkvRopeParams& qp, int M, int N,
+                                              uint32_t tbase, long long row_base, int nb, int quarter, int lane,
+                                              uint8_t* epi_stage, bool staged_kind, bool segment_kind,
+                                              bool seg_e4m3) {
+  const int rit = quarter * 32 + lane;
+  const long long row = row_base + rit;
+  const long long row0 = row_base + quarter * 32;
+  const bool staged = staged_kind && row0 + 32 <= M;
+  QkvRow qr{};
+  if (ep.kind == EPI_QKV_ROPE && row < M) qr = qkv_row_info(qp, row);
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    uint32_t r[32];
+    tmem_ld32(tbase + c0, r);
+    tmem_ld_wait();
+    const long long col = static_cast<long long>(nb) * BN + c0;
+    if (segment_kind && col + 32 <= N) {
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      uint32_t w[16];
+      void* dst = nullptr;
+      if (row < M) {
+        if (ep.row_scale) {
+          apply_operand_scales(ep, row, col, v);
+        }
+        dst = segment_words(ep, qp, qr, row, col, v, w);
+      }
+      if (seg_e4m3)
+        store_row_words_staged<8>(dst, w, epi_stage, lane);
+      else
+        store_row_words_staged<16>(dst, w, epi_stage, lane);
+    } else if (staged && col + 32 <= N) {
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      if (ep.row_scale) {
+        apply_operand_scales(ep, row, col, v);
+      }
+      if (ep.kind == EPI_RESID_GATED)
+        epilogue_resid_warp<true>(ep, row0, col, v, epi_stage, lane);
+      else
+        epilogue_resid_warp<false>(ep, row0, col, v, epi_stage, lane);
+    } else if (row < M && col < N) {
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      if (ep.row_scale) {
+        apply_operand_scales(ep, row, col, v);
+      }
+      if (segment_kind) {
+        uint32_t w[16];
+        store_row_words_direct(segment_words(ep, qp, qr, row, col, v, w), w, seg_e4m3 ? 8 : 16);
+      } else {
+        epilogue_row32(ep, row, col, v);
+      }
+    }
+  }
+}
+
 template <int BN, bool FP8>
 __global__ void __launch_bounds__(192, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -501,7 +570,6 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     }
   } else {
     const int quarter = warp & 3;
-    const int rit = quarter * 32 + lane;
     uint8_t* epi_stage = smem + C::STAGES * C::STAGE_BYTES + 256 + (warp - 2) * EPI_WARP_BYTES;
     // the residual kinds take the staged path when the warp's 32 rows are all in
     // range and h32 / out rows start on 16-byte boundaries
@@ -520,60 +588,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       tile_coords(tile, num_m, num_n, mb, nb);
       if (!mbar_wait(&tfull[acc], acc_phase, err)) { abort_flag = 1; break; }
       tc_fence_after();
-      const long long row = static_cast<long long>(mb) * BM + rit;
-      const long long row0 = static_cast<long long>(mb) * BM + quarter * 32;
-      const bool staged = staged_kind && row0 + 32 <= M;
-      QkvRow qr{};
-      if (ep.kind == EPI_QKV_ROPE && row < M) qr = qkv_row_info(qp, row);
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tbase + c0, r);
-        tmem_ld_wait();
-        const long long col = static_cast<long long>(nb) * BN + c0;
-        if (segment_kind && col + 32 <= N) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          uint32_t w[16];
-          void* dst = nullptr;
-          if (row < M) {
-            if (ep.row_scale) {
-              apply_operand_scales(ep, row, col, v);
-            }
-            dst = segment_words(ep, qp, qr, row, col, v, w);
-          }
-          if (seg_e4m3)
-            store_row_words_staged<8>(dst, w, epi_stage, lane);
-          else
-            store_row_words_staged<16>(dst, w, epi_stage, lane);
-        } else if (staged && col + 32 <= N) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          if (ep.row_scale) {
-            apply_operand_scales(ep, row, col, v);
-          }
-          if (ep.kind == EPI_RESID_GATED)
-            epilogue_resid_warp<true>(ep, row0, col, v, epi_stage, lane);
-          else
-            epilogue_resid_warp<false>(ep, row0, col, v, epi_stage, lane);
-        } else if (row < M && col < N) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          if (ep.row_scale) {
-            apply_operand_scales(ep, row, col, v);
-          }
-          if (segment_kind) {
-            uint32_t w[16];
-            store_row_words_direct(segment_words(ep, qp, qr, row, col, v, w), w, seg_e4m3 ? 8 : 16);
-          } else {
-            epilogue_row32(ep, row, col, v);
-          }
-        }
-      }
+      epilogue_tile<BN>(ep, qp, M, N, tbase_of(tmem, quarter, acc * BN), static_cast<long long>(mb) * BM, nb,
+                        quarter, lane, epi_stage, staged_kind, segment_kind, seg_e4m3);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -587,6 +603,227 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// ---------------------------------------------------------------------------
+// The same GEMM on CTA pairs (bf16, BN = 256): a cluster of two CTAs computes a
+// 256 x BN tile with tcgen05.mma.cta_group::2 (M = 256), CTA r holding rows
+// 128r .. 128r+127 of A and columns BN/2 r .. of W in its shared memory (the
+// tensor cores exchange the W halves), so each CTA stages 16 KB of A and 16 KB
+// of W a k-block and the ring is PAIR_STAGES deep in the same shared memory.
+// Each CTA's tensor memory holds its 128 rows of the two BN-column
+// accumulators, and its epilogue warps run epilogue_tile on them as above.
+//   warp 0 (both CTAs)   TMA producer; the copies complete on the leader's
+//                        (even CTA's) full[] barriers, which expect both CTAs'
+//                        bytes (the cta_group::2 copy form, no multicast);
+//   warp 1 (leader)      issues the MMAs; its commits release empty[] and
+//                        tfull[] in both CTAs;
+//   warps 2-5 (both)     epilogue; each warp hands its accumulator back on the
+//                        leader's tempty[] (8 arrivals).
+// Every wait is bounded; a wait that gives up raises the device error word and
+// sets both CTAs' abort flags, and both CTAs meet at the final cluster barrier.
+constexpr int PAIR_STAGES = 6;
+
+template <int BN>
+struct PairCfg {
+  static constexpr uint32_t A_BYTES = BM * BK_BYTES;            // this CTA's 128 rows
+  static constexpr uint32_t B_BYTES = (BN / 2) * BK_BYTES;      // this CTA's BN/2 columns
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr size_t SMEM = 1024 + PAIR_STAGES * STAGE_BYTES + 256 + 4 * EPI_WARP_BYTES;
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+template <int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const __grid_constant__ GemmEpiParams ep, const __grid_constant__ QkvRopeParams qp, int M, int N, int K,
+            int* err) {
+  using C = PairCfg<BN>;
+  constexpr int ST = PAIR_STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + ST * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES);
+  uint64_t* empty = full + ST;
+  uint64_t* tfull = empty + ST;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ volatile int abort_flag;
+
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);   // one arrive per epilogue warp of each CTA
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    tma_prefetch_map(&tmA);
+    tma_prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t abort_peer = smem_peer(const_cast<int*>(&abort_flag), rank ^ 1u);
+  auto set_abort = [&]() {
+    abort_flag = 1;
+    st_cluster_u32(abort_peer, 1u);
+  };
+
+  const int num_m = (M + 2 * BM - 1) / (2 * BM);
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  constexpr int BK = 64;
+  const int kblocks = (K + BK - 1) / BK;
+  constexpr uint32_t idesc = idesc_bf16(2 * BM, BN, false, false);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[ST];
+      for (int i = 0; i < ST; ++i) last_parity[i] = -1;
+      for (int tile = pair; tile < num_tiles && !abort_flag; tile += npairs) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, mb, nb);
+        const int arow = mb * 2 * BM + static_cast<int>(rank) * BM;
+        const int brow = nb * BN + static_cast<int>(rank) * (BN / 2);
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, err)) { ok = false; break; }
+          const uint32_t bar = smem_peer(&full[stage], 0);
+          if (leader) mbar_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kb * BK, arow);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kb * BK, brow);
+          last_parity[stage] = static_cast<int>(phase);
+          if (++stage == ST) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) { set_abort(); break; }
+      }
+      // the leader's full[] phases count both CTAs' bytes: every issued copy has
+      // landed once they complete (at once on the normal path)
+      if (leader)
+        for (int i = 0; i < ST; ++i)
+          if (last_parity[i] >= 0) mbar_wait(&full[i], static_cast<uint32_t>(last_parity[i]), err);
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tile = pair; tile < num_tiles; tile += npairs) {
+        if (abort_flag) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, err)) { set_abort(); break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK_BYTES / 32; ++kk)
+            umma_bf16_ss_pair(d_tmem, sdesc_kmajor(a0 + kk * 32), sdesc_kmajor(b0 + kk * 32), idesc,
+                              (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == ST) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) { set_abort(); break; }
+        umma_commit_pair_mc(&tfull[acc], 0x3);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      // all issued MMAs complete before either CTA releases its tensor memory
+      umma_commit_pair(drain);
+      mbar_wait(drain, 0, err);
+    }
+  } else {
+    const int quarter = warp & 3;
+    uint8_t* epi_stage = smem + ST * C::STAGE_BYTES + 256 + (warp - 2) * EPI_WARP_BYTES;
+    const bool staged_kind = (ep.kind == EPI_RESID || ep.kind == EPI_RESID_GATED) && (ep.ld % 8) == 0 &&
+                             (reinterpret_cast<uintptr_t>(ep.h32) & 15) == 0 &&
+                             (reinterpret_cast<uintptr_t>(ep.out) & 15) == 0;
+    const bool segment_kind = ep.kind == EPI_STORE || ep.kind == EPI_GELU || ep.kind == EPI_QKV_ROPE;
+    const bool seg_e4m3 = ep.kind == EPI_QKV_ROPE && qp.fp8_inv != nullptr;
+    const uint32_t tempty_leader = smem_peer(&tempty[0], 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs) {
+      if (abort_flag) break;
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, mb, nb);
+      if (!mbar_wait(&tfull[acc], acc_phase, err)) { set_abort(); break; }
+      tc_fence_after();
+      epilogue_tile<BN>(ep, qp, M, N, tbase_of(tmem, quarter, acc * BN),
+                        static_cast<long long>(mb) * 2 * BM + static_cast<long long>(rank) * BM, nb, quarter, lane,
+                        epi_stage, staged_kind, segment_kind, seg_e4m3);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&tempty[acc]);
+        else
+          mbar_arrive_remote(tempty_leader + acc * 8);
+      }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();          // the leader's MMAs into the follower's tensor memory are done
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN>
+cudaError_t launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep,
+                        const QkvRopeParams& qp, int M, int N, int K, int* err, int num_sms, cudaStream_t st) {
+  using C = PairCfg<BN>;
+  auto kern = k_gemm_pair<BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
+  if (e != cudaSuccess) return e;
+  // persistent: as many pairs as can be resident at once (one CTA an SM), at most one a tile
+  static int max_pairs = -1;
+  if (max_pairs < 0) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * (num_sms / 2));
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    max_pairs = (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) ? n : num_sms / 2;
+    cudaGetLastError();
+  }
+  const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN);
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  kern<<<2 * pairs, 192, C::SMEM, st>>>(tmA, tmB, ep, qp, M, N, K, err);
+  return cudaGetLastError();
 }
 
 template <int BN, bool FP8>
@@ -604,6 +841,8 @@ cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const Gemm
 
 }  // namespace
 
+int gemm_tc_b_box_rows(int bn) { return bn == 256 ? bn / 2 : bn; }
+
 int gemm_tc_pick_bn(int N) {
   if (N % 256 == 0 && N >= 1024) return 256;
   if (N % 128 == 0) return 128;
@@ -615,7 +854,7 @@ cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const
   QkvRopeParams none{};
   const QkvRopeParams& q = qp ? *qp : none;
   switch (bn) {
-    case 256: return launch_bn<256, false>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
+    case 256: return launch_pair<256>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
     case 128: return launch_bn<128, false>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
     default: return launch_bn<64, false>(tmA, tmB, ep, q, M, N, K, err, num_sms, st);
   }

@@ -12,6 +12,9 @@ int op_error_word(int** out);
 
 // ---- tcgen05 (bf16) ----------------------------------------------------------------
 int gemm_tc_pick_bn(int N);
+// Rows of the W box of a bf16 tensor map for launch_gemm_tc with that bn: the
+// bn = 256 tiles run on CTA pairs, each CTA loading half of the tile's W rows.
+int gemm_tc_b_box_rows(int bn);
 // qp: parameters of the EPI_QKV_ROPE epilogue (NULL for the others).
 cudaError_t launch_gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmEpiParams& ep, int M, int N,
                            int K, int bn, int* err, int num_sms, cudaStream_t st, const QkvRopeParams* qp = nullptr);

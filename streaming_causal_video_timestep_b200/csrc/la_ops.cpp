@@ -47,7 +47,7 @@ int la_op_gemm(int32_t dtype, int32_t epilogue, const void* A, const void* W, vo
     if (!tmap_init(err)) return LA_ECUDA;
     const int bn = gemm_tc_pick_bn(static_cast<int>(N));
     CUtensorMap ta, tb;
-    if (!tmap_2d_bf16(&ta, A, M, K, K, 128, err) || !tmap_2d_bf16(&tb, W, N, K, K, bn, err)) return LA_ECUDA;
+    if (!tmap_2d_bf16(&ta, A, M, K, K, 128, err) || !tmap_2d_bf16(&tb, W, N, K, K, gemm_tc_b_box_rows(bn), err)) return LA_ECUDA;
     int* dev_err = nullptr;
     if (op_error_word(&dev_err) != LA_OK) return LA_ECUDA;
     return ret(launch_gemm_tc(ta, tb, ep, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), bn, dev_err,

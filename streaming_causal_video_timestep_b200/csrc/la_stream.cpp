@@ -1292,8 +1292,8 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
     s->tm_wqkv.resize(L);
     s->tm_wout.resize(L);
     for (int l = 0; l < L && ok; ++l) {
-      ok = ok && tmap_2d_bf16(&s->tm_wqkv[l], s->w_qkv[l], 3 * D, D, D, bn_qkv, s->err);
-      ok = ok && tmap_2d_bf16(&s->tm_wout[l], s->w_out[l], D, D, D, bn_d, s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_wqkv[l], s->w_qkv[l], 3 * D, D, D, gemm_tc_b_box_rows(bn_qkv), s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_wout[l], s->w_out[l], D, D, D, gemm_tc_b_box_rows(bn_d), s->err);
     }
     if (s->dit) {
       const long long Ff = s->Fffn;
@@ -1302,8 +1302,8 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
       s->tm_w1.resize(L);
       s->tm_w2.resize(L);
       for (int l = 0; l < L && ok; ++l) {
-        ok = ok && tmap_2d_bf16(&s->tm_w1[l], s->w_ffn1[l], Ff, D, D, gemm_tc_pick_bn(s->Fffn), s->err);
-        ok = ok && tmap_2d_bf16(&s->tm_w2[l], s->w_ffn2[l], D, Ff, Ff, bn_d, s->err);
+        ok = ok && tmap_2d_bf16(&s->tm_w1[l], s->w_ffn1[l], Ff, D, D, gemm_tc_b_box_rows(gemm_tc_pick_bn(s->Fffn)), s->err);
+        ok = ok && tmap_2d_bf16(&s->tm_w2[l], s->w_ffn2[l], D, Ff, Ff, gemm_tc_b_box_rows(bn_d), s->err);
       }
     }
     if (s->cross) {
@@ -1314,9 +1314,9 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
       s->tm_wkvc.resize(L);
       s->tm_woc.resize(L);
       for (int l = 0; l < L && ok; ++l) {
-        ok = ok && tmap_2d_bf16(&s->tm_wqc[l], s->w_qc[l], D, D, D, bn_d, s->err);
-        ok = ok && tmap_2d_bf16(&s->tm_wkvc[l], s->w_kvc[l], 2 * D, s->Da, s->Da, gemm_tc_pick_bn(2 * s->D), s->err);
-        ok = ok && tmap_2d_bf16(&s->tm_woc[l], s->w_oc[l], D, D, D, bn_d, s->err);
+        ok = ok && tmap_2d_bf16(&s->tm_wqc[l], s->w_qc[l], D, D, D, gemm_tc_b_box_rows(bn_d), s->err);
+        ok = ok && tmap_2d_bf16(&s->tm_wkvc[l], s->w_kvc[l], 2 * D, s->Da, s->Da, gemm_tc_b_box_rows(gemm_tc_pick_bn(2 * s->D)), s->err);
+        ok = ok && tmap_2d_bf16(&s->tm_woc[l], s->w_oc[l], D, D, D, gemm_tc_b_box_rows(bn_d), s->err);
       }
       ok = ok && tmap_planes_bf16(&s->maps_cross.q, s->qc_heads, d, T, H, NB, s->err);
       ok = ok && tmap_planes_bf16(&s->maps_cross.k[0], s->audio_k, d, Aa, H, L * NB, s->err);
@@ -1325,8 +1325,8 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
     if (!s->id_in) {
       ok = ok && tmap_2d_bf16(&s->tm_xop, s->xop, NB * T, C, C, 128, s->err);
       ok = ok && tmap_2d_bf16(&s->tm_s_xop, s->s_xop, F, C, C, 128, s->err);
-      ok = ok && tmap_2d_bf16(&s->tm_win, s->w_in, D, C, C, bn_d, s->err);
-      ok = ok && tmap_2d_bf16(&s->tm_whead, s->w_head, C, D, D, bn_c, s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_win, s->w_in, D, C, C, gemm_tc_b_box_rows(bn_d), s->err);
+      ok = ok && tmap_2d_bf16(&s->tm_whead, s->w_head, C, D, D, gemm_tc_b_box_rows(bn_c), s->err);
     }
     if (s->afp8) {
       ok = ok && tmap_planes_u8(&s->maps_stream.q, s->q_rope, d, T, H, NB, s->err);

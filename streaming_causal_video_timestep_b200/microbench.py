@@ -4,7 +4,7 @@
     python -m streaming_causal_video_timestep_b200.microbench gemm  [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench gemm_out [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench euler [--iters N]
-    python -m streaming_causal_video_timestep_b200.microbench rerope [--iters N]
+    python -m streaming_causal_video_timestep_b200.microbench rerope [--iters N] [--layers L]
     python -m streaming_causal_video_timestep_b200.microbench gemm_fp8 [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench attn_fp8 [--iters N]
 
@@ -155,10 +155,10 @@ def bench_euler(iters):
             "bytes": nbytes}
 
 
-def bench_rerope(iters):
+def bench_rerope(iters, layers=8):
     from types import SimpleNamespace
     from .stream import LaStream
-    cfg = SimpleNamespace(num_layers=8, hidden=5120, heads=40, head_dim=128, latent_ch=64, grid_h=30, grid_w=52,
+    cfg = SimpleNamespace(num_layers=layers, hidden=5120, heads=40, head_dim=128, latent_ch=64, grid_h=30, grid_w=52,
                           frames_per_block=3, sink_frames=1, window_blocks=1, timesteps=(1.0, 0.75, 0.5, 0.25, 0.0),
                           rope_split=(22, 21, 21), pairs=(22, 21, 21), rope_theta=10000.0, sink_mode=0, rolling_rope=1,
                           sink_offset_frames=3, schedule=0, dtype=0)
@@ -193,13 +193,15 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("mode", choices=["attn", "attn_fp8", "gemm", "gemm_out", "euler", "rerope", "gemm_fp8", "all"])
     ap.add_argument("--iters", type=int, default=10)
+    ap.add_argument("--layers", type=int, default=8, help="rerope: sublayers of the stream (one launch covers all)")
     args = ap.parse_args()
     modes = ["attn", "attn_fp8", "gemm", "gemm_out", "gemm_fp8", "euler", "rerope"] if args.mode == "all" else [args.mode]
     for m in modes:
         clocks = ClockSampler(torch.cuda.current_device())
         clocks.start()
         r = {"attn": bench_attn, "attn_fp8": bench_attn_fp8, "gemm": bench_gemm, "gemm_out": bench_gemm_out,
-             "euler": bench_euler, "rerope": bench_rerope, "gemm_fp8": bench_gemm_fp8}[m](args.iters)
+             "euler": bench_euler, "rerope": lambda it: bench_rerope(it, args.layers),
+             "gemm_fp8": bench_gemm_fp8}[m](args.iters)
         r["clocks"] = clocks.stop()
         print(json.dumps(r), flush=True)
 

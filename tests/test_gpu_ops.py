@@ -31,7 +31,9 @@ def _np(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-GEMM_SHAPES = [(300, 256, 320), (130, 64, 64), (1000, 1536, 512), (4680 + 37, 192, 64), (17, 512, 1024)]
+# N = 256 multiples >= 1024 run on CTA pairs (256-row tiles); the others on one CTA
+GEMM_SHAPES = [(300, 256, 320), (130, 64, 64), (1000, 1536, 512), (4680 + 37, 192, 64), (17, 512, 1024),
+               (17, 1024, 128), (129, 2048, 192), (4680 + 37, 1024, 320), (300, 5120, 64)]
 
 
 @pytest.mark.parametrize("dtype", [DTYPE_BF16, DTYPE_FP32])
@@ -62,10 +64,11 @@ def test_gemm_store_and_resid(dtype, M, N, K):
 
 
 @pytest.mark.parametrize("dtype", [DTYPE_BF16, DTYPE_FP32])
-def test_gemm_set32_and_euler_epilogues(dtype):
+@pytest.mark.parametrize("N", [64, 1024])
+def test_gemm_set32_and_euler_epilogues(dtype, N):
     from streaming_causal_video_timestep_b200 import op_gemm
     rnd = bf16_round if dtype == DTYPE_BF16 else (lambda a: a.astype(np.float32))
-    M, N, K, G = 4 * 180, 64, 256, 4
+    M, K, G = 4 * 180, 256, 4
     A = rnd(random_array(1, (M, K)))
     W = rnd(random_array(2, (N, K), scale=0.05))
     ref = A.astype(np.float64) @ W.astype(np.float64).T
