@@ -9,7 +9,8 @@
 //                64-column 128-byte-swizzled boxes: a 2-stage ring for bf16,
 //                4 stages for e4m3, see kv_stages());
 //                warp 1: TMEM owner (512 columns: S_A | S_B | O_A | O_B) and
-//                MMA issuer; warps 2-3 idle.  Drops to 56 registers a thread.
+//                MMA issuer (the whole warp waits, one elected lane issues);
+//                warps 2-3 idle.  Drops to 56 registers a thread.
 //   warpgroup 1  softmax of tile A, warpgroup 2 softmax of tile B: one thread
 //                per query row (= TMEM lane).  Raised to 224 registers a thread
 //                so that a row's 128 scores of a key tile stay in registers
@@ -313,8 +314,12 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
       mbar_wait(q_full, 0, err);
       for (int i = 0; i < NS; ++i)
         if (last_parity[i] >= 0) mbar_wait(&kv_full[i], static_cast<uint32_t>(last_parity[i]), err);
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
       // -------------------------------------------------------------- MMA issuer
+      // The whole warp runs the loop and waits (one outcome for all lanes), and
+      // one elected lane issues the MMAs and commits: measured 9-12 % faster per
+      // clock than the same loop run by a single thread.
+      auto wwait = [&](uint64_t* bar, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(bar, par, err)); };
       // The tensor core queues only a few MMAs, so the issue loop is kept lean:
       // descriptors are precomputed and advanced by adding offsets, pv_done is
       // committed only for the last key tile (the commit of S(t) already covers
@@ -346,21 +351,25 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
         }
         umma_commit(&s_full[w]);
       };
-      bool ok = mbar_wait(q_full, 0, err) && (nt == 0 || mbar_wait(&kv_full[0], 0, err));
+      bool ok = wwait(q_full, 0) && (nt == 0 || wwait(&kv_full[0], 0));
       if (ok && nt > 0) {
         tc_fence_after();
-        for (int w = 0; w < nq; ++w) issue_s(w, 0);
-        umma_commit(&kv_empty[0]);
+        if (elect_one()) {
+          for (int w = 0; w < nq; ++w) issue_s(w, 0);
+          umma_commit(&kv_empty[0]);
+        }
+        __syncwarp();
       }
       // step t reads ring step t+1 = [V(t) | K(t+1)]: stage (t+1) % NS, phase ((t+1) / NS) & 1
       uint32_t vs = 1 % NS, vpar = (1 / NS) & 1;
       for (int t = 0; t < nt && ok; ++t) {
         const bool more = t + 1 < nt;
-        ok = mbar_wait(&kv_full[vs], vpar, err);
+        ok = wwait(&kv_full[vs], vpar);
         if (!ok) break;
         for (int w = 0; w < nq; ++w) {
-          if (!mbar_wait(&p_full[w], static_cast<uint32_t>(t & 1), err)) { ok = false; break; }
+          if (!wwait(&p_full[w], static_cast<uint32_t>(t & 1))) { ok = false; break; }
           tc_fence_after();
+          if (elect_one()) {
           // One K step is 8 tensor-memory columns of P (16 bf16 or 32 e4m3 keys)
           // and 16 or 32 key rows of the V tile (128 bytes each).
           if (FP8) {
@@ -378,14 +387,18 @@ k_attn_tc(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnPar
             issue_s(w, vs);
           else
             umma_commit(&pv_done[w]);
+          }
+          __syncwarp();
         }
         if (!ok) break;
-        umma_commit(&kv_empty[vs]);
+        if (elect_one()) umma_commit(&kv_empty[vs]);
+        __syncwarp();
         if (++vs == NS) { vs = 0; vpar ^= 1u; }
       }
       if (!ok) abort_flag = 1;
-      umma_commit(drain);
-      mbar_wait(drain, 0, err);
+      if (elect_one()) umma_commit(drain);
+      __syncwarp();
+      wwait(drain, 0);
     }
   } else {
     regs_inc<REGS_HIGH>();
