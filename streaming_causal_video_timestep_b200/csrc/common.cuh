@@ -113,6 +113,12 @@ struct GemmEpiParams {
   const float* row_scale;   // optional [M]: acc *= row_scale[row] * col_scale[col] first (FP8 operands)
   const float* col_scale;   // [N], set together with row_scale
   const float* gate[LA_MAX_STEPS];   // RESID_GATED: per row group, [N]
+  // The per-token RMS norm folded into the GEMMs (n(h) W^T = diag(1 / rms(h)) (h W^T)):
+  float* ssq_out;        // optional [M][ssq_ld]: each row's sum of squares of the new values over this
+                         // tile's BN columns, at column-tile index (SET32 / RESID kinds)
+  const float* ssq_in;   // optional [M][ssq_ld]: acc *= 1 / sqrt(sum_j ssq_in[row][j] / ssq_n + 1e-6) first
+  int ssq_ld;            // partial sums a row (column tiles of the producing GEMM)
+  float ssq_n;           // values a row the mean is over
 };
 
 // tanh-approximated GELU: u/2 (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))).

@@ -407,6 +407,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmEpiParams& ep, const Qkv
   const bool staged = staged_kind && row0 + 32 <= M;
   QkvRow qr{};
   if (ep.kind == EPI_QKV_ROPE && row < M) qr = qkv_row_info(qp, row);
+  // the row's RMS norm from the partial sums the producing GEMM left (folded norm)
+  float inv_rms = 1.0f;
+  if (ep.ssq_in && row < M) {
+    float t = 0.f;
+    for (int j = 0; j < ep.ssq_ld; ++j) t += ep.ssq_in[row * ep.ssq_ld + j];
+    inv_rms = rsqrtf(t / ep.ssq_n + 1e-6f);
+  }
+  float ss = 0.f;              // sum of squares of the row's new values over this tile
 #pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += 32) {
     uint32_t r[32];
@@ -416,7 +424,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmEpiParams& ep, const Qkv
     if (segment_kind && col + 32 <= N) {
       float v[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * inv_rms;
       uint32_t w[16];
       void* dst = nullptr;
       if (row < M) {
@@ -432,7 +440,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmEpiParams& ep, const Qkv
     } else if (staged && col + 32 <= N) {
       float v[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * inv_rms;
       if (ep.row_scale) {
         apply_operand_scales(ep, row, col, v);
       }
@@ -440,10 +448,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmEpiParams& ep, const Qkv
         epilogue_resid_warp<true>(ep, row0, col, v, epi_stage, lane);
       else
         epilogue_resid_warp<false>(ep, row0, col, v, epi_stage, lane);
+      if (ep.ssq_out) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);   // v now holds the row's new values
+      }
     } else if (row < M && col < N) {
       float v[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * inv_rms;
       if (ep.row_scale) {
         apply_operand_scales(ep, row, col, v);
       }
@@ -452,9 +464,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmEpiParams& ep, const Qkv
         store_row_words_direct(segment_words(ep, qp, qr, row, col, v, w), w, seg_e4m3 ? 8 : 16);
       } else {
         epilogue_row32(ep, row, col, v);
+        if (ep.ssq_out) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);   // SET32 / RESID leave the new values in v
+        }
       }
     }
   }
+  if (ep.ssq_out && row < M) ep.ssq_out[row * ep.ssq_ld + nb] = ss;
 }
 
 template <int BN, bool FP8>

@@ -199,7 +199,14 @@ struct la_stream {
   std::vector<void*> allocs;
   float* xs = nullptr;      // [nbuf][T][C]
   float* h32 = nullptr;     // [nbuf*T][D] residual stream
-  void* hop = nullptr;      // [nbuf*T][D] normalised GEMM operand, dtype (fp32: == hn32)
+  void* hop = nullptr;      // [nbuf*T][D] normalised GEMM operand, dtype (fp32: == hn32); with the folded
+                            // norm, the residual itself rounded to bf16
+  // The per-token RMS norm folded into the GEMMs (bf16 attention sublayers with an in-projection and a
+  // head, no e4m3 projections): the in- and output projections' epilogues leave each row's sum of squares
+  // per column tile in ssq, and the QKV and head epilogues scale their rows by 1 / rms from it.
+  bool fold = false;
+  float* ssq = nullptr;     // [nbuf*T][ssq_ld]
+  int ssq_ld = 0;
   float* hn32 = nullptr;    // [nbuf*T][D] fp32 normalised residual (fp32 streams, identity head)
   void* xop = nullptr;      // [nbuf*T][C] bf16 (bf16 with an in-projection)
   float* qkv = nullptr;     // fp32 [nbuf*T][3D] (fp32 streams; bf16 fuses it into the GEMM)
@@ -453,6 +460,20 @@ int gemm(la_stream* s, int kind, const CUtensorMap* tmA, const CUtensorMap* tmB,
   });
 }
 
+// The folded norm: a GEMM whose epilogue produces the residual leaves each row's
+// partial sums of squares; one that consumes its operand scales rows by 1 / rms.
+void fold_out(la_stream* s, GemmEpiParams& e) {
+  if (!s->fold) return;
+  e.ssq_out = s->ssq;
+  e.ssq_ld = s->ssq_ld;
+}
+void fold_in(la_stream* s, GemmEpiParams& e) {
+  if (!s->fold) return;
+  e.ssq_in = s->ssq;
+  e.ssq_ld = s->ssq_ld;
+  e.ssq_n = static_cast<float>(s->D);
+}
+
 GemmEpiParams epi(int kind, void* out, float* h32, long long ld) {
   GemmEpiParams e{};
   e.kind = kind;
@@ -689,14 +710,16 @@ int run_pass(la_stream* s, const PassDesc& pd) {
            return launch_cvt_bf16(s->xs, s->xop, static_cast<long long>(rows) * C, s->st);
          })) != LA_OK)
       return r;
-    GemmEpiParams e = epi(EPI_SET32, nullptr, s->h32, D);
+    GemmEpiParams e = epi(EPI_SET32, s->fold ? s->hop : nullptr, s->h32, D);
+    fold_out(s, e);
     if ((r = gemm(s, LA_KIND_IN_PROJ, &s->tm_xop, &s->tm_win, s->xs, s->w_in, e, rows, D, C)) != LA_OK) return r;
   }
   if (s->capture && (r = capture_pass(s, pd, -1)) != LA_OK) return r;
   // timestep index of each buffer's AdaLN vectors (the DiT block)
   int tidx[LA_MAX_STEPS] = {};
   for (int b = 0; b < pd.nbuf; ++b) tidx[b] = pd.active[b] ? std::min(pd.step[b], S) : 0;
-  if (!s->dit && (r = normalise(s, s->h32, rows, s->hop, s->bf16 ? nullptr : s->hn32)) != LA_OK) return r;
+  if (!s->dit && !s->fold && (r = normalise(s, s->h32, rows, s->hop, s->bf16 ? nullptr : s->hn32)) != LA_OK)
+    return r;
 
   RopeArgs ra = rope_args(s);
   AttnParams ap{};
@@ -762,6 +785,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
       // QKV projection with Rolling RoPE + ring append fused into the epilogue
       qp.ring_slice0 = ra.ring_slice0;
       GemmEpiParams eq = epi(EPI_QKV_ROPE, nullptr, nullptr, 3LL * D);
+      fold_in(s, eq);
       const int bn = gemm_tc_pick_bn(3 * D);
       if (s->fp8) {
         if ((r = proj_fp8(s, LA_KIND_QKV_GEMM, s->hop, s->tm_a8, s->tm_wq8[l], s->wq8s[l], eq, rows, 3 * D, D, &qp)) !=
@@ -803,7 +827,8 @@ int run_pass(la_stream* s, const PassDesc& pd) {
       if ((r = launch(s, LA_KIND_ATTN, [&] { return launch_attn_f32(ap, s->st); })) != LA_OK) return r;
     }
     // output projection + residual, then the next operand (next layer or head)
-    GemmEpiParams eo = epi(EPI_RESID, nullptr, s->h32, D);
+    GemmEpiParams eo = epi(EPI_RESID, s->fold ? s->hop : nullptr, s->h32, D);
+    fold_out(s, eo);
     if (s->dit) set_gates(s, eo, T, tidx, pd.nbuf, l, 2);
     if (s->fp8) {
       if ((r = proj_fp8(s, LA_KIND_OUT_GEMM, s->attn_o, s->tm_a8, s->tm_wo8[l], s->wo8s[l], eo, rows, D, D)) != LA_OK)
@@ -837,7 +862,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
     if (s->capture && (r = capture_pass(s, pd, l)) != LA_OK) return r;
     const bool last = l == s->L - 1;
     const bool want_f32 = !s->bf16 || (last && s->id_head);
-    if ((!s->dit || last) &&
+    if ((!s->dit || last) && !s->fold &&
         (r = normalise(s, s->h32, rows, (s->bf16 && !(last && s->id_head)) ? s->hop : nullptr,
                        want_f32 ? s->hn32 : nullptr)) != LA_OK)
       return r;
@@ -858,6 +883,7 @@ int run_pass(la_stream* s, const PassDesc& pd) {
       e.active[i] = pd.active[i];
     }
     e.vtap = vtap;
+    fold_in(s, e);
     if ((r = gemm(s, LA_KIND_HEAD, &s->tm_hop, &s->tm_whead, s->hn32, s->w_head, e, rows, C, D)) != LA_OK)
       return r;
   }
@@ -1152,6 +1178,8 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   s->Da = s->cross ? cfg->audio_dim : 0;
   s->eq = s->afp8 ? 1 : s->ea;
   s->id_in = w->w_in == nullptr; s->id_head = w->w_head == nullptr;
+  s->fold = s->bf16 && !s->fp8 && !s->dit && !s->id_in && !s->id_head;
+  s->ssq_ld = s->fold ? ceil_div_i(s->D, gemm_tc_pick_bn(s->D)) : 0;
   s->nbuf = cfg->schedule == LA_SCHED_PIPELINED ? s->S : 1;
   s->st = static_cast<cudaStream_t>(cuda_stream);
   s->w_in = w->w_in; s->w_head = w->w_head;
@@ -1216,6 +1244,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   if (!s->bf16) ALLOC_OR_BAIL(s->qkv, NB * T * 3 * D * 4);
   ALLOC_OR_BAIL(s->q_rope, NB * T * D * eq);
   ALLOC_OR_BAIL(s->attn_o, NB * T * D * es);
+  if (s->fold) ALLOC_OR_BAIL(s->ssq, NB * T * s->ssq_ld * 4);
   ALLOC_OR_BAIL(s->sk_rope, L * NB * H * F * d * eq);
   ALLOC_OR_BAIL(s->ring_k, L * S * E * H * T * d * eq);
   ALLOC_OR_BAIL(s->ring_v, L * S * E * H * T * d * eq);

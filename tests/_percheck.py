@@ -14,7 +14,7 @@ import numpy as np
 
 import math
 
-from oracle import block_causal_attention, euler_step, rms_norm, rope_rotate
+from oracle import RMS_EPS, block_causal_attention, euler_step, rms_norm, rope_rotate
 from oracle.dit import gelu_tanh, modulate
 from oracle.fp8 import (attention_fp8, attn_fp8_scales, dequantize_weight, project, quantize_heads,
                         quantize_rows)
@@ -37,6 +37,20 @@ def _normed_operand(h, cfg):
 
 def _dit(cfg):
     return getattr(cfg, "block_kind", 0) == 1
+
+
+def _folded(cfg, W):
+    """Whether the stream folds the RMS norm into its GEMMs (bf16 attention
+    sublayers with an in-projection and a head, bf16 projections): the QKV and head
+    GEMMs then consume the residual itself rounded to bf16, and scale each product
+    row by the row's 1 / rms, taken from the fp32 residual."""
+    return (cfg.dtype == DTYPE_BF16 and not getattr(cfg, "proj_fp8", 0) and not _dit(cfg)
+            and W.w_in is not None and W.w_head is not None)
+
+
+def _inv_rms(h):
+    h = np.asarray(h, np.float64)
+    return 1.0 / np.sqrt(np.mean(h * h, axis=-1, keepdims=True) + RMS_EPS)
 
 
 def _attn_operand(h, cfg, W, l, t_idx):
@@ -176,8 +190,11 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None, audio
     want = x_in[R] if w_in is None else _operand(x_in[R], cfg) @ w_in.T
     chk(h_in[R], want, "in-proj h")
     h_prev = h_in
+    fold = _folded(cfg, W)
     for l in range(L):
-        op = _attn_operand(h_prev[R], cfg, W, l, i)
+        # folded norm: n(h) W^T taken as diag(1 / rms(h)) (bf16(h) W^T)
+        op = _operand(h_prev[R], cfg) if fold else _attn_operand(h_prev[R], cfg, W, l, i)
+        rs = _inv_rms(h_prev[R]) if fold else 1.0
         if getattr(cfg, "proj_fp8", 0) or getattr(cfg, "attn_fp8", 0):
             # e4m3 operands downstream: check the normalisation on its own, then go on
             # from the operand the GPU consumed (a one-ulp bf16 difference there moves
@@ -185,7 +202,7 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None, audio
             op_gpu = to_np(s.tap("hop", l, i))[R].astype(np.float64)
             chk(op_gpu, op, f"norm operand l{l}")
             op = op_gpu
-        qkv = _proj(op, W.w_qkv[l], cfg)
+        qkv = _proj(op, W.w_qkv[l], cfg) * rs
         q = qkv[:, :D].reshape(len(R), H, d)
         k = qkv[:, D:2 * D].reshape(len(R), H, d)
         v = qkv[:, 2 * D:].reshape(len(R), H, d)
@@ -234,8 +251,12 @@ def check_step(s, cfg, W, b, i, rows=None, tag="", report=None, sink=None, audio
         want = h_prev[R].astype(np.float64) + _proj(_operand(o_gpu[R], cfg), W.w_out[l], cfg)
         chk(h_next[R], want, f"h l{l}")
         h_prev = h_next
-    vel = (rms_norm(h_prev[R].astype(np.float64)) if w_head is None
-           else _normed_operand(h_prev[R], cfg) @ w_head.T)
+    if w_head is None:
+        vel = rms_norm(h_prev[R].astype(np.float64))
+    elif fold:
+        vel = (_operand(h_prev[R], cfg) @ w_head.T) * _inv_rms(h_prev[R])
+    else:
+        vel = _normed_operand(h_prev[R], cfg) @ w_head.T
     chk(to_np(s.tap("v", 0, i))[R], vel, "velocity")
     x_want = euler_step(x_in[R], vel, cfg.timesteps[i], cfg.timesteps[i + 1])
     chk(to_np(s.tap("x_out", 0, i))[R], x_want, "x")
