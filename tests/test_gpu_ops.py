@@ -170,11 +170,12 @@ def test_euler_standalone_matches_oracle():
     assert_close(_np(x), want, DTYPE_FP32, "euler")
 
 
-@pytest.mark.parametrize("emu", [3, 4])
+@pytest.mark.parametrize("emu", [0, 3, 4])
 def test_attention_with_polynomial_exp2_share_matches_oracle(emu, tmp_path):
     """LA_ATTN_EMU=k computes k of every 8 exponential pairs of full key tiles
-    with the FMA-pipe polynomial; the setting is read once per process, so the
-    case runs in a child process and the parity check runs here."""
+    with the FMA-pipe polynomial (bf16 default 2, covered by every other
+    attention test; 0 is ex2 alone); the setting is read once per process, so
+    the case runs in a child process and the parity check runs here."""
     import os
     import subprocess
     import sys
