@@ -95,6 +95,11 @@ struct QkvRopeParams {
   const float* tcos; const float* tsin;   // [LA_MAX_STEPS][LA_TROWS][LA_MAX_PT]
   const float* rcos; const float* rsin;   // [grid_h][ph]
   const float* ccos; const float* csin;   // [grid_w][pw]
+  // (cos, sin) of every pair of every token of the pass, [d/2][rowtab_ld] with
+  // the grouped row (buffer * T + token) fastest, gathered once a pass from the
+  // three tables above; NULL: the epilogue gathers from them itself
+  const float2* rowtab;
+  long long rowtab_ld;
   void* q_rope;              // [nbuf][H][T][d]
   void* ring_k; void* ring_v;// [L][S][E][H][T][d]
   const float* fp8_inv;      // NULL, or [3][H] inverse scales of q, K, V: write e4m3 codes of

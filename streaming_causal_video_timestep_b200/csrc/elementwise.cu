@@ -67,6 +67,39 @@ __device__ __forceinline__ void rotate8(float (&v)[8], int ch, int buf, int trow
   }
 }
 
+// One (pair, token) of an active buffer a thread, token fastest (coalesced
+// stores); the same three-way table choice as rotate8.
+__global__ void k_rope_rows(const __grid_constant__ PassDesc pd, const __grid_constant__ RopeArgs a,
+                            float2* __restrict__ out, long long ld) {
+  const int half = a.d / 2;
+  const long long per_buf = static_cast<long long>(half) * a.T;
+  const long long total = pd.nactive * per_buf;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int ai = static_cast<int>(i / per_buf);
+    const long long rem = i - ai * per_buf;
+    const int j = static_cast<int>(rem / a.T), n = static_cast<int>(rem - static_cast<long long>(j) * a.T);
+    const int buf = pd.active_buf[ai];
+    const int f = n / a.F, m = n - f * a.F;
+    const int rr = m / a.grid_w, cc = m - rr * a.grid_w;
+    float c, s;
+    if (j < a.pt) {
+      const int idx = (buf * LA_TROWS + f) * LA_MAX_PT + j;
+      c = a.tcos[idx];
+      s = a.tsin[idx];
+    } else if (j < a.pt + a.ph) {
+      const int idx = rr * a.ph + (j - a.pt);
+      c = a.rcos[idx];
+      s = a.rsin[idx];
+    } else {
+      const int idx = cc * a.pw + (j - a.pt - a.ph);
+      c = a.ccos[idx];
+      s = a.csin[idx];
+    }
+    out[static_cast<long long>(j) * ld + static_cast<long long>(buf) * a.T + n] = make_float2(c, s);
+  }
+}
+
 __global__ void k_rope_ttab(const __grid_constant__ PassDesc pd, int fpb, int pt, const double* __restrict__ omega,
                             float* tcos, float* tsin) {
   const int rows = fpb + 1;
@@ -401,6 +434,14 @@ int grid_for(long long n, int per_block = 256) {
 }
 
 }  // namespace
+
+cudaError_t launch_rope_rows(const PassDesc& pd, const RopeArgs& a, float2* out, long long ld, cudaStream_t st) {
+  if (pd.nactive <= 0) return cudaSuccess;
+  if (a.d % 2 != 0 || a.T <= 0 || a.F <= 0 || a.grid_w <= 0) return cudaErrorInvalidValue;
+  const long long total = static_cast<long long>(pd.nactive) * (a.d / 2) * a.T;
+  k_rope_rows<<<grid_for(total, 256), 256, 0, st>>>(pd, a, out, ld);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rope_ttab(const PassDesc& pd, int fpb, int pt, const double* omega_t, float* tcos, float* tsin,
                              cudaStream_t st) {

@@ -98,7 +98,18 @@ __device__ __forceinline__ void* qkv_rope_words(const QkvRopeParams& qp, const Q
   const int part = c32 / qp.D;
   const int cc = c32 - part * qp.D;
   const int h = cc / qp.d, e0 = cc - h * qp.d;
-  if (part < 2) {
+  if (part < 2 && qp.rowtab) {
+    // lanes are consecutive tokens: each pair's load is one contiguous run of (cos, sin)
+    const float2* tab = qp.rowtab + static_cast<long long>(e0 >> 1) * qp.rowtab_ld +
+                        (static_cast<long long>(qr.buf) * qp.T + qr.n);
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const float2 cs = __ldg(tab + jj * qp.rowtab_ld);
+      const float x0 = acc[2 * jj], x1 = acc[2 * jj + 1];
+      acc[2 * jj] = x0 * cs.x - x1 * cs.y;
+      acc[2 * jj + 1] = x0 * cs.y + x1 * cs.x;
+    }
+  } else if (part < 2) {
     const int pw_base = qp.pt + qp.ph;
 #pragma unroll
     for (int jj = 0; jj < 16; ++jj) {

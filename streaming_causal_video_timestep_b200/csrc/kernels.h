@@ -64,6 +64,12 @@ cudaError_t launch_attn_f32(const AttnParams& p, cudaStream_t st);
 cudaError_t launch_rope_ttab(const PassDesc& pd, int fpb, int pt, const double* omega_t, float* tcos, float* tsin,
                              cudaStream_t st);
 
+struct RopeArgs;
+// The per-token RoPE table of a pass for the QKV epilogue: (cos, sin) of every
+// pair j < d/2 of every token of every active buffer into out[j * ld + buf * T +
+// token], gathered from the pass's temporal table and the height / width tables.
+cudaError_t launch_rope_rows(const PassDesc& pd, const RopeArgs& a, float2* out, long long ld, cudaStream_t st);
+
 struct RopeArgs {
   int T, F, H, d, D, grid_w, fpb;
   int pt, ph, pw;

@@ -233,6 +233,7 @@ struct la_stream {
   float* tcos = nullptr;
   float* tsin = nullptr;
   float *rcos = nullptr, *rsin = nullptr, *ccos = nullptr, *csin = nullptr;
+  float2* rope_rows = nullptr;   // [d/2][nbuf*T] (cos, sin) of the pass (bf16 QKV epilogue)
   int* dev_err = nullptr;
 
   CUtensorMap tm_hop{}, tm_xop{}, tm_o{}, tm_win{}, tm_whead{};
@@ -697,6 +698,11 @@ int run_pass(la_stream* s, const PassDesc& pd) {
          return launch_rope_ttab(pd, s->fpb, s->pt, s->omega_t, s->tcos, s->tsin, s->st);
        })) != LA_OK)
     return r;
+  if (s->bf16 && (r = launch(s, LA_KIND_OTHER, [&] {
+                    return launch_rope_rows(pd, rope_args(s), s->rope_rows, static_cast<long long>(s->nbuf) * T,
+                                            s->st);
+                  })) != LA_OK)
+    return r;
 
   // in-projection into the fp32 residual stream, then its normalised operand
   if (s->id_in) {
@@ -754,6 +760,8 @@ int run_pass(la_stream* s, const PassDesc& pd) {
   }
   qp.tcos = s->tcos; qp.tsin = s->tsin; qp.rcos = s->rcos; qp.rsin = s->rsin; qp.ccos = s->ccos; qp.csin = s->csin;
   qp.q_rope = s->q_rope; qp.ring_k = s->ring_k; qp.ring_v = s->ring_v;
+  qp.rowtab = s->rope_rows;
+  qp.rowtab_ld = static_cast<long long>(s->nbuf) * T;
   ap.out32 = (s->bf16 && s->capture) ? s->cap_oall : nullptr;
   ap.q_prescaled = s->bf16 ? 1 : 0;
 
@@ -1281,6 +1289,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   ALLOC_OR_BAIL(s->rcos, std::max(1, cfg->grid_h * s->ph) * 4);
   ALLOC_OR_BAIL(s->rsin, std::max(1, cfg->grid_h * s->ph) * 4);
   ALLOC_OR_BAIL(s->ccos, std::max(1, cfg->grid_w * s->pw) * 4);
+  if (s->bf16) ALLOC_OR_BAIL(s->rope_rows, static_cast<long long>(d / 2) * NB * T * 8);
   ALLOC_OR_BAIL(s->csin, std::max(1, cfg->grid_w * s->pw) * 4);
   ALLOC_OR_BAIL(s->dev_err, 64);
 

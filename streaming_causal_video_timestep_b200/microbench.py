@@ -7,6 +7,7 @@
     python -m streaming_causal_video_timestep_b200.microbench rerope [--iters N] [--layers L]
     python -m streaming_causal_video_timestep_b200.microbench gemm_fp8 [--iters N]
     python -m streaming_causal_video_timestep_b200.microbench attn_fp8 [--iters N]
+    python -m streaming_causal_video_timestep_b200.microbench qkv_stream [--iters N] [--fp8]
 
 attn : one block's attention in steady state at the 14B-like shape: 4680
        queries x 40 heads x 128 over [sink 1560 | 2 window blocks | block]
@@ -22,6 +23,11 @@ rerope: the per-block sink re-rope of the 8-sublayer stream (30x52 grid, 40x128
        heads, 4 slots), one launch a tick for all layers: reads each layer's
        fp32 un-roped sink K (32 MB) once and writes 4 bf16 roped copies (64 MB),
        766 MB a launch; timed by the stream's profiling counters.
+qkv_stream: the QKV projection with its fused RoPE / ring-append epilogue and
+       the output projection with its residual epilogue, as they run in the
+       4-slot grouped stream ([18720, 5120] x [15360, 5120]^T and x [5120,
+       5120]^T), in a one-sublayer stream at the 14B-like shape; bf16, or with
+       --fp8 on e4m3 operands; timed by the stream's profiling counters.
 Inputs exceed L2 (126 MB) except the per-slot attention keys (160 MB K/V +
 48 MB q).  Each timed loop spans at least 1.5 s; prints one JSON line per mode
 with the SM clock record (median under load, throttle reasons) taken around it.
@@ -189,11 +195,59 @@ def bench_rerope(iters, layers=8):
             "ms": round(ms, 4), "gbs": round(nbytes / ms / 1e6, 1), "bytes": nbytes}
 
 
+def bench_qkv_stream(iters, fp8=False):
+    from types import SimpleNamespace
+    from .stream import LaStream
+    cfg = SimpleNamespace(num_layers=1, hidden=5120, heads=40, head_dim=128, latent_ch=64, grid_h=30, grid_w=52,
+                          frames_per_block=3, sink_frames=1, window_blocks=2, timesteps=(1.0, 0.75, 0.5, 0.25, 0.0),
+                          rope_split=(22, 21, 21), pairs=(22, 21, 21), rope_theta=10000.0, sink_mode=0, rolling_rope=1,
+                          sink_offset_frames=3, schedule=0, dtype=0, proj_fp8=1 if fp8 else 0)
+    D, C, F, T = cfg.hidden, cfg.latent_ch, cfg.grid_h * cfg.grid_w, 3 * cfg.grid_h * cfg.grid_w
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    rnd = lambda *sh: (torch.randn(*sh, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    w = dict(w_qkv=[rnd(3 * D, D)], w_out=[rnd(D, D)], w_in=rnd(D, C), w_head=rnd(C, D))
+    s = LaStream(cfg, w)
+    s.set_sink(torch.randn(F, C, generator=g, device="cuda"))
+    x = torch.randn(T, C, generator=g, device="cuda")
+    out = torch.empty(T, C, device="cuda")
+    for _ in range(3 + 3 + 3):          # fill: every slot active with a full window
+        s.step(x, out)
+    s.synchronize()
+    s.profile(True)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    n = 0
+    while True:                         # at least iters ticks and 1.5 s
+        s.step(x, out)
+        n += 1
+        if n >= iters and n % 10 == 0:
+            t1.record()
+            t1.synchronize()
+            if t0.elapsed_time(t1) >= 1500.0:
+                break
+    s.synchronize()
+    res = {"mode": "qkv_stream", "dtype": "e4m3 operands" if fp8 else "bf16", "ticks": n}
+    M = 4 * T
+    for kind, N, what in (("qkv_gemm", 3 * D, "QKV + RoPE/ring append"), ("out_gemm", D, "output + residual")):
+        cnt, tot = s.profile_read(kind)
+        ms = tot / cnt
+        flops = 2.0 * M * N * D
+        res[kind] = {"shape": f"{M}x{N}x{D}", "epilogue": what, "ms": round(ms, 4),
+                     "tflops": round(flops / ms / 1e9, 1), "launches": cnt}
+    s.profile(False)
+    s.close()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("mode", choices=["attn", "attn_fp8", "gemm", "gemm_out", "euler", "rerope", "gemm_fp8", "all"])
+    ap.add_argument("mode", choices=["attn", "attn_fp8", "gemm", "gemm_out", "euler", "rerope", "gemm_fp8",
+                                     "qkv_stream", "all"])
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--layers", type=int, default=8, help="rerope: sublayers of the stream (one launch covers all)")
+    ap.add_argument("--fp8", action="store_true", help="qkv_stream: e4m3 projections")
     args = ap.parse_args()
     modes = ["attn", "attn_fp8", "gemm", "gemm_out", "gemm_fp8", "euler", "rerope"] if args.mode == "all" else [args.mode]
     for m in modes:
@@ -201,7 +255,7 @@ def main():
         clocks.start()
         r = {"attn": bench_attn, "attn_fp8": bench_attn_fp8, "gemm": bench_gemm, "gemm_out": bench_gemm_out,
              "euler": bench_euler, "rerope": lambda it: bench_rerope(it, args.layers),
-             "gemm_fp8": bench_gemm_fp8}[m](args.iters)
+             "gemm_fp8": bench_gemm_fp8, "qkv_stream": lambda it: bench_qkv_stream(it, args.fp8)}[m](args.iters)
         r["clocks"] = clocks.stop()
         print(json.dumps(r), flush=True)
 
