@@ -746,7 +746,12 @@ def main():
     line = run_gpu(args, rank, world, local_rank)
     from workloads import STREAM
     if world > 1 and world % STREAM.cfg.num_steps == 0 and not args.no_tpp:
-        tpp = run_tpp(args, rank, world, local_rank)
+        # the pipeline arm must not cost the replicas line: an error in it (or a rank
+        # that times out in one of its collectives) is reported in the record instead
+        try:
+            tpp = run_tpp(args, rank, world, local_rank)
+        except Exception as e:       # noqa: BLE001 - any failure of the sub-record
+            tpp = {"error": f"{type(e).__name__}: {e}"[:300]}
         if rank == 0:
             line["tpp"] = tpp
     if rank == 0:
