@@ -38,9 +38,10 @@ WORKLOAD = dict(
 
 # DRAM bytes (read + write) of one slot's attention launch (4680 queries x 15,600 keys x 40 heads x 128,
 # bf16 q/K/V and output) from one ncu capture of the one-slot attention microbenchmark of the kernel with
-# the warp-wide MMA issuer: 386.9 MB read + 44.4 MB written, against 415.2 MB of algorithmic bytes.  The
-# grouped launch of the stream reads the disjoint q / K / V of its S slots, so its traffic is S times this.
-ATTN_DRAM_BYTES_PER_SLOT = 431.3e6
+# the warp-wide MMA issuer and 2 of 8 exponential pairs on the FMA pipe: 385.2 MB read + 43.3 MB written,
+# against 415.2 MB of algorithmic bytes.  The grouped launch of the stream reads the disjoint q / K / V of
+# its S slots, so its traffic is S times this.
+ATTN_DRAM_BYTES_PER_SLOT = 428.5e6
 # FFN width of the full DiT block in the ablation: the 14B Wan-style DiT's 13824 (2.7 x 5120)
 DIT_FFN = 13824
 # Audio of a block for the DiT block's cross-attention (synthetic sizes; the pages give none):
