@@ -207,14 +207,14 @@ __device__ __forceinline__ void* segment_words(const GemmEpiParams& ep, const Qk
   return reinterpret_cast<__nv_bfloat16*>(ep.out) + row * ep.ld + col;
 }
 
-// h32 (+)= [gate *] acc for the 32 rows row0 .. row0+31 of one epilogue warp and
+// h32 (+)= [gate *] acc (SET: h32 = acc) for the 32 rows row0 .. row0+31 of one epilogue warp and
 // the 32 columns col .. col+31 (all in range), plus the bf16 copy to ep.out.
 // Lane t holds row t's values in acc.  The chunk passes through the warp's
 // shared-memory stage: loaded and stored by lanes 8 to a 128-byte row segment
 // (bf16: 4 to a 64-byte segment), combined by lanes one row each.  16-byte
 // slots in the stage are XOR-swizzled by row, so neither access pattern has
 // bank conflicts beyond the 4 wavefronts that 512 bytes take.
-template <bool GATED>
+template <bool GATED, bool SET = false>
 __device__ __forceinline__ void epilogue_resid_warp(const GemmEpiParams& ep, long long row0, long long col,
                                                    float (&acc)[32], uint8_t* stage, int lane) {
   float4* sf = reinterpret_cast<float4*>(stage);
@@ -226,28 +226,35 @@ __device__ __forceinline__ void epilogue_resid_warp(const GemmEpiParams& ep, lon
 #pragma unroll
     for (int i = 0; i < 8; ++i) gvs[i] = __ldg(g4 + i);
   }
-  float4 hv[8];
+  if (!SET) {
+    float4 hv[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int r = 4 * k + sub;
-    hv[k] = *reinterpret_cast<const float4*>(ep.h32 + (row0 + r) * ep.ld + col + 4 * ch);
-  }
+    for (int k = 0; k < 8; ++k) {
+      const int r = 4 * k + sub;
+      hv[k] = *reinterpret_cast<const float4*>(ep.h32 + (row0 + r) * ep.ld + col + 4 * ch);
+    }
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int r = 4 * k + sub;
-    sf[r * 8 + (ch ^ (r & 7))] = hv[k];
+    for (int k = 0; k < 8; ++k) {
+      const int r = 4 * k + sub;
+      sf[r * 8 + (ch ^ (r & 7))] = hv[k];
+    }
+    __syncwarp();
   }
-  __syncwarp();
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     float4& slot = sf[lane * 8 + (c ^ (lane & 7))];
-    float4 h = slot;
-    if (GATED) {
+    float4 h;
+    if (SET) {
+      // the chunk is the new value itself (h32 = acc), staged only for the coalesced stores
+      h = make_float4(acc[4 * c + 0], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+    } else if (GATED) {
+      h = slot;
       h.x = fmaf(gvs[c].x, acc[4 * c + 0], h.x);
       h.y = fmaf(gvs[c].y, acc[4 * c + 1], h.y);
       h.z = fmaf(gvs[c].z, acc[4 * c + 2], h.z);
       h.w = fmaf(gvs[c].w, acc[4 * c + 3], h.w);
     } else {
+      h = slot;
       h.x += acc[4 * c + 0];
       h.y += acc[4 * c + 1];
       h.z += acc[4 * c + 2];
@@ -457,6 +464,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmEpiParams& ep, const Qkv
       }
       if (ep.kind == EPI_RESID_GATED)
         epilogue_resid_warp<true>(ep, row0, col, v, epi_stage, lane);
+      else if (ep.kind == EPI_SET32)
+        epilogue_resid_warp<false, true>(ep, row0, col, v, epi_stage, lane);
       else
         epilogue_resid_warp<false>(ep, row0, col, v, epi_stage, lane);
       if (ep.ssq_out) {
@@ -599,9 +608,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   } else {
     const int quarter = warp & 3;
     uint8_t* epi_stage = smem + C::STAGES * C::STAGE_BYTES + 256 + (warp - 2) * EPI_WARP_BYTES;
-    // the residual kinds take the staged path when the warp's 32 rows are all in
+    // the residual kinds and SET32 take the staged path when the warp's 32 rows are all in
     // range and h32 / out rows start on 16-byte boundaries
-    const bool staged_kind = (ep.kind == EPI_RESID || ep.kind == EPI_RESID_GATED) && (ep.ld % 8) == 0 &&
+    const bool staged_kind = (ep.kind == EPI_RESID || ep.kind == EPI_RESID_GATED || ep.kind == EPI_SET32) &&
+                             (ep.ld % 8) == 0 &&
                              (reinterpret_cast<uintptr_t>(ep.h32) & 15) == 0 &&
                              (reinterpret_cast<uintptr_t>(ep.out) & 15) == 0;
     // the kinds that end in one packed segment a row (64 bytes of bf16, or 32 of
@@ -785,7 +795,8 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   } else {
     const int quarter = warp & 3;
     uint8_t* epi_stage = smem + ST * C::STAGE_BYTES + 256 + (warp - 2) * EPI_WARP_BYTES;
-    const bool staged_kind = (ep.kind == EPI_RESID || ep.kind == EPI_RESID_GATED) && (ep.ld % 8) == 0 &&
+    const bool staged_kind = (ep.kind == EPI_RESID || ep.kind == EPI_RESID_GATED || ep.kind == EPI_SET32) &&
+                             (ep.ld % 8) == 0 &&
                              (reinterpret_cast<uintptr_t>(ep.h32) & 15) == 0 &&
                              (reinterpret_cast<uintptr_t>(ep.out) & 15) == 0;
     const bool segment_kind = ep.kind == EPI_STORE || ep.kind == EPI_GELU || ep.kind == EPI_QKV_ROPE;
