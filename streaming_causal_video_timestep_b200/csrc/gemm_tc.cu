@@ -10,10 +10,14 @@
 //               per k-block (32 bytes of K each);
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //               32*(w%4) .. +31 = tile rows), fused epilogue, global stores.
-//               The residual epilogues move each 32 x 32 chunk of the fp32
-//               residual through a per-warp shared-memory stage, so that the
-//               global loads and stores cover whole 128-byte row segments.
+//               The residual and set epilogues move each 32 x 32 chunk of the
+//               fp32 residual through a per-warp shared-memory stage, so that the
+//               global loads and stores cover whole 128-byte row segments.  The
+//               epilogues also carry the per-token RMS norm folded into the
+//               GEMMs: the residual writers leave each row's sum of squares per
+//               column tile, the QKV and head GEMMs scale rows by 1 / rms.
 // The two accumulators let the epilogue of tile n overlap the main loop of n+1.
+// 256-column bf16 tiles run on CTA pairs instead (k_gemm_pair below).
 // Tiles are visited in bands of GROUP_M row-blocks so the A band and the W
 // tiles in flight stay L2-resident.
 #include <cuda_fp16.h>
