@@ -743,6 +743,9 @@ def main():
         import torch
         import torch.distributed as tdist
         torch.cuda.set_device(local_rank)
+        # a collective that times out aborts its communicator and raises in the waiting
+        # call (instead of tearing the process down), so rank 0 can still print its line
+        os.environ.setdefault("TORCH_NCCL_ASYNC_ERROR_HANDLING", "2")
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     line = run_gpu(args, rank, world, local_rank)
     from workloads import STREAM
