@@ -313,8 +313,11 @@ int la_debug_capture(la_stream* s, int32_t enable);
 #define LA_TAP_SINK_KROPE 10 /* attn [H, F, d] sink K as roped for the slot's last step          */
 #define LA_TAP_SINK_H    11 /* fp32 [F, D] sink residual entering layer `layer` in the last sink
                                pass (la_set_sink or the AAS replacement; slot ignored)           */
-#define LA_TAP_HOP       12 /* bf16 [T_b, D] normalised residual as the QKV projection of layer
-                               `layer` consumed it at the slot's step (bf16 streams)             */
+#define LA_TAP_HOP       12 /* bf16 [T_b, D] the QKV projection's operand of layer `layer` at the
+                               slot's step (bf16 streams): the normalised residual, or, where
+                               the stream folds the norm into its GEMMs (bf16 attention
+                               sublayers with w_in, w_head and bf16 projections), the residual
+                               itself rounded to bf16 (the GEMM scales its rows by 1 / rms)  */
 #define LA_TAP_SINK_HOP  13 /* bf16 [F, D] the same in the last sink pass (slot ignored)         */
 /* With attn_fp8 the Q, RING_K, RING_V and SINK_KROPE taps hold uint8 e4m3 codes
  * (value = code * scale of its layer, part and head; Q not pre-scaled), and: */
