@@ -391,20 +391,15 @@ def run_tpp(args, rank, world, local_rank):
     # the hand-off alone: the message a rank sends each tick (block id + T x C fp32),
     # rank r -> r + 1 of every pipeline at once, timed on each rank, max over ranks
     msg = [torch.zeros(1, dtype=torch.int64, device=dev), torch.zeros((T, C), dtype=torch.float32, device=dev)]
-    inbox = [torch.empty_like(t) for t in msg]
+    layout = [(tuple(t.shape), t.dtype) for t in msg]
     tdist.barrier()
     torch.cuda.synchronize()
     hev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     reps = 20
     hev[0].record()
     for _ in range(reps):
-        works = []
-        if r < S - 1:
-            works += [tdist.isend(t, pid * S + r + 1, group=groups[pid]) for t in msg]
-        if r > 0:
-            works += [tdist.irecv(t, pid * S + r - 1, group=groups[pid]) for t in inbox]
-        for w in works:
-            w.wait()
+        # the pipeline's own exchange: one batched send / receive a rank
+        tr.exchange(msg if r < S - 1 else None, layout if r > 0 else None)
     hev[1].record()
     torch.cuda.synchronize()
     hand_ms = max_over_ranks(hev[0].elapsed_time(hev[1]) / reps, "cuda")
