@@ -484,8 +484,8 @@ def cpu_baseline(rows=1560, reps=1):
         smp.step()
     dt = (time.perf_counter() - t0) / reps
     return {"value": round(smp.frames_per_s(dt), 6), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
-            "sample": (f"fp64 numpy oracle, one attention sublayer of one slot, {rows} of 4680 query rows over "
-                       f"15,600 keys ({dt:.1f} s), scaled x{4680 / rows:.0f} rows x 4 slots x 8 layers per tick")}
+            "sample": (f"1 sublayer, 1 slot, {rows}/4680 rows x 15600 keys, {dt:.1f} s; "
+                       f"x{4680 / rows:.0f} rows x4 slots x8 layers")}
 
 
 def run_sweep(args):
@@ -688,8 +688,7 @@ def run_reference(args):
         smp.step()
     dt = (time.perf_counter() - t0) / args.steps
     v = smp.frames_per_s(dt)
-    sample = (f"fp64 numpy oracle, per step one attention sublayer of one slot for 234 of 4680 query rows "
-              f"({dt:.2f} s), scaled to a tick (x20 rows x 4 slots x 8 layers)")
+    sample = f"per step: 1 sublayer, 1 slot, 234/4680 rows, {dt:.2f} s; x20 rows x4 slots x8 layers"
     return {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1000.0, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
