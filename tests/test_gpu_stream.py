@@ -93,6 +93,21 @@ def test_tiny_fp32_stream_every_tick_matches_oracle():
     _run_teacher_forced(TINY)
 
 
+@pytest.mark.parametrize("window,nblocks", [(0, 6), (4, 3)])
+def test_tiny_fp32_stream_window_edges_match_oracle(window, nblocks):
+    """The window's degenerate ends: no prior blocks at all (each block attends to
+    the sink and itself), and a stream that ends before its window fills."""
+    wl = Workload(f"tiny-w{window}", TINY.cfg.replace(window_blocks=window), TINY.seed, nblocks, TINY.w_std)
+    _run_teacher_forced(wl)
+
+
+def test_small_bf16_stream_window_0_teacher_forced():
+    """bf16 with no cache window: ring entries of one block each, sink + self keys."""
+    wl = Workload("small-bf16-w0", SMALL_BF16.cfg.replace(window_blocks=0), SMALL_BF16.seed, 6,
+                  SMALL_BF16.w_std, SMALL_BF16.head_std)
+    _run_teacher_forced(wl)
+
+
 def test_tiny_fp32_stream_free_running_trajectory():
     """No teacher forcing: the fp32 trajectory itself stays within 1e-5."""
     wl = TINY
