@@ -206,3 +206,106 @@ def test_tpp_two_pipelines_in_one_job_over_their_own_groups():
         blocks, err = out[pid]
         assert blocks == list(range(6))
         assert err < 2e-6
+
+
+class _RendezvousHub:
+    """Ranks as threads, with the blocking semantics of a GPU communicator: a send
+    completes only once its receiver has taken the message, and a broadcast only
+    once every rank has reached it.  (gloo buffers its sends, so the gloo tests
+    cannot show a send and a collective waiting on each other.)  Every wait is
+    bounded: a protocol that deadlocks fails the test instead of hanging it."""
+
+    def __init__(self, world, limit_s=20.0):
+        import threading
+        self.world, self.limit = world, limit_s
+        self.cv = threading.Condition()
+        self.links = {}                     # (sender, seq) -> message
+        self.taken = set()
+        self.bar = threading.Barrier(world, timeout=limit_s)
+        self.slot = [None]
+
+    def _wait(self, pred, what):
+        if not self.cv.wait_for(pred, timeout=self.limit):
+            raise TimeoutError(f"deadlock: {what}")
+
+    def endpoint(self, rank):
+        return _RendezvousEnd(self, rank)
+
+
+class _RendezvousEnd:
+    def __init__(self, hub, rank):
+        self.hub, self.rank = hub, rank
+        self.sent = self.recvd = 0
+
+    def exchange(self, send, recv_layout):
+        h, out = self.hub, None
+        with h.cv:
+            key = None
+            if send is not None:                       # post the send (both halves of the batch are posted
+                key = (self.rank, self.sent)           # before either is waited on)
+                self.sent += 1
+                h.links[key] = [t.clone() for t in send]
+                h.cv.notify_all()
+            if recv_layout is not None:
+                want = (self.rank - 1, self.recvd)
+                self.recvd += 1
+                h._wait(lambda: want in h.links, f"rank {self.rank} receiving {want}")
+                out = h.links.pop(want)
+                h.taken.add(want)
+                h.cv.notify_all()
+            if key is not None:
+                h._wait(lambda: key in h.taken, f"rank {self.rank} sending {key}")
+        return out
+
+    def bcast_from_last(self, t):
+        h = self.hub
+        if self.rank == h.world - 1:
+            h.slot[0] = t.clone()
+        h.bar.wait()
+        if self.rank != h.world - 1:
+            t.copy_(h.slot[0])
+        h.bar.wait()
+        return t
+
+
+@pytest.mark.parametrize("aas", [True, False])
+def test_tpp_completes_with_rendezvous_sends(aas):
+    """The pipeline's protocol under unbuffered sends (rank threads, one batched
+    exchange a tick before the sink broadcast) finishes every block and matches
+    the single-process pipelined stream."""
+    import threading
+
+    from streaming_causal_video_timestep_b200.tpp import TppRank
+    from workloads import make_weights
+    wl = _workload(aas)
+    W = make_weights(wl)
+    S = wl.cfg.num_steps
+    hub = _RendezvousHub(S)
+    ranks = [TppRank(OracleSlot(wl, W, r), r, S, hub.endpoint(r), "cpu", S, wl.cfg.sink_tokens, aas)
+             for r in range(S)]
+    seq = _inputs(wl)
+    done, errors = {}, []
+
+    def run(r):
+        try:
+            for item in seq:
+                x_new = item[0] if (item is not None and r.rank == 0) else None
+                blk, lat = r.tick(x_new)
+                if blk >= 0:
+                    done[blk] = lat
+            r.close()
+        except Exception as e:      # noqa: BLE001 - reported below
+            errors.append(f"rank {r.rank}: {type(e).__name__}: {e}")
+            hub.bar.abort()
+
+    threads = [threading.Thread(target=run, args=(r,)) for r in ranks]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not errors, errors
+    assert not any(t.is_alive() for t in threads)
+    want = _single_process(wl, W)
+    assert sorted(done) == list(range(wl.num_blocks))
+    for b in range(wl.num_blocks):
+        np.testing.assert_allclose(done[b].numpy(), want[b], rtol=2e-6, atol=2e-6)
