@@ -293,6 +293,24 @@ int64_t la_index_state_size(const la_stream* s);
  */
 int la_get_index_state(const la_stream* s, int32_t* host_buf, int64_t n);
 
+/* The tick scheduler on the host alone: no stream, no GPU, no device memory.
+ * la_sched_trace runs the scheduling of `nticks` la_denoise_step calls on a
+ * fresh stream of configuration cfg (has_new[k] != 0: call k brings a new
+ * block; the sequential and slot schedules need one on every call), in the
+ * order a call makes them (plan the tick, append each running (slot, block) to
+ * its ring, the clean-cache refresh, finish), and writes the index state after
+ * each call (the layout of la_get_index_state, la_sched_state_size(cfg) int32
+ * values each) to out[k * size ...].  Only the scheduling fields of cfg are read
+ * (frames_per_block, window_blocks, num_steps, sink_mode, schedule, slot_index,
+ * cache_mode, cache_step, rolling_rope, sink_offset_frames).
+ * Returns LA_EINVAL for a bad configuration, NULL pointers or out_len below
+ * nticks * size; LA_ESTATE at a call the schedule does not allow (then out holds
+ * the states of the calls before it).  la_sched_state_size returns -1 for a bad
+ * configuration.  A stream's AAS sink replacement by the caller
+ * (la_replace_sink, slot schedule) is not modelled. */
+int64_t la_sched_state_size(const la_config* cfg);
+int la_sched_trace(const la_config* cfg, int32_t nticks, const uint8_t* has_new, int32_t* out, int64_t out_len);
+
 /* Enable (1) / disable (0) capture of per-slot intermediates for la_debug_tap.
  * Allocates capture buffers on enable. */
 int la_debug_capture(la_stream* s, int32_t enable);

@@ -10,7 +10,7 @@ from ._lib import LaError, exported_symbols, load  # noqa: F401
 
 def __getattr__(name):
     if name in ("LaStream", "op_gemm", "op_attention", "op_euler", "op_quantize_e4m3", "op_gemm_fp8",
-                "op_attention_fp8", "torch_dtype"):
+                "op_attention_fp8", "torch_dtype", "sched_trace"):
         from . import stream
         return getattr(stream, name)
     raise AttributeError(name)

@@ -71,6 +71,8 @@ def load():
         "la_status_string": (c_char_p, [c_int]),
         "la_index_state_size": (c_int64, [c_void_p]),
         "la_get_index_state": (c_int, [c_void_p, POINTER(c_int32), c_int64]),
+        "la_sched_state_size": (c_int64, [c_void_p]),
+        "la_sched_trace": (c_int, [c_void_p, c_int32, c_void_p, POINTER(c_int32), c_int64]),
         "la_debug_capture": (c_int, [c_void_p, c_int32]),
         "la_debug_tap": (c_int, [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_int64]),
         "la_debug_set_slot_input": (c_int, [c_void_p, c_int32, c_void_p]),
@@ -112,7 +114,7 @@ def exported_symbols():
         "la_debug_capture", "la_debug_tap", "la_debug_set_slot_input", "la_profile_enable", "la_profile_read",
         "la_launch_count", "la_op_gemm", "la_op_attention", "la_op_euler", "la_op_attention_static",
         "la_debug_wait_timeout", "la_op_quantize_e4m3", "la_op_gemm_fp8", "la_op_attention_fp8",
-        "la_debug_op_wait_timeout", "la_op_status",
+        "la_debug_op_wait_timeout", "la_op_status", "la_sched_state_size", "la_sched_trace",
     ]
 
 

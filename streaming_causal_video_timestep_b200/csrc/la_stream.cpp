@@ -350,28 +350,11 @@ int dalloc(la_stream* s, void** p, size_t bytes) {
     ptr = reinterpret_cast<decltype(ptr)>(p_);                                          \
   } while (0)
 
-int validate(const la_config* c, const la_weights* w, std::string& msg) {
-  if (!c || !w) { msg = "NULL config or weights"; return LA_EINVAL; }
-  if (c->num_layers < 1 || c->hidden < 1 || c->heads < 1 || c->head_dim < 2 || c->latent_ch < 1 ||
-      c->grid_h < 1 || c->grid_w < 1) { msg = "sizes must be positive"; return LA_EINVAL; }
-  if (static_cast<long long>(c->heads) * c->head_dim != c->hidden) { msg = "hidden != heads*head_dim"; return LA_EINVAL; }
-  if (c->head_dim % 8 != 0 || c->head_dim > 128) { msg = "head_dim must be a multiple of 8 and <= 128"; return LA_EINVAL; }
-  if (c->dtype == LA_BF16 && c->head_dim != 128) { msg = "the bf16 path needs head_dim == 128"; return LA_EINVAL; }
-  if (c->dtype != LA_BF16 && c->dtype != LA_FP32) { msg = "dtype must be LA_BF16 or LA_FP32"; return LA_EINVAL; }
+// The fields the tick scheduler reads (shared by stream creation and la_sched_trace).
+int validate_schedule(const la_config* c, std::string& msg) {
   if (c->frames_per_block < 1 || c->frames_per_block > LA_MAX_FPB) { msg = "frames_per_block out of range"; return LA_EINVAL; }
-  if (c->sink_frames != 1) { msg = "sink_frames must be 1"; return LA_EINVAL; }
   if (c->window_blocks < 0 || c->window_blocks > LA_MAX_WINDOW) { msg = "window_blocks out of range"; return LA_EINVAL; }
   if (c->num_steps < 1 || c->num_steps > LA_MAX_STEPS) { msg = "num_steps out of range"; return LA_EINVAL; }
-  if (!c->timesteps) { msg = "NULL timesteps"; return LA_EINVAL; }
-  for (int i = 0; i <= c->num_steps; ++i)
-    if (!std::isfinite(c->timesteps[i])) { msg = "timesteps must be finite"; return LA_EINVAL; }
-  for (int i = 0; i < c->num_steps; ++i)
-    if (!(c->timesteps[i + 1] < c->timesteps[i])) { msg = "timesteps must be strictly descending"; return LA_EINVAL; }
-  const int P = c->head_dim / 2;
-  if (c->rope_split[0] < 0 || c->rope_split[1] < 0 || c->rope_split[2] < 0 ||
-      c->rope_split[0] + c->rope_split[1] + c->rope_split[2] != P) { msg = "rope_split must sum to head_dim/2"; return LA_EINVAL; }
-  if (c->rope_split[0] > LA_MAX_PT) { msg = "too many temporal rotary pairs"; return LA_EINVAL; }
-  if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) { msg = "rope_theta must be positive"; return LA_EINVAL; }
   if (c->sink_mode != LA_SINK_FIXED && c->sink_mode != LA_SINK_AAS) { msg = "bad sink_mode"; return LA_EINVAL; }
   if (c->schedule != LA_SCHED_PIPELINED && c->schedule != LA_SCHED_SEQUENTIAL && c->schedule != LA_SCHED_SLOT) {
     msg = "bad schedule";
@@ -390,6 +373,35 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
     if (c->schedule != LA_SCHED_SEQUENTIAL) { msg = "the fixed-noise cache runs in the sequential schedule"; return LA_EINVAL; }
     if (c->cache_step < 0 || c->cache_step >= c->num_steps) { msg = "cache_step must name one of the steps"; return LA_EINVAL; }
   }
+  if (c->cache_mode == LA_CACHE_CLEAN_REFRESH && c->schedule != LA_SCHED_SEQUENTIAL) {
+    msg = "the clean-cache refresh needs the sequential schedule";
+    return LA_EINVAL;
+  }
+  if (c->rolling_rope != 0 && c->rolling_rope != 1) { msg = "rolling_rope must be 0 or 1"; return LA_EINVAL; }
+  if (c->sink_offset_frames < 0) { msg = "sink_offset_frames must be >= 0"; return LA_EINVAL; }
+  return LA_OK;
+}
+
+int validate(const la_config* c, const la_weights* w, std::string& msg) {
+  if (!c || !w) { msg = "NULL config or weights"; return LA_EINVAL; }
+  if (c->num_layers < 1 || c->hidden < 1 || c->heads < 1 || c->head_dim < 2 || c->latent_ch < 1 ||
+      c->grid_h < 1 || c->grid_w < 1) { msg = "sizes must be positive"; return LA_EINVAL; }
+  if (static_cast<long long>(c->heads) * c->head_dim != c->hidden) { msg = "hidden != heads*head_dim"; return LA_EINVAL; }
+  if (c->head_dim % 8 != 0 || c->head_dim > 128) { msg = "head_dim must be a multiple of 8 and <= 128"; return LA_EINVAL; }
+  if (c->dtype == LA_BF16 && c->head_dim != 128) { msg = "the bf16 path needs head_dim == 128"; return LA_EINVAL; }
+  if (c->dtype != LA_BF16 && c->dtype != LA_FP32) { msg = "dtype must be LA_BF16 or LA_FP32"; return LA_EINVAL; }
+  if (c->sink_frames != 1) { msg = "sink_frames must be 1"; return LA_EINVAL; }
+  if (const int r = validate_schedule(c, msg); r != LA_OK) return r;
+  if (!c->timesteps) { msg = "NULL timesteps"; return LA_EINVAL; }
+  for (int i = 0; i <= c->num_steps; ++i)
+    if (!std::isfinite(c->timesteps[i])) { msg = "timesteps must be finite"; return LA_EINVAL; }
+  for (int i = 0; i < c->num_steps; ++i)
+    if (!(c->timesteps[i + 1] < c->timesteps[i])) { msg = "timesteps must be strictly descending"; return LA_EINVAL; }
+  const int P = c->head_dim / 2;
+  if (c->rope_split[0] < 0 || c->rope_split[1] < 0 || c->rope_split[2] < 0 ||
+      c->rope_split[0] + c->rope_split[1] + c->rope_split[2] != P) { msg = "rope_split must sum to head_dim/2"; return LA_EINVAL; }
+  if (c->rope_split[0] > LA_MAX_PT) { msg = "too many temporal rotary pairs"; return LA_EINVAL; }
+  if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) { msg = "rope_theta must be positive"; return LA_EINVAL; }
   if (c->proj_fp8 != 0 && c->proj_fp8 != 1) { msg = "proj_fp8 must be 0 or 1"; return LA_EINVAL; }
   if (c->proj_fp8 && c->dtype != LA_BF16) { msg = "e4m3 projections need the bf16 stream"; return LA_EINVAL; }
   if (c->attn_fp8 != 0 && c->attn_fp8 != 1) { msg = "attn_fp8 must be 0 or 1"; return LA_EINVAL; }
@@ -407,12 +419,6 @@ int validate(const la_config* c, const la_weights* w, std::string& msg) {
     msg = "e4m3 attention needs the bf16 stream and head_dim 128";
     return LA_EINVAL;
   }
-  if (c->cache_mode == LA_CACHE_CLEAN_REFRESH && c->schedule != LA_SCHED_SEQUENTIAL) {
-    msg = "the clean-cache refresh needs the sequential schedule";
-    return LA_EINVAL;
-  }
-  if (c->rolling_rope != 0 && c->rolling_rope != 1) { msg = "rolling_rope must be 0 or 1"; return LA_EINVAL; }
-  if (c->sink_offset_frames < 0) { msg = "sink_offset_frames must be >= 0"; return LA_EINVAL; }
   if ((w->w_in == nullptr) != (w->w_head == nullptr)) { msg = "w_in and w_head must both be set or both NULL"; return LA_EINVAL; }
   if (w->w_in == nullptr && c->latent_ch != c->hidden) { msg = "identity projections need latent_ch == hidden"; return LA_EINVAL; }
   if (!w->w_qkv || !w->w_out) { msg = "NULL layer weight arrays"; return LA_EINVAL; }
@@ -1489,6 +1495,41 @@ int64_t la_index_state_size(const la_stream* s) { return s ? s->sched.state_size
 int la_get_index_state(const la_stream* s, int32_t* host_buf, int64_t n) {
   if (!s || !host_buf || n < s->sched.state_size()) return LA_EINVAL;
   s->sched.export_state(host_buf);
+  return LA_OK;
+}
+
+int64_t la_sched_state_size(const la_config* cfg) {
+  std::string msg;
+  if (!cfg || validate_schedule(cfg, msg) != LA_OK) return -1;
+  return 4 + static_cast<int64_t>(cfg->num_steps) * (8 + 3 * (cfg->window_blocks + 1));
+}
+
+int la_sched_trace(const la_config* cfg, int32_t nticks, const uint8_t* has_new, int32_t* out, int64_t out_len) {
+  std::string msg;
+  if (!cfg || nticks < 0 || (nticks > 0 && (!has_new || !out))) return LA_EINVAL;
+  if (validate_schedule(cfg, msg) != LA_OK) {
+    std::fprintf(stderr, "la_sched_trace: %s\n", msg.c_str());
+    return LA_EINVAL;
+  }
+  Scheduler sc;
+  sc.init(*cfg);
+  const long long n = sc.state_size();
+  if (out_len < n * nticks) return LA_EINVAL;
+  std::vector<std::pair<int, long long>> run;
+  std::vector<long long> next_held;
+  for (int k = 0; k < nticks; ++k) {
+    // the scheduling calls of one la_denoise_step, in its order, without the passes
+    const bool nw = has_new[k] != 0;
+    if (!sc.pipelined && !nw) return LA_ESTATE;
+    if (nw && (sc.blocks_in + 1) * static_cast<long long>(sc.fpb) > 0x7FFFFFF0LL) return LA_ESTATE;
+    long long finished = -1;
+    sc.plan(nw, run, finished, next_held);
+    sc.begin(nw, next_held);
+    for (auto& [slot, b] : run) sc.append(slot, b);
+    if (!sc.pipelined && sc.clean) sc.append_refresh(finished);
+    sc.finish(finished);
+    sc.export_state(out + n * k);
+  }
   return LA_OK;
 }
 

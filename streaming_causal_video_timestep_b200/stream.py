@@ -12,7 +12,7 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import LaConfig, LaWeights, check, load
+from ._lib import LA_EINVAL, LaConfig, LaError, LaWeights, check, load
 
 
 def _dtype_code(dtype):
@@ -57,28 +57,7 @@ class LaStream:
         self.stream = stream if stream is not None else torch.cuda.current_stream()
         self.dtype = _dtype_code(cfg.dtype)
         self.tdtype = torch_dtype(self.dtype)
-        ts = [float(t) for t in cfg.timesteps]
-        self._ts = (c_float * len(ts))(*ts)
-        pairs = getattr(cfg, "pairs", None) or cfg.rope_split
-        c = LaConfig()
-        c.num_layers, c.hidden, c.heads, c.head_dim = cfg.num_layers, cfg.hidden, cfg.heads, cfg.head_dim
-        c.latent_ch, c.grid_h, c.grid_w = cfg.latent_ch, cfg.grid_h, cfg.grid_w
-        c.frames_per_block, c.sink_frames, c.window_blocks = cfg.frames_per_block, cfg.sink_frames, cfg.window_blocks
-        c.num_steps = len(ts) - 1
-        c.timesteps = ctypes.cast(self._ts, ctypes.POINTER(c_float))
-        c.rope_split = (c_int32 * 3)(*pairs)
-        c.rope_theta = float(cfg.rope_theta)
-        c.sink_mode, c.rolling_rope, c.sink_offset_frames = cfg.sink_mode, cfg.rolling_rope, cfg.sink_offset_frames
-        c.schedule, c.dtype = cfg.schedule, self.dtype
-        c.cache_mode = getattr(cfg, "cache_mode", 0)
-        c.proj_fp8 = getattr(cfg, "proj_fp8", 0)
-        c.attn_fp8 = getattr(cfg, "attn_fp8", 0)
-        c.cache_step = getattr(cfg, "cache_step", 0)
-        c.block_kind = getattr(cfg, "block_kind", 0)
-        c.ffn_dim = getattr(cfg, "ffn_dim", 0)
-        c.audio_tokens = getattr(cfg, "audio_tokens", 0)
-        c.audio_dim = getattr(cfg, "audio_dim", 0)
-        c.slot_index = getattr(cfg, "slot_index", 0)
+        c, self._ts = _la_config(cfg, self.dtype)
         self.cfg = cfg
         self.c = c
         self.T = cfg.frames_per_block * cfg.grid_h * cfg.grid_w
@@ -228,6 +207,49 @@ class LaStream:
 
     def launch_count(self):
         return self.lib.la_launch_count(self.h)
+
+
+def _la_config(cfg, dtype_code):
+    """The C configuration of cfg, and the timestep array it points into (keep it alive)."""
+    ts = [float(t) for t in cfg.timesteps]
+    ts_arr = (c_float * len(ts))(*ts)
+    pairs = getattr(cfg, "pairs", None) or cfg.rope_split
+    c = LaConfig()
+    c.num_layers, c.hidden, c.heads, c.head_dim = cfg.num_layers, cfg.hidden, cfg.heads, cfg.head_dim
+    c.latent_ch, c.grid_h, c.grid_w = cfg.latent_ch, cfg.grid_h, cfg.grid_w
+    c.frames_per_block, c.sink_frames, c.window_blocks = cfg.frames_per_block, cfg.sink_frames, cfg.window_blocks
+    c.num_steps = len(ts) - 1
+    c.timesteps = ctypes.cast(ts_arr, ctypes.POINTER(c_float))
+    c.rope_split = (c_int32 * 3)(*pairs)
+    c.rope_theta = float(cfg.rope_theta)
+    c.sink_mode, c.rolling_rope, c.sink_offset_frames = cfg.sink_mode, cfg.rolling_rope, cfg.sink_offset_frames
+    c.schedule, c.dtype = cfg.schedule, dtype_code
+    c.cache_mode = getattr(cfg, "cache_mode", 0)
+    c.proj_fp8 = getattr(cfg, "proj_fp8", 0)
+    c.attn_fp8 = getattr(cfg, "attn_fp8", 0)
+    c.cache_step = getattr(cfg, "cache_step", 0)
+    c.block_kind = getattr(cfg, "block_kind", 0)
+    c.ffn_dim = getattr(cfg, "ffn_dim", 0)
+    c.audio_tokens = getattr(cfg, "audio_tokens", 0)
+    c.audio_dim = getattr(cfg, "audio_dim", 0)
+    c.slot_index = getattr(cfg, "slot_index", 0)
+    return c, ts_arr
+
+
+def sched_trace(cfg, has_new):
+    """The tick scheduler alone, on the host (la_sched_trace; no GPU): the index
+    state after each of len(has_new) calls (has_new[k]: call k brings a new
+    block), int32 [calls, la_sched_state_size]."""
+    lib = load()
+    c, _keep = _la_config(cfg, _dtype_code(cfg.dtype))
+    size = lib.la_sched_state_size(ctypes.byref(c))
+    if size < 0:
+        raise LaError(LA_EINVAL, "bad scheduling configuration")
+    n = len(has_new)
+    flags = (ctypes.c_uint8 * max(n, 1))(*[1 if x else 0 for x in has_new])
+    out = np.zeros((n, size), np.int32)
+    check(lib.la_sched_trace(ctypes.byref(c), n, flags, out.ctypes.data_as(ctypes.POINTER(c_int32)), out.size))
+    return out
 
 
 # ---- op-level wrappers -------------------------------------------------------------------
