@@ -334,8 +334,8 @@ int la_debug_capture(la_stream* s, int32_t enable);
 #define LA_TAP_HOP       12 /* bf16 [T_b, D] the QKV projection's operand of layer `layer` at the
                                slot's step (bf16 streams): the normalised residual, or, where
                                the stream folds the norm into its GEMMs (bf16 attention
-                               sublayers with w_in, w_head and bf16 projections), the residual
-                               itself rounded to bf16 (the GEMM scales its rows by 1 / rms)  */
+                               sublayers with w_in and w_head), the residual itself rounded
+                               to bf16 (the GEMM scales its rows by 1 / rms)                 */
 #define LA_TAP_SINK_HOP  13 /* bf16 [F, D] the same in the last sink pass (slot ignored)         */
 /* With attn_fp8 the Q, RING_K, RING_V and SINK_KROPE taps hold uint8 e4m3 codes
  * (value = code * scale of its layer, part and head; Q not pre-scaled), and: */

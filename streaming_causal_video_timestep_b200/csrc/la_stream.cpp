@@ -202,8 +202,9 @@ struct la_stream {
   void* hop = nullptr;      // [nbuf*T][D] normalised GEMM operand, dtype (fp32: == hn32); with the folded
                             // norm, the residual itself rounded to bf16
   // The per-token RMS norm folded into the GEMMs (bf16 attention sublayers with an in-projection and a
-  // head, no e4m3 projections): the in- and output projections' epilogues leave each row's sum of squares
-  // per column tile in ssq, and the QKV and head epilogues scale their rows by 1 / rms from it.
+  // head): the in- and output projections' epilogues leave each row's sum of squares per column tile in
+  // ssq, and the QKV and head epilogues scale their rows by 1 / rms from it (with e4m3 projections, on
+  // top of the operand's per-row scale: per-row scaling makes the codes of h those of h / rms).
   bool fold = false;
   float* ssq = nullptr;     // [nbuf*T][ssq_ld]
   int ssq_ld = 0;
@@ -1192,7 +1193,7 @@ int la_stream_create(const la_config* cfg, const la_weights* w, void* cuda_strea
   s->Da = s->cross ? cfg->audio_dim : 0;
   s->eq = s->afp8 ? 1 : s->ea;
   s->id_in = w->w_in == nullptr; s->id_head = w->w_head == nullptr;
-  s->fold = s->bf16 && !s->fp8 && !s->dit && !s->id_in && !s->id_head;
+  s->fold = s->bf16 && !s->dit && !s->id_in && !s->id_head;
   s->ssq_ld = s->fold ? ceil_div_i(s->D, gemm_tc_pick_bn(s->D)) : 0;
   s->nbuf = cfg->schedule == LA_SCHED_PIPELINED ? s->S : 1;
   s->st = static_cast<cudaStream_t>(cuda_stream);

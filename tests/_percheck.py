@@ -41,10 +41,11 @@ def _dit(cfg):
 
 def _folded(cfg, W):
     """Whether the stream folds the RMS norm into its GEMMs (bf16 attention
-    sublayers with an in-projection and a head, bf16 projections): the QKV and head
-    GEMMs then consume the residual itself rounded to bf16, and scale each product
-    row by the row's 1 / rms, taken from the fp32 residual."""
-    return (cfg.dtype == DTYPE_BF16 and not getattr(cfg, "proj_fp8", 0) and not _dit(cfg)
+    sublayers with an in-projection and a head): the QKV and head GEMMs then
+    consume the residual itself rounded to bf16 (with e4m3 projections, quantized
+    per row from it), and scale each product row by the row's 1 / rms, taken from
+    the fp32 residual."""
+    return (cfg.dtype == DTYPE_BF16 and not _dit(cfg)
             and W.w_in is not None and W.w_head is not None)
 
 
