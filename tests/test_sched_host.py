@@ -102,3 +102,22 @@ def test_bad_scheduling_configuration_is_rejected(over):
         cfg = TINY.cfg.replace(**over)
     with pytest.raises(LaError):
         _trace(cfg, [1, 1])
+
+
+@pytest.mark.parametrize("window,r", [(2, 0), (2, 3), (0, 1), (5, 2)])
+def test_slot_schedule_follows_the_pipelined_slot(window, r):
+    """A slot stream (LA_SCHED_SLOT, one rank of the timestep pipeline) keeps step r's
+    ring exactly as slot r of the grouped pipelined stream does: its call k runs block
+    k, as the pipelined stream's slot r does at call k + r."""
+    from workloads import SCHED_SLOT
+    n = 40
+    base = TINY.cfg.replace(window_blocks=window, sink_mode=SINK_FIXED)
+    S = base.num_steps
+    slot = _trace(base.replace(schedule=SCHED_SLOT, slot_index=r), [1] * n)
+    pipe = _trace(base.replace(schedule=SCHED_PIPELINED), [1] * (n + S - 1))
+    per = 8 + 3 * base.ring_entries
+    for k in range(n):
+        a = slot[k][4 + r * per: 4 + (r + 1) * per]
+        b = pipe[k + r][4 + r * per: 4 + (r + 1) * per]
+        np.testing.assert_array_equal(a, b)
+        assert a[0] == k
